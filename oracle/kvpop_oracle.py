@@ -1,0 +1,291 @@
+"""Plain CPU oracle for KVpop's decode-time hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module: it
+is used by tests/, by __graft_entry__.smoke() and by the cpu_baseline leg of
+bench.py.  It shares no code with the CUDA library (it does not import the
+package, its kernels, or its binding).
+
+Source: "KVpop -- Key-Value Cache Compression with Predictive Online Pruning"
+(paperlayer.ai summary page of arXiv 2607.05061v2).  Each function names the
+section it follows.  Everything is float64 numpy unless stated; ranking
+decisions use float32 scores, because the page's §F (Experiment Details,
+training setup) states that top-k ranking/selection runs in float32.
+
+Readings of points the page leaves open (each one is also listed in the
+design notes):
+
+* Total order on tokens (tie rule): key(j) = (s_j, -j).  A higher score ranks
+  higher; on equal scores the older token ranks higher.  A newcomer replaces
+  the current minimum only if its key is strictly larger.  NaN scores rank as
+  -inf; -0.0 equals +0.0.
+* Window = the W most recent positions {q-W+1 .. q} (current token included),
+  positions >= S only.  The token u = q - W leaves the window at q (§E.4
+  Delayed Readout: "newly eligible token is u = q - w").
+* Delay D > 0: a D-slot staging ring between window and the eligible region.
+  Staged tokens stay in the cache and are attended (§E.1: keys and values
+  remain cached until the eviction decision); they sit outside B = S+W+K.
+  The eligible set at q is {S <= j <= q - W - D}.
+* Update before attend: the query at position q attends to its own token and
+  to the set decided at q (§C.1 Mask Definition / §I Pseudocode: past tokens
+  that are sinks, recent, eligible and selected).
+* Attention scale 1/sqrt(d).  Scorer input x = [k; v] (§E.1), MLP
+  s = w2 . relu(W1 x + b1) + b2 (§E.2 stateless headwise MLP scorer).
+* Slot placement (needed only to compare slot maps): a prefill chunk keeps the
+  surviving long-range tokens in their slots and gives the admitted newcomers,
+  in ascending position, the free-or-vacated top-k slots in ascending slot
+  order; one decode step is the one-newcomer case (next free slot, else the
+  slot of the evicted minimum).  Window slot of token t: S + (t mod W);
+  staging slot: S + W + (t mod D); sink slot: t.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+NEG_INF = float("-inf")
+
+
+# ---------------------------------------------------------------------------
+# Scorer (§E.1 Headwise Inputs, §E.2 Stateless Linear and MLP Scorers)
+# ---------------------------------------------------------------------------
+
+def head_input(k: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """x = [k; v]: the scorer sees only cached quantities of the KV head (§E.1)."""
+    return np.concatenate([np.asarray(k, np.float64), np.asarray(v, np.float64)], axis=-1)
+
+
+def mlp_score(x: np.ndarray, w1: np.ndarray, b1: np.ndarray, w2: np.ndarray, b2: float) -> np.ndarray:
+    """Stateless headwise MLP score s = w2 . relu(W1 x + b1) + b2, float64 (§E.2).
+
+    x: [..., 2d]; w1: [hidden, 2d]; b1: [hidden]; w2: [hidden]; b2: scalar.
+    """
+    x = np.asarray(x, np.float64)
+    hidden = np.maximum(x @ np.asarray(w1, np.float64).T + np.asarray(b1, np.float64), 0.0)
+    return hidden @ np.asarray(w2, np.float64) + float(b2)
+
+
+def ranking_score(s) -> np.ndarray:
+    """Round scores to float32, the precision of top-k ranking (§F)."""
+    return np.asarray(s, np.float64).astype(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Retention policy (§3 Fixed-budget pruning; §C.1 Mask Definition; §I)
+# ---------------------------------------------------------------------------
+
+def rank_key(score: float, pos: int):
+    """Total order used for every retention decision: (score, -position)."""
+    s = float(score)
+    if math.isnan(s):
+        s = NEG_INF
+    return (s, -int(pos))
+
+
+def eligible_positions(q: int, S: int, W: int, D: int) -> range:
+    """Tokens that have left the protected window (and the staging ring) by query q."""
+    return range(S, max(S, q - W - D + 1))
+
+
+def running_topk(scores: Sequence[float], q: int, S: int, W: int, D: int, K: int) -> List[int]:
+    """Brute-force running prefix top-k: the K best eligible tokens at q, by rank_key.
+
+    Returned in ascending position order.  If at most K tokens are eligible all
+    of them are kept (§C.1: the budget is enforced once the sequence is long
+    enough).
+    """
+    elig = list(eligible_positions(q, S, W, D))
+    ranked = sorted(elig, key=lambda j: rank_key(scores[j], j), reverse=True)
+    return sorted(ranked[:K])
+
+
+def sink_positions(q: int, S: int) -> List[int]:
+    return list(range(0, min(S, q + 1)))
+
+
+def recent_positions(q: int, S: int, W: int, D: int) -> List[int]:
+    """Window {q-W+1..q} plus staging {q-W-D+1..q-W}, positions >= S only."""
+    return list(range(max(S, q - W - D + 1), q + 1))
+
+
+def attended_positions(q: int, S: int, W: int, D: int, topk: Sequence[int]) -> List[int]:
+    """Sinks, recent and selected long-range tokens (§C.1, §I), ascending."""
+    return sorted(set(sink_positions(q, S)) | set(recent_positions(q, S, W, D)) | set(topk))
+
+
+# ---------------------------------------------------------------------------
+# Attention over the retained set (§C.1: decoding attends directly over the
+# retained cache entries)
+# ---------------------------------------------------------------------------
+
+def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray):
+    """Softmax attention of query heads q [G][d] over keys/values [n][d], float64.
+
+    Returns (out [G][d], weights [G][n]).  Scale 1/sqrt(d).
+    """
+    q = np.asarray(q, np.float64)
+    keys = np.asarray(keys, np.float64)
+    values = np.asarray(values, np.float64)
+    d = q.shape[-1]
+    logits = (q @ keys.T) / math.sqrt(d)
+    logits = logits - logits.max(axis=-1, keepdims=True)
+    w = np.exp(logits)
+    w = w / w.sum(axis=-1, keepdims=True)
+    return w @ values, w
+
+
+# ---------------------------------------------------------------------------
+# Slot simulator: the incremental rule, slot by slot (for slot-map parity).
+# ---------------------------------------------------------------------------
+
+@dataclass
+class SlotState:
+    S: int
+    W: int
+    D: int
+    K: int
+    slot_pos: List[int] = field(default_factory=list)     # slot -> position (-1 = empty)
+    slot_score: List[float] = field(default_factory=list)  # top-k slots' ranking scores
+    n_seen: int = 0
+    n_topk: int = 0
+
+    def __post_init__(self):
+        n = self.S + self.W + self.D + self.K
+        self.slot_pos = [-1] * n
+        self.slot_score = [NEG_INF] * n
+
+    @property
+    def topk_base(self) -> int:
+        return self.S + self.W + self.D
+
+    def window_slot(self, t: int) -> int:
+        return self.S + (t % self.W)
+
+    def staging_slot(self, t: int) -> int:
+        return self.S + self.W + (t % self.D)
+
+    def topk_positions(self) -> List[int]:
+        b = self.topk_base
+        return sorted(p for p in self.slot_pos[b:b + self.K] if p >= 0)
+
+    def _admit(self, newcomers: Sequence[int], scores: Sequence[float]):
+        """Merge newly eligible tokens into the long-range slots (see module notes)."""
+        if not newcomers:
+            return
+        b = self.topk_base
+        current = [(self.slot_pos[b + i], b + i) for i in range(self.n_topk)]
+        pool = [(rank_key(scores[p], p), p) for p, _ in current] + \
+               [(rank_key(scores[p], p), p) for p in newcomers]
+        pool.sort(reverse=True)
+        keep = {p for _, p in pool[:self.K]}
+        vacated = [s for p, s in current if p not in keep]
+        free = list(range(b + self.n_topk, b + self.K))
+        targets = sorted(vacated + free)
+        admitted = sorted(p for p in newcomers if p in keep)
+        for slot in vacated:
+            self.slot_pos[slot] = -1
+            self.slot_score[slot] = NEG_INF
+        for slot, p in zip(targets, admitted):
+            self.slot_pos[slot] = p
+            self.slot_score[slot] = float(scores[p])
+        self.n_topk = min(self.K, self.n_topk + len(newcomers))
+
+    def append_chunk(self, n_new: int, scores: Sequence[float]):
+        """Prefill a chunk of n_new tokens (positions n_seen .. n_seen+n_new-1)."""
+        S, W, D = self.S, self.W, self.D
+        old, new = self.n_seen, self.n_seen + n_new
+        # newly eligible: positions in [S, new-W-D) not eligible before
+        lo = max(S, old - W - D)
+        hi = max(S, new - W - D)
+        newcomers = list(range(lo, hi))
+        # staging / window / sink contents follow directly from n_seen
+        self.n_seen = new
+        self._admit(newcomers, scores)
+        self._refresh_recent()
+
+    def decode(self, scores: Sequence[float]):
+        """One decode step: token p = n_seen arrives."""
+        self.append_chunk(1, scores)
+
+    def _refresh_recent(self):
+        S, W, D, n = self.S, self.W, self.D, self.n_seen
+        q = n - 1
+        for t in range(0, min(S, n)):
+            self.slot_pos[t] = t
+        for i in range(W):
+            self.slot_pos[S + i] = -1
+        for i in range(D):
+            self.slot_pos[S + W + i] = -1
+        for t in range(max(S, q - W + 1), q + 1):
+            self.slot_pos[self.window_slot(t)] = t
+        for t in range(max(S, q - W - D + 1), max(S, q - W + 1)):
+            self.slot_pos[self.staging_slot(t)] = t
+
+
+# ---------------------------------------------------------------------------
+# One (batch row, layer, KV head) unit, end to end.
+# ---------------------------------------------------------------------------
+
+@dataclass
+class UnitResult:
+    outputs: np.ndarray                 # [n_steps][G][d]
+    slot_maps: List[List[int]]          # after prefill, then after each step
+    topk_sets: List[List[int]]          # brute-force T_q after prefill and each step
+    weight_sums: np.ndarray             # [n_steps][G] softmax row sums
+    attended_counts: List[int]
+
+
+def run_unit(k_all: np.ndarray, v_all: np.ndarray, q_steps: np.ndarray, scores: Sequence[float],
+             S: int, W: int, D: int, K: int, P: int,
+             prefill_chunks: Optional[Sequence[int]] = None,
+             check_simulator: bool = True) -> UnitResult:
+    """Run prefill of P tokens, then len(q_steps) decode steps, for one unit.
+
+    k_all, v_all: [P + n_steps][d] keys/values of every token (prompt then
+    decode tokens); q_steps: [n_steps][G][d] queries of the decode steps;
+    scores: ranking scores of every token (already in ranking precision).
+    The attended set at every step is the brute-force definition; the slot
+    simulator runs beside it and must hold the same long-range set.
+    """
+    n_steps = len(q_steps)
+    state = SlotState(S, W, D, K)
+    chunks = list(prefill_chunks) if prefill_chunks else ([P] if P > 0 else [])
+    assert sum(chunks) == P
+    for c in chunks:
+        state.append_chunk(c, scores)
+    slot_maps = [list(state.slot_pos)]
+    topk_sets = [running_topk(scores, P - 1, S, W, D, K)] if P > 0 else [[]]
+    if check_simulator and P > 0:
+        assert state.topk_positions() == topk_sets[0], "slot simulator disagrees with brute force"
+    outs, sums, counts = [], [], []
+    for i in range(n_steps):
+        q = P + i
+        state.decode(scores)
+        T = running_topk(scores, q, S, W, D, K)
+        if check_simulator:
+            assert state.topk_positions() == T, f"slot simulator disagrees at q={q}"
+        A = attended_positions(q, S, W, D, T)
+        o, w = attention(q_steps[i], k_all[A], v_all[A])
+        outs.append(o)
+        sums.append(w.sum(axis=-1))
+        counts.append(len(A))
+        slot_maps.append(list(state.slot_pos))
+        topk_sets.append(T)
+    G = q_steps.shape[1] if n_steps else 0
+    d = k_all.shape[-1]
+    return UnitResult(outputs=np.array(outs).reshape(n_steps, G, d), slot_maps=slot_maps,
+                      topk_sets=topk_sets, weight_sums=np.array(sums).reshape(n_steps, G),
+                      attended_counts=counts)
+
+
+def unit_scores_mlp(k_all, v_all, w1, b1, w2, b2) -> np.ndarray:
+    """Ranking scores of every token of a unit from the MLP scorer (§E.2, §F)."""
+    return ranking_score(mlp_score(head_input(k_all, v_all), w1, b1, w2, b2))
+
+
+def dense_causal_attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray) -> np.ndarray:
+    """Plain dense attention of one query [G][d] over all keys/values up to itself."""
+    o, _ = attention(q, keys, values)
+    return o

@@ -1,0 +1,167 @@
+"""Pins of the CPU oracle against what the KVpop page and plain mathematics fix.
+
+Each pin raises AssertionError on failure.  They are plain functions so that
+test_oracle_pins.py runs them and test_oracle_mutations.py can check that a
+planted mistake in the oracle makes at least one of them fail.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+from oracle import kvpop_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def pin_mlp_hand_example():
+    g = _load("mlp_hand_example.json")
+    x = orc.head_input(np.array(g["k"]), np.array(g["v"]))
+    s = orc.mlp_score(x, np.array(g["w1"]), np.array(g["b1"]), np.array(g["w2"]), g["b2"])
+    assert abs(float(s) - g["score"]) < 1e-12, (float(s), g["score"])
+
+
+def _trace(name):
+    g = _load(name)
+    S, W, D, K, P = g["S"], g["W"], g["D"], g["K"], g["P"]
+    scores = g["scores"]
+    st = orc.SlotState(S, W, D, K)
+    st.append_chunk(P, scores)
+    assert st.slot_pos == g["slot_map_after_prefill"], (st.slot_pos, g["slot_map_after_prefill"])
+    for step in g["steps"]:
+        q = step["q"]
+        st.decode(scores)
+        assert st.n_seen == q + 1
+        T = orc.running_topk(scores, q, S, W, D, K)
+        assert T == step["topk"], (q, T, step["topk"])
+        assert orc.attended_positions(q, S, W, D, T) == step["attended"], (q, step["attended"])
+        assert st.slot_pos == step["slot_map"], (q, st.slot_pos, step["slot_map"])
+
+
+def pin_retention_trace_d0():
+    _trace("retention_trace_s1_w2_d0_k2.json")
+
+
+def pin_retention_trace_d1():
+    _trace("retention_trace_s1_w2_d1_k1.json")
+
+
+def pin_prefill_chunk_placement():
+    g = _load("prefill_chunk_placement_s1_w1_k2.json")
+    for mode in ("chunked", "single"):
+        st = orc.SlotState(g["S"], g["W"], g["D"], g["K"])
+        for n, expect in zip(g[mode]["chunks"], g[mode]["slot_map_after_chunk"]):
+            st.append_chunk(n, g["scores"])
+            assert st.slot_pos == expect, (mode, st.slot_pos, expect)
+        assert st.topk_positions() == g["topk"]
+
+
+def _rand_unit(seed, n_tokens, n_steps, G, d, tie_levels=0):
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((n_tokens, d))
+    v = rng.standard_normal((n_tokens, d))
+    q = rng.standard_normal((n_steps, G, d))
+    s = rng.standard_normal(n_tokens)
+    if tie_levels:
+        s = np.floor(s * tie_levels)
+    return k, v, q, orc.ranking_score(s)
+
+
+def pin_dense_when_budget_covers_context():
+    """Budget >= context: the output is plain dense attention (torch SDPA, float64)."""
+    S, W, D, K, P, n, G, d = 3, 5, 2, 64, 20, 30, 4, 16
+    k, v, q, s = _rand_unit(1, P + n, n, G, d)
+    res = orc.run_unit(k, v, q, s, S, W, D, K, P)
+    for i in range(n):
+        t = P + i
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q[i][:, None, :]), torch.tensor(k[None, :t + 1]),
+            torch.tensor(v[None, :t + 1])).numpy()[:, 0, :]
+        np.testing.assert_allclose(res.outputs[i], ref, rtol=1e-10, atol=1e-12)
+
+
+def pin_budget_invariant_and_structure():
+    """|sinks| + |window + staging| + |top-k| = B + D once the context is long enough;
+    sinks are always kept; the recent block is exactly the last W + D positions;
+    an evicted token never comes back; the long-range set is the brute-force top-K."""
+    for (S, W, D, K) in [(4, 16, 0, 44), (2, 5, 3, 7), (0, 3, 0, 4), (1, 1, 0, 3)]:
+        P, n = 40, 60
+        k, v, q, s = _rand_unit(S * 100 + W, P + n, n, 2, 8, tie_levels=3)
+        res = orc.run_unit(k, v, q, s, S, W, D, K, P)
+        evicted = set()
+        for i in range(n):
+            t = P + i
+            T = res.topk_sets[i + 1]
+            A = orc.attended_positions(t, S, W, D, T)
+            assert len(A) == res.attended_counts[i]
+            if t + 1 >= S + W + D + K:
+                assert len(A) == S + W + D + K, (S, W, D, K, t, len(A))
+            assert set(range(min(S, t + 1))) <= set(A)
+            recent = [j for j in A if j >= t - W - D + 1 and j >= S]
+            assert recent == list(range(max(S, t - W - D + 1), t + 1))
+            elig = list(range(S, max(S, t - W - D + 1)))
+            assert set(T) <= set(elig) and len(T) == min(K, len(elig))
+            # brute force over every subset size: T is the set of the K best keys
+            if T:
+                worst_kept = min(orc.rank_key(s[j], j) for j in T)
+                for j in elig:
+                    if j not in T:
+                        assert orc.rank_key(s[j], j) < worst_kept
+            assert not (set(T) & evicted), "evicted token came back"
+            prev = res.topk_sets[i]
+            evicted |= set(prev) - set(T)
+
+
+def pin_softmax_rows_sum_to_one():
+    k, v, q, s = _rand_unit(7, 50, 20, 3, 8)
+    res = orc.run_unit(k, v, q, s, 2, 4, 0, 6, 30)
+    np.testing.assert_allclose(res.weight_sums, 1.0, rtol=0, atol=1e-12)
+
+
+def pin_delay_equivalence():
+    """Stateless scorer: (W, D) behaves as (W + D, 0) with the same K; D = 0 is immediate."""
+    S, W, D, K, P, n, G, d = 2, 4, 3, 5, 25, 25, 2, 8
+    k, v, q, s = _rand_unit(11, P + n, n, G, d, tie_levels=2)
+    a = orc.run_unit(k, v, q, s, S, W, D, K, P)
+    b = orc.run_unit(k, v, q, s, S, W + D, 0, K, P)
+    np.testing.assert_allclose(a.outputs, b.outputs, rtol=0, atol=1e-14)
+    assert a.topk_sets == b.topk_sets
+
+
+def pin_prefill_is_running_topk():
+    """Prefill of P tokens equals prefill of P - m tokens followed by m decode steps."""
+    S, W, D, K, G, d = 3, 4, 0, 6, 2, 8
+    P, n, m = 30, 10, 7
+    k, v, q, s = _rand_unit(5, P + n, n + m, G, d, tie_levels=3)
+    a = orc.run_unit(k, v, q[m:], s, S, W, D, K, P)
+    b = orc.run_unit(k, v, q, s, S, W, D, K, P - m)
+    assert a.topk_sets == b.topk_sets[m:]
+    np.testing.assert_allclose(a.outputs, b.outputs[m:], rtol=0, atol=1e-14)
+
+
+def pin_attention_closed_forms():
+    d = 4
+    keys = np.array([[1.0, 0, 0, 0], [1.0, 0, 0, 0], [0, 1.0, 0, 0]])
+    vals = np.array([[1.0, 2, 3, 4], [3.0, 2, 1, 0], [0, 0, 0, 8]])
+    # equal logits on all keys -> mean of the values
+    q = np.zeros((1, d))
+    o, w = orc.attention(q, keys, vals)
+    np.testing.assert_allclose(o[0], vals.mean(axis=0), atol=1e-15)
+    # logits (q.k)/sqrt(d): q = [2 ln 3, 0, 0, 0] * sqrt(d)/2 -> keys 0,1 get ln 3, key 2 gets 0
+    q = np.array([[math.log(3.0) * math.sqrt(d), 0, 0, 0]])
+    o, w = orc.attention(q, keys, vals)
+    np.testing.assert_allclose(w[0], [3 / 7, 3 / 7, 1 / 7], atol=1e-15)
+    np.testing.assert_allclose(o[0], (3 * vals[0] + 3 * vals[1] + vals[2]) / 7, atol=1e-14)
+
+
+ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1,
+            pin_prefill_chunk_placement, pin_dense_when_budget_covers_context,
+            pin_budget_invariant_and_structure, pin_softmax_rows_sum_to_one,
+            pin_delay_equivalence, pin_prefill_is_running_topk, pin_attention_closed_forms]

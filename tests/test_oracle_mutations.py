@@ -1,0 +1,122 @@
+"""Planted mistakes in the CPU oracle must make at least one pin fail.
+
+Each case monkeypatches one oracle function with a plausible slip (a dropped
+term, a wrong sign or index, a swapped operand) and runs every pin; the case
+passes only if some pin raises.  This is what makes the pins evidence.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle_pins as pins
+from oracle import kvpop_oracle as orc
+
+
+def _ties_to_newer(score, pos):
+    s = float(score)
+    return (s, int(pos))
+
+
+def _elig_off_by_one(q, S, W, D):
+    return range(S, max(S, q - W - D + 2))
+
+
+def _no_scale(q, keys, values):
+    q = np.asarray(q, np.float64)
+    logits = q @ np.asarray(keys, np.float64).T
+    logits -= logits.max(axis=-1, keepdims=True)
+    w = np.exp(logits)
+    w /= w.sum(axis=-1, keepdims=True)
+    return w @ np.asarray(values, np.float64), w
+
+
+def _vk_order(k, v):
+    return np.concatenate([np.asarray(v, np.float64), np.asarray(k, np.float64)], axis=-1)
+
+
+def _drop_b1(x, w1, b1, w2, b2):
+    h = np.maximum(np.asarray(x, np.float64) @ np.asarray(w1).T, 0.0)
+    return h @ np.asarray(w2) + float(b2)
+
+
+def _drop_b2(x, w1, b1, w2, b2):
+    h = np.maximum(np.asarray(x, np.float64) @ np.asarray(w1).T + np.asarray(b1), 0.0)
+    return h @ np.asarray(w2)
+
+
+def _no_relu(x, w1, b1, w2, b2):
+    h = np.asarray(x, np.float64) @ np.asarray(w1).T + np.asarray(b1)
+    return h @ np.asarray(w2) + float(b2)
+
+
+def _recent_without_current(q, S, W, D):
+    return list(range(max(S, q - W - D + 1), q))
+
+
+def _recent_ignores_staging(q, S, W, D):
+    return list(range(max(S, q - W + 1), q + 1))
+
+
+def _topk_keeps_lowest(scores, q, S, W, D, K):
+    elig = list(orc.eligible_positions(q, S, W, D))
+    ranked = sorted(elig, key=lambda j: orc.rank_key(scores[j], j))
+    return sorted(ranked[:K])
+
+
+def _topk_keeps_k_minus_1(scores, q, S, W, D, K):
+    elig = list(orc.eligible_positions(q, S, W, D))
+    ranked = sorted(elig, key=lambda j: orc.rank_key(scores[j], j), reverse=True)
+    return sorted(ranked[:max(K - 1, 0)])
+
+
+def _sinks_off_by_one(q, S):
+    return list(range(0, min(S - 1, q + 1)))
+
+
+def _softmax_without_max_shift_wrong_norm(q, keys, values):
+    q = np.asarray(q, np.float64)
+    logits = (q @ np.asarray(keys, np.float64).T) / math.sqrt(q.shape[-1])
+    w = np.exp(logits)
+    w /= w.shape[-1]
+    return w @ np.asarray(values, np.float64), w
+
+
+def _window_slot_wrong(self, t):
+    return self.S + ((t + 1) % self.W)
+
+
+MUTATIONS = {
+    "tie_goes_to_newer": ("rank_key", _ties_to_newer),
+    "eligible_off_by_one": ("eligible_positions", _elig_off_by_one),
+    "attention_no_scale": ("attention", _no_scale),
+    "scorer_input_v_then_k": ("head_input", _vk_order),
+    "scorer_drops_b1": ("mlp_score", _drop_b1),
+    "scorer_drops_b2": ("mlp_score", _drop_b2),
+    "scorer_no_relu": ("mlp_score", _no_relu),
+    "recent_excludes_current": ("recent_positions", _recent_without_current),
+    "recent_ignores_staging": ("recent_positions", _recent_ignores_staging),
+    "topk_keeps_lowest": ("running_topk", _topk_keeps_lowest),
+    "topk_keeps_k_minus_1": ("running_topk", _topk_keeps_k_minus_1),
+    "sinks_off_by_one": ("sink_positions", _sinks_off_by_one),
+    "softmax_wrong_normaliser": ("attention", _softmax_without_max_shift_wrong_norm),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(orc, attr, fn)
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError, ZeroDivisionError):
+            failed.append(pin.__name__)
+    assert failed, f"mutation {name} passed every pin"
+
+
+def test_slot_placement_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(orc.SlotState, "window_slot", _window_slot_wrong)
+    with pytest.raises(AssertionError):
+        pins.pin_retention_trace_d0()
