@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""KVpop decode benchmark on B200: decode tokens/s and achieved HBM bandwidth.
+
+One step = one KVpop decode step of every layer of the workload for every
+batch row: per layer, window append + boundary scoring + argmin-replace
+(kvpop_decode_append) and GQA attention over the bounded cache
+(kvpop_decode_attend), through the C ABI.  Default workload: Qwen3-4B-shaped,
+87.5% compression (36 layers, 32 q / 8 kv heads, d 128, bf16, batch 64,
+budget 1024 = 4 sinks + 128 window + 892 long-range, prompt 8192).  Data are
+synthetic (seeded), shaped like the pages' workloads; the cache (9.7 GB) is
+far larger than L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle
+instead (the reference arm).  Multi-GPU: one replica per rank (the path
+shards into independent (batch row, KV head) units; no data-path
+collective), timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import kvpop_workloads as wl  # noqa: E402
+
+WORKLOADS = {"cr88": wl.QWEN3_4B_CR88, "cr75": wl.QWEN3_4B_CR75, "8b_d32": wl.QWEN3_8B_D32}
+METRIC = "decode tokens/s and achieved HBM GB/s (% of peak) at 75%/88% KV compression"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kvpop", "reference"], default="kvpop")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cr88")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--input-sets", type=int, default=32, help="distinct decode input sets, cycled")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (small cases for ncu captures; renames the workload)")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+
+def attention_bytes(w: wl.Workload) -> int:
+    """Bytes one attention launch (one layer, all units) must move at steady
+    state: every occupied slot row [k | v] once, q in, output out."""
+    es = 2 if w.dtype == "bf16" else 4
+    units = w.batch * w.n_kv_heads
+    slots = w.sinks + w.window + w.delay + w.topk
+    return units * slots * 2 * w.head_dim * es + 2 * w.batch * w.n_q_heads * w.head_dim * es
+
+
+def step_bytes(w: wl.Workload) -> int:
+    """Algorithmic HBM bytes of one whole decode step (all layers, all rows):
+    K/V read + q + out + new K/V write + boundary K/V read + replace copy +
+    long-range score scan, per (batch row, layer); scorer weights once."""
+    es = 2 if w.dtype == "bf16" else 4
+    d, Hkv, Hq = w.head_dim, w.n_kv_heads, w.n_q_heads
+    per_row_layer = (Hkv * (w.sinks + w.window + w.delay + w.topk) * 2 * d * es
+                     + Hq * d * es + Hq * d * es
+                     + Hkv * 3 * 2 * d * es
+                     + Hkv * w.topk * 8)
+    weights = w.n_layers * Hkv * (w.scorer_hidden * 2 * d + 2 * w.scorer_hidden + 1) * 4
+    return w.batch * w.n_layers * per_row_layer + weights
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """A bounded sample of the workload on the CPU oracle: `n_units` units of
+    the workload's shape (prompt of P tokens prefilled, untimed), stepped one
+    decode token at a time."""
+
+    def __init__(self, w: wl.Workload, n_units: int, max_steps: int, seed: int = 1):
+        import numpy as np
+        from oracle import kvpop_oracle as orc
+        self.orc = orc
+        one = w.replace(batch=1, n_layers=1)
+        k, v = wl.prompt_kv(one, 0, master=seed)
+        qd, kd, vd = wl.decode_inputs_batched(one, 0, max_steps, master=seed)
+        w1, b1, w2, b2 = wl.scorer_weights(one, master=seed)
+        self.units = []
+        G = w.group
+        for u in range(n_units):
+            h = u % w.n_kv_heads
+            k_all = np.concatenate([k[0, h].double().numpy(), kd[:, 0, h].double().numpy()])
+            v_all = np.concatenate([v[0, h].double().numpy(), vd[:, 0, h].double().numpy()])
+            q_steps = qd[:, 0, h * G:(h + 1) * G].double().numpy()
+            s = orc.unit_scores_mlp(k_all, v_all, w1[0, h].double().numpy(), b1[0, h].double().numpy(),
+                                    w2[0, h].double().numpy(), float(b2[0, h]))
+            unit = orc.OracleUnit(k_all, v_all, s, w.sinks, w.window, w.delay, w.topk, w.prefill,
+                                  check_simulator=False)
+            self.units.append((unit, q_steps))
+        self.i = 0
+
+    def step(self):
+        for unit, q_steps in self.units:
+            unit.step(q_steps[self.i])
+        self.i += 1
+
+
+def cpu_threads_limit():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=1)
+    except Exception:
+        return None
+
+
+def oracle_tokens_per_s(w: wl.Workload, seconds: float):
+    """Times the oracle's decode steps on a bounded sample; returns
+    (tokens/s, description)."""
+    units_per_token = w.n_layers * w.n_kv_heads
+    n_units, max_steps = 4, 400
+    lim = cpu_threads_limit()
+    sample = OracleSample(w, n_units, max_steps)
+    t0 = time.perf_counter()
+    steps = 0
+    while steps < max_steps and (time.perf_counter() - t0 < seconds or steps < 2):
+        sample.step()
+        steps += 1
+    dt = time.perf_counter() - t0
+    if lim is not None:
+        lim.unregister() if hasattr(lim, "unregister") else None
+    unit_steps = n_units * steps
+    tok_s = unit_steps / units_per_token / dt
+    desc = (f"{n_units} (batch row, KV head) units of the {w.name} shape, prompt {w.prefill} prefilled "
+            f"untimed, {steps} decode steps each timed ({unit_steps} unit-steps, {dt:.1f} s); one decode "
+            f"token = {units_per_token} unit-steps (all layers and KV heads of one batch row)")
+    return tok_s, desc
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    units_per_token = w.n_layers * w.n_kv_heads
+    n_units = 2
+    lim = cpu_threads_limit()
+    sample = OracleSample(w, n_units, args.warmup + args.steps + 1)
+    for _ in range(args.warmup):
+        sample.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        sample.step()
+    dt = time.perf_counter() - t0
+    tok_s = n_units * args.steps / units_per_token / dt
+    desc = (f"each step: one decode step of {n_units} units of the {w.name} shape on the CPU oracle "
+            f"(prompt {w.prefill} prefilled untimed); tokens = unit-steps / {units_per_token}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "sample": desc},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def build_cache(w: wl.Workload, torch):
+    import fixed_budget_kv_kvpop_b200 as kp
+    weights = tuple(t.cuda() for t in wl.scorer_weights(w))
+    w1, b1, w2, b2 = weights
+    cfg = kp.make_config(batch=w.batch, n_layers=w.n_layers, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                         head_dim=w.head_dim, sinks=w.sinks, window=w.window, topk=w.topk, delay=w.delay,
+                         ref_context=w.prefill, compression_ratio=w.compression_ratio,
+                         max_prefill_chunk=w.prefill, dtype=w.dtype, scorer_hidden=w.scorer_hidden,
+                         w1=w1, b1=b1, w2=w2, b2=b2)
+    cache = kp.KVPopCache(cfg, keepalive=weights)
+    for layer in range(w.n_layers):
+        k, v = wl.prompt_kv(w, layer, device="cuda")
+        cache.prefill(layer, k, v)
+        del k, v
+    torch.cuda.synchronize()
+    return cache
+
+
+def run_gpu(args, w, rank, world, torch):
+    dev = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    t_setup = time.perf_counter()
+    cache = build_cache(w, torch)
+    NI = max(1, min(args.input_sets, args.steps + args.warmup))
+    qs, ks, vs = [], [], []
+    for layer in range(w.n_layers):
+        q, k, v = wl.decode_inputs_batched(w, layer, NI, device="cuda")
+        qs.append(q); ks.append(k); vs.append(v)
+    outs = [torch.empty_like(qs[0][0]) for _ in range(w.n_layers)]
+    torch.cuda.synchronize()
+    setup_s = time.perf_counter() - t_setup
+    L = w.n_layers
+
+    def one_step(i, ev=None):
+        j = i % NI
+        for layer in range(L):
+            cache.decode_append(layer, ks[layer][j], vs[layer][j], stream=stream)
+            if ev is not None:
+                ev[0][layer].record(stream)
+            cache.decode_attend(layer, qs[layer][j], outs[layer], stream=stream)
+            if ev is not None:
+                ev[1][layer].record(stream)
+
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize()
+    st, bits = cache.get_error()
+    if st != 0:
+        raise RuntimeError(f"device error after warm-up: status {st} bits {bits}")
+
+    evs = [([torch.cuda.Event(enable_timing=True) for _ in range(L)],
+            [torch.cuda.Event(enable_timing=True) for _ in range(L)]) for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    smi_idx = dev
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            smi_idx = int(vis.split(",")[dev])
+        except ValueError:
+            smi_idx = dev
+    sampler = ClockSampler(smi_idx)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for s in range(args.steps):
+        one_step(args.warmup + s, evs[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = start.elapsed_time(end)
+    attn_ms = [evs[s][0][l].elapsed_time(evs[s][1][l]) for s in range(args.steps) for l in range(L)]
+    st, bits = cache.get_error()
+    if st != 0:
+        raise RuntimeError(f"device error in timed region: status {st} bits {bits}")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    tokens = w.batch * args.steps * world
+    value = tokens / (elapsed_ms / 1e3)
+    peak, peak_kind = measured_peaks()
+    sbytes = step_bytes(w)
+    step_gbs = sbytes * args.steps / (elapsed_ms / 1e3) / 1e9
+    abytes = attention_bytes(w)
+    attn_mean_ms = statistics.fmean(attn_ms)
+    attn_gbs = abytes / (attn_mean_ms / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, cache, torch, world)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "layers": w.n_layers, "q_heads": w.n_q_heads,
+                   "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "sinks": w.sinks, "window": w.window,
+                   "topk": w.topk, "delay": w.delay, "budget": w.budget, "prompt": w.prefill,
+                   "compression": round(w.compression_ratio, 4), "parallelism": f"replicas x{world}",
+                   "l2": "no flush: inputs (cache %.1f GB) larger than L2" % (w.n_layers * attention_bytes(w) / 1e9),
+                   "input_sets": NI},
+        "hbm": {"step_bytes": sbytes, "achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
+                "frac_of_8tbs": step_gbs / 8000.0, "peak_kind": peak_kind},
+        "roofline": {"kernel": "decode_attention_kernel<bf16,128,4>", "bound": "hbm", "achieved": attn_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": attn_gbs / peak, "traffic": None,
+                     "bytes_per_launch": abytes, "mean_launch_us": attn_mean_ms * 1e3,
+                     "launches": len(attn_ms), "peak_kind": peak_kind},
+        "gpu_launches": 2 * L * args.steps,
+        "clocks": clocks,
+        "setup_s": setup_s,
+    }
+    if e2e is not None:
+        res["e2e"] = e2e
+    return res
+
+
+def run_e2e(args, w, cache, torch, world):
+    """Same metric through the C ABI with the step's inputs in pinned HOST
+    memory: each step copies q/k/v of all layers host->device, runs the step,
+    and copies the outputs device->host, pipelined over two buffers and three
+    streams (copy-in, compute, copy-out)."""
+    L, K = w.n_layers, max(1, args.e2e_steps)
+    NI = 4
+    hq = [torch.empty((L,) + (w.batch, w.n_q_heads, w.head_dim), dtype=w.torch_dtype()).pin_memory()
+          for _ in range(NI)]
+    hk = [torch.empty((L, w.batch, w.n_kv_heads, w.head_dim), dtype=w.torch_dtype()).pin_memory()
+          for _ in range(NI)]
+    hv = [torch.empty_like(hk[0]).pin_memory() for _ in range(NI)]
+    for i in range(NI):
+        for layer in range(L):
+            q, k, v = wl.decode_inputs(w, layer, 10_000 + i)
+            hq[i][layer].copy_(q); hk[i][layer].copy_(k); hv[i][layer].copy_(v)
+    hout = [torch.empty_like(hq[0]).pin_memory() for _ in range(2)]
+    dq = [torch.empty_like(hq[0], device="cuda") for _ in range(2)]
+    dk = [torch.empty_like(hk[0], device="cuda") for _ in range(2)]
+    dv = [torch.empty_like(hk[0], device="cuda") for _ in range(2)]
+    dout = [torch.empty_like(hq[0], device="cuda") for _ in range(2)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+
+    def step(s, first):
+        b = s % 2
+        with torch.cuda.stream(s_in):
+            if not first[b]:
+                s_in.wait_event(ev_cmp[b])
+            dq[b].copy_(hq[s % NI], non_blocking=True)
+            dk[b].copy_(hk[s % NI], non_blocking=True)
+            dv[b].copy_(hv[s % NI], non_blocking=True)
+            ev_in[b].record(s_in)
+        s_cmp.wait_event(ev_in[b])
+        if not first[b]:
+            s_cmp.wait_event(ev_out[b])
+        for layer in range(L):
+            cache.decode_append(layer, dk[b][layer], dv[b][layer], stream=s_cmp)
+            cache.decode_attend(layer, dq[b][layer], dout[b][layer], stream=s_cmp)
+        ev_cmp[b].record(s_cmp)
+        s_out.wait_event(ev_cmp[b])
+        with torch.cuda.stream(s_out):
+            hout[b].copy_(dout[b], non_blocking=True)
+            ev_out[b].record(s_out)
+        first[b] = False
+
+    first = [True, True]
+    for s in range(3):
+        step(s, first)
+    torch.cuda.synchronize()
+    start.record(s_in)
+    for s in range(K):
+        step(3 + s, first)
+    end.record(s_out)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    es = 2 if w.dtype == "bf16" else 4
+    h2d = L * w.batch * (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim * es
+    d2h = L * w.batch * w.n_q_heads * w.head_dim * es
+    return {"value": w.batch * K * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": K, "ms_per_step": ms / K}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+    if args.layers and args.layers != w.n_layers:
+        w = w.replace(name=f"{w.name}_L{args.layers}", n_layers=args.layers)
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_gpu(args, w, rank, world, torch)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, desc = oracle_tokens_per_s(w, args.cpu_seconds)
+            res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

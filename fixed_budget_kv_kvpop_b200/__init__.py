@@ -1,0 +1,224 @@
+"""Python binding of libkvpop.so (the KVpop fixed-budget KV cache C ABI).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels behind include/kvpop.h.  PyTorch supplies device memory and streams.
+Importing this module loads the in-tree libkvpop.so and fails loudly if it is
+missing; there is no fallback implementation.
+
+Names follow the C ABI: kvpop_cache_bytes, kvpop_create, kvpop_prefill,
+kvpop_decode_step, kvpop_inspect, kvpop_get_layout, kvpop_get_error,
+kvpop_clear_error, kvpop_debug_poison_error, kvpop_destroy,
+kvpop_status_string.  `KVPopCache` bundles a handle with its device buffer.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvpop.so")
+
+KVPOP_OK = 0
+KVPOP_ERR_INVALID_ARG = -1
+KVPOP_ERR_BAD_SHAPE = -2
+KVPOP_ERR_ORDER = -3
+KVPOP_ERR_CONTEXT_OVERFLOW = -4
+KVPOP_ERR_CUDA = -5
+KVPOP_ERR_DEVICE = -6
+KVPOP_ERR_TIMEOUT = -7
+
+KVPOP_DTYPE_F32 = 0
+KVPOP_DTYPE_BF16 = 1
+KVPOP_FLAG_EXTERNAL_SCORES = 1
+KVPOP_FLAG_DEBUG_CHECKS = 2
+
+KVPOP_DEVERR_CONTEXT_OVERFLOW = 1
+KVPOP_DEVERR_TIMEOUT = 2
+KVPOP_DEVERR_BAD_INDEX = 4
+KVPOP_DEVERR_NAN_SCORE = 8
+KVPOP_DEVERR_STATE_MISMATCH = 16
+
+EXPORTED_SYMBOLS = (
+    "kvpop_cache_bytes", "kvpop_create", "kvpop_prefill", "kvpop_decode_step", "kvpop_decode_append",
+    "kvpop_decode_attend", "kvpop_inspect",
+    "kvpop_get_layout", "kvpop_get_error", "kvpop_clear_error", "kvpop_debug_poison_error",
+    "kvpop_destroy", "kvpop_status_string",
+)
+
+
+class kvpop_config(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_layers", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("sinks", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("topk", ctypes.c_int32), ("delay", ctypes.c_int32),
+        ("ref_context", ctypes.c_int32), ("compression_ratio", ctypes.c_float),
+        ("max_context", ctypes.c_int32), ("max_prefill_chunk", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("scorer_hidden", ctypes.c_int32),
+        ("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+class kvpop_layout_info(ctypes.Structure):
+    _fields_ = [
+        ("kv_offset", ctypes.c_size_t), ("kv_layer_stride", ctypes.c_size_t),
+        ("pos_offset", ctypes.c_size_t), ("pos_layer_stride", ctypes.c_size_t),
+        ("score_offset", ctypes.c_size_t), ("score_layer_stride", ctypes.c_size_t),
+        ("state_offset", ctypes.c_size_t), ("state_layer_stride", ctypes.c_size_t),
+        ("slots_per_unit", ctypes.c_int32), ("units", ctypes.c_int32), ("row_bytes", ctypes.c_int32),
+        ("topk_base", ctypes.c_int32),
+    ]
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"libkvpop.so not built at {path}: run "
+                          "`python fixed_budget_kv_kvpop_b200/csrc/build.py` (no CPU fallback exists)")
+    lib = ctypes.CDLL(path)
+    P, I32, U32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t
+    sig = {
+        "kvpop_cache_bytes": ([ctypes.POINTER(kvpop_config), ctypes.POINTER(SZ)], ctypes.c_int),
+        "kvpop_create": ([ctypes.POINTER(kvpop_config), P, SZ, ctypes.POINTER(P)], ctypes.c_int),
+        "kvpop_prefill": ([P, I32, P, P, I32, P, P], ctypes.c_int),
+        "kvpop_decode_step": ([P, I32, P, P, P, P, P, P], ctypes.c_int),
+        "kvpop_decode_append": ([P, I32, P, P, P, P], ctypes.c_int),
+        "kvpop_decode_attend": ([P, I32, P, P, P], ctypes.c_int),
+        "kvpop_inspect": ([P, I32, P, P, P, P], ctypes.c_int),
+        "kvpop_get_layout": ([P, ctypes.POINTER(kvpop_layout_info)], ctypes.c_int),
+        "kvpop_get_error": ([P, ctypes.POINTER(I32)], ctypes.c_int),
+        "kvpop_clear_error": ([P, P], ctypes.c_int),
+        "kvpop_debug_poison_error": ([P, I32, P], ctypes.c_int),
+        "kvpop_destroy": ([P], ctypes.c_int),
+        "kvpop_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = load_library()
+
+
+class KVPopError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.kvpop_status_string(status).decode()} ({status})")
+
+
+def _check(status: int, what: str) -> None:
+    if status != KVPOP_OK:
+        raise KVPopError(status, what)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream or None
+
+
+def make_config(*, batch, n_layers, n_q_heads, n_kv_heads, head_dim, sinks, window, topk, delay=0,
+                ref_context=0, compression_ratio=0.0, max_context=1 << 30, max_prefill_chunk=0,
+                dtype="bf16", scorer_hidden=64, w1=None, b1=None, w2=None, b2=None,
+                external_scores=False, debug_checks=False) -> kvpop_config:
+    c = kvpop_config()
+    c.batch, c.n_layers, c.n_q_heads, c.n_kv_heads, c.head_dim = batch, n_layers, n_q_heads, n_kv_heads, head_dim
+    c.sinks, c.window, c.topk, c.delay = sinks, window, topk, delay
+    c.ref_context, c.compression_ratio = ref_context, compression_ratio
+    c.max_context, c.max_prefill_chunk = max_context, max_prefill_chunk
+    c.dtype = KVPOP_DTYPE_F32 if dtype in ("f32", "float32") else KVPOP_DTYPE_BF16
+    c.scorer_hidden = scorer_hidden
+    c.w1, c.b1, c.w2, c.b2 = _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)
+    c.flags = (KVPOP_FLAG_EXTERNAL_SCORES if external_scores else 0) | (KVPOP_FLAG_DEBUG_CHECKS if debug_checks else 0)
+    return c
+
+
+def cache_bytes(cfg: kvpop_config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.kvpop_cache_bytes(ctypes.byref(cfg), ctypes.byref(n)), "kvpop_cache_bytes")
+    return n.value
+
+
+class KVPopCache:
+    """A handle plus the device buffer it lives in (allocated with torch).
+
+    The scorer weights passed to make_config must stay alive as long as this
+    object; they are kept referenced here.
+    """
+
+    def __init__(self, cfg: kvpop_config, device=None, keepalive=()):
+        import torch
+        self.cfg = cfg
+        self._keep = tuple(keepalive)
+        self.nbytes = cache_bytes(cfg)
+        self.buffer = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        base = self.buffer.data_ptr()
+        self._off = (-base) % 256
+        self.handle = ctypes.c_void_p()
+        _check(lib.kvpop_create(ctypes.byref(cfg), ctypes.c_void_p(base + self._off), self.nbytes,
+                                ctypes.byref(self.handle)), "kvpop_create")
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            lib.kvpop_destroy(h)
+            self.handle = None
+
+    def prefill(self, layer: int, k, v, ext_scores=None, stream=None):
+        n = int(k.shape[2]) if k is not None else 0
+        _check(lib.kvpop_prefill(self.handle, layer, _ptr(k), _ptr(v), n, _ptr(ext_scores),
+                                 _stream_ptr(stream)), "kvpop_prefill")
+
+    def decode_step(self, layer: int, q, k_new, v_new, out, ext_score=None, stream=None):
+        _check(lib.kvpop_decode_step(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                     _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step")
+
+    def decode_append(self, layer: int, k_new, v_new, ext_score=None, stream=None):
+        _check(lib.kvpop_decode_append(self.handle, layer, _ptr(k_new), _ptr(v_new), _ptr(ext_score),
+                                       _stream_ptr(stream)), "kvpop_decode_append")
+
+    def decode_attend(self, layer: int, q, out, stream=None):
+        _check(lib.kvpop_decode_attend(self.handle, layer, _ptr(q), _ptr(out), _stream_ptr(stream)),
+               "kvpop_decode_attend")
+
+    def inspect(self, layer: int, stream=None):
+        import numpy as np
+        lay = self.layout()
+        n = lay.units * lay.slots_per_unit
+        pos = np.empty(n, np.int32)
+        score = np.empty(n, np.float32)
+        state = np.empty(lay.units * 4, np.int32)
+        _check(lib.kvpop_inspect(self.handle, layer, pos.ctypes.data, score.ctypes.data, state.ctypes.data,
+                                 _stream_ptr(stream)), "kvpop_inspect")
+        return (pos.reshape(lay.units, lay.slots_per_unit), score.reshape(lay.units, lay.slots_per_unit),
+                state.reshape(lay.units, 4))
+
+    def layout(self) -> kvpop_layout_info:
+        info = kvpop_layout_info()
+        _check(lib.kvpop_get_layout(self.handle, ctypes.byref(info)), "kvpop_get_layout")
+        return info
+
+    def kv_rows(self, layer: int):
+        """View of layer `layer`'s cache rows as a byte tensor [units][slots][row_bytes]."""
+        lay = self.layout()
+        start = self._off + lay.kv_offset + layer * lay.kv_layer_stride
+        n = lay.units * lay.slots_per_unit * lay.row_bytes
+        return self.buffer[start:start + n].view(lay.units, lay.slots_per_unit, lay.row_bytes)
+
+    def get_error(self):
+        bits = ctypes.c_int32(0)
+        st = lib.kvpop_get_error(self.handle, ctypes.byref(bits))
+        return st, bits.value
+
+    def clear_error(self, stream=None):
+        _check(lib.kvpop_clear_error(self.handle, _stream_ptr(stream)), "kvpop_clear_error")
+
+    def poison_error(self, bits: int, stream=None):
+        _check(lib.kvpop_debug_poison_error(self.handle, bits, _stream_ptr(stream)), "kvpop_debug_poison_error")

@@ -1,0 +1,235 @@
+// Internal definitions shared by the KVpop CUDA kernels and the C-ABI host code.
+//
+// Method: "KVpop -- Key-Value Cache Compression with Predictive Online Pruning"
+// (summary page of arXiv 2607.05061v2).  Each KV head keeps a bounded cache of
+// S sink tokens, a protected window of the W most recent tokens, an optional
+// D-slot staging ring for delayed scoring, and K long-range slots holding the
+// running top-k of the tokens that have left the window (§3 Fixed-budget
+// pruning, §C.1 Mask Definition, §I Pseudocode).
+//
+// Device cache layout of one layer (all row-major, one "unit" = one
+// (batch row, KV head) pair, unit = b * Hkv + h):
+//   kv    [units][NS][2][d]  element type T; per slot the key row then the value
+//                            row, so one slot is one contiguous 2*d*sizeof(T) row
+//   pos   [units][NS]  int32 position held by each slot, -1 = empty
+//   score [units][NS]  fp32  ranking score (long-range slots; with caller
+//                            scores also the window/staging slots)
+//   state [units][4]   int32 {n_seen, n_topk, 0, 0}
+// Slot map: sinks [0, S) hold positions 0..S-1; window slot of token t is
+// S + (t mod W); staging slot is S + W + (t mod D); long-range slots start at
+// S + W + D and fill as a prefix.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace kvpop {
+
+// Device error bits, OR-ed into the error word (read by kvpop_get_error).
+enum : int32_t {
+  DEVERR_CONTEXT_OVERFLOW = 1,
+  DEVERR_TIMEOUT = 2,
+  DEVERR_BAD_INDEX = 4,
+  DEVERR_NAN_SCORE = 8,
+  DEVERR_STATE_MISMATCH = 16,
+};
+
+constexpr int kMaxSeg = 64;         // split-K partials per unit (upper bound)
+constexpr int kTileSlots = 16;      // slots per consumer-warp tile in the decode kernel
+constexpr int kConsumerWarps = 8;   // consumer warps per decode CTA
+constexpr int kStagesPerWarp = 3;   // smem pipeline depth per consumer warp
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
+
+struct LayerArgs {
+  uint8_t* kv;          // this layer's [units][NS][2][d]
+  int32_t* pos;         // [units][NS]
+  float* score;         // [units][NS]
+  int32_t* state;       // [units][4]
+  const float* w1;      // this layer's scorer [Hkv][hidden][2d]
+  const float* b1;      // [Hkv][hidden]
+  const float* w2;      // [Hkv][hidden]
+  const float* b2;      // [Hkv]
+  int32_t* err;         // device error word
+  int units, Hkv, Hq, G, d, S, W, D, K, NS, hidden;
+  int max_context;
+  uint32_t flags;
+  int row_bytes;        // 2 * d * sizeof(T)
+};
+
+constexpr uint32_t FLAG_EXTERNAL_SCORES = 1u;
+constexpr uint32_t FLAG_DEBUG_CHECKS = 2u;
+
+// --- total order on tokens: key = (score, -position), packed in 64 bits ---
+// Higher score ranks higher; on equal score the older (smaller) position ranks
+// higher.  -0.0 is folded onto +0.0 and NaN ranks below -inf.
+__host__ __device__ __forceinline__ uint64_t rank_key(float s, int32_t pos) {
+  uint32_t u;
+#ifdef __CUDA_ARCH__
+  u = __float_as_uint(s);
+#else
+  __builtin_memcpy(&u, &s, 4);
+#endif
+  uint32_t ordered;
+  if ((u & 0x7fffffffu) > 0x7f800000u) {
+    ordered = 0u;                       // NaN
+  } else {
+    if ((u & 0x7fffffffu) == 0u) u = 0u;  // -0 -> +0
+    ordered = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
+  return (static_cast<uint64_t>(ordered) << 32) | static_cast<uint32_t>(0xffffffffu - static_cast<uint32_t>(pos));
+}
+
+// --- slot helpers ---
+__host__ __device__ __forceinline__ int window_slot(int t, int S, int W) { return S + (t % W); }
+__host__ __device__ __forceinline__ int staging_slot(int t, int S, int W, int D) { return S + W + (t % D); }
+__host__ __device__ __forceinline__ int topk_base(int S, int W, int D) { return S + W + D; }
+
+// Split-K work decomposition of the decode kernel (host and device agree on it).
+// total tiles = units * tpu; nw = number of consumer warps that get work; warp
+// w covers tiles [w*total/nw, (w+1)*total/nw).
+__host__ __device__ __forceinline__ int64_t seg_lo(int64_t w, int64_t total, int64_t nw) {
+  return (w * total) / nw;
+}
+__host__ __device__ __forceinline__ int64_t warp_of_tile(int64_t x, int64_t total, int64_t nw) {
+  return ((x + 1) * nw - 1) / total;
+}
+__host__ __device__ __forceinline__ int64_t decode_active_warps(int64_t total, int64_t tpu, int64_t launched) {
+  int64_t nw = launched < total ? launched : total;
+  // every unit must be covered by at most kMaxSeg warps
+  int64_t min_tiles = (tpu + (kMaxSeg - 2)) / (kMaxSeg - 1);
+  if (min_tiles < 1) min_tiles = 1;
+  int64_t cap = total / min_tiles;
+  if (cap < 1) cap = 1;
+  return nw < cap ? nw : cap;
+}
+
+// --- element conversions ---
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f32(float x) { return x; }
+  static __device__ __forceinline__ float from_f32(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f32(float x) { return __float2bfloat16_rn(x); }
+};
+
+// Unpack 16 bytes (one uint4) into fp32 values.
+__device__ __forceinline__ void unpack16(const uint4& r, float* out, float) {
+  out[0] = __uint_as_float(r.x); out[1] = __uint_as_float(r.y);
+  out[2] = __uint_as_float(r.z); out[3] = __uint_as_float(r.w);
+}
+__device__ __forceinline__ void unpack16(const uint4& r, float* out, __nv_bfloat16) {
+  out[0] = __uint_as_float(r.x << 16); out[1] = __uint_as_float(r.x & 0xffff0000u);
+  out[2] = __uint_as_float(r.y << 16); out[3] = __uint_as_float(r.y & 0xffff0000u);
+  out[4] = __uint_as_float(r.z << 16); out[5] = __uint_as_float(r.z & 0xffff0000u);
+  out[6] = __uint_as_float(r.w << 16); out[7] = __uint_as_float(r.w & 0xffff0000u);
+}
+
+// --- mbarrier / bulk-copy wrappers (sm_90+ PTX, used here on sm_100a) ---
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+               :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: returns false (and the caller records DEVERR_TIMEOUT) when the
+// phase does not complete within kWaitLimitNs of wall time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+// One contiguous global -> shared bulk copy (no multicast), completion counted
+// in bytes on the mbarrier.  dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void set_error(int32_t* err, int32_t bits) {
+  atomicOr(err, bits);
+}
+
+// Scorer: s = w2 . relu(W1 x + b1) + b2 for x = [k; v] of one slot row
+// (KVpop page §E.1 headwise inputs, §E.2 stateless MLP scorer).  Accumulated
+// in fp64 (the inputs and fp32 weights are exact in fp64) and rounded once to
+// fp32, the ranking precision (§F).  Called by a whole CTA; `xs` is shared
+// scratch of 2d floats, `red` shared scratch of at least blockDim.x/32
+// doubles.  Returns the score in every thread.
+template <typename T>
+__device__ float mlp_score_block(const T* row, int d, const float* w1, const float* b1, const float* w2,
+                                 float b2, int hidden, float* xs, double* red) {
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarp = nthr >> 5;
+  for (int i = tid; i < 2 * d; i += nthr) xs[i] = Elem<T>::to_f32(row[i]);
+  __syncthreads();
+  double part = 0.0;
+  for (int j = warp; j < hidden; j += nwarp) {
+    const float* wr = w1 + static_cast<size_t>(j) * 2 * d;
+    double acc = 0.0;
+    for (int i = lane; i < 2 * d; i += 32) acc = fma(static_cast<double>(wr[i]), static_cast<double>(xs[i]), acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const double h = fmax(acc + static_cast<double>(b1[j]), 0.0);
+    part = fma(static_cast<double>(w2[j]), h, part);   // identical in all lanes
+  }
+  if (lane == 0) red[warp] = part;
+  __syncthreads();
+  double s = static_cast<double>(b2);
+  for (int w = 0; w < nwarp; ++w) s += red[w];
+  __syncthreads();
+  return static_cast<float>(s);
+}
+
+// Decode kernel scratch (split-K partials), shared by the layers of a handle.
+struct DecodeScratch {
+  float* part_acc;    // [units][kMaxSeg][G][d]
+  float* part_ml;     // [units][kMaxSeg][G][2]
+  int32_t* ticket;    // [units]
+};
+
+// Kernel launchers (defined in the .cu files).
+int launch_update(const LayerArgs& a, int dtype, const void* k_new, const void* v_new,
+                  const float* ext_score, cudaStream_t st);
+int launch_attention(const LayerArgs& a, int dtype, const DecodeScratch& sc, const void* q, void* out,
+                     int num_sms, cudaStream_t st);
+
+struct PrefillScratch {
+  float* new_score;   // [units][cap]
+  int32_t* tgt;       // [units][K]
+  int cap;            // capacity of newly eligible tokens per unit per chunk
+};
+int launch_prefill(const LayerArgs& a, int dtype, const PrefillScratch& ps, const void* k, const void* v,
+                   int n_tokens, int n_seen_before, int n_topk_before, const float* ext_scores,
+                   cudaStream_t st);
+
+}  // namespace kvpop

@@ -1,0 +1,389 @@
+// Prefill builder: appends a chunk of prompt tokens to the KVpop cache.
+//
+// After a chunk the cache holds exactly what the running prefix top-k rule
+// (KVpop page §I Pseudocode, §C.1 Mask Definition) gives at the chunk's last
+// token: positions < S in the sink slots, the last W tokens in the window
+// ring, the D tokens before them in the staging ring, and the K best tokens
+// (key = (score, -position), fp32 scores as in §F) among all tokens that have
+// left the window/staging, in the long-range slots.
+//
+// Placement: long-range tokens that survive the chunk keep their slots; the
+// admitted newcomers, in ascending position, take the free-or-vacated
+// long-range slots in ascending slot order (for a first chunk this is
+// ascending position order).
+//
+// Kernels, in stream order:
+//   P1 score:  MLP score of every newly eligible token (or caller's score),
+//              as a small register-blocked GEMM with W1 held in smem, fp64
+//              accumulation rounded once to fp32.
+//   P2 select: per unit, radix select of the K-th largest 64-bit key among the
+//              current long-range tokens and the newcomers, then slot
+//              assignment by block prefix sums and row copies.
+//   P3 move:   window tokens that enter the staging ring move there.
+//   P4 write:  chunk tokens go to their sink / window / staging slots.
+#include "kvpop_internal.cuh"
+
+namespace kvpop {
+
+namespace {
+
+struct ChunkGeom {
+  int n0, n1, e0, e1, c0;  // tokens before/after, newly eligible [e0, e1), long-range used before
+};
+
+// Where does token t's row live during this chunk?  (t < n0: cache ring)
+template <typename T>
+__device__ __forceinline__ const uint8_t* token_row(const LayerArgs& a, const ChunkGeom& cg, int u, int t,
+                                                    const T* k, const T* v, int n, const uint8_t*& vsrc) {
+  if (t >= cg.n0) {
+    const size_t off = (static_cast<size_t>(u) * n + (t - cg.n0)) * a.d;
+    vsrc = reinterpret_cast<const uint8_t*>(v + off);
+    return reinterpret_cast<const uint8_t*>(k + off);
+  }
+  const int slot = (t >= cg.n0 - a.W) ? window_slot(t, a.S, a.W) : staging_slot(t, a.S, a.W, a.D);
+  const uint8_t* row = a.kv + (static_cast<size_t>(u) * a.NS + slot) * a.row_bytes;
+  vsrc = row + a.d * sizeof(T);
+  return row;
+}
+
+template <typename T>
+__device__ __forceinline__ int token_slot_in_cache(const LayerArgs& a, const ChunkGeom& cg, int t) {
+  return (t >= cg.n0 - a.W) ? window_slot(t, a.S, a.W) : staging_slot(t, a.S, a.W, a.D);
+}
+
+// ---------------- P1: scoring ----------------
+constexpr int kScoreThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k,
+                                                              const T* __restrict__ v, int n,
+                                                              const float* __restrict__ ext,
+                                                              float* __restrict__ out, int cap) {
+  extern __shared__ float sm[];
+  const int u = blockIdx.y;
+  const int h = u % a.Hkv;
+  const int n_new = cg.e1 - cg.e0;
+  const int d2 = 2 * a.d;
+  const int HQ = a.hidden / 4;                 // threads per token quad
+  const int TT = 4 * (kScoreThreads / HQ);     // tokens per tile
+  const int tok0 = blockIdx.x * TT;
+  if (tok0 >= n_new) return;
+  const int ntok = min(TT, n_new - tok0);
+  const int tid = threadIdx.x;
+
+  if (a.flags & FLAG_EXTERNAL_SCORES) {
+    for (int i = tid; i < ntok; i += blockDim.x) {
+      const int t = cg.e0 + tok0 + i;
+      float s;
+      if (t >= cg.n0) s = ext[static_cast<size_t>(u) * n + (t - cg.n0)];
+      else s = a.score[static_cast<size_t>(u) * a.NS + token_slot_in_cache<T>(a, cg, t)];
+      out[static_cast<size_t>(u) * cap + tok0 + i] = s;
+    }
+    return;
+  }
+
+  float* Ws = sm;                          // [d2][hidden]  (W1 transposed)
+  float* Xs = sm + d2 * a.hidden;          // [TT][d2]
+  const float* w1 = a.w1 + static_cast<size_t>(h) * a.hidden * d2;
+  for (int idx = tid; idx < a.hidden * d2; idx += blockDim.x) {
+    const int j = idx / d2, i = idx % d2;
+    Ws[i * a.hidden + j] = w1[idx];
+  }
+  for (int idx = tid; idx < TT * d2; idx += blockDim.x) {
+    const int tt = idx / d2, i = idx % d2;
+    float x = 0.f;
+    if (tt < ntok) {
+      const int t = cg.e0 + tok0 + tt;
+      const uint8_t* vs;
+      const uint8_t* ks = token_row<T>(a, cg, u, t, k, v, n, vs);
+      x = (i < a.d) ? Elem<T>::to_f32(reinterpret_cast<const T*>(ks)[i])
+                    : Elem<T>::to_f32(reinterpret_cast<const T*>(vs)[i - a.d]);
+    }
+    Xs[tt * d2 + i] = x;
+  }
+  __syncthreads();
+  const int tq = tid / HQ, hq = tid % HQ;
+  // fp64 accumulation, one rounding to fp32 at the end (ranking precision)
+  double acc[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
+  for (int i = 0; i < d2; ++i) {
+    const float4 wv = *reinterpret_cast<const float4*>(Ws + i * a.hidden + 4 * hq);
+    const double w0 = wv.x, w1v = wv.y, w2v = wv.z, w3 = wv.w;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const double xv = Xs[(4 * tq + r) * d2 + i];
+      acc[r][0] = fma(xv, w0, acc[r][0]);
+      acc[r][1] = fma(xv, w1v, acc[r][1]);
+      acc[r][2] = fma(xv, w2v, acc[r][2]);
+      acc[r][3] = fma(xv, w3, acc[r][3]);
+    }
+  }
+  const float* b1 = a.b1 + static_cast<size_t>(h) * a.hidden;
+  const float* w2 = a.w2 + static_cast<size_t>(h) * a.hidden;
+  double part[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    part[r] = 0.0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      part[r] = fma(static_cast<double>(w2[4 * hq + c]),
+                    fmax(acc[r][c] + static_cast<double>(b1[4 * hq + c]), 0.0), part[r]);
+  }
+  // reduce over the HQ threads of a token quad (consecutive lanes, HQ | 32)
+  for (int off = 1; off < HQ; off <<= 1)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+  if (hq == 0) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int tt = 4 * tq + r;
+      if (tt < ntok) out[static_cast<size_t>(u) * cap + tok0 + tt] = static_cast<float>(part[r] + static_cast<double>(a.b2[h]));
+    }
+  }
+}
+
+// ---------------- P2: select + place ----------------
+constexpr int kSelThreads = 1024;
+
+// Exclusive block prefix sum of a 0/1 flag; returns the offset, sets *total.
+__device__ __forceinline__ int block_scan_flag(int flag, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const unsigned ball = __ballot_sync(0xffffffffu, flag);
+  const int in_warp = __popc(ball & ((1u << lane) - 1u));
+  if (lane == 0) warp_sums[warp] = __popc(ball);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int w = 0; w < nw; ++w) { const int c = warp_sums[w]; warp_sums[w] = run; run += c; }
+    warp_sums[nw] = run;
+  }
+  __syncthreads();
+  const int res = warp_sums[warp] + in_warp;
+  *total = warp_sums[nw];
+  __syncthreads();
+  return res;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k,
+                                                             const T* __restrict__ v, int n,
+                                                             const float* __restrict__ new_score, int cap,
+                                                             int32_t* __restrict__ tgt_all) {
+  __shared__ unsigned hist[256];
+  __shared__ int warp_sums[kSelThreads / 32 + 1];
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_need;
+  __shared__ int s_list_tok[kSelThreads];
+  __shared__ int s_list_slot[kSelThreads];
+
+  const int u = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int K = a.K;
+  const int base = topk_base(a.S, a.W, a.D);
+  const int n_new = cg.e1 - cg.e0;
+  const int c0 = cg.c0;
+  int32_t* pos = a.pos + static_cast<size_t>(u) * a.NS;
+  float* score = a.score + static_cast<size_t>(u) * a.NS;
+  const float* ns = new_score + static_cast<size_t>(u) * cap;
+  int32_t* tgt = tgt_all + static_cast<size_t>(u) * (K > 0 ? K : 1);
+  uint8_t* kv = a.kv + static_cast<size_t>(u) * a.NS * a.row_bytes;
+
+  if (tid == 0) {
+    a.state[4 * u + 0] = cg.n1;
+    a.state[4 * u + 1] = min(K, c0 + n_new);
+  }
+  if (n_new == 0 || K == 0) return;
+
+  const int ncand = c0 + n_new;
+  auto cand_key = [&](int i) -> unsigned long long {
+    if (i < c0) return rank_key(score[base + i], pos[base + i]);
+    return rank_key(ns[i - c0], cg.e0 + (i - c0));
+  };
+
+  unsigned long long thr = 0ull;   // admit keys >= thr
+  if (ncand > K) {
+    if (tid == 0) { s_prefix = 0ull; s_need = K; }
+    unsigned long long mask = 0ull;
+    for (int pass = 0; pass < 8; ++pass) {
+      const int shift = 56 - 8 * pass;
+      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0u;
+      __syncthreads();
+      const unsigned long long prefix = s_prefix;
+      for (int i = tid; i < ncand; i += blockDim.x) {
+        const unsigned long long key = cand_key(i);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255ull], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int need = s_need;
+        int cum = 0;
+        int sel = 0;
+        for (int dgt = 255; dgt >= 0; --dgt) {
+          const int c = static_cast<int>(hist[dgt]);
+          if (cum + c >= need) { sel = dgt; need -= cum; break; }
+          cum += c;
+        }
+        s_need = need;
+        s_prefix = prefix | (static_cast<unsigned long long>(sel) << shift);
+      }
+      mask |= 255ull << shift;
+      __syncthreads();
+    }
+    thr = s_prefix;
+  }
+
+  // target slots: free or vacated long-range slots, ascending
+  int n_tgt = 0;
+  for (int i0 = 0; i0 < K; i0 += blockDim.x) {
+    const int i = i0 + tid;
+    int flag = 0;
+    if (i < K) flag = (i >= c0) || (cand_key(i) < thr);
+    int total;
+    const int off = block_scan_flag(flag, warp_sums, &total);
+    if (flag) tgt[n_tgt + off] = base + i;
+    n_tgt += total;
+  }
+  __syncthreads();
+  // admitted newcomers, ascending position -> tgt[rank]
+  int n_adm = 0;
+  for (int r0 = 0; r0 < n_new; r0 += blockDim.x) {
+    const int r = r0 + tid;
+    int flag = 0;
+    if (r < n_new) flag = (ncand <= K) || (rank_key(ns[r], cg.e0 + r) >= thr);
+    int total;
+    const int off = block_scan_flag(flag, warp_sums, &total);
+    if (flag) {
+      s_list_tok[off] = cg.e0 + r;
+      s_list_slot[off] = __ldcg(&tgt[n_adm + off]);
+    }
+    __syncthreads();
+    // copy the rows: one warp per admitted token
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int j = warp; j < total; j += blockDim.x / 32) {
+      const int t = s_list_tok[j];
+      const int slot = s_list_slot[j];
+      const uint8_t* vs;
+      const uint8_t* ks = token_row<T>(a, cg, u, t, k, v, n, vs);
+      uint8_t* dst = kv + static_cast<size_t>(slot) * a.row_bytes;
+      const int half = a.d * sizeof(T);
+      for (int b = lane * 16; b < half; b += 32 * 16) {
+        *reinterpret_cast<uint4*>(dst + b) = *reinterpret_cast<const uint4*>(ks + b);
+        *reinterpret_cast<uint4*>(dst + half + b) = *reinterpret_cast<const uint4*>(vs + b);
+      }
+      if (lane == 0) {
+        pos[slot] = t;
+        score[slot] = ns[t - cg.e0];
+      }
+    }
+    n_adm += total;
+    __syncthreads();
+  }
+  // When the candidates overflow K every target slot is refilled
+  // (|targets| == |admitted| == K - survivors); while filling up, the
+  // admitted newcomers take the first free slots.
+  if ((a.flags & FLAG_DEBUG_CHECKS) && tid == 0) {
+    const bool bad = (ncand > K) ? (n_adm != n_tgt || n_adm > K) : (n_adm != n_new || n_adm > n_tgt);
+    if (bad) set_error(a.err, DEVERR_STATE_MISMATCH);
+  }
+}
+
+// ---------------- P3: window -> staging moves ----------------
+template <typename T>
+__global__ void move_kernel(LayerArgs a, ChunkGeom cg) {
+  const int u = blockIdx.x;
+  // window tokens before the chunk: [max(S, n0-W), n0); those in [n1-W-D, n1-W) now sit in staging
+  const int lo = max(max(a.S, cg.n0 - a.W), cg.n1 - a.W - a.D);
+  const int hi = min(cg.n0, cg.n1 - a.W);
+  uint8_t* kv = a.kv + static_cast<size_t>(u) * a.NS * a.row_bytes;
+  int32_t* pos = a.pos + static_cast<size_t>(u) * a.NS;
+  float* score = a.score + static_cast<size_t>(u) * a.NS;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = lo + warp; t < hi; t += blockDim.x / 32) {
+    const int src = window_slot(t, a.S, a.W), dst = staging_slot(t, a.S, a.W, a.D);
+    for (int b = lane * 16; b < a.row_bytes; b += 32 * 16)
+      *reinterpret_cast<uint4*>(kv + static_cast<size_t>(dst) * a.row_bytes + b) =
+          *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(src) * a.row_bytes + b);
+    if (lane == 0) { pos[dst] = t; score[dst] = score[src]; }
+  }
+}
+
+// ---------------- P4: chunk tokens -> sink / window / staging ----------------
+template <typename T>
+__global__ void write_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k, const T* __restrict__ v, int n,
+                             const float* __restrict__ ext) {
+  const int u = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = cg.n0 + blockIdx.x * (blockDim.x / 32) + warp;
+  if (t >= cg.n1) return;
+  int slot;
+  if (t < a.S) slot = t;
+  else if (t >= cg.n1 - a.W) slot = window_slot(t, a.S, a.W);
+  else if (a.D > 0 && t >= cg.n1 - a.W - a.D) slot = staging_slot(t, a.S, a.W, a.D);
+  else return;  // already eligible: handled by the select step
+  uint8_t* dst = a.kv + (static_cast<size_t>(u) * a.NS + slot) * a.row_bytes;
+  const size_t off = (static_cast<size_t>(u) * n + (t - cg.n0)) * a.d;
+  const uint8_t* ks = reinterpret_cast<const uint8_t*>(k + off);
+  const uint8_t* vs = reinterpret_cast<const uint8_t*>(v + off);
+  const int half = a.d * sizeof(T);
+  for (int b = lane * 16; b < half; b += 32 * 16) {
+    *reinterpret_cast<uint4*>(dst + b) = *reinterpret_cast<const uint4*>(ks + b);
+    *reinterpret_cast<uint4*>(dst + half + b) = *reinterpret_cast<const uint4*>(vs + b);
+  }
+  if (lane == 0) {
+    a.pos[static_cast<size_t>(u) * a.NS + slot] = t;
+    a.score[static_cast<size_t>(u) * a.NS + slot] =
+        (a.flags & FLAG_EXTERNAL_SCORES) ? ext[static_cast<size_t>(u) * n + (t - cg.n0)] : 0.f;
+  }
+}
+
+template <typename T>
+int launch_prefill_t(const LayerArgs& a, const PrefillScratch& ps, const T* k, const T* v, int n, int n0, int c0,
+                     const float* ext, cudaStream_t st) {
+  ChunkGeom cg;
+  cg.n0 = n0;
+  cg.n1 = n0 + n;
+  cg.e0 = max(a.S, n0 - a.W - a.D);
+  cg.e1 = max(a.S, cg.n1 - a.W - a.D);
+  cg.c0 = c0;
+  const int n_new = cg.e1 - cg.e0;
+  if (n_new > ps.cap) return -2;
+  if (n_new > 0) {
+    const int HQ = a.hidden / 4;
+    const int TT = 4 * (kScoreThreads / HQ);
+    const size_t smem = (a.flags & FLAG_EXTERNAL_SCORES) ? 0
+                        : (static_cast<size_t>(2 * a.d) * a.hidden + static_cast<size_t>(TT) * 2 * a.d) * sizeof(float);
+    static size_t smem_set = 0;
+    if (smem > 48 * 1024 && smem > smem_set) {
+      if (cudaFuncSetAttribute(score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return -1;
+      smem_set = smem;
+    }
+    dim3 grid((n_new + TT - 1) / TT, a.units);
+    score_kernel<T><<<grid, kScoreThreads, smem, st>>>(a, cg, k, v, n, ext, ps.new_score, ps.cap);
+  }
+  select_kernel<T><<<a.units, kSelThreads, 0, st>>>(a, cg, k, v, n, ps.new_score, ps.cap, ps.tgt);
+  if (a.D > 0) move_kernel<T><<<a.units, 256, 0, st>>>(a, cg);
+  if (n > 0) {
+    dim3 grid((n + 7) / 8, a.units);
+    write_kernel<T><<<grid, 256, 0, st>>>(a, cg, k, v, n, ext);
+  }
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace
+
+int launch_prefill(const LayerArgs& a, int dtype, const PrefillScratch& ps, const void* k, const void* v,
+                   int n_tokens, int n_seen_before, int n_topk_before, const float* ext_scores, cudaStream_t st) {
+  if (dtype == 0)
+    return launch_prefill_t<float>(a, ps, static_cast<const float*>(k), static_cast<const float*>(v), n_tokens,
+                                   n_seen_before, n_topk_before, ext_scores, st);
+  return launch_prefill_t<__nv_bfloat16>(a, ps, static_cast<const __nv_bfloat16*>(k),
+                                         static_cast<const __nv_bfloat16*>(v), n_tokens, n_seen_before,
+                                         n_topk_before, ext_scores, st);
+}
+
+}  // namespace kvpop

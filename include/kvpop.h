@@ -1,0 +1,195 @@
+/*
+ * kvpop.h -- C ABI of the KVpop fixed-budget KV cache, decode-time hot path.
+ *
+ * Method: "KVpop -- Key-Value Cache Compression with Predictive Online
+ * Pruning" (summary page of arXiv 2607.05061v2).  Every KV head keeps a
+ * bounded cache of budget B = S + W + K tokens, the same for every head:
+ * S attention-sink tokens, a protected window of the W most recent tokens,
+ * and K long-range slots holding the running top-k of the tokens that have
+ * left the window, ranked by a small headwise scorer on [k; v]
+ * (page §3 "Fixed-budget pruning", §C.1 "Mask Definition", §E.1-§E.2,
+ * §I "KVpop Pseudocode").  Optional delayed scoring (page §3 "Stateful
+ * scorers", §E.4 "Delayed Readout") is a D-slot staging ring between the
+ * window and the long-range slots: a token is scored D steps after it leaves
+ * the window.  Staged tokens stay cached and are attended.
+ *
+ * Conventions for every call:
+ *  - Return value: KVPOP_OK (0) or a negative KVPOP_ERR_* code.  Nothing
+ *    throws or aborts across the ABI.  Arguments are validated before any
+ *    work is enqueued; a call that fails validation enqueues nothing.
+ *  - Device pointers point to memory on the device the handle was created on.
+ *    The library never allocates or frees device memory: the caller owns all
+ *    of it and lends it for the duration of the call (inputs) or the handle's
+ *    lifetime (the cache buffer).
+ *  - Work is asynchronous on the caller's CUDA stream (`stream`, a
+ *    cudaStream_t; NULL = legacy default stream).  Only kvpop_create,
+ *    kvpop_inspect and kvpop_get_error synchronise.
+ *  - Calls on one handle must be ordered on one stream (or by the caller's
+ *    events): the handle's split-K scratch is shared by its layers.
+ *  - All batch rows share one sequence length.  Layers are independent and
+ *    each keeps its own position counter (on the device).
+ *  - Element type of q, k, v, the cache and the output: config.dtype.
+ *    Scores are fp32 (the page, §F, ranks and selects in float32).
+ */
+#ifndef KVPOP_H
+#define KVPOP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define KVPOP_OK 0
+#define KVPOP_ERR_INVALID_ARG -1      /* null pointer, out-of-range layer, bad flag */
+#define KVPOP_ERR_BAD_SHAPE -2        /* shape combination not valid / not built */
+#define KVPOP_ERR_ORDER -3            /* call out of order (e.g. prefill after decode) */
+#define KVPOP_ERR_CONTEXT_OVERFLOW -4 /* position counter would pass max_context */
+#define KVPOP_ERR_CUDA -5             /* a CUDA runtime call failed */
+#define KVPOP_ERR_DEVICE -6           /* a kernel recorded an error (see kvpop_get_error) */
+#define KVPOP_ERR_TIMEOUT -7          /* a bounded device-side wait gave up */
+
+/* Element types. */
+#define KVPOP_DTYPE_F32 0
+#define KVPOP_DTYPE_BF16 1
+
+/* Flags. */
+#define KVPOP_FLAG_EXTERNAL_SCORES 1u /* caller supplies every token's score instead of the MLP */
+#define KVPOP_FLAG_DEBUG_CHECKS 2u    /* kernels check slot bookkeeping and NaN scores */
+
+/* Device error bits reported by kvpop_get_error. */
+#define KVPOP_DEVERR_CONTEXT_OVERFLOW 1
+#define KVPOP_DEVERR_TIMEOUT 2
+#define KVPOP_DEVERR_BAD_INDEX 4
+#define KVPOP_DEVERR_NAN_SCORE 8
+#define KVPOP_DEVERR_STATE_MISMATCH 16
+
+typedef struct kvpop_config {
+  int32_t batch;        /* batch rows b >= 1 */
+  int32_t n_layers;     /* layers L >= 1 */
+  int32_t n_q_heads;    /* query heads Hq, a multiple of n_kv_heads (GQA) */
+  int32_t n_kv_heads;   /* KV heads Hkv >= 1 */
+  int32_t head_dim;     /* d: 64 or 128 (bf16), 64 (fp32) */
+  int32_t sinks;        /* S >= 0 */
+  int32_t window;       /* W >= 1 */
+  int32_t topk;         /* K >= 0 long-range slots; budget B = S + W + K */
+  int32_t delay;        /* D >= 0 staging slots for delayed scoring (outside B) */
+  int32_t ref_context;  /* prompt length the compression ratio is quoted against; 0 = no check */
+  float compression_ratio; /* redundant, checked: |(1 - CR) * ref_context - B| <= 0.5 */
+  int32_t max_context;  /* positions must stay below this (int32 positions) */
+  int32_t max_prefill_chunk; /* largest n_tokens of one kvpop_prefill call */
+  int32_t dtype;        /* KVPOP_DTYPE_F32 or KVPOP_DTYPE_BF16 */
+  int32_t scorer_hidden; /* MLP 2d -> hidden -> 1; hidden in {32, 64, 128} */
+  /* Scorer weights, device fp32, borrowed for the handle's lifetime
+   * (may be NULL with KVPOP_FLAG_EXTERNAL_SCORES):
+   *   w1 [L][Hkv][hidden][2d]  (input x = [k; v], page §E.1)
+   *   b1 [L][Hkv][hidden], w2 [L][Hkv][hidden], b2 [L][Hkv]
+   * score = w2 . relu(W1 x + b1) + b2 (page §E.2, stateless MLP scorer). */
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+  uint32_t flags;       /* KVPOP_FLAG_* */
+} kvpop_config;
+
+typedef struct kvpop_handle kvpop_handle;
+
+/* Offsets (bytes, from dev_mem) of the cache arrays, for inspection and tests.
+ * Layer l's arrays start at offset + l * *_layer_stride. */
+typedef struct kvpop_layout_info {
+  size_t kv_offset, kv_layer_stride;       /* [units][slots][2][d] (key row, value row) */
+  size_t pos_offset, pos_layer_stride;     /* int32 [units][slots], -1 = empty */
+  size_t score_offset, score_layer_stride; /* fp32 [units][slots] */
+  size_t state_offset, state_layer_stride; /* int32 [units][4] = {n_seen, n_topk, 0, 0} */
+  int32_t slots_per_unit;                  /* S + W + D + K */
+  int32_t units;                           /* batch * n_kv_heads; unit = b * Hkv + h */
+  int32_t row_bytes;                       /* 2 * d * sizeof(dtype) */
+  int32_t topk_base;                       /* first long-range slot, S + W + D */
+} kvpop_layout_info;
+
+/* Device bytes the caller must allocate for `cfg` (cache, slot metadata,
+ * split-K and prefill scratch).  Validates cfg.  Host only. */
+int kvpop_cache_bytes(const kvpop_config* cfg, size_t* bytes);
+
+/* Binds a caller-allocated device buffer (>= kvpop_cache_bytes, 256-byte
+ * aligned, on the current device) and initialises it (empty cache,
+ * synchronously).  The buffer must outlive the handle.  *out receives the
+ * handle (host memory owned by the library until kvpop_destroy). */
+int kvpop_create(const kvpop_config* cfg, void* dev_mem, size_t bytes, kvpop_handle** out);
+
+/* Appends a chunk of n_tokens prompt tokens to layer `layer` (positions
+ * n_seen .. n_seen + n_tokens - 1).  k, v: device [b][Hkv][n_tokens][d].
+ * ext_scores: device fp32 [b][Hkv][n_tokens] (required with
+ * KVPOP_FLAG_EXTERNAL_SCORES, ignored otherwise).  After the call the layer
+ * holds the running prefix top-k state at its last token (page §I): the
+ * long-range slots keep the K best eligible tokens; survivors keep their
+ * slots and admitted tokens fill free/vacated slots in ascending order.
+ * Must precede the layer's first decode step (else KVPOP_ERR_ORDER);
+ * 0 <= n_tokens <= max_prefill_chunk. */
+int kvpop_prefill(kvpop_handle* h, int32_t layer, const void* k, const void* v, int32_t n_tokens,
+                  const float* ext_scores, void* stream);
+
+/* One decode step of one layer for all batch rows.  With p = the layer's
+ * position counter:
+ *  1. window append and boundary update: the token leaving the window (after
+ *     D staging steps when D > 0) is scored by the MLP on [k; v] (or its
+ *     caller score) and replaces the minimum of the long-range set only if
+ *     its key (score, -position) is strictly larger; while the long-range set
+ *     is not full it takes the next free slot; the new token's k/v is written
+ *     to its window slot;
+ *  2. GQA attention of the new queries over all occupied slots (softmax,
+ *     scale 1/sqrt(d), fp32 accumulation).
+ * q: device [b][Hq][d]; k_new, v_new: device [b][Hkv][d]; out: device
+ * [b][Hq][d] (same element type); ext_score: device fp32 [b][Hkv], the score
+ * of the token being appended (required with KVPOP_FLAG_EXTERNAL_SCORES).
+ * The position counter then advances by one. */
+int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void* k_new, const void* v_new,
+                      void* out, const float* ext_score, void* stream);
+
+/* The two halves of kvpop_decode_step, for callers that schedule them apart
+ * (same arguments and semantics; append must precede attend for each step).
+ * kvpop_decode_append: step 1 only (window append, boundary scoring and
+ * argmin-replace); advances the position counter.
+ * kvpop_decode_attend: step 2 only, over the cache as it stands (the query of
+ * the token appended last).  Calling attend again without an append repeats
+ * the same attention. */
+int kvpop_decode_append(kvpop_handle* h, int32_t layer, const void* k_new, const void* v_new,
+                        const float* ext_score, void* stream);
+int kvpop_decode_attend(kvpop_handle* h, int32_t layer, const void* q, void* out, void* stream);
+
+/* Copies layer `layer`'s slot -> position map (int32 [units][slots]), slot
+ * scores (fp32 [units][slots]) and per-unit state (int32 [units][4]) to HOST
+ * buffers; any of them may be NULL.  Synchronises `stream`.  For tests and
+ * debugging. */
+int kvpop_inspect(kvpop_handle* h, int32_t layer, int32_t* pos_out, float* score_out, int32_t* state_out,
+                  void* stream);
+
+/* Fills *out with the layout of the device buffer. */
+int kvpop_get_layout(const kvpop_handle* h, kvpop_layout_info* out);
+
+/* Synchronises the device and reads the device error word.  Returns KVPOP_OK
+ * if no kernel recorded an error, KVPOP_ERR_CONTEXT_OVERFLOW / _TIMEOUT /
+ * _DEVICE otherwise (device_bits, if not NULL, receives the KVPOP_DEVERR_*
+ * bits), or KVPOP_ERR_CUDA if the device reported an asynchronous error. */
+int kvpop_get_error(kvpop_handle* h, int32_t* device_bits);
+
+/* Clears the device error word (asynchronously, on `stream`). */
+int kvpop_clear_error(kvpop_handle* h, void* stream);
+
+/* Test hook: ORs `bits` into the device error word on `stream`, so host-side
+ * failure handling can be exercised without making any kernel fail. */
+int kvpop_debug_poison_error(kvpop_handle* h, int32_t bits, void* stream);
+
+/* Releases the handle's host state.  Does not touch the device buffer. */
+int kvpop_destroy(kvpop_handle* h);
+
+/* Static description of a status code. */
+const char* kvpop_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVPOP_H */

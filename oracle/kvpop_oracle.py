@@ -237,6 +237,44 @@ class UnitResult:
     attended_counts: List[int]
 
 
+class OracleUnit:
+    """One (batch row, layer, KV head) unit stepped one decode token at a time.
+
+    k_all, v_all: [n_tokens][d] keys/values of every token the unit will see
+    (prompt, then decode tokens); scores: ranking score of every token.  The
+    constructor prefills P tokens (in `prefill_chunks` if given); step(q)
+    decodes the next token: slot-simulator update, brute-force running top-k
+    at the new position, attention of q [G][d] over the attended set.
+    """
+
+    def __init__(self, k_all, v_all, scores, S, W, D, K, P, prefill_chunks=None, check_simulator=True):
+        self.k_all, self.v_all, self.scores = k_all, v_all, scores
+        self.S, self.W, self.D, self.K, self.P = S, W, D, K, P
+        self.check = check_simulator
+        self.state = SlotState(S, W, D, K)
+        chunks = list(prefill_chunks) if prefill_chunks else ([P] if P > 0 else [])
+        assert sum(chunks) == P
+        for c in chunks:
+            self.state.append_chunk(c, scores)
+        self.topk = running_topk(scores, P - 1, S, W, D, K) if P > 0 else []
+        if check_simulator and P > 0:
+            assert self.state.topk_positions() == self.topk, "slot simulator disagrees with brute force"
+        self.q = P  # position of the next decode token
+
+    def step(self, qvec):
+        q = self.q
+        S, W, D, K = self.S, self.W, self.D, self.K
+        self.state.decode(self.scores)
+        T = running_topk(self.scores, q, S, W, D, K)
+        if self.check:
+            assert self.state.topk_positions() == T, f"slot simulator disagrees at q={q}"
+        A = attended_positions(q, S, W, D, T)
+        o, w = attention(qvec, self.k_all[A], self.v_all[A])
+        self.topk = T
+        self.q = q + 1
+        return o, w, T, A
+
+
 def run_unit(k_all: np.ndarray, v_all: np.ndarray, q_steps: np.ndarray, scores: Sequence[float],
              S: int, W: int, D: int, K: int, P: int,
              prefill_chunks: Optional[Sequence[int]] = None,
@@ -250,28 +288,16 @@ def run_unit(k_all: np.ndarray, v_all: np.ndarray, q_steps: np.ndarray, scores: 
     simulator runs beside it and must hold the same long-range set.
     """
     n_steps = len(q_steps)
-    state = SlotState(S, W, D, K)
-    chunks = list(prefill_chunks) if prefill_chunks else ([P] if P > 0 else [])
-    assert sum(chunks) == P
-    for c in chunks:
-        state.append_chunk(c, scores)
-    slot_maps = [list(state.slot_pos)]
-    topk_sets = [running_topk(scores, P - 1, S, W, D, K)] if P > 0 else [[]]
-    if check_simulator and P > 0:
-        assert state.topk_positions() == topk_sets[0], "slot simulator disagrees with brute force"
+    unit = OracleUnit(k_all, v_all, scores, S, W, D, K, P, prefill_chunks, check_simulator)
+    slot_maps = [list(unit.state.slot_pos)]
+    topk_sets = [list(unit.topk)]
     outs, sums, counts = [], [], []
     for i in range(n_steps):
-        q = P + i
-        state.decode(scores)
-        T = running_topk(scores, q, S, W, D, K)
-        if check_simulator:
-            assert state.topk_positions() == T, f"slot simulator disagrees at q={q}"
-        A = attended_positions(q, S, W, D, T)
-        o, w = attention(q_steps[i], k_all[A], v_all[A])
+        o, w, T, A = unit.step(q_steps[i])
         outs.append(o)
         sums.append(w.sum(axis=-1))
         counts.append(len(A))
-        slot_maps.append(list(state.slot_pos))
+        slot_maps.append(list(unit.state.slot_pos))
         topk_sets.append(T)
     G = q_steps.shape[1] if n_steps else 0
     d = k_all.shape[-1]

@@ -1,0 +1,110 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import kvpop_workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+gh = pytest.importorskip("gpu_harness")
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def test_tiny_workload_full_run_matches_oracle():
+    """The tiny fp32 workload end to end: 128-token prefill, 128 decode steps,
+    MLP scorer on the GPU; outputs within fp32 tolerance at every step, GPU
+    scores within 1e-4 relative, long-range sets equal (up to near-ties)."""
+    _need_gpu()
+    w = wl.TINY
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode)
+    for unit in range(w.batch * w.n_kv_heads):
+        gh.check_unit(run, 0, unit, exact_slots=False, atol=gh.F32_ATOL)
+
+
+@pytest.mark.parametrize("dtype,d,hq,hkv", [("f32", 64, 4, 2), ("bf16", 64, 8, 2), ("bf16", 128, 8, 2),
+                                            ("bf16", 128, 4, 4), ("bf16", 64, 16, 2)])
+@pytest.mark.parametrize("S,W,D,K", [(4, 16, 0, 44), (2, 8, 5, 20), (0, 1, 0, 7), (3, 4, 0, 0)])
+def test_external_scores_bit_exact_slots(dtype, d, hq, hkv, S, W, D, K):
+    """Identical (tie-heavy) score arrays on both sides: the slot -> position
+    map must equal the oracle's slot simulator bit for bit at every step."""
+    _need_gpu()
+    w = wl.Workload("ext_case", batch=3, n_layers=2, n_q_heads=hq, n_kv_heads=hkv, head_dim=d, dtype=dtype,
+                    sinks=S, window=W, topk=K, delay=D, prefill=57, decode=40, scorer_hidden=32,
+                    heavy_hitter_frac=0.02 if dtype == "bf16" else 0.0)
+    run = gh.run_gpu(w, n_layers=2, n_steps=w.decode, external=True, tie_levels=3, layers_to_keep=(1,))
+    atol = gh.F32_ATOL if dtype == "f32" else gh.BF16_ATOL
+    for unit in range(w.batch * w.n_kv_heads):
+        gh.check_unit(run, 1, unit, exact_slots=True, atol=atol)
+
+
+@pytest.mark.parametrize("chunks", [[10, 30, 17], [1] * 12 + [45], [56, 1]])
+def test_chunked_prefill_bit_exact(chunks):
+    """Prefill in chunks: survivors keep their slots, newcomers fill free or
+    vacated slots in ascending order; then decode continues exactly."""
+    _need_gpu()
+    w = wl.Workload("chunk_case", batch=2, n_layers=1, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=3, window=6, topk=9, delay=2, prefill=sum(chunks), decode=20, scorer_hidden=64)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, external=True, tie_levels=2, chunks=chunks)
+    for unit in range(w.batch * w.n_kv_heads):
+        gh.check_unit(run, 0, unit, exact_slots=True, atol=gh.BF16_ATOL, chunks=chunks)
+
+
+def test_budget_covering_context_is_dense_attention():
+    """Budget >= context: every token is attended (dense causal attention)."""
+    _need_gpu()
+    w = wl.Workload("dense_case", batch=2, n_layers=1, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=4, window=32, topk=300, delay=0, prefill=100, decode=60, scorer_hidden=64,
+                    heavy_hitter_frac=0.02)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode)
+    for unit in range(4):
+        res = gh.check_unit(run, 0, unit, exact_slots=False, atol=gh.BF16_ATOL)
+        assert res.attended_counts == [w.prefill + i + 1 for i in range(w.decode)]
+
+
+def test_decode_from_empty_cache():
+    """No prompt at all: sinks, window and long-range slots fill during decode."""
+    _need_gpu()
+    w = wl.Workload("empty_case", batch=2, n_layers=1, n_q_heads=4, n_kv_heads=2, head_dim=64, dtype="f32",
+                    sinks=4, window=8, topk=10, delay=3, prefill=0, decode=50, scorer_hidden=32)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, external=True, tie_levels=3)
+    for unit in range(4):
+        gh.check_unit(run, 0, unit, exact_slots=True, atol=gh.F32_ATOL, chunks=[])
+
+
+def test_many_segments_per_unit_merge():
+    """Few units with long caches: each unit's slots are split over many
+    consumer warps, so the split-K merge (atomic ticket, LSE combine) runs."""
+    _need_gpu()
+    w = wl.Workload("merge_case", batch=1, n_layers=1, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=4, window=64, topk=1980, delay=0, prefill=2600, decode=6, scorer_hidden=64,
+                    heavy_hitter_frac=0.02)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode)
+    for unit in range(2):
+        gh.check_unit(run, 0, unit, exact_slots=False, atol=gh.BF16_ATOL)
+
+
+def test_nonfinite_free_outputs_and_rows_hold_tokens():
+    """Every occupied slot row holds exactly the k/v of the token its position
+    says (checks the in-place copies of append, staging move and replace)."""
+    _need_gpu()
+    w = wl.Workload("rows_case", batch=2, n_layers=1, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=2, window=5, topk=11, delay=3, prefill=40, decode=25, scorer_hidden=64)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, external=True, tie_levels=4)
+    rows = run.cache.kv_rows(0).cpu()
+    pos, _, state = run.cache.inspect(0)
+    for unit in range(4):
+        k_all, v_all, _ = gh.unit_inputs(run, 0, unit)
+        for slot, p in enumerate(pos[unit]):
+            if p < 0:
+                continue
+            r = rows[unit, slot].view(torch.bfloat16).double().numpy()
+            np.testing.assert_array_equal(r[:128], k_all[p])
+            np.testing.assert_array_equal(r[128:], v_all[p])
+        assert state[unit][0] == w.prefill + w.decode
+    for o in run.outs[0]:
+        assert torch.isfinite(o).all()
