@@ -2,9 +2,9 @@
 """KVpop decode benchmark on B200: decode tokens/s and achieved HBM bandwidth.
 
 One step = one KVpop decode step of every layer of the workload for every
-batch row: per layer, window append + boundary scoring + argmin-replace
-(kvpop_decode_append) and GQA attention over the bounded cache
-(kvpop_decode_attend), through the C ABI.  Default workload: Qwen3-4B-shaped,
+batch row: per layer one kvpop_decode_step call (window append, boundary
+scoring, argmin-replace and GQA attention over the bounded cache, fused in one
+kernel launch), through the C ABI.  Default workload: Qwen3-4B-shaped,
 87.5% compression (36 layers, 32 q / 8 kv heads, d 128, bf16, batch 64,
 budget 1024 = 4 sinks + 128 window + 892 long-range, prompt 8192).  Data are
 synthetic (seeded), shaped like the pages' workloads; the cache (9.7 GB) is
@@ -273,10 +273,9 @@ def run_gpu(args, w, rank, world, torch):
     def one_step(i, ev=None):
         j = i % NI
         for layer in range(L):
-            cache.decode_append(layer, ks[layer][j], vs[layer][j], stream=stream)
             if ev is not None:
                 ev[0][layer].record(stream)
-            cache.decode_attend(layer, qs[layer][j], outs[layer], stream=stream)
+            cache.decode_step(layer, qs[layer][j], ks[layer][j], vs[layer][j], outs[layer], stream=stream)
             if ev is not None:
                 ev[1][layer].record(stream)
 
@@ -325,7 +324,7 @@ def run_gpu(args, w, rank, world, torch):
     peak, peak_kind = measured_peaks()
     sbytes = step_bytes(w)
     step_gbs = sbytes * args.steps / (elapsed_ms / 1e3) / 1e9
-    abytes = attention_bytes(w)
+    abytes = sbytes // L   # one fused launch = one layer's share of the step
     attn_mean_ms = statistics.fmean(attn_ms)
     attn_gbs = abytes / (attn_mean_ms / 1e3) / 1e9
 
@@ -345,11 +344,12 @@ def run_gpu(args, w, rank, world, torch):
                    "input_sets": NI},
         "hbm": {"step_bytes": sbytes, "achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
                 "frac_of_8tbs": step_gbs / 8000.0, "peak_kind": peak_kind},
-        "roofline": {"kernel": "decode_attention_kernel<bf16,128,4>", "bound": "hbm", "achieved": attn_gbs,
+        "roofline": {"kernel": "decode_kernel<bf16,128,4,8,3> (fused append + attend, one launch per layer)",
+                     "bound": "hbm", "achieved": attn_gbs,
                      "peak": peak, "unit": "GB/s", "frac": attn_gbs / peak, "traffic": None,
                      "bytes_per_launch": abytes, "mean_launch_us": attn_mean_ms * 1e3,
                      "launches": len(attn_ms), "peak_kind": peak_kind},
-        "gpu_launches": 2 * L * args.steps,
+        "gpu_launches": L * args.steps,
         "clocks": clocks,
         "setup_s": setup_s,
     }
@@ -399,8 +399,7 @@ def run_e2e(args, w, cache, torch, world):
         if not first[b]:
             s_cmp.wait_event(ev_out[b])
         for layer in range(L):
-            cache.decode_append(layer, dk[b][layer], dv[b][layer], stream=s_cmp)
-            cache.decode_attend(layer, dq[b][layer], dout[b][layer], stream=s_cmp)
+            cache.decode_step(layer, dq[b][layer], dk[b][layer], dv[b][layer], dout[b][layer], stream=s_cmp)
         ev_cmp[b].record(s_cmp)
         s_out.wait_event(ev_cmp[b])
         with torch.cuda.stream(s_out):

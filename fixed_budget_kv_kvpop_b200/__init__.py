@@ -17,7 +17,8 @@ import os
 from typing import Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkvpop.so")
+# KVPOP_LIBRARY may point at another build of the same library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("KVPOP_LIBRARY") or os.path.join(_HERE, "libkvpop.so")
 
 KVPOP_OK = 0
 KVPOP_ERR_INVALID_ARG = -1

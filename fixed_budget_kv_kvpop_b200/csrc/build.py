@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
-SOURCES = ["kvpop_api.cu", "kvpop_update.cu", "kvpop_attention.cu", "kvpop_prefill.cu"]
+SOURCES = ["kvpop_api.cu", "kvpop_decode.cu", "kvpop_prefill.cu"]
 HEADERS = ["kvpop_internal.cuh", os.path.join(ROOT, "include", "kvpop.h")]
 OUT = os.path.join(PKG, "libkvpop.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -28,10 +28,10 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, out: str = OUT, defines=()) -> str:
+    if out == OUT and not defines and not force and not _stale():
         return OUT
-    cmd = [NVCC] + FLAGS + [os.path.join(HERE, s) for s in SOURCES] + ["-o", OUT + ".tmp"]
+    cmd = [NVCC] + FLAGS + ["-D" + d for d in defines] + [os.path.join(HERE, s) for s in SOURCES] + ["-o", out + ".tmp"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -40,8 +40,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed building libkvpop.so")
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(OUT + ".tmp", OUT)
-    return OUT
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":

@@ -8,10 +8,6 @@
 #include "../../include/kvpop.h"
 #include "kvpop_internal.cuh"
 
-namespace kvpop {
-int attention_supported(int dtype, int d, int G);
-}
-
 using namespace kvpop;
 
 namespace {
@@ -21,6 +17,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 struct Layout {
   int units, NS, G, esize, row_bytes, cap, kslots;
   size_t kv_off, kv_stride, pos_off, pos_stride, score_off, score_stride, state_off, state_stride;
+  size_t layer_off, dec_off, dec_stride;
   size_t pacc_off, pml_off, ticket_off, pre_score_off, pre_tgt_off, err_off, total;
 };
 
@@ -35,7 +32,7 @@ int validate(const kvpop_config* c) {
   if (c->max_context < 1 || c->max_prefill_chunk < 0) return KVPOP_ERR_BAD_SHAPE;
   if ((c->flags & ~(KVPOP_FLAG_EXTERNAL_SCORES | KVPOP_FLAG_DEBUG_CHECKS)) != 0) return KVPOP_ERR_INVALID_ARG;
   const int G = c->n_q_heads / c->n_kv_heads;
-  if (!attention_supported(c->dtype, c->head_dim, G)) return KVPOP_ERR_BAD_SHAPE;
+  if (!decode_supported(c->dtype, c->head_dim, G)) return KVPOP_ERR_BAD_SHAPE;
   if (!(c->flags & KVPOP_FLAG_EXTERNAL_SCORES)) {
     if (!hidden_supported(c->scorer_hidden)) return KVPOP_ERR_BAD_SHAPE;
     if (!c->w1 || !c->b1 || !c->w2 || !c->b2) return KVPOP_ERR_INVALID_ARG;
@@ -68,6 +65,9 @@ Layout make_layout(const kvpop_config* c) {
   L.score_off = off; off += layers * L.score_stride;
   L.state_stride = align256(units * 16);
   L.state_off = off; off += layers * L.state_stride;
+  L.layer_off = off; off += align256(layers * sizeof(LayerState));
+  L.dec_stride = align256(2 * units * sizeof(Decision));
+  L.dec_off = off; off += layers * L.dec_stride;
   L.pacc_off = off; off += align256(units * kMaxSeg * L.G * c->head_dim * 4);
   L.pml_off = off; off += align256(units * kMaxSeg * L.G * 2 * 4);
   L.ticket_off = off; off += align256(units * 4);
@@ -89,6 +89,7 @@ struct kvpop_handle {
   std::vector<int> n_seen;   // host mirror of each layer's position counter
   std::vector<int> n_topk;   // host mirror of each layer's long-range fill
   std::vector<char> decoding;
+  std::vector<CUtensorMap> maps;  // per layer: TMA view of the cache rows
 };
 
 namespace {
@@ -101,6 +102,8 @@ LayerArgs layer_args(const kvpop_handle* h, int layer) {
   a.pos = reinterpret_cast<int32_t*>(h->mem + L.pos_off + layer * L.pos_stride);
   a.score = reinterpret_cast<float*>(h->mem + L.score_off + layer * L.score_stride);
   a.state = reinterpret_cast<int32_t*>(h->mem + L.state_off + layer * L.state_stride);
+  a.layer = reinterpret_cast<LayerState*>(h->mem + L.layer_off) + layer;
+  a.dec = reinterpret_cast<Decision*>(h->mem + L.dec_off + layer * L.dec_stride);
   const size_t hid = c.scorer_hidden, d2 = 2 * static_cast<size_t>(c.head_dim), H = c.n_kv_heads;
   if (c.w1) {
     a.w1 = c.w1 + layer * H * hid * d2;
@@ -133,6 +136,8 @@ DecodeScratch decode_scratch(const kvpop_handle* h) {
   s.ticket = reinterpret_cast<int32_t*>(h->mem + h->lay.ticket_off);
   return s;
 }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool on_device(const void* p) {
   if (!p) return false;
@@ -180,12 +185,22 @@ int kvpop_create(const kvpop_config* cfg, void* dev_mem, size_t bytes, kvpop_han
   h->n_seen.assign(cfg->n_layers, 0);
   h->n_topk.assign(cfg->n_layers, 0);
   h->decoding.assign(cfg->n_layers, 0);
+  h->maps.resize(cfg->n_layers);
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    if (make_decode_tensor_map(&h->maps[l], h->mem + L.kv_off + l * L.kv_stride, cfg->dtype, cfg->head_dim,
+                               static_cast<int64_t>(L.units) * L.NS, L.row_bytes) != 0) {
+      delete h;
+      return KVPOP_ERR_CUDA;
+    }
+  }
   uint8_t* m = h->mem;
   bool ok = cudaMemset(m + L.kv_off, 0, cfg->n_layers * L.kv_stride) == cudaSuccess &&
             cudaMemset(m + L.pos_off, 0xff, cfg->n_layers * L.pos_stride) == cudaSuccess &&
             cudaMemset(m + L.score_off, 0, cfg->n_layers * L.score_stride) == cudaSuccess &&
-            cudaMemset(m + L.state_off, 0, L.total - L.state_off) == cudaSuccess &&
-            cudaDeviceSynchronize() == cudaSuccess;
+            cudaMemset(m + L.state_off, 0, L.total - L.state_off) == cudaSuccess;
+  for (int l = 0; ok && l < cfg->n_layers; ++l)
+    ok = launch_decide(layer_args(h, l), cfg->dtype, 0, 0, nullptr) == 0;
+  ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
     delete h;
     return KVPOP_ERR_CUDA;
@@ -216,36 +231,46 @@ int kvpop_prefill(kvpop_handle* h, int32_t layer, const void* k, const void* v, 
   if (r != 0) return KVPOP_ERR_CUDA;
   const int S = h->cfg.sinks, W = h->cfg.window, D = h->cfg.delay;
   const int e0 = std::max(S, n0 - W - D), e1 = std::max(S, n0 + n_tokens - W - D);
-  h->n_seen[layer] = n0 + n_tokens;
-  h->n_topk[layer] = std::min(h->cfg.topk, c0 + (e1 - e0));
+  const int n1 = n0 + n_tokens, c1 = std::min(h->cfg.topk, c0 + (e1 - e0));
+  if (launch_decide(a, h->cfg.dtype, n1, c1, static_cast<cudaStream_t>(stream)) != 0) return KVPOP_ERR_CUDA;
+  h->n_seen[layer] = n1;
+  h->n_topk[layer] = c1;
   return KVPOP_OK;
 }
 
-int kvpop_decode_append(kvpop_handle* h, int32_t layer, const void* k_new, const void* v_new,
-                        const float* ext_score, void* stream) {
-  if (!h || layer < 0 || layer >= h->cfg.n_layers) return KVPOP_ERR_INVALID_ARG;
-  if (!k_new || !v_new) return KVPOP_ERR_INVALID_ARG;
-  const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
-  if (ext && !ext_score) return KVPOP_ERR_INVALID_ARG;
-  if (h->n_seen[layer] >= h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
-  const LayerArgs a = layer_args(h, layer);
-  if (launch_update(a, h->cfg.dtype, k_new, v_new, ext ? ext_score : nullptr, static_cast<cudaStream_t>(stream)) != 0)
-    return KVPOP_ERR_CUDA;
+namespace {
+void advance_mirror(kvpop_handle* h, int layer) {
   const int S = h->cfg.sinks, W = h->cfg.window, D = h->cfg.delay;
   const int p = h->n_seen[layer];
   if (p - W - D >= S && h->n_topk[layer] < h->cfg.topk) h->n_topk[layer] += 1;
   h->n_seen[layer] = p + 1;
   h->decoding[layer] = 1;
+}
+}  // namespace
+
+int kvpop_decode_append(kvpop_handle* h, int32_t layer, const void* k_new, const void* v_new,
+                        const float* ext_score, void* stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers) return KVPOP_ERR_INVALID_ARG;
+  if (!k_new || !v_new) return KVPOP_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new)) return KVPOP_ERR_INVALID_ARG;
+  const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
+  if (ext && !ext_score) return KVPOP_ERR_INVALID_ARG;
+  if (h->n_seen[layer] >= h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
+  const LayerArgs a = layer_args(h, layer);
+  if (launch_append(a, h->cfg.dtype, k_new, v_new, ext ? ext_score : nullptr, static_cast<cudaStream_t>(stream)) != 0)
+    return KVPOP_ERR_CUDA;
+  advance_mirror(h, layer);
   return KVPOP_OK;
 }
 
 int kvpop_decode_attend(kvpop_handle* h, int32_t layer, const void* q, void* out, void* stream) {
   if (!h || layer < 0 || layer >= h->cfg.n_layers) return KVPOP_ERR_INVALID_ARG;
   if (!q || !out) return KVPOP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out)) return KVPOP_ERR_INVALID_ARG;
   if (h->n_seen[layer] == 0) return KVPOP_ERR_ORDER;
   const LayerArgs a = layer_args(h, layer);
-  const int r = launch_attention(a, h->cfg.dtype, decode_scratch(h), q, out, h->num_sms,
-                                 static_cast<cudaStream_t>(stream));
+  const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, decode_scratch(h), MODE_ATTEND, q, nullptr, nullptr,
+                              nullptr, out, h->num_sms, static_cast<cudaStream_t>(stream));
   if (r == -2) return KVPOP_ERR_BAD_SHAPE;
   return r == 0 ? KVPOP_OK : KVPOP_ERR_CUDA;
 }
@@ -253,10 +278,18 @@ int kvpop_decode_attend(kvpop_handle* h, int32_t layer, const void* q, void* out
 int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void* k_new, const void* v_new,
                       void* out, const float* ext_score, void* stream) {
   if (!h || layer < 0 || layer >= h->cfg.n_layers) return KVPOP_ERR_INVALID_ARG;
-  if (!q || !out) return KVPOP_ERR_INVALID_ARG;
-  const int r = kvpop_decode_append(h, layer, k_new, v_new, ext_score, stream);
-  if (r != KVPOP_OK) return r;
-  return kvpop_decode_attend(h, layer, q, out, stream);
+  if (!q || !out || !k_new || !v_new) return KVPOP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_new) || !aligned16(v_new)) return KVPOP_ERR_INVALID_ARG;
+  const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
+  if (ext && !ext_score) return KVPOP_ERR_INVALID_ARG;
+  if (h->n_seen[layer] >= h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
+  const LayerArgs a = layer_args(h, layer);
+  const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, decode_scratch(h), MODE_STEP, q, k_new, v_new,
+                              ext ? ext_score : nullptr, out, h->num_sms, static_cast<cudaStream_t>(stream));
+  if (r == -2) return KVPOP_ERR_BAD_SHAPE;
+  if (r != 0) return KVPOP_ERR_CUDA;
+  advance_mirror(h, layer);
+  return KVPOP_OK;
 }
 
 int kvpop_inspect(kvpop_handle* h, int32_t layer, int32_t* pos_out, float* score_out, int32_t* state_out,

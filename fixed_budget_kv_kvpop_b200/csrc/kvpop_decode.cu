@@ -1,0 +1,1045 @@
+// KVpop decode step: fused cache update + split-K flash decode (sm_100a).
+//
+// Method: KVpop page §3 (fixed-budget pruning), §C.1 (mask definition:
+// decoding attends directly over the retained cache entries: sinks, recent
+// window, selected long-range tokens), §E.1-§E.2 (headwise MLP scorer on
+// [k; v]), §E.4 / §I (a token is scored when it reaches the eviction
+// boundary u = q - w; with delayed scoring D more steps later).
+//
+// One launch per layer and step does all of it.  The step that appends token
+// N (position p = N) changes the attended set by exactly one token out and
+// one in: the boundary token b = N - W - D either replaces the long-range
+// minimum e (e leaves) or is dropped (b leaves), and the new token N enters;
+// every other token only changes slot.  So the kernel
+//   * attends over the cache as it stood after step N-1, masking the single
+//     slot `evict` of this step's decision, and adds the new token's (k, v)
+//     from the input as one extra term in the final merge;
+//   * takes the NEXT step's eviction decision (score of token N+1-W-D, block
+//     argmin of the long-range keys, with this step's replacement applied) in
+//     a dedicated decider warp while the other warps stream the cache;
+//   * lets the last warp to finish a unit merge the split-K partials, write
+//     the output and commit this step's row moves (boundary token into its
+//     long-range slot, window token into the staging ring, new token into its
+//     window slot), after every reader of those rows has finished.
+// MODE_ATTEND is the attention part alone over the cache as it stands.
+//
+// Streaming layout: the tiles of all units (16 slots, one 2*d*sizeof(T) row
+// [k | v] per slot) form one sequence cut into equal contiguous ranges, one
+// per consumer warp (stream-K).  Each consumer warp feeds its own shared-memory
+// ring: lane j issues one cp.async.bulk (no multicast) for row j of the tile
+// into a row padded by 16 bytes, completion counted on the stage's mbarrier.
+// QK: lane (j, h) computes slot j's dot products over half h of the dims for
+// all G heads, q broadcast from shared memory, packed fp32 FMA
+// (fma.rn.f32x2); one shuffle joins the halves.  Softmax in the exp2 domain
+// with lazy rescaling (the running max moves only when a tile exceeds it by
+// 2^8).  PV: lanes own 16-byte chunks of the value row, slot groups split the
+// tile, p broadcast from shared memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kvpop_internal.cuh"
+
+namespace kvpop {
+
+namespace {
+
+constexpr int TS = 16;                               // slots per tile
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kLazy = 8.0f;                        // lazy rescale threshold (log2 units)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Launch shape of the decode kernel: consumer warps per CTA, shared-memory
+// stages per consumer warp, decider warps per CTA.
+#ifndef KVPOP_NCW
+#define KVPOP_NCW 10
+#endif
+#ifndef KVPOP_NSTG
+#define KVPOP_NSTG 2
+#endif
+#ifndef KVPOP_NDW
+#define KVPOP_NDW 2
+#endif
+constexpr int NDW = KVPOP_NDW;
+
+// A tile is TS rows [k | v]; it lands in shared memory as NBLK boxes of
+// TS rows x 128 bytes (box b holds bytes [128 b, 128 b + 128) of every row),
+// swizzled by the tensor-map TMA: 16-byte chunk c of box row j sits at chunk
+// c ^ (j & 7).  Column reads of 8 consecutive rows and row reads of 8
+// consecutive chunks both hit 8 distinct bank groups.
+template <typename T, int DH, int G>
+struct Geo {
+  static constexpr int ESZ = sizeof(T);
+  static constexpr int ROW = 2 * DH * ESZ;      // bytes per slot row [k | v]
+  static constexpr int NCHK = DH * ESZ / 16;    // 16-byte chunks per k (or v) row
+  static constexpr int NBLK = ROW / 128;        // 128-byte boxes per row
+  static constexpr int BOX = TS * 128;          // bytes per box in shared memory
+  static constexpr int BOXELEMS = 128 / ESZ;    // elements per box row
+  static constexpr int CH = NCHK / 2;           // chunks per QK half
+  static constexpr int EPC = 16 / ESZ;          // elements per chunk
+  static constexpr int LPS = NCHK;              // PV: lanes per slot
+  static constexpr int SG = 32 / LPS;           // PV: slot groups
+  static constexpr int SPG = TS / SG;           // PV: slots per group
+  static constexpr int STAGE = TS * ROW;
+  static constexpr int QHALF = CH * G * EPC * 4;     // bytes of one q half
+  static constexpr int QBYTES = 2 * QHALF + 16;      // + pad between halves
+  static constexpr int PSLOT = 2 * G * 4;            // p pairs (p, p) per slot
+  static constexpr int PBYTES = TS * PSLOT + SG * 16;
+  static_assert(NCHK == 8 || NCHK == 16, "k row must be 128 or 256 bytes");
+  // byte offset of 16-byte chunk c (0 <= c < 2 NCHK; v row from NCHK) of slot j
+  static __device__ __forceinline__ int off(int j, int c) {
+    return (c >> 3) * BOX + j * 128 + (((c & 7) ^ (j & 7)) << 4);
+  }
+};
+
+constexpr int kMergeCap = 256;   // per-CTA queue of units ready to merge
+
+template <typename T, int DH, int G, int NCW, int NSTG>
+struct Smem {
+  using GE = Geo<T, DH, G>;
+  static constexpr int QRB = (G * DH + 2 * DH) * GE::ESZ;   // raw q | k_new | v_new of one unit
+  static constexpr int RINGS = 0;
+  static constexpr int Q = RINGS + NCW * NSTG * GE::STAGE;
+  static constexpr int P = Q + NCW * GE::QBYTES;
+  static constexpr int QRAW = P + NCW * GE::PBYTES;
+  static constexpr int XS = QRAW + NCW * 2 * QRB;
+  static constexpr int MQ = XS + NDW * 2 * DH * 4;
+  static constexpr int BAR = MQ + (kMergeCap + 4) * 4;
+  static constexpr int TOTAL = BAR + NCW * (NSTG + 2) * 8;
+  static_assert(GE::STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+  static_assert(Q % 16 == 0 && P % 16 == 0 && QRAW % 16 == 0 && QRB % 16 == 0 && XS % 16 == 0 && MQ % 16 == 0 &&
+                    BAR % 8 == 0,
+                "smem alignment");
+  static_assert(TOTAL <= 232448, "shared memory per CTA exceeds 227 KB");
+};
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Validity of a slot of the cache holding tokens 0..p (fill-up phases only).
+struct ValidGeom {
+  int p, S, W, D, nse;
+  bool full;
+  __device__ __forceinline__ bool slot_ok(int i) const {
+    if (i >= nse) return false;
+    if (full) return true;
+    if (i < S) return i <= p;
+    if (i < S + W) {
+      if (p < S) return false;
+      const int idx = i - S;
+      const int t = p - (((p - idx) % W) + W) % W;
+      return t >= S;
+    }
+    if (i < S + W + D) {
+      const int q0 = p - W;
+      if (q0 < S) return false;
+      const int idx = i - S - W;
+      const int t = q0 - (((q0 - idx) % D) + D) % D;
+      return t >= S;
+    }
+    return true;  // long-range slots below nse are occupied
+  }
+};
+
+// Eviction decision for the step that appends token N, taken by one warp.
+// pending == nullptr: the cache as committed (holds tokens 0..N-1).
+// pending != nullptr: the cache before the commit of the step appending token
+// N-1 (described by *pending); token N-1 is then (kn, vn, ext_new).
+// ntk = long-range slots in use once that step is committed.
+template <typename T>
+__device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, int ntk, const Decision* pending,
+                                const T* kn, const T* vn, float ext_new, float* xs) {
+  const int lane = threadIdx.x & 31;
+  const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
+  Decision r;
+  r.p = N; r.bpos = -1; r.bslot = -1; r.tgt = -1; r.evict = -1; r.sb = 0.f; r.pad[0] = r.pad[1] = 0;
+  const int b = N - W - D;
+  if (b < S) return r;
+  const int base = topk_base(S, W, D);
+  const T* kv = reinterpret_cast<const T*>(a.kv + static_cast<size_t>(u) * NS * a.row_bytes);
+  const int32_t* pos = a.pos + static_cast<size_t>(u) * NS;
+  const float* score = a.score + static_cast<size_t>(u) * NS;
+  r.bpos = b;
+  r.bslot = (D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D);
+  // Prefetch the long-range keys of the first argmin batch before the scorer
+  // runs, so both sets of loads are in flight together.
+  constexpr int kB = 16;   // keys per lane per round trip
+  const bool need_argmin = (ntk >= K) && (K > 0);
+  float sc0[kB];
+  int32_t ps0[kB];
+  if (need_argmin) {
+#pragma unroll
+    for (int t = 0; t < kB; ++t) {
+      const int i = lane + 32 * t;
+      if (i < K) { sc0[t] = score[base + i]; ps0[t] = pos[base + i]; }
+    }
+  }
+  // where b's row is now
+  const T* krow;
+  bool from_input = false;
+  int rslot;
+  if (pending != nullptr && b == N - 1) {
+    from_input = true;
+    rslot = -1;
+    krow = kn;
+  } else {
+    rslot = (pending != nullptr && D <= 1) ? window_slot(b, S, W) : r.bslot;
+    krow = kv + static_cast<size_t>(rslot) * (2 * a.d);
+  }
+  const T* vrow = from_input ? vn : krow + a.d;
+  float sb;
+  if (a.flags & FLAG_EXTERNAL_SCORES) {
+    sb = from_input ? ext_new : score[rslot];
+  } else {
+    const int h = u % a.Hkv;
+    sb = mlp_score_warp<T>(krow, vrow, a.d, a.w1 + static_cast<size_t>(h) * a.hidden * 2 * a.d,
+                           a.b1 + static_cast<size_t>(h) * a.hidden, a.w2 + static_cast<size_t>(h) * a.hidden,
+                           a.b2[h], a.hidden, xs);
+  }
+  r.sb = sb;
+  if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0) {
+    if (!from_input && pos[rslot] != b) set_error(a.err, DEVERR_STATE_MISMATCH);
+    if (sb != sb) set_error(a.err, DEVERR_NAN_SCORE);
+  }
+  if (ntk < K) {
+    r.tgt = base + ntk;     // fill-up: next free long-range slot, nobody leaves
+    r.evict = -1;
+  } else if (K == 0) {
+    r.evict = r.bslot;
+  } else {
+    // block argmin of the long-range keys (keys are unique: positions are)
+    uint64_t best = ~0ull;
+    int mslot = -1;
+    for (int i0 = 0; i0 < K; i0 += 32 * kB) {
+      float sc[kB];
+      int32_t ps[kB];
+#pragma unroll
+      for (int t = 0; t < kB; ++t) {
+        const int i = i0 + lane + 32 * t;
+        if (i0 == 0) { sc[t] = sc0[t]; ps[t] = ps0[t]; }
+        else if (i < K) { sc[t] = score[base + i]; ps[t] = pos[base + i]; }
+      }
+#pragma unroll
+      for (int t = 0; t < kB; ++t) {
+        const int i = i0 + lane + 32 * t;
+        if (i < K) {
+          const int sl = base + i;
+          const uint64_t key = (pending != nullptr && sl == pending->tgt) ? rank_key(pending->sb, pending->bpos)
+                                                                          : rank_key(sc[t], ps[t]);
+          if (key < best) { best = key; mslot = sl; }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t ok = __shfl_xor_sync(0xffffffffu, best, o);
+      const int os = __shfl_xor_sync(0xffffffffu, mslot, o);
+      if (ok < best) { best = ok; mslot = os; }
+    }
+    if (rank_key(sb, b) > best) {
+      r.tgt = mslot;
+      r.evict = mslot;
+    } else {
+      r.evict = r.bslot;
+    }
+  }
+  return r;
+}
+
+// Commit of the step appending token N for unit u (one warp): moves rows as
+// the decision says, writes the new token, updates the unit's counters.
+template <typename T>
+__device__ void commit_warp(const LayerArgs& a, int u, int N, int ntk_after, const Decision& r, const T* kn,
+                            const T* vn, float ext_new) {
+  const int lane = threadIdx.x & 31;
+  const int S = a.S, W = a.W, D = a.D, NS = a.NS, RB = a.row_bytes;
+  uint8_t* kv = a.kv + static_cast<size_t>(u) * NS * RB;
+  int32_t* pos = a.pos + static_cast<size_t>(u) * NS;
+  float* score = a.score + static_cast<size_t>(u) * NS;
+  if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0) {
+    if (r.p != N) set_error(a.err, DEVERR_STATE_MISMATCH);
+    if (r.bpos >= 0 && pos[r.bslot] != r.bpos) set_error(a.err, DEVERR_STATE_MISMATCH);
+  }
+  const int p = N;
+  const int ns = p < S ? p : window_slot(p, S, W);
+  const int o = (p >= S && p - W >= S) ? p - W : -1;
+  const int st = (D > 0 && o >= 0) ? staging_slot(o, S, W, D) : -1;
+  const int half = a.d * static_cast<int>(sizeof(T));
+  // Read every source row first (one round trip), then write: the moves are
+  // tgt <- bslot, st <- ns, ns <- new, and bslot may equal st.
+  constexpr int kMaxChunks = 2;   // 16-byte chunks per lane per row (rows <= 1024 bytes)
+  uint4 rb[kMaxChunks], rn[kMaxChunks], rw[kMaxChunks];
+#pragma unroll
+  for (int t = 0; t < kMaxChunks; ++t) {
+    const int i = (lane + 32 * t) * 16;
+    if (i < RB) {
+      if (r.tgt >= 0) rb[t] = *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(r.bslot) * RB + i);
+      if (st >= 0) rn[t] = *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(ns) * RB + i);
+      rw[t] = (i < half) ? *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(kn) + i)
+                         : *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vn) + (i - half));
+    }
+  }
+  const float sns = (st >= 0) ? score[ns] : 0.f;
+  __syncwarp();
+#pragma unroll
+  for (int t = 0; t < kMaxChunks; ++t) {
+    const int i = (lane + 32 * t) * 16;
+    if (i < RB) {
+      if (r.tgt >= 0) *reinterpret_cast<uint4*>(kv + static_cast<size_t>(r.tgt) * RB + i) = rb[t];
+      if (st >= 0) *reinterpret_cast<uint4*>(kv + static_cast<size_t>(st) * RB + i) = rn[t];
+      *reinterpret_cast<uint4*>(kv + static_cast<size_t>(ns) * RB + i) = rw[t];
+    }
+  }
+  if (lane == 0) {
+    if (r.tgt >= 0) { pos[r.tgt] = r.bpos; score[r.tgt] = r.sb; }
+    if (st >= 0) { pos[st] = o; score[st] = sns; }
+    pos[ns] = p;
+    score[ns] = (a.flags & FLAG_EXTERNAL_SCORES) ? ext_new : 0.f;
+    a.state[4 * u + 0] = p + 1;
+    a.state[4 * u + 1] = ntk_after;
+  }
+  __syncwarp();
+}
+
+// Merge the split-K partials of a unit, write the output, and (in a step)
+// commit the step's row moves.  Run by one warp once every contributor of the
+// unit has arrived; kept out of line so streaming loops do not carry its
+// registers.  The new token was already folded into the first partial.
+template <typename T, int DH, int G>
+__device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch& sc, bool step, int N, int ntk_after,
+                                        int64_t unit, int nseg, const T* __restrict__ k_new,
+                                        const T* __restrict__ v_new, const float* __restrict__ ext,
+                                        T* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  constexpr int DPL = DH / 32;   // output dims per lane (contiguous)
+  const float* pm = sc.part_ml + unit * kMaxSeg * (G * 2);
+  const float* pa = sc.part_acc + unit * kMaxSeg * (G * DH);
+  T* ou = out + unit * (G * DH);
+  float M[G], L[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float mx = kNegInf;
+    for (int s0 = 0; s0 < nseg; s0 += 32) {
+      const float ms = (s0 + lane < nseg) ? __ldcg(pm + (s0 + lane) * G * 2 + 2 * g) : kNegInf;
+      mx = fmaxf(mx, ms);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    M[g] = mx;
+    float lsum = 0.f;
+    for (int s0 = 0; s0 < nseg; s0 += 32) {
+      const int sI = s0 + lane;
+      if (sI < nseg) {
+        const float ms = __ldcg(pm + sI * G * 2 + 2 * g);
+        if (ms != kNegInf) lsum += __ldcg(pm + sI * G * 2 + 2 * g + 1) * exp2f(ms - mx);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    L[g] = lsum;
+  }
+  float o_acc[G][DPL];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o_acc[g][e] = 0.f;
+  constexpr int kSB = 2;   // segments per round trip
+  for (int s0 = 0; s0 < nseg; s0 += kSB) {
+    float pv[kSB][G][DPL];
+    float ws[kSB][G];
+#pragma unroll
+    for (int t = 0; t < kSB; ++t) {
+      if (s0 + t < nseg) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float ms = __ldcg(pm + (s0 + t) * G * 2 + 2 * g);
+          ws[t][g] = (ms != kNegInf) ? exp2f(ms - M[g]) : 0.f;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) pv[t][g][e] = __ldcg(pa + (s0 + t) * G * DH + g * DH + lane * DPL + e);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kSB; ++t) {
+      if (s0 + t < nseg) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) o_acc[g][e] = fmaf(pv[t][g][e], ws[t][g], o_acc[g][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float inv = L[g] > 0.f ? 1.f / L[g] : 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) ou[g * DH + lane * DPL + e] = Elem<T>::from_f32(o_acc[g][e] * inv);
+  }
+  if (step) {
+    const Decision r = a.dec[static_cast<size_t>(N & 1) * a.units + unit];
+    commit_warp<T>(a, static_cast<int>(unit), N, ntk_after, r, k_new + unit * DH, v_new + unit * DH,
+                   ext ? ext[unit] : 0.f);
+  }
+}
+
+template <typename T, int DH, int G, int NCW, int NSTG>
+__global__ void __launch_bounds__((NCW + NDW) * 32, 1)
+decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ LayerArgs a,
+              const __grid_constant__ DecodeScratch sc, const int mode, const T* __restrict__ q,
+              const T* __restrict__ k_new, const T* __restrict__ v_new, const float* __restrict__ ext,
+              T* __restrict__ out) {
+  using GE = Geo<T, DH, G>;
+  using SM = Smem<T, DH, G, NCW, NSTG>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + SM::BAR);   // [NCW][NSTG]
+  uint64_t* q_bar = full_bar + NCW * NSTG;                             // [NCW][2]
+  int* mq = reinterpret_cast<int*>(smem + SM::MQ);                     // entries, then tail, head, done
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool step = (mode == MODE_STEP);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NCW * (NSTG + 2); ++i) mbar_init(&full_bar[i], 1);
+    mbar_fence_init();
+  }
+  for (int i = threadIdx.x; i < kMergeCap + 4; i += blockDim.x) mq[i] = 0;
+  // Programmatic dependent launch: let the next kernel in the stream start its
+  // prologue as SMs free up, and wait here until the previous one has
+  // completed and its writes are visible (everything below reads its results).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __syncthreads();
+  if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled boxes need 1024-byte alignment
+    if (threadIdx.x == 0) set_error(a.err, DEVERR_BAD_INDEX);
+    return;
+  }
+
+  const int N = a.layer->n_seen;      // the cache holds tokens 0..N-1
+  const int ntk = a.layer->n_topk;
+  const int S = a.S, W = a.W, D = a.D, K = a.K;
+  if (step && N >= a.max_context) {
+    if (threadIdx.x == 0) set_error(a.err, DEVERR_CONTEXT_OVERFLOW);
+    return;
+  }
+  const int ntk_after = ntk + ((step && N - W - D >= S && ntk < K) ? 1 : 0);
+  ValidGeom vg;
+  vg.p = N - 1; vg.S = S; vg.W = W; vg.D = D;
+  vg.nse = S + W + D + ntk;
+  vg.full = N >= S + W + D;
+  const int tpu = (vg.nse + TS - 1) / TS;
+  const int64_t total = static_cast<int64_t>(a.units) * tpu;
+  const int64_t nw = decode_active_warps(total, tpu, static_cast<int64_t>(gridDim.x) * NCW);
+  const float qscale = kLog2e * rsqrtf(static_cast<float>(DH));
+
+  auto nseg_of = [&](int64_t unit) -> int {
+    return static_cast<int>(warp_of_tile(unit * tpu + tpu - 1, total, nw) - warp_of_tile(unit * tpu, total, nw) + 1);
+  };
+  auto do_merge = [&](int64_t unit) {
+    merge_unit<T, DH, G>(a, sc, step, N, ntk_after, unit, nseg_of(unit), k_new, v_new, ext, out);
+    __syncwarp();
+    if (lane == 0) sc.ticket[unit] = 0;
+  };
+  // Count one finished contributor of `unit`.  The last one either queues the
+  // merge for this CTA's helpers (defer) or runs it at once.
+  auto arrive = [&](int64_t unit, bool defer) {
+    const int need = nseg_of(unit) + (step ? 1 : 0);
+    __threadfence();
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0) prev = atomicAdd(&sc.ticket[unit], 1);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != need - 1) return;
+    __threadfence();
+    int slot = kMergeCap;
+    if (defer) {
+      if (lane == 0) {
+        slot = atomicAdd(&mq[kMergeCap], 1);
+        if (slot < kMergeCap) atomicExch(&mq[slot], static_cast<int>(unit) + 1);
+      }
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+    }
+    if (slot >= kMergeCap) do_merge(unit);
+  };
+  // Pop queued merges until every consumer warp of the CTA has finished and
+  // the queue is drained (bounded wait; all traffic is this CTA's shared memory).
+  auto help = [&]() {
+    const uint64_t t0 = global_ns();
+    while (true) {
+      int got = -1;
+      if (lane == 0) {
+        const int tail = min(atomicAdd(&mq[kMergeCap], 0), kMergeCap);
+        const int head = atomicAdd(&mq[kMergeCap + 1], 0);
+        if (head < tail) {
+          if (atomicCAS(&mq[kMergeCap + 1], head, head + 1) == head) {
+            int v;
+            while ((v = atomicAdd(&mq[head], 0)) == 0) {
+              if (global_ns() - t0 > kWaitLimitNs) break;
+            }
+            got = v > 0 ? v - 1 : -3;
+          }
+        } else if (atomicAdd(&mq[kMergeCap + 2], 0) == NCW) {
+          const int tail2 = min(atomicAdd(&mq[kMergeCap], 0), kMergeCap);
+          if (head >= tail2) got = -2;
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (got == -2) break;
+      if (got == -3) {
+        if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+        break;
+      }
+      if (got >= 0) {
+        do_merge(got);
+        continue;
+      }
+      if (global_ns() - t0 > kWaitLimitNs) {
+        if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+        break;
+      }
+      __nanosleep(256);
+    }
+  };
+  auto consumer_done = [&]() {
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      atomicAdd(&mq[kMergeCap + 2], 1);
+    }
+    __syncwarp();
+  };
+  // Every warp of a step launch reports here once; the last one advances the
+  // layer counters (nobody reads them again in this launch).
+  auto finish_launch = [&]() {
+    if (!step) return;
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      const int prev = atomicAdd(&a.layer->ticket, 1);
+      if (prev == static_cast<int>(gridDim.x) * (NCW + NDW) - 1) {
+        a.layer->n_seen = N + 1;
+        a.layer->n_topk = ntk_after;
+        a.layer->ticket = 0;
+        __threadfence();
+      }
+    }
+  };
+
+  if (warp >= NCW) {
+    // ---------------- deciders, then merge helpers ----------------
+    if (step) {
+      const int dw = warp - NCW;
+      float* xs = reinterpret_cast<float*>(smem + SM::XS) + dw * 2 * DH;
+      for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
+        const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
+        const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, &cur, k_new + static_cast<size_t>(u) * DH,
+                                           v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f, xs);
+        if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+        arrive(u, false);
+      }
+    }
+    help();
+    finish_launch();
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * NCW + warp;
+  if (gw >= nw) {
+    consumer_done();
+    help();
+    finish_launch();
+    return;
+  }
+  const int64_t lo = seg_lo(gw, total, nw);
+  const int cnt = static_cast<int>(seg_lo(gw + 1, total, nw) - lo);
+  const int last_unit = static_cast<int>((lo + cnt - 1) / tpu);
+  uint8_t* ring = smem + SM::RINGS + warp * NSTG * GE::STAGE;
+  uint8_t* qsm = smem + SM::Q + warp * GE::QBYTES;
+  uint8_t* psm = smem + SM::P + warp * GE::PBYTES;
+  uint8_t* qraw = smem + SM::QRAW + warp * 2 * SM::QRB;
+  uint64_t* fb = full_bar + warp * NSTG;
+  uint64_t* qb = q_bar + warp * 2;
+  const int NS = a.NS;
+
+  // q (and in a step the new token's k, v) of a unit -> raw buffer `buf`
+  auto issue_q = [&](int unit, int buf) {
+    constexpr uint32_t kq = G * DH * GE::ESZ, kr = DH * GE::ESZ;
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&qb[buf], kq + (step ? 2 * kr : 0));
+      uint8_t* dst = qraw + buf * SM::QRB;
+      bulk_g2s(dst, q + static_cast<int64_t>(unit) * (G * DH), kq, &qb[buf]);
+      if (step) {
+        bulk_g2s(dst + kq, k_new + static_cast<int64_t>(unit) * DH, kr, &qb[buf]);
+        bulk_g2s(dst + kq + kr, v_new + static_cast<int64_t>(unit) * DH, kr, &qb[buf]);
+      }
+    }
+  };
+
+  // issue cursor (tile index within the range -> unit, tile of the unit)
+  int iu = static_cast<int>(lo / tpu), ij = static_cast<int>(lo - static_cast<int64_t>(iu) * tpu);
+  int istage = 0;
+  auto issue_next = [&]() {
+    if (lane == 0) mbar_arrive_expect_tx(&fb[istage], GE::STAGE);
+    __syncwarp();
+    if (lane < GE::NBLK)
+      tma_load_2d(ring + istage * GE::STAGE + lane * GE::BOX, &tmap, lane * GE::BOXELEMS, iu * NS + ij * TS,
+                  &fb[istage]);
+    if (++ij == tpu) { ij = 0; ++iu; }
+    if (++istage == NSTG) istage = 0;
+  };
+
+  const int j = lane & 15;        // QK: slot of the tile
+  const int h = lane >> 4;        // QK: half of the dims
+  const int gq = lane / GE::LPS;  // PV: slot group
+  const int c = lane % GE::LPS;   // PV: chunk of the value row
+
+  float2 acc[G][GE::EPC / 2];
+  float m[G], lp[G];
+  int evict = -1;
+  int cur = -1;
+  int qbuf = 0;
+  uint32_t qphase = 0;   // bit b = parity of raw buffer b's next completion
+
+  // Start a unit segment: q into the fp32 layout, reset the softmax state,
+  // fold the new token in if this warp holds the unit's first tile, and
+  // prefetch the next unit's q.
+  auto start_unit = [&](int unit, bool first_tile) {
+    if (!mbar_wait(&qb[qbuf], (qphase >> qbuf) & 1u)) {
+      if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+    }
+    qphase ^= 1u << qbuf;
+    const uint8_t* raw = qraw + qbuf * SM::QRB;
+    __syncwarp();
+    float* qf = reinterpret_cast<float*>(qsm);
+    const T* qr = reinterpret_cast<const T*>(raw);
+    for (int idx = lane; idx < G * DH; idx += 32) {
+      const int g = idx / DH, dim = idx % DH;
+      const int ch = dim / GE::EPC, e = dim % GE::EPC;
+      const int hh = ch / GE::CH, cc = ch % GE::CH;
+      qf[hh * ((GE::QHALF + 16) / 4) + (cc * G + g) * GE::EPC + e] = Elem<T>::to_f32(qr[idx]) * qscale;
+    }
+    evict = step ? a.dec[static_cast<size_t>(N & 1) * a.units + unit].evict : -1;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = kNegInf;
+      lp[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = make_float2(0.f, 0.f);
+    }
+    if (step && first_tile) {
+      // the appended token: score q . k_new and take it as the first slot
+      constexpr int DPL = DH / 32;
+      const T* kn = reinterpret_cast<const T*>(raw + G * DH * GE::ESZ);
+      const T* vn = kn + DH;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float part = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e)
+          part = fmaf(Elem<T>::to_f32(qr[g * DH + lane * DPL + e]), Elem<T>::to_f32(kn[lane * DPL + e]), part);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        m[g] = part * qscale;   // p = exp2(s - m) = 1
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) lp[g] = 1.f;
+      }
+      if (gq == 0) {
+        const uint4 vr = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vn) + c * 16);
+        float2 v2[GE::EPC / 2];
+        if constexpr (sizeof(T) == 2) {
+          v2[0] = bf2_to_f2(vr.x); v2[1] = bf2_to_f2(vr.y); v2[2] = bf2_to_f2(vr.z); v2[3] = bf2_to_f2(vr.w);
+        } else {
+          v2[0] = make_float2(__uint_as_float(vr.x), __uint_as_float(vr.y));
+          v2[1] = make_float2(__uint_as_float(vr.z), __uint_as_float(vr.w));
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = v2[e];
+      }
+    }
+    __syncwarp();
+    if (unit < last_unit) issue_q(unit + 1, qbuf ^ 1);
+    qbuf ^= 1;
+  };
+
+  auto finalize = [&](int unit) {
+    float l[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float v = lp[g];
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      l[g] = v;
+    }
+#pragma unroll
+    for (int o = GE::LPS; o < 32; o <<= 1)
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < GE::EPC / 2; ++e) {
+          acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, o);
+          acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, o);
+        }
+    const int64_t first = warp_of_tile(static_cast<int64_t>(unit) * tpu, total, nw);
+    const int seg = static_cast<int>(gw - first);
+    if (seg >= kMaxSeg) {  // cannot happen: decode_active_warps bounds the segments
+      if (lane == 0) set_error(a.err, DEVERR_BAD_INDEX);
+      return;
+    }
+    float* pa = sc.part_acc + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * DH);
+    float* pmv = sc.part_ml + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * 2);
+    if (lane < GE::LPS) {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < GE::EPC / 2; ++e)
+          *reinterpret_cast<float2*>(pa + g * DH + c * GE::EPC + 2 * e) = acc[g][e];
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) { pmv[2 * g] = m[g]; pmv[2 * g + 1] = l[g]; }
+    }
+    arrive(unit, true);
+  };
+
+  // consume cursor
+  int cu = static_cast<int>(lo / tpu), cj = static_cast<int>(lo - static_cast<int64_t>(cu) * tpu);
+  // first unit's q before the tile burst (it would queue behind it otherwise)
+  issue_q(cu, 0);
+  {
+    const int npre = cnt < NSTG ? cnt : NSTG;
+    for (int i = 0; i < npre; ++i) issue_next();
+  }
+  int cstage = 0;
+  uint32_t cphase = 0;
+  bool failed = false;
+  int failed_at = -1;
+  for (int i = 0; i < cnt; ++i) {
+    const int s0 = cj * TS;
+    const int nsl = min(TS, vg.nse - s0);
+    if (cu != cur) {
+      if (cur >= 0) finalize(cur);
+      cur = cu;
+      start_unit(cu, cj == 0);
+    }
+    if (!mbar_wait(&fb[cstage], cphase)) {
+      if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+      failed = true;
+      failed_at = i;
+      break;
+    }
+    const uint8_t* tile = ring + cstage * GE::STAGE;
+
+    // ---- QK: lane (j, h) = slot j, dims of half h, all G heads ----
+    float s[G];
+    {
+      float2 sa[G][2];
+#pragma unroll
+      for (int g = 0; g < G; ++g) { sa[g][0] = make_float2(0.f, 0.f); sa[g][1] = make_float2(0.f, 0.f); }
+      const float* qh = reinterpret_cast<const float*>(qsm + h * (GE::QHALF + 16));
+#pragma unroll
+      for (int cc = 0; cc < GE::CH; ++cc) {
+        const uint4 kr = *reinterpret_cast<const uint4*>(tile + GE::off(j, h * GE::CH + cc));
+        float2 k2[GE::EPC / 2];
+        if constexpr (sizeof(T) == 2) {
+          k2[0] = bf2_to_f2(kr.x); k2[1] = bf2_to_f2(kr.y); k2[2] = bf2_to_f2(kr.z); k2[3] = bf2_to_f2(kr.w);
+        } else {
+          k2[0] = make_float2(__uint_as_float(kr.x), __uint_as_float(kr.y));
+          k2[1] = make_float2(__uint_as_float(kr.z), __uint_as_float(kr.w));
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float4* qp = reinterpret_cast<const float4*>(qh + (cc * G + g) * GE::EPC);
+#pragma unroll
+          for (int e4 = 0; e4 < GE::EPC / 4; ++e4) {
+            const float4 qv = qp[e4];
+            sa[g][e4 & 1] = ffma2(make_float2(qv.x, qv.y), k2[2 * e4], sa[g][e4 & 1]);
+            sa[g][e4 & 1] = ffma2(make_float2(qv.z, qv.w), k2[2 * e4 + 1], sa[g][e4 & 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float v = (sa[g][0].x + sa[g][0].y) + (sa[g][1].x + sa[g][1].y);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        s[g] = v;
+      }
+    }
+    const int slot = s0 + j;
+    const bool valid = (j < nsl) && (slot != evict) && vg.slot_ok(slot);
+    const uint32_t vmask = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+    // ---- online softmax (exp2 domain, lazy rescale) ----
+    float p[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float sv = valid ? s[g] : kNegInf;
+      float mt = sv;
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+      if (mt > m[g] + kLazy) {   // warp-uniform
+        const float alpha = (m[g] == kNegInf) ? 0.f : fast_exp2(m[g] - mt);
+        m[g] = mt;
+        lp[g] *= alpha;
+#pragma unroll
+        for (int e = 0; e < GE::EPC / 2; ++e) {
+          acc[g][e].x *= alpha;
+          acc[g][e].y *= alpha;
+        }
+      }
+      p[g] = valid ? fast_exp2(sv - m[g]) : 0.f;
+      lp[g] += p[g];
+    }
+    if (h == 0) {
+      float* pd = reinterpret_cast<float*>(psm + j * GE::PSLOT + (j / GE::SPG) * 16);
+#pragma unroll
+      for (int g = 0; g < G; g += 2) {
+        if (g + 1 < G)
+          *reinterpret_cast<float4*>(pd + 2 * g) = make_float4(p[g], p[g], p[g + 1], p[g + 1]);
+        else
+          *reinterpret_cast<float2*>(pd + 2 * g) = make_float2(p[g], p[g]);
+      }
+    }
+    __syncwarp();
+    // ---- PV: lane (gq, c) = slots of group gq, value chunk c ----
+    auto pv_slot = [&](int j2) {
+      const float* pp = reinterpret_cast<const float*>(psm + j2 * GE::PSLOT + (j2 / GE::SPG) * 16);
+      float2 pr[G];
+#pragma unroll
+      for (int g = 0; g < G; g += 2) {
+        if (g + 1 < G) {
+          const float4 t4 = *reinterpret_cast<const float4*>(pp + 2 * g);
+          pr[g] = make_float2(t4.x, t4.y);
+          pr[g + 1] = make_float2(t4.z, t4.w);
+        } else {
+          pr[g] = *reinterpret_cast<const float2*>(pp + 2 * g);
+        }
+      }
+      const uint4 vr = *reinterpret_cast<const uint4*>(tile + GE::off(j2, GE::NCHK + c));
+      float2 v2[GE::EPC / 2];
+      if constexpr (sizeof(T) == 2) {
+        v2[0] = bf2_to_f2(vr.x); v2[1] = bf2_to_f2(vr.y); v2[2] = bf2_to_f2(vr.z); v2[3] = bf2_to_f2(vr.w);
+      } else {
+        v2[0] = make_float2(__uint_as_float(vr.x), __uint_as_float(vr.y));
+        v2[1] = make_float2(__uint_as_float(vr.z), __uint_as_float(vr.w));
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = ffma2(pr[g], v2[e], acc[g][e]);
+    };
+    if (vmask == 0xffffu) {
+#pragma unroll
+      for (int jj = 0; jj < GE::SPG; ++jj) pv_slot(gq * GE::SPG + jj);
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < GE::SPG; ++jj) {
+        const int j2 = gq * GE::SPG + jj;
+        if ((vmask >> j2) & 1u) pv_slot(j2);
+      }
+    }
+    __syncwarp();
+    if (i + NSTG < cnt) {
+      fence_proxy_async_smem();
+      issue_next();
+    }
+    if (++cj == tpu) { cj = 0; ++cu; }
+    if (++cstage == NSTG) { cstage = 0; cphase ^= 1u; }
+  }
+  if (failed) {
+    // let this warp's copies still in flight land (bounded) before it exits
+    int st2 = cstage;
+    uint32_t ph2 = cphase;
+    for (int k2 = failed_at + 1; k2 < cnt && k2 < failed_at + NSTG; ++k2) {
+      if (++st2 == NSTG) { st2 = 0; ph2 ^= 1u; }
+      mbar_wait(&fb[st2], ph2);
+    }
+  } else if (cur >= 0) {
+    finalize(cur);
+  }
+  consumer_done();
+  help();
+  finish_launch();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) append_kernel(const LayerArgs a, const T* __restrict__ k_new,
+                                                     const T* __restrict__ v_new, const float* __restrict__ ext) {
+  __shared__ __align__(16) float xs[4][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * 4 + warp;
+  const int N = a.layer->n_seen;
+  const int ntk = a.layer->n_topk;
+  const int ntk_after = ntk + ((N - a.W - a.D >= a.S && ntk < a.K) ? 1 : 0);
+  if (N >= a.max_context) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_error(a.err, DEVERR_CONTEXT_OVERFLOW);
+    return;
+  }
+  if (u < a.units) {
+    const T* kn = k_new + static_cast<size_t>(u) * a.d;
+    const T* vn = v_new + static_cast<size_t>(u) * a.d;
+    const float en = ext ? ext[u] : 0.f;
+    const Decision r = a.dec[static_cast<size_t>(N & 1) * a.units + u];
+    commit_warp<T>(a, u, N, ntk_after, r, kn, vn, en);
+    __threadfence();
+    __syncwarp();
+    const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, nullptr, kn, vn, en, xs[warp]);
+    if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+  }
+  // last warp of the launch advances the layer counters
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence();
+    const int prev = atomicAdd(&a.layer->ticket, 1);
+    if (prev == static_cast<int>(gridDim.x) * 4 - 1) {
+      a.layer->n_seen = N + 1;
+      a.layer->n_topk = ntk_after;
+      a.layer->ticket = 0;
+      __threadfence();
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) decide_kernel(const LayerArgs a, int N, int ntk) {
+  __shared__ __align__(16) float xs[4][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * 4 + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.layer->n_seen = N;
+    a.layer->n_topk = ntk;
+    a.layer->ticket = 0;
+  }
+  if (u >= a.units) return;
+  const Decision r = decide_warp<T>(a, u, N, ntk, nullptr, nullptr, nullptr, 0.f, xs[warp]);
+  if (lane == 0) {
+    a.dec[static_cast<size_t>(N & 1) * a.units + u] = r;
+    a.state[4 * u + 0] = N;
+    a.state[4 * u + 1] = ntk;
+  }
+}
+
+template <typename T, int DH, int G, int NCW, int NSTG>
+int launch_t(const CUtensorMap& tmap, const LayerArgs& a, const DecodeScratch& sc, int mode, const void* q,
+             const void* kn, const void* vn, const float* ext, void* out, int num_sms, cudaStream_t st) {
+  using SM = Smem<T, DH, G, NCW, NSTG>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(decode_kernel<T, DH, G, NCW, NSTG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SM::TOTAL) != cudaSuccess)
+      return -1;
+    attr_set = true;
+  }
+  const int64_t tpu_max = (a.NS + TS - 1) / TS;
+  const int64_t total_max = static_cast<int64_t>(a.units) * tpu_max;
+  int64_t grid = (total_max + NCW - 1) / NCW;
+  if (grid > num_sms) grid = num_sms;
+  if (grid < 1) grid = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3((NCW + NDW) * 32);
+  cfg.dynamicSmemBytes = SM::TOTAL;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<T, DH, G, NCW, NSTG>, tmap, a, sc, mode,
+                                           static_cast<const T*>(q), static_cast<const T*>(kn),
+                                           static_cast<const T*>(vn), ext, static_cast<T*>(out));
+  return e == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace
+
+int make_decode_tensor_map(CUtensorMap* map, void* layer_kv, int dtype, int d, int64_t rows, int row_bytes) {
+  // The driver entry point is fetched through the runtime, so the library
+  // needs no link-time dependency on libcuda.
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess || fn == nullptr)
+      return -1;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const int esz = dtype == 0 ? 4 : 2;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(2 * d), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(TS)};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = encode(map, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                            layer_kv, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+int decode_supported(int dtype, int d, int G) {
+  if (dtype == 1 && d == 128) return G == 1 || G == 2 || G == 4;
+  if (d == 64) return G == 1 || G == 2 || G == 4 || G == 8;
+  return 0;
+}
+
+int launch_decode(const CUtensorMap& tmap, const LayerArgs& a, int dtype, const DecodeScratch& sc, int mode,
+                  const void* q, const void* k_new, const void* v_new, const float* ext_score, void* out, int num_sms,
+                  cudaStream_t st) {
+#define KVPOP_DISPATCH(TT, DD, GG) \
+  if (a.d == DD && a.G == GG)      \
+    return launch_t<TT, DD, GG, (GG > 4 ? 8 : KVPOP_NCW), (GG > 4 ? 2 : KVPOP_NSTG)>(tmap, a, sc, mode, q, k_new,  \
+                                                                             v_new, ext_score, out, num_sms, st);
+  if (dtype == 1) {
+    KVPOP_DISPATCH(__nv_bfloat16, 128, 4)
+    KVPOP_DISPATCH(__nv_bfloat16, 128, 2)
+    KVPOP_DISPATCH(__nv_bfloat16, 128, 1)
+    KVPOP_DISPATCH(__nv_bfloat16, 64, 8)
+    KVPOP_DISPATCH(__nv_bfloat16, 64, 4)
+    KVPOP_DISPATCH(__nv_bfloat16, 64, 2)
+    KVPOP_DISPATCH(__nv_bfloat16, 64, 1)
+  } else {
+    KVPOP_DISPATCH(float, 64, 8)
+    KVPOP_DISPATCH(float, 64, 4)
+    KVPOP_DISPATCH(float, 64, 2)
+    KVPOP_DISPATCH(float, 64, 1)
+  }
+#undef KVPOP_DISPATCH
+  return -2;
+}
+
+int launch_append(const LayerArgs& a, int dtype, const void* k_new, const void* v_new, const float* ext_score,
+                  cudaStream_t st) {
+  const int grid = (a.units + 3) / 4;
+  if (dtype == 0)
+    append_kernel<float><<<grid, 128, 0, st>>>(a, static_cast<const float*>(k_new),
+                                               static_cast<const float*>(v_new), ext_score);
+  else
+    append_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a, static_cast<const __nv_bfloat16*>(k_new),
+                                                       static_cast<const __nv_bfloat16*>(v_new), ext_score);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_decide(const LayerArgs& a, int dtype, int n_seen, int n_topk, cudaStream_t st) {
+  const int grid = (a.units + 3) / 4;
+  if (dtype == 0)
+    decide_kernel<float><<<grid, 128, 0, st>>>(a, n_seen, n_topk);
+  else
+    decide_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a, n_seen, n_topk);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace kvpop

@@ -14,13 +14,19 @@
 //   pos   [units][NS]  int32 position held by each slot, -1 = empty
 //   score [units][NS]  fp32  ranking score (long-range slots; with caller
 //                            scores also the window/staging slots)
-//   state [units][4]   int32 {n_seen, n_topk, 0, 0}
+//   state [units][4]   int32 {n_seen, n_topk, 0, 0} (per unit, for inspection)
+//   layer  LayerState  {n_seen, n_topk, ticket}: the counters every kernel of
+//                      the layer reads; updated only by the last warp of a
+//                      launch, so all warps of a launch see the same values
+//   dec   [2][units]   Decision: the eviction decision of the step appending
+//                      token N lives in dec[N & 1] (taken one step ahead)
 // Slot map: sinks [0, S) hold positions 0..S-1; window slot of token t is
 // S + (t mod W); staging slot is S + W + (t mod D); long-range slots start at
 // S + W + D and fill as a prefix.
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -36,16 +42,35 @@ enum : int32_t {
 };
 
 constexpr int kMaxSeg = 64;         // split-K partials per unit (upper bound)
-constexpr int kTileSlots = 16;      // slots per consumer-warp tile in the decode kernel
-constexpr int kConsumerWarps = 8;   // consumer warps per decode CTA
-constexpr int kStagesPerWarp = 3;   // smem pipeline depth per consumer warp
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
+
+// Per-layer counters shared by all units (all batch rows share one length).
+struct LayerState {
+  int32_t n_seen;   // tokens in the cache; the next decode step appends token n_seen
+  int32_t n_topk;   // long-range slots in use (a prefix of the long-range region)
+  int32_t ticket;   // warps of the current launch that have finished
+  int32_t pad;
+};
+
+// Eviction decision of the decode step that appends token p, for one unit.
+// The token b = p - W - D reaches the eviction boundary at that step.
+struct Decision {
+  int32_t p;       // position the decision is for
+  int32_t bpos;    // boundary token position, -1 if none
+  int32_t bslot;   // its slot before the step's moves
+  int32_t tgt;     // long-range slot it moves to, -1 if dropped (or none)
+  int32_t evict;   // slot whose token leaves the attended set at this step, -1 if none
+  float sb;        // its ranking score
+  int32_t pad[2];
+};
 
 struct LayerArgs {
   uint8_t* kv;          // this layer's [units][NS][2][d]
   int32_t* pos;         // [units][NS]
   float* score;         // [units][NS]
   int32_t* state;       // [units][4]
+  LayerState* layer;    // this layer's counters
+  Decision* dec;        // [2][units]
   const float* w1;      // this layer's scorer [Hkv][hidden][2d]
   const float* b1;      // [Hkv][hidden]
   const float* w2;      // [Hkv][hidden]
@@ -181,33 +206,87 @@ __device__ __forceinline__ void set_error(int32_t* err, int32_t bits) {
 }
 
 // Scorer: s = w2 . relu(W1 x + b1) + b2 for x = [k; v] of one slot row
-// (KVpop page §E.1 headwise inputs, §E.2 stateless MLP scorer).  Accumulated
-// in fp64 (the inputs and fp32 weights are exact in fp64) and rounded once to
-// fp32, the ranking precision (§F).  Called by a whole CTA; `xs` is shared
-// scratch of 2d floats, `red` shared scratch of at least blockDim.x/32
-// doubles.  Returns the score in every thread.
-template <typename T>
-__device__ float mlp_score_block(const T* row, int d, const float* w1, const float* b1, const float* w2,
-                                 float b2, int hidden, float* xs, double* red) {
-  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarp = nthr >> 5;
-  for (int i = tid; i < 2 * d; i += nthr) xs[i] = Elem<T>::to_f32(row[i]);
-  __syncthreads();
-  double part = 0.0;
-  for (int j = warp; j < hidden; j += nwarp) {
-    const float* wr = w1 + static_cast<size_t>(j) * 2 * d;
-    double acc = 0.0;
-    for (int i = lane; i < 2 * d; i += 32) acc = fma(static_cast<double>(wr[i]), static_cast<double>(xs[i]), acc);
+// (KVpop page §E.1 headwise inputs, §E.2 stateless MLP scorer), computed by
+// one warp.  Accumulated in fp64 (inputs and fp32 weights are exact in fp64)
+// and rounded once to fp32, the ranking precision (§F).  `xs` is warp-private
+// shared scratch of 2d floats, 16-byte aligned.  Lane j owns hidden units
+// j, j + 32, ...; its W1 row is read as float4.  Returns the score in every
+// lane.
+template <typename T, int ROWS>
+__device__ double mlp_hidden_part(const float* xs, int d, const float* w1, const float* b1, const float* w2) {
+  // lane j owns hidden rows j, j + 32, ... (ROWS of them); W1 rows are read
+  // as float4 in batches of 16 / ROWS per row, so each round trip brings
+  // 8 KB per warp
+  const int lane = threadIdx.x & 31;
+  constexpr int kBatch = 16 / ROWS;
+  const int n4 = (2 * d) / 4;
+  const float4* xv = reinterpret_cast<const float4*>(xs);
+  const float4* wr[ROWS];
+  double acc[ROWS];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    const double h = fmax(acc + static_cast<double>(b1[j]), 0.0);
-    part = fma(static_cast<double>(w2[j]), h, part);   // identical in all lanes
+  for (int r = 0; r < ROWS; ++r) {
+    wr[r] = reinterpret_cast<const float4*>(w1 + static_cast<size_t>(lane + 32 * r) * 2 * d);
+    acc[r] = 0.0;
   }
-  if (lane == 0) red[warp] = part;
-  __syncthreads();
-  double s = static_cast<double>(b2);
-  for (int w = 0; w < nwarp; ++w) s += red[w];
-  __syncthreads();
-  return static_cast<float>(s);
+  for (int i0 = 0; i0 < n4; i0 += kBatch) {
+    float4 w[ROWS][kBatch];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+      for (int t = 0; t < kBatch; ++t) w[r][t] = __ldg(wr[r] + i0 + t);
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const float4 x = xv[i0 + t];
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        double a = acc[r];
+        a = fma(static_cast<double>(w[r][t].x), static_cast<double>(x.x), a);
+        a = fma(static_cast<double>(w[r][t].y), static_cast<double>(x.y), a);
+        a = fma(static_cast<double>(w[r][t].z), static_cast<double>(x.z), a);
+        a = fma(static_cast<double>(w[r][t].w), static_cast<double>(x.w), a);
+        acc[r] = a;
+      }
+    }
+  }
+  double part = 0.0;
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r) {
+    const int j = lane + 32 * r;
+    part = fma(static_cast<double>(w2[j]), fmax(acc[r] + static_cast<double>(b1[j]), 0.0), part);
+  }
+  return part;
+}
+
+// hidden in {32, 64, 128}; 2d a multiple of 64 (d = 64 or 128)
+template <typename T>
+__device__ float mlp_score_warp(const T* krow, const T* vrow, int d, const float* w1, const float* b1,
+                                const float* w2, float b2, int hidden, float* xs) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < d; i += 32) {
+    xs[i] = Elem<T>::to_f32(krow[i]);
+    xs[d + i] = Elem<T>::to_f32(vrow[i]);
+  }
+  __syncwarp();
+  double part;
+  if (hidden == 32) part = mlp_hidden_part<T, 1>(xs, d, w1, b1, w2);
+  else if (hidden == 64) part = mlp_hidden_part<T, 2>(xs, d, w1, b1, w2);
+  else part = mlp_hidden_part<T, 4>(xs, d, w1, b1, w2);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  __syncwarp();
+  return static_cast<float>(part + static_cast<double>(b2));
+}
+
+// Packed fp32 FMA (sm_100 FFMA2): d = a * b + c on both halves, round-to-nearest.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// bf16x2 word -> (lo, hi) as fp32 (exact).
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Decode kernel scratch (split-K partials), shared by the layers of a handle.
@@ -218,10 +297,21 @@ struct DecodeScratch {
 };
 
 // Kernel launchers (defined in the .cu files).
-int launch_update(const LayerArgs& a, int dtype, const void* k_new, const void* v_new,
-                  const float* ext_score, cudaStream_t st);
-int launch_attention(const LayerArgs& a, int dtype, const DecodeScratch& sc, const void* q, void* out,
-                     int num_sms, cudaStream_t st);
+enum DecodeMode : int { MODE_STEP = 0, MODE_ATTEND = 1 };
+// One fused decode step (MODE_STEP) or attention over the cache as it stands
+// (MODE_ATTEND).  ext_score may be null.
+int launch_decode(const CUtensorMap& tmap, const LayerArgs& a, int dtype, const DecodeScratch& sc, int mode,
+                  const void* q, const void* k_new, const void* v_new, const float* ext_score, void* out, int num_sms,
+                  cudaStream_t st);
+// Tensor map over one layer's cache rows for the decode kernel's TMA loads.
+int make_decode_tensor_map(CUtensorMap* map, void* layer_kv, int dtype, int d, int64_t rows, int row_bytes);
+// The cache update of a decode step without attention.
+int launch_append(const LayerArgs& a, int dtype, const void* k_new, const void* v_new, const float* ext_score,
+                  cudaStream_t st);
+// Takes the eviction decision for the next decode step from the cache as it
+// stands and sets the layer counters to (n_seen, n_topk).
+int launch_decide(const LayerArgs& a, int dtype, int n_seen, int n_topk, cudaStream_t st);
+int decode_supported(int dtype, int d, int G);
 
 struct PrefillScratch {
   float* new_score;   // [units][cap]

@@ -144,7 +144,8 @@ int kvpop_prefill(kvpop_handle* h, int32_t layer, const void* k, const void* v, 
  * q: device [b][Hq][d]; k_new, v_new: device [b][Hkv][d]; out: device
  * [b][Hq][d] (same element type); ext_score: device fp32 [b][Hkv], the score
  * of the token being appended (required with KVPOP_FLAG_EXTERNAL_SCORES).
- * The position counter then advances by one. */
+ * q, k_new, v_new and out must be 16-byte aligned (KVPOP_ERR_INVALID_ARG
+ * otherwise).  The position counter then advances by one. */
 int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void* k_new, const void* v_new,
                       void* out, const float* ext_score, void* stream);
 

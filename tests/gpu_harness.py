@@ -57,7 +57,7 @@ def build_cache(w: wl.Workload, n_layers: int, external: bool, weights=None, max
 
 def run_gpu(w: wl.Workload, n_layers: int, n_steps: int, *, external: bool = False, chunks=None,
             inspect_every: int = 1, layers_to_keep: Sequence[int] = (0,), tie_levels: int = 0,
-            master: int = 0, gen_device: str = "cpu", debug=True) -> Run:
+            master: int = 0, gen_device: str = "cpu", debug=True, split: bool = False) -> Run:
     """Prefill + n_steps decode steps of every layer on the GPU, through the C ABI."""
     dev = "cuda"
     weights = None
@@ -103,7 +103,11 @@ def run_gpu(w: wl.Workload, n_layers: int, n_steps: int, *, external: bool = Fal
                 es = wl.external_scores(w, layer, w.prefill + n_steps, master=master, device=gen_device,
                                         tie_levels=tie_levels)[:, :, w.prefill + i].contiguous().to(dev)
             out = torch.empty_like(q)
-            cache.decode_step(layer, q, kn, vn, out, es)
+            if split:
+                cache.decode_append(layer, kn, vn, es)
+                cache.decode_attend(layer, q, out)
+            else:
+                cache.decode_step(layer, q, kn, vn, out, es)
             if layer in run.layers:
                 run.dec_q[layer].append(q)
                 run.dec_k[layer].append(kn)

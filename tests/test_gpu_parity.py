@@ -108,3 +108,44 @@ def test_nonfinite_free_outputs_and_rows_hold_tokens():
         assert state[unit][0] == w.prefill + w.decode
     for o in run.outs[0]:
         assert torch.isfinite(o).all()
+
+
+@pytest.mark.parametrize("S,W,D,K", [(4, 16, 0, 44), (2, 8, 5, 20), (0, 1, 0, 7), (2, 3, 1, 6)])
+def test_split_append_attend_matches_fused_step(S, W, D, K):
+    """kvpop_decode_append + kvpop_decode_attend (two launches) and the fused
+    kvpop_decode_step agree: identical slot maps, outputs equal up to fp32
+    summation order."""
+    _need_gpu()
+    w = wl.Workload("split_case", batch=2, n_layers=1, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=S, window=W, topk=K, delay=D, prefill=50, decode=30, scorer_hidden=64,
+                    heavy_hitter_frac=0.02)
+    a = gh.run_gpu(w, n_layers=1, n_steps=w.decode)
+    b = gh.run_gpu(w, n_layers=1, n_steps=w.decode, split=True)
+    for i in range(w.decode + 1):
+        np.testing.assert_array_equal(a.slot_pos[0][i], b.slot_pos[0][i])
+    for i in range(w.decode):
+        np.testing.assert_allclose(a.outs[0][i].numpy(), b.outs[0][i].numpy(), rtol=0, atol=1.6e-2)
+    for unit in range(4):
+        gh.check_unit(b, 0, unit, exact_slots=False, atol=gh.BF16_ATOL)
+
+
+def test_mlp_scores_match_oracle_exactly_in_fp32():
+    """The scorer accumulates in fp64 and rounds once, so the long-range slots'
+    fp32 scores equal the oracle's float64-then-float32 scores."""
+    _need_gpu()
+    w = wl.Workload("score_case", batch=2, n_layers=1, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=4, window=16, topk=40, delay=2, prefill=120, decode=24, scorer_hidden=64,
+                    heavy_hitter_frac=0.02)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode)
+    pos, score, _ = run.cache.inspect(0)
+    base = w.sinks + w.window + w.delay
+    n_exact = n_total = 0
+    for unit in range(4):
+        k_all, v_all, _ = gh.unit_inputs(run, 0, unit)
+        ref = gh.unit_scores(run, 0, unit, k_all, v_all)
+        for sl in range(base, pos.shape[1]):
+            if pos[unit, sl] >= 0:
+                n_total += 1
+                n_exact += int(np.float32(ref[pos[unit, sl]]) == score[unit, sl])
+    assert n_total == 4 * w.topk
+    assert n_exact == n_total, f"{n_total - n_exact} of {n_total} scores differ from the oracle's fp32 value"
