@@ -91,12 +91,12 @@ struct Geo {
   }
 };
 
-constexpr int kMergeCap = 256;   // per-CTA queue of units ready to merge
+constexpr int kMergeCap = 512;   // per-CTA ring of units ready to merge
 
 template <typename T, int DH, int G, int NCW, int NSTG>
 struct Smem {
   using GE = Geo<T, DH, G>;
-  static constexpr int QRB = (G * DH + 2 * DH) * GE::ESZ;   // raw q | k_new | v_new of one unit
+  static constexpr int QRB = (G * DH + 2 * DH) * GE::ESZ + 32;   // raw q | k_new | v_new | decision of one unit
   static constexpr int RINGS = 0;
   static constexpr int Q = RINGS + NCW * NSTG * GE::STAGE;
   static constexpr int P = Q + NCW * GE::QBYTES;
@@ -117,6 +117,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Ticket increment with acquire-release semantics at GPU scope: the caller's
+// (and, after __syncwarp, its warp's) earlier writes are visible to whoever
+// observes the new count.
+__device__ __forceinline__ int ticket_add(int32_t* t) {
+  int prev;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(prev) : "l"(t) : "memory");
+  return prev;
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -170,19 +179,7 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
   const float* score = a.score + static_cast<size_t>(u) * NS;
   r.bpos = b;
   r.bslot = (D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D);
-  // Prefetch the long-range keys of the first argmin batch before the scorer
-  // runs, so both sets of loads are in flight together.
-  constexpr int kB = 16;   // keys per lane per round trip
-  const bool need_argmin = (ntk >= K) && (K > 0);
-  float sc0[kB];
-  int32_t ps0[kB];
-  if (need_argmin) {
-#pragma unroll
-    for (int t = 0; t < kB; ++t) {
-      const int i = lane + 32 * t;
-      if (i < K) { sc0[t] = score[base + i]; ps0[t] = pos[base + i]; }
-    }
-  }
+  constexpr int kB = 16;   // long-range keys per lane per round trip
   // where b's row is now
   const T* krow;
   bool from_input = false;
@@ -225,8 +222,7 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
 #pragma unroll
       for (int t = 0; t < kB; ++t) {
         const int i = i0 + lane + 32 * t;
-        if (i0 == 0) { sc[t] = sc0[t]; ps[t] = ps0[t]; }
-        else if (i < K) { sc[t] = score[base + i]; ps[t] = pos[base + i]; }
+        if (i < K) { sc[t] = score[base + i]; ps[t] = pos[base + i]; }
       }
 #pragma unroll
       for (int t = 0; t < kB; ++t) {
@@ -311,9 +307,12 @@ __device__ void commit_warp(const LayerArgs& a, int u, int N, int ntk_after, con
 }
 
 // Merge the split-K partials of a unit, write the output, and (in a step)
-// commit the step's row moves.  Run by one warp once every contributor of the
-// unit has arrived; kept out of line so streaming loops do not carry its
-// registers.  The new token was already folded into the first partial.
+// commit the step's row moves: boundary token into its long-range slot,
+// window token into the staging ring, new token into its window slot.  Run by
+// one warp once every contributor of the unit has arrived.  Two dependent
+// round trips: (1) every segment's (m, l) and the step's decision; (2) every
+// segment's accumulators and the rows the commit moves.  The new token was
+// already folded into the first partial.
 template <typename T, int DH, int G>
 __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch& sc, bool step, int N, int ntk_after,
                                         int64_t unit, int nseg, const T* __restrict__ k_new,
@@ -321,60 +320,99 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
                                         T* __restrict__ out) {
   const int lane = threadIdx.x & 31;
   constexpr int DPL = DH / 32;   // output dims per lane (contiguous)
+  static_assert(DPL == 2 || DPL == 4, "head_dim 64 or 128");
   const float* pm = sc.part_ml + unit * kMaxSeg * (G * 2);
   const float* pa = sc.part_acc + unit * kMaxSeg * (G * DH);
   T* ou = out + unit * (G * DH);
-  float M[G], L[G];
+  const int S = a.S, W = a.W, D = a.D, NS = a.NS, RB = a.row_bytes;
+
+  // ---- round trip 1: segment maxima/sums (lane s holds segment s, s + 32) and the decision ----
+  float mlA[2 * G], mlB[2 * G];
+#pragma unroll
+  for (int t = 0; t < 2 * G; ++t) {
+    mlA[t] = (lane < nseg) ? __ldcg(pm + lane * G * 2 + t) : 0.f;
+    mlB[t] = (lane + 32 < nseg) ? __ldcg(pm + (lane + 32) * G * 2 + t) : 0.f;
+  }
+  Decision r;
+  r.tgt = -1; r.bslot = -1; r.bpos = -1; r.p = N; r.evict = -1; r.sb = 0.f;
+  if (step) r = a.dec[static_cast<size_t>(N & 1) * a.units + unit];
+  float M[G], L[G], wA[G], wB[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    float mx = kNegInf;
-    for (int s0 = 0; s0 < nseg; s0 += 32) {
-      const float ms = (s0 + lane < nseg) ? __ldcg(pm + (s0 + lane) * G * 2 + 2 * g) : kNegInf;
-      mx = fmaxf(mx, ms);
-    }
+    const float ma = (lane < nseg) ? mlA[2 * g] : kNegInf;
+    const float mb = (lane + 32 < nseg) ? mlB[2 * g] : kNegInf;
+    float mx = fmaxf(ma, mb);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     M[g] = mx;
-    float lsum = 0.f;
-    for (int s0 = 0; s0 < nseg; s0 += 32) {
-      const int sI = s0 + lane;
-      if (sI < nseg) {
-        const float ms = __ldcg(pm + sI * G * 2 + 2 * g);
-        if (ms != kNegInf) lsum += __ldcg(pm + sI * G * 2 + 2 * g + 1) * exp2f(ms - mx);
+    wA[g] = (ma != kNegInf) ? fast_exp2(ma - mx) : 0.f;
+    wB[g] = (mb != kNegInf) ? fast_exp2(mb - mx) : 0.f;
+    float ls = wA[g] * mlA[2 * g + 1] + wB[g] * mlB[2 * g + 1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    L[g] = ls;
+  }
+
+  // ---- round trip 2: commit source rows (issued first) and segment accumulators ----
+  const int p = N;
+  const int ns = p < S ? p : window_slot(p, S, W);
+  const int o = (p >= S && p - W >= S) ? p - W : -1;
+  const int st = (D > 0 && o >= 0) ? staging_slot(o, S, W, D) : -1;
+  uint8_t* kv = a.kv + static_cast<size_t>(unit) * NS * RB;
+  int32_t* pos = a.pos + static_cast<size_t>(unit) * NS;
+  float* score = a.score + static_cast<size_t>(unit) * NS;
+  const int half = DH * static_cast<int>(sizeof(T));
+  constexpr int kMaxChunks = 2;   // 16-byte chunks per lane per row (rows <= 1024 bytes)
+  uint4 rb[kMaxChunks], rn[kMaxChunks], rw[kMaxChunks];
+  float sns = 0.f;
+  if (step) {
+#pragma unroll
+    for (int t = 0; t < kMaxChunks; ++t) {
+      const int i = (lane + 32 * t) * 16;
+      if (i < RB) {
+        if (r.tgt >= 0) rb[t] = *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(r.bslot) * RB + i);
+        if (st >= 0) rn[t] = *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(ns) * RB + i);
+        rw[t] = (i < half) ? *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(k_new + unit * DH) + i)
+                           : *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(v_new + unit * DH) +
+                                                             (i - half));
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    L[g] = lsum;
+    if (st >= 0) sns = score[ns];
   }
   float o_acc[G][DPL];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < DPL; ++e) o_acc[g][e] = 0.f;
-  constexpr int kSB = 2;   // segments per round trip
+  constexpr int kSB = 4;   // segments per batch of loads
   for (int s0 = 0; s0 < nseg; s0 += kSB) {
     float pv[kSB][G][DPL];
-    float ws[kSB][G];
 #pragma unroll
     for (int t = 0; t < kSB; ++t) {
       if (s0 + t < nseg) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float ms = __ldcg(pm + (s0 + t) * G * 2 + 2 * g);
-          ws[t][g] = (ms != kNegInf) ? exp2f(ms - M[g]) : 0.f;
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) pv[t][g][e] = __ldcg(pa + (s0 + t) * G * DH + g * DH + lane * DPL + e);
+          const float* src = pa + (s0 + t) * G * DH + g * DH + lane * DPL;
+          if constexpr (DPL == 4) {
+            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src));
+            pv[t][g][0] = v4.x; pv[t][g][1] = v4.y; pv[t][g][2] = v4.z; pv[t][g][3] = v4.w;
+          } else {
+            const float2 v2 = __ldcg(reinterpret_cast<const float2*>(src));
+            pv[t][g][0] = v2.x; pv[t][g][1] = v2.y;
+          }
         }
       }
     }
 #pragma unroll
     for (int t = 0; t < kSB; ++t) {
-      if (s0 + t < nseg) {
+      const int sI = s0 + t;
+      if (sI < nseg) {
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+        for (int g = 0; g < G; ++g) {
+          const float wsv = __shfl_sync(0xffffffffu, sI < 32 ? wA[g] : wB[g], sI & 31);
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) o_acc[g][e] = fmaf(pv[t][g][e], ws[t][g], o_acc[g][e]);
+          for (int e = 0; e < DPL; ++e) o_acc[g][e] = fmaf(pv[t][g][e], wsv, o_acc[g][e]);
+        }
       }
     }
   }
@@ -384,11 +422,30 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
 #pragma unroll
     for (int e = 0; e < DPL; ++e) ou[g * DH + lane * DPL + e] = Elem<T>::from_f32(o_acc[g][e] * inv);
   }
-  if (step) {
-    const Decision r = a.dec[static_cast<size_t>(N & 1) * a.units + unit];
-    commit_warp<T>(a, static_cast<int>(unit), N, ntk_after, r, k_new + unit * DH, v_new + unit * DH,
-                   ext ? ext[unit] : 0.f);
+  if (!step) return;
+  if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0) {
+    if (r.p != N) set_error(a.err, DEVERR_STATE_MISMATCH);
+    if (r.bpos >= 0 && pos[r.bslot] != r.bpos) set_error(a.err, DEVERR_STATE_MISMATCH);
   }
+  __syncwarp();
+#pragma unroll
+  for (int t = 0; t < kMaxChunks; ++t) {
+    const int i = (lane + 32 * t) * 16;
+    if (i < RB) {
+      if (r.tgt >= 0) *reinterpret_cast<uint4*>(kv + static_cast<size_t>(r.tgt) * RB + i) = rb[t];
+      if (st >= 0) *reinterpret_cast<uint4*>(kv + static_cast<size_t>(st) * RB + i) = rn[t];
+      *reinterpret_cast<uint4*>(kv + static_cast<size_t>(ns) * RB + i) = rw[t];
+    }
+  }
+  if (lane == 0) {
+    if (r.tgt >= 0) { pos[r.tgt] = r.bpos; score[r.tgt] = r.sb; }
+    if (st >= 0) { pos[st] = o; score[st] = sns; }
+    pos[ns] = p;
+    score[ns] = (a.flags & FLAG_EXTERNAL_SCORES) ? ext[unit] : 0.f;
+    a.state[4 * unit + 0] = p + 1;
+    a.state[4 * unit + 1] = ntk_after;
+  }
+  __syncwarp();
 }
 
 template <typename T, int DH, int G, int NCW, int NSTG>
@@ -449,27 +506,30 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     __syncwarp();
     if (lane == 0) sc.ticket[unit] = 0;
   };
-  // Count one finished contributor of `unit`.  The last one either queues the
-  // merge for this CTA's helpers (defer) or runs it at once.
-  auto arrive = [&](int64_t unit, bool defer) {
-    const int need = nseg_of(unit) + (step ? 1 : 0);
-    __threadfence();
+  // Queue a unit whose contributors have all arrived, for this CTA's merge
+  // helpers.  The queue is a ring of kMergeCap entries (0 = empty, else unit + 1);
+  // when it is full the pusher waits for the helpers (bounded).
+  auto push_merge = [&](int64_t unit) {
+    if (lane == 0) {
+      const int slot = atomicAdd(&mq[kMergeCap], 1);
+      const uint64_t t0 = global_ns();
+      while (slot - atomicAdd(&mq[kMergeCap + 1], 0) >= kMergeCap) {
+        if (global_ns() - t0 > kWaitLimitNs) { set_error(a.err, DEVERR_TIMEOUT); break; }
+        __nanosleep(128);
+      }
+      atomicExch(&mq[slot % kMergeCap], static_cast<int>(unit) + 1);
+    }
+    __syncwarp();
+  };
+  // Count one finished contributor of `unit`; returns the previous count (lane 0's
+  // value in every lane).  The caller pushes the merge if it was the last.
+  auto arrive = [&](int64_t unit) -> int {
     __syncwarp();
     int prev = 0;
-    if (lane == 0) prev = atomicAdd(&sc.ticket[unit], 1);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev != need - 1) return;
-    __threadfence();
-    int slot = kMergeCap;
-    if (defer) {
-      if (lane == 0) {
-        slot = atomicAdd(&mq[kMergeCap], 1);
-        if (slot < kMergeCap) atomicExch(&mq[slot], static_cast<int>(unit) + 1);
-      }
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-    }
-    if (slot >= kMergeCap) do_merge(unit);
+    if (lane == 0) prev = ticket_add(&sc.ticket[unit]);
+    return prev;
   };
+  auto need_of = [&](int64_t unit) -> int { return nseg_of(unit) + (step ? 1 : 0); };
   // Pop queued merges until every consumer warp of the CTA has finished and
   // the queue is drained (bounded wait; all traffic is this CTA's shared memory).
   auto help = [&]() {
@@ -477,19 +537,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     while (true) {
       int got = -1;
       if (lane == 0) {
-        const int tail = min(atomicAdd(&mq[kMergeCap], 0), kMergeCap);
+        const int tail = atomicAdd(&mq[kMergeCap], 0);
         const int head = atomicAdd(&mq[kMergeCap + 1], 0);
         if (head < tail) {
           if (atomicCAS(&mq[kMergeCap + 1], head, head + 1) == head) {
             int v;
-            while ((v = atomicAdd(&mq[head], 0)) == 0) {
+            while ((v = atomicExch(&mq[head % kMergeCap], 0)) == 0) {
               if (global_ns() - t0 > kWaitLimitNs) break;
             }
             got = v > 0 ? v - 1 : -3;
           }
         } else if (atomicAdd(&mq[kMergeCap + 2], 0) == NCW) {
-          const int tail2 = min(atomicAdd(&mq[kMergeCap], 0), kMergeCap);
-          if (head >= tail2) got = -2;
+          if (head >= atomicAdd(&mq[kMergeCap], 0)) got = -2;
         }
       }
       got = __shfl_sync(0xffffffffu, got, 0);
@@ -499,6 +558,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
         break;
       }
       if (got >= 0) {
+        __threadfence();
         do_merge(got);
         continue;
       }
@@ -544,7 +604,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
         const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, &cur, k_new + static_cast<size_t>(u) * DH,
                                            v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f, xs);
         if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
-        arrive(u, false);
+        const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
+        if (prev == need_of(u) - 1) push_merge(u);
       }
     }
     help();
@@ -576,12 +637,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     constexpr uint32_t kq = G * DH * GE::ESZ, kr = DH * GE::ESZ;
     if (lane == 0) {
       fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&qb[buf], kq + (step ? 2 * kr : 0));
+      mbar_arrive_expect_tx(&qb[buf], kq + (step ? 2 * kr + 32 : 0));
       uint8_t* dst = qraw + buf * SM::QRB;
       bulk_g2s(dst, q + static_cast<int64_t>(unit) * (G * DH), kq, &qb[buf]);
       if (step) {
         bulk_g2s(dst + kq, k_new + static_cast<int64_t>(unit) * DH, kr, &qb[buf]);
         bulk_g2s(dst + kq + kr, v_new + static_cast<int64_t>(unit) * DH, kr, &qb[buf]);
+        bulk_g2s(dst + kq + 2 * kr, a.dec + static_cast<size_t>(N & 1) * a.units + unit, 32, &qb[buf]);
       }
     }
   };
@@ -608,6 +670,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   float m[G], lp[G];
   int evict = -1;
   int cur = -1;
+  int pend_unit = -1, pend_prev = 0;   // last finished segment, its ticket result
   int qbuf = 0;
   uint32_t qphase = 0;   // bit b = parity of raw buffer b's next completion
 
@@ -629,7 +692,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
       const int hh = ch / GE::CH, cc = ch % GE::CH;
       qf[hh * ((GE::QHALF + 16) / 4) + (cc * G + g) * GE::EPC + e] = Elem<T>::to_f32(qr[idx]) * qscale;
     }
-    evict = step ? a.dec[static_cast<size_t>(N & 1) * a.units + unit].evict : -1;
+    evict = step ? reinterpret_cast<const Decision*>(raw + G * DH * GE::ESZ + 2 * DH * GE::ESZ)->evict : -1;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       m[g] = kNegInf;
@@ -713,7 +776,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
 #pragma unroll
       for (int g = 0; g < G; ++g) { pmv[2 * g] = m[g]; pmv[2 * g + 1] = l[g]; }
     }
-    arrive(unit, true);
+    pend_unit = unit;
+    pend_prev = arrive(unit);   // checked later, so the atomic's round trip overlaps streaming
+  };
+  auto check_pending = [&]() {
+    if (pend_unit < 0) return;
+    const int prev = __shfl_sync(0xffffffffu, pend_prev, 0);
+    if (prev == need_of(pend_unit) - 1) push_merge(pend_unit);
+    pend_unit = -1;
   };
 
   // consume cursor
@@ -732,7 +802,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     const int s0 = cj * TS;
     const int nsl = min(TS, vg.nse - s0);
     if (cu != cur) {
-      if (cur >= 0) finalize(cur);
+      if (cur >= 0) {
+        check_pending();
+        finalize(cur);
+      }
       cur = cu;
       start_unit(cu, cj == 0);
     }
@@ -868,7 +941,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
       mbar_wait(&fb[st2], ph2);
     }
   } else if (cur >= 0) {
+    check_pending();
     finalize(cur);
+    check_pending();
   }
   consumer_done();
   help();

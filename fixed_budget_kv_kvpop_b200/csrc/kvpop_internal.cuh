@@ -215,10 +215,10 @@ __device__ __forceinline__ void set_error(int32_t* err, int32_t bits) {
 template <typename T, int ROWS>
 __device__ double mlp_hidden_part(const float* xs, int d, const float* w1, const float* b1, const float* w2) {
   // lane j owns hidden rows j, j + 32, ... (ROWS of them); W1 rows are read
-  // as float4 in batches of 16 / ROWS per row, so each round trip brings
-  // 8 KB per warp
+  // as float4 in batches of 32 / ROWS per row, so each round trip brings
+  // 16 KB per warp
   const int lane = threadIdx.x & 31;
-  constexpr int kBatch = 16 / ROWS;
+  constexpr int kBatch = 32 / ROWS;
   const int n4 = (2 * d) / 4;
   const float4* xv = reinterpret_cast<const float4*>(xs);
   const float4* wr[ROWS];
