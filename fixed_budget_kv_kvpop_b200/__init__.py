@@ -28,6 +28,9 @@ KVPOP_ERR_CONTEXT_OVERFLOW = -4
 KVPOP_ERR_CUDA = -5
 KVPOP_ERR_DEVICE = -6
 KVPOP_ERR_TIMEOUT = -7
+KVPOP_ERR_SCRATCH_LIMIT = -8
+
+KVPOP_NOALLOC_SCRATCH_BYTES = 16 << 20   # static split-K buffer behind decode_step_noalloc
 
 KVPOP_DTYPE_F32 = 0
 KVPOP_DTYPE_BF16 = 1
@@ -44,7 +47,7 @@ EXPORTED_SYMBOLS = (
     "kvpop_cache_bytes", "kvpop_create", "kvpop_prefill", "kvpop_decode_step", "kvpop_decode_append",
     "kvpop_decode_attend", "kvpop_inspect",
     "kvpop_get_layout", "kvpop_get_error", "kvpop_clear_error", "kvpop_debug_poison_error",
-    "kvpop_destroy", "kvpop_status_string",
+    "kvpop_destroy", "kvpop_status_string", "kvpop_decode_step_noalloc",
 )
 
 
@@ -92,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvpop_debug_poison_error": ([P, I32, P], ctypes.c_int),
         "kvpop_destroy": ([P], ctypes.c_int),
         "kvpop_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "kvpop_decode_step_noalloc": ([P, I32, P, P, P, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -180,6 +184,15 @@ class KVPopCache:
     def decode_step(self, layer: int, q, k_new, v_new, out, ext_score=None, stream=None):
         _check(lib.kvpop_decode_step(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                      _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step")
+
+    def decode_step_noalloc(self, layer: int, q, k_new, v_new, out, ext_score=None, stream=None):
+        """decode_step for callers that cannot allocate device memory: the
+        split-K scratch comes from the library's static 16 MiB buffer instead
+        of this handle's buffer, so the call allocates nothing.  Its first
+        call on a device looks up that buffer once (make it before any stream
+        capture); calls that overlap on the GPU share the buffer and race."""
+        _check(lib.kvpop_decode_step_noalloc(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                             _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step_noalloc")
 
     def decode_append(self, layer: int, k_new, v_new, ext_score=None, stream=None):
         _check(lib.kvpop_decode_append(self.handle, layer, _ptr(k_new), _ptr(v_new), _ptr(ext_score),

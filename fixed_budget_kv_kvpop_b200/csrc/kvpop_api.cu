@@ -2,6 +2,7 @@
 // layout, host mirrors of the per-layer counters, kernel launches.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -366,8 +367,84 @@ const char* kvpop_status_string(int s) {
     case KVPOP_ERR_CUDA: return "CUDA runtime error";
     case KVPOP_ERR_DEVICE: return "device-side error recorded";
     case KVPOP_ERR_TIMEOUT: return "device-side wait timed out";
+    case KVPOP_ERR_SCRATCH_LIMIT: return "problem needs more split-K scratch than the 16 MiB static buffer holds";
     default: return "unknown status";
   }
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// kvpop_decode_step_noalloc: the decode step with its split-K scratch in a
+// static device buffer, for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+
+// Split-K partials [units][kMaxSeg][G][d] and [units][kMaxSeg][G][2] (fp32)
+// and arrival tickets [units] (int32) of kvpop_decode_step_noalloc.  One copy
+// per GPU, part of the module image; host code must not hand this name to a
+// kernel (on the host it only stands for the symbol): the device address
+// comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[KVPOP_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+uint8_t* g_noalloc_base[kNoallocMaxDevices];   // device address per device, looked up once
+
+// Device address of g_noalloc_scratch on `dev`, which must be current.  The
+// first call per device does the lookup (this is the set-up step that must
+// happen before any stream capture).
+int noalloc_base(int dev, uint8_t** base) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_base[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return KVPOP_ERR_CUDA;
+    }
+    g_noalloc_base[dev] = static_cast<uint8_t*>(p);
+  }
+  *base = g_noalloc_base[dev];
+  return KVPOP_OK;
+}
+
+}  // namespace
+
+extern "C" int kvpop_decode_step_noalloc(kvpop_handle* h, int32_t layer, const void* q, const void* k_new,
+                                         const void* v_new, void* out, const float* ext_score, void* stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers) return KVPOP_ERR_INVALID_ARG;
+  if (!q || !out || !k_new || !v_new) return KVPOP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_new) || !aligned16(v_new)) return KVPOP_ERR_INVALID_ARG;
+  const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
+  if (ext && !ext_score) return KVPOP_ERR_INVALID_ARG;
+  if (h->n_seen[layer] >= h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
+  // the same split-K layout as the handle's own region, packed from offset 0
+  const size_t units = h->lay.units, G = h->lay.G, d = h->cfg.head_dim;
+  const size_t acc_bytes = align256(units * kMaxSeg * G * d * 4);
+  const size_t ml_bytes = align256(units * kMaxSeg * G * 2 * 4);
+  const size_t ticket_bytes = units * 4;
+  if (acc_bytes + ml_bytes + align256(ticket_bytes) > KVPOP_NOALLOC_SCRATCH_BYTES) return KVPOP_ERR_SCRATCH_LIMIT;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVPOP_ERR_CUDA;
+  if (dev != h->device || dev < 0 || dev >= kNoallocMaxDevices) return KVPOP_ERR_INVALID_ARG;
+  uint8_t* base = nullptr;
+  const int rb = noalloc_base(dev, &base);
+  if (rb != KVPOP_OK) return rb;
+  DecodeScratch sc;
+  sc.part_acc = reinterpret_cast<float*>(base);
+  sc.part_ml = reinterpret_cast<float*>(base + acc_bytes);
+  sc.ticket = reinterpret_cast<int32_t*>(base + acc_bytes + ml_bytes);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the tickets count arrivals from zero; a call that gave up on a wait can
+  // leave them non-zero, and another handle may have used more units
+  if (cudaMemsetAsync(sc.ticket, 0, ticket_bytes, st) != cudaSuccess) return KVPOP_ERR_CUDA;
+  const LayerArgs a = layer_args(h, layer);
+  const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, sc, MODE_STEP, q, k_new, v_new,
+                              ext ? ext_score : nullptr, out, h->num_sms, st);
+  if (r == -2) return KVPOP_ERR_BAD_SHAPE;
+  if (r != 0) return KVPOP_ERR_CUDA;
+  advance_mirror(h, layer);
+  return KVPOP_OK;
+}

@@ -50,6 +50,11 @@ extern "C" {
 #define KVPOP_ERR_CUDA -5             /* a CUDA runtime call failed */
 #define KVPOP_ERR_DEVICE -6           /* a kernel recorded an error (see kvpop_get_error) */
 #define KVPOP_ERR_TIMEOUT -7          /* a bounded device-side wait gave up */
+#define KVPOP_ERR_SCRATCH_LIMIT -8    /* needs more scratch than kvpop_decode_step_noalloc's static buffer */
+
+/* Size of the static split-K scratch buffer behind kvpop_decode_step_noalloc
+ * (16 MiB on every GPU that loads the library, held until the process exits). */
+#define KVPOP_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 /* Element types. */
 #define KVPOP_DTYPE_F32 0
@@ -148,6 +153,38 @@ int kvpop_prefill(kvpop_handle* h, int32_t layer, const void* k, const void* v, 
  * otherwise).  The position counter then advances by one. */
 int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void* k_new, const void* v_new,
                       void* out, const float* ext_score, void* stream);
+
+/* kvpop_decode_step for callers that cannot allocate device memory.
+ * The KVpop pages have no counterpart: this is a deployment variant.
+ *
+ * Who needs it: code that runs where nobody may call cudaMalloc -- a plugin
+ * inside a serving engine whose memory planner owns every device byte and
+ * hands the plugin only the tensors it planned, or a latency-critical decode
+ * loop that must not risk the device-wide synchronisation a cudaMalloc or
+ * cudaFree can cause.  This call allocates nothing and calls no allocating
+ * routine.  Its split-K partials and arrival tickets live in one static
+ * device buffer that is part of the library image
+ * (KVPOP_NOALLOC_SCRATCH_BYTES per GPU), not in the handle's buffer; the
+ * handle's own split-K region is left untouched.
+ *
+ * Arguments, results and errors are those of kvpop_decode_step, plus:
+ *  - KVPOP_ERR_SCRATCH_LIMIT (nothing enqueued) when the handle needs more
+ *    scratch than the static buffer holds.  The need is
+ *    units * 64 * G * (head_dim + 2) * 4 bytes plus units * 4, each part
+ *    rounded up to 256 bytes (units = batch * n_kv_heads, G = n_q_heads /
+ *    n_kv_heads); with G = 4, head_dim = 128 that is up to 126 units.
+ *  - KVPOP_ERR_INVALID_ARG when the current device is not the handle's.
+ *  - Set-up: the first call on a device (with that device current) looks up
+ *    the buffer's device address once and keeps it for the process; make
+ *    that first call before any stream capture begins.
+ *  - Every call on a device shares the one buffer, which keeps what the last
+ *    call left there.  The call clears the arrival tickets (the only part
+ *    that must start at zero) on `stream` before its kernel; the partials
+ *    are always written before they are read.  Calls whose work overlaps on
+ *    the GPU (other streams, other handles, other host threads) race on the
+ *    buffer and give wrong results: order them on one stream or by events. */
+int kvpop_decode_step_noalloc(kvpop_handle* h, int32_t layer, const void* q, const void* k_new,
+                              const void* v_new, void* out, const float* ext_score, void* stream);
 
 /* The two halves of kvpop_decode_step, for callers that schedule them apart
  * (same arguments and semantics; append must precede attend for each step).
