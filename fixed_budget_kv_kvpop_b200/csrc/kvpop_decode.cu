@@ -26,8 +26,12 @@
 // Streaming layout: the tiles of all units (16 slots, one 2*d*sizeof(T) row
 // [k | v] per slot) form one sequence cut into equal contiguous ranges, one
 // per consumer warp (stream-K).  Each consumer warp feeds its own shared-memory
-// ring: lane j issues one cp.async.bulk (no multicast) for row j of the tile
-// into a row padded by 16 bytes, completion counted on the stage's mbarrier.
+// ring (NSTG stages of one tile): the layer's rows are one 2-D tensor map
+// (inner dimension 2*d elements, outer units*NS rows) and a tile is 2*d*size/128
+// TMA boxes of 16 rows x 128 bytes with the 128-byte swizzle, issued by that
+// many lanes (cp.async.bulk.tensor, no multicast), completion counted on the
+// stage's mbarrier.  The swizzle makes the row-per-lane QK reads and the
+// chunk-per-lane PV reads of 16-byte vectors conflict-free.
 // QK: lane (j, h) computes slot j's dot products over half h of the dims for
 // all G heads, q broadcast from shared memory, packed fp32 FMA
 // (fma.rn.f32x2); one shuffle joins the halves.  Softmax in the exp2 domain
