@@ -53,7 +53,8 @@ constexpr float kLazy = 8.0f;                        // lazy rescale threshold (
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Launch shape of the decode kernel: consumer warps per CTA, shared-memory
-// stages per consumer warp, decider warps per CTA.
+// stages per consumer warp, decider warps per CTA, tiles per consumer warp
+// prefetched into L2 before the wait for the previous kernel.
 #ifndef KVPOP_NCW
 #define KVPOP_NCW 10
 #endif
@@ -62,6 +63,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 #endif
 #ifndef KVPOP_NDW
 #define KVPOP_NDW 2
+#endif
+#ifndef KVPOP_PFT
+#define KVPOP_PFT 2
 #endif
 constexpr int NDW = KVPOP_NDW;
 
@@ -452,6 +456,68 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
   __syncwarp();
 }
 
+// Before the kernel waits for its predecessor in the stream: warm L2 with
+// what this warp reads first, so the HBM idles less across the launch
+// boundary.  Only L2 prefetches are issued (hints: nothing is read into the
+// SM); the layer counters read here may be stale when the predecessor is a
+// launch of this same layer, so they only choose addresses, each clamped to
+// its array.  Consumer warps: the first kPrefetchTiles tiles of their range.
+// Decider warps: the long-range keys and candidate boundary rows of their
+// units, and (one CTA per KV head) that head's scorer weights.
+template <int NCW>
+__device__ __forceinline__ void l2_warmup(const LayerArgs& a, bool step, int warp, int lane) {
+  constexpr int kPrefetchTiles = KVPOP_PFT;
+  if (lane != 0) return;
+  const int N = ld_relaxed(&a.layer->n_seen);
+  const int ntk = ld_relaxed(&a.layer->n_topk);
+  const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
+  if (N < 1 || N > a.max_context || ntk < 0 || ntk > K) return;
+  const int64_t rb = a.row_bytes;
+  if (warp < NCW) {
+    if (kPrefetchTiles == 0) return;
+    const int tpu = (S + W + D + ntk + TS - 1) / TS;
+    const int64_t total = static_cast<int64_t>(a.units) * tpu;
+    const int64_t nw = decode_active_warps(total, tpu, static_cast<int64_t>(gridDim.x) * NCW);
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * NCW + warp;
+    if (gw >= nw) return;
+    const int64_t lo = seg_lo(gw, total, nw);
+    const int64_t cnt = seg_lo(gw + 1, total, nw) - lo;
+    for (int i = 0; i < kPrefetchTiles && i < cnt; ++i) {
+      const int64_t t = lo + i;
+      const int64_t u = t / tpu;
+      const int jt = static_cast<int>(t - u * tpu);
+      const int rows = min(TS, NS - jt * TS);
+      if (rows > 0) prefetch_l2(a.kv + (u * NS + static_cast<int64_t>(jt) * TS) * rb, static_cast<uint32_t>(rows * rb));
+    }
+    return;
+  }
+  if (!step) return;
+  const int dw = warp - NCW;
+  const int base = topk_base(S, W, D);
+  const int b = N + 1 - W - D;   // boundary token of the decision taken in this launch
+  for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
+    if (K > 0) {
+      // [lo, hi) byte range of the unit's long-range scores / positions, in 16-byte units
+      const int64_t lo = (static_cast<int64_t>(u) * NS + base) * 4 / 16 * 16;
+      const int64_t hi = (static_cast<int64_t>(u) * NS + base + K) * 4 / 16 * 16;
+      if (hi > lo) {
+        prefetch_l2(reinterpret_cast<const uint8_t*>(a.score) + lo, static_cast<uint32_t>(hi - lo));
+        prefetch_l2(reinterpret_cast<const uint8_t*>(a.pos) + lo, static_cast<uint32_t>(hi - lo));
+      }
+    }
+    if (b >= S && b < N) {
+      const uint8_t* ur = a.kv + static_cast<int64_t>(u) * NS * rb;
+      prefetch_l2(ur + static_cast<int64_t>(window_slot(b, S, W)) * rb, static_cast<uint32_t>(rb));
+      if (D > 0) prefetch_l2(ur + static_cast<int64_t>(staging_slot(b, S, W, D)) * rb, static_cast<uint32_t>(rb));
+    }
+  }
+  if (dw == 0 && blockIdx.x < a.Hkv && !(a.flags & FLAG_EXTERNAL_SCORES) && a.w1 != nullptr) {
+    const float* w1 = a.w1 + static_cast<size_t>(blockIdx.x) * a.hidden * 2 * a.d;
+    if ((reinterpret_cast<uintptr_t>(w1) & 15u) == 0)
+      prefetch_l2(w1, static_cast<uint32_t>(a.hidden) * 2 * a.d * 4);
+  }
+}
+
 template <typename T, int DH, int G, int NCW, int NSTG>
 __global__ void __launch_bounds__((NCW + NDW) * 32, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ LayerArgs a,
@@ -478,6 +544,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   // prologue as SMs free up, and wait here until the previous one has
   // completed and its writes are visible (everything below reads its results).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  l2_warmup<NCW>(a, step, warp, lane);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
   if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled boxes need 1024-byte alignment
