@@ -334,7 +334,11 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
   T* ou = out + unit * (G * DH);
   const int S = a.S, W = a.W, D = a.D, NS = a.NS, RB = a.row_bytes;
 
-  // ---- round trip 1: segment maxima/sums (lane s holds segment s, s + 32) and the decision ----
+  // ---- one round trip: every load below is issued before any result is used.
+  // segment maxima/sums (lane s holds segments s, s + 32), the decision, the
+  // rows the commit moves (their slots follow from N alone: the boundary
+  // token's row is read even when it is dropped), and the accumulators of the
+  // first kSB segments.
   float mlA[2 * G], mlB[2 * G];
 #pragma unroll
   for (int t = 0; t < 2 * G; ++t) {
@@ -344,28 +348,12 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
   Decision r;
   r.tgt = -1; r.bslot = -1; r.bpos = -1; r.p = N; r.evict = -1; r.sb = 0.f;
   if (step) r = a.dec[static_cast<size_t>(N & 1) * a.units + unit];
-  float M[G], L[G], wA[G], wB[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float ma = (lane < nseg) ? mlA[2 * g] : kNegInf;
-    const float mb = (lane + 32 < nseg) ? mlB[2 * g] : kNegInf;
-    float mx = fmaxf(ma, mb);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    M[g] = mx;
-    wA[g] = (ma != kNegInf) ? fast_exp2(ma - mx) : 0.f;
-    wB[g] = (mb != kNegInf) ? fast_exp2(mb - mx) : 0.f;
-    float ls = wA[g] * mlA[2 * g + 1] + wB[g] * mlB[2 * g + 1];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-    L[g] = ls;
-  }
-
-  // ---- round trip 2: commit source rows (issued first) and segment accumulators ----
   const int p = N;
   const int ns = p < S ? p : window_slot(p, S, W);
   const int o = (p >= S && p - W >= S) ? p - W : -1;
   const int st = (D > 0 && o >= 0) ? staging_slot(o, S, W, D) : -1;
+  const int bb = N - W - D;   // boundary token of this step
+  const int bslot = (bb >= S) ? ((D == 0) ? window_slot(bb, S, W) : staging_slot(bb, S, W, D)) : -1;
   uint8_t* kv = a.kv + static_cast<size_t>(unit) * NS * RB;
   int32_t* pos = a.pos + static_cast<size_t>(unit) * NS;
   float* score = a.score + static_cast<size_t>(unit) * NS;
@@ -378,7 +366,7 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
     for (int t = 0; t < kMaxChunks; ++t) {
       const int i = (lane + 32 * t) * 16;
       if (i < RB) {
-        if (r.tgt >= 0) rb[t] = *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(r.bslot) * RB + i);
+        if (bslot >= 0) rb[t] = *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(bslot) * RB + i);
         if (st >= 0) rn[t] = *reinterpret_cast<const uint4*>(kv + static_cast<size_t>(ns) * RB + i);
         rw[t] = (i < half) ? *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(k_new + unit * DH) + i)
                            : *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(v_new + unit * DH) +
@@ -387,14 +375,9 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
     }
     if (st >= 0) sns = score[ns];
   }
-  float o_acc[G][DPL];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) o_acc[g][e] = 0.f;
-  constexpr int kSB = 4;   // segments per batch of loads
-  for (int s0 = 0; s0 < nseg; s0 += kSB) {
-    float pv[kSB][G][DPL];
+  constexpr int kSB = 4;   // segments per batch of accumulator loads
+  float pv[kSB][G][DPL];
+  auto load_batch = [&](int s0) {
 #pragma unroll
     for (int t = 0; t < kSB; ++t) {
       if (s0 + t < nseg) {
@@ -411,6 +394,33 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
         }
       }
     }
+  };
+  load_batch(0);
+
+  float M[G], L[G], wA[G], wB[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float ma = (lane < nseg) ? mlA[2 * g] : kNegInf;
+    const float mb = (lane + 32 < nseg) ? mlB[2 * g] : kNegInf;
+    float mx = fmaxf(ma, mb);
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+    M[g] = mx;
+    wA[g] = (ma != kNegInf) ? fast_exp2(ma - mx) : 0.f;
+    wB[g] = (mb != kNegInf) ? fast_exp2(mb - mx) : 0.f;
+    float ls = wA[g] * mlA[2 * g + 1] + wB[g] * mlB[2 * g + 1];
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o2);
+    L[g] = ls;
+  }
+
+  float o_acc[G][DPL];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o_acc[g][e] = 0.f;
+  for (int s0 = 0; s0 < nseg; s0 += kSB) {
+    if (s0 > 0) load_batch(s0);
 #pragma unroll
     for (int t = 0; t < kSB; ++t) {
       const int sI = s0 + t;
@@ -434,13 +444,14 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
   if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0) {
     if (r.p != N) set_error(a.err, DEVERR_STATE_MISMATCH);
     if (r.bpos >= 0 && pos[r.bslot] != r.bpos) set_error(a.err, DEVERR_STATE_MISMATCH);
+    if (r.tgt >= 0 && r.bslot != bslot) set_error(a.err, DEVERR_STATE_MISMATCH);
   }
   __syncwarp();
 #pragma unroll
   for (int t = 0; t < kMaxChunks; ++t) {
     const int i = (lane + 32 * t) * 16;
     if (i < RB) {
-      if (r.tgt >= 0) *reinterpret_cast<uint4*>(kv + static_cast<size_t>(r.tgt) * RB + i) = rb[t];
+      if (r.tgt >= 0 && bslot >= 0) *reinterpret_cast<uint4*>(kv + static_cast<size_t>(r.tgt) * RB + i) = rb[t];
       if (st >= 0) *reinterpret_cast<uint4*>(kv + static_cast<size_t>(st) * RB + i) = rn[t];
       *reinterpret_cast<uint4*>(kv + static_cast<size_t>(ns) * RB + i) = rw[t];
     }
