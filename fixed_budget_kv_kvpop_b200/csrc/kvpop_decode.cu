@@ -934,28 +934,47 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
         s[g] = v;
       }
     }
-    const int slot = s0 + j;
-    const bool valid = (j < nsl) && (slot != evict) && vg.slot_ok(slot);
-    const uint32_t vmask = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+    // Slot validity: a tile of occupied slots without the evicted one (the
+    // common case) needs no per-slot test.
+    bool valid = true;
+    uint32_t vmask = 0xffffu;
+    if (!(vg.full && s0 + TS <= vg.nse && (evict < s0 || evict >= s0 + TS))) {
+      const int slot = s0 + j;
+      valid = (j < nsl) && (slot != evict) && vg.slot_ok(slot);
+      vmask = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+    }
     // ---- online softmax (exp2 domain, lazy rescale) ----
+    float sv[G];
+    bool in_range = true;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      sv[g] = valid ? s[g] : kNegInf;
+      in_range = in_range && (sv[g] <= m[g] + kLazy);
+    }
+    // The running max moves only when a tile exceeds it by 2^kLazy; one vote
+    // tells whether any score of the tile does, else no tile max is needed.
+    if (!__all_sync(0xffffffffu, in_range)) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float mt = sv[g];
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+        if (mt > m[g] + kLazy) {   // warp-uniform
+          const float alpha = (m[g] == kNegInf) ? 0.f : fast_exp2(m[g] - mt);
+          m[g] = mt;
+          lp[g] *= alpha;
+#pragma unroll
+          for (int e = 0; e < GE::EPC / 2; ++e) {
+            acc[g][e].x *= alpha;
+            acc[g][e].y *= alpha;
+          }
+        }
+      }
+    }
     float p[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float sv = valid ? s[g] : kNegInf;
-      float mt = sv;
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-      if (mt > m[g] + kLazy) {   // warp-uniform
-        const float alpha = (m[g] == kNegInf) ? 0.f : fast_exp2(m[g] - mt);
-        m[g] = mt;
-        lp[g] *= alpha;
-#pragma unroll
-        for (int e = 0; e < GE::EPC / 2; ++e) {
-          acc[g][e].x *= alpha;
-          acc[g][e].y *= alpha;
-        }
-      }
-      p[g] = valid ? fast_exp2(sv - m[g]) : 0.f;
+      p[g] = valid ? fast_exp2(sv[g] - m[g]) : 0.f;
       lp[g] += p[g];
     }
     if (h == 0) {
