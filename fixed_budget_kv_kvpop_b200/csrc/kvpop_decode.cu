@@ -109,12 +109,11 @@ struct Smem {
   static constexpr int Q = RINGS + NCW * NSTG * GE::STAGE;
   static constexpr int P = Q + NCW * GE::QBYTES;
   static constexpr int QRAW = P + NCW * GE::PBYTES;
-  static constexpr int XS = QRAW + NCW * 2 * QRB;
-  static constexpr int MQ = XS + NDW * 2 * DH * 4;
+  static constexpr int MQ = QRAW + NCW * 2 * QRB;
   static constexpr int BAR = MQ + (kMergeCap + 4) * 4;
   static constexpr int TOTAL = BAR + NCW * (NSTG + 2) * 8;
   static_assert(GE::STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
-  static_assert(Q % 16 == 0 && P % 16 == 0 && QRAW % 16 == 0 && QRB % 16 == 0 && XS % 16 == 0 && MQ % 16 == 0 &&
+  static_assert(Q % 16 == 0 && P % 16 == 0 && QRAW % 16 == 0 && QRB % 16 == 0 && MQ % 16 == 0 &&
                     BAR % 8 == 0,
                 "smem alignment");
   static_assert(TOTAL <= 232448, "shared memory per CTA exceeds 227 KB");
@@ -174,7 +173,7 @@ struct ValidGeom {
 // ntk = long-range slots in use once that step is committed.
 template <typename T>
 __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, int ntk, const Decision* pending,
-                                const T* kn, const T* vn, float ext_new, float* xs) {
+                                const T* kn, const T* vn, float ext_new) {
   const int lane = threadIdx.x & 31;
   const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
   Decision r;
@@ -208,7 +207,7 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
     const int h = u % a.Hkv;
     sb = mlp_score_warp<T>(krow, vrow, a.d, a.w1 + static_cast<size_t>(h) * a.hidden * 2 * a.d,
                            a.b1 + static_cast<size_t>(h) * a.hidden, a.w2 + static_cast<size_t>(h) * a.hidden,
-                           a.b2[h], a.hidden, xs);
+                           a.b2[h], a.hidden);
   }
   r.sb = sb;
   if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0) {
@@ -680,11 +679,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     // ---------------- deciders, then merge helpers ----------------
     if (step) {
       const int dw = warp - NCW;
-      float* xs = reinterpret_cast<float*>(smem + SM::XS) + dw * 2 * DH;
       for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
         const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
         const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, &cur, k_new + static_cast<size_t>(u) * DH,
-                                           v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f, xs);
+                                           v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f);
         if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
         const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
         if (prev == need_of(u) - 1) push_merge(u);
@@ -1054,7 +1052,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
 template <typename T>
 __global__ void __launch_bounds__(128) append_kernel(const LayerArgs a, const T* __restrict__ k_new,
                                                      const T* __restrict__ v_new, const float* __restrict__ ext) {
-  __shared__ __align__(16) float xs[4][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * 4 + warp;
   const int N = a.layer->n_seen;
@@ -1072,7 +1069,7 @@ __global__ void __launch_bounds__(128) append_kernel(const LayerArgs a, const T*
     commit_warp<T>(a, u, N, ntk_after, r, kn, vn, en);
     __threadfence();
     __syncwarp();
-    const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, nullptr, kn, vn, en, xs[warp]);
+    const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, nullptr, kn, vn, en);
     if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
   }
   // last warp of the launch advances the layer counters
@@ -1091,7 +1088,6 @@ __global__ void __launch_bounds__(128) append_kernel(const LayerArgs a, const T*
 
 template <typename T>
 __global__ void __launch_bounds__(128) decide_kernel(const LayerArgs a, int N, int ntk) {
-  __shared__ __align__(16) float xs[4][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * 4 + warp;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -1100,7 +1096,7 @@ __global__ void __launch_bounds__(128) decide_kernel(const LayerArgs a, int N, i
     a.layer->ticket = 0;
   }
   if (u >= a.units) return;
-  const Decision r = decide_warp<T>(a, u, N, ntk, nullptr, nullptr, nullptr, 0.f, xs[warp]);
+  const Decision r = decide_warp<T>(a, u, N, ntk, nullptr, nullptr, nullptr, 0.f);
   if (lane == 0) {
     a.dec[static_cast<size_t>(N & 1) * a.units + u] = r;
     a.state[4 * u + 0] = N;

@@ -217,76 +217,82 @@ __device__ __forceinline__ void set_error(int32_t* err, int32_t bits) {
   atomicOr(err, bits);
 }
 
-// Scorer: s = w2 . relu(W1 x + b1) + b2 for x = [k; v] of one slot row
-// (KVpop page §E.1 headwise inputs, §E.2 stateless MLP scorer), computed by
-// one warp.  Accumulated in fp64 (inputs and fp32 weights are exact in fp64)
-// and rounded once to fp32, the ranking precision (§F).  `xs` is warp-private
-// shared scratch of 2d floats, 16-byte aligned.  Lane j owns hidden units
-// j, j + 32, ...; its W1 row is read as float4.  Returns the score in every
-// lane.
-template <typename T, int ROWS>
-__device__ double mlp_hidden_part(const float* xs, int d, const float* w1, const float* b1, const float* w2) {
-  // lane j owns hidden rows j, j + 32, ... (ROWS of them); W1 rows are read
-  // as float4 in batches of 32 / ROWS per row, so each round trip brings
-  // 16 KB per warp
+// Scorer: s = w2 . relu(W1 x + b1) + b2 for x = [k; v] of one token (KVpop
+// page §E.1 headwise inputs, §E.2 stateless MLP scorer), computed by one warp.
+// Accumulated in fp64 (bf16/fp32 inputs and fp32 weights are exact in fp64)
+// and rounded once to fp32, the ranking precision (§F).  Lane l holds inputs
+// [l * X, l * X + X) of [k; v] (X = 2d / 32) in fp64; for each hidden row the
+// warp reads the whole W1 row (coalesced: 4 cache lines per instruction), each
+// lane forms its X-term partial sum, and a butterfly reduction over 16 rows at
+// a time leaves lane l (< 16) with the pre-activation of row 16 * block + l.
+template <typename T, int D2>
+__device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, const float* w1, const float* b1,
+                                                const float* w2, float b2, int hidden) {
+  constexpr int X = D2 / 32;      // inputs per lane (4 or 8)
+  constexpr int D = D2 / 2;
   const int lane = threadIdx.x & 31;
-  constexpr int kBatch = 32 / ROWS;
-  const int n4 = (2 * d) / 4;
-  const float4* xv = reinterpret_cast<const float4*>(xs);
-  const float4* wr[ROWS];
-  double acc[ROWS];
+  const int i0 = lane * X;
+  const T* src = (i0 < D) ? krow + i0 : vrow + (i0 - D);
+  constexpr int kBytes = X * static_cast<int>(sizeof(T));   // 8, 16 or 32: rows are 16-byte aligned
+  alignas(16) T xr[X];
+  if constexpr (kBytes % 16 == 0) {
 #pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
-    wr[r] = reinterpret_cast<const float4*>(w1 + static_cast<size_t>(lane + 32 * r) * 2 * d);
-    acc[r] = 0.0;
+    for (int q = 0; q < kBytes / 16; ++q) reinterpret_cast<uint4*>(xr)[q] = reinterpret_cast<const uint4*>(src)[q];
+  } else {
+    reinterpret_cast<uint2*>(xr)[0] = reinterpret_cast<const uint2*>(src)[0];
   }
-  for (int i0 = 0; i0 < n4; i0 += kBatch) {
-    float4 w[ROWS][kBatch];
+  double x[X];
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r)
+  for (int e = 0; e < X; ++e) x[e] = static_cast<double>(Elem<T>::to_f32(xr[e]));
+  double part = 0.0;
+  for (int blk = 0; blk < hidden; blk += 16) {
+    double v[16];
 #pragma unroll
-      for (int t = 0; t < kBatch; ++t) w[r][t] = __ldg(wr[r] + i0 + t);
+    for (int r = 0; r < 16; ++r) {
+      const float4* wr = reinterpret_cast<const float4*>(w1 + static_cast<size_t>(blk + r) * D2 + i0);
+      double acc = 0.0;
 #pragma unroll
-    for (int t = 0; t < kBatch; ++t) {
-      const float4 x = xv[i0 + t];
+      for (int q = 0; q < X / 4; ++q) {
+        const float4 w = __ldg(wr + q);
+        acc = fma(static_cast<double>(w.x), x[4 * q + 0], acc);
+        acc = fma(static_cast<double>(w.y), x[4 * q + 1], acc);
+        acc = fma(static_cast<double>(w.z), x[4 * q + 2], acc);
+        acc = fma(static_cast<double>(w.w), x[4 * q + 3], acc);
+      }
+      v[r] = acc;
+    }
+    // fold the two half-warps, then reduce-scatter over the 16 lanes of each:
+    // after the step with offset o, lane l keeps the half of its values whose
+    // index has bit o equal to l's; lanes l and l ^ 16 end with row l & 15
 #pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        double a = acc[r];
-        a = fma(static_cast<double>(w[r][t].x), static_cast<double>(x.x), a);
-        a = fma(static_cast<double>(w[r][t].y), static_cast<double>(x.y), a);
-        a = fma(static_cast<double>(w[r][t].z), static_cast<double>(x.z), a);
-        a = fma(static_cast<double>(w[r][t].w), static_cast<double>(x.w), a);
-        acc[r] = a;
+    for (int r = 0; r < 16; ++r) v[r] += __shfl_xor_sync(0xffffffffu, v[r], 16);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < o; ++i) {
+        const double keep = up ? v[i + o] : v[i];
+        const double send = up ? v[i] : v[i + o];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
       }
     }
+    if (lane < 16) {
+      const int j = blk + lane;
+      part = fma(static_cast<double>(w2[j]), fmax(v[0] + static_cast<double>(b1[j]), 0.0), part);
+    }
   }
-  double part = 0.0;
-#pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
-    const int j = lane + 32 * r;
-    part = fma(static_cast<double>(w2[j]), fmax(acc[r] + static_cast<double>(b1[j]), 0.0), part);
-  }
-  return part;
-}
-
-// hidden in {32, 64, 128}; 2d a multiple of 64 (d = 64 or 128)
-template <typename T>
-__device__ float mlp_score_warp(const T* krow, const T* vrow, int d, const float* w1, const float* b1,
-                                const float* w2, float b2, int hidden, float* xs) {
-  const int lane = threadIdx.x & 31;
-  for (int i = lane; i < d; i += 32) {
-    xs[i] = Elem<T>::to_f32(krow[i]);
-    xs[d + i] = Elem<T>::to_f32(vrow[i]);
-  }
-  __syncwarp();
-  double part;
-  if (hidden == 32) part = mlp_hidden_part<T, 1>(xs, d, w1, b1, w2);
-  else if (hidden == 64) part = mlp_hidden_part<T, 2>(xs, d, w1, b1, w2);
-  else part = mlp_hidden_part<T, 4>(xs, d, w1, b1, w2);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  __syncwarp();
   return static_cast<float>(part + static_cast<double>(b2));
+}
+
+// hidden in {32, 64, 128}; d = 64 or 128; krow, vrow 16-byte aligned.  Returns
+// the score in every lane.
+template <typename T>
+__device__ __noinline__ float mlp_score_warp(const T* krow, const T* vrow, int d, const float* w1, const float* b1,
+                                             const float* w2, float b2, int hidden) {
+  if (d == 128) return mlp_score_rows<T, 256>(krow, vrow, w1, b1, w2, b2, hidden);
+  return mlp_score_rows<T, 128>(krow, vrow, w1, b1, w2, b2, hidden);
 }
 
 // Packed fp32 FMA (sm_100 FFMA2): d = a * b + c on both halves, round-to-nearest.
