@@ -225,9 +225,9 @@ __device__ __forceinline__ void set_error(int32_t* err, int32_t bits) {
 // warp reads the whole W1 row (coalesced: 4 cache lines per instruction), each
 // lane forms its X-term partial sum, and a butterfly reduction over 16 rows at
 // a time leaves lane l (< 16) with the pre-activation of row 16 * block + l.
-template <typename T, int D2>
+template <typename T, int D2, int HID>
 __device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, const float* w1, const float* b1,
-                                                const float* w2, float b2, int hidden) {
+                                                const float* w2, float b2) {
   constexpr int X = D2 / 32;      // inputs per lane (4 or 8)
   constexpr int D = D2 / 2;
   const int lane = threadIdx.x & 31;
@@ -245,7 +245,10 @@ __device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, co
 #pragma unroll
   for (int e = 0; e < X; ++e) x[e] = static_cast<double>(Elem<T>::to_f32(xr[e]));
   double part = 0.0;
-  for (int blk = 0; blk < hidden; blk += 16) {
+  for (int blk = 0; blk < HID; blk += 16) {
+    // b1 and w2 of the row this lane finishes, issued with the block's W1 loads
+    const float b1j = (lane < 16) ? __ldg(b1 + blk + lane) : 0.f;
+    const float w2j = (lane < 16) ? __ldg(w2 + blk + lane) : 0.f;
     double v[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
@@ -276,10 +279,7 @@ __device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, co
         v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
       }
     }
-    if (lane < 16) {
-      const int j = blk + lane;
-      part = fma(static_cast<double>(w2[j]), fmax(v[0] + static_cast<double>(b1[j]), 0.0), part);
-    }
+    if (lane < 16) part = fma(static_cast<double>(w2j), fmax(v[0] + static_cast<double>(b1j), 0.0), part);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -291,8 +291,14 @@ __device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, co
 template <typename T>
 __device__ __noinline__ float mlp_score_warp(const T* krow, const T* vrow, int d, const float* w1, const float* b1,
                                              const float* w2, float b2, int hidden) {
-  if (d == 128) return mlp_score_rows<T, 256>(krow, vrow, w1, b1, w2, b2, hidden);
-  return mlp_score_rows<T, 128>(krow, vrow, w1, b1, w2, b2, hidden);
+  if (d == 128) {
+    if (hidden == 32) return mlp_score_rows<T, 256, 32>(krow, vrow, w1, b1, w2, b2);
+    if (hidden == 64) return mlp_score_rows<T, 256, 64>(krow, vrow, w1, b1, w2, b2);
+    return mlp_score_rows<T, 256, 128>(krow, vrow, w1, b1, w2, b2);
+  }
+  if (hidden == 32) return mlp_score_rows<T, 128, 32>(krow, vrow, w1, b1, w2, b2);
+  if (hidden == 64) return mlp_score_rows<T, 128, 64>(krow, vrow, w1, b1, w2, b2);
+  return mlp_score_rows<T, 128, 128>(krow, vrow, w1, b1, w2, b2);
 }
 
 // Packed fp32 FMA (sm_100 FFMA2): d = a * b + c on both halves, round-to-nearest.
