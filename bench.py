@@ -92,8 +92,8 @@ def step_bytes(w: wl.Workload) -> int:
 # of `bench.py --layers 2 --steps 2 --warmup 1` (the cr88 shape, 2 layers),
 # valid only for the kernel sources whose hash is recorded with it.
 TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024",
-                   "sources_sha256": "34e5352dcee16b2779d522c478505336774746d417be2fdab8e9e92f54ecd306",
-                   "dram_bytes": 275_159_808 + 5_022_720, "algorithmic_bytes": 274_452_512}
+                   "sources_sha256": "ad23ba1c4b1371eb2d358b5005b50bfb421ed43c3f1ee060dedd210ebbebae73",
+                   "dram_bytes": 279_510_272 + 5_801_984, "algorithmic_bytes": 274_452_512}
 
 
 def kernel_sources_sha256() -> str:
