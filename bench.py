@@ -282,19 +282,39 @@ def build_cache(w: wl.Workload, torch):
                          max_prefill_chunk=w.prefill, dtype=w.dtype, scorer_hidden=w.scorer_hidden,
                          w1=w1, b1=b1, w2=w2, b2=b2)
     cache = kp.KVPopCache(cfg, keepalive=weights)
+    stream = torch.cuda.current_stream()
+    prefill_ms = []
     for layer in range(w.n_layers):
         k, v = wl.prompt_kv(w, layer, device="cuda")
-        cache.prefill(layer, k, v)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.prefill(layer, k, v, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        prefill_ms.append(e0.elapsed_time(e1))
         del k, v
     torch.cuda.synchronize()
-    return cache
+    return cache, prefill_ms
+
+
+def prefill_summary(w: wl.Workload, prefill_ms):
+    """The prefill build (one kvpop_prefill per layer, whole prompt in one
+    chunk): time per layer, prompt tokens per second, and the fp64 rate of its
+    scorer (2 * 2d * hidden flops for every token that leaves the window)."""
+    ms = statistics.median(prefill_ms)
+    eligible = max(0, w.prefill - w.window - w.delay - w.sinks)
+    flops = w.batch * w.n_kv_heads * eligible * 2.0 * (2 * w.head_dim) * w.scorer_hidden
+    return {"ms_per_layer": ms, "prompt_tokens_per_s": w.batch * w.prefill / (ms / 1e3),
+            "scorer_fp64_tflops_lower_bound": flops / (ms / 1e3) / 1e12, "layers_timed": len(prefill_ms),
+            "note": "one-off per prompt, not in the decode tokens/s; the TFLOP/s figure divides the scorer's "
+                    "flops by the whole prefill time (select, move and write included)"}
 
 
 def run_gpu(args, w, rank, world, torch):
     dev = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
     t_setup = time.perf_counter()
-    cache = build_cache(w, torch)
+    cache, prefill_ms = build_cache(w, torch)
     NI = max(1, min(args.input_sets, args.steps + args.warmup))
     qs, ks, vs = [], [], []
     for layer in range(w.n_layers):
@@ -384,6 +404,7 @@ def run_gpu(args, w, rank, world, torch):
                      "bytes_per_launch": abytes, "mean_launch_us": attn_mean_ms * 1e3,
                      "launches": n_launches, "peak_kind": peak_kind},
         "gpu_launches": n_launches,
+        "prefill": prefill_summary(w, prefill_ms),
         "clocks": clocks,
         "setup_s": setup_s,
     }

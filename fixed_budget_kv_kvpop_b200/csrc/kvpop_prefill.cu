@@ -145,6 +145,142 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, Chunk
   }
 }
 
+// P1 for the common shapes (2d in {128, 256}, hidden in {32, 64}): the same
+// scores as score_kernel, with W1 (transposed) and the token tile held in
+// shared memory as fp64, so the inner loop is 4 shared loads of 2 doubles per
+// 16 fp64 FMAs and nothing is converted there.  Thread (tq, hq) computes the
+// pre-activations of tokens 4tq..4tq+3 x hidden 4hq..4hq+3; the 16 threads of
+// a token quad then finish w2 . relu(. + b1) by shuffles.  Each block keeps
+// W1 resident and walks kTilesPerBlock token tiles of its unit.
+constexpr int kScore64Threads = 128;
+constexpr int kTilesPerBlock = 8;
+
+template <int D2, int HID>
+struct Score64Geom {
+  static constexpr int TT = 4 * (kScore64Threads / (HID / 4));   // tokens per tile: 32 (HID 64) or 64 (HID 32)
+  static constexpr int WP = HID + 2;                             // padded row of the transposed W1 (doubles)
+  static constexpr int XP = TT + 2;                              // padded row of the transposed tile (doubles)
+  static constexpr int SMEM = (D2 * WP + D2 * XP) * 8;
+};
+
+template <typename T, int D2, int HID>
+__global__ void __launch_bounds__(kScore64Threads) score64_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k,
+                                                                  const T* __restrict__ v, int n,
+                                                                  float* __restrict__ out, int cap) {
+  using SG = Score64Geom<D2, HID>;
+  constexpr int TT = SG::TT, WP = SG::WP, XP = SG::XP;
+  constexpr int HQN = HID / 4;   // threads per token quad
+  extern __shared__ __align__(16) double sm64[];
+  double* Wd = sm64;             // [D2][WP]: Wd[i][j] = W1[j][i]
+  double* Xd = sm64 + D2 * WP;   // [D2][XP]: Xd[i][t] = x_t[i]
+  const int u = blockIdx.y;
+  const int h = u % a.Hkv;
+  const int n_new = cg.e1 - cg.e0;
+  const int tid = threadIdx.x;
+  const int tile0 = blockIdx.x * kTilesPerBlock;
+  if (tile0 * TT >= n_new) return;
+
+  const float* w1 = a.w1 + static_cast<size_t>(h) * HID * D2;
+  {
+    // thread -> a contiguous stretch of one W1 row; 8 float4 loads in flight
+    constexpr int FPT = HID * D2 / kScore64Threads;   // floats per thread (a divisor of D2)
+    const int j = (tid * FPT) / D2, i0 = (tid * FPT) % D2;
+    const float4* src = reinterpret_cast<const float4*>(w1 + static_cast<size_t>(j) * D2 + i0);
+#pragma unroll
+    for (int q0 = 0; q0 < FPT / 4; q0 += 8) {
+      float4 wv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) wv[q] = __ldg(src + q0 + q);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int i = i0 + 4 * (q0 + q);
+        Wd[(i + 0) * WP + j] = static_cast<double>(wv[q].x);
+        Wd[(i + 1) * WP + j] = static_cast<double>(wv[q].y);
+        Wd[(i + 2) * WP + j] = static_cast<double>(wv[q].z);
+        Wd[(i + 3) * WP + j] = static_cast<double>(wv[q].w);
+      }
+    }
+  }
+  const int tq = tid / HQN, hq = tid % HQN;
+  const float* b1 = a.b1 + static_cast<size_t>(h) * HID;
+  const float* w2 = a.w2 + static_cast<size_t>(h) * HID;
+  double b1v[4], w2v[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    b1v[c] = static_cast<double>(b1[4 * hq + c]);
+    w2v[c] = static_cast<double>(w2[4 * hq + c]);
+  }
+  const double b2 = static_cast<double>(a.b2[h]);
+
+  for (int tile = tile0; tile < tile0 + kTilesPerBlock && tile * TT < n_new; ++tile) {
+    const int tok0 = tile * TT;
+    const int ntok = min(TT, n_new - tok0);
+    __syncthreads();   // W1 written (first tile) / previous tile's reads done
+    {
+      // thread -> (token tt, part p): a contiguous stretch of EPT inputs, all
+      // within k or within v; every 16-byte load is issued before any is used
+      constexpr int TPT = kScore64Threads / TT;   // threads per token (2 or 4)
+      constexpr int EPT = D2 / TPT;               // inputs per thread
+      constexpr int NV = EPT * static_cast<int>(sizeof(T)) / 16;
+      const int tt = tid / TPT, p = tid % TPT;
+      alignas(16) T xr[EPT];
+      if (tt < ntok) {
+        const int t = cg.e0 + tok0 + tt;
+        const uint8_t* vs;
+        const uint8_t* ks = token_row<T>(a, cg, u, t, k, v, n, vs);
+        const int i0 = p * EPT;
+        const uint4* src = reinterpret_cast<const uint4*>(
+            (i0 < D2 / 2) ? ks + i0 * sizeof(T) : vs + (i0 - D2 / 2) * sizeof(T));
+#pragma unroll
+        for (int q = 0; q < NV; ++q) reinterpret_cast<uint4*>(xr)[q] = src[q];
+      } else {
+#pragma unroll
+        for (int q = 0; q < NV; ++q) reinterpret_cast<uint4*>(xr)[q] = make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) Xd[(p * EPT + e) * XP + tt] = static_cast<double>(Elem<T>::to_f32(xr[e]));
+    }
+    __syncthreads();
+    double acc[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
+#pragma unroll 4
+    for (int i = 0; i < D2; ++i) {
+      const double2 x01 = *reinterpret_cast<const double2*>(Xd + i * XP + 4 * tq);
+      const double2 x23 = *reinterpret_cast<const double2*>(Xd + i * XP + 4 * tq + 2);
+      const double2 w01 = *reinterpret_cast<const double2*>(Wd + i * WP + 4 * hq);
+      const double2 w23 = *reinterpret_cast<const double2*>(Wd + i * WP + 4 * hq + 2);
+      const double xr[4] = {x01.x, x01.y, x23.x, x23.y};
+      const double wc[4] = {w01.x, w01.y, w23.x, w23.y};
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fma(xr[r], wc[c], acc[r][c]);
+    }
+    double part[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      part[r] = 0.0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) part[r] = fma(w2v[c], fmax(acc[r][c] + b1v[c], 0.0), part[r]);
+    }
+    // reduce over the HQN threads of a token quad (consecutive lanes, HQN | 32)
+#pragma unroll
+    for (int off = 1; off < HQN; off <<= 1)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
+    if (hq == 0) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int tt = 4 * tq + r;
+        if (tt < ntok) out[static_cast<size_t>(u) * cap + tok0 + tt] = static_cast<float>(part[r] + b2);
+      }
+    }
+  }
+}
+
 // ---------------- P2: select + place ----------------
 constexpr int kSelThreads = 1024;
 
@@ -339,6 +475,23 @@ __global__ void write_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k,
   }
 }
 
+template <typename T, int D2, int HID>
+int launch_score64(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T* v, int n, const PrefillScratch& ps,
+                   int n_new, cudaStream_t st) {
+  using SG = Score64Geom<D2, HID>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(score64_kernel<T, D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM) !=
+        cudaSuccess)
+      return -1;
+    attr_set = true;
+  }
+  const int tiles = (n_new + SG::TT - 1) / SG::TT;
+  dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
+  score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, ps.new_score, ps.cap);
+  return 0;
+}
+
 template <typename T>
 int launch_prefill_t(const LayerArgs& a, const PrefillScratch& ps, const T* k, const T* v, int n, int n0, int c0,
                      const float* ext, cudaStream_t st) {
@@ -350,7 +503,16 @@ int launch_prefill_t(const LayerArgs& a, const PrefillScratch& ps, const T* k, c
   cg.c0 = c0;
   const int n_new = cg.e1 - cg.e0;
   if (n_new > ps.cap) return -2;
-  if (n_new > 0) {
+  const bool use64 = !(a.flags & FLAG_EXTERNAL_SCORES) && (a.hidden == 32 || a.hidden == 64) &&
+                     (a.d == 64 || a.d == 128);
+  if (n_new > 0 && use64) {
+    int r = 0;
+    if (a.d == 128 && a.hidden == 64) r = launch_score64<T, 256, 64>(a, cg, k, v, n, ps, n_new, st);
+    else if (a.d == 128) r = launch_score64<T, 256, 32>(a, cg, k, v, n, ps, n_new, st);
+    else if (a.hidden == 64) r = launch_score64<T, 128, 64>(a, cg, k, v, n, ps, n_new, st);
+    else r = launch_score64<T, 128, 32>(a, cg, k, v, n, ps, n_new, st);
+    if (r != 0) return r;
+  } else if (n_new > 0) {
     const int HQ = a.hidden / 4;
     const int TT = 4 * (kScoreThreads / HQ);
     const size_t smem = (a.flags & FLAG_EXTERNAL_SCORES) ? 0
