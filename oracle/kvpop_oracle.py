@@ -36,6 +36,8 @@ design notes):
   order; one decode step is the one-newcomer case (next free slot, else the
   slot of the evicted minimum).  Window slot of token t: S + (t mod W);
   staging slot: S + W + (t mod D); sink slot: t.
+* Temporal decay (optional, §B.3): log-space, ranking by the static priority
+  p_j = s_j - (j + W + D) ln gamma_h in float32 (see decayed_priority).
 """
 from __future__ import annotations
 
@@ -70,6 +72,67 @@ def mlp_score(x: np.ndarray, w1: np.ndarray, b1: np.ndarray, w2: np.ndarray, b2:
 def ranking_score(s) -> np.ndarray:
     """Round scores to float32, the precision of top-k ranking (§F)."""
     return np.asarray(s, np.float64).astype(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Temporal decay (§B.3 Temporal Decay and Static Priorities; teacher policy)
+# ---------------------------------------------------------------------------
+#
+# The page gives shared per-head decay factors 0 < gamma_h < 1 on effective
+# scores (a recency bias) and names the equivalent "static priorities", but no
+# formula.  Reading: log-space decay.  Token j becomes eligible at step
+# e_j = j + W + D; at step q >= e_j its effective score is
+#     eff_q(j) = s_j + (q - e_j) * ln gamma_h,
+# and since q * ln gamma_h is common to every token at step q, ranking by
+# eff_q is ranking by the static priority
+#     p_j = s_j - e_j * ln gamma_h,
+# formed once, in float32 (§F), as one rounding of the exact value.
+
+def round_to_float32(x) -> float:
+    """Round an exact rational (Fraction) or float to the nearest float32,
+    ties to even, in one step (no intermediate float64 rounding)."""
+    from fractions import Fraction
+    fr = Fraction(x)
+    if fr == 0:
+        return 0.0
+    neg = fr < 0
+    a = -fr if neg else fr
+    e = a.numerator.bit_length() - a.denominator.bit_length()   # 2^e <= a < 2^(e+2)
+    while a >= Fraction(2) ** (e + 1):
+        e += 1
+    while a < Fraction(2) ** e:
+        e -= 1
+    q = max(e, -126) - 23                  # weight of the last mantissa bit (subnormals below 2^-126)
+    m = a / Fraction(2) ** q
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    val = float(n) * 2.0 ** q
+    if val > float(np.finfo(np.float32).max):
+        val = math.inf
+    return -val if neg else val
+
+
+def decayed_priority(scores: Sequence[float], W: int, D: int, log_gamma: float) -> np.ndarray:
+    """Static priorities p_j = fl32(s_j - (j + W + D) * ln gamma) of tokens
+    0..n-1 (scores already float32-valued), one rounding of the exact value."""
+    from fractions import Fraction
+    lg = Fraction(float(np.float32(log_gamma)))
+    out = np.empty(len(scores), np.float64)
+    for j, sj in enumerate(scores):
+        sj = float(sj)
+        if math.isnan(sj) or math.isinf(sj):
+            out[j] = sj
+            continue
+        out[j] = round_to_float32(Fraction(sj) - (j + W + D) * lg)
+    return out
+
+
+def effective_score(s_j: float, j: int, q: int, W: int, D: int, log_gamma: float):
+    """eff_q(j) = s_j + (q - e_j) * ln gamma, exactly (a Fraction), for q >= e_j."""
+    from fractions import Fraction
+    return Fraction(float(s_j)) + (q - (j + W + D)) * Fraction(float(np.float32(log_gamma)))
 
 
 # ---------------------------------------------------------------------------

@@ -161,7 +161,65 @@ def pin_attention_closed_forms():
     np.testing.assert_allclose(o[0], (3 * vals[0] + 3 * vals[1] + vals[2]) / 7, atol=1e-14)
 
 
+def pin_decay_hand_example():
+    """§B.3 decay, hand-derived: S=0, W=1, D=0, K=1, every score 0.  Token j
+    becomes eligible at step j + 1 with priority (j + 1) / 8 for
+    ln gamma = -1/8, so the newest eligible token always wins; without decay
+    the scores tie and the oldest token stays.  Priorities of [1, .5, .5] at
+    W=2, D=1, ln gamma = -1/4: 1 + 3/4, 1/2 + 4/4, 1/2 + 5/4."""
+    pr = orc.decayed_priority([1.0, 0.5, 0.5], 2, 1, -0.25)
+    assert list(pr) == [1.75, 1.5, 1.75], list(pr)
+    n = 12
+    zeros = [0.0] * n
+    dec = orc.decayed_priority(zeros, 1, 0, -0.125)
+    assert list(dec) == [(j + 1) / 8 for j in range(n)], list(dec)
+    for q in range(1, n):
+        assert orc.running_topk(dec, q, 0, 1, 0, 1) == [q - 1]
+        assert orc.running_topk(zeros, q, 0, 1, 0, 1) == [0]
+    # ln gamma = 0 leaves the scores as they are
+    sc = orc.ranking_score(np.random.default_rng(3).standard_normal(50))
+    assert np.array_equal(orc.decayed_priority(sc, 5, 2, 0.0), sc)
+
+
+def pin_decay_static_priority_is_effective_score_topk():
+    """The static priority ranks like the effective score at every step: the
+    top-K of eff_q(j) = s_j + (q - e_j) ln gamma, computed exactly for each q
+    by brute force, equals the top-K of the priorities, and the slot
+    simulator (incremental argmin-replace) keeps that same set."""
+    rng = np.random.default_rng(11)
+    S, W, D, K, n = 2, 3, 1, 4, 60
+    lg = float(np.float32(-0.07))
+    sc = orc.ranking_score(rng.standard_normal(n))
+    pr = orc.decayed_priority(sc, W, D, lg)
+    st = orc.SlotState(S, W, D, K)
+    st.append_chunk(S + W + D + 1, pr)   # holds tokens 0..q for q = S + W + D
+    for q in range(S + W + D, n):
+        if q > S + W + D:
+            st.decode(pr)
+        elig = list(orc.eligible_positions(q, S, W, D))
+        brute = sorted(elig, key=lambda j: (orc.effective_score(sc[j], j, q, W, D, lg), -j), reverse=True)[:K]
+        assert sorted(brute) == orc.running_topk(pr, q, S, W, D, K), q
+        assert sorted(brute) == st.topk_positions(), q
+
+
+def pin_float32_single_rounding():
+    """Priorities are rounded once to float32 from the exact value: ties go
+    to even, and a value just above a halfway point rounds up even where a
+    detour through float64 would land on the tie and round down."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    for x in rng.standard_normal(500) * 1e3:
+        assert orc.round_to_float32(float(x)) == float(np.float32(x))
+    one = Fraction(1)
+    assert orc.round_to_float32(one + Fraction(1, 2 ** 24)) == 1.0
+    assert orc.round_to_float32(one + Fraction(3, 2 ** 24)) == 1.0 + 2.0 ** -22
+    assert orc.round_to_float32(one + Fraction(1, 2 ** 24) + Fraction(1, 2 ** 80)) == 1.0 + 2.0 ** -23
+    assert orc.round_to_float32(-(one + Fraction(1, 2 ** 24) + Fraction(1, 2 ** 80))) == -(1.0 + 2.0 ** -23)
+
+
 ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1,
             pin_prefill_chunk_placement, pin_dense_when_budget_covers_context,
             pin_budget_invariant_and_structure, pin_softmax_rows_sum_to_one,
-            pin_delay_equivalence, pin_prefill_is_running_topk, pin_attention_closed_forms]
+            pin_delay_equivalence, pin_prefill_is_running_topk, pin_attention_closed_forms,
+            pin_decay_hand_example, pin_decay_static_priority_is_effective_score_topk,
+            pin_float32_single_rounding]

@@ -86,6 +86,22 @@ def _window_slot_wrong(self, t):
     return self.S + ((t + 1) % self.W)
 
 
+def _decay_sign_flipped(scores, W, D, log_gamma):
+    from fractions import Fraction
+    lg = Fraction(float(np.float32(log_gamma)))
+    return np.array([orc.round_to_float32(Fraction(float(s)) + (j + W + D) * lg) for j, s in enumerate(scores)])
+
+
+def _decay_eligibility_off_by_one(scores, W, D, log_gamma):
+    from fractions import Fraction
+    lg = Fraction(float(np.float32(log_gamma)))
+    return np.array([orc.round_to_float32(Fraction(float(s)) - (j + W + D - 1) * lg) for j, s in enumerate(scores)])
+
+
+def _round_via_float64(x):
+    return float(np.float32(float(x)))
+
+
 MUTATIONS = {
     "tie_goes_to_newer": ("rank_key", _ties_to_newer),
     "eligible_off_by_one": ("eligible_positions", _elig_off_by_one),
@@ -100,6 +116,9 @@ MUTATIONS = {
     "topk_keeps_k_minus_1": ("running_topk", _topk_keeps_k_minus_1),
     "sinks_off_by_one": ("sink_positions", _sinks_off_by_one),
     "softmax_wrong_normaliser": ("attention", _softmax_without_max_shift_wrong_norm),
+    "decay_sign_flipped": ("decayed_priority", _decay_sign_flipped),
+    "decay_eligibility_off_by_one": ("decayed_priority", _decay_eligibility_off_by_one),
+    "priority_double_rounding": ("round_to_float32", _round_via_float64),
 }
 
 
