@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--input-sets", type=int, default=32, help="distinct decode input sets, cycled")
+    ap.add_argument("--log-decay", type=float, default=None,
+                    help="temporal decay: ln(gamma) <= 0 for every KV head (default: no decay)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small cases for ncu captures; renames the workload)")
     return ap.parse_args()
@@ -272,15 +274,19 @@ def run_reference(args, w, rank, world):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def build_cache(w: wl.Workload, torch):
+def build_cache(w: wl.Workload, torch, log_decay=None):
     import fixed_budget_kv_kvpop_b200 as kp
     weights = tuple(t.cuda() for t in wl.scorer_weights(w))
     w1, b1, w2, b2 = weights
+    decay = None
+    if log_decay is not None:
+        decay = torch.full((w.n_layers, w.n_kv_heads), float(log_decay), dtype=torch.float32, device="cuda")
+        weights = weights + (decay,)
     cfg = kp.make_config(batch=w.batch, n_layers=w.n_layers, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                          head_dim=w.head_dim, sinks=w.sinks, window=w.window, topk=w.topk, delay=w.delay,
                          ref_context=w.prefill, compression_ratio=w.compression_ratio,
                          max_prefill_chunk=w.prefill, dtype=w.dtype, scorer_hidden=w.scorer_hidden,
-                         w1=w1, b1=b1, w2=w2, b2=b2)
+                         w1=w1, b1=b1, w2=w2, b2=b2, log_decay=decay)
     cache = kp.KVPopCache(cfg, keepalive=weights)
     stream = torch.cuda.current_stream()
     prefill_ms = []
@@ -314,7 +320,7 @@ def run_gpu(args, w, rank, world, torch):
     dev = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
     t_setup = time.perf_counter()
-    cache, prefill_ms = build_cache(w, torch)
+    cache, prefill_ms = build_cache(w, torch, args.log_decay)
     NI = max(1, min(args.input_sets, args.steps + args.warmup))
     qs, ks, vs = [], [], []
     for layer in range(w.n_layers):
@@ -394,7 +400,7 @@ def run_gpu(args, w, rank, world, torch):
                    "topk": w.topk, "delay": w.delay, "budget": w.budget, "prompt": w.prefill,
                    "compression": round(w.compression_ratio, 4), "parallelism": f"replicas x{world}",
                    "l2": "no flush: inputs (cache %.1f GB) larger than L2" % (w.n_layers * attention_bytes(w) / 1e9),
-                   "input_sets": NI},
+                   "input_sets": NI, "log_decay": args.log_decay},
         "hbm": {"step_bytes": sbytes, "achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
                 "frac_of_8tbs": step_gbs / 8000.0, "peak_kind": peak_kind},
         "roofline": {"kernel": "decode_kernel (fused append + attend, one launch per layer)",

@@ -60,7 +60,7 @@ class kvpop_config(ctypes.Structure):
         ("max_context", ctypes.c_int32), ("max_prefill_chunk", ctypes.c_int32),
         ("dtype", ctypes.c_int32), ("scorer_hidden", ctypes.c_int32),
         ("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
-        ("flags", ctypes.c_uint32),
+        ("flags", ctypes.c_uint32), ("log_decay", ctypes.c_void_p),
     ]
 
 
@@ -130,9 +130,14 @@ def _stream_ptr(stream) -> Optional[int]:
 
 
 def make_config(*, batch, n_layers, n_q_heads, n_kv_heads, head_dim, sinks, window, topk, delay=0,
-                ref_context=0, compression_ratio=0.0, max_context=1 << 30, max_prefill_chunk=0,
+                ref_context=0, compression_ratio=0.0, max_context=None, max_prefill_chunk=0,
                 dtype="bf16", scorer_hidden=64, w1=None, b1=None, w2=None, b2=None,
-                external_scores=False, debug_checks=False) -> kvpop_config:
+                external_scores=False, debug_checks=False, log_decay=None) -> kvpop_config:
+    """log_decay: optional device fp32 tensor [n_layers][n_kv_heads] of
+    ln(gamma_h) <= 0 (temporal decay); max_context defaults to 2^30, or 2^24
+    with decay."""
+    if max_context is None:
+        max_context = (1 << 24) if log_decay is not None else (1 << 30)
     c = kvpop_config()
     c.batch, c.n_layers, c.n_q_heads, c.n_kv_heads, c.head_dim = batch, n_layers, n_q_heads, n_kv_heads, head_dim
     c.sinks, c.window, c.topk, c.delay = sinks, window, topk, delay
@@ -142,6 +147,7 @@ def make_config(*, batch, n_layers, n_q_heads, n_kv_heads, head_dim, sinks, wind
     c.scorer_hidden = scorer_hidden
     c.w1, c.b1, c.w2, c.b2 = _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)
     c.flags = (KVPOP_FLAG_EXTERNAL_SCORES if external_scores else 0) | (KVPOP_FLAG_DEBUG_CHECKS if debug_checks else 0)
+    c.log_decay = _ptr(log_decay)
     return c
 
 

@@ -31,6 +31,7 @@ int validate(const kvpop_config* c) {
   if (c->dtype != KVPOP_DTYPE_F32 && c->dtype != KVPOP_DTYPE_BF16) return KVPOP_ERR_INVALID_ARG;
   if (c->sinks < 0 || c->window < 1 || c->topk < 0 || c->delay < 0) return KVPOP_ERR_BAD_SHAPE;
   if (c->max_context < 1 || c->max_prefill_chunk < 0) return KVPOP_ERR_BAD_SHAPE;
+  if (c->log_decay != nullptr && c->max_context > (1 << 24)) return KVPOP_ERR_BAD_SHAPE;
   if ((c->flags & ~(KVPOP_FLAG_EXTERNAL_SCORES | KVPOP_FLAG_DEBUG_CHECKS)) != 0) return KVPOP_ERR_INVALID_ARG;
   const int G = c->n_q_heads / c->n_kv_heads;
   if (!decode_supported(c->dtype, c->head_dim, G)) return KVPOP_ERR_BAD_SHAPE;
@@ -127,6 +128,7 @@ LayerArgs layer_args(const kvpop_handle* h, int layer) {
   a.max_context = c.max_context;
   a.flags = c.flags;
   a.row_bytes = L.row_bytes;
+  a.log_decay = c.log_decay ? c.log_decay + static_cast<size_t>(layer) * H : nullptr;
   return a;
 }
 

@@ -209,6 +209,7 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
                            a.b1 + static_cast<size_t>(h) * a.hidden, a.w2 + static_cast<size_t>(h) * a.hidden,
                            a.b2[h], a.hidden);
   }
+  sb = ranking_priority(a, u, N, sb);   // b becomes eligible at step b + W + D = N
   r.sb = sb;
   if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0) {
     if (!from_input && pos[rslot] != b) set_error(a.err, DEVERR_STATE_MISMATCH);

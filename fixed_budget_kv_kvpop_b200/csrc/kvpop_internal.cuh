@@ -80,7 +80,16 @@ struct LayerArgs {
   int max_context;
   uint32_t flags;
   int row_bytes;        // 2 * d * sizeof(T)
+  const float* log_decay;   // this layer's ln(gamma) [Hkv], or null (no temporal decay)
 };
+
+// Ranking priority of a token that becomes eligible at step e: its score, or
+// with temporal decay the static priority s - e * ln(gamma_h) in one fp32
+// rounding (page §B.3; e <= 2^24 is exact in fp32).
+__device__ __forceinline__ float ranking_priority(const LayerArgs& a, int unit, int e, float s) {
+  if (a.log_decay == nullptr) return s;
+  return __fmaf_rn(-static_cast<float>(e), a.log_decay[unit % a.Hkv], s);
+}
 
 constexpr uint32_t FLAG_EXTERNAL_SCORES = 1u;
 constexpr uint32_t FLAG_DEBUG_CHECKS = 2u;

@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, Chunk
       float s;
       if (t >= cg.n0) s = ext[static_cast<size_t>(u) * n + (t - cg.n0)];
       else s = a.score[static_cast<size_t>(u) * a.NS + token_slot_in_cache<T>(a, cg, t)];
-      out[static_cast<size_t>(u) * cap + tok0 + i] = s;
+      out[static_cast<size_t>(u) * cap + tok0 + i] = ranking_priority(a, u, t + a.W + a.D, s);
     }
     return;
   }
@@ -140,7 +140,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, Chunk
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int tt = 4 * tq + r;
-      if (tt < ntok) out[static_cast<size_t>(u) * cap + tok0 + tt] = static_cast<float>(part[r] + static_cast<double>(a.b2[h]));
+      if (tt < ntok)
+        out[static_cast<size_t>(u) * cap + tok0 + tt] =
+            ranking_priority(a, u, cg.e0 + tok0 + tt + a.W + a.D, static_cast<float>(part[r] + static_cast<double>(a.b2[h])));
     }
   }
 }
@@ -275,7 +277,9 @@ __global__ void __launch_bounds__(kScore64Threads) score64_kernel(LayerArgs a, C
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int tt = 4 * tq + r;
-        if (tt < ntok) out[static_cast<size_t>(u) * cap + tok0 + tt] = static_cast<float>(part[r] + b2);
+        if (tt < ntok)
+          out[static_cast<size_t>(u) * cap + tok0 + tt] =
+              ranking_priority(a, u, cg.e0 + tok0 + tt + a.W + a.D, static_cast<float>(part[r] + b2));
       }
     }
   }

@@ -97,6 +97,15 @@ typedef struct kvpop_config {
   const float* w2;
   const float* b2;
   uint32_t flags;       /* KVPOP_FLAG_* */
+  /* Optional temporal decay (page §B.3 "Temporal Decay and Static
+   * Priorities"): device fp32 [L][Hkv] holding ln(gamma_h), each finite and
+   * <= 0 (0 < gamma_h <= 1), borrowed for the handle's lifetime; NULL = no
+   * decay.  Token j becomes eligible at step e_j = j + W + D; its effective
+   * score at step q is s_j + (q - e_j) ln gamma_h, which ranks like the
+   * static priority p_j = s_j - e_j ln gamma_h.  The library ranks by p_j,
+   * formed once in fp32 (one rounding, like fmaf), and stores p_j as the
+   * long-range slots' scores.  Requires max_context <= 2^24. */
+  const float* log_decay;
 } kvpop_config;
 
 typedef struct kvpop_handle kvpop_handle;

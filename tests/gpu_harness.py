@@ -37,9 +37,11 @@ class Run:
     ext_dec: Optional[dict] = None
     weights: Optional[tuple] = None
     cache: object = None
+    log_decay: Optional[np.ndarray] = None   # [L][Hkv] ln gamma, or None
 
 
-def build_cache(w: wl.Workload, n_layers: int, external: bool, weights=None, max_chunk=None, debug=True):
+def build_cache(w: wl.Workload, n_layers: int, external: bool, weights=None, max_chunk=None, debug=True,
+                log_decay=None):
     import fixed_budget_kv_kvpop_b200 as kp
     keep = ()
     kw = {}
@@ -51,23 +53,30 @@ def build_cache(w: wl.Workload, n_layers: int, external: bool, weights=None, max
                          head_dim=w.head_dim, sinks=w.sinks, window=w.window, topk=w.topk, delay=w.delay,
                          max_prefill_chunk=max_chunk if max_chunk is not None else max(w.prefill, 1),
                          dtype=w.dtype, scorer_hidden=w.scorer_hidden, external_scores=external,
-                         debug_checks=debug, **kw)
+                         debug_checks=debug, log_decay=log_decay, **kw)
+    if log_decay is not None:
+        keep = tuple(keep) + (log_decay,)
     return kp.KVPopCache(cfg, device="cuda", keepalive=keep)
 
 
 def run_gpu(w: wl.Workload, n_layers: int, n_steps: int, *, external: bool = False, chunks=None,
             inspect_every: int = 1, layers_to_keep: Sequence[int] = (0,), tie_levels: int = 0,
-            master: int = 0, gen_device: str = "cpu", debug=True, split: bool = False) -> Run:
-    """Prefill + n_steps decode steps of every layer on the GPU, through the C ABI."""
+            master: int = 0, gen_device: str = "cpu", debug=True, split: bool = False,
+            log_decay: Optional[np.ndarray] = None) -> Run:
+    """Prefill + n_steps decode steps of every layer on the GPU, through the C ABI.
+    log_decay: optional float32 [n_layers][Hkv] ln gamma (temporal decay)."""
     dev = "cuda"
     weights = None
     if not external:
         weights = tuple(t.to(dev) for t in wl.scorer_weights(w.replace(n_layers=n_layers), master=master))
     chunks = list(chunks) if chunks else ([w.prefill] if w.prefill > 0 else [])
-    cache = build_cache(w, n_layers, external, weights, max_chunk=max(chunks) if chunks else 1, debug=debug)
+    dec_dev = None if log_decay is None else torch.tensor(np.asarray(log_decay, np.float32), device=dev)
+    cache = build_cache(w, n_layers, external, weights, max_chunk=max(chunks) if chunks else 1, debug=debug,
+                        log_decay=dec_dev)
     run = Run(w=w, layers=list(layers_to_keep), prompt_k={}, prompt_v={}, dec_q={}, dec_k={}, dec_v={},
               outs={}, slot_pos={}, slot_score={}, ext_prompt={} if external else None,
-              ext_dec={} if external else None, weights=weights, cache=cache)
+              ext_dec={} if external else None, weights=weights, cache=cache,
+              log_decay=None if log_decay is None else np.asarray(log_decay, np.float32))
     for layer in range(n_layers):
         k, v = wl.prompt_kv(w, layer, master=master, device=gen_device)
         k, v = k.to(dev), v.to(dev)
@@ -143,14 +152,20 @@ def unit_inputs(run: Run, layer: int, unit: int):
 
 
 def unit_scores(run: Run, layer: int, unit: int, k_all, v_all):
+    """The oracle's ranking value of every token of a unit: its float32 score,
+    or with temporal decay its static priority."""
     w = run.w
     b, h = divmod(unit, w.n_kv_heads)
     if run.ext_prompt is not None:
         pr = run.ext_prompt[layer][b, h].double().cpu().numpy()
         dc = np.array([t[b, h].item() for t in run.ext_dec[layer]], dtype=np.float64)
-        return orc.ranking_score(np.concatenate([pr, dc]))
-    w1, b1, w2, b2 = (t.double().cpu().numpy() for t in run.weights)
-    return orc.unit_scores_mlp(k_all, v_all, w1[layer, h], b1[layer, h], w2[layer, h], b2[layer, h])
+        s = orc.ranking_score(np.concatenate([pr, dc]))
+    else:
+        w1, b1, w2, b2 = (t.double().cpu().numpy() for t in run.weights)
+        s = orc.unit_scores_mlp(k_all, v_all, w1[layer, h], b1[layer, h], w2[layer, h], b2[layer, h])
+    if run.log_decay is not None:
+        s = orc.decayed_priority(s, w.window, w.delay, float(run.log_decay[layer, h]))
+    return s
 
 
 def score_tol(s_ref: np.ndarray, all_scores: np.ndarray) -> np.ndarray:

@@ -149,3 +149,34 @@ def test_mlp_scores_match_oracle_exactly_in_fp32():
                 n_exact += int(np.float32(ref[pos[unit, sl]]) == score[unit, sl])
     assert n_total == 4 * w.topk
     assert n_exact == n_total, f"{n_total - n_exact} of {n_total} scores differ from the oracle's fp32 value"
+
+
+@pytest.mark.parametrize("external,S,W,D,K", [(True, 4, 16, 0, 44), (True, 2, 3, 2, 9), (False, 4, 16, 0, 44),
+                                              (False, 2, 8, 5, 20)])
+def test_temporal_decay_matches_oracle(external, S, W, D, K):
+    """Temporal decay (per-head ln gamma, different per layer and head):
+    with identical caller scores the slot maps equal the oracle's bit for
+    bit; with the MLP scorer the long-range slots' fp32 priorities equal the
+    oracle's exactly.  Outputs match at every step.  Includes a chunked
+    prefill, so prompt tokens and decode tokens both take the priority."""
+    _need_gpu()
+    w = wl.Workload("decay_case", batch=2, n_layers=2, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=S, window=W, topk=K, delay=D, prefill=90, decode=40, scorer_hidden=64,
+                    heavy_hitter_frac=0.02)
+    lg = -np.array([[0.003, 0.04], [0.0, 0.2]], np.float32)   # [L][Hkv]; includes no decay (0)
+    chunks = [30, 60]
+    run = gh.run_gpu(w, n_layers=2, n_steps=w.decode, external=external, tie_levels=3 if external else 0,
+                     layers_to_keep=(0, 1), chunks=chunks, log_decay=lg)
+    for layer in (0, 1):
+        for unit in range(w.batch * w.n_kv_heads):
+            gh.check_unit(run, layer, unit, exact_slots=external, atol=gh.BF16_ATOL, chunks=chunks)
+    if not external:
+        base = S + W + D
+        for layer in (0, 1):
+            pos, score, _ = run.cache.inspect(layer)
+            for unit in range(w.batch * w.n_kv_heads):
+                k_all, v_all, _ = gh.unit_inputs(run, layer, unit)
+                pr = gh.unit_scores(run, layer, unit, k_all, v_all)
+                for sl in range(base, pos.shape[1]):
+                    if pos[unit, sl] >= 0:
+                        assert np.float32(pr[pos[unit, sl]]) == score[unit, sl], (layer, unit, sl)
