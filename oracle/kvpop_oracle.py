@@ -369,6 +369,16 @@ def run_unit(k_all: np.ndarray, v_all: np.ndarray, q_steps: np.ndarray, scores: 
                       attended_counts=counts)
 
 
+def linear_score(x: np.ndarray, w: np.ndarray, b: float) -> np.ndarray:
+    """Stateless headwise linear scorer s = w . x + b (§E.2), float64."""
+    return np.asarray(x, np.float64) @ np.asarray(w, np.float64) + float(b)
+
+
+def unit_scores_linear(k_all, v_all, w, b) -> np.ndarray:
+    """Ranking scores of every token of a unit from the linear scorer (§E.2, §F)."""
+    return ranking_score(linear_score(head_input(k_all, v_all), w, b))
+
+
 def unit_scores_mlp(k_all, v_all, w1, b1, w2, b2) -> np.ndarray:
     """Ranking scores of every token of a unit from the MLP scorer (§E.2, §F)."""
     return ranking_score(mlp_score(head_input(k_all, v_all), w1, b1, w2, b2))

@@ -217,9 +217,24 @@ def pin_float32_single_rounding():
     assert orc.round_to_float32(-(one + Fraction(1, 2 ** 24) + Fraction(1, 2 ** 80))) == -(1.0 + 2.0 ** -23)
 
 
+def pin_linear_scorer():
+    """§E.2 linear scorer: a hand example (x = [k; v] = [1, 2, -1, 0.5],
+    w = [0.5, -0.25, 2, 4], b = 0.125: 0.5 - 0.5 - 2 + 2 + 0.125), and the
+    identity relu(t) - relu(-t) = t: an MLP with hidden rows [w; -w],
+    w2 = [1, -1], b1 = 0 is the linear scorer w . x + b2."""
+    s = orc.linear_score(orc.head_input(np.array([1.0, 2.0]), np.array([-1.0, 0.5])),
+                         np.array([0.5, -0.25, 2.0, 4.0]), 0.125)
+    assert float(s) == 0.125, float(s)
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((20, 8))
+    w = rng.standard_normal(8)
+    mlp = orc.mlp_score(x, np.stack([w, -w]), np.zeros(2), np.array([1.0, -1.0]), 0.3)
+    assert np.allclose(mlp, orc.linear_score(x, w, 0.3), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1,
             pin_prefill_chunk_placement, pin_dense_when_budget_covers_context,
             pin_budget_invariant_and_structure, pin_softmax_rows_sum_to_one,
             pin_delay_equivalence, pin_prefill_is_running_topk, pin_attention_closed_forms,
             pin_decay_hand_example, pin_decay_static_priority_is_effective_score_topk,
-            pin_float32_single_rounding]
+            pin_float32_single_rounding, pin_linear_scorer]

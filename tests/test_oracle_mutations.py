@@ -102,6 +102,10 @@ def _round_via_float64(x):
     return float(np.float32(float(x)))
 
 
+def _linear_drops_bias(x, w, b):
+    return np.asarray(x, np.float64) @ np.asarray(w, np.float64)
+
+
 MUTATIONS = {
     "tie_goes_to_newer": ("rank_key", _ties_to_newer),
     "eligible_off_by_one": ("eligible_positions", _elig_off_by_one),
@@ -119,6 +123,7 @@ MUTATIONS = {
     "decay_sign_flipped": ("decayed_priority", _decay_sign_flipped),
     "decay_eligibility_off_by_one": ("decayed_priority", _decay_eligibility_off_by_one),
     "priority_double_rounding": ("round_to_float32", _round_via_float64),
+    "linear_drops_bias": ("linear_score", _linear_drops_bias),
 }
 
 
