@@ -22,7 +22,7 @@ struct Layout {
   size_t pacc_off, pml_off, ticket_off, pre_score_off, pre_tgt_off, err_off, total;
 };
 
-bool hidden_supported(int h) { return h == 32 || h == 64 || h == 128; }
+bool hidden_supported(int h) { return h == 0 || h == 32 || h == 64 || h == 128; }   // 0: linear scorer
 
 int validate(const kvpop_config* c) {
   if (!c) return KVPOP_ERR_INVALID_ARG;
@@ -37,7 +37,7 @@ int validate(const kvpop_config* c) {
   if (!decode_supported(c->dtype, c->head_dim, G)) return KVPOP_ERR_BAD_SHAPE;
   if (!(c->flags & KVPOP_FLAG_EXTERNAL_SCORES)) {
     if (!hidden_supported(c->scorer_hidden)) return KVPOP_ERR_BAD_SHAPE;
-    if (!c->w1 || !c->b1 || !c->w2 || !c->b2) return KVPOP_ERR_INVALID_ARG;
+    if (!c->w1 || !c->b2 || (c->scorer_hidden > 0 && (!c->b1 || !c->w2))) return KVPOP_ERR_INVALID_ARG;
   }
   const double budget = static_cast<double>(c->sinks) + c->window + c->topk;
   if (budget + c->delay > 2147483647.0 / 2) return KVPOP_ERR_BAD_SHAPE;
@@ -108,9 +108,9 @@ LayerArgs layer_args(const kvpop_handle* h, int layer) {
   a.dec = reinterpret_cast<Decision*>(h->mem + L.dec_off + layer * L.dec_stride);
   const size_t hid = c.scorer_hidden, d2 = 2 * static_cast<size_t>(c.head_dim), H = c.n_kv_heads;
   if (c.w1) {
-    a.w1 = c.w1 + layer * H * hid * d2;
-    a.b1 = c.b1 + layer * H * hid;
-    a.w2 = c.w2 + layer * H * hid;
+    a.w1 = c.w1 + layer * H * (hid > 0 ? hid : 1) * d2;   // linear scorer: one row per head
+    a.b1 = (hid > 0 && c.b1) ? c.b1 + layer * H * hid : nullptr;
+    a.w2 = (hid > 0 && c.w2) ? c.w2 + layer * H * hid : nullptr;
     a.b2 = c.b2 + layer * H;
   }
   a.err = reinterpret_cast<int32_t*>(h->mem + L.err_off);

@@ -205,9 +205,7 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
     sb = from_input ? ext_new : score[rslot];
   } else {
     const int h = u % a.Hkv;
-    sb = mlp_score_warp<T>(krow, vrow, a.d, a.w1 + static_cast<size_t>(h) * a.hidden * 2 * a.d,
-                           a.b1 + static_cast<size_t>(h) * a.hidden, a.w2 + static_cast<size_t>(h) * a.hidden,
-                           a.b2[h], a.hidden);
+    sb = mlp_score_warp<T>(krow, vrow, a.d, head_w1(a, h), head_b1(a, h), head_w2(a, h), a.b2[h], a.hidden);
   }
   sb = ranking_priority(a, u, N, sb);   // b becomes eligible at step b + W + D = N
   r.sb = sb;
@@ -523,9 +521,9 @@ __device__ __forceinline__ void l2_warmup(const LayerArgs& a, bool step, int war
     }
   }
   if (dw == 0 && blockIdx.x < a.Hkv && !(a.flags & FLAG_EXTERNAL_SCORES) && a.w1 != nullptr) {
-    const float* w1 = a.w1 + static_cast<size_t>(blockIdx.x) * a.hidden * 2 * a.d;
+    const float* w1 = head_w1(a, blockIdx.x);
     if ((reinterpret_cast<uintptr_t>(w1) & 15u) == 0)
-      prefetch_l2(w1, static_cast<uint32_t>(a.hidden) * 2 * a.d * 4);
+      prefetch_l2(w1, static_cast<uint32_t>(a.hidden > 0 ? a.hidden : 1) * 2 * a.d * 4);
   }
 }
 

@@ -83,6 +83,18 @@ struct LayerArgs {
   const float* log_decay;   // this layer's ln(gamma) [Hkv], or null (no temporal decay)
 };
 
+// Scorer weights of KV head h in this layer: W1 rows (one row for the linear
+// scorer), b1 and w2 (null for the linear scorer).
+__host__ __device__ __forceinline__ const float* head_w1(const LayerArgs& a, int h) {
+  return a.w1 + static_cast<size_t>(h) * (a.hidden > 0 ? a.hidden : 1) * 2 * a.d;
+}
+__host__ __device__ __forceinline__ const float* head_b1(const LayerArgs& a, int h) {
+  return a.hidden > 0 ? a.b1 + static_cast<size_t>(h) * a.hidden : nullptr;
+}
+__host__ __device__ __forceinline__ const float* head_w2(const LayerArgs& a, int h) {
+  return a.hidden > 0 ? a.w2 + static_cast<size_t>(h) * a.hidden : nullptr;
+}
+
 // Ranking priority of a token that becomes eligible at step e: its score, or
 // with temporal decay the static priority s - e * ln(gamma_h) in one fp32
 // rounding (page §B.3; e <= 2^24 is exact in fp32).
@@ -295,11 +307,48 @@ __device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, co
   return static_cast<float>(part + static_cast<double>(b2));
 }
 
-// hidden in {32, 64, 128}; d = 64 or 128; krow, vrow 16-byte aligned.  Returns
-// the score in every lane.
+// Stateless headwise linear scorer s = w . [k; v] + b (page §E.2), one warp:
+// lane l holds inputs [l * X, l * X + X) and the matching weights; fp64 dot
+// product, warp reduction, one rounding to fp32.
+template <typename T, int D2>
+__device__ __forceinline__ float linear_score_rows(const T* krow, const T* vrow, const float* w, float b) {
+  constexpr int X = D2 / 32;
+  constexpr int D = D2 / 2;
+  const int lane = threadIdx.x & 31;
+  const int i0 = lane * X;
+  const T* src = (i0 < D) ? krow + i0 : vrow + (i0 - D);
+  constexpr int kBytes = X * static_cast<int>(sizeof(T));
+  alignas(16) T xr[X];
+  if constexpr (kBytes % 16 == 0) {
+#pragma unroll
+    for (int q = 0; q < kBytes / 16; ++q) reinterpret_cast<uint4*>(xr)[q] = reinterpret_cast<const uint4*>(src)[q];
+  } else {
+    reinterpret_cast<uint2*>(xr)[0] = reinterpret_cast<const uint2*>(src)[0];
+  }
+  double acc = 0.0;
+#pragma unroll
+  for (int q = 0; q < X / 4; ++q) {
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(w + i0) + q);
+    acc = fma(static_cast<double>(wv.x), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 0])), acc);
+    acc = fma(static_cast<double>(wv.y), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 1])), acc);
+    acc = fma(static_cast<double>(wv.z), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 2])), acc);
+    acc = fma(static_cast<double>(wv.w), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 3])), acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return static_cast<float>(acc + static_cast<double>(b));
+}
+
+// hidden in {32, 64, 128} (MLP) or 0 (linear: w1 is the weight row, b2 the
+// bias); d = 64 or 128; krow, vrow 16-byte aligned.  Returns the score in
+// every lane.
 template <typename T>
 __device__ __noinline__ float mlp_score_warp(const T* krow, const T* vrow, int d, const float* w1, const float* b1,
                                              const float* w2, float b2, int hidden) {
+  if (hidden == 0) {
+    if (d == 128) return linear_score_rows<T, 256>(krow, vrow, w1, b2);
+    return linear_score_rows<T, 128>(krow, vrow, w1, b2);
+  }
   if (d == 128) {
     if (hidden == 32) return mlp_score_rows<T, 256, 32>(krow, vrow, w1, b1, w2, b2);
     if (hidden == 64) return mlp_score_rows<T, 256, 64>(krow, vrow, w1, b1, w2, b2);

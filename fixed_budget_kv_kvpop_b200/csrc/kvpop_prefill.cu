@@ -285,6 +285,34 @@ __global__ void __launch_bounds__(kScore64Threads) score64_kernel(LayerArgs a, C
   }
 }
 
+// P1 with the stateless headwise linear scorer (page §E.2), s = w . [k; v] + b:
+// one warp per token, the weight row in registers, fp64 dot product.
+constexpr int kLinearThreads = 256;
+constexpr int kLinearTokensPerWarp = 8;
+
+template <typename T, int D2>
+__global__ void __launch_bounds__(kLinearThreads) linear_score_kernel(LayerArgs a, ChunkGeom cg,
+                                                                      const T* __restrict__ k,
+                                                                      const T* __restrict__ v, int n,
+                                                                      float* __restrict__ out, int cap) {
+  const int u = blockIdx.y;
+  const int h = u % a.Hkv;
+  const int n_new = cg.e1 - cg.e0;
+  const int warp = threadIdx.x >> 5;
+  const int tok0 = (blockIdx.x * (kLinearThreads / 32) + warp) * kLinearTokensPerWarp;
+  const float* w = head_w1(a, h);
+  const float b = a.b2[h];
+  for (int i = 0; i < kLinearTokensPerWarp; ++i) {
+    const int r = tok0 + i;
+    if (r >= n_new) break;
+    const int t = cg.e0 + r;
+    const uint8_t* vs;
+    const uint8_t* ks = token_row<T>(a, cg, u, t, k, v, n, vs);
+    const float s = linear_score_rows<T, D2>(reinterpret_cast<const T*>(ks), reinterpret_cast<const T*>(vs), w, b);
+    if ((threadIdx.x & 31) == 0) out[static_cast<size_t>(u) * cap + r] = ranking_priority(a, u, t + a.W + a.D, s);
+  }
+}
+
 // ---------------- P2: select + place ----------------
 constexpr int kSelThreads = 1024;
 
@@ -516,6 +544,13 @@ int launch_prefill_t(const LayerArgs& a, const PrefillScratch& ps, const T* k, c
     else if (a.hidden == 64) r = launch_score64<T, 128, 64>(a, cg, k, v, n, ps, n_new, st);
     else r = launch_score64<T, 128, 32>(a, cg, k, v, n, ps, n_new, st);
     if (r != 0) return r;
+  } else if (n_new > 0 && a.hidden == 0 && !(a.flags & FLAG_EXTERNAL_SCORES)) {
+    constexpr int per_block = (kLinearThreads / 32) * kLinearTokensPerWarp;
+    dim3 grid((n_new + per_block - 1) / per_block, a.units);
+    if (a.d == 128)
+      linear_score_kernel<T, 256><<<grid, kLinearThreads, 0, st>>>(a, cg, k, v, n, ps.new_score, ps.cap);
+    else
+      linear_score_kernel<T, 128><<<grid, kLinearThreads, 0, st>>>(a, cg, k, v, n, ps.new_score, ps.cap);
   } else if (n_new > 0) {
     const int HQ = a.hidden / 4;
     const int TT = 4 * (kScoreThreads / HQ);

@@ -86,12 +86,14 @@ typedef struct kvpop_config {
   int32_t max_context;  /* positions must stay below this (int32 positions) */
   int32_t max_prefill_chunk; /* largest n_tokens of one kvpop_prefill call */
   int32_t dtype;        /* KVPOP_DTYPE_F32 or KVPOP_DTYPE_BF16 */
-  int32_t scorer_hidden; /* MLP 2d -> hidden -> 1; hidden in {32, 64, 128} */
+  int32_t scorer_hidden; /* MLP 2d -> hidden -> 1 with hidden in {32, 64, 128}, or 0 = linear scorer */
   /* Scorer weights, device fp32, borrowed for the handle's lifetime
    * (may be NULL with KVPOP_FLAG_EXTERNAL_SCORES):
    *   w1 [L][Hkv][hidden][2d]  (input x = [k; v], page §E.1)
    *   b1 [L][Hkv][hidden], w2 [L][Hkv][hidden], b2 [L][Hkv]
-   * score = w2 . relu(W1 x + b1) + b2 (page §E.2, stateless MLP scorer). */
+   * score = w2 . relu(W1 x + b1) + b2 (page §E.2, stateless MLP scorer).
+   * With scorer_hidden = 0 (page §E.2, stateless headwise linear scorer):
+   * w1 [L][Hkv][2d] and b2 [L][Hkv], score = w1 . x + b2; b1, w2 may be NULL. */
   const float* w1;
   const float* b1;
   const float* w2;

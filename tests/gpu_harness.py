@@ -68,7 +68,9 @@ def run_gpu(w: wl.Workload, n_layers: int, n_steps: int, *, external: bool = Fal
     dev = "cuda"
     weights = None
     if not external:
-        weights = tuple(t.to(dev) for t in wl.scorer_weights(w.replace(n_layers=n_layers), master=master))
+        # scorer_hidden 0 = linear scorer: one weight row per head (w1[..., 0, :]) and b2
+        wshape = w.replace(n_layers=n_layers, scorer_hidden=max(w.scorer_hidden, 1))
+        weights = tuple(t.to(dev) for t in wl.scorer_weights(wshape, master=master))
     chunks = list(chunks) if chunks else ([w.prefill] if w.prefill > 0 else [])
     dec_dev = None if log_decay is None else torch.tensor(np.asarray(log_decay, np.float32), device=dev)
     cache = build_cache(w, n_layers, external, weights, max_chunk=max(chunks) if chunks else 1, debug=debug,
@@ -162,7 +164,10 @@ def unit_scores(run: Run, layer: int, unit: int, k_all, v_all):
         s = orc.ranking_score(np.concatenate([pr, dc]))
     else:
         w1, b1, w2, b2 = (t.double().cpu().numpy() for t in run.weights)
-        s = orc.unit_scores_mlp(k_all, v_all, w1[layer, h], b1[layer, h], w2[layer, h], b2[layer, h])
+        if w.scorer_hidden == 0:
+            s = orc.unit_scores_linear(k_all, v_all, w1[layer, h, 0], b2[layer, h])
+        else:
+            s = orc.unit_scores_mlp(k_all, v_all, w1[layer, h], b1[layer, h], w2[layer, h], b2[layer, h])
     if run.log_decay is not None:
         s = orc.decayed_priority(s, w.window, w.delay, float(run.log_decay[layer, h]))
     return s

@@ -180,3 +180,27 @@ def test_temporal_decay_matches_oracle(external, S, W, D, K):
                 for sl in range(base, pos.shape[1]):
                     if pos[unit, sl] >= 0:
                         assert np.float32(pr[pos[unit, sl]]) == score[unit, sl], (layer, unit, sl)
+
+
+@pytest.mark.parametrize("dtype,d,hq,hkv", [("bf16", 128, 8, 2), ("f32", 64, 4, 2)])
+def test_linear_scorer_matches_oracle(dtype, d, hq, hkv):
+    """Stateless headwise linear scorer (scorer_hidden = 0): GPU scores of
+    the long-range tokens equal the oracle's float64-then-float32 scores
+    exactly, sets and outputs match at every step, over a chunked prefill
+    and decode with a staging ring."""
+    _need_gpu()
+    w = wl.Workload("linear_case", batch=2, n_layers=1, n_q_heads=hq, n_kv_heads=hkv, head_dim=d, dtype=dtype,
+                    sinks=3, window=10, topk=30, delay=2, prefill=100, decode=30, scorer_hidden=0,
+                    heavy_hitter_frac=0.02 if dtype == "bf16" else 0.0)
+    chunks = [37, 63]
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, chunks=chunks)
+    atol = gh.F32_ATOL if dtype == "f32" else gh.BF16_ATOL
+    pos, score, _ = run.cache.inspect(0)
+    base = w.sinks + w.window + w.delay
+    for unit in range(w.batch * w.n_kv_heads):
+        gh.check_unit(run, 0, unit, exact_slots=False, atol=atol, chunks=chunks)
+        k_all, v_all, _ = gh.unit_inputs(run, 0, unit)
+        ref = gh.unit_scores(run, 0, unit, k_all, v_all)
+        for sl in range(base, pos.shape[1]):
+            assert pos[unit, sl] >= 0
+            assert np.float32(ref[pos[unit, sl]]) == score[unit, sl], (unit, sl)
