@@ -96,8 +96,8 @@ def step_bytes(w: wl.Workload) -> int:
 # of `bench.py --layers 2 --steps 2 --warmup 1` (the cr88 shape, 2 layers),
 # valid only for the kernel sources whose hash is recorded with it.
 TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024",
-                   "sources_sha256": "ad23ba1c4b1371eb2d358b5005b50bfb421ed43c3f1ee060dedd210ebbebae73",
-                   "dram_bytes": 279_510_272 + 5_801_984, "algorithmic_bytes": 274_452_512}
+                   "sources_sha256": "85a54fb15d497557650e5e985170016fa1eabd1f08cea0b8e3115cc976a3580b",
+                   "dram_bytes": 279_369_472 + 5_617_920, "algorithmic_bytes": 274_452_512}
 
 
 def kernel_sources_sha256() -> str:

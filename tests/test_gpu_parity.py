@@ -204,3 +204,23 @@ def test_linear_scorer_matches_oracle(dtype, d, hq, hkv):
         for sl in range(base, pos.shape[1]):
             assert pos[unit, sl] >= 0
             assert np.float32(ref[pos[unit, sl]]) == score[unit, sl], (unit, sl)
+
+
+def test_full_size_target_config_sampled_units():
+    """The 87.5%-compression target shape at full size (64 rows x 8 KV heads,
+    prompt 8192, B = 1024 = 4 + 128 + 892, G = 4, bf16, MLP scorer), one
+    layer, in the launch configuration bench.py times (one CTA per SM, 10
+    consumer + 2 decider warps, 64 tiles per unit split over ~3 warps).
+    Prefill plus 4 fused decode steps; three sampled units (first, middle,
+    last) checked against the oracle at every step: outputs, long-range sets
+    and exact fp32 scores."""
+    _need_gpu()
+    w = wl.QWEN3_4B_CR88.replace(name="full_size_case", n_layers=1, decode=4)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, gen_device="cuda", debug=False)
+    units = w.batch * w.n_kv_heads
+    for unit in (0, units // 2 + 3, units - 1):
+        gh.check_unit(run, 0, unit, exact_slots=False, atol=gh.BF16_ATOL)
+    pos, score, state = run.cache.inspect(0)
+    base = w.sinks + w.window + w.delay
+    assert (pos[:, base:] >= 0).all()                       # every long-range slot filled
+    assert (state[:, 0] == w.prefill + w.decode).all()     # every unit advanced
