@@ -273,6 +273,26 @@ def run_reference(args, w, rank, world):
 
 
 # ---------------------------------------------------------------------------
+# Multi-GPU: independent replicas, one per rank (no data-path collective)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(value: float, world: int, torch, device) -> float:
+    """The slowest rank's time: every rank must call this at the same point
+    (one all-reduce, MAX); device 'cuda' under NCCL, 'cpu' under gloo."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(batch: int, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job decode tokens/s: every rank decodes `batch` rows for `steps`
+    steps, and the job takes the slowest rank's time."""
+    return batch * steps * world / (elapsed_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 
@@ -389,13 +409,8 @@ def run_gpu(args, w, rank, world, torch):
     st, bits = cache.get_error()
     if st != 0:
         raise RuntimeError(f"device error in timed region: status {st} bits {bits}")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-
-    tokens = w.batch * args.steps * world
-    value = tokens / (elapsed_ms / 1e3)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, torch, "cuda")
+    value = replica_throughput(w.batch, args.steps, world, elapsed_ms)
     peak, peak_kind = measured_peaks()
     sbytes = step_bytes(w)
     step_gbs = sbytes * args.steps / (elapsed_ms / 1e3) / 1e9
@@ -500,14 +515,11 @@ def run_e2e(args, w, cache, torch, world):
     end.record(s_out)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, torch, "cuda")
     es = 2 if w.dtype == "bf16" else 4
     h2d = L * w.batch * (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim * es
     d2h = L * w.batch * w.n_q_heads * w.head_dim * es
-    return {"value": w.batch * K * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    return {"value": replica_throughput(w.batch, K, world, ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": K, "ms_per_step": ms / K}
 
 
