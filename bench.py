@@ -214,6 +214,20 @@ class OracleSample:
         self.i += 1
 
 
+def host_info():
+    """The host the CPU oracle runs on: logical CPUs and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_threads_limit():
     try:
         from threadpoolctl import threadpool_limits
@@ -266,7 +280,8 @@ def run_reference(args, w, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name, "sample": desc},
-        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc,
+                         "host": host_info()},
         "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -543,7 +558,8 @@ def main():
         res = run_gpu(args, w, rank, world, torch)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             v, desc = oracle_tokens_per_s(w, args.cpu_seconds)
-            res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc}
+            res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc,
+                                   "host": host_info()}
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
