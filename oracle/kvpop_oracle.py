@@ -38,6 +38,9 @@ design notes):
   staging slot: S + W + (t mod D); sink slot: t.
 * Temporal decay (optional, §B.3): log-space, ranking by the static priority
   p_j = s_j - (j + W + D) ln gamma_h in float32 (see decayed_priority).
+* Parallel prefill attention (§C.1, §C.2): every prompt position q attends to
+  the set a decode step at q would attend to.  Running cutoff of token j: with
+  m = q - W - D, j is kept exactly for m in [j, c_j) (see running_cutoffs).
 """
 from __future__ import annotations
 
@@ -388,3 +391,72 @@ def dense_causal_attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray) 
     """Plain dense attention of one query [G][d] over all keys/values up to itself."""
     o, _ = attention(q, keys, values)
     return o
+
+
+# ---------------------------------------------------------------------------
+# Parallel sparse prefill attention (§C Efficient Running Top-k Sparse
+# Attention: §C.1 Mask Definition, §C.2 Fenwick-Tree Cutoff Computation)
+# ---------------------------------------------------------------------------
+#
+# Over a whole prompt of n tokens, query position q attends to exactly the
+# set a decode step at q would attend to: sinks, the recent W + D positions
+# and the running top-k of the eligible tokens at q (update before attend).
+# The page computes, per head, one "running cutoff" per token and evaluates
+# the mask from it on the fly.  Reading of the cutoff: with m = q - W - D the
+# newest eligible position at query q, token j is in the long-range set at
+# exactly the steps whose m lies in [j, c_j); the oracle computes c_j by its
+# definition (the first m at which j is not kept), not by the tree.
+
+INT32_MAX = 2 ** 31 - 1
+
+
+def running_cutoffs(scores: Sequence[float], n: int, S: int, W: int, D: int, K: int) -> List[int]:
+    """Running cutoff c_j of every token of a length-n prompt, by brute force.
+
+    c_j (S <= j <= n-1-W-D) = the first newest-eligible position m >= j at
+    which j is not in running_topk (c_j = j: never admitted), or INT32_MAX if
+    j is still kept at the last position.  Tokens that never become eligible
+    in the prompt (sinks, the last W + D positions) get -1.
+    """
+    c = [-1] * n
+    m_last = n - 1 - W - D
+    for j in range(S, m_last + 1):
+        c[j] = INT32_MAX
+    for m in range(S, m_last + 1):
+        kept = set(running_topk(scores, m + W + D, S, W, D, K))
+        for j in range(S, m + 1):
+            if c[j] == INT32_MAX and j not in kept:
+                c[j] = m
+    return c
+
+
+def attention_lse(q: np.ndarray, keys: np.ndarray) -> np.ndarray:
+    """Log-normaliser log sum_j exp(q_g . k_j / sqrt(d)) of each query head, float64."""
+    q = np.asarray(q, np.float64)
+    logits = (q @ np.asarray(keys, np.float64).T) / math.sqrt(q.shape[-1])
+    mx = logits.max(axis=-1)
+    return mx + np.log(np.exp(logits - mx[:, None]).sum(axis=-1))
+
+
+def prefill_attention(q_all: np.ndarray, k_all: np.ndarray, v_all: np.ndarray, scores: Sequence[float],
+                      S: int, W: int, D: int, K: int):
+    """Attention outputs of every prompt position under the fixed-budget mask.
+
+    q_all: [n][G][d] queries; k_all, v_all: [n][d]; scores: ranking scores of
+    the n tokens.  Position q attends to attended_positions(q, ...) with the
+    brute-force running top-k at q (§C.1, §I).  Returns (out [n][G][d],
+    lse [n][G] log-normalisers, counts [n] attended tokens per position).
+    """
+    n = len(k_all)
+    G, d = q_all.shape[1], q_all.shape[2]
+    out = np.zeros((n, G, d))
+    lse = np.zeros((n, G))
+    counts = []
+    for q in range(n):
+        T = running_topk(scores, q, S, W, D, K)
+        A = attended_positions(q, S, W, D, T)
+        o, _ = attention(q_all[q], k_all[A], v_all[A])
+        out[q] = o
+        lse[q] = attention_lse(q_all[q], k_all[A])
+        counts.append(len(A))
+    return out, lse, counts

@@ -232,9 +232,131 @@ def pin_linear_scorer():
     assert np.allclose(mlp, orc.linear_score(x, w, 0.3), rtol=0, atol=1e-12)
 
 
+
+# ---------------------------------------------------------------------------
+# Parallel sparse prefill attention (§C.1 Mask Definition, §C.2 Fenwick-Tree
+# Cutoff Computation)
+# ---------------------------------------------------------------------------
+
+def pin_prefill_mask_hand_example():
+    """Hand-derived cutoffs and attended sets; with zero queries and one-hot
+    values the prefill output of row q is the indicator of its attended set
+    divided by its size, and the log-normaliser is log |A_q|."""
+    g = _load("prefill_mask_s1_w1_d0_k1.json")
+    S, W, D, K, s = g["S"], g["W"], g["D"], g["K"], g["scores"]
+    n = len(s)
+    assert orc.running_cutoffs(s, n, S, W, D, K) == g["cutoffs"]
+    for q in range(n):
+        T = orc.running_topk(s, q, S, W, D, K)
+        assert orc.attended_positions(q, S, W, D, T) == g["attended"][q], q
+    out, lse, counts = orc.prefill_attention(np.zeros((n, 1, n)), np.zeros((n, n)), np.eye(n), s, S, W, D, K)
+    for q in range(n):
+        A = g["attended"][q]
+        expect = np.zeros(n)
+        expect[A] = 1.0 / len(A)
+        np.testing.assert_allclose(out[q, 0], expect, rtol=0, atol=1e-15)
+        assert abs(lse[q, 0] - math.log(len(A))) < 1e-14
+        assert counts[q] == len(A)
+
+
+def _fenwick_cutoffs(scores, n, S, W, D, K):
+    """The tree method of §C.2, written independently of the oracle: visit the
+    eligible tokens best first (score, then older first; NaN lowest); before
+    inserting token j, the K-th smallest position among the tokens already in
+    a Fenwick tree over positions (those ranked above j) is the step at which
+    j leaves the long-range set; fewer than K above it means it never leaves."""
+    c = [-1] * n
+    elig = list(range(S, n - W - D))
+    tree = [0] * (n + 1)
+
+    def add(i):
+        i += 1
+        while i <= n:
+            tree[i] += 1
+            i += i & -i
+
+    def kth(k):
+        pos, rem, step = 0, k, 1 << n.bit_length()
+        while step:
+            if pos + step <= n and tree[pos + step] < rem:
+                pos += step
+                rem -= tree[pos]
+            step >>= 1
+        return pos
+
+    def key(j):
+        x = float(scores[j])
+        return (-math.inf if math.isnan(x) else x, -j)
+
+    for r, j in enumerate(sorted(elig, key=key, reverse=True)):
+        if r < K:
+            c[j] = 2 ** 31 - 1
+        else:
+            c[j] = max(j, kth(K)) if K > 0 else j
+        add(j)
+    return c
+
+
+def pin_running_cutoffs_match_fenwick():
+    for i, (S, W, D, K, n, ties) in enumerate([(2, 3, 0, 4, 40, 3), (0, 1, 0, 1, 30, 2), (1, 2, 2, 5, 45, 0),
+                                               (3, 4, 1, 0, 20, 2), (1, 1, 0, 50, 30, 0), (0, 2, 0, 3, 25, 1),
+                                               (4, 2, 3, 6, 12, 0)]):
+        _, _, _, s = _rand_unit(100 + i, n, 0, 1, 2, tie_levels=ties)
+        assert orc.running_cutoffs(s, n, S, W, D, K) == _fenwick_cutoffs(s, n, S, W, D, K), (S, W, D, K)
+
+
+def pin_running_cutoffs_are_intervals():
+    """Token j is in the running top-k at newest-eligible position m exactly when
+    j <= m < c_j (an evicted token never returns, §C.2)."""
+    S, W, D, K, n = 2, 3, 1, 4, 36
+    _, _, _, s = _rand_unit(21, n, 0, 1, 2, tie_levels=2)
+    c = orc.running_cutoffs(s, n, S, W, D, K)
+    for m in range(S, n - W - D):
+        kept = set(orc.running_topk(s, m + W + D, S, W, D, K))
+        for j in range(S, n - W - D):
+            assert (j in kept) == (j <= m < c[j]), (m, j, c[j])
+
+
+def pin_prefill_attention_dense_when_budget_covers_context():
+    """K >= n: every row is causal dense attention (torch SDPA, float64) and its
+    log-normaliser is torch.logsumexp of the causal logits."""
+    S, W, D, K, n, G, d = 2, 3, 1, 64, 40, 2, 8
+    rng = np.random.default_rng(3)
+    k, v = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    q = rng.standard_normal((n, G, d))
+    s = orc.ranking_score(rng.standard_normal(n))
+    out, lse, _ = orc.prefill_attention(q, k, v, s, S, W, D, K)
+    qt = torch.tensor(q).permute(1, 0, 2)  # [G][n][d]
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, torch.tensor(k)[None], torch.tensor(v)[None],
+                                                           is_causal=True)
+    np.testing.assert_allclose(out, ref.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+    logits = (qt @ torch.tensor(k).T) / math.sqrt(d)
+    logits = logits.masked_fill(torch.triu(torch.ones(n, n, dtype=torch.bool), 1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(logits, -1).T.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def pin_prefill_attention_matches_slot_simulator():
+    """Row q equals attention over the slot simulator's whole cache content after
+    token q arrives one token at a time (sinks, window, staging, long-range slots),
+    and it attends to min(q + 1, S + W + D + K) tokens."""
+    for (S, W, D, K, n) in [(2, 4, 0, 5, 40), (1, 3, 2, 4, 36), (0, 2, 0, 3, 30)]:
+        G, d = 2, 8
+        k, v, qq, s = _rand_unit(S * 10 + W + D, n, n, G, d, tie_levels=3)
+        out, lse, counts = orc.prefill_attention(qq, k, v, s, S, W, D, K)
+        st = orc.SlotState(S, W, D, K)
+        for q in range(n):
+            st.decode(s)
+            A = sorted(p for p in st.slot_pos if p >= 0)
+            assert counts[q] == len(A) == min(q + 1, S + W + D + K), (q, counts[q], len(A))
+            o, w = orc.attention(qq[q], k[A], v[A])
+            np.testing.assert_allclose(out[q], o, rtol=0, atol=1e-13)
+
 ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1,
             pin_prefill_chunk_placement, pin_dense_when_budget_covers_context,
             pin_budget_invariant_and_structure, pin_softmax_rows_sum_to_one,
             pin_delay_equivalence, pin_prefill_is_running_topk, pin_attention_closed_forms,
             pin_decay_hand_example, pin_decay_static_priority_is_effective_score_topk,
-            pin_float32_single_rounding, pin_linear_scorer]
+            pin_float32_single_rounding, pin_linear_scorer,
+            pin_prefill_mask_hand_example, pin_running_cutoffs_match_fenwick,
+            pin_running_cutoffs_are_intervals, pin_prefill_attention_dense_when_budget_covers_context,
+            pin_prefill_attention_matches_slot_simulator]

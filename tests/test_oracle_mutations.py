@@ -106,6 +106,33 @@ def _linear_drops_bias(x, w, b):
     return np.asarray(x, np.float64) @ np.asarray(w, np.float64)
 
 
+def _cutoff_last_kept(scores, n, S, W, D, K):
+    c = _ORIG_CUTOFFS(scores, n, S, W, D, K)
+    return [x - 1 if 0 <= x < 2 ** 31 - 1 else x for x in c]
+
+
+def _prefill_stale_topk(q_all, k_all, v_all, scores, S, W, D, K):
+    n = len(k_all)
+    G, d = q_all.shape[1], q_all.shape[2]
+    out, lse, counts = np.zeros((n, G, d)), np.zeros((n, G)), []
+    for q in range(n):
+        T = orc.running_topk(scores, max(q - 1, 0), S, W, D, K)
+        A = orc.attended_positions(q, S, W, D, T)
+        out[q] = orc.attention(q_all[q], k_all[A], v_all[A])[0]
+        lse[q] = orc.attention_lse(q_all[q], k_all[A])
+        counts.append(len(A))
+    return out, lse, counts
+
+
+def _lse_unscaled(q, keys):
+    logits = np.asarray(q, np.float64) @ np.asarray(keys, np.float64).T
+    mx = logits.max(axis=-1)
+    return mx + np.log(np.exp(logits - mx[:, None]).sum(axis=-1))
+
+
+_ORIG_CUTOFFS = orc.running_cutoffs
+
+
 MUTATIONS = {
     "tie_goes_to_newer": ("rank_key", _ties_to_newer),
     "eligible_off_by_one": ("eligible_positions", _elig_off_by_one),
@@ -124,6 +151,9 @@ MUTATIONS = {
     "decay_eligibility_off_by_one": ("decayed_priority", _decay_eligibility_off_by_one),
     "priority_double_rounding": ("round_to_float32", _round_via_float64),
     "linear_drops_bias": ("linear_score", _linear_drops_bias),
+    "cutoff_records_last_kept_step": ("running_cutoffs", _cutoff_last_kept),
+    "prefill_attends_before_update": ("prefill_attention", _prefill_stale_topk),
+    "prefill_lse_unscaled": ("attention_lse", _lse_unscaled),
 }
 
 
