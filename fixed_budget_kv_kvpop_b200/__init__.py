@@ -48,6 +48,7 @@ EXPORTED_SYMBOLS = (
     "kvpop_decode_attend", "kvpop_inspect",
     "kvpop_get_layout", "kvpop_get_error", "kvpop_clear_error", "kvpop_debug_poison_error",
     "kvpop_destroy", "kvpop_status_string", "kvpop_decode_step_noalloc",
+    "kvpop_prefill_attention_workspace_bytes", "kvpop_prefill_attention",
 )
 
 
@@ -96,6 +97,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvpop_destroy": ([P], ctypes.c_int),
         "kvpop_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "kvpop_decode_step_noalloc": ([P, I32, P, P, P, P, P, P], ctypes.c_int),
+        "kvpop_prefill_attention_workspace_bytes": ([P, I32, ctypes.POINTER(SZ)], ctypes.c_int),
+        "kvpop_prefill_attention": ([P, I32, P, P, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -176,10 +179,10 @@ class KVPopCache:
         _check(lib.kvpop_create(ctypes.byref(cfg), ctypes.c_void_p(base + self._off), self.nbytes,
                                 ctypes.byref(self.handle)), "kvpop_create")
 
-    def __del__(self):
+    def __del__(self, _lib=lib):
         h = getattr(self, "handle", None)
         if h:
-            lib.kvpop_destroy(h)
+            _lib.kvpop_destroy(h)
             self.handle = None
 
     def prefill(self, layer: int, k, v, ext_scores=None, stream=None):
@@ -199,6 +202,25 @@ class KVPopCache:
         capture); calls that overlap on the GPU share the buffer and race."""
         _check(lib.kvpop_decode_step_noalloc(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                              _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step_noalloc")
+
+    def prefill_attention_workspace_bytes(self, n_tokens: int) -> int:
+        out = ctypes.c_size_t()
+        _check(lib.kvpop_prefill_attention_workspace_bytes(self.handle, n_tokens, ctypes.byref(out)),
+               "kvpop_prefill_attention_workspace_bytes")
+        return out.value
+
+    def prefill_attention(self, layer: int, q, k, v, out, lse=None, workspace=None, ext_scores=None, stream=None):
+        """Attention outputs of every prompt position under the running top-k
+        mask.  q, out: [b][Hq][n][d]; k, v: [b][Hkv][n][d]; lse: optional fp32
+        [b][Hq][n]; workspace: a uint8 device tensor of at least
+        prefill_attention_workspace_bytes(n) bytes, 16-byte aligned (its first
+        units * n int32 are the running cutoffs afterwards).  Does not touch
+        the cache."""
+        n = int(k.shape[2])
+        _check(lib.kvpop_prefill_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
+                                           _ptr(out), _ptr(lse), _ptr(workspace),
+                                           int(workspace.numel() * workspace.element_size()) if workspace is not None
+                                           else 0, _stream_ptr(stream)), "kvpop_prefill_attention")
 
     def decode_append(self, layer: int, k_new, v_new, ext_score=None, stream=None):
         _check(lib.kvpop_decode_append(self.handle, layer, _ptr(k_new), _ptr(v_new), _ptr(ext_score),

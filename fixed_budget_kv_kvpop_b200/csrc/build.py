@@ -10,8 +10,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
-SOURCES = ["kvpop_api.cu", "kvpop_decode.cu", "kvpop_prefill.cu"]
-HEADERS = ["kvpop_internal.cuh", os.path.join(ROOT, "include", "kvpop.h")]
+SOURCES = ["kvpop_api.cu", "kvpop_decode.cu", "kvpop_prefill.cu", "kvpop_prefill_attn.cu"]
+HEADERS = ["kvpop_internal.cuh", "kvpop_prefill_attn.cuh", os.path.join(ROOT, "include", "kvpop.h")]
 OUT = os.path.join(PKG, "libkvpop.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

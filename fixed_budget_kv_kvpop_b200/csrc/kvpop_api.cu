@@ -8,6 +8,7 @@
 
 #include "../../include/kvpop.h"
 #include "kvpop_internal.cuh"
+#include "kvpop_prefill_attn.cuh"
 
 using namespace kvpop;
 
@@ -351,6 +352,36 @@ int kvpop_debug_poison_error(kvpop_handle* h, int32_t bits, void* stream) {
   poison_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<int32_t*>(h->mem + h->lay.err_off),
                                                                 bits);
   return cudaGetLastError() == cudaSuccess ? KVPOP_OK : KVPOP_ERR_CUDA;
+}
+
+int kvpop_prefill_attention_workspace_bytes(const kvpop_handle* h, int32_t n_tokens, size_t* bytes) {
+  if (!h || !bytes || n_tokens < 0) return KVPOP_ERR_INVALID_ARG;
+  if (n_tokens > h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
+  PrefillAttnPlan p;
+  if (plan_prefill_attention(layer_args(h, 0), n_tokens, &p) != 0) return KVPOP_ERR_BAD_SHAPE;
+  *bytes = p.total;
+  return KVPOP_OK;
+}
+
+int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const void* k, const void* v,
+                            int32_t n_tokens, const float* ext_scores, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers || n_tokens < 0) return KVPOP_ERR_INVALID_ARG;
+  if (n_tokens > h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
+  if (n_tokens == 0) return KVPOP_OK;
+  if (!q || !k || !v || !out || !workspace) return KVPOP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return KVPOP_ERR_INVALID_ARG;
+  const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
+  if (ext && !ext_scores) return KVPOP_ERR_INVALID_ARG;
+  const LayerArgs a = layer_args(h, layer);
+  PrefillAttnPlan p;
+  if (plan_prefill_attention(a, n_tokens, &p) != 0 || a.units > 65535) return KVPOP_ERR_BAD_SHAPE;
+  if (workspace_bytes < p.total) return KVPOP_ERR_INVALID_ARG;
+  const int r = launch_prefill_attention(a, h->cfg.dtype, p, q, k, v, ext ? ext_scores : nullptr, out, lse,
+                                         static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+  if (r == -2) return KVPOP_ERR_BAD_SHAPE;
+  return r == 0 ? KVPOP_OK : KVPOP_ERR_CUDA;
 }
 
 int kvpop_destroy(kvpop_handle* h) {

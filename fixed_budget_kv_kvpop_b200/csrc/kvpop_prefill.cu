@@ -22,6 +22,7 @@
 //   P3 move:   window tokens that enter the staging ring move there.
 //   P4 write:  chunk tokens go to their sink / window / staging slots.
 #include "kvpop_internal.cuh"
+#include "kvpop_prefill_attn.cuh"
 
 namespace kvpop {
 
@@ -508,7 +509,7 @@ __global__ void write_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k,
 }
 
 template <typename T, int D2, int HID>
-int launch_score64(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T* v, int n, const PrefillScratch& ps,
+int launch_score64(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T* v, int n, float* out, int cap,
                    int n_new, cudaStream_t st) {
   using SG = Score64Geom<D2, HID>;
   static bool attr_set = false;
@@ -520,7 +521,46 @@ int launch_score64(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T*
   }
   const int tiles = (n_new + SG::TT - 1) / SG::TT;
   dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
-  score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, ps.new_score, ps.cap);
+  score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap);
+  return 0;
+}
+
+// P1 for the tokens [cg.e0, cg.e1): ranking priority of each into out[u * cap + (t - cg.e0)].
+template <typename T>
+int launch_scores_t(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T* v, int n, const float* ext,
+                    float* out, int cap, cudaStream_t st) {
+  const int n_new = cg.e1 - cg.e0;
+  const bool use64 = !(a.flags & FLAG_EXTERNAL_SCORES) && (a.hidden == 32 || a.hidden == 64) &&
+                     (a.d == 64 || a.d == 128);
+  if (n_new > 0 && use64) {
+    int r = 0;
+    if (a.d == 128 && a.hidden == 64) r = launch_score64<T, 256, 64>(a, cg, k, v, n, out, cap, n_new, st);
+    else if (a.d == 128) r = launch_score64<T, 256, 32>(a, cg, k, v, n, out, cap, n_new, st);
+    else if (a.hidden == 64) r = launch_score64<T, 128, 64>(a, cg, k, v, n, out, cap, n_new, st);
+    else r = launch_score64<T, 128, 32>(a, cg, k, v, n, out, cap, n_new, st);
+    if (r != 0) return r;
+  } else if (n_new > 0 && a.hidden == 0 && !(a.flags & FLAG_EXTERNAL_SCORES)) {
+    constexpr int per_block = (kLinearThreads / 32) * kLinearTokensPerWarp;
+    dim3 grid((n_new + per_block - 1) / per_block, a.units);
+    if (a.d == 128)
+      linear_score_kernel<T, 256><<<grid, kLinearThreads, 0, st>>>(a, cg, k, v, n, out, cap);
+    else
+      linear_score_kernel<T, 128><<<grid, kLinearThreads, 0, st>>>(a, cg, k, v, n, out, cap);
+  } else if (n_new > 0) {
+    const int HQ = a.hidden / 4;
+    const int TT = 4 * (kScoreThreads / HQ);
+    const size_t smem = (a.flags & FLAG_EXTERNAL_SCORES) ? 0
+                        : (static_cast<size_t>(2 * a.d) * a.hidden + static_cast<size_t>(TT) * 2 * a.d) * sizeof(float);
+    static size_t smem_set = 0;
+    if (smem > 48 * 1024 && smem > smem_set) {
+      if (cudaFuncSetAttribute(score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return -1;
+      smem_set = smem;
+    }
+    dim3 grid((n_new + TT - 1) / TT, a.units);
+    score_kernel<T><<<grid, kScoreThreads, smem, st>>>(a, cg, k, v, n, ext, out, cap);
+  }
   return 0;
 }
 
@@ -535,37 +575,8 @@ int launch_prefill_t(const LayerArgs& a, const PrefillScratch& ps, const T* k, c
   cg.c0 = c0;
   const int n_new = cg.e1 - cg.e0;
   if (n_new > ps.cap) return -2;
-  const bool use64 = !(a.flags & FLAG_EXTERNAL_SCORES) && (a.hidden == 32 || a.hidden == 64) &&
-                     (a.d == 64 || a.d == 128);
-  if (n_new > 0 && use64) {
-    int r = 0;
-    if (a.d == 128 && a.hidden == 64) r = launch_score64<T, 256, 64>(a, cg, k, v, n, ps, n_new, st);
-    else if (a.d == 128) r = launch_score64<T, 256, 32>(a, cg, k, v, n, ps, n_new, st);
-    else if (a.hidden == 64) r = launch_score64<T, 128, 64>(a, cg, k, v, n, ps, n_new, st);
-    else r = launch_score64<T, 128, 32>(a, cg, k, v, n, ps, n_new, st);
-    if (r != 0) return r;
-  } else if (n_new > 0 && a.hidden == 0 && !(a.flags & FLAG_EXTERNAL_SCORES)) {
-    constexpr int per_block = (kLinearThreads / 32) * kLinearTokensPerWarp;
-    dim3 grid((n_new + per_block - 1) / per_block, a.units);
-    if (a.d == 128)
-      linear_score_kernel<T, 256><<<grid, kLinearThreads, 0, st>>>(a, cg, k, v, n, ps.new_score, ps.cap);
-    else
-      linear_score_kernel<T, 128><<<grid, kLinearThreads, 0, st>>>(a, cg, k, v, n, ps.new_score, ps.cap);
-  } else if (n_new > 0) {
-    const int HQ = a.hidden / 4;
-    const int TT = 4 * (kScoreThreads / HQ);
-    const size_t smem = (a.flags & FLAG_EXTERNAL_SCORES) ? 0
-                        : (static_cast<size_t>(2 * a.d) * a.hidden + static_cast<size_t>(TT) * 2 * a.d) * sizeof(float);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-      if (cudaFuncSetAttribute(score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return -1;
-      smem_set = smem;
-    }
-    dim3 grid((n_new + TT - 1) / TT, a.units);
-    score_kernel<T><<<grid, kScoreThreads, smem, st>>>(a, cg, k, v, n, ext, ps.new_score, ps.cap);
-  }
+  const int r = launch_scores_t<T>(a, cg, k, v, n, ext, ps.new_score, ps.cap, st);
+  if (r != 0) return r;
   select_kernel<T><<<a.units, kSelThreads, 0, st>>>(a, cg, k, v, n, ps.new_score, ps.cap, ps.tgt);
   if (a.D > 0) move_kernel<T><<<a.units, 256, 0, st>>>(a, cg);
   if (n > 0) {
@@ -576,6 +587,25 @@ int launch_prefill_t(const LayerArgs& a, const PrefillScratch& ps, const T* k, c
 }
 
 }  // namespace
+
+int launch_prompt_scores(const LayerArgs& a, int dtype, const void* k, const void* v, int n, const float* ext,
+                         float* out, int cap, cudaStream_t st) {
+  ChunkGeom cg;
+  cg.n0 = 0;
+  cg.n1 = n;
+  cg.e0 = a.S;
+  cg.e1 = max(a.S, n - a.W - a.D);
+  cg.c0 = 0;
+  if (cg.e1 - cg.e0 > cap) return -2;
+  int r;
+  if (dtype == 0)
+    r = launch_scores_t<float>(a, cg, static_cast<const float*>(k), static_cast<const float*>(v), n, ext, out, cap, st);
+  else
+    r = launch_scores_t<__nv_bfloat16>(a, cg, static_cast<const __nv_bfloat16*>(k),
+                                       static_cast<const __nv_bfloat16*>(v), n, ext, out, cap, st);
+  if (r != 0) return r;
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
 
 int launch_prefill(const LayerArgs& a, int dtype, const PrefillScratch& ps, const void* k, const void* v,
                    int n_tokens, int n_seen_before, int n_topk_before, const float* ext_scores, cudaStream_t st) {

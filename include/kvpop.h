@@ -208,6 +208,41 @@ int kvpop_decode_append(kvpop_handle* h, int32_t layer, const void* k_new, const
                         const float* ext_score, void* stream);
 int kvpop_decode_attend(kvpop_handle* h, int32_t layer, const void* q, void* out, void* stream);
 
+/* Parallel sparse prefill attention (page §C "Efficient Running Top-k Sparse
+ * Attention": §C.1 Mask Definition, §C.2 Fenwick-Tree Cutoff Computation).
+ * Computes, for every position q of a prompt of n_tokens tokens (positions
+ * 0 .. n_tokens - 1) and every query head, the attention output under the
+ * fixed-budget mask: q attends to exactly the set a decode step at q would
+ * attend to -- the sinks, the recent W + D positions (its own included) and
+ * the running top-k of the tokens eligible at q (scored as kvpop_prefill
+ * scores them, decay included) -- with softmax scale 1/sqrt(d) and fp32
+ * accumulation.  Does not read or change the cache or its position counter;
+ * any layer's scorer weights may be used at any time.
+ *
+ * Running cutoffs: with m = q - W - D, token j (S <= j <= n_tokens-1-W-D)
+ * is in the long-range set exactly for m in [j, c_j); c_j = INT32_MAX when j
+ * is still kept at the last position, c_j = j when it is never admitted.
+ * Tokens that never become eligible in the prompt get -1.
+ *
+ * q: device [b][Hq][n_tokens][d]; k, v: device [b][Hkv][n_tokens][d];
+ * out: device [b][Hq][n_tokens][d] (config.dtype); lse: device fp32
+ * [b][Hq][n_tokens] receiving each row's natural-log softmax normaliser
+ * log sum_j exp(q.k_j / sqrt(d)), or NULL; ext_scores: device fp32
+ * [b][Hkv][n_tokens] (required with KVPOP_FLAG_EXTERNAL_SCORES, ignored
+ * otherwise).  q, k, v, out and workspace must be 16-byte aligned.
+ * workspace: caller-owned device scratch of at least
+ * kvpop_prefill_attention_workspace_bytes(n_tokens) bytes; after the call its
+ * first units * n_tokens int32 hold the cutoffs c_j ([units][n_tokens]).
+ * Errors: KVPOP_ERR_INVALID_ARG (null or misaligned pointer, workspace too
+ * small, bad layer), KVPOP_ERR_BAD_SHAPE (G not dividing 64, head_dim other
+ * than 64/128, S + K + W + D + 64/G above 16384, more than 65535 units),
+ * KVPOP_ERR_CONTEXT_OVERFLOW (n_tokens > max_context); nothing is enqueued
+ * then.  n_tokens = 0 is a no-op. */
+int kvpop_prefill_attention_workspace_bytes(const kvpop_handle* h, int32_t n_tokens, size_t* bytes);
+int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const void* k, const void* v,
+                            int32_t n_tokens, const float* ext_scores, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /* Copies layer `layer`'s slot -> position map (int32 [units][slots]), slot
  * scores (fp32 [units][slots]) and per-unit state (int32 [units][4]) to HOST
  * buffers; any of them may be NULL.  Synchronises `stream`.  For tests and

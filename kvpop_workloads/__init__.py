@@ -153,6 +153,13 @@ def prompt_kv(w: Workload, layer: int, n_tokens: Optional[int] = None, master: i
     return k.to(dt), v.to(dt)
 
 
+def prompt_queries(w: Workload, layer: int, n_tokens: Optional[int] = None, master: int = 0, device="cpu"):
+    """Queries of every prompt position for one layer: [batch][q_heads][n][d] in w's dtype."""
+    n = w.prefill if n_tokens is None else n_tokens
+    q = _normal((w.batch, w.n_q_heads, n, w.head_dim), _gen(device, master, w.name, layer, "pq", n), device)
+    return q.to(w.torch_dtype())
+
+
 def decode_inputs(w: Workload, layer: int, step: int, master: int = 0, device="cpu"):
     """One decode step's inputs for one layer: q [b][Hq][d], k_new/v_new [b][Hkv][d]."""
     q = _normal((w.batch, w.n_q_heads, w.head_dim), _gen(device, master, w.name, layer, "q", step), device)

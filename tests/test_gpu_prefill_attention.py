@@ -1,0 +1,213 @@
+"""Parity of the parallel sparse prefill attention (CUDA, through the C ABI)
+with the CPU oracle: running cutoffs bit-exact, outputs and log-normalisers
+within the dtype's tolerance, on seeded inputs of several tiles with ragged
+tails, and the edge cases of the mask (nothing eligible, K = 0, K covering the
+prompt, one token)."""
+import numpy as np
+import pytest
+import torch
+
+import kvpop_workloads as wl
+from oracle import kvpop_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+gh = pytest.importorskip("gpu_harness")
+
+LSE_ATOL = {"f32": 1e-4, "bf16": 1e-3}   # fp32 sums of at most a few thousand terms
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+class PaRun:
+    pass
+
+
+def run_prefill_attention(w, n, *, external=False, tie_levels=0, log_decay=None, layer=0, master=0,
+                          gen_device="cpu", with_lse=True):
+    """One prefill-attention call for `layer` of a one-layer-per-call cache."""
+    import fixed_budget_kv_kvpop_b200 as kp
+    n_layers = layer + 1
+    weights = None
+    if not external:
+        wshape = w.replace(n_layers=n_layers, scorer_hidden=max(w.scorer_hidden, 1))
+        weights = tuple(t.cuda() for t in wl.scorer_weights(wshape, master=master))
+    dec = None if log_decay is None else torch.tensor(np.asarray(log_decay, np.float32), device="cuda")
+    cache = gh.build_cache(w, n_layers, external, weights, max_chunk=1, debug=True, log_decay=dec)
+    k, v = wl.prompt_kv(w, layer, n_tokens=n, master=master, device=gen_device)
+    q = wl.prompt_queries(w, layer, n, master=master, device=gen_device)
+    k, v, q = k.cuda(), v.cuda(), q.cuda()
+    ext = None
+    if external:
+        ext = wl.external_scores(w, layer, n, master=master, device=gen_device, tie_levels=tie_levels).cuda()
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full((w.batch, w.n_q_heads, n), float("nan"), device="cuda") if with_lse else None
+    ws = torch.empty(cache.prefill_attention_workspace_bytes(n), dtype=torch.uint8, device="cuda")
+    cache.prefill_attention(layer, q, k, v, out, lse, ws, ext)
+    torch.cuda.synchronize()
+    st, bits = cache.get_error()
+    assert st == 0, f"device error status {st} bits {bits}"
+    units = w.batch * w.n_kv_heads
+    r = PaRun()
+    r.w, r.n, r.layer, r.cache, r.weights = w, n, layer, cache, weights
+    r.q, r.k, r.v, r.ext, r.out, r.lse = q, k, v, ext, out, lse
+    r.cut = ws[:units * n * 4].view(torch.int32).reshape(units, n).cpu().numpy() if n > 0 else None
+    r.log_decay = None if log_decay is None else np.asarray(log_decay, np.float32)
+    return r
+
+
+def unit_view(r, unit):
+    w = r.w
+    b, h = divmod(unit, w.n_kv_heads)
+    G = w.group
+    k = r.k[b, h].double().cpu().numpy()
+    v = r.v[b, h].double().cpu().numpy()
+    q = r.q[b, h * G:(h + 1) * G].double().cpu().numpy().transpose(1, 0, 2)   # [n][G][d]
+    out = r.out[b, h * G:(h + 1) * G].double().cpu().numpy().transpose(1, 0, 2)
+    lse = None if r.lse is None else r.lse[b, h * G:(h + 1) * G].double().cpu().numpy().T
+    if r.ext is not None:
+        s = orc.ranking_score(r.ext[b, h].double().cpu().numpy())
+    else:
+        w1, b1, w2, b2 = (t.double().cpu().numpy() for t in r.weights)
+        if w.scorer_hidden == 0:
+            s = orc.unit_scores_linear(k, v, w1[r.layer, h, 0], b2[r.layer, h])
+        else:
+            s = orc.unit_scores_mlp(k, v, w1[r.layer, h], b1[r.layer, h], w2[r.layer, h], b2[r.layer, h])
+    if r.log_decay is not None:
+        s = orc.decayed_priority(s, w.window, w.delay, float(r.log_decay[r.layer, h]))
+    return k, v, q, out, lse, s
+
+
+def check_all_rows(r, units=None, atol=None):
+    w = r.w
+    atol = atol if atol is not None else (gh.F32_ATOL if w.dtype == "f32" else gh.BF16_ATOL)
+    for unit in (range(w.batch * w.n_kv_heads) if units is None else units):
+        k, v, q, out, lse, s = unit_view(r, unit)
+        cut = orc.running_cutoffs(s, r.n, w.sinks, w.window, w.delay, w.topk)
+        assert list(r.cut[unit]) == cut, f"unit {unit}: cutoffs differ"
+        ref, ref_lse, _ = orc.prefill_attention(q, k, v, s, w.sinks, w.window, w.delay, w.topk)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=atol, err_msg=f"unit {unit}")
+        if lse is not None:
+            np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=LSE_ATOL[w.dtype], err_msg=f"unit {unit} lse")
+
+
+def _case(dtype, d, hq, hkv, *, S, W, D, K, hidden, batch=1):
+    return wl.Workload(f"pa_{dtype}_d{d}_g{hq // hkv}_s{S}w{W}d{D}k{K}_h{hidden}", batch=batch, n_layers=1,
+                       n_q_heads=hq, n_kv_heads=hkv, head_dim=d, dtype=dtype, sinks=S, window=W, topk=K,
+                       delay=D, prefill=0, decode=0, scorer_hidden=hidden, heavy_hitter_frac=0.02)
+
+
+def test_tiny_shape_mlp_scorer():
+    """The tiny workload's shape (fp32, d 64, G 2, S 4, W 16, K 44, MLP 32):
+    300 prompt positions = 9 full query tiles of 32 plus a ragged one."""
+    _need_gpu()
+    r = run_prefill_attention(wl.TINY.replace(prefill=0), 300)
+    check_all_rows(r)
+
+
+@pytest.mark.parametrize("dtype,d,hq,hkv,S,W,D,K,hidden,n,ties", [
+    ("bf16", 128, 8, 2, 4, 16, 0, 40, 64, 500, 2),
+    ("bf16", 128, 8, 2, 2, 12, 5, 30, 64, 333, 0),
+    ("bf16", 64, 16, 2, 1, 8, 0, 20, 32, 257, 3),
+    ("f32", 64, 2, 2, 0, 4, 3, 50, 32, 401, 1),
+    ("bf16", 64, 8, 8, 4, 32, 0, 64, 64, 190, 0),
+])
+def test_external_scores_with_ties(dtype, d, hq, hkv, S, W, D, K, hidden, n, ties):
+    """Caller scores (quantised so that equal scores are common): cutoffs
+    bit-exact under the (score, -position) order, outputs and normalisers."""
+    _need_gpu()
+    w = _case(dtype, d, hq, hkv, S=S, W=W, D=D, K=K, hidden=hidden)
+    r = run_prefill_attention(w, n, external=True, tie_levels=ties)
+    check_all_rows(r)
+
+
+@pytest.mark.parametrize("dtype,d,hq,hkv,S,W,D,K,hidden,n", [
+    ("bf16", 128, 8, 2, 4, 16, 0, 40, 64, 400),
+    ("bf16", 128, 4, 1, 3, 10, 4, 25, 64, 300),
+    ("f32", 64, 4, 2, 2, 8, 0, 30, 0, 280),
+    ("bf16", 64, 8, 2, 4, 16, 2, 20, 128, 220),
+])
+def test_gpu_scorer(dtype, d, hq, hkv, S, W, D, K, hidden, n):
+    """The scores come from the library's own scorer (MLP of hidden 64 / 128,
+    or the linear scorer), as kvpop_prefill computes them."""
+    _need_gpu()
+    w = _case(dtype, d, hq, hkv, S=S, W=W, D=D, K=K, hidden=hidden, batch=2)
+    r = run_prefill_attention(w, n)
+    check_all_rows(r)
+
+
+def test_temporal_decay():
+    """Ranking by the decayed static priority (ln gamma per KV head)."""
+    _need_gpu()
+    w = _case("bf16", 128, 8, 2, S=4, W=16, D=0, K=40, hidden=64)
+    r = run_prefill_attention(w, 350, log_decay=np.array([[-0.01, -0.2]], np.float32))
+    check_all_rows(r)
+
+
+@pytest.mark.parametrize("S,W,D,K,n", [
+    (4, 16, 0, 40, 1),          # one token
+    (4, 16, 0, 40, 19),         # nothing ever eligible (n <= S + W + D)
+    (4, 16, 2, 40, 23),         # exactly one eligible token at the last position
+    (4, 16, 0, 0, 150),         # K = 0: sinks + window only
+    (4, 16, 0, 500, 150),       # K covers the prompt: dense causal attention
+    (0, 1, 0, 1, 90),           # no sinks, window 1, one long-range slot
+])
+def test_mask_edge_cases(S, W, D, K, n):
+    _need_gpu()
+    w = _case("bf16", 128, 8, 2, S=S, W=W, D=D, K=K, hidden=64)
+    r = run_prefill_attention(w, n, external=True, tie_levels=2)
+    check_all_rows(r)
+    if K >= n:
+        # every row is plain causal attention
+        qt = r.q.double().cpu()
+        kt = r.k.double().cpu().repeat_interleave(w.group, dim=1)
+        vt = r.v.double().cpu().repeat_interleave(w.group, dim=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+        np.testing.assert_allclose(r.out.double().cpu().numpy(), ref.numpy(), rtol=0, atol=gh.BF16_ATOL)
+
+
+def test_repeat_call_is_deterministic_and_leaves_cache_alone():
+    """Two calls give identical bits; the cache's position counter is untouched."""
+    _need_gpu()
+    w = _case("bf16", 128, 8, 2, S=4, W=16, D=0, K=40, hidden=64)
+    r = run_prefill_attention(w, 200)
+    first = r.out.clone()
+    ws = torch.empty(r.cache.prefill_attention_workspace_bytes(200), dtype=torch.uint8, device="cuda")
+    r.cache.prefill_attention(0, r.q, r.k, r.v, r.out, r.lse, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(first, r.out)
+    _, _, state = r.cache.inspect(0)
+    assert (state[:, 0] == 0).all()
+
+
+def test_full_size_target_shape_sampled_rows():
+    """The 87.5%-compression target shape at full size (64 rows x 8 KV heads,
+    prompt 8192, S 4 + W 128 + K 892, G 4, bf16, MLP scorer 64), in the launch
+    configuration bench.py times.  Sampled units and positions: the mask each
+    position gets from the GPU's cutoffs equals the oracle's attended set, and
+    the output row and normaliser match attention over that set."""
+    _need_gpu()
+    w = wl.QWEN3_4B_CR88.replace(name="pa_full_size", n_layers=1, decode=0)
+    n = w.prefill
+    r = run_prefill_attention(w, n, gen_device="cuda")
+    units = w.batch * w.n_kv_heads
+    S, W, D, K = w.sinks, w.window, w.delay, w.topk
+    rng = np.random.default_rng(7)
+    for unit in (0, units // 2 + 3, units - 1):
+        k, v, q, out, lse, s = unit_view(r, unit)
+        c = r.cut[unit]
+        rows = sorted(set([0, S, S + W, S + W + K + 3, n - 1] + list(rng.integers(0, n, 6))))
+        for qp in rows:
+            T = orc.running_topk(s, qp, S, W, D, K)
+            A = orc.attended_positions(qp, S, W, D, T)
+            m = qp - W - D
+            gpu_set = sorted(set(range(min(S, qp + 1))) | set(range(max(S, m + 1), qp + 1)) |
+                             {j for j in range(S, m + 1) if c[j] > m})
+            assert gpu_set == A, (unit, qp)
+            o, _ = orc.attention(q[qp], k[A], v[A])
+            np.testing.assert_allclose(out[qp], o, rtol=0, atol=gh.BF16_ATOL, err_msg=f"unit {unit} q {qp}")
+            np.testing.assert_allclose(lse[qp], orc.attention_lse(q[qp], k[A]), rtol=0, atol=LSE_ATOL["bf16"])
+    assert torch.isfinite(r.out).all()
