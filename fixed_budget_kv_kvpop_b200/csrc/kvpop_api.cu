@@ -358,7 +358,7 @@ int kvpop_prefill_attention_workspace_bytes(const kvpop_handle* h, int32_t n_tok
   if (!h || !bytes || n_tokens < 0) return KVPOP_ERR_INVALID_ARG;
   if (n_tokens > h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
   PrefillAttnPlan p;
-  if (plan_prefill_attention(layer_args(h, 0), n_tokens, &p) != 0) return KVPOP_ERR_BAD_SHAPE;
+  if (plan_prefill_attention(layer_args(h, 0), h->cfg.dtype, n_tokens, &p) != 0) return KVPOP_ERR_BAD_SHAPE;
   *bytes = p.total;
   return KVPOP_OK;
 }
@@ -376,7 +376,7 @@ int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const
   if (ext && !ext_scores) return KVPOP_ERR_INVALID_ARG;
   const LayerArgs a = layer_args(h, layer);
   PrefillAttnPlan p;
-  if (plan_prefill_attention(a, n_tokens, &p) != 0 || a.units > 65535) return KVPOP_ERR_BAD_SHAPE;
+  if (plan_prefill_attention(a, h->cfg.dtype, n_tokens, &p) != 0 || a.units > 65535) return KVPOP_ERR_BAD_SHAPE;
   if (workspace_bytes < p.total) return KVPOP_ERR_INVALID_ARG;
   const int r = launch_prefill_attention(a, h->cfg.dtype, p, q, k, v, ext ? ext_scores : nullptr, out, lse,
                                          static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));

@@ -24,7 +24,10 @@
 // long-range tokens still kept at its first query (c_j > m0; at most K), and
 // the recent positions of its queries.  It then streams them in tiles of
 // kPaKeys through shared memory with an online softmax in fp32 (FMA pipes),
-// masking each (query, key) pair by the rule above.
+// masking each (query, key) pair by the rule above.  bf16 inputs take the
+// tensor-core kernel instead (sparse_attn_mma_kernel: 128 rows per CTA,
+// m16n8k16 bf16 MMAs with fp32 accumulation, keys gathered by cp.async);
+// fp32 inputs keep the FMA kernel so that no product is rounded.
 #include "kvpop_prefill_attn.cuh"
 
 namespace kvpop {
@@ -136,25 +139,44 @@ template <> struct PaIo<float> {
   }
   static __device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 };
-template <> struct PaIo<__nv_bfloat16> {
-  static __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* o) {
-    const uint4 r = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+
+// Candidate keys of a tile of query positions [q0, q1) with m0 = q0 - W - D,
+// in ascending position: the sinks, the long-range tokens still kept at m0
+// (c_j > m0; at most K of them) and the recent block [max(S, m0 + 1), q1).
+// Every key a query of the tile may attend to is among them.  Block-wide
+// (all NT threads); returns the count (at most cap).
+template <int NT>
+__device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1, int cap) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ns = min(S, q1);
+  for (int i = tid; i < ns; i += NT) cand[i] = i;
+  int count = ns;
+  for (int base = S; base <= m0; base += NT) {
+    const int j = base + tid;
+    const bool f = j <= m0 && cu[j] > m0;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) wtot[warp] = __popc(bal);
+    __syncthreads();
+    int off = count, total = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      o[2 * i] = __uint_as_float(w[i] << 16);
-      o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    for (int w = 0; w < NT / 32; ++w) {
+      const int t = wtot[w];
+      off += (w < warp) ? t : 0;
+      total += t;
     }
+    const int slot = off + __popc(bal & ((1u << lane) - 1u));
+    if (f && slot < cap) cand[slot] = j;
+    count += total;
+    __syncthreads();
   }
-  static __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
-    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
-    const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
-    uint2 r;
-    r.x = *reinterpret_cast<const uint32_t*>(&a);
-    r.y = *reinterpret_cast<const uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(p) = r;
-  }
-};
+  const int r0 = max(S, m0 + 1);
+  const int nr = max(0, q1 - r0);
+  for (int i = tid; i < nr; i += NT)
+    if (count + i < cap) cand[count + i] = r0 + i;
+  count += nr;
+  __syncthreads();
+  return min(count, cap);   // count <= cap always: S + K + qt + W + D bounds it
+}
 
 template <int DH>
 struct PaSmem {
@@ -185,7 +207,7 @@ __global__ void __launch_bounds__(kPaThreads) sparse_attn_kernel(PaArgs p) {
   int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
   int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int rg = tid >> 3, kg = tid & 7;
   const int u = blockIdx.y;
   const int b = u / p.Hkv, hk = u % p.Hkv;
@@ -213,36 +235,7 @@ __global__ void __launch_bounds__(kPaThreads) sparse_attn_kernel(PaArgs p) {
     dst[1] = make_float4(x[4] * p.scale_log2, x[5] * p.scale_log2, x[6] * p.scale_log2, x[7] * p.scale_log2);
   }
 
-  // candidate keys: sinks, long-range tokens kept at the first query, recent block
-  const int m0 = q0 - WD;
-  const int ns = min(S, q1);
-  for (int i = tid; i < ns; i += kPaThreads) cand[i] = i;
-  int count = ns;
-  for (int base = S; base <= m0; base += kPaThreads) {
-    const int j = base + tid;
-    const bool f = j <= m0 && cu[j] > m0;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) wtot[warp] = __popc(bal);
-    __syncthreads();
-    int off = count, total = 0;
-#pragma unroll
-    for (int w = 0; w < kPaThreads / 32; ++w) {
-      const int t = wtot[w];
-      off += (w < warp) ? t : 0;
-      total += t;
-    }
-    const int slot = off + __popc(bal & ((1u << lane) - 1u));
-    if (f && slot < p.cand_cap) cand[slot] = j;
-    count += total;
-    __syncthreads();
-  }
-  const int r0 = max(S, m0 + 1);
-  const int nr = max(0, q1 - r0);
-  for (int i = tid; i < nr; i += kPaThreads)
-    if (count + i < p.cand_cap) cand[count + i] = r0 + i;
-  count += nr;
-  if (count > p.cand_cap) count = p.cand_cap;   // cannot happen: S + K + qt + W + D bounds it
-  __syncthreads();
+  const int count = gather_candidates<kPaThreads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
 
   float4 o[4][NC];
   float mrow[4], lrow[4];
@@ -389,24 +382,285 @@ __global__ void __launch_bounds__(kPaThreads) sparse_attn_kernel(PaArgs p) {
   }
 }
 
-template <typename T, int DH>
-int launch_attn(const PaArgs& pa, int units, int n, cudaStream_t st) {
+// ---------------- bf16 attention on the tensor cores (mma.sync) ----------------
+// One CTA of 8 warps per (unit, 128 / G query positions): each warp owns 16
+// query rows (Q fragments held in registers), the CTA streams its candidate
+// keys in tiles of 64 through a two-stage cp.async ring, S = Q K^T and
+// O += P V run as m16n8k16 bf16 MMAs with fp32 accumulators, and the mask and
+// online softmax run on the S fragments in registers.
+constexpr int kMmaThreads = 256;
+constexpr int kMmaKeys = 64;
+
+template <int DH>
+struct MmaSmem {
+  static constexpr int RS = DH + 8;   // bf16 row stride: 16-byte pad keeps ldmatrix rows on distinct banks
+  static constexpr size_t Q_OFF = 0;
+  static constexpr size_t KV_OFF = Q_OFF + 2ull * kPaMmaRows * RS;
+  static constexpr size_t TILE = 2ull * kMmaKeys * RS;       // one K or V tile
+  static constexpr size_t POS_OFF = KV_OFF + 4 * TILE;       // stages x {K, V}
+  static constexpr size_t CUT_OFF = POS_OFF + sizeof(int) * 2 * kMmaKeys;
+  static constexpr size_t WT_OFF = CUT_OFF + sizeof(int) * 2 * kMmaKeys;
+  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);
+  static size_t bytes(int cand_cap) { return CAND_OFF + sizeof(int) * static_cast<size_t>(cand_cap); }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+               "{%8, %9}, {%0, %1, %2, %3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs p) {
+  using SM = MmaSmem<DH>;
+  constexpr int KS = DH / 16;      // k-steps of Q K^T
+  constexpr int NT = kMmaKeys / 8; // key n-tiles of S
+  constexpr int DT = DH / 8;       // d n-tiles of O
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smem_raw + SM::Q_OFF);
+  int* kpos = reinterpret_cast<int*>(smem_raw + SM::POS_OFF);
+  int* kcut = reinterpret_cast<int*>(smem_raw + SM::CUT_OFF);
+  int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
+  int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g8 = lane >> 2, tig = lane & 3;
+  const int u = blockIdx.y;
+  const int b = u / p.Hkv, hk = u % p.Hkv;
+  const int n = p.n, S = p.S, WD = p.W + p.D, G = p.G;
+  const int q0 = blockIdx.x * p.qt;
+  const int q1 = min(n, q0 + p.qt);
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
+  const __nv_bfloat16* kgp = static_cast<const __nv_bfloat16*>(p.k) + static_cast<size_t>(u) * n * DH;
+  const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
+  const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
+
+  // query rows (row = position offset * G + head), zero beyond the prompt
+  for (int c = tid; c < kPaMmaRows * (DH / 8); c += kMmaThreads) {
+    const int row = c / (DH / 8), ch = c % (DH / 8);
+    const int qpos = q0 + row / G, g = row % G;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (qpos < q1) x = *reinterpret_cast<const uint4*>(qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos) * DH + ch * 8);
+    *reinterpret_cast<uint4*>(Qs + row * SM::RS + ch * 8) = x;
+  }
+  const int count = gather_candidates<kMmaThreads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
+  const int ntiles = (count + kMmaKeys - 1) / kMmaKeys;
+
+  auto issue = [&](int t) {
+    const int st = t & 1;
+    const int t0 = t * kMmaKeys;
+    if (tid < kMmaKeys) {
+      const int idx = t0 + tid;
+      const int j = idx < count ? cand[idx] : -1;
+      kpos[st * kMmaKeys + tid] = j;
+      kcut[st * kMmaKeys + tid] = j >= 0 ? cu[j] : 0;
+    }
+    const uint32_t kbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st) * SM::TILE);
+    const uint32_t vbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st + 1) * SM::TILE);
+    for (int c = tid; c < kMmaKeys * (DH / 8); c += kMmaThreads) {
+      const int key = c / (DH / 8), ch = c % (DH / 8);
+      const int idx = t0 + key;
+      const int j = idx < count ? cand[idx] : -1;
+      const size_t off = j >= 0 ? static_cast<size_t>(j) * DH + ch * 8 : 0;
+      const uint32_t so = static_cast<uint32_t>((key * SM::RS + ch * 8) * 2);
+      cp_async16(kbase + so, kgp + off, j >= 0 ? 16 : 0);
+      cp_async16(vbase + so, vgp + off, j >= 0 ? 16 : 0);
+    }
+    cp_async_commit();
+  };
+  if (ntiles > 0) issue(0);
+
+  // Q fragments of the warp's 16 rows
+  uint32_t qa[KS][4];
+  {
+    const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int row = warp * 16 + (mi & 1) * 8 + ri, col = ks * 16 + (mi >> 1) * 8;
+      ldsm_x4(smem_u32(Qs + row * SM::RS + col), qa[ks]);
+    }
+  }
+  const int row_lo = warp * 16 + g8;
+  const int qlo = q0 + row_lo / G, qhi = q0 + (row_lo + 8) / G;
+  const int mlo = qlo - WD, mhi = qhi - WD;
+  const bool vlo = qlo < q1, vhi = qhi < q1;
+
+  float o[DT][4];
+#pragma unroll
+  for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+
+  for (int t = 0; t < ntiles; ++t) {
+    if (t + 1 < ntiles) {
+      issue(t + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int st = t & 1;
+    const uint32_t kbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st) * SM::TILE);
+    const uint32_t vbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st + 1) * SM::TILE);
+
+    float sc[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+    {
+      const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+        for (int jp = 0; jp < NT / 2; ++jp) {
+          uint32_t r[4];
+          const int key = jp * 16 + (mi >> 1) * 8 + ri, col = ks * 16 + (mi & 1) * 8;
+          ldsm_x4(kbase + static_cast<uint32_t>((key * SM::RS + col) * 2), r);
+          mma_bf16_16816(sc[2 * jp], qa[ks], r[0], r[1]);
+          mma_bf16_16816(sc[2 * jp + 1], qa[ks], r[2], r[3]);
+        }
+      }
+    }
+
+    // mask by the running top-k rule, base-2 logits, online softmax
+    const int* kp = kpos + st * kMmaKeys;
+    const int* kc = kcut + st * kMmaKeys;
+    float tmax_lo = -INFINITY, tmax_hi = -INFINITY;
+#pragma unroll
+    for (int jn = 0; jn < NT; ++jn) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = jn * 8 + tig * 2 + e;
+        const int j = kp[key], c = kc[key];
+        const bool ok_lo = j >= 0 && vlo && j <= qlo && (j < S || j > mlo || c > mlo);
+        const bool ok_hi = j >= 0 && vhi && j <= qhi && (j < S || j > mhi || c > mhi);
+        sc[jn][e] = ok_lo ? sc[jn][e] * p.scale_log2 : -INFINITY;
+        sc[jn][2 + e] = ok_hi ? sc[jn][2 + e] * p.scale_log2 : -INFINITY;
+        tmax_lo = fmaxf(tmax_lo, sc[jn][e]);
+        tmax_hi = fmaxf(tmax_hi, sc[jn][2 + e]);
+      }
+    }
+    tmax_lo = fmaxf(tmax_lo, __shfl_xor_sync(0xffffffffu, tmax_lo, 1));
+    tmax_lo = fmaxf(tmax_lo, __shfl_xor_sync(0xffffffffu, tmax_lo, 2));
+    tmax_hi = fmaxf(tmax_hi, __shfl_xor_sync(0xffffffffu, tmax_hi, 1));
+    tmax_hi = fmaxf(tmax_hi, __shfl_xor_sync(0xffffffffu, tmax_hi, 2));
+    const float nm_lo = fmaxf(m_lo, tmax_lo), nm_hi = fmaxf(m_hi, tmax_hi);
+    const float a_lo = (nm_lo == -INFINITY) ? 1.f : exp2f(m_lo - nm_lo);
+    const float a_hi = (nm_hi == -INFINITY) ? 1.f : exp2f(m_hi - nm_hi);
+    float ps_lo = 0.f, ps_hi = 0.f;
+    uint32_t pa[NT / 2][4];
+#pragma unroll
+    for (int jn = 0; jn < NT; ++jn) {
+      const float p0 = sc[jn][0] == -INFINITY ? 0.f : exp2f(sc[jn][0] - nm_lo);
+      const float p1 = sc[jn][1] == -INFINITY ? 0.f : exp2f(sc[jn][1] - nm_lo);
+      const float p2 = sc[jn][2] == -INFINITY ? 0.f : exp2f(sc[jn][2] - nm_hi);
+      const float p3 = sc[jn][3] == -INFINITY ? 0.f : exp2f(sc[jn][3] - nm_hi);
+      ps_lo += p0 + p1;
+      ps_hi += p2 + p3;
+      pa[jn >> 1][(jn & 1) * 2 + 0] = pack_bf16(p0, p1);
+      pa[jn >> 1][(jn & 1) * 2 + 1] = pack_bf16(p2, p3);
+    }
+    ps_lo += __shfl_xor_sync(0xffffffffu, ps_lo, 1);
+    ps_lo += __shfl_xor_sync(0xffffffffu, ps_lo, 2);
+    ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 1);
+    ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 2);
+    l_lo = l_lo * a_lo + ps_lo;
+    l_hi = l_hi * a_hi + ps_hi;
+    m_lo = nm_lo;
+    m_hi = nm_hi;
+#pragma unroll
+    for (int i = 0; i < DT; ++i) {
+      o[i][0] *= a_lo;
+      o[i][1] *= a_lo;
+      o[i][2] *= a_hi;
+      o[i][3] *= a_hi;
+    }
+
+    // O += P V
+    {
+      const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+      for (int kk = 0; kk < kMmaKeys / 16; ++kk) {
+#pragma unroll
+        for (int dp = 0; dp < DT / 2; ++dp) {
+          uint32_t r[4];
+          const int key = kk * 16 + (mi & 1) * 8 + ri, col = dp * 16 + (mi >> 1) * 8;
+          ldsm_x4_t(vbase + static_cast<uint32_t>((key * SM::RS + col) * 2), r);
+          mma_bf16_16816(o[2 * dp], pa[kk], r[0], r[1]);
+          mma_bf16_16816(o[2 * dp + 1], pa[kk], r[2], r[3]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int row = row_lo + 8 * h;
+    const int qpos = h ? qhi : qlo;
+    if (qpos >= q1) continue;
+    const int g = row % G;
+    const size_t rowi = (static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos;
+    const float inv = 1.f / (h ? l_hi : l_lo);
+#pragma unroll
+    for (int i = 0; i < DT; ++i)
+      *reinterpret_cast<uint32_t*>(og + rowi * DH + i * 8 + tig * 2) = pack_bf16(o[i][2 * h] * inv, o[i][2 * h + 1] * inv);
+    if (p.lse != nullptr && tig == 0)
+      p.lse[rowi] = ((h ? m_hi : m_lo) + log2f(h ? l_hi : l_lo)) * 0.69314718055994531f;
+  }
+}
+
+template <int DH>
+int launch_attn_f32(const PaArgs& pa, int units, int n, cudaStream_t st) {
   const size_t smem = PaSmem<DH>::bytes(pa.cand_cap);
   static size_t smem_set = 0;
   if (smem > 48 * 1024 && smem > smem_set) {
-    if (cudaFuncSetAttribute(sparse_attn_kernel<T, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(sparse_attn_kernel<float, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return -1;
     smem_set = smem;
   }
   dim3 grid((n + pa.qt - 1) / pa.qt, units);
-  sparse_attn_kernel<T, DH><<<grid, kPaThreads, smem, st>>>(pa);
+  sparse_attn_kernel<float, DH><<<grid, kPaThreads, smem, st>>>(pa);
+  return 0;
+}
+
+template <int DH>
+int launch_attn_bf16(const PaArgs& pa, int units, int n, cudaStream_t st) {
+  const size_t smem = MmaSmem<DH>::bytes(pa.cand_cap);
+  static size_t smem_set = 0;
+  if (smem > 48 * 1024 && smem > smem_set) {
+    if (cudaFuncSetAttribute(sparse_attn_mma_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return -1;
+    smem_set = smem;
+  }
+  dim3 grid((n + pa.qt - 1) / pa.qt, units);
+  sparse_attn_mma_kernel<DH><<<grid, kMmaThreads, smem, st>>>(pa);
   return 0;
 }
 
 }  // namespace
 
-int plan_prefill_attention(const LayerArgs& a, int n, PrefillAttnPlan* p) {
+int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan* p) {
   if (n < 0 || kPaRows % a.G != 0) return -2;
   if (a.d != 64 && a.d != 128) return -2;
   PrefillAttnPlan P{};
@@ -414,7 +668,7 @@ int plan_prefill_attention(const LayerArgs& a, int n, PrefillAttnPlan* p) {
   P.ne = max(0, n - a.W - a.D - a.S);
   P.npow = next_pow2(max(P.ne, 1));
   P.words = max(1, (P.ne + 31) / 32);
-  P.qt = kPaRows / a.G;
+  P.qt = (dtype == 0 ? kPaRows : kPaMmaRows) / a.G;
   const int64_t cc = static_cast<int64_t>(a.S) + a.K + P.qt + a.W + a.D;
   if (cc > (1 << 14)) return -2;   // the candidate list lives in shared memory
   P.cand_cap = static_cast<int>(cc);
@@ -480,10 +734,9 @@ int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPla
   pa.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.d));
   int r;
   if (dtype == 0)
-    r = (a.d == 128) ? launch_attn<float, 128>(pa, a.units, p.n, st) : launch_attn<float, 64>(pa, a.units, p.n, st);
+    r = (a.d == 128) ? launch_attn_f32<128>(pa, a.units, p.n, st) : launch_attn_f32<64>(pa, a.units, p.n, st);
   else
-    r = (a.d == 128) ? launch_attn<__nv_bfloat16, 128>(pa, a.units, p.n, st)
-                     : launch_attn<__nv_bfloat16, 64>(pa, a.units, p.n, st);
+    r = (a.d == 128) ? launch_attn_bf16<128>(pa, a.units, p.n, st) : launch_attn_bf16<64>(pa, a.units, p.n, st);
   if (r != 0) return r;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

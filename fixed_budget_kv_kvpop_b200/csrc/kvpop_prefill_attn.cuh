@@ -14,8 +14,10 @@ namespace kvpop {
 int launch_prompt_scores(const LayerArgs& a, int dtype, const void* k, const void* v, int n, const float* ext,
                          float* out, int cap, cudaStream_t st);
 
-// Rows of query heads one attention CTA computes (query positions x G).
+// Rows of query heads one attention CTA computes (query positions x G):
+// fp32 kernel (FMA pipes) and bf16 kernel (tensor cores).
 constexpr int kPaRows = 64;
+constexpr int kPaMmaRows = 128;
 // Candidate keys staged per tile.
 constexpr int kPaKeys = 32;
 // Largest sort handled in shared memory (keys); larger sorts run in the workspace.
@@ -28,14 +30,14 @@ struct PrefillAttnPlan {
   int ne;           // tokens that become eligible in the prompt: max(0, n - W - D - S)
   int npow;         // sort length: next power of two >= max(ne, 1)
   int words;        // bitmap words: (ne + 31) / 32, at least 1
-  int qt;           // query positions per attention CTA: kPaRows / G
+  int qt;           // query positions per attention CTA: kPaRows / G (fp32) or kPaMmaRows / G (bf16)
   int cand_cap;     // candidate keys of one CTA at most: S + K + qt + W + D
   size_t cut_off, score_off, keys_off, bits_off, total;   // workspace layout (bytes)
   bool keys_global, bits_global;
 };
 
 // Plans the workspace and launch shapes; returns 0 or -2 (shape not supported).
-int plan_prefill_attention(const LayerArgs& a, int n, PrefillAttnPlan* p);
+int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan* p);
 
 // Cutoffs then attention, on `st`.  cut, scores, keys and bits point into the
 // caller's workspace at the plan's offsets.  Returns 0, -1 (CUDA) or -2.
