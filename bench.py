@@ -10,6 +10,11 @@ budget 1024 = 4 sinks + 128 window + 892 long-range, prompt 8192).  Data are
 synthetic (seeded), shaped like the pages' workloads; the cache (9.7 GB) is
 far larger than L2, so no flush is needed between steps.
 
+`--path prefill-attention` times instead the parallel sparse prefill
+attention of one layer of the same shape (kvpop_prefill_attention: prompt
+scores, running cutoffs and the masked attention of all 8192 positions) and
+prints its own line, with the roofline against the bf16 tensor peak.
+
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle
 instead (the reference arm).  Multi-GPU: one replica per rank (the path
 shards into independent (batch row, KV head) units; no data-path
@@ -38,9 +43,13 @@ METRIC = "decode tokens/s and achieved HBM GB/s (% of peak) at 75%/88% KV compre
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 200 decode, 10 prefill-attention)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kvpop", "reference"], default="kvpop")
+    ap.add_argument("--path", choices=["decode", "prefill-attention"], default="decode",
+                    help="decode (the headline) or the parallel sparse prefill attention of one layer")
+    ap.add_argument("--pa-batch", type=int, default=0,
+                    help="prefill-attention path: batch rows (default: the workload's; smaller for profiling)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cr88")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-e2e", action="store_true")
@@ -538,6 +547,121 @@ def run_e2e(args, w, cache, torch, world):
             "d2h_bytes_per_step": d2h, "steps": K, "ms_per_step": ms / K}
 
 
+PA_METRIC = "prefill attention tokens/s under the running top-k mask (one layer: scores, cutoffs, attention)"
+
+
+def prefill_attention_flops(w: wl.Workload) -> float:
+    """Algorithmic flops of one layer's prefill attention: 2 * d for q.k and
+    2 * d for p.v per attended (position, query head) pair; position q attends
+    to min(q + 1, S + W + D + K) tokens."""
+    B = w.sinks + w.window + w.delay + w.topk
+    pairs = sum(min(q + 1, B) for q in range(w.prefill))
+    return 4.0 * w.head_dim * pairs * w.n_q_heads * w.batch
+
+
+def oracle_prefill_rows_per_s(w: wl.Workload, seconds: float):
+    """The oracle's per-position computation (running top-k at q, attended set,
+    attention) on rows sampled evenly over one unit's prompt."""
+    import numpy as np
+    from oracle import kvpop_oracle as orc
+    one = w.replace(batch=1, n_layers=1)
+    k, v = wl.prompt_kv(one, 0, master=1)
+    q = wl.prompt_queries(one, 0, master=1)
+    w1, b1, w2, b2 = wl.scorer_weights(one, master=1)
+    G = w.group
+    kk, vv = k[0, 0].double().numpy(), v[0, 0].double().numpy()
+    qq = q[0, :G].double().numpy().transpose(1, 0, 2)
+    s = orc.unit_scores_mlp(kk, vv, w1[0, 0].double().numpy(), b1[0, 0].double().numpy(),
+                            w2[0, 0].double().numpy(), float(b2[0, 0]))
+    rows = np.linspace(0, w.prefill - 1, 2048).astype(int)
+    t0 = time.perf_counter()
+    done = 0
+    for qp in rows:
+        T = orc.running_topk(s, int(qp), w.sinks, w.window, w.delay, w.topk)
+        A = orc.attended_positions(int(qp), w.sinks, w.window, w.delay, T)
+        orc.attention(qq[qp], kk[A], vv[A])
+        done += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    tok_s = done / dt / w.n_kv_heads
+    desc = (f"{done} prompt positions of one (batch row, KV head) unit of the {w.name} shape, spread evenly "
+            f"over the {w.prefill}-token prompt, scores untimed ({dt:.1f} s); one prompt token = "
+            f"{w.n_kv_heads} unit-rows (all KV heads of one batch row, one layer)")
+    return tok_s, desc
+
+
+def run_prefill_attention(args, w, torch):
+    import fixed_budget_kv_kvpop_b200 as kp
+    steps = args.steps if args.steps is not None else 10
+    one = w.replace(name=w.name + "_L1", n_layers=1)
+    if args.pa_batch:
+        one = one.replace(name=f"{w.name}_L1_b{args.pa_batch}", batch=args.pa_batch)
+    weights = tuple(t.cuda() for t in wl.scorer_weights(one))
+    w1, b1, w2, b2 = weights
+    cfg = kp.make_config(batch=one.batch, n_layers=1, n_q_heads=one.n_q_heads, n_kv_heads=one.n_kv_heads,
+                         head_dim=one.head_dim, sinks=one.sinks, window=one.window, topk=one.topk,
+                         delay=one.delay, ref_context=one.prefill, compression_ratio=one.compression_ratio,
+                         max_prefill_chunk=1, dtype=one.dtype, scorer_hidden=one.scorer_hidden,
+                         w1=w1, b1=b1, w2=w2, b2=b2)
+    cache = kp.KVPopCache(cfg, keepalive=weights)
+    n = one.prefill
+    k, v = wl.prompt_kv(one, 0, device="cuda")
+    q = wl.prompt_queries(one, 0, device="cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty((one.batch, one.n_q_heads, n), dtype=torch.float32, device="cuda")
+    ws = torch.empty(cache.prefill_attention_workspace_bytes(n), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        cache.prefill_attention(0, q, k, v, out, lse, ws, stream=stream)
+    torch.cuda.synchronize()
+    st, bits = cache.get_error()
+    if st != 0:
+        raise RuntimeError(f"device error after warm-up: status {st} bits {bits}")
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        cache.prefill_attention(0, q, k, v, out, lse, ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / steps
+    st, bits = cache.get_error()
+    if st != 0:
+        raise RuntimeError(f"device error in timed region: status {st} bits {bits}")
+    flops = prefill_attention_flops(one)
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, kind = float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    achieved = flops / (ms / 1e3) / 1e12
+    res = {
+        "metric": PA_METRIC, "value": one.batch * n / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": one.dtype, "data": "synthetic",
+        "config": {"workload": one.name, "batch": one.batch, "layers": 1, "q_heads": one.n_q_heads,
+                   "kv_heads": one.n_kv_heads, "head_dim": one.head_dim, "sinks": one.sinks,
+                   "window": one.window, "topk": one.topk, "delay": one.delay, "prompt": n,
+                   "l2": "no flush: q, k, v (%.1f GB) larger than L2" % ((q.numel() + 2 * k.numel()) * 2 / 1e9)},
+        "roofline": {"kernel": "whole call: prompt scorer + cutoff_kernel + sparse_attn_mma_kernel",
+                     "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "flops_per_call": flops, "peak_kind": kind,
+                     "note": "flops of the attention alone over the time of the whole call; the launch list "
+                             "under profiles/ gives each kernel's share"},
+        "gpu_launches": 3 * steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        v_, desc = oracle_prefill_rows_per_s(one, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc,
+                               "host": host_info()}
+    return res
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -547,10 +671,19 @@ def main():
     if args.layers and args.layers != w.n_layers:
         w = w.replace(name=f"{w.name}_L{args.layers}", n_layers=args.layers)
     if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 200
         run_reference(args, w, rank, world)
         return
     import torch
     torch.cuda.set_device(local)
+    if args.path == "prefill-attention":
+        if world > 1 and rank != 0:
+            return
+        print(json.dumps(run_prefill_attention(args, w, torch)), flush=True)
+        return
+    if args.steps is None:
+        args.steps = 200
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))

@@ -464,6 +464,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs 
   }
   const int count = gather_candidates<kMmaThreads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
   const int ntiles = (count + kMmaKeys - 1) / kMmaKeys;
+  const int m1 = q1 - 1 - WD;   // newest eligible position of the tile's last query
+  int* tile_full = wtot + 8;      // [stage][2 warps]: every key visible to every query of the tile
 
   auto issue = [&](int t) {
     const int st = t & 1;
@@ -471,8 +473,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs 
     if (tid < kMmaKeys) {
       const int idx = t0 + tid;
       const int j = idx < count ? cand[idx] : -1;
+      const int c = j >= 0 ? cu[j] : 0;
       kpos[st * kMmaKeys + tid] = j;
-      kcut[st * kMmaKeys + tid] = j >= 0 ? cu[j] : 0;
+      kcut[st * kMmaKeys + tid] = c;
+      const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
+      const unsigned bal = __ballot_sync(0xffffffffu, full);
+      if (lane == 0) tile_full[st * 2 + warp] = (bal == 0xffffffffu);
     }
     const uint32_t kbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st) * SM::TILE);
     const uint32_t vbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st + 1) * SM::TILE);
@@ -539,22 +545,36 @@ __global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs 
       }
     }
 
-    // mask by the running top-k rule, base-2 logits, online softmax
-    const int* kp = kpos + st * kMmaKeys;
-    const int* kc = kcut + st * kMmaKeys;
+    // mask by the running top-k rule, base-2 logits, online softmax.  Most
+    // tiles hold only keys that every query of the CTA attends to.
     float tmax_lo = -INFINITY, tmax_hi = -INFINITY;
+    if (tile_full[st * 2] && tile_full[st * 2 + 1]) {
 #pragma unroll
-    for (int jn = 0; jn < NT; ++jn) {
+      for (int jn = 0; jn < NT; ++jn) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int key = jn * 8 + tig * 2 + e;
-        const int j = kp[key], c = kc[key];
-        const bool ok_lo = j >= 0 && vlo && j <= qlo && (j < S || j > mlo || c > mlo);
-        const bool ok_hi = j >= 0 && vhi && j <= qhi && (j < S || j > mhi || c > mhi);
-        sc[jn][e] = ok_lo ? sc[jn][e] * p.scale_log2 : -INFINITY;
-        sc[jn][2 + e] = ok_hi ? sc[jn][2 + e] * p.scale_log2 : -INFINITY;
-        tmax_lo = fmaxf(tmax_lo, sc[jn][e]);
-        tmax_hi = fmaxf(tmax_hi, sc[jn][2 + e]);
+        for (int e = 0; e < 2; ++e) {
+          sc[jn][e] = vlo ? sc[jn][e] * p.scale_log2 : -INFINITY;
+          sc[jn][2 + e] = vhi ? sc[jn][2 + e] * p.scale_log2 : -INFINITY;
+          tmax_lo = fmaxf(tmax_lo, sc[jn][e]);
+          tmax_hi = fmaxf(tmax_hi, sc[jn][2 + e]);
+        }
+      }
+    } else {
+      const int* kp = kpos + st * kMmaKeys;
+      const int* kc = kcut + st * kMmaKeys;
+#pragma unroll
+      for (int jn = 0; jn < NT; ++jn) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = jn * 8 + tig * 2 + e;
+          const int j = kp[key], c = kc[key];
+          const bool ok_lo = j >= 0 && vlo && j <= qlo && (j < S || j > mlo || c > mlo);
+          const bool ok_hi = j >= 0 && vhi && j <= qhi && (j < S || j > mhi || c > mhi);
+          sc[jn][e] = ok_lo ? sc[jn][e] * p.scale_log2 : -INFINITY;
+          sc[jn][2 + e] = ok_hi ? sc[jn][2 + e] * p.scale_log2 : -INFINITY;
+          tmax_lo = fmaxf(tmax_lo, sc[jn][e]);
+          tmax_hi = fmaxf(tmax_hi, sc[jn][2 + e]);
+        }
       }
     }
     tmax_lo = fmaxf(tmax_lo, __shfl_xor_sync(0xffffffffu, tmax_lo, 1));
