@@ -144,18 +144,32 @@ template <> struct PaIo<float> {
 // in ascending position: the sinks, the long-range tokens still kept at m0
 // (c_j > m0; at most K of them) and the recent block [max(S, m0 + 1), q1).
 // Every key a query of the tile may attend to is among them.  Block-wide
-// (all NT threads); returns the count (at most cap).
+// (all NT threads); returns the count (at most cap).  Each thread scans 8
+// consecutive positions per round (8 cutoff loads in flight), and one block
+// scan per NT * 8 positions places the kept ones.
 template <int NT>
 __device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1, int cap) {
+  constexpr int R = 8;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ns = min(S, q1);
   for (int i = tid; i < ns; i += NT) cand[i] = i;
   int count = ns;
-  for (int base = S; base <= m0; base += NT) {
-    const int j = base + tid;
-    const bool f = j <= m0 && cu[j] > m0;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) wtot[warp] = __popc(bal);
+  for (int base = S; base <= m0; base += NT * R) {
+    const int j0 = base + tid * R;
+    int c[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) c[r] = (j0 + r <= m0) ? cu[j0 + r] : 0;
+    unsigned mine = 0u;
+#pragma unroll
+    for (int r = 0; r < R; ++r) mine |= (j0 + r <= m0 && c[r] > m0) ? (1u << r) : 0u;
+    const int cnt = __popc(mine);
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    if (lane == 31) wtot[warp] = inc;
     __syncthreads();
     int off = count, total = 0;
 #pragma unroll
@@ -164,8 +178,14 @@ __device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S,
       off += (w < warp) ? t : 0;
       total += t;
     }
-    const int slot = off + __popc(bal & ((1u << lane) - 1u));
-    if (f && slot < cap) cand[slot] = j;
+    off += inc - cnt;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if ((mine >> r) & 1u) {
+        if (off < cap) cand[off] = j0 + r;
+        ++off;
+      }
+    }
     count += total;
     __syncthreads();
   }
@@ -467,19 +487,29 @@ __global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs 
   const int m1 = q1 - 1 - WD;   // newest eligible position of the tile's last query
   int* tile_full = wtot + 8;      // [stage][2 warps]: every key visible to every query of the tile
 
-  auto issue = [&](int t) {
-    const int st = t & 1;
-    const int t0 = t * kMmaKeys;
+  // Key metadata of tile t: the first kMmaKeys threads load (position,
+  // cutoff) early and publish them to shared memory after the current tile's
+  // math, so the cutoff loads' latency hides behind the MMAs.
+  auto load_meta = [&](int t, int& j, int& c) {
     if (tid < kMmaKeys) {
-      const int idx = t0 + tid;
-      const int j = idx < count ? cand[idx] : -1;
-      const int c = j >= 0 ? cu[j] : 0;
+      const int idx = t * kMmaKeys + tid;
+      j = idx < count ? cand[idx] : -1;
+      c = j >= 0 ? cu[j] : 0;
+    }
+  };
+  auto store_meta = [&](int t, int j, int c) {
+    if (tid < kMmaKeys) {
+      const int st = t & 1;
       kpos[st * kMmaKeys + tid] = j;
       kcut[st * kMmaKeys + tid] = c;
       const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
       const unsigned bal = __ballot_sync(0xffffffffu, full);
       if (lane == 0) tile_full[st * 2 + warp] = (bal == 0xffffffffu);
     }
+  };
+  auto issue = [&](int t) {
+    const int st = t & 1;
+    const int t0 = t * kMmaKeys;
     const uint32_t kbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st) * SM::TILE);
     const uint32_t vbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st + 1) * SM::TILE);
     for (int c = tid; c < kMmaKeys * (DH / 8); c += kMmaThreads) {
@@ -493,7 +523,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs 
     }
     cp_async_commit();
   };
-  if (ntiles > 0) issue(0);
+  if (ntiles > 0) {
+    int j0 = -1, c0 = 0;
+    load_meta(0, j0, c0);
+    store_meta(0, j0, c0);
+    issue(0);
+  }
 
   // Q fragments of the warp's 16 rows
   uint32_t qa[KS][4];
@@ -516,7 +551,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs 
   float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
 
   for (int t = 0; t < ntiles; ++t) {
+    int jn = -1, cn = 0;
     if (t + 1 < ntiles) {
+      load_meta(t + 1, jn, cn);
       issue(t + 1);
       cp_async_wait<1>();
     } else {
@@ -628,6 +665,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) sparse_attn_mma_kernel(PaArgs 
         }
       }
     }
+    if (t + 1 < ntiles) store_meta(t + 1, jn, cn);   // stage (t+1)&1 was last read in tile t-1
     __syncthreads();
   }
 
