@@ -85,6 +85,10 @@ def test_null_arguments():
     assert kp.lib.kvpop_decode_step(None, 0, None, None, None, None, None, None) == kp.KVPOP_ERR_INVALID_ARG
     assert kp.lib.kvpop_destroy(None) == kp.KVPOP_ERR_INVALID_ARG
     assert kp.lib.kvpop_get_error(None, None) == kp.KVPOP_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    assert kp.lib.kvpop_prefill_attention_workspace_bytes(None, 16, ctypes.byref(n)) == kp.KVPOP_ERR_INVALID_ARG
+    assert kp.lib.kvpop_prefill_attention(None, 0, None, None, None, 16, None, None, None, None, 0,
+                                          None) == kp.KVPOP_ERR_INVALID_ARG
 
 
 def test_create_rejects_host_memory():

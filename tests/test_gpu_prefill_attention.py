@@ -211,3 +211,33 @@ def test_full_size_target_shape_sampled_rows():
             np.testing.assert_allclose(out[qp], o, rtol=0, atol=gh.BF16_ATOL, err_msg=f"unit {unit} q {qp}")
             np.testing.assert_allclose(lse[qp], orc.attention_lse(q[qp], k[A]), rtol=0, atol=LSE_ATOL["bf16"])
     assert torch.isfinite(r.out).all()
+
+
+def test_argument_errors_enqueue_nothing():
+    """Misaligned or missing pointers, a short workspace and a bad layer are
+    rejected before any work is enqueued; the output stays untouched."""
+    _need_gpu()
+    import fixed_budget_kv_kvpop_b200 as kp
+    w = _case("bf16", 128, 8, 2, S=4, W=16, D=0, K=40, hidden=64)
+    r = run_prefill_attention(w, 64)
+    n = 64
+    need = r.cache.prefill_attention_workspace_bytes(n)
+    out = torch.full_like(r.q, 7.0)
+    ws = torch.empty(need + 64, dtype=torch.uint8, device="cuda")
+    lib, h = kp.lib, r.cache.handle
+
+    def call(layer=0, q=r.q.data_ptr(), out_p=out.data_ptr(), ws_p=ws.data_ptr(), ws_n=need, n_tok=n):
+        return lib.kvpop_prefill_attention(h, layer, q, r.k.data_ptr(), r.v.data_ptr(), n_tok, None, out_p, None,
+                                           ws_p, ws_n, None)
+    assert call(ws_n=need - 1) == kp.KVPOP_ERR_INVALID_ARG
+    assert call(ws_p=ws.data_ptr() + 4) == kp.KVPOP_ERR_INVALID_ARG
+    assert call(q=r.q.data_ptr() + 2) == kp.KVPOP_ERR_INVALID_ARG
+    assert call(out_p=None) == kp.KVPOP_ERR_INVALID_ARG
+    assert call(layer=1) == kp.KVPOP_ERR_INVALID_ARG
+    assert call(n_tok=-1) == kp.KVPOP_ERR_INVALID_ARG
+    assert call(n_tok=0) == kp.KVPOP_OK
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
+    assert call() == kp.KVPOP_OK
+    torch.cuda.synchronize()
+    assert torch.equal(out, r.out)
