@@ -48,7 +48,7 @@ EXPORTED_SYMBOLS = (
     "kvpop_decode_attend", "kvpop_inspect",
     "kvpop_get_layout", "kvpop_get_error", "kvpop_clear_error", "kvpop_debug_poison_error",
     "kvpop_destroy", "kvpop_status_string", "kvpop_decode_step_noalloc",
-    "kvpop_prefill_attention_workspace_bytes", "kvpop_prefill_attention",
+    "kvpop_prefill_attention_workspace_bytes", "kvpop_prefill_attention", "kvpop_prefill_with_attention",
 )
 
 
@@ -99,6 +99,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvpop_decode_step_noalloc": ([P, I32, P, P, P, P, P, P], ctypes.c_int),
         "kvpop_prefill_attention_workspace_bytes": ([P, I32, ctypes.POINTER(SZ)], ctypes.c_int),
         "kvpop_prefill_attention": ([P, I32, P, P, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
+        "kvpop_prefill_with_attention": ([P, I32, P, P, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -221,6 +222,18 @@ class KVPopCache:
                                            _ptr(out), _ptr(lse), _ptr(workspace),
                                            int(workspace.numel() * workspace.element_size()) if workspace is not None
                                            else 0, _stream_ptr(stream)), "kvpop_prefill_attention")
+
+    def prefill_with_attention(self, layer: int, q, k, v, out, lse=None, workspace=None, ext_scores=None,
+                               stream=None):
+        """prefill (whole prompt, empty layer) and prefill_attention in one
+        call: the prompt is scored once; afterwards the layer holds the cache
+        kvpop_prefill would build and is ready for decode steps."""
+        n = int(k.shape[2])
+        _check(lib.kvpop_prefill_with_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
+                                                _ptr(out), _ptr(lse), _ptr(workspace),
+                                                int(workspace.numel() * workspace.element_size())
+                                                if workspace is not None else 0, _stream_ptr(stream)),
+               "kvpop_prefill_with_attention")
 
     def decode_append(self, layer: int, k_new, v_new, ext_score=None, stream=None):
         _check(lib.kvpop_decode_append(self.handle, layer, _ptr(k_new), _ptr(v_new), _ptr(ext_score),

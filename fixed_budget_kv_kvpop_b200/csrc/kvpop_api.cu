@@ -384,6 +384,37 @@ int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const
   return r == 0 ? KVPOP_OK : KVPOP_ERR_CUDA;
 }
 
+int kvpop_prefill_with_attention(kvpop_handle* h, int32_t layer, const void* q, const void* k, const void* v,
+                                 int32_t n_tokens, const float* ext_scores, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers || n_tokens < 0) return KVPOP_ERR_INVALID_ARG;
+  if (h->decoding[layer] || h->n_seen[layer] != 0) return KVPOP_ERR_ORDER;
+  if (n_tokens > h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
+  if (n_tokens == 0) return KVPOP_OK;
+  if (!q || !k || !v || !out || !workspace) return KVPOP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return KVPOP_ERR_INVALID_ARG;
+  const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
+  if (ext && !ext_scores) return KVPOP_ERR_INVALID_ARG;
+  const LayerArgs a = layer_args(h, layer);
+  PrefillAttnPlan p;
+  if (plan_prefill_attention(a, h->cfg.dtype, n_tokens, &p) != 0 || a.units > 65535) return KVPOP_ERR_BAD_SHAPE;
+  if (workspace_bytes < p.total) return KVPOP_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float* es = ext ? ext_scores : nullptr;
+  int r = launch_prefill_attention(a, h->cfg.dtype, p, q, k, v, es, out, lse, ws, st);
+  if (r == -2) return KVPOP_ERR_BAD_SHAPE;
+  if (r != 0) return KVPOP_ERR_CUDA;
+  if (launch_place_kept(a, h->cfg.dtype, p, k, v, ws, st) != 0) return KVPOP_ERR_CUDA;
+  if (launch_prompt_write(a, h->cfg.dtype, k, v, n_tokens, es, st) != 0) return KVPOP_ERR_CUDA;
+  const int c1 = std::min(h->cfg.topk, p.ne);
+  if (launch_decide(a, h->cfg.dtype, n_tokens, c1, st) != 0) return KVPOP_ERR_CUDA;
+  h->n_seen[layer] = n_tokens;
+  h->n_topk[layer] = c1;
+  return KVPOP_OK;
+}
+
 int kvpop_destroy(kvpop_handle* h) {
   if (!h) return KVPOP_ERR_INVALID_ARG;
   delete h;

@@ -607,6 +607,24 @@ int launch_prompt_scores(const LayerArgs& a, int dtype, const void* k, const voi
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
+int launch_prompt_write(const LayerArgs& a, int dtype, const void* k, const void* v, int n, const float* ext,
+                        cudaStream_t st) {
+  ChunkGeom cg;
+  cg.n0 = 0;
+  cg.n1 = n;
+  cg.e0 = a.S;
+  cg.e1 = max(a.S, n - a.W - a.D);
+  cg.c0 = 0;
+  if (n <= 0) return 0;
+  dim3 grid((n + 7) / 8, a.units);
+  if (dtype == 0)
+    write_kernel<float><<<grid, 256, 0, st>>>(a, cg, static_cast<const float*>(k), static_cast<const float*>(v), n, ext);
+  else
+    write_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a, cg, static_cast<const __nv_bfloat16*>(k),
+                                                      static_cast<const __nv_bfloat16*>(v), n, ext);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
 int launch_prefill(const LayerArgs& a, int dtype, const PrefillScratch& ps, const void* k, const void* v,
                    int n_tokens, int n_seen_before, int n_topk_before, const float* ext_scores, cudaStream_t st) {
   if (dtype == 0)

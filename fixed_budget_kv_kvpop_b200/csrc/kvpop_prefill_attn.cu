@@ -719,7 +719,63 @@ int launch_attn_bf16(const PaArgs& pa, int units, int n, cudaStream_t st) {
   return 0;
 }
 
+// ---------------- cache build from the cutoffs ----------------
+// Long-range set at the last prompt position = the tokens whose cutoff is
+// "never"; a whole-prompt prefill places them in ascending position order.
+__global__ void __launch_bounds__(256) place_kept_kernel(LayerArgs a, const int32_t* __restrict__ cut,
+                                                         const float* __restrict__ scores, int score_cap, int n,
+                                                         int ne, const uint8_t* __restrict__ k,
+                                                         const uint8_t* __restrict__ v, int half) {
+  __shared__ int wtot[8];
+  const int u = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* cu = cut + static_cast<size_t>(u) * n;
+  const int base_slot = a.S + a.W + a.D;
+  int count = 0;
+  for (int b0 = 0; b0 < ne; b0 += 256) {
+    const int i = b0 + tid;
+    const int j = a.S + i;
+    const bool f = i < ne && cu[j] == kNever;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) wtot[warp] = __popc(bal);
+    __syncthreads();
+    int off = count, total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      off += (w < warp) ? wtot[w] : 0;
+      total += wtot[w];
+    }
+    off += __popc(bal & ((1u << lane) - 1u));
+    if (f && off < a.K) {
+      const int slot = base_slot + off;
+      uint8_t* dst = a.kv + (static_cast<size_t>(u) * a.NS + slot) * a.row_bytes;
+      const uint8_t* ks = k + (static_cast<size_t>(u) * n + j) * half;
+      const uint8_t* vs = v + (static_cast<size_t>(u) * n + j) * half;
+      for (int b = 0; b < half; b += 16) {
+        *reinterpret_cast<uint4*>(dst + b) = *reinterpret_cast<const uint4*>(ks + b);
+        *reinterpret_cast<uint4*>(dst + half + b) = *reinterpret_cast<const uint4*>(vs + b);
+      }
+      a.pos[static_cast<size_t>(u) * a.NS + slot] = j;
+      a.score[static_cast<size_t>(u) * a.NS + slot] = scores[static_cast<size_t>(u) * score_cap + i];
+    }
+    count += total;
+    __syncthreads();
+  }
+  if ((a.flags & FLAG_DEBUG_CHECKS) && tid == 0 && count != min(a.K, ne)) set_error(a.err, DEVERR_STATE_MISMATCH);
+}
+
 }  // namespace
+
+int launch_place_kept(const LayerArgs& a, int dtype, const PrefillAttnPlan& p, const void* k, const void* v,
+                      const uint8_t* workspace, cudaStream_t st) {
+  if (p.ne <= 0 || a.K <= 0) return 0;
+  const int half = a.d * (dtype == 0 ? 4 : 2);
+  place_kept_kernel<<<a.units, 256, 0, st>>>(a, reinterpret_cast<const int32_t*>(workspace + p.cut_off),
+                                             reinterpret_cast<const float*>(workspace + p.score_off), p.ne, p.n,
+                                             p.ne, static_cast<const uint8_t*>(k), static_cast<const uint8_t*>(v),
+                                             half);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
 
 int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan* p) {
   if (n < 0 || kPaRows % a.G != 0) return -2;

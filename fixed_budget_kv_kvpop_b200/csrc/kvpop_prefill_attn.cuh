@@ -45,4 +45,16 @@ int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPla
                              const void* v, const float* ext, void* out, float* lse, uint8_t* workspace,
                              cudaStream_t st);
 
+// Whole-prompt cache build from the cutoffs of a launch_prefill_attention on
+// the same workspace (the layer must be empty): the tokens kept to the end
+// (cutoff "never") go to the long-range slots in ascending position order,
+// with their ranking priorities.  Returns 0 or -1.
+int launch_place_kept(const LayerArgs& a, int dtype, const PrefillAttnPlan& p, const void* k, const void* v,
+                      const uint8_t* workspace, cudaStream_t st);
+
+// The prompt's sinks, window and staging tokens to their slots (the prefill
+// builder's write step for one whole-prompt chunk).  Returns 0 or -1.
+int launch_prompt_write(const LayerArgs& a, int dtype, const void* k, const void* v, int n, const float* ext,
+                        cudaStream_t st);
+
 }  // namespace kvpop

@@ -243,6 +243,21 @@ int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const
                             int32_t n_tokens, const float* ext_scores, void* out, float* lse, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* kvpop_prefill and kvpop_prefill_attention in one call, for a whole prompt
+ * on an empty layer: the prompt is scored once, its attention outputs (and
+ * log-normalisers, if lse is not NULL) are computed under the running top-k
+ * mask, and the layer's cache is built from the same scores and cutoffs --
+ * the long-range slots receive the tokens whose cutoff is INT32_MAX (kept at
+ * the last position) in ascending position order, exactly what kvpop_prefill
+ * of the whole prompt as one chunk places.  Afterwards the layer is ready for
+ * decode steps (position counter n_tokens).  Arguments, layouts, workspace
+ * and errors as kvpop_prefill_attention, plus KVPOP_ERR_ORDER when the layer
+ * has seen any token.  Page §C.1 / §C.2 (mask and cutoffs) and §I (running
+ * prefix top-k). */
+int kvpop_prefill_with_attention(kvpop_handle* h, int32_t layer, const void* q, const void* k, const void* v,
+                                 int32_t n_tokens, const float* ext_scores, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* Copies layer `layer`'s slot -> position map (int32 [units][slots]), slot
  * scores (fp32 [units][slots]) and per-unit state (int32 [units][4]) to HOST
  * buffers; any of them may be NULL.  Synchronises `stream`.  For tests and

@@ -241,3 +241,82 @@ def test_argument_errors_enqueue_nothing():
     assert call() == kp.KVPOP_OK
     torch.cuda.synchronize()
     assert torch.equal(out, r.out)
+
+
+@pytest.mark.parametrize("dtype,d,hq,hkv,S,W,D,K,hidden,n,external,ties,decay", [
+    ("bf16", 128, 8, 2, 4, 16, 0, 40, 64, 300, False, 0, None),
+    ("bf16", 128, 8, 2, 2, 12, 3, 30, 64, 257, True, 2, None),
+    ("f32", 64, 4, 2, 4, 16, 0, 44, 0, 200, False, 0, None),
+    ("bf16", 64, 8, 2, 4, 16, 2, 20, 32, 180, False, 0, -0.05),
+    ("bf16", 128, 8, 2, 4, 16, 0, 500, 64, 120, True, 1, None),   # fewer eligible tokens than K
+])
+def test_fused_prefill_matches_prefill_then_attention(dtype, d, hq, hkv, S, W, D, K, hidden, n, external, ties,
+                                                      decay):
+    """kvpop_prefill_with_attention (one scoring pass; long-range slots from
+    the cutoffs) leaves bit for bit the cache kvpop_prefill builds (slot map,
+    scores, rows, counters), returns bit for bit the outputs of
+    kvpop_prefill_attention, and the decode steps after it agree bit for bit."""
+    _need_gpu()
+    w = _case(dtype, d, hq, hkv, S=S, W=W, D=D, K=K, hidden=hidden, batch=2)
+    weights = None
+    if not external:
+        weights = tuple(t.cuda() for t in wl.scorer_weights(w.replace(scorer_hidden=max(hidden, 1))))
+    dec = None if decay is None else torch.full((1, hkv), decay, dtype=torch.float32, device="cuda")
+    caches = [gh.build_cache(w, 1, external, weights, max_chunk=n, debug=True, log_decay=dec) for _ in range(2)]
+    k, v = (t.cuda() for t in wl.prompt_kv(w, 0, n_tokens=n))
+    q = wl.prompt_queries(w, 0, n).cuda()
+    steps = 3
+    ext_all = wl.external_scores(w, 0, n + steps, tie_levels=ties).cuda() if external else None
+    ext = ext_all[:, :, :n].contiguous() if external else None
+    outs, lses = [], []
+    for i, c in enumerate(caches):
+        out = torch.full_like(q, float("nan"))
+        lse = torch.full((w.batch, w.n_q_heads, n), float("nan"), device="cuda")
+        ws = torch.empty(c.prefill_attention_workspace_bytes(n), dtype=torch.uint8, device="cuda")
+        if i == 0:
+            c.prefill(0, k, v, ext)
+            c.prefill_attention(0, q, k, v, out, lse, ws, ext)
+        else:
+            c.prefill_with_attention(0, q, k, v, out, lse, ws, ext)
+        outs.append(out)
+        lses.append(lse)
+    torch.cuda.synchronize()
+    for c in caches:
+        st, bits = c.get_error()
+        assert st == 0, (st, bits)
+    assert torch.equal(outs[0], outs[1])
+    assert torch.equal(lses[0], lses[1])
+    ia, ib = caches[0].inspect(0), caches[1].inspect(0)
+    for xa, xb, what in zip(ia, ib, ("slot map", "scores", "state")):
+        assert np.array_equal(xa, xb), what
+    assert torch.equal(caches[0].kv_rows(0), caches[1].kv_rows(0))
+    # with the MLP scorer some long-range slots must be in use, and they must be ascending
+    base = S + W + D
+    pos = ia[0].reshape(w.batch * w.n_kv_heads, -1)[:, base:]
+    for row in pos:
+        kept = [int(x) for x in row if x >= 0]
+        assert kept == sorted(kept) and len(kept) == min(K, max(0, n - W - D - S))
+    for i in range(steps):
+        qd, kn, vn = wl.decode_inputs(w, 0, i)
+        qd, kn, vn = qd.cuda(), kn.cuda(), vn.cuda()
+        es = ext_all[:, :, n + i].contiguous() if external else None
+        res = []
+        for c in caches:
+            o = torch.empty_like(qd)
+            c.decode_step(0, qd, kn, vn, o, es)
+            res.append(o)
+        torch.cuda.synchronize()
+        assert torch.equal(res[0], res[1]), f"decode step {i}"
+
+
+def test_fused_prefill_rejects_a_used_layer():
+    _need_gpu()
+    import fixed_budget_kv_kvpop_b200 as kp
+    w = _case("bf16", 128, 8, 2, S=4, W=16, D=0, K=40, hidden=64)
+    r = run_prefill_attention(w, 64)
+    k, v = r.k, r.v
+    r.cache.prefill(0, k[:, :, :1].contiguous(), v[:, :, :1].contiguous())   # the layer has seen a token
+    ws = torch.empty(r.cache.prefill_attention_workspace_bytes(64), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(r.q)
+    with pytest.raises(kp.KVPopError):
+        r.cache.prefill_with_attention(0, r.q, k, v, out, None, ws)
