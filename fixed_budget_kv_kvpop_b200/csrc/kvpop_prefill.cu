@@ -512,13 +512,10 @@ template <typename T, int D2, int HID>
 int launch_score64(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T* v, int n, float* out, int cap,
                    int n_new, cudaStream_t st) {
   using SG = Score64Geom<D2, HID>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(score64_kernel<T, D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM) !=
-        cudaSuccess)
-      return -1;
-    attr_set = true;
-  }
+  // set on every call: the attribute belongs to the current device
+  if (cudaFuncSetAttribute(score64_kernel<T, D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM) !=
+      cudaSuccess)
+    return -1;
   const int tiles = (n_new + SG::TT - 1) / SG::TT;
   dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
   score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap);
@@ -551,13 +548,9 @@ int launch_scores_t(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T
     const int TT = 4 * (kScoreThreads / HQ);
     const size_t smem = (a.flags & FLAG_EXTERNAL_SCORES) ? 0
                         : (static_cast<size_t>(2 * a.d) * a.hidden + static_cast<size_t>(TT) * 2 * a.d) * sizeof(float);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-      if (cudaFuncSetAttribute(score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return -1;
-      smem_set = smem;
-    }
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem)) != cudaSuccess)
+      return -1;
     dim3 grid((n_new + TT - 1) / TT, a.units);
     score_kernel<T><<<grid, kScoreThreads, smem, st>>>(a, cg, k, v, n, ext, out, cap);
   }

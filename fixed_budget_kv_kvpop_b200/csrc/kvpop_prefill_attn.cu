@@ -692,13 +692,11 @@ __global__ void __launch_bounds__(kMmaThreads, 2) sparse_attn_mma_kernel(PaArgs 
 template <int DH>
 int launch_attn_f32(const PaArgs& pa, int units, int n, cudaStream_t st) {
   const size_t smem = PaSmem<DH>::bytes(pa.cand_cap);
-  static size_t smem_set = 0;
-  if (smem > 48 * 1024 && smem > smem_set) {
-    if (cudaFuncSetAttribute(sparse_attn_kernel<float, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return -1;
-    smem_set = smem;
-  }
+  // set on every call: the attribute belongs to the current device
+  if (smem > 48 * 1024 && cudaFuncSetAttribute(sparse_attn_kernel<float, DH>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem)) != cudaSuccess)
+    return -1;
   dim3 grid((n + pa.qt - 1) / pa.qt, units);
   sparse_attn_kernel<float, DH><<<grid, kPaThreads, smem, st>>>(pa);
   return 0;
@@ -707,13 +705,10 @@ int launch_attn_f32(const PaArgs& pa, int units, int n, cudaStream_t st) {
 template <int DH>
 int launch_attn_bf16(const PaArgs& pa, int units, int n, cudaStream_t st) {
   const size_t smem = MmaSmem<DH>::bytes(pa.cand_cap);
-  static size_t smem_set = 0;
-  if (smem > 48 * 1024 && smem > smem_set) {
-    if (cudaFuncSetAttribute(sparse_attn_mma_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return -1;
-    smem_set = smem;
-  }
+  if (smem > 48 * 1024 && cudaFuncSetAttribute(sparse_attn_mma_kernel<DH>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem)) != cudaSuccess)
+    return -1;
   dim3 grid((n + pa.qt - 1) / pa.qt, units);
   sparse_attn_mma_kernel<DH><<<grid, kMmaThreads, smem, st>>>(pa);
   return 0;
@@ -822,13 +817,9 @@ int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPla
   }
   const size_t cut_smem = (p.keys_global ? 0 : static_cast<size_t>(p.npow) * 8) +
                           (p.bits_global ? 0 : static_cast<size_t>(p.words) * 4);
-  static bool cut_attr = false;
-  if (!cut_attr) {
-    const int mx = kPaSmemSortKeys * 8 + kPaSmemBitmapWords * 4;
-    if (cudaFuncSetAttribute(cutoff_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess)
-      return -1;
-    cut_attr = true;
-  }
+  if (cudaFuncSetAttribute(cutoff_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kPaSmemSortKeys * 8 + kPaSmemBitmapWords * 4) != cudaSuccess)
+    return -1;
   cutoff_kernel<<<a.units, kCutThreads, cut_smem, st>>>(scores, max(p.ne, 1), cut, p.n, p.ne, p.npow, p.words, a.S,
                                                         a.K, keys, bits, p.keys_global ? 1 : 0,
                                                         p.bits_global ? 1 : 0, a.err);
