@@ -460,3 +460,105 @@ def prefill_attention(q_all: np.ndarray, k_all: np.ndarray, v_all: np.ndarray, s
         lse[q] = attention_lse(q_all[q], k_all[A])
         counts.append(len(A))
     return out, lse, counts
+
+
+# ---------------------------------------------------------------------------
+# Stateful mLSTM scorer with delayed readout (§A Background: Linear Attention
+# and mLSTM; §E.3 mLSTM Scorer; §E.4 Delayed Readout).  Oracle only.
+# ---------------------------------------------------------------------------
+#
+# The pages name the parts but give no formulas; readings (each one also in
+# the design notes):
+# * Input x_t = [k_t; v_t] (§E.1).  Write features phi(W_k x_t), value
+#   W_v x_t, read features phi(W_q x_u) of the token being scored.
+# * Hedgehog feature map (§E.3): project to p dims, then [softmax(z); softmax(-z)]
+#   (2p features: "halves the projected dimension before positive and negative
+#   softmax features").
+# * Scalar gates from headwise projections: input pre-activation
+#   i~_t = w_i . x_t + b_i used as exp(i~_t); forget gate sigmoid(w_f . x_t + b_f)
+#   (log-sigmoid in the stabilised form).  No output gate (§A: removed).
+# * The numerically stabilised mLSTM recurrence (§E.3) with C_0 = 0, n_0 = 0,
+#   m_0 = 0:  m_t = max(log f_t + m_{t-1}, i~_t),  i'_t = exp(i~_t - m_t),
+#   f'_t = exp(log f_t + m_{t-1} - m_t),  C_t = f'_t C_{t-1} + i'_t v_t phi_t^T,
+#   n_t = f'_t n_{t-1} + i'_t phi_t,  readout h = C r / max(|n . r|, exp(-m)).
+# * Delayed readout (§E.4): the token u that becomes eligible at step
+#   q = u + W + D is read with the state after token q; score =
+#   w_o . SiLU(h) + b_o (the "SiLU-based transformation with a bias term"; the
+#   optional normalisation is left out).  The score is fixed from then on, so
+#   the running top-k rule above applies unchanged.
+
+def hedgehog(z: np.ndarray) -> np.ndarray:
+    """[softmax(z); softmax(-z)] along the last axis, float64 (§E.3)."""
+    z = np.asarray(z, np.float64)
+    a = np.exp(z - z.max(axis=-1, keepdims=True))
+    b = np.exp(-z - (-z).max(axis=-1, keepdims=True))
+    return np.concatenate([a / a.sum(axis=-1, keepdims=True), b / b.sum(axis=-1, keepdims=True)], axis=-1)
+
+
+def log_sigmoid(x: float) -> float:
+    x = float(x)
+    return -math.log1p(math.exp(-x)) if x >= 0 else x - math.log1p(math.exp(x))
+
+
+@dataclass
+class MlstmParams:
+    """Headwise mLSTM scorer weights: wq, wk [p][2d]; wv [dv][2d];
+    wi, wf [2d]; bi, bf scalars; wo [dv]; bo scalar."""
+    wq: np.ndarray
+    wk: np.ndarray
+    wv: np.ndarray
+    wi: np.ndarray
+    bi: float
+    wf: np.ndarray
+    bf: float
+    wo: np.ndarray
+    bo: float
+
+
+def mlstm_states(x_all: np.ndarray, P: MlstmParams):
+    """Stabilised recurrence over tokens 0..n-1; returns the list of
+    (C_t, n_t, m_t) after each token t (§E.3)."""
+    x_all = np.asarray(x_all, np.float64)
+    dv, f2 = P.wv.shape[0], 2 * P.wk.shape[0]
+    C, nv, m = np.zeros((dv, f2)), np.zeros(f2), 0.0
+    out = []
+    for x in x_all:
+        phi = hedgehog(P.wk @ x)
+        val = P.wv @ x
+        it = float(P.wi @ x) + P.bi
+        lf = log_sigmoid(float(P.wf @ x) + P.bf)
+        m_new = max(lf + m, it)
+        ip, fp = math.exp(it - m_new), math.exp(lf + m - m_new)
+        C = fp * C + ip * np.outer(val, phi)
+        nv = fp * nv + ip * phi
+        m = m_new
+        out.append((C.copy(), nv.copy(), m))
+    return out
+
+
+def mlstm_readout(C: np.ndarray, nv: np.ndarray, m: float, r: np.ndarray) -> np.ndarray:
+    """h = C r / max(|n . r|, exp(-m)) (§A: normalised retrieval from the summary)."""
+    return (C @ r) / max(abs(float(nv @ r)), math.exp(-m))
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def unit_scores_mlstm(k_all, v_all, P: MlstmParams, S: int, W: int, D: int) -> np.ndarray:
+    """Delayed-readout score of every token u >= S whose eligibility step
+    q = u + W + D lies inside the sequence, rounded to float32 (§E.4, §F);
+    NaN for the others (sinks, and tokens not yet eligible at the end)."""
+    x_all = head_input(k_all, v_all)
+    n = len(x_all)
+    states = mlstm_states(x_all, P)
+    s = np.full(n, np.nan)
+    for u in range(S, n):
+        q = u + W + D
+        if q >= n:
+            break
+        C, nv, m = states[q]
+        h = mlstm_readout(C, nv, m, hedgehog(P.wq @ x_all[u]))
+        s[u] = float(P.wo @ silu(h)) + P.bo
+    return ranking_score(s)

@@ -351,6 +351,97 @@ def pin_prefill_attention_matches_slot_simulator():
             o, w = orc.attention(qq[q], k[A], v[A])
             np.testing.assert_allclose(out[q], o, rtol=0, atol=1e-13)
 
+
+# ---------------------------------------------------------------------------
+# Stateful mLSTM scorer with delayed readout (§A, §E.3, §E.4)
+# ---------------------------------------------------------------------------
+
+def _mlstm_params(seed, d, p, dv, bi, bf):
+    rng = np.random.default_rng(seed)
+    return orc.MlstmParams(wq=rng.normal(size=(p, 2 * d)) * 0.7, wk=rng.normal(size=(p, 2 * d)) * 0.7,
+                           wv=rng.normal(size=(dv, 2 * d)), wi=rng.normal(size=2 * d) * 0.3, bi=bi,
+                           wf=rng.normal(size=2 * d) * 0.3, bf=bf, wo=rng.normal(size=dv), bo=0.1)
+
+
+def pin_hedgehog_feature_map():
+    """[softmax(z); softmax(-z)] as torch.softmax computes it; each half sums
+    to 1; negating z swaps the halves."""
+    z = np.random.default_rng(5).normal(size=(6, 7)) * 3.0
+    phi = orc.hedgehog(z)
+    zt = torch.tensor(z)
+    ref = torch.cat([torch.softmax(zt, -1), torch.softmax(-zt, -1)], -1).numpy()
+    np.testing.assert_allclose(phi, ref, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(phi[:, :7].sum(-1), 1.0, atol=1e-14)
+    np.testing.assert_allclose(orc.hedgehog(-z), np.concatenate([phi[:, 7:], phi[:, :7]], -1), atol=1e-15)
+
+
+def pin_mlstm_stabilised_equals_closed_form():
+    """The stabilised recurrence reads out what the closed form of the gated
+    outer-product sum gives (§A: recurrent and parallel forms agree): with
+    g_t = exp(i~_t) * prod_{s=t+1..q} sigmoid(f~_s), C = sum_t g_t v_t phi_t^T,
+    n = sum_t g_t phi_t and h = C r / max(|n . r|, 1).  A strongly negative
+    input bias drives |n . r| below 1 so that the floor is exercised."""
+    d, p, dv, n = 3, 4, 2, 18
+    floor_used = False
+    for seed, (bi, bf) in enumerate([(-4.0, 1.0), (0.5, -0.5), (3.0, 2.0)]):
+        P = _mlstm_params(40 + seed, d, p, dv, bi, bf)
+        x = np.random.default_rng(60 + seed).normal(size=(n, 2 * d))
+        states = orc.mlstm_states(x, P)
+        ig = [math.exp(float(P.wi @ xt) + P.bi) for xt in x]
+        fg = [1.0 / (1.0 + math.exp(-(float(P.wf @ xt) + P.bf))) for xt in x]
+        rr = np.random.default_rng(80 + seed).normal(size=(n, 2 * d))
+        for q in range(n):
+            C = np.zeros((dv, 2 * p))
+            nn = np.zeros(2 * p)
+            for t in range(q + 1):
+                g = ig[t] * math.prod(fg[t + 1:q + 1])
+                phi = orc.hedgehog(P.wk @ x[t])
+                C += g * np.outer(P.wv @ x[t], phi)
+                nn += g * phi
+            r = orc.hedgehog(P.wq @ rr[q])
+            den = abs(float(nn @ r))
+            floor_used |= den < 1.0
+            h_ref = (C @ r) / max(den, 1.0)
+            np.testing.assert_allclose(orc.mlstm_readout(*states[q], r), h_ref, rtol=1e-10, atol=1e-12)
+    assert floor_used
+
+
+def pin_mlstm_delayed_readout_is_causal_and_forward_looking():
+    """The score of token u (eligible at q = u + W + D) does not change when a
+    later token changes, and does change when token q changes: the state it is
+    read from has processed exactly the tokens through q (§E.4)."""
+    S, W, D, d, n = 2, 4, 1, 3, 30
+    P = _mlstm_params(7, d, 4, 2, 0.0, 1.0)
+    rng = np.random.default_rng(9)
+    k, v = rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    s = orc.unit_scores_mlstm(k, v, P, S, W, D)
+    assert np.isnan(s[:S]).all() and np.isnan(s[n - W - D:]).all() and np.isfinite(s[S:n - W - D]).all()
+    u = 10
+    q = u + W + D
+    k2 = k.copy()
+    k2[q + 1] += 5.0
+    s2 = orc.unit_scores_mlstm(k2, v, P, S, W, D)
+    np.testing.assert_array_equal(s2[:q + 1 - W - D], s[:q + 1 - W - D])
+    k3 = k.copy()
+    k3[q] += 5.0
+    s3 = orc.unit_scores_mlstm(k3, v, P, S, W, D)
+    assert s3[u] != s[u]
+    np.testing.assert_array_equal(s3[:u], s[:u])
+
+
+def pin_mlstm_scores_drive_the_running_topk():
+    """Scores fixed at eligibility plug into the retention rule unchanged: the
+    slot simulator holds the brute-force top-k at every decode step."""
+    S, W, D, K, d, P_len, steps = 2, 4, 2, 5, 3, 20, 15
+    P = _mlstm_params(11, d, 4, 2, 0.0, 1.0)
+    rng = np.random.default_rng(12)
+    n = P_len + steps
+    k, v = rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    q = rng.normal(size=(steps, 2, d))
+    s = orc.unit_scores_mlstm(k, v, P, S, W, D)
+    res = orc.run_unit(k, v, q, s, S, W, D, K, P_len)
+    assert all(len(t) == min(K, max(0, P_len + i - W - D - S + 1)) for i, t in enumerate(res.topk_sets[1:]))
+
 ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1,
             pin_prefill_chunk_placement, pin_dense_when_budget_covers_context,
             pin_budget_invariant_and_structure, pin_softmax_rows_sum_to_one,
@@ -359,4 +450,6 @@ ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1
             pin_float32_single_rounding, pin_linear_scorer,
             pin_prefill_mask_hand_example, pin_running_cutoffs_match_fenwick,
             pin_running_cutoffs_are_intervals, pin_prefill_attention_dense_when_budget_covers_context,
-            pin_prefill_attention_matches_slot_simulator]
+            pin_prefill_attention_matches_slot_simulator, pin_hedgehog_feature_map,
+            pin_mlstm_stabilised_equals_closed_form, pin_mlstm_delayed_readout_is_causal_and_forward_looking,
+            pin_mlstm_scores_drive_the_running_topk]

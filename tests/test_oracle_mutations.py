@@ -133,6 +133,48 @@ def _lse_unscaled(q, keys):
 _ORIG_CUTOFFS = orc.running_cutoffs
 
 
+def _hedgehog_positive_only(z):
+    z = np.asarray(z, np.float64)
+    a = np.exp(z - z.max(axis=-1, keepdims=True))
+    a = a / a.sum(axis=-1, keepdims=True)
+    return np.concatenate([a, a], axis=-1)
+
+
+def _mlstm_forget_not_log(x_all, P):
+    x_all = np.asarray(x_all, np.float64)
+    dv, f2 = P.wv.shape[0], 2 * P.wk.shape[0]
+    C, nv, m = np.zeros((dv, f2)), np.zeros(f2), 0.0
+    out = []
+    for x in x_all:
+        phi = orc.hedgehog(P.wk @ x)
+        it = float(P.wi @ x) + P.bi
+        f = 1.0 / (1.0 + math.exp(-(float(P.wf @ x) + P.bf)))
+        m_new = max(f + m, it)
+        ip, fp = math.exp(it - m_new), math.exp(f + m - m_new)
+        C = fp * C + ip * np.outer(P.wv @ x, phi)
+        nv = fp * nv + ip * phi
+        m = m_new
+        out.append((C.copy(), nv.copy(), m))
+    return out
+
+
+def _mlstm_readout_no_floor(C, nv, m, r):
+    return (C @ r) / abs(float(nv @ r))
+
+
+def _mlstm_not_delayed(k_all, v_all, P, S, W, D):
+    x_all = orc.head_input(k_all, v_all)
+    n = len(x_all)
+    states = orc.mlstm_states(x_all, P)
+    s = np.full(n, np.nan)
+    for u in range(S, n):
+        if u + W + D >= n:
+            break
+        C, nv, m = states[u]
+        s[u] = float(P.wo @ orc.silu(orc.mlstm_readout(C, nv, m, orc.hedgehog(P.wq @ x_all[u])))) + P.bo
+    return orc.ranking_score(s)
+
+
 MUTATIONS = {
     "tie_goes_to_newer": ("rank_key", _ties_to_newer),
     "eligible_off_by_one": ("eligible_positions", _elig_off_by_one),
@@ -154,6 +196,10 @@ MUTATIONS = {
     "cutoff_records_last_kept_step": ("running_cutoffs", _cutoff_last_kept),
     "prefill_attends_before_update": ("prefill_attention", _prefill_stale_topk),
     "prefill_lse_unscaled": ("attention_lse", _lse_unscaled),
+    "hedgehog_positive_only": ("hedgehog", _hedgehog_positive_only),
+    "mlstm_forget_gate_not_in_log_space": ("mlstm_states", _mlstm_forget_not_log),
+    "mlstm_normaliser_without_floor": ("mlstm_readout", _mlstm_readout_no_floor),
+    "mlstm_readout_not_delayed": ("unit_scores_mlstm", _mlstm_not_delayed),
 }
 
 
