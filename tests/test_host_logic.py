@@ -48,3 +48,19 @@ def test_decode_work_split(units, tpu):
     random.seed(units * 1000 + tpu)
     for launched in (8, 9 * 8, 148 * 8, 1184):
         _check(units, tpu, launched)
+
+
+def test_prefill_attention_flop_count():
+    """bench.py's flop count of one prefill-attention call: 4 d flops per
+    attended (position, query head) pair, position q attending min(q + 1, B + D)
+    tokens; checked against the sum written out for a small shape and the
+    closed form sum_{q<B'} (q + 1) + (n - B') B' for the target shape."""
+    import bench
+    import kvpop_workloads as wl
+    small = wl.TINY.replace(prefill=30)          # B + D = 4 + 16 + 44 = 64 > 30: every position dense
+    assert bench.prefill_attention_flops(small) == 4.0 * 64 * sum(q + 1 for q in range(30)) * 4 * 1
+    w = wl.QWEN3_4B_CR88.replace(n_layers=1)
+    Bp = w.sinks + w.window + w.delay + w.topk
+    n = w.prefill
+    pairs = Bp * (Bp + 1) // 2 + (n - Bp) * Bp
+    assert bench.prefill_attention_flops(w) == 4.0 * w.head_dim * pairs * w.n_q_heads * w.batch
