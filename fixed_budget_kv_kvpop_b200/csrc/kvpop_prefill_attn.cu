@@ -27,7 +27,13 @@
 // masking each (query, key) pair by the rule above.  bf16 inputs take the
 // tensor-core kernel instead (sparse_attn_mma_kernel: 128 rows per CTA,
 // m16n8k16 bf16 MMAs with fp32 accumulation, keys gathered by cp.async);
-// fp32 inputs keep the FMA kernel so that no product is rounded.
+// fp32 inputs keep the FMA kernel so that they are never rounded to a
+// tensor-core input type.
+//
+// Cache build.  The tokens whose cutoff is "never" are the running top-k at
+// the last prompt position; place_kept_kernel writes them to the long-range
+// slots in ascending position order (what a one-chunk prefill places), so a
+// whole-prompt prefill and its attention outputs share one scoring pass.
 #include "kvpop_prefill_attn.cuh"
 
 namespace kvpop {
