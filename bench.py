@@ -109,6 +109,34 @@ TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024",
                    "dram_bytes": 279_369_472 + 5_617_920, "algorithmic_bytes": 274_452_512}
 
 
+# ncu capture of the prefill attention's tensor-core kernel (the small case of
+# profiles/sparse_attn_mma_kernel_cr88_b4_full.md: 4 rows x 8 KV heads =
+# 32 units, prompt 8192): DRAM read + write of one launch.  Traffic grows with
+# the units a launch covers (every unit reads its own q, k, v and writes its
+# own output), so a launch of U units moves dram_bytes * U / 32.
+PA_TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024", "units": 32,
+                      "kernel_sha256": "1f1c1014d2f6de3dc158726e42a2f3ebf1274cc7b39c2c482fff3bf644f079bf",
+                      "dram_bytes": 403_806_208 + 238_022_144}
+
+
+def _strip_code(src: str) -> str:
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(ln.strip() for ln in src.splitlines() if ln.strip())
+
+
+def mma_kernel_sha256() -> str:
+    """sha256 of the prefill attention's tensor-core kernel (its section of
+    kvpop_prefill_attn.cu, comments and blank lines removed)."""
+    import hashlib
+    with open(os.path.join(ROOT, "fixed_budget_kv_kvpop_b200", "csrc", "kvpop_prefill_attn.cu")) as fh:
+        src = fh.read()
+    a = src.index("bf16 attention on the tensor cores")
+    b = src.index("int launch_attn_f32(")
+    return hashlib.sha256(_strip_code(src[a:b]).encode()).hexdigest()
+
+
 def kernel_sources_sha256() -> str:
     """sha256 of the decode kernel's code: its two source files with comments
     and blank lines removed (a comment edit does not change the kernel)."""
@@ -639,6 +667,13 @@ def run_prefill_attention(args, w, torch):
     except Exception:
         peak, kind = 1590.0, "fallback"
     achieved = flops / (ms / 1e3) / 1e12
+    cap = PA_TRAFFIC_CAPTURE
+    units = one.batch * one.n_kv_heads
+    traffic = None
+    if w.name.startswith(cap["workload"]) and mma_kernel_sha256() == cap["kernel_sha256"]:
+        traffic = cap["dram_bytes"] * units / cap["units"]
+    esize = 2 if one.dtype == "bf16" else 4
+    io_bytes = (2 * q.numel() + 2 * k.numel()) * esize   # q, k, v read; output written
     res = {
         "metric": PA_METRIC, "value": one.batch * n / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
@@ -649,9 +684,11 @@ def run_prefill_attention(args, w, torch):
                    "l2": "no flush: q, k, v (%.1f GB) larger than L2" % ((q.numel() + 2 * k.numel()) * 2 / 1e9)},
         "roofline": {"kernel": "whole call: prompt scorer + cutoff_kernel + sparse_attn_mma_kernel",
                      "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "flops_per_call": flops, "peak_kind": kind,
+                     "frac": achieved / peak, "traffic": traffic, "flops_per_call": flops, "peak_kind": kind,
+                     "attention_io_bytes": io_bytes,
                      "note": "flops of the attention alone over the time of the whole call; the launch list "
-                             "under profiles/ gives each kernel's share"},
+                             "under profiles/ gives each kernel's share; traffic = the attention kernel's DRAM "
+                             "bytes per launch from an ncu capture of 32 units, scaled by units"},
         "gpu_launches": 3 * steps,
         "clocks": clocks,
     }
