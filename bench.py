@@ -602,6 +602,7 @@ def oracle_prefill_rows_per_s(w: wl.Workload, seconds: float):
     s = orc.unit_scores_mlp(kk, vv, w1[0, 0].double().numpy(), b1[0, 0].double().numpy(),
                             w2[0, 0].double().numpy(), float(b2[0, 0]))
     rows = np.linspace(0, w.prefill - 1, 2048).astype(int)
+    lim = cpu_threads_limit()   # one core, as the line's "cores" says
     t0 = time.perf_counter()
     done = 0
     for qp in rows:
@@ -612,6 +613,8 @@ def oracle_prefill_rows_per_s(w: wl.Workload, seconds: float):
         if time.perf_counter() - t0 > seconds:
             break
     dt = time.perf_counter() - t0
+    if lim is not None and hasattr(lim, "unregister"):
+        lim.unregister()
     tok_s = done / dt / w.n_kv_heads
     desc = (f"{done} prompt positions of one (batch row, KV head) unit of the {w.name} shape, spread evenly "
             f"over the {w.prefill}-token prompt, scores untimed ({dt:.1f} s); one prompt token = "
