@@ -2,7 +2,9 @@
 with the CPU oracle: running cutoffs bit-exact, outputs and log-normalisers
 within the dtype's tolerance, on seeded inputs of several tiles with ragged
 tails, and the edge cases of the mask (nothing eligible, K = 0, K covering the
-prompt, one token)."""
+prompt, one token); and the fused whole-prompt call
+(kvpop_prefill_with_attention) bit for bit against kvpop_prefill followed by
+kvpop_prefill_attention."""
 import numpy as np
 import pytest
 import torch

@@ -64,3 +64,16 @@ def test_prefill_attention_flop_count():
     n = w.prefill
     pairs = Bp * (Bp + 1) // 2 + (n - Bp) * Bp
     assert bench.prefill_attention_flops(w) == 4.0 * w.head_dim * pairs * w.n_q_heads * w.batch
+
+
+def test_bench_arguments(monkeypatch):
+    """Default steps stay unset until the chosen path fills them in (200 decode
+    steps, 10 prefill-attention calls); the prefill-attention options parse."""
+    import sys
+    import bench
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    a = bench.parse_args()
+    assert a.path == "decode" and a.steps is None and a.pa_batch == 0
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--path", "prefill-attention", "--pa-batch", "4", "--steps", "2"])
+    a = bench.parse_args()
+    assert a.path == "prefill-attention" and a.pa_batch == 4 and a.steps == 2
