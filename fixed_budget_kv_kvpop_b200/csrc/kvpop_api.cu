@@ -372,6 +372,7 @@ int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const
   if (!q || !k || !v || !out || !workspace) return KVPOP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
     return KVPOP_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return KVPOP_ERR_INVALID_ARG;
   const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
   if (ext && !ext_scores) return KVPOP_ERR_INVALID_ARG;
   const LayerArgs a = layer_args(h, layer);
@@ -394,6 +395,7 @@ int kvpop_prefill_with_attention(kvpop_handle* h, int32_t layer, const void* q, 
   if (!q || !k || !v || !out || !workspace) return KVPOP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
     return KVPOP_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return KVPOP_ERR_INVALID_ARG;
   const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
   if (ext && !ext_scores) return KVPOP_ERR_INVALID_ARG;
   const LayerArgs a = layer_args(h, layer);

@@ -229,7 +229,8 @@ int kvpop_decode_attend(kvpop_handle* h, int32_t layer, const void* q, void* out
  * [b][Hq][n_tokens] receiving each row's natural-log softmax normaliser
  * log sum_j exp(q.k_j / sqrt(d)), or NULL; ext_scores: device fp32
  * [b][Hkv][n_tokens] (required with KVPOP_FLAG_EXTERNAL_SCORES, ignored
- * otherwise).  q, k, v, out and workspace must be 16-byte aligned.
+ * otherwise).  q, k, v, out and workspace must be 16-byte aligned, lse 4-byte
+ * aligned.
  * workspace: caller-owned device scratch of at least
  * kvpop_prefill_attention_workspace_bytes(n_tokens) bytes; after the call its
  * first units * n_tokens int32 hold the cutoffs c_j ([units][n_tokens]).
