@@ -442,6 +442,30 @@ def pin_mlstm_scores_drive_the_running_topk():
     res = orc.run_unit(k, v, q, s, S, W, D, K, P_len)
     assert all(len(t) == min(K, max(0, P_len + i - W - D - S + 1)) for i, t in enumerate(res.topk_sets[1:]))
 
+
+def pin_mlstm_readout_hand_example():
+    """A hand-worked delayed readout (golden/mlstm_readout_hand_example.json):
+    with one-dimensional Hedgehog projections every feature vector is [1, 1],
+    so the readout h is a decayed average of the values and the score head
+    w_o . SiLU(h) + b_o can be checked by eye (§E.4 Delayed Readout)."""
+    g = _load("mlstm_readout_hand_example.json")
+    P = orc.MlstmParams(wq=np.array(g["wq"]), wk=np.array(g["wk"]), wv=np.array(g["wv"]), wi=np.array(g["wi"]),
+                        bi=g["bi"], wf=np.array(g["wf"]), bf=g["bf"], wo=np.array(g["wo"]), bo=g["bo"])
+    k = np.array(g["k"])[:, None]
+    v = np.array(g["v"])[:, None]
+    x = orc.head_input(k, v)
+    states = orc.mlstm_states(x, P)
+    for u, h_ref in enumerate(g["h"]):
+        q = u + g["W"] + g["D"]
+        h = orc.mlstm_readout(*states[q], orc.hedgehog(P.wq @ x[u]))
+        np.testing.assert_allclose(h, h_ref, rtol=0, atol=1e-12)
+    s = orc.unit_scores_mlstm(k, v, P, g["S"], g["W"], g["D"])
+    for u, ref in enumerate(g["scores"]):
+        if ref is None:
+            assert math.isnan(s[u]), (u, s[u])
+        else:
+            assert s[u] == float(np.float32(ref)), (u, s[u], ref)
+
 ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1,
             pin_prefill_chunk_placement, pin_dense_when_budget_covers_context,
             pin_budget_invariant_and_structure, pin_softmax_rows_sum_to_one,
@@ -452,4 +476,4 @@ ALL_PINS = [pin_mlp_hand_example, pin_retention_trace_d0, pin_retention_trace_d1
             pin_running_cutoffs_are_intervals, pin_prefill_attention_dense_when_budget_covers_context,
             pin_prefill_attention_matches_slot_simulator, pin_hedgehog_feature_map,
             pin_mlstm_stabilised_equals_closed_form, pin_mlstm_delayed_readout_is_causal_and_forward_looking,
-            pin_mlstm_scores_drive_the_running_topk]
+            pin_mlstm_scores_drive_the_running_topk, pin_mlstm_readout_hand_example]

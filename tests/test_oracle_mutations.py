@@ -175,6 +175,23 @@ def _mlstm_not_delayed(k_all, v_all, P, S, W, D):
     return orc.ranking_score(s)
 
 
+def _sigmoid_for_silu(x):
+    x = np.asarray(x, np.float64)
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _identity_for_silu(x):
+    return np.asarray(x, np.float64)
+
+
+def _mlstm_score_drops_bias(k_all, v_all, P, S, W, D):
+    import dataclasses
+    return _ORIG_MLSTM_SCORES(k_all, v_all, dataclasses.replace(P, bo=0.0), S, W, D)
+
+
+_ORIG_MLSTM_SCORES = orc.unit_scores_mlstm
+
+
 MUTATIONS = {
     "tie_goes_to_newer": ("rank_key", _ties_to_newer),
     "eligible_off_by_one": ("eligible_positions", _elig_off_by_one),
@@ -200,6 +217,9 @@ MUTATIONS = {
     "mlstm_forget_gate_not_in_log_space": ("mlstm_states", _mlstm_forget_not_log),
     "mlstm_normaliser_without_floor": ("mlstm_readout", _mlstm_readout_no_floor),
     "mlstm_readout_not_delayed": ("unit_scores_mlstm", _mlstm_not_delayed),
+    "mlstm_score_head_sigmoid_for_silu": ("silu", _sigmoid_for_silu),
+    "mlstm_score_head_identity_for_silu": ("silu", _identity_for_silu),
+    "mlstm_score_head_drops_bias": ("unit_scores_mlstm", _mlstm_score_drops_bias),
 }
 
 
