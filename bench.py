@@ -51,7 +51,13 @@ def parse_args():
     ap.add_argument("--pa-batch", type=int, default=0,
                     help="prefill-attention path: batch rows (default: the workload's; smaller for profiling)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cr88")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=None, help="e2e timed steps (default: --steps)")
+    ap.add_argument("--e2e-warmup", type=int, default=None, help="e2e warm-up steps (default: --warmup)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations (75%% compression, 8B with delayed scoring) and the sweep")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the bandwidth sweep")
+    ap.add_argument("--cpu-workers", type=int, default=0,
+                    help="processes of the parallel oracle leg (default: min(host CPUs, 16))")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -296,6 +302,50 @@ def oracle_tokens_per_s(w: wl.Workload, seconds: float):
     return tok_s, desc
 
 
+def _oracle_worker(w, seed, seconds, max_steps, barrier, results):
+    """One process of the parallel oracle leg: one unit of the workload's
+    shape, prefilled (untimed), then decode steps for `seconds` after every
+    worker is ready."""
+    import threadpoolctl
+    with threadpoolctl.threadpool_limits(limits=1):
+        sample = OracleSample(w, 1, max_steps, seed=seed)
+        barrier.wait(timeout=600)
+        t0 = time.perf_counter()
+        steps = 0
+        while steps < max_steps and (time.perf_counter() - t0 < seconds or steps < 2):
+            sample.step()
+            steps += 1
+        results.put((steps, time.perf_counter() - t0))
+
+
+def oracle_parallel_tokens_per_s(w: wl.Workload, seconds: float, workers: int):
+    """The oracle on `workers` host cores at once: one process per core
+    (started with spawn, safe after CUDA initialisation), each stepping its
+    own unit of the workload's shape.  Units are independent, so the
+    throughput is the sum of the processes' unit-step rates.  Returns
+    (tokens/s, cores used, description)."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    barrier = ctx.Barrier(workers)
+    results = ctx.Queue()
+    max_steps = 4000
+    procs = [ctx.Process(target=_oracle_worker, args=(w, 100 + i, seconds, max_steps, barrier, results))
+             for i in range(workers)]
+    for p_ in procs:
+        p_.start()
+    got = [results.get(timeout=900) for _ in procs]
+    for p_ in procs:
+        p_.join(timeout=60)
+    units_per_token = w.n_layers * w.n_kv_heads
+    rate = sum(st / dt for st, dt in got)          # unit-steps per second, all processes together
+    steps = sum(st for st, _ in got)
+    mean_dt = sum(dt for _, dt in got) / len(got)
+    desc = (f"{workers} processes on {workers} host cores, each one (batch row, KV head) unit of the {w.name} "
+            f"shape (prompt {w.prefill} prefilled untimed), stepped for {mean_dt:.1f} s on average after all "
+            f"were ready ({steps} unit-steps in all); one decode token = {units_per_token} unit-steps")
+    return rate / units_per_token, workers, desc
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return
@@ -348,8 +398,11 @@ def replica_throughput(batch: int, steps: int, world: int, elapsed_ms: float) ->
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def build_cache(w: wl.Workload, torch, log_decay=None):
+def build_cache(w: wl.Workload, torch, log_decay=None, prompt=None):
+    """A cache for every layer of `w`, each layer prefilled with `prompt`
+    tokens (default: the workload's prompt) in one kvpop_prefill call."""
     import fixed_budget_kv_kvpop_b200 as kp
+    P = w.prefill if prompt is None else prompt
     weights = tuple(t.cuda() for t in wl.scorer_weights(w))
     w1, b1, w2, b2 = weights
     decay = None
@@ -359,13 +412,13 @@ def build_cache(w: wl.Workload, torch, log_decay=None):
     cfg = kp.make_config(batch=w.batch, n_layers=w.n_layers, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                          head_dim=w.head_dim, sinks=w.sinks, window=w.window, topk=w.topk, delay=w.delay,
                          ref_context=w.prefill, compression_ratio=w.compression_ratio,
-                         max_prefill_chunk=w.prefill, dtype=w.dtype, scorer_hidden=w.scorer_hidden,
+                         max_prefill_chunk=P, dtype=w.dtype, scorer_hidden=w.scorer_hidden,
                          w1=w1, b1=b1, w2=w2, b2=b2, log_decay=decay)
     cache = kp.KVPopCache(cfg, keepalive=weights)
     stream = torch.cuda.current_stream()
     prefill_ms = []
     for layer in range(w.n_layers):
-        k, v = wl.prompt_kv(w, layer, device="cuda")
+        k, v = wl.prompt_kv(w, layer, n_tokens=P, device="cuda")
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         cache.prefill(layer, k, v, stream=stream)
@@ -390,20 +443,31 @@ def prefill_summary(w: wl.Workload, prefill_ms):
                     "flops by the whole prefill time (select, move and write included)"}
 
 
-def run_gpu(args, w, rank, world, torch):
+def smi_index(torch):
     dev = torch.cuda.current_device()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[dev])
+        except (ValueError, IndexError):
+            return dev
+    return dev
+
+
+def time_decode(w, cache, steps, warmup, torch, world, input_sets=32, graph=False):
+    """Times `steps` decode steps (every layer, every batch row) after
+    `warmup` untimed ones, on the current stream, with CUDA events around the
+    launches and nvidia-smi sampling the clocks; the time is the max over
+    ranks.  Returns the measurement as a dict."""
     stream = torch.cuda.current_stream()
-    t_setup = time.perf_counter()
-    cache, prefill_ms = build_cache(w, torch, args.log_decay)
-    NI = max(1, min(args.input_sets, args.steps + args.warmup))
+    L = w.n_layers
+    NI = max(1, min(input_sets, steps + warmup))
     qs, ks, vs = [], [], []
-    for layer in range(w.n_layers):
+    for layer in range(L):
         q, k, v = wl.decode_inputs_batched(w, layer, NI, device="cuda")
         qs.append(q); ks.append(k); vs.append(v)
-    outs = [torch.empty_like(qs[0][0]) for _ in range(w.n_layers)]
+    outs = [torch.empty_like(qs[0][0]) for _ in range(L)]
     torch.cuda.synchronize()
-    setup_s = time.perf_counter() - t_setup
-    L = w.n_layers
 
     def launch_step(j, st):
         for layer in range(L):
@@ -417,10 +481,10 @@ def run_gpu(args, w, rank, world, torch):
         else:
             launch_step(i % NI, stream)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         one_step(i)
     torch.cuda.synchronize()
-    if args.graph:
+    if graph:
         # Capture (not run) one step per input set.  Each replay advances the
         # layers' device-side counters like an eager step; only the library's
         # host mirrors (used for argument validation) run ahead.
@@ -435,25 +499,17 @@ def run_gpu(args, w, rank, world, torch):
     st, bits = cache.get_error()
     if st != 0:
         raise RuntimeError(f"device error after warm-up: status {st} bits {bits}")
-
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    smi_idx = dev
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    if vis:
-        try:
-            smi_idx = int(vis.split(",")[dev])
-        except ValueError:
-            smi_idx = dev
-    sampler = ClockSampler(smi_idx)
+    sampler = ClockSampler(smi_index(torch))
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
     start.record(stream)
-    for s in range(args.steps):
-        one_step(args.warmup + s)
+    for s in range(steps):
+        one_step(warmup + s)
     end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -462,50 +518,122 @@ def run_gpu(args, w, rank, world, torch):
     if st != 0:
         raise RuntimeError(f"device error in timed region: status {st} bits {bits}")
     elapsed_ms = max_over_ranks(elapsed_ms, world, torch, "cuda")
-    value = replica_throughput(w.batch, args.steps, world, elapsed_ms)
     peak, peak_kind = measured_peaks()
     sbytes = step_bytes(w)
-    step_gbs = sbytes * args.steps / (elapsed_ms / 1e3) / 1e9
-    abytes = sbytes // L   # one fused launch = one layer's share of the step
+    step_gbs = sbytes * steps / (elapsed_ms / 1e3) / 1e9
     # The timed region holds nothing but these launches, back to back on one
     # stream (no event between them, so programmatic dependent launch can
     # overlap one launch's tail with the next one's prologue): the average
     # launch duration is the region's duration over the launch count.
-    n_launches = L * args.steps
-    attn_mean_ms = elapsed_ms / n_launches
-    attn_gbs = abytes / (attn_mean_ms / 1e3) / 1e9
+    n_launches = L * steps
+    del graphs
+    return {"elapsed_ms": elapsed_ms, "ms_per_step": elapsed_ms / steps,
+            "tokens_per_s": replica_throughput(w.batch, steps, world, elapsed_ms),
+            "step_bytes": sbytes, "achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
+            "frac_of_8tbs": step_gbs / 8000.0, "peak_kind": peak_kind,
+            "mean_launch_us": elapsed_ms / n_launches * 1e3, "launches": n_launches,
+            "bytes_per_launch": sbytes // L, "clocks": clocks, "input_sets": len(graphs) if graph else NI}
+
+
+def run_gpu(args, w, rank, world, torch):
+    t_setup = time.perf_counter()
+    cache, prefill_ms = build_cache(w, torch, args.log_decay)
+    torch.cuda.synchronize()
+    setup_s = time.perf_counter() - t_setup
+    m = time_decode(w, cache, args.steps, args.warmup, torch, world, args.input_sets, args.graph)
+    L = w.n_layers
+    abytes = m["bytes_per_launch"]
+    attn_gbs = abytes / (m["mean_launch_us"] / 1e6) / 1e9
 
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, cache, torch, world)
 
     res = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": m["tokens_per_s"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "layers": w.n_layers, "q_heads": w.n_q_heads,
                    "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "sinks": w.sinks, "window": w.window,
                    "topk": w.topk, "delay": w.delay, "budget": w.budget, "prompt": w.prefill,
                    "compression": round(w.compression_ratio, 4), "parallelism": f"replicas x{world}",
                    "l2": "no flush: inputs (cache %.1f GB) larger than L2" % (w.n_layers * attention_bytes(w) / 1e9),
-                   "input_sets": len(graphs) if graphs else NI, "log_decay": args.log_decay,
-                   "cuda_graph": bool(graphs)},
-        "hbm": {"step_bytes": sbytes, "achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
-                "frac_of_8tbs": step_gbs / 8000.0, "peak_kind": peak_kind},
+                   "input_sets": m["input_sets"], "log_decay": args.log_decay, "cuda_graph": bool(args.graph)},
+        "hbm": {k: m[k] for k in ("step_bytes", "achieved_gbs", "peak_gbs", "frac", "frac_of_8tbs", "peak_kind")},
         "roofline": {"kernel": "decode_kernel (fused append + attend, one launch per layer)",
                      "bound": "hbm", "achieved": attn_gbs,
-                     "peak": peak, "unit": "GB/s", "frac": attn_gbs / peak,
+                     "peak": m["peak_gbs"], "unit": "GB/s", "frac": attn_gbs / m["peak_gbs"],
                      "traffic": measured_traffic(w, abytes),
-                     "bytes_per_launch": abytes, "mean_launch_us": attn_mean_ms * 1e3,
-                     "launches": n_launches, "peak_kind": peak_kind},
-        "gpu_launches": n_launches,
+                     "bytes_per_launch": abytes, "mean_launch_us": m["mean_launch_us"],
+                     "launches": m["launches"], "peak_kind": m["peak_kind"]},
+        "gpu_launches": m["launches"],
         "prefill": prefill_summary(w, prefill_ms),
-        "clocks": clocks,
+        "clocks": m["clocks"],
         "setup_s": setup_s,
     }
     if e2e is not None:
         res["e2e"] = e2e
+    del cache
+    torch.cuda.empty_cache()
     return res
+
+
+def other_config(args, w, torch, world, prompt=None, note=None):
+    """Decode throughput of another configuration, timed like the headline
+    (same steps and warm-up; no e2e or CPU leg)."""
+    t0 = time.perf_counter()
+    cache, prefill_ms = build_cache(w, torch, None, prompt)
+    m = time_decode(w, cache, args.steps, args.warmup, torch, world, args.input_sets)
+    del cache
+    torch.cuda.empty_cache()
+    out = {"workload": w.name, "batch": w.batch, "layers": w.n_layers, "budget": w.budget, "delay": w.delay,
+           "prompt": w.prefill if prompt is None else prompt, "compression": round(w.compression_ratio, 4),
+           "tokens_per_s": m["tokens_per_s"], "ms_per_step": m["ms_per_step"],
+           "achieved_gbs": m["achieved_gbs"], "frac": m["frac"], "frac_of_8tbs": m["frac_of_8tbs"],
+           "mean_launch_us": m["mean_launch_us"], "bytes_per_launch": m["bytes_per_launch"],
+           "launches": m["launches"], "clocks": m["clocks"], "prefill_ms_per_layer": statistics.median(prefill_ms),
+           "wall_s": time.perf_counter() - t0}
+    if note:
+        out["note"] = note
+    return out
+
+
+SWEEP_CACHE_CAP = 80e9   # bytes of cache a sweep point may hold (HBM is 180 GB)
+
+
+def sweep_plan(budgets=wl.SWEEP_BUDGETS, batches=wl.SWEEP_BATCHES, cap=SWEEP_CACHE_CAP):
+    """The bandwidth sweep on the Qwen3-8B shape: per (budget, batch) the
+    workload, the layers it runs (36, or fewer when the 36-layer cache would
+    exceed `cap`), and the prompt it prefills (budget + 256 tokens: a decode
+    step reads the whole bounded cache, whose size does not depend on how
+    long the prompt was once the long-range slots are full)."""
+    plan = []
+    for B in budgets:
+        for b in batches:
+            w = wl.sweep_point(B, b)
+            per_layer = attention_bytes(w)
+            layers = max(1, min(w.n_layers, int(cap // per_layer)))
+            plan.append({"budget": B, "batch": b, "workload": w.replace(n_layers=layers), "layers": layers,
+                         "full_cache_gb": per_layer * w.n_layers / 1e9, "prompt": B + 256})
+    return plan
+
+
+def run_sweep(args, torch, world):
+    points = []
+    for pt in sweep_plan():
+        w = pt["workload"]
+        notes = [f"prompt shortened from {w.prefill} to {pt['prompt']} tokens: the decode step reads the full "
+                 "bounded cache either way"]
+        if pt["layers"] < 36:
+            notes.append(f"layers reduced to {pt['layers']} of 36: the 36-layer cache is "
+                         f"{pt['full_cache_gb']:.0f} GB" + (", more than the 180 GB of HBM"
+                                                             if pt["full_cache_gb"] > 180 else ""))
+        r = other_config(args, w, torch, world, prompt=pt["prompt"], note="; ".join(notes))
+        r.update({"budget": pt["budget"], "batch": pt["batch"], "layers_full": 36,
+                  "layers_reduced": pt["layers"] < 36})
+        points.append(r)
+    return {"shape": "Qwen3-8B (36 layers, 32 q / 8 kv heads, d 128, bf16), 4 sinks, window 128, K = B - 132, D 0",
+            "points": points}
 
 
 def run_e2e(args, w, cache, torch, world):
@@ -513,7 +641,9 @@ def run_e2e(args, w, cache, torch, world):
     memory: each step copies q/k/v of all layers host->device, runs the step,
     and copies the outputs device->host, pipelined over two buffers and three
     streams (copy-in, compute, copy-out)."""
-    L, K = w.n_layers, max(1, args.e2e_steps)
+    L = w.n_layers
+    K = max(1, args.e2e_steps if args.e2e_steps is not None else args.steps)
+    WU = max(1, args.e2e_warmup if args.e2e_warmup is not None else args.warmup)
     NI = 4
     hq = [torch.empty((L,) + (w.batch, w.n_q_heads, w.head_dim), dtype=w.torch_dtype()).pin_memory()
           for _ in range(NI)]
@@ -558,12 +688,12 @@ def run_e2e(args, w, cache, torch, world):
         first[b] = False
 
     first = [True, True]
-    for s in range(3):
+    for s in range(WU):
         step(s, first)
     torch.cuda.synchronize()
     start.record(s_in)
     for s in range(K):
-        step(3 + s, first)
+        step(WU + s, first)
     end.record(s_out)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
@@ -572,7 +702,10 @@ def run_e2e(args, w, cache, torch, world):
     h2d = L * w.batch * (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim * es
     d2h = L * w.batch * w.n_q_heads * w.head_dim * es
     return {"value": replica_throughput(w.batch, K, world, ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": K, "ms_per_step": ms / K}
+            "d2h_bytes_per_step": d2h, "steps": K, "warmup": WU, "ms_per_step": ms / K,
+            "note": "same step count and warm-up as the device-timed region; the copies of step s+1 and s-1 "
+                    "overlap step s's launches (two buffers, three streams), so e2e can come out at or even "
+                    "slightly below the device-only step time"}
 
 
 PA_METRIC = "prefill attention tokens/s under the running top-k mask (one layer: scores, cutoffs, attention)"
@@ -684,7 +817,7 @@ def run_prefill_attention(args, w, torch):
         "config": {"workload": one.name, "batch": one.batch, "layers": 1, "q_heads": one.n_q_heads,
                    "kv_heads": one.n_kv_heads, "head_dim": one.head_dim, "sinks": one.sinks,
                    "window": one.window, "topk": one.topk, "delay": one.delay, "prompt": n,
-                   "l2": "no flush: q, k, v (%.1f GB) larger than L2" % ((q.numel() + 2 * k.numel()) * 2 / 1e9)},
+                   "l2": "no flush: q, k, v (%.1f GB) larger than L2" % ((q.numel() + 2 * k.numel()) * esize / 1e9)},
         "roofline": {"kernel": "whole call: prompt scorer + cutoff_kernel + sparse_attn_mma_kernel",
                      "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "flops_per_call": flops, "peak_kind": kind,
@@ -729,10 +862,27 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
         res = run_gpu(args, w, rank, world, torch)
+        # The other configurations of the metric, timed the same way (single
+        # GPU runs only: under torchrun every rank would have to repeat them).
+        if world == 1 and not args.no_extras:
+            extras = {}
+            for key in ("cr75", "cr88", "8b_d32"):
+                if WORKLOADS[key].name != w.name and not args.layers:
+                    extras[key] = other_config(args, WORKLOADS[key], torch, world)
+            res["configs"] = extras
+            if not args.no_sweep:
+                res["sweep"] = run_sweep(args, torch, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            v, desc = oracle_tokens_per_s(w, args.cpu_seconds)
-            res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc,
-                                   "host": host_info()}
+            v1, desc1 = oracle_tokens_per_s(w, args.cpu_seconds)
+            single = {"value": v1, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc1}
+            workers = args.cpu_workers or max(1, min(os.cpu_count() or 1, 16))
+            try:
+                vp, cores, descp = oracle_parallel_tokens_per_s(w, args.cpu_seconds, workers)
+                res["cpu_baseline"] = {"value": vp, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                       "sample": descp, "single_core": single, "host": host_info()}
+            except Exception as exc:   # the single-core figure still stands
+                single.update({"host": host_info(), "parallel_leg_failed": repr(exc)[:200]})
+                res["cpu_baseline"] = single
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -133,6 +133,49 @@ def _stream_ptr(stream) -> Optional[int]:
     return stream.cuda_stream or None
 
 
+_DTYPE_NAMES = {"f32": KVPOP_DTYPE_F32, "float32": KVPOP_DTYPE_F32, "fp32": KVPOP_DTYPE_F32,
+                "bf16": KVPOP_DTYPE_BF16, "bfloat16": KVPOP_DTYPE_BF16}
+
+
+def dtype_code(dtype) -> int:
+    """KVPOP_DTYPE_* of an element-type name ('f32', 'float32', 'fp32',
+    'bf16', 'bfloat16') or of torch.float32 / torch.bfloat16; anything else
+    raises ValueError."""
+    if isinstance(dtype, str):
+        if dtype in _DTYPE_NAMES:
+            return _DTYPE_NAMES[dtype]
+    else:
+        import torch
+        if dtype == torch.float32:
+            return KVPOP_DTYPE_F32
+        if dtype == torch.bfloat16:
+            return KVPOP_DTYPE_BF16
+    raise ValueError(f"unsupported element type {dtype!r}: use one of {sorted(_DTYPE_NAMES)}")
+
+
+def _torch_dtype(code: int):
+    import torch
+    return torch.float32 if code == KVPOP_DTYPE_F32 else torch.bfloat16
+
+
+def check_tensor(t, name: str, shape, dtype, device) -> None:
+    """Raises ValueError unless `t` is a contiguous CUDA tensor on `device`
+    (a torch.device) with exactly `shape` and `dtype`.  The C ABI sees only
+    raw pointers, so every tensor is checked here before its address is
+    passed on."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device.type != "cuda" or t.device != device:
+        raise ValueError(f"{name}: on {t.device}, the cache lives on {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
 def make_config(*, batch, n_layers, n_q_heads, n_kv_heads, head_dim, sinks, window, topk, delay=0,
                 ref_context=0, compression_ratio=0.0, max_context=None, max_prefill_chunk=0,
                 dtype="bf16", scorer_hidden=64, w1=None, b1=None, w2=None, b2=None,
@@ -147,7 +190,7 @@ def make_config(*, batch, n_layers, n_q_heads, n_kv_heads, head_dim, sinks, wind
     c.sinks, c.window, c.topk, c.delay = sinks, window, topk, delay
     c.ref_context, c.compression_ratio = ref_context, compression_ratio
     c.max_context, c.max_prefill_chunk = max_context, max_prefill_chunk
-    c.dtype = KVPOP_DTYPE_F32 if dtype in ("f32", "float32") else KVPOP_DTYPE_BF16
+    c.dtype = dtype_code(dtype)
     c.scorer_hidden = scorer_hidden
     c.w1, c.b1, c.w2, c.b2 = _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)
     c.flags = (KVPOP_FLAG_EXTERNAL_SCORES if external_scores else 0) | (KVPOP_FLAG_DEBUG_CHECKS if debug_checks else 0)
@@ -179,6 +222,20 @@ class KVPopCache:
         self.handle = ctypes.c_void_p()
         _check(lib.kvpop_create(ctypes.byref(cfg), ctypes.c_void_p(base + self._off), self.nbytes,
                                 ctypes.byref(self.handle)), "kvpop_create")
+        self.device = self.buffer.device
+        self.dtype = _torch_dtype(cfg.dtype)
+
+    # -- argument checks (shapes from include/kvpop.h) --
+    def _elems(self, name, t, shape):
+        check_tensor(t, name, shape, self.dtype, self.device)
+
+    def _f32(self, name, t, shape):
+        import torch
+        check_tensor(t, name, shape, torch.float32, self.device)
+
+    def _dims(self):
+        c = self.cfg
+        return c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim
 
     def __del__(self, _lib=lib):
         h = getattr(self, "handle", None)
@@ -188,10 +245,26 @@ class KVPopCache:
 
     def prefill(self, layer: int, k, v, ext_scores=None, stream=None):
         n = int(k.shape[2]) if k is not None else 0
+        if k is not None or v is not None:
+            b, _, hkv, d = self._dims()
+            self._elems("k", k, (b, hkv, n, d))
+            self._elems("v", v, (b, hkv, n, d))
+            if ext_scores is not None:
+                self._f32("ext_scores", ext_scores, (b, hkv, n))
         _check(lib.kvpop_prefill(self.handle, layer, _ptr(k), _ptr(v), n, _ptr(ext_scores),
                                  _stream_ptr(stream)), "kvpop_prefill")
 
+    def _check_step(self, q, k_new, v_new, out, ext_score):
+        b, hq, hkv, d = self._dims()
+        self._elems("q", q, (b, hq, d))
+        self._elems("k_new", k_new, (b, hkv, d))
+        self._elems("v_new", v_new, (b, hkv, d))
+        self._elems("out", out, (b, hq, d))
+        if ext_score is not None:
+            self._f32("ext_score", ext_score, (b, hkv))
+
     def decode_step(self, layer: int, q, k_new, v_new, out, ext_score=None, stream=None):
+        self._check_step(q, k_new, v_new, out, ext_score)
         _check(lib.kvpop_decode_step(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                      _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step")
 
@@ -201,6 +274,7 @@ class KVPopCache:
         of this handle's buffer, so the call allocates nothing.  Its first
         call on a device looks up that buffer once (make it before any stream
         capture); calls that overlap on the GPU share the buffer and race."""
+        self._check_step(q, k_new, v_new, out, ext_score)
         _check(lib.kvpop_decode_step_noalloc(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                              _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step_noalloc")
 
@@ -217,7 +291,7 @@ class KVPopCache:
         prefill_attention_workspace_bytes(n) bytes, 16-byte aligned (its first
         units * n int32 are the running cutoffs afterwards).  Does not touch
         the cache."""
-        n = int(k.shape[2])
+        n = self._check_prompt(q, k, v, out, lse, workspace, ext_scores)
         _check(lib.kvpop_prefill_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
                                            _ptr(out), _ptr(lse), _ptr(workspace),
                                            int(workspace.numel() * workspace.element_size()) if workspace is not None
@@ -228,18 +302,42 @@ class KVPopCache:
         """prefill (whole prompt, empty layer) and prefill_attention in one
         call: the prompt is scored once; afterwards the layer holds the cache
         kvpop_prefill would build and is ready for decode steps."""
-        n = int(k.shape[2])
+        n = self._check_prompt(q, k, v, out, lse, workspace, ext_scores)
         _check(lib.kvpop_prefill_with_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
                                                 _ptr(out), _ptr(lse), _ptr(workspace),
                                                 int(workspace.numel() * workspace.element_size())
                                                 if workspace is not None else 0, _stream_ptr(stream)),
                "kvpop_prefill_with_attention")
 
+    def _check_prompt(self, q, k, v, out, lse, workspace, ext_scores) -> int:
+        import torch
+        b, hq, hkv, d = self._dims()
+        n = int(k.shape[2]) if isinstance(k, torch.Tensor) and k.dim() == 4 else -1
+        self._elems("k", k, (b, hkv, n, d))
+        self._elems("v", v, (b, hkv, n, d))
+        self._elems("q", q, (b, hq, n, d))
+        self._elems("out", out, (b, hq, n, d))
+        if lse is not None:
+            self._f32("lse", lse, (b, hq, n))
+        if ext_scores is not None:
+            self._f32("ext_scores", ext_scores, (b, hkv, n))
+        if workspace is not None:
+            check_tensor(workspace, "workspace", (workspace.numel(),), torch.uint8, self.device)
+        return n
+
     def decode_append(self, layer: int, k_new, v_new, ext_score=None, stream=None):
+        b, _, hkv, d = self._dims()
+        self._elems("k_new", k_new, (b, hkv, d))
+        self._elems("v_new", v_new, (b, hkv, d))
+        if ext_score is not None:
+            self._f32("ext_score", ext_score, (b, hkv))
         _check(lib.kvpop_decode_append(self.handle, layer, _ptr(k_new), _ptr(v_new), _ptr(ext_score),
                                        _stream_ptr(stream)), "kvpop_decode_append")
 
     def decode_attend(self, layer: int, q, out, stream=None):
+        b, hq, _, d = self._dims()
+        self._elems("q", q, (b, hq, d))
+        self._elems("out", out, (b, hq, d))
         _check(lib.kvpop_decode_attend(self.handle, layer, _ptr(q), _ptr(out), _stream_ptr(stream)),
                "kvpop_decode_attend")
 

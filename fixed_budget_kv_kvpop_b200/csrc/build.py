@@ -29,18 +29,40 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, out: str = OUT, defines=()) -> str:
+    """Compiles every source to an object in parallel, then links the shared
+    library (each translation unit's device code is self-contained, so no
+    device link step is needed)."""
     if out == OUT and not defines and not force and not _stale():
         return OUT
-    cmd = [NVCC] + FLAGS + ["-D" + d for d in defines] + [os.path.join(HERE, s) for s in SOURCES] + ["-o", out + ".tmp"]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
+    import tempfile
+    from concurrent.futures import ThreadPoolExecutor
+    tmp = tempfile.mkdtemp(prefix="kvpop_build_")
+    extra = ["-D" + d for d in defines] + (["-Xptxas=-v"] if verbose else [])
+    compile_flags = [f for f in FLAGS if f != "-shared"]
+
+    def compile_one(src):
+        obj = os.path.join(tmp, os.path.splitext(src)[0] + ".o")
+        cmd = [NVCC] + compile_flags + extra + ["-c", os.path.join(HERE, src), "-o", obj]
+        return obj, subprocess.run(cmd, capture_output=True, text=True)
+
+    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+        results = list(ex.map(compile_one, SOURCES))
+    for obj, res in results:
+        if res.returncode != 0:
+            sys.stderr.write(res.stdout + res.stderr)
+            raise RuntimeError("nvcc failed building libkvpop.so")
+        if verbose:
+            sys.stderr.write(res.stderr)
+    link = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC"] + \
+        [obj for obj, _ in results] + ["-o", out + ".tmp"]
+    res = subprocess.run(link, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libkvpop.so")
-    if verbose:
-        sys.stderr.write(res.stderr)
+        raise RuntimeError("nvcc failed linking libkvpop.so")
     os.replace(out + ".tmp", out)
+    for obj, _ in results:
+        os.remove(obj)
+    os.rmdir(tmp)
     return out
 
 

@@ -588,16 +588,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   };
   // Queue a unit whose contributors have all arrived, for this CTA's merge
   // helpers.  The queue is a ring of kMergeCap entries (0 = empty, else unit + 1);
-  // when it is full the pusher waits for the helpers (bounded).
+  // when it is full the pusher waits for the helpers (bounded).  If that wait
+  // gives up, the entry is not written (its ring slot still holds a unit not
+  // yet merged): the error word reports the timeout and the step's outputs
+  // are undefined, but no other unit's merge is lost.
   auto push_merge = [&](int64_t unit) {
     if (lane == 0) {
       const int slot = atomicAdd(&mq[kMergeCap], 1);
       const uint64_t t0 = global_ns();
+      bool full = false;
       while (slot - atomicAdd(&mq[kMergeCap + 1], 0) >= kMergeCap) {
-        if (global_ns() - t0 > kWaitLimitNs) { set_error(a.err, DEVERR_TIMEOUT); break; }
+        if (global_ns() - t0 > kWaitLimitNs) { set_error(a.err, DEVERR_TIMEOUT); full = true; break; }
         __nanosleep(128);
       }
-      atomicExch(&mq[slot % kMergeCap], static_cast<int>(unit) + 1);
+      if (!full) atomicExch(&mq[slot % kMergeCap], static_cast<int>(unit) + 1);
     }
     __syncwarp();
   };
@@ -1107,12 +1111,17 @@ template <typename T, int DH, int G, int NCW, int NSTG>
 int launch_t(const CUtensorMap& tmap, const LayerArgs& a, const DecodeScratch& sc, int mode, const void* q,
              const void* kn, const void* vn, const float* ext, void* out, int num_sms, cudaStream_t st) {
   using SM = Smem<T, DH, G, NCW, NSTG>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The shared-memory attribute belongs to the current device: set it once per
+  // device (devices beyond the table get it on every call).
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
     if (cudaFuncSetAttribute(decode_kernel<T, DH, G, NCW, NSTG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SM::TOTAL) != cudaSuccess)
       return -1;
-    attr_set = true;
+    if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
   }
   const int64_t tpu_max = (a.NS + TS - 1) / TS;
   const int64_t total_max = static_cast<int64_t>(a.units) * tpu_max;

@@ -126,16 +126,35 @@ typedef struct kvpop_layout_info {
 } kvpop_layout_info;
 
 /* Device bytes the caller must allocate for `cfg` (cache, slot metadata,
- * split-K and prefill scratch).  Validates cfg.  Host only. */
+ * split-K and prefill scratch).  Validates cfg.  Host only.
+ * Page §3 "Fixed-budget pruning" and §C.1 "Mask Definition": every KV head
+ * keeps at most B = S + W + K tokens, the same budget for every head, so the
+ * cache of a layer is units x (S + W + D + K) slots, fixed at creation
+ * (D = the staging ring of delayed scoring, §E.4).  The pages quote
+ * compression ratios (75%, 88%) without a formula; this library reads them
+ * as CR = 1 - B / ref_context and checks cfg.compression_ratio against it.
+ * Errors: KVPOP_ERR_INVALID_ARG (null argument; bad dtype, flag or scorer
+ * pointer; compression ratio out of [0, 1) or not matching the budget),
+ * KVPOP_ERR_BAD_SHAPE (shape outside the supported set). */
 int kvpop_cache_bytes(const kvpop_config* cfg, size_t* bytes);
 
 /* Binds a caller-allocated device buffer (>= kvpop_cache_bytes, 256-byte
  * aligned, on the current device) and initialises it (empty cache,
  * synchronously).  The buffer must outlive the handle.  *out receives the
- * handle (host memory owned by the library until kvpop_destroy). */
+ * handle (host memory owned by the library until kvpop_destroy).
+ * Page §3 "Fixed-budget pruning" (a hard, fixed-size cache: eviction is
+ * permanent, so the cache never grows past its budget) and §C.1 (the budget
+ * is reached once the sequence is long enough; until then every slot that
+ * holds a token is attended).  Errors: KVPOP_ERR_INVALID_ARG (null, short or
+ * misaligned buffer, buffer not device memory), KVPOP_ERR_BAD_SHAPE (cfg
+ * outside the supported shapes), KVPOP_ERR_CUDA (a CUDA call failed); *out
+ * is NULL then. */
 int kvpop_create(const kvpop_config* cfg, void* dev_mem, size_t bytes, kvpop_handle** out);
 
-/* Appends a chunk of n_tokens prompt tokens to layer `layer` (positions
+/* Page §I "KVpop Pseudocode" (score every KV entry, keep the sinks, the
+ * recent window and the running-prefix top-k of the eligible tokens) and
+ * §C.1 "Mask Definition", applied to a whole prompt chunk at once.
+ * Appends a chunk of n_tokens prompt tokens to layer `layer` (positions
  * n_seen .. n_seen + n_tokens - 1).  k, v: device [b][Hkv][n_tokens][d].
  * ext_scores: device fp32 [b][Hkv][n_tokens] (required with
  * KVPOP_FLAG_EXTERNAL_SCORES, ignored otherwise).  After the call the layer
@@ -143,11 +162,20 @@ int kvpop_create(const kvpop_config* cfg, void* dev_mem, size_t bytes, kvpop_han
  * long-range slots keep the K best eligible tokens; survivors keep their
  * slots and admitted tokens fill free/vacated slots in ascending order.
  * Must precede the layer's first decode step (else KVPOP_ERR_ORDER);
- * 0 <= n_tokens <= max_prefill_chunk. */
+ * 0 <= n_tokens <= max_prefill_chunk.  Errors (nothing enqueued):
+ * KVPOP_ERR_INVALID_ARG (bad handle or layer, negative n_tokens, null k or v,
+ * missing ext_scores), KVPOP_ERR_BAD_SHAPE (n_tokens > max_prefill_chunk),
+ * KVPOP_ERR_ORDER, KVPOP_ERR_CONTEXT_OVERFLOW (positions would reach
+ * max_context); KVPOP_ERR_CUDA if a launch fails. */
 int kvpop_prefill(kvpop_handle* h, int32_t layer, const void* k, const void* v, int32_t n_tokens,
                   const float* ext_scores, void* stream);
 
-/* One decode step of one layer for all batch rows.  With p = the layer's
+/* One decode step of one layer for all batch rows: page §3 "Fixed-budget
+ * pruning" (sinks + protected window + running top-k, eviction permanent),
+ * §C.1 "Mask Definition" (during decoding attention runs directly over the
+ * retained cache entries), §E.4 "Delayed Readout" (the token u = q - w
+ * becomes eligible at q; with the staging ring, D steps later) and §I
+ * "KVpop Pseudocode" (the running prefix top-k rule).  With p = the layer's
  * position counter:
  *  1. window append and boundary update: the token leaving the window (after
  *     D staging steps when D > 0) is scored by the MLP on [k; v] (or its
@@ -161,7 +189,12 @@ int kvpop_prefill(kvpop_handle* h, int32_t layer, const void* k, const void* v, 
  * [b][Hq][d] (same element type); ext_score: device fp32 [b][Hkv], the score
  * of the token being appended (required with KVPOP_FLAG_EXTERNAL_SCORES).
  * q, k_new, v_new and out must be 16-byte aligned (KVPOP_ERR_INVALID_ARG
- * otherwise).  The position counter then advances by one. */
+ * otherwise).  The position counter then advances by one.  Errors (nothing
+ * enqueued): KVPOP_ERR_INVALID_ARG (bad handle or layer, null or misaligned
+ * pointer, missing ext_score), KVPOP_ERR_CONTEXT_OVERFLOW (the position
+ * counter has reached max_context), KVPOP_ERR_BAD_SHAPE; KVPOP_ERR_CUDA if
+ * the launch fails.  Device-side failures (a bounded wait that gave up,
+ * debug-check mismatches) are reported later by kvpop_get_error. */
 int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void* k_new, const void* v_new,
                       void* out, const float* ext_score, void* stream);
 
@@ -197,7 +230,8 @@ int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void*
 int kvpop_decode_step_noalloc(kvpop_handle* h, int32_t layer, const void* q, const void* k_new,
                               const void* v_new, void* out, const float* ext_score, void* stream);
 
-/* The two halves of kvpop_decode_step, for callers that schedule them apart
+/* The two halves of kvpop_decode_step (same passages: page §3, §C.1, §E.4,
+ * §I), for callers that schedule them apart
  * (same arguments and semantics; append must precede attend for each step).
  * kvpop_decode_append: step 1 only (window append, boundary scoring and
  * argmin-replace); advances the position counter.
@@ -262,31 +296,38 @@ int kvpop_prefill_with_attention(kvpop_handle* h, int32_t layer, const void* q, 
 
 /* Copies layer `layer`'s slot -> position map (int32 [units][slots]), slot
  * scores (fp32 [units][slots]) and per-unit state (int32 [units][4]) to HOST
- * buffers; any of them may be NULL.  Synchronises `stream`.  For tests and
- * debugging. */
+ * buffers; any of them may be NULL.  Synchronises `stream`.  Test and
+ * diagnostic call; no passage of the pages defines it.  Errors:
+ * KVPOP_ERR_INVALID_ARG (bad handle or layer), KVPOP_ERR_CUDA. */
 int kvpop_inspect(kvpop_handle* h, int32_t layer, int32_t* pos_out, float* score_out, int32_t* state_out,
                   void* stream);
 
-/* Fills *out with the layout of the device buffer. */
+/* Fills *out with the layout of the device buffer.  Diagnostic call; no
+ * passage of the pages defines it.  KVPOP_ERR_INVALID_ARG on a null argument. */
 int kvpop_get_layout(const kvpop_handle* h, kvpop_layout_info* out);
 
-/* Synchronises the device and reads the device error word.  Returns KVPOP_OK
+/* Failure reporting of this library (no passage of the pages defines it).
+ * Synchronises the device and reads the device error word.  Returns KVPOP_OK
  * if no kernel recorded an error, KVPOP_ERR_CONTEXT_OVERFLOW / _TIMEOUT /
  * _DEVICE otherwise (device_bits, if not NULL, receives the KVPOP_DEVERR_*
  * bits), or KVPOP_ERR_CUDA if the device reported an asynchronous error. */
 int kvpop_get_error(kvpop_handle* h, int32_t* device_bits);
 
-/* Clears the device error word (asynchronously, on `stream`). */
+/* Clears the device error word (asynchronously, on `stream`).  Failure
+ * reporting of this library; no passage of the pages defines it. */
 int kvpop_clear_error(kvpop_handle* h, void* stream);
 
-/* Test hook: ORs `bits` into the device error word on `stream`, so host-side
- * failure handling can be exercised without making any kernel fail. */
+/* Test hook (no passage of the pages defines it): ORs `bits` into the device
+ * error word on `stream`, so host-side failure handling can be exercised
+ * without making any kernel fail. */
 int kvpop_debug_poison_error(kvpop_handle* h, int32_t bits, void* stream);
 
-/* Releases the handle's host state.  Does not touch the device buffer. */
+/* Releases the handle's host state.  Does not touch the device buffer.
+ * Resource management of this library; no passage of the pages defines it.
+ * KVPOP_ERR_INVALID_ARG on NULL. */
 int kvpop_destroy(kvpop_handle* h);
 
-/* Static description of a status code. */
+/* Static description of a status code (diagnostic; no passage defines it). */
 const char* kvpop_status_string(int status);
 
 #ifdef __cplusplus

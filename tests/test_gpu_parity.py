@@ -224,3 +224,42 @@ def test_full_size_target_config_sampled_units():
     base = w.sinks + w.window + w.delay
     assert (pos[:, base:] >= 0).all()                       # every long-range slot filled
     assert (state[:, 0] == w.prefill + w.decode).all()     # every unit advanced
+
+
+def test_full_size_cr75_sampled_units():
+    """The 75%-compression Qwen3-4B shape at full size (16 rows x 8 KV heads,
+    prompt 8192, B = 2048 = 4 + 128 + 1916, G = 4, bf16, MLP scorer), one
+    layer, bench.py's launch configuration.  Prefill plus 4 fused decode
+    steps; first, middle and last units against the oracle at every step:
+    outputs, long-range sets and exact fp32 scores."""
+    _need_gpu()
+    w = wl.QWEN3_4B_CR75.replace(name="full_size_cr75_case", n_layers=1, decode=4)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, gen_device="cuda", debug=False)
+    units = w.batch * w.n_kv_heads
+    for unit in (0, units // 2 + 3, units - 1):
+        gh.check_unit(run, 0, unit, exact_slots=False, atol=gh.BF16_ATOL)
+    pos, score, state = run.cache.inspect(0)
+    base = w.sinks + w.window + w.delay
+    assert (pos[:, base:] >= 0).all()
+    assert (state[:, 0] == w.prefill + w.decode).all()
+
+
+def test_full_size_8b_delayed_scoring_sampled_units():
+    """The Qwen3-8B shape with delayed scoring at full size (32 rows x 8 KV
+    heads, prompt 32768, B = 4096 = 4 + 256 + 3836 plus a D = 32 staging ring,
+    G = 4, bf16, MLP scorer), one layer.  Prefill plus 4 fused decode steps;
+    first, middle and last units against the oracle at every step, including
+    the staged tokens being attended and scored 32 steps after they leave the
+    window."""
+    _need_gpu()
+    w = wl.QWEN3_8B_D32.replace(name="full_size_8b_case", n_layers=1, decode=4)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, gen_device="cuda", debug=False)
+    units = w.batch * w.n_kv_heads
+    for unit in (0, units // 2 + 3, units - 1):
+        res = gh.check_unit(run, 0, unit, exact_slots=False, atol=gh.BF16_ATOL)
+        assert res.attended_counts == [w.budget + w.delay] * w.decode
+    pos, score, state = run.cache.inspect(0)
+    base = w.sinks + w.window + w.delay
+    assert (pos[:, base:] >= 0).all()
+    assert (pos[:, w.sinks + w.window:base] >= 0).all()     # the staging ring is full
+    assert (state[:, 0] == w.prefill + w.decode).all()

@@ -215,6 +215,90 @@ def test_full_size_target_shape_sampled_rows():
     assert torch.isfinite(r.out).all()
 
 
+def _fenwick_cutoffs(s, n, S, W, D, K):
+    import oracle_pins
+    return oracle_pins._fenwick_cutoffs(s, n, S, W, D, K)
+
+
+def _check_large_unit(r, unit, m_samples, rows, atol):
+    """Cutoffs of one unit at a size the brute-force cutoffs cannot reach:
+    equal to the pinned Fenwick-tree computation, and at sampled newest-
+    eligible positions m the GPU's cutoffs give exactly the oracle's running
+    top-k (j kept iff j <= m < c_j); sampled rows against the oracle's
+    attention over its attended set."""
+    w = r.w
+    S, W, D, K = w.sinks, w.window, w.delay, w.topk
+    k, v, q, out, lse, s = unit_view(r, unit)
+    c = r.cut[unit]
+    assert list(c) == _fenwick_cutoffs(s, r.n, S, W, D, K), f"unit {unit}: cutoffs differ from the Fenwick tree"
+    for m in m_samples:
+        kept = set(orc.running_topk(s, m + W + D, S, W, D, K))
+        gpu = {j for j in range(S, m + 1) if c[j] > m}
+        assert gpu == kept, (unit, m)
+    for qp in rows:
+        T = orc.running_topk(s, qp, S, W, D, K)
+        A = orc.attended_positions(qp, S, W, D, T)
+        o, _ = orc.attention(q[qp], k[A], v[A])
+        np.testing.assert_allclose(out[qp], o, rtol=0, atol=atol, err_msg=f"unit {unit} q {qp}")
+        if lse is not None:
+            np.testing.assert_allclose(lse[qp], orc.attention_lse(q[qp], k[A]), rtol=0, atol=LSE_ATOL[w.dtype])
+
+
+def test_cutoffs_sorted_in_the_workspace():
+    """More than 16,384 eligible tokens in a unit: cutoff_kernel sorts the
+    rank keys in the caller's workspace instead of shared memory (bitmap
+    still in shared memory).  One unit, 17,000 prompt tokens, bf16 d 128 G 4,
+    the 87.5% budget (4 + 128 + 892), caller scores with ties."""
+    _need_gpu()
+    w = _case("bf16", 128, 4, 1, S=4, W=128, D=0, K=892, hidden=64)
+    n = 17000
+    r = run_prefill_attention(w, n, external=True, tie_levels=3, gen_device="cuda")
+    rng = np.random.default_rng(3)
+    m_last = n - 1 - w.window - w.delay
+    ms = sorted(set([w.sinks, w.sinks + w.topk - 1, w.sinks + w.topk, m_last] +
+                    list(rng.integers(w.sinks, m_last + 1, 8))))
+    rows = sorted(set([0, n - 1, 16500] + list(rng.integers(0, n, 8))))
+    _check_large_unit(r, 0, ms, rows, gh.BF16_ATOL)
+    assert torch.isfinite(r.out).all()
+
+
+def test_cutoffs_with_the_bitmap_in_the_workspace():
+    """More than 131,072 eligible tokens in a unit: cutoff_kernel keeps both
+    the sort keys and the position bitmap in the workspace.  One unit of
+    131,594 prompt tokens (131,572 eligible), fp32 d 64 G 2, S 4 + W 16 +
+    D 2 + K 300, the library's MLP scorer."""
+    _need_gpu()
+    w = _case("f32", 64, 2, 1, S=4, W=16, D=2, K=300, hidden=32)
+    n = 131072 + 22 + 500
+    r = run_prefill_attention(w, n, gen_device="cuda")
+    rng = np.random.default_rng(4)
+    m_last = n - 1 - w.window - w.delay
+    ms = sorted(set([w.sinks, w.sinks + w.topk, 131100, m_last] + list(rng.integers(w.sinks, m_last + 1, 4))))
+    rows = sorted(set([0, n - 1, 131090] + list(rng.integers(0, n, 6))))
+    _check_large_unit(r, 0, ms, rows, gh.F32_ATOL)
+    assert torch.isfinite(r.out).all()
+
+
+def test_full_size_8b_delayed_shape_sampled_rows():
+    """The Qwen3-8B delayed-scoring shape at full size (32 rows x 8 KV heads,
+    prompt 32768, S 4 + W 256 + D 32 + K 3836, G 4, bf16, MLP scorer): 32,476
+    eligible tokens per unit, so every unit's cutoffs are sorted in the
+    workspace.  Sampled units: cutoffs against the Fenwick tree and the
+    oracle's running top-k at sampled positions, and sampled output rows."""
+    _need_gpu()
+    w = wl.QWEN3_8B_D32.replace(name="pa_full_size_8b", n_layers=1, decode=0)
+    n = w.prefill
+    r = run_prefill_attention(w, n, gen_device="cuda")
+    units = w.batch * w.n_kv_heads
+    rng = np.random.default_rng(8)
+    m_last = n - 1 - w.window - w.delay
+    for unit in (0, units - 1):
+        ms = sorted(set([w.sinks, w.sinks + w.topk, m_last] + list(rng.integers(w.sinks, m_last + 1, 3))))
+        rows = sorted(set([0, w.sinks + w.window + w.delay + w.topk + 5, n - 1] + list(rng.integers(0, n, 4))))
+        _check_large_unit(r, unit, ms, rows, gh.BF16_ATOL)
+    assert torch.isfinite(r.out).all()
+
+
 def test_argument_errors_enqueue_nothing():
     """Misaligned or missing pointers, a short workspace and a bad layer are
     rejected before any work is enqueued; the output stays untouched."""

@@ -77,3 +77,58 @@ def test_bench_arguments(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--path", "prefill-attention", "--pa-batch", "4", "--steps", "2"])
     a = bench.parse_args()
     assert a.path == "prefill-attention" and a.pa_batch == 4 and a.steps == 2
+
+
+def test_sweep_plan_covers_the_grid_and_bounds_memory():
+    """Every (budget, batch) point of the bandwidth sweep is planned once;
+    the 36-layer cache is kept whole where it fits under the cap, and the
+    points where it does not (b256 x B8192 = 309 GB is larger than HBM) run
+    fewer layers, each point's cache within the cap; the prompt fills the
+    long-range slots (prompt - W - S >= K)."""
+    import bench
+    import kvpop_workloads as wl
+    plan = bench.sweep_plan()
+    assert {(p["budget"], p["batch"]) for p in plan} == {(B, b) for B in wl.SWEEP_BUDGETS
+                                                           for b in wl.SWEEP_BATCHES}
+    assert len(plan) == len(wl.SWEEP_BUDGETS) * len(wl.SWEEP_BATCHES)
+    for p in plan:
+        w = p["workload"]
+        per_layer = bench.attention_bytes(w)
+        assert 1 <= p["layers"] <= 36 and w.n_layers == p["layers"]
+        assert p["layers"] == 36 or per_layer * (p["layers"] + 1) > bench.SWEEP_CACHE_CAP
+        assert per_layer * p["layers"] <= bench.SWEEP_CACHE_CAP
+        assert p["prompt"] - w.window - w.sinks >= w.topk
+        assert w.budget == p["budget"] and w.batch == p["batch"]
+    big = [p for p in plan if p["budget"] == 8192 and p["batch"] == 256][0]
+    assert big["full_cache_gb"] > 180 and big["layers"] < 36
+    small = [p for p in plan if p["budget"] == 512 and p["batch"] == 1][0]
+    assert small["layers"] == 36
+
+
+def test_dtype_names_are_explicit():
+    """make_config accepts only known element-type names; a typo raises
+    instead of silently building a bf16 cache."""
+    import torch
+    import fixed_budget_kv_kvpop_b200 as kp
+    for name in ("f32", "float32", "fp32", torch.float32):
+        assert kp.dtype_code(name) == kp.KVPOP_DTYPE_F32
+    for name in ("bf16", "bfloat16", torch.bfloat16):
+        assert kp.dtype_code(name) == kp.KVPOP_DTYPE_BF16
+    for bad in ("float", "fp16", "bf 16", torch.float16, None):
+        with pytest.raises(ValueError):
+            kp.dtype_code(bad)
+
+
+def test_tensor_checks_reject_host_tensors():
+    """The binding checks every tensor before passing its address on: a
+    host tensor, a wrong dtype, shape or layout raises ValueError."""
+    import torch
+    import fixed_budget_kv_kvpop_b200 as kp
+    dev = torch.device("cuda", 0)
+    with pytest.raises(ValueError, match="cuda"):
+        kp.check_tensor(torch.zeros(2, 3), "q", (2, 3), torch.float32, dev)
+    with pytest.raises(ValueError, match="torch.Tensor"):
+        kp.check_tensor([1.0], "q", (1,), torch.float32, dev)
+    meta = torch.empty(2, 3, device="meta")
+    with pytest.raises(ValueError):
+        kp.check_tensor(meta, "q", (2, 3), torch.float32, dev)
