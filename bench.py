@@ -398,13 +398,23 @@ def replica_throughput(batch: int, steps: int, world: int, elapsed_ms: float) ->
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def build_cache(w: wl.Workload, torch, log_decay=None, prompt=None):
+MLSTM_DIMS = (16, 16)   # mLSTM scorer of the bench: Hedgehog projection p, value size dv
+
+
+def build_cache(w: wl.Workload, torch, log_decay=None, prompt=None, scorer="mlp"):
     """A cache for every layer of `w`, each layer prefilled with `prompt`
-    tokens (default: the workload's prompt) in one kvpop_prefill call."""
+    tokens (default: the workload's prompt) in one kvpop_prefill call.
+    scorer: 'mlp' (the workload's MLP) or 'mlstm' (the stateful scorer with
+    seeded weights, p = dv = 16)."""
     import fixed_budget_kv_kvpop_b200 as kp
     P = w.prefill if prompt is None else prompt
     weights = tuple(t.cuda() for t in wl.scorer_weights(w))
     w1, b1, w2, b2 = weights
+    extra = {}
+    if scorer == "mlstm":
+        packed = wl.mlstm_weights(w, *MLSTM_DIMS).cuda()
+        weights = weights + (packed,)
+        extra = dict(scorer="mlstm", mlstm_p=MLSTM_DIMS[0], mlstm_dv=MLSTM_DIMS[1], mlstm_w=packed)
     decay = None
     if log_decay is not None:
         decay = torch.full((w.n_layers, w.n_kv_heads), float(log_decay), dtype=torch.float32, device="cuda")
@@ -413,7 +423,7 @@ def build_cache(w: wl.Workload, torch, log_decay=None, prompt=None):
                          head_dim=w.head_dim, sinks=w.sinks, window=w.window, topk=w.topk, delay=w.delay,
                          ref_context=w.prefill, compression_ratio=w.compression_ratio,
                          max_prefill_chunk=P, dtype=w.dtype, scorer_hidden=w.scorer_hidden,
-                         w1=w1, b1=b1, w2=w2, b2=b2, log_decay=decay)
+                         w1=w1, b1=b1, w2=w2, b2=b2, log_decay=decay, **extra)
     cache = kp.KVPopCache(cfg, keepalive=weights)
     stream = torch.cuda.current_stream()
     prefill_ms = []
@@ -578,11 +588,11 @@ def run_gpu(args, w, rank, world, torch):
     return res
 
 
-def other_config(args, w, torch, world, prompt=None, note=None):
+def other_config(args, w, torch, world, prompt=None, note=None, scorer="mlp"):
     """Decode throughput of another configuration, timed like the headline
     (same steps and warm-up; no e2e or CPU leg)."""
     t0 = time.perf_counter()
-    cache, prefill_ms = build_cache(w, torch, None, prompt)
+    cache, prefill_ms = build_cache(w, torch, None, prompt, scorer)
     m = time_decode(w, cache, args.steps, args.warmup, torch, world, args.input_sets)
     del cache
     torch.cuda.empty_cache()
@@ -870,6 +880,13 @@ def main():
                 if WORKLOADS[key].name != w.name and not args.layers:
                     extras[key] = other_config(args, WORKLOADS[key], torch, world)
             res["configs"] = extras
+            # the stateful mLSTM scorer with delayed readout on the headline shape
+            res["mlstm"] = other_config(
+                args, w, torch, world, scorer="mlstm",
+                note=f"mLSTM scorer (p = {MLSTM_DIMS[0]}, dv = {MLSTM_DIMS[1]}, seeded weights): per layer and step "
+                     "one mlstm_step_kernel (state update with the new token, delayed readout of the boundary "
+                     "token, argmin decision) and one decode_kernel")
+            res["mlstm"]["gpu_launches"] = 2 * res["mlstm"]["launches"]
             if not args.no_sweep:
                 res["sweep"] = run_sweep(args, torch, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

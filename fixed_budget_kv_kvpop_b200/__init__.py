@@ -49,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "kvpop_get_layout", "kvpop_get_error", "kvpop_clear_error", "kvpop_debug_poison_error",
     "kvpop_destroy", "kvpop_status_string", "kvpop_decode_step_noalloc",
     "kvpop_prefill_attention_workspace_bytes", "kvpop_prefill_attention", "kvpop_prefill_with_attention",
+    "kvpop_debug_set_hook",
 )
 
 
@@ -62,7 +63,20 @@ class kvpop_config(ctypes.Structure):
         ("dtype", ctypes.c_int32), ("scorer_hidden", ctypes.c_int32),
         ("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
         ("flags", ctypes.c_uint32), ("log_decay", ctypes.c_void_p),
+        ("scorer_kind", ctypes.c_int32), ("mlstm_p", ctypes.c_int32), ("mlstm_dv", ctypes.c_int32),
+        ("mlstm_w", ctypes.c_void_p),
     ]
+
+
+KVPOP_SCORER_MLP = 0
+KVPOP_SCORER_MLSTM = 1
+
+
+def mlstm_head_floats(p: int, dv: int, d: int) -> int:
+    """Floats of one (layer, KV head) block of the mLSTM weights (include/kvpop.h
+    KVPOP_MLSTM_HEAD_FLOATS): W_q, W_k [p][2d], W_v [dv][2d], w_i, w_f [2d],
+    then w_o [dv], b_i, b_f, b_o, padded to a multiple of 4."""
+    return (2 * p + dv + 2) * 2 * d + ((dv + 3 + 3) // 4) * 4
 
 
 class kvpop_layout_info(ctypes.Structure):
@@ -100,6 +114,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvpop_prefill_attention_workspace_bytes": ([P, I32, ctypes.POINTER(SZ)], ctypes.c_int),
         "kvpop_prefill_attention": ([P, I32, P, P, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
         "kvpop_prefill_with_attention": ([P, I32, P, P, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
+        "kvpop_debug_set_hook": ([P, I32], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -179,10 +194,15 @@ def check_tensor(t, name: str, shape, dtype, device) -> None:
 def make_config(*, batch, n_layers, n_q_heads, n_kv_heads, head_dim, sinks, window, topk, delay=0,
                 ref_context=0, compression_ratio=0.0, max_context=None, max_prefill_chunk=0,
                 dtype="bf16", scorer_hidden=64, w1=None, b1=None, w2=None, b2=None,
-                external_scores=False, debug_checks=False, log_decay=None) -> kvpop_config:
+                external_scores=False, debug_checks=False, log_decay=None, scorer="mlp", mlstm_p=0,
+                mlstm_dv=0, mlstm_w=None) -> kvpop_config:
     """log_decay: optional device fp32 tensor [n_layers][n_kv_heads] of
     ln(gamma_h) <= 0 (temporal decay); max_context defaults to 2^30, or 2^24
-    with decay."""
+    with decay.  scorer: 'mlp' (w1/b1/w2/b2; the linear scorer when
+    scorer_hidden = 0) or 'mlstm' (mlstm_p, mlstm_dv and the packed device
+    weights mlstm_w [n_layers][n_kv_heads][mlstm_head_floats(p, dv, d)])."""
+    if scorer not in ("mlp", "mlstm"):
+        raise ValueError(f"unknown scorer {scorer!r}: 'mlp' or 'mlstm'")
     if max_context is None:
         max_context = (1 << 24) if log_decay is not None else (1 << 30)
     c = kvpop_config()
@@ -195,12 +215,15 @@ def make_config(*, batch, n_layers, n_q_heads, n_kv_heads, head_dim, sinks, wind
     c.w1, c.b1, c.w2, c.b2 = _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)
     c.flags = (KVPOP_FLAG_EXTERNAL_SCORES if external_scores else 0) | (KVPOP_FLAG_DEBUG_CHECKS if debug_checks else 0)
     c.log_decay = _ptr(log_decay)
+    c.scorer_kind = KVPOP_SCORER_MLSTM if scorer == "mlstm" else KVPOP_SCORER_MLP
+    c.mlstm_p, c.mlstm_dv = mlstm_p, mlstm_dv
+    c.mlstm_w = _ptr(mlstm_w)
     return c
 
 
-def cache_bytes(cfg: kvpop_config) -> int:
+def cache_bytes(cfg: kvpop_config, library=None) -> int:
     n = ctypes.c_size_t(0)
-    _check(lib.kvpop_cache_bytes(ctypes.byref(cfg), ctypes.byref(n)), "kvpop_cache_bytes")
+    _check((library or lib).kvpop_cache_bytes(ctypes.byref(cfg), ctypes.byref(n)), "kvpop_cache_bytes")
     return n.value
 
 
@@ -211,16 +234,19 @@ class KVPopCache:
     object; they are kept referenced here.
     """
 
-    def __init__(self, cfg: kvpop_config, device=None, keepalive=()):
+    def __init__(self, cfg: kvpop_config, device=None, keepalive=(), library=None):
+        """library: another build of the same library loaded with
+        load_library (the test-hook build, for instance); default libkvpop.so."""
         import torch
         self.cfg = cfg
+        self._lib = library or lib
         self._keep = tuple(keepalive)
-        self.nbytes = cache_bytes(cfg)
+        self.nbytes = cache_bytes(cfg, self._lib)
         self.buffer = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
         base = self.buffer.data_ptr()
         self._off = (-base) % 256
         self.handle = ctypes.c_void_p()
-        _check(lib.kvpop_create(ctypes.byref(cfg), ctypes.c_void_p(base + self._off), self.nbytes,
+        _check(self._lib.kvpop_create(ctypes.byref(cfg), ctypes.c_void_p(base + self._off), self.nbytes,
                                 ctypes.byref(self.handle)), "kvpop_create")
         self.device = self.buffer.device
         self.dtype = _torch_dtype(cfg.dtype)
@@ -237,10 +263,10 @@ class KVPopCache:
         c = self.cfg
         return c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim
 
-    def __del__(self, _lib=lib):
+    def __del__(self):
         h = getattr(self, "handle", None)
         if h:
-            _lib.kvpop_destroy(h)
+            self._lib.kvpop_destroy(h)
             self.handle = None
 
     def prefill(self, layer: int, k, v, ext_scores=None, stream=None):
@@ -251,7 +277,7 @@ class KVPopCache:
             self._elems("v", v, (b, hkv, n, d))
             if ext_scores is not None:
                 self._f32("ext_scores", ext_scores, (b, hkv, n))
-        _check(lib.kvpop_prefill(self.handle, layer, _ptr(k), _ptr(v), n, _ptr(ext_scores),
+        _check(self._lib.kvpop_prefill(self.handle, layer, _ptr(k), _ptr(v), n, _ptr(ext_scores),
                                  _stream_ptr(stream)), "kvpop_prefill")
 
     def _check_step(self, q, k_new, v_new, out, ext_score):
@@ -265,7 +291,7 @@ class KVPopCache:
 
     def decode_step(self, layer: int, q, k_new, v_new, out, ext_score=None, stream=None):
         self._check_step(q, k_new, v_new, out, ext_score)
-        _check(lib.kvpop_decode_step(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+        _check(self._lib.kvpop_decode_step(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                      _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step")
 
     def decode_step_noalloc(self, layer: int, q, k_new, v_new, out, ext_score=None, stream=None):
@@ -275,12 +301,12 @@ class KVPopCache:
         call on a device looks up that buffer once (make it before any stream
         capture); calls that overlap on the GPU share the buffer and race."""
         self._check_step(q, k_new, v_new, out, ext_score)
-        _check(lib.kvpop_decode_step_noalloc(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+        _check(self._lib.kvpop_decode_step_noalloc(self.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                              _ptr(ext_score), _stream_ptr(stream)), "kvpop_decode_step_noalloc")
 
     def prefill_attention_workspace_bytes(self, n_tokens: int) -> int:
         out = ctypes.c_size_t()
-        _check(lib.kvpop_prefill_attention_workspace_bytes(self.handle, n_tokens, ctypes.byref(out)),
+        _check(self._lib.kvpop_prefill_attention_workspace_bytes(self.handle, n_tokens, ctypes.byref(out)),
                "kvpop_prefill_attention_workspace_bytes")
         return out.value
 
@@ -292,7 +318,7 @@ class KVPopCache:
         units * n int32 are the running cutoffs afterwards).  Does not touch
         the cache."""
         n = self._check_prompt(q, k, v, out, lse, workspace, ext_scores)
-        _check(lib.kvpop_prefill_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
+        _check(self._lib.kvpop_prefill_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
                                            _ptr(out), _ptr(lse), _ptr(workspace),
                                            int(workspace.numel() * workspace.element_size()) if workspace is not None
                                            else 0, _stream_ptr(stream)), "kvpop_prefill_attention")
@@ -303,7 +329,7 @@ class KVPopCache:
         call: the prompt is scored once; afterwards the layer holds the cache
         kvpop_prefill would build and is ready for decode steps."""
         n = self._check_prompt(q, k, v, out, lse, workspace, ext_scores)
-        _check(lib.kvpop_prefill_with_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
+        _check(self._lib.kvpop_prefill_with_attention(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(ext_scores),
                                                 _ptr(out), _ptr(lse), _ptr(workspace),
                                                 int(workspace.numel() * workspace.element_size())
                                                 if workspace is not None else 0, _stream_ptr(stream)),
@@ -331,14 +357,14 @@ class KVPopCache:
         self._elems("v_new", v_new, (b, hkv, d))
         if ext_score is not None:
             self._f32("ext_score", ext_score, (b, hkv))
-        _check(lib.kvpop_decode_append(self.handle, layer, _ptr(k_new), _ptr(v_new), _ptr(ext_score),
+        _check(self._lib.kvpop_decode_append(self.handle, layer, _ptr(k_new), _ptr(v_new), _ptr(ext_score),
                                        _stream_ptr(stream)), "kvpop_decode_append")
 
     def decode_attend(self, layer: int, q, out, stream=None):
         b, hq, _, d = self._dims()
         self._elems("q", q, (b, hq, d))
         self._elems("out", out, (b, hq, d))
-        _check(lib.kvpop_decode_attend(self.handle, layer, _ptr(q), _ptr(out), _stream_ptr(stream)),
+        _check(self._lib.kvpop_decode_attend(self.handle, layer, _ptr(q), _ptr(out), _stream_ptr(stream)),
                "kvpop_decode_attend")
 
     def inspect(self, layer: int, stream=None):
@@ -348,14 +374,14 @@ class KVPopCache:
         pos = np.empty(n, np.int32)
         score = np.empty(n, np.float32)
         state = np.empty(lay.units * 4, np.int32)
-        _check(lib.kvpop_inspect(self.handle, layer, pos.ctypes.data, score.ctypes.data, state.ctypes.data,
+        _check(self._lib.kvpop_inspect(self.handle, layer, pos.ctypes.data, score.ctypes.data, state.ctypes.data,
                                  _stream_ptr(stream)), "kvpop_inspect")
         return (pos.reshape(lay.units, lay.slots_per_unit), score.reshape(lay.units, lay.slots_per_unit),
                 state.reshape(lay.units, 4))
 
     def layout(self) -> kvpop_layout_info:
         info = kvpop_layout_info()
-        _check(lib.kvpop_get_layout(self.handle, ctypes.byref(info)), "kvpop_get_layout")
+        _check(self._lib.kvpop_get_layout(self.handle, ctypes.byref(info)), "kvpop_get_layout")
         return info
 
     def kv_rows(self, layer: int):
@@ -367,11 +393,15 @@ class KVPopCache:
 
     def get_error(self):
         bits = ctypes.c_int32(0)
-        st = lib.kvpop_get_error(self.handle, ctypes.byref(bits))
+        st = self._lib.kvpop_get_error(self.handle, ctypes.byref(bits))
         return st, bits.value
 
     def clear_error(self, stream=None):
-        _check(lib.kvpop_clear_error(self.handle, _stream_ptr(stream)), "kvpop_clear_error")
+        _check(self._lib.kvpop_clear_error(self.handle, _stream_ptr(stream)), "kvpop_clear_error")
 
     def poison_error(self, bits: int, stream=None):
-        _check(lib.kvpop_debug_poison_error(self.handle, bits, _stream_ptr(stream)), "kvpop_debug_poison_error")
+        _check(self._lib.kvpop_debug_poison_error(self.handle, bits, _stream_ptr(stream)), "kvpop_debug_poison_error")
+
+    def set_test_hook(self, hook: int):
+        """Failure injection of a KVPOP_TEST_HOOKS build (kvpop_debug_set_hook)."""
+        _check(self._lib.kvpop_debug_set_hook(self.handle, hook), "kvpop_debug_set_hook")

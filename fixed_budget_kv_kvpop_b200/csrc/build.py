@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
-SOURCES = ["kvpop_api.cu", "kvpop_decode.cu", "kvpop_prefill.cu", "kvpop_prefill_attn.cu"]
+SOURCES = ["kvpop_api.cu", "kvpop_decode.cu", "kvpop_prefill.cu", "kvpop_prefill_attn.cu", "kvpop_mlstm.cu"]
 HEADERS = ["kvpop_internal.cuh", "kvpop_prefill_attn.cuh", os.path.join(ROOT, "include", "kvpop.h")]
 OUT = os.path.join(PKG, "libkvpop.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -66,5 +66,23 @@ def build(force: bool = False, verbose: bool = False, out: str = OUT, defines=()
     return out
 
 
+TEST_HOOKS_OUT = os.path.join(PKG, "libkvpop_testhooks.so")
+# The failure-injection build: kvpop_debug_set_hook works, and the decode
+# kernel's merge-queue waits give up after 50 ms instead of 2 s.
+TEST_HOOKS_DEFINES = ("KVPOP_TEST_HOOKS", "KVPOP_MERGE_WAIT_LIMIT_NS=50000000ull")
+
+
+def build_test_hooks(force: bool = False) -> str:
+    if not force and os.path.exists(TEST_HOOKS_OUT):
+        t = os.path.getmtime(TEST_HOOKS_OUT)
+        deps = [os.path.join(HERE, s) for s in SOURCES] + [os.path.join(HERE, h) if not os.path.isabs(h) else h
+                                                          for h in HEADERS] + [__file__]
+        if all(os.path.getmtime(p) <= t for p in deps):
+            return TEST_HOOKS_OUT
+    return build(out=TEST_HOOKS_OUT, defines=TEST_HOOKS_DEFINES)
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--test-hooks" in sys.argv:
+        print(build_test_hooks(force="--force" in sys.argv))

@@ -21,7 +21,13 @@ struct Layout {
   size_t kv_off, kv_stride, pos_off, pos_stride, score_off, score_stride, state_off, state_stride;
   size_t layer_off, dec_off, dec_stride;
   size_t pacc_off, pml_off, ticket_off, pre_score_off, pre_tgt_off, err_off, total;
+  size_t mlstm_off, mlstm_stride;   // mLSTM states per layer (0 bytes for the stateless scorers)
 };
+
+// The mLSTM scorer decides (not caller scores).
+bool mlstm_active(const kvpop_config* c) {
+  return c->scorer_kind == KVPOP_SCORER_MLSTM && !(c->flags & KVPOP_FLAG_EXTERNAL_SCORES);
+}
 
 bool hidden_supported(int h) { return h == 0 || h == 32 || h == 64 || h == 128; }   // 0: linear scorer
 
@@ -36,7 +42,13 @@ int validate(const kvpop_config* c) {
   if ((c->flags & ~(KVPOP_FLAG_EXTERNAL_SCORES | KVPOP_FLAG_DEBUG_CHECKS)) != 0) return KVPOP_ERR_INVALID_ARG;
   const int G = c->n_q_heads / c->n_kv_heads;
   if (!decode_supported(c->dtype, c->head_dim, G)) return KVPOP_ERR_BAD_SHAPE;
-  if (!(c->flags & KVPOP_FLAG_EXTERNAL_SCORES)) {
+  if (c->scorer_kind != KVPOP_SCORER_MLP && c->scorer_kind != KVPOP_SCORER_MLSTM) return KVPOP_ERR_INVALID_ARG;
+  if (c->scorer_kind == KVPOP_SCORER_MLSTM) {
+    if (c->mlstm_p < 1 || c->mlstm_p > 16 || c->mlstm_dv < 1 || c->mlstm_dv > 32) return KVPOP_ERR_BAD_SHAPE;
+    if (c->head_dim != 64 && c->head_dim != 128) return KVPOP_ERR_BAD_SHAPE;
+    if (mlstm_active(c) && (!c->mlstm_w || (reinterpret_cast<uintptr_t>(c->mlstm_w) & 15u) != 0))
+      return KVPOP_ERR_INVALID_ARG;
+  } else if (!(c->flags & KVPOP_FLAG_EXTERNAL_SCORES)) {
     if (!hidden_supported(c->scorer_hidden)) return KVPOP_ERR_BAD_SHAPE;
     if (!c->w1 || !c->b2 || (c->scorer_hidden > 0 && (!c->b1 || !c->w2))) return KVPOP_ERR_INVALID_ARG;
   }
@@ -68,6 +80,11 @@ Layout make_layout(const kvpop_config* c) {
   L.score_off = off; off += layers * L.score_stride;
   L.state_stride = align256(units * 16);
   L.state_off = off; off += layers * L.state_stride;
+  // after state_off: zeroed at creation (an mLSTM state starts at C = 0, n = 0, m = 0)
+  L.mlstm_stride = c->scorer_kind == KVPOP_SCORER_MLSTM
+                       ? align256(units * static_cast<size_t>(mlstm_state_doubles(c->mlstm_p, c->mlstm_dv)) * 8)
+                       : 0;
+  L.mlstm_off = off; off += layers * L.mlstm_stride;
   L.layer_off = off; off += align256(layers * sizeof(LayerState));
   L.dec_stride = align256(2 * units * sizeof(Decision));
   L.dec_off = off; off += layers * L.dec_stride;
@@ -93,6 +110,7 @@ struct kvpop_handle {
   std::vector<int> n_topk;   // host mirror of each layer's long-range fill
   std::vector<char> decoding;
   std::vector<CUtensorMap> maps;  // per layer: TMA view of the cache rows
+  int test_hook = 0;              // failure injection (KVPOP_TEST_HOOKS builds only)
 };
 
 namespace {
@@ -130,6 +148,15 @@ LayerArgs layer_args(const kvpop_handle* h, int layer) {
   a.flags = c.flags;
   a.row_bytes = L.row_bytes;
   a.log_decay = c.log_decay ? c.log_decay + static_cast<size_t>(layer) * H : nullptr;
+  a.test_hook = h->test_hook;
+  a.mlstm = mlstm_active(&c) ? 1 : 0;
+  if (c.scorer_kind == KVPOP_SCORER_MLSTM) {
+    a.mp = c.mlstm_p;
+    a.mdv = c.mlstm_dv;
+    a.mw = c.mlstm_w ? c.mlstm_w + static_cast<size_t>(layer) * H * mlstm_head_floats(c.mlstm_p, c.mlstm_dv, c.head_dim)
+                     : nullptr;
+    a.mstate = reinterpret_cast<double*>(h->mem + L.mlstm_off + layer * L.mlstm_stride);
+  }
   return a;
 }
 
@@ -261,6 +288,8 @@ int kvpop_decode_append(kvpop_handle* h, int32_t layer, const void* k_new, const
   if (ext && !ext_score) return KVPOP_ERR_INVALID_ARG;
   if (h->n_seen[layer] >= h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
   const LayerArgs a = layer_args(h, layer);
+  if (a.mlstm && launch_mlstm_step(a, h->cfg.dtype, k_new, v_new, static_cast<cudaStream_t>(stream)) != 0)
+    return KVPOP_ERR_CUDA;
   if (launch_append(a, h->cfg.dtype, k_new, v_new, ext ? ext_score : nullptr, static_cast<cudaStream_t>(stream)) != 0)
     return KVPOP_ERR_CUDA;
   advance_mirror(h, layer);
@@ -288,8 +317,11 @@ int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void*
   if (ext && !ext_score) return KVPOP_ERR_INVALID_ARG;
   if (h->n_seen[layer] >= h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
   const LayerArgs a = layer_args(h, layer);
-  const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, decode_scratch(h), MODE_STEP, q, k_new, v_new,
-                              ext ? ext_score : nullptr, out, h->num_sms, static_cast<cudaStream_t>(stream));
+  if (a.mlstm && launch_mlstm_step(a, h->cfg.dtype, k_new, v_new, static_cast<cudaStream_t>(stream)) != 0)
+    return KVPOP_ERR_CUDA;
+  const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, decode_scratch(h), a.mlstm ? MODE_STEP_NODECIDE : MODE_STEP,
+                              q, k_new, v_new, ext ? ext_score : nullptr, out, h->num_sms,
+                              static_cast<cudaStream_t>(stream));
   if (r == -2) return KVPOP_ERR_BAD_SHAPE;
   if (r != 0) return KVPOP_ERR_CUDA;
   advance_mirror(h, layer);
@@ -417,6 +449,18 @@ int kvpop_prefill_with_attention(kvpop_handle* h, int32_t layer, const void* q, 
   return KVPOP_OK;
 }
 
+int kvpop_debug_set_hook(kvpop_handle* h, int32_t hook) {
+#ifdef KVPOP_TEST_HOOKS
+  if (!h || hook < 0 || hook > TEST_HOOK_WITHHOLD_DONE) return KVPOP_ERR_INVALID_ARG;
+  h->test_hook = hook;
+  return KVPOP_OK;
+#else
+  (void)h;
+  (void)hook;
+  return KVPOP_ERR_INVALID_ARG;   // not a test build: no hook exists
+#endif
+}
+
 int kvpop_destroy(kvpop_handle* h) {
   if (!h) return KVPOP_ERR_INVALID_ARG;
   delete h;
@@ -507,8 +551,9 @@ extern "C" int kvpop_decode_step_noalloc(kvpop_handle* h, int32_t layer, const v
   // leave them non-zero, and another handle may have used more units
   if (cudaMemsetAsync(sc.ticket, 0, ticket_bytes, st) != cudaSuccess) return KVPOP_ERR_CUDA;
   const LayerArgs a = layer_args(h, layer);
-  const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, sc, MODE_STEP, q, k_new, v_new,
-                              ext ? ext_score : nullptr, out, h->num_sms, st);
+  if (a.mlstm && launch_mlstm_step(a, h->cfg.dtype, k_new, v_new, st) != 0) return KVPOP_ERR_CUDA;
+  const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, sc, a.mlstm ? MODE_STEP_NODECIDE : MODE_STEP, q, k_new,
+                              v_new, ext ? ext_score : nullptr, out, h->num_sms, st);
   if (r == -2) return KVPOP_ERR_BAD_SHAPE;
   if (r != 0) return KVPOP_ERR_CUDA;
   advance_mirror(h, layer);

@@ -542,7 +542,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const bool step = (mode == MODE_STEP);
+  const bool step = (mode != MODE_ATTEND);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NCW * (NSTG + 2); ++i) mbar_init(&full_bar[i], 1);
@@ -598,7 +598,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
       const uint64_t t0 = global_ns();
       bool full = false;
       while (slot - atomicAdd(&mq[kMergeCap + 1], 0) >= kMergeCap) {
-        if (global_ns() - t0 > kWaitLimitNs) { set_error(a.err, DEVERR_TIMEOUT); full = true; break; }
+        if (global_ns() - t0 > kMergeWaitLimitNs) { set_error(a.err, DEVERR_TIMEOUT); full = true; break; }
         __nanosleep(128);
       }
       if (!full) atomicExch(&mq[slot % kMergeCap], static_cast<int>(unit) + 1);
@@ -627,7 +627,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
           if (atomicCAS(&mq[kMergeCap + 1], head, head + 1) == head) {
             int v;
             while ((v = atomicExch(&mq[head % kMergeCap], 0)) == 0) {
-              if (global_ns() - t0 > kWaitLimitNs) break;
+              if (global_ns() - t0 > kMergeWaitLimitNs) break;
             }
             got = v > 0 ? v - 1 : -3;
           }
@@ -646,7 +646,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
         do_merge(got);
         continue;
       }
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > kMergeWaitLimitNs) {
         if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
         break;
       }
@@ -655,6 +655,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   };
   auto consumer_done = [&]() {
     __syncwarp();
+#ifdef KVPOP_TEST_HOOKS
+    if (a.test_hook == TEST_HOOK_WITHHOLD_DONE && blockIdx.x == 0 && warp == 0) return;
+#endif
     if (lane == 0) {
       __threadfence_block();
       atomicAdd(&mq[kMergeCap + 2], 1);
@@ -683,10 +686,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     if (step) {
       const int dw = warp - NCW;
       for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
-        const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
-        const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, &cur, k_new + static_cast<size_t>(u) * DH,
-                                           v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f);
-        if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+        if (mode == MODE_STEP) {   // MODE_STEP_NODECIDE: the next step's kernel decides
+          const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
+          const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, &cur, k_new + static_cast<size_t>(u) * DH,
+                                             v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f);
+          if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+        }
         const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
         if (prev == need_of(u) - 1) push_merge(u);
       }
@@ -1072,8 +1077,10 @@ __global__ void __launch_bounds__(128) append_kernel(const LayerArgs a, const T*
     commit_warp<T>(a, u, N, ntk_after, r, kn, vn, en);
     __threadfence();
     __syncwarp();
-    const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, nullptr, kn, vn, en);
-    if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+    if (!a.mlstm) {   // the mLSTM scorer decides in the next step's own kernel
+      const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, nullptr, kn, vn, en);
+      if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+    }
   }
   // last warp of the launch advances the layer counters
   __syncwarp();
@@ -1099,9 +1106,11 @@ __global__ void __launch_bounds__(128) decide_kernel(const LayerArgs a, int N, i
     a.layer->ticket = 0;
   }
   if (u >= a.units) return;
-  const Decision r = decide_warp<T>(a, u, N, ntk, nullptr, nullptr, nullptr, 0.f);
+  if (!a.mlstm) {   // the mLSTM scorer decides in the step's own kernel
+    const Decision r = decide_warp<T>(a, u, N, ntk, nullptr, nullptr, nullptr, 0.f);
+    if (lane == 0) a.dec[static_cast<size_t>(N & 1) * a.units + u] = r;
+  }
   if (lane == 0) {
-    a.dec[static_cast<size_t>(N & 1) * a.units + u] = r;
     a.state[4 * u + 0] = N;
     a.state[4 * u + 1] = ntk;
   }

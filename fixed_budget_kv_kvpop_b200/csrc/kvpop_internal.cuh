@@ -43,6 +43,12 @@ enum : int32_t {
 
 constexpr int kMaxSeg = 64;         // split-K partials per unit (upper bound)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
+// Bound of the decode kernel's merge-queue waits (shared memory only, no copy
+// in flight).  Test builds shorten it to make such a wait run out quickly.
+#ifndef KVPOP_MERGE_WAIT_LIMIT_NS
+#define KVPOP_MERGE_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kMergeWaitLimitNs = KVPOP_MERGE_WAIT_LIMIT_NS;
 
 // Per-layer counters shared by all units (all batch rows share one length).
 struct LayerState {
@@ -81,7 +87,27 @@ struct LayerArgs {
   uint32_t flags;
   int row_bytes;        // 2 * d * sizeof(T)
   const float* log_decay;   // this layer's ln(gamma) [Hkv], or null (no temporal decay)
+  // Stateful mLSTM scorer (page §A, §E.3, §E.4); mlstm = 0 when the stateless
+  // scorer or caller scores decide.
+  int mlstm;            // 1: each step's decision waits for the step's own token
+  int mp, mdv;          // Hedgehog projection size p (2p features), value size dv
+  const float* mw;      // this layer's weights [Hkv][mlstm_head_floats(p, dv, d)]
+  double* mstate;       // this layer's states [units][mlstm_state_doubles(p, dv)]
+  int test_hook;        // failure injection, honoured only by builds with KVPOP_TEST_HOOKS
 };
+
+// test_hook values (KVPOP_TEST_HOOKS builds): consumer warp 0 of CTA 0 does
+// its work but never reports that it is done, so the CTA's merge helpers wait
+// until kMergeWaitLimitNs and record DEVERR_TIMEOUT.
+constexpr int TEST_HOOK_WITHHOLD_DONE = 1;
+
+// mLSTM weights of one (layer, KV head): rows of 2d floats W_q [p], W_k [p],
+// W_v [dv], w_i, w_f; then w_o [dv], b_i, b_f, b_o, padded to 4 floats.
+__host__ __device__ __forceinline__ int mlstm_head_floats(int p, int dv, int d) {
+  return (2 * p + dv + 2) * 2 * d + ((dv + 3 + 3) / 4) * 4;
+}
+// State of one unit, fp64: C [2p][dv] (feature-major), n [2p], m, pad.
+__host__ __device__ __forceinline__ int mlstm_state_doubles(int p, int dv) { return 2 * p * dv + 2 * p + 2; }
 
 // Scorer weights of KV head h in this layer: W1 rows (one row for the linear
 // scorer), b1 and w2 (null for the linear scorer).
@@ -379,9 +405,11 @@ struct DecodeScratch {
 };
 
 // Kernel launchers (defined in the .cu files).
-enum DecodeMode : int { MODE_STEP = 0, MODE_ATTEND = 1 };
-// One fused decode step (MODE_STEP) or attention over the cache as it stands
-// (MODE_ATTEND).  ext_score may be null.
+enum DecodeMode : int { MODE_STEP = 0, MODE_ATTEND = 1, MODE_STEP_NODECIDE = 2 };
+// One fused decode step (MODE_STEP), the same step taking its decision from a
+// kernel launched just before it instead of deciding the next step
+// (MODE_STEP_NODECIDE, the mLSTM scorer), or attention over the cache as it
+// stands (MODE_ATTEND).  ext_score may be null.
 int launch_decode(const CUtensorMap& tmap, const LayerArgs& a, int dtype, const DecodeScratch& sc, int mode,
                   const void* q, const void* k_new, const void* v_new, const float* ext_score, void* out, int num_sms,
                   cudaStream_t st);
@@ -403,5 +431,15 @@ struct PrefillScratch {
 int launch_prefill(const LayerArgs& a, int dtype, const PrefillScratch& ps, const void* k, const void* v,
                    int n_tokens, int n_seen_before, int n_topk_before, const float* ext_scores,
                    cudaStream_t st);
+
+// mLSTM scorer (kvpop_mlstm.cu).  Decode: updates every unit's state with the
+// step's token and writes the step's eviction decision (dec[N & 1]) for the
+// decode kernel that follows in MODE_STEP_NODECIDE.  Prefill: runs the
+// recurrence over the chunk of tokens [n0, n0 + n) and writes the ranking
+// priority of every token that becomes eligible in it into
+// out[u * cap + (t - e0)].  Both return 0 or -1 (launch failed).
+int launch_mlstm_step(const LayerArgs& a, int dtype, const void* k_new, const void* v_new, cudaStream_t st);
+int launch_mlstm_prefill(const LayerArgs& a, int dtype, const void* k, const void* v, int n, int n0, int e0,
+                         float* out, int cap, cudaStream_t st);
 
 }  // namespace kvpop

@@ -568,7 +568,8 @@ int launch_prefill_t(const LayerArgs& a, const PrefillScratch& ps, const T* k, c
   cg.c0 = c0;
   const int n_new = cg.e1 - cg.e0;
   if (n_new > ps.cap) return -2;
-  const int r = launch_scores_t<T>(a, cg, k, v, n, ext, ps.new_score, ps.cap, st);
+  const int r = a.mlstm ? launch_mlstm_prefill(a, sizeof(T) == 4 ? 0 : 1, k, v, n, n0, cg.e0, ps.new_score, ps.cap, st)
+                        : launch_scores_t<T>(a, cg, k, v, n, ext, ps.new_score, ps.cap, st);
   if (r != 0) return r;
   select_kernel<T><<<a.units, kSelThreads, 0, st>>>(a, cg, k, v, n, ps.new_score, ps.cap, ps.tgt);
   if (a.D > 0) move_kernel<T><<<a.units, 256, 0, st>>>(a, cg);

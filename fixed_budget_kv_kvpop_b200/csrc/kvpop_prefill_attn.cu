@@ -780,6 +780,7 @@ int launch_place_kept(const LayerArgs& a, int dtype, const PrefillAttnPlan& p, c
 
 int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan* p) {
   if (n < 0 || kPaRows % a.G != 0) return -2;
+  if (a.mlstm) return -2;   // the prompt scores come from the stateless scorers or the caller
   if (a.d != 64 && a.d != 128) return -2;
   PrefillAttnPlan P{};
   P.n = n;

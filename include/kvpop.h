@@ -60,6 +60,15 @@ extern "C" {
 #define KVPOP_DTYPE_F32 0
 #define KVPOP_DTYPE_BF16 1
 
+/* Scorer kinds (kvpop_config.scorer_kind). */
+#define KVPOP_SCORER_MLP 0    /* stateless MLP, or the linear scorer when scorer_hidden = 0 (page §E.2) */
+#define KVPOP_SCORER_MLSTM 1  /* stateful mLSTM scorer with delayed readout (page §A, §E.3, §E.4) */
+
+/* Floats of one (layer, KV head) block of kvpop_config.mlstm_w: rows of 2d
+ * weights W_q (p rows), W_k (p), W_v (dv), w_i, w_f, then w_o (dv), b_i, b_f,
+ * b_o, padded to a multiple of 4. */
+#define KVPOP_MLSTM_HEAD_FLOATS(p, dv, d) ((2 * (p) + (dv) + 2) * 2 * (d) + (((dv) + 3 + 3) / 4) * 4)
+
 /* Flags. */
 #define KVPOP_FLAG_EXTERNAL_SCORES 1u /* caller supplies every token's score instead of the MLP */
 #define KVPOP_FLAG_DEBUG_CHECKS 2u    /* kernels check slot bookkeeping and NaN scores */
@@ -108,6 +117,28 @@ typedef struct kvpop_config {
    * formed once in fp32 (one rounding, like fmaf), and stores p_j as the
    * long-range slots' scores.  Requires max_context <= 2^24. */
   const float* log_decay;
+  /* Scorer kind: KVPOP_SCORER_MLP (w1/b1/w2/b2 above) or KVPOP_SCORER_MLSTM
+   * (the fields below; w1/b1/w2/b2 and scorer_hidden are then unused).  The
+   * mLSTM scorer (page §A "Background: Linear Attention and mLSTM", §E.3
+   * "mLSTM Scorer", §E.4 "Delayed Readout"): per KV head a recurrent state
+   * (matrix memory C [2p][dv], normaliser n [2p], stabiliser m) in fp64 in
+   * the cache buffer, updated by every token t with x_t = [k_t; v_t]:
+   *   phi_t = [softmax(W_k x_t); softmax(-W_k x_t)] (Hedgehog feature map),
+   *   i~ = w_i . x_t + b_i, log f = log sigmoid(w_f . x_t + b_f),
+   *   m' = max(log f + m, i~), C' = e^(log f + m - m') C + e^(i~ - m') phi_t (W_v x_t)^T,
+   *   n' = e^(log f + m - m') n + e^(i~ - m') phi_t;
+   * the token u that becomes eligible at step q = u + W + D is read out from
+   * the state after token q with r = Hedgehog(W_q x_u):
+   *   h = C^T r / max(|n . r|, e^-m),  score = w_o . SiLU(h) + b_o,
+   * rounded once to fp32.  Each decode step updates the state with the new
+   * token before deciding the boundary token, so the decision is taken in
+   * the step itself (one extra small launch per layer and step).  The
+   * prefill attention calls do not take this scorer (KVPOP_ERR_BAD_SHAPE). */
+  int32_t scorer_kind;
+  int32_t mlstm_p;        /* Hedgehog projection size p, 1..16 (2p features) */
+  int32_t mlstm_dv;       /* value size dv, 1..32 */
+  const float* mlstm_w;   /* device fp32 [L][Hkv][KVPOP_MLSTM_HEAD_FLOATS(p, dv, d)], 16-byte aligned,
+                             borrowed for the handle's lifetime (may be NULL with KVPOP_FLAG_EXTERNAL_SCORES) */
 } kvpop_config;
 
 typedef struct kvpop_handle kvpop_handle;
@@ -321,6 +352,16 @@ int kvpop_clear_error(kvpop_handle* h, void* stream);
  * error word on `stream`, so host-side failure handling can be exercised
  * without making any kernel fail. */
 int kvpop_debug_poison_error(kvpop_handle* h, int32_t bits, void* stream);
+
+/* Test hook (no passage of the pages defines it), honoured only by builds of
+ * this library compiled with KVPOP_TEST_HOOKS, which also shorten the decode
+ * kernel's merge-queue waits; other builds return KVPOP_ERR_INVALID_ARG and
+ * change nothing.  hook = 1: in every later decode step, one consumer warp
+ * finishes its work but never reports that it is done, so its CTA's merge
+ * helpers wait until their bound runs out and the error word records
+ * KVPOP_DEVERR_TIMEOUT (the kernel still returns; no copy is in flight
+ * during that wait).  hook = 0 turns it off. */
+int kvpop_debug_set_hook(kvpop_handle* h, int32_t hook);
 
 /* Releases the handle's host state.  Does not touch the device buffer.
  * Resource management of this library; no passage of the pages defines it.

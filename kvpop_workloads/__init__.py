@@ -196,6 +196,42 @@ def scorer_weights(w: Workload, master: int = 0, device="cpu"):
     return w1.contiguous(), b1, w2.contiguous(), b2
 
 
+def mlstm_weights(w: Workload, p: int = 16, dv: int = 16, master: int = 0, device="cpu"):
+    """Seeded weights of the stateful mLSTM scorer, packed per (layer, KV head)
+    as the C ABI takes them: fp32 [L][Hkv][(2p + dv + 2) * 2d + pad] holding
+    the rows W_q [p], W_k [p], W_v [dv], w_i, w_f (each 2d long), then w_o
+    [dv], b_i, b_f, b_o and zero padding to a multiple of 4.
+
+    Reading of the recipe (the pages give no trained weights): W_q, W_k, W_v
+    and w_o ~ N(0, 0.1^2); w_i, w_f ~ N(0, 0.05^2); b_i = 0, b_f = 3 (a
+    forget gate near sigmoid(3) = 0.95, the stable early memory the page's
+    §E.5 initialisation aims at); b_o = 0."""
+    L, H, d2 = w.n_layers, w.n_kv_heads, 2 * w.head_dim
+    rows = 2 * p + dv + 2
+    tail = ((dv + 3 + 3) // 4) * 4
+    g = _gen(device, master, w.name, "mlstm", p, dv)
+    mat = _normal((L, H, rows, d2), g, device)
+    scale = torch.full((rows,), 0.1, device=device)
+    scale[2 * p + dv:] = 0.05
+    mat = mat * scale[:, None]
+    t = torch.zeros((L, H, tail), device=device)
+    t[..., :dv] = _normal((L, H, dv), g, device) * 0.1
+    t[..., dv + 1] = 3.0
+    return torch.cat([mat.reshape(L, H, rows * d2), t], dim=-1).contiguous()
+
+
+def unpack_mlstm(packed_head, p: int, dv: int, d: int) -> dict:
+    """One (layer, KV head) block of mlstm_weights as named float64 numpy
+    arrays: wq, wk [p][2d], wv [dv][2d], wi, wf [2d], wo [dv]; bi, bf, bo."""
+    x = packed_head.double().cpu().numpy()
+    d2 = 2 * d
+    rows = 2 * p + dv + 2
+    m = x[:rows * d2].reshape(rows, d2)
+    t = x[rows * d2:]
+    return {"wq": m[:p], "wk": m[p:2 * p], "wv": m[2 * p:2 * p + dv], "wi": m[2 * p + dv], "wf": m[2 * p + dv + 1],
+            "wo": t[:dv], "bi": float(t[dv]), "bf": float(t[dv + 1]), "bo": float(t[dv + 2])}
+
+
 def external_scores(w: Workload, layer: int, n_tokens: int, master: int = 0, device="cpu",
                     tag: str = "ext", tie_levels: int = 0):
     """Caller-supplied per-token scores [b][Hkv][n] (fp32).

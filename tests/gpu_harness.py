@@ -38,14 +38,19 @@ class Run:
     weights: Optional[tuple] = None
     cache: object = None
     log_decay: Optional[np.ndarray] = None   # [L][Hkv] ln gamma, or None
+    mlstm: Optional[tuple] = None            # (packed device weights, p, dv) of the mLSTM scorer, or None
 
 
 def build_cache(w: wl.Workload, n_layers: int, external: bool, weights=None, max_chunk=None, debug=True,
-                log_decay=None):
+                log_decay=None, mlstm=None, library=None):
     import fixed_budget_kv_kvpop_b200 as kp
     keep = ()
     kw = {}
-    if not external:
+    if mlstm is not None:
+        packed, p, dv = mlstm
+        kw = dict(scorer="mlstm", mlstm_p=p, mlstm_dv=dv, mlstm_w=packed)
+        keep = (packed,)
+    elif not external:
         w1, b1, w2, b2 = weights
         kw = dict(w1=w1, b1=b1, w2=w2, b2=b2)
         keep = weights
@@ -56,29 +61,37 @@ def build_cache(w: wl.Workload, n_layers: int, external: bool, weights=None, max
                          debug_checks=debug, log_decay=log_decay, **kw)
     if log_decay is not None:
         keep = tuple(keep) + (log_decay,)
-    return kp.KVPopCache(cfg, device="cuda", keepalive=keep)
+    return kp.KVPopCache(cfg, device="cuda", keepalive=keep, library=library)
 
 
 def run_gpu(w: wl.Workload, n_layers: int, n_steps: int, *, external: bool = False, chunks=None,
             inspect_every: int = 1, layers_to_keep: Sequence[int] = (0,), tie_levels: int = 0,
             master: int = 0, gen_device: str = "cpu", debug=True, split: bool = False,
-            log_decay: Optional[np.ndarray] = None) -> Run:
+            log_decay: Optional[np.ndarray] = None, mlstm_dims: Optional[tuple] = None, library=None,
+            step_hook=None) -> Run:
     """Prefill + n_steps decode steps of every layer on the GPU, through the C ABI.
-    log_decay: optional float32 [n_layers][Hkv] ln gamma (temporal decay)."""
+    log_decay: optional float32 [n_layers][Hkv] ln gamma (temporal decay).
+    mlstm_dims: (p, dv) to score with the stateful mLSTM scorer instead of the MLP.
+    library: another build of libkvpop (load_library); step_hook(cache, i, when)
+    is called with when = "before" / "after" around decode step i."""
     dev = "cuda"
     weights = None
-    if not external:
+    mlstm = None
+    if mlstm_dims is not None:
+        p_, dv_ = mlstm_dims
+        mlstm = (wl.mlstm_weights(w.replace(n_layers=n_layers), p_, dv_, master=master).to(dev), p_, dv_)
+    elif not external:
         # scorer_hidden 0 = linear scorer: one weight row per head (w1[..., 0, :]) and b2
         wshape = w.replace(n_layers=n_layers, scorer_hidden=max(w.scorer_hidden, 1))
         weights = tuple(t.to(dev) for t in wl.scorer_weights(wshape, master=master))
     chunks = list(chunks) if chunks else ([w.prefill] if w.prefill > 0 else [])
     dec_dev = None if log_decay is None else torch.tensor(np.asarray(log_decay, np.float32), device=dev)
     cache = build_cache(w, n_layers, external, weights, max_chunk=max(chunks) if chunks else 1, debug=debug,
-                        log_decay=dec_dev)
+                        log_decay=dec_dev, mlstm=mlstm, library=library)
     run = Run(w=w, layers=list(layers_to_keep), prompt_k={}, prompt_v={}, dec_q={}, dec_k={}, dec_v={},
               outs={}, slot_pos={}, slot_score={}, ext_prompt={} if external else None,
               ext_dec={} if external else None, weights=weights, cache=cache,
-              log_decay=None if log_decay is None else np.asarray(log_decay, np.float32))
+              log_decay=None if log_decay is None else np.asarray(log_decay, np.float32), mlstm=mlstm)
     for layer in range(n_layers):
         k, v = wl.prompt_kv(w, layer, master=master, device=gen_device)
         k, v = k.to(dev), v.to(dev)
@@ -106,6 +119,8 @@ def run_gpu(w: wl.Workload, n_layers: int, n_steps: int, *, external: bool = Fal
         else:
             del k, v
     for i in range(n_steps):
+        if step_hook is not None:
+            step_hook(cache, i, "before")
         for layer in range(n_layers):
             q, kn, vn = wl.decode_inputs(w, layer, i, master=master, device=gen_device)
             q, kn, vn = q.to(dev), kn.to(dev), vn.to(dev)
@@ -133,6 +148,8 @@ def run_gpu(w: wl.Workload, n_layers: int, n_steps: int, *, external: bool = Fal
                 else:
                     run.slot_pos[layer].append(None)
                     run.slot_score[layer].append(None)
+        if step_hook is not None:
+            step_hook(cache, i, "after")
     torch.cuda.synchronize()
     st, bits = cache.get_error()
     assert st == 0, f"device error status {st} bits {bits}"
@@ -162,6 +179,10 @@ def unit_scores(run: Run, layer: int, unit: int, k_all, v_all):
         pr = run.ext_prompt[layer][b, h].double().cpu().numpy()
         dc = np.array([t[b, h].item() for t in run.ext_dec[layer]], dtype=np.float64)
         s = orc.ranking_score(np.concatenate([pr, dc]))
+    elif run.mlstm is not None:
+        packed, p_, dv_ = run.mlstm
+        P = orc.MlstmParams(**wl.unpack_mlstm(packed[layer, h], p_, dv_, w.head_dim))
+        s = orc.unit_scores_mlstm(k_all, v_all, P, w.sinks, w.window, w.delay)
     else:
         w1, b1, w2, b2 = (t.double().cpu().numpy() for t in run.weights)
         if w.scorer_hidden == 0:
@@ -174,7 +195,11 @@ def unit_scores(run: Run, layer: int, unit: int, k_all, v_all):
 
 
 def score_tol(s_ref: np.ndarray, all_scores: np.ndarray) -> np.ndarray:
-    rms = float(np.sqrt(np.mean(np.square(all_scores)))) if all_scores.size else 0.0
+    """|ds| allowed per token: 1e-4 of max(|s|, 1e-2 RMS of the unit's scores).
+    Tokens without a score (NaN: not yet eligible under a delayed readout)
+    are left out of the RMS."""
+    fin = all_scores[np.isfinite(all_scores)]
+    rms = float(np.sqrt(np.mean(np.square(fin)))) if fin.size else 0.0
     return SCORE_RTOL * np.maximum(np.abs(s_ref), 1e-2 * rms)
 
 
