@@ -133,6 +133,7 @@ struct PaArgs {
   const int32_t* cut;
   int n, S, W, D, G, Hq, Hkv, qt, cand_cap;
   float scale_log2;   // log2(e) / sqrt(d): logits in base-2 units
+  int32_t* err;       // device error word (bounded waits that give up)
 };
 
 template <typename T> struct PaIo;
@@ -695,6 +696,355 @@ __global__ void __launch_bounds__(kMmaThreads, 2) sparse_attn_mma_kernel(PaArgs 
   }
 }
 
+
+// ---------------- bf16 attention on the 5th-generation tensor cores ----------------
+// One CTA of 4 warps per (unit, 128 / G query positions): thread t owns query
+// row t, which is also TMEM lane t.  Per tile of kTcKeys candidate keys:
+//   1. all threads gather the tile's K and V rows with cp.async into shared
+//      memory (one tile ahead, two stages);
+//   2. one thread issues S = Q K^T as tcgen05.mma (bf16 operands from shared
+//      memory, fp32 accumulator in TMEM, M = 128, N = kTcKeys, K = 16 per
+//      instruction) and commits it to an mbarrier;
+//   3. every thread loads its row of S from TMEM (tcgen05.ld), applies the
+//      running top-k mask and an exp2-domain online softmax (the running max
+//      moves only when a tile exceeds it by 2^8; the O row in TMEM is then
+//      rescaled by tcgen05.ld / st), and writes its row of P (bf16) to shared
+//      memory;
+//   4. one thread issues O += P V (M = 128, N = d, K = 16 per instruction)
+//      into the TMEM accumulator.
+// Operands use the canonical no-swizzle layout: 16-byte cells stored
+// chunk-major ([16-byte chunk][row]), so every 8 x 16-byte core matrix is
+// 128 contiguous bytes.  K-major (Q, K, P): leading offset = the chunk stride,
+// stride offset = 128 bytes (8 rows).  V is the MN-major B operand of P V:
+// stride offset = the chunk stride (8 more dims), leading offset = 128 bytes
+// (8 more keys).  Two CTAs share an SM (shared memory and 2 x 256 TMEM
+// columns), so one CTA's softmax overlaps the other's MMAs.
+constexpr int kTcThreads = 128;
+constexpr int kTcKeys = 32;
+constexpr int kTcRows = 128;
+constexpr uint32_t kTcCols = 256;          // TMEM columns per CTA: S at 0, O at 128
+constexpr size_t kTcMinSmem = 80 * 1024;   // keeps at most two CTAs (2 x 256 TMEM columns) per SM
+constexpr float kTcLazy = 8.0f;            // lazy rescale threshold (log2 units)
+
+template <int DH>
+struct TcSmem {
+  static constexpr int QCH = DH / 8;                                   // 16-byte chunks per row
+  static constexpr size_t Q_OFF = 0;                                   // [QCH][kTcRows] cells
+  static constexpr size_t KV_TILE = static_cast<size_t>(QCH) * kTcKeys * 16;   // [QCH][kTcKeys] cells
+  static constexpr size_t KV_OFF = Q_OFF + static_cast<size_t>(QCH) * kTcRows * 16;   // [stage][K, V]
+  static constexpr size_t P_OFF = KV_OFF + 4 * KV_TILE;                // [kTcKeys / 8][kTcRows] cells
+  static constexpr size_t META_OFF = P_OFF + static_cast<size_t>(kTcKeys / 8) * kTcRows * 16;
+  static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * (4 * kTcKeys + 4);
+  static constexpr size_t TADDR_OFF = BAR_OFF + 16;
+  static constexpr size_t WT_OFF = TADDR_OFF + 16;
+  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);
+  static_assert(BAR_OFF % 8 == 0 && KV_OFF % 16 == 0 && P_OFF % 16 == 0, "shared-memory alignment");
+  static size_t bytes(int cand_cap) {
+    const size_t b = CAND_OFF + sizeof(int) * static_cast<size_t>(cand_cap);
+    return b > kTcMinSmem ? b : kTcMinSmem;
+  }
+};
+
+// Shared-memory matrix descriptor, no swizzle (start, leading and stride
+// byte offsets in 16-byte units; descriptor version 1).
+__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, M x N,
+// B K-major (b_mn = 0) or MN-major (b_mn = 1), A K-major.
+__host__ __device__ constexpr uint32_t tc_idesc(int M, int N, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               :: "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      :: "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+         "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])),
+         "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+         "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+         "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+         "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+         "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+         "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+         "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+         "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kTcThreads) sparse_attn_tc_kernel(PaArgs p) {
+  using SM = TcSmem<DH>;
+  constexpr int QCH = SM::QCH;
+  constexpr uint32_t kIdescS = tc_idesc(kTcRows, kTcKeys, 0);
+  constexpr uint32_t kIdescPV = tc_idesc(kTcRows, DH, 1);
+  constexpr uint32_t kRowCells = kTcRows * 16;   // bytes of one chunk column of Q or P
+  constexpr uint32_t kKeyCells = kTcKeys * 16;   // bytes of one chunk column of a K or V tile
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  int* kpos = reinterpret_cast<int*>(smem_raw + SM::META_OFF);   // [2][kTcKeys]
+  int* kcut = kpos + 2 * kTcKeys;                                  // [2][kTcKeys]
+  int* tfull = kcut + 2 * kTcKeys;                                 // [2]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + SM::BAR_OFF);
+  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_raw + SM::TADDR_OFF);
+  int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
+  int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int u = blockIdx.y;
+  const int b = u / p.Hkv, hk = u % p.Hkv;
+  const int n = p.n, S = p.S, WD = p.W + p.D, G = p.G;
+  const int q0 = blockIdx.x * p.qt;
+  const int q1 = min(n, q0 + p.qt);
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
+  const __nv_bfloat16* kgp = static_cast<const __nv_bfloat16*>(p.k) + static_cast<size_t>(u) * n * DH;
+  const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
+  const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(taddr_s)), "r"(kTcCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  // query rows (row = position offset * G + head), zero beyond the prompt
+  for (int c = tid; c < kTcRows * QCH; c += kTcThreads) {
+    const int row = c / QCH, ch = c % QCH;
+    const int qpos = q0 + row / G, g = row % G;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (qpos < q1)
+      x = *reinterpret_cast<const uint4*>(qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos) * DH + ch * 8);
+    *reinterpret_cast<uint4*>(smem_raw + SM::Q_OFF + (static_cast<size_t>(ch) * kTcRows + row) * 16) = x;
+  }
+  fence_proxy_async_smem();   // Q (generic-proxy stores) is read by the tensor cores
+  const int count = gather_candidates<kTcThreads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *taddr_s;
+  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;   // this warp's TMEM lanes
+  const int ntiles = (count + kTcKeys - 1) / kTcKeys;
+  const int m1 = q1 - 1 - WD;
+
+  // gather tile t into stage t & 1: K and V rows (16-byte cells, zero past the
+  // candidates) and the keys' positions and cutoffs
+  auto issue = [&](int t) {
+    const int st = t & 1;
+    const uint32_t kbase = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
+    const uint32_t vbase = kbase + static_cast<uint32_t>(SM::KV_TILE);
+    for (int i = tid; i < kTcKeys * QCH; i += kTcThreads) {
+      const int key = i / QCH, ch = i % QCH;
+      const int idx = t * kTcKeys + key;
+      const int j = idx < count ? cand[idx] : -1;
+      const size_t off = j >= 0 ? static_cast<size_t>(j) * DH + ch * 8 : 0;
+      const uint32_t so = static_cast<uint32_t>((ch * kTcKeys + key) * 16);
+      cp_async16(kbase + so, kgp + off, j >= 0 ? 16 : 0);
+      cp_async16(vbase + so, vgp + off, j >= 0 ? 16 : 0);
+    }
+    cp_async_commit();
+    if (tid < kTcKeys) {
+      const int idx = t * kTcKeys + tid;
+      const int j = idx < count ? cand[idx] : -1;
+      const int c = j >= 0 ? cu[j] : 0;
+      kpos[st * kTcKeys + tid] = j;
+      kcut[st * kTcKeys + tid] = c;
+      const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
+      const unsigned bal = __ballot_sync(0xffffffffu, full);
+      if (lane == 0) tfull[st] = (bal == 0xffffffffu);
+    }
+  };
+
+  const int row = tid;
+  const int qpos = q0 + row / G;
+  const bool vrow = qpos < q1;
+  const int mrow = qpos - WD;
+  float m_run = -INFINITY, l_run = 0.f;
+  uint32_t phase = 0;
+  bool failed = false;
+
+  if (ntiles > 0) issue(0);
+  for (int t = 0; t < ntiles; ++t) {
+    const int st = t & 1;
+    if (t + 1 < ntiles) {
+      issue(t + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    fence_proxy_async_smem();   // this thread's cp.async rows -> the tensor cores' view
+    __syncthreads();
+    const uint32_t kt = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
+    const uint32_t vt = kt + static_cast<uint32_t>(SM::KV_TILE);
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < DH / 16; ++ks)
+        tc_mma(tS, tc_desc(sbase + static_cast<uint32_t>(SM::Q_OFF) + ks * 2 * kRowCells, kRowCells, 128),
+               tc_desc(kt + ks * 2 * kKeyCells, kKeyCells, 128), kIdescS, ks > 0 ? 1u : 0u);
+      tc_commit(bar);
+    }
+    bool ok = mbar_wait(bar, phase);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+    float s[32];
+    tc_ld32(tS + lrow, s);
+
+    // running top-k mask, base-2 logits, online softmax with lazy rescaling
+    float tmax = -INFINITY;
+    if (tfull[st]) {
+#pragma unroll
+      for (int i = 0; i < kTcKeys; ++i) {
+        s[i] = vrow ? s[i] * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, s[i]);
+      }
+    } else {
+      const int* kp = kpos + st * kTcKeys;
+      const int* kc = kcut + st * kTcKeys;
+#pragma unroll
+      for (int i = 0; i < kTcKeys; ++i) {
+        const int j = kp[i];
+        const bool vis = j >= 0 && vrow && j <= qpos && (j < S || j > mrow || kc[i] > mrow);
+        s[i] = vis ? s[i] * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, s[i]);
+      }
+    }
+    float alpha = 1.f;
+    bool resc = false;
+    if (tmax > m_run + kTcLazy) {
+      resc = (m_run != -INFINITY);   // an O row that has seen no key is still zero
+      alpha = resc ? exp2f(m_run - tmax) : 0.f;
+      l_run *= alpha;
+      m_run = tmax;
+    }
+    float psum = 0.f;
+    uint32_t pk[kTcKeys / 2];
+#pragma unroll
+    for (int i = 0; i < kTcKeys; i += 2) {
+      const float p0 = s[i] == -INFINITY ? 0.f : exp2f(s[i] - m_run);
+      const float p1 = s[i + 1] == -INFINITY ? 0.f : exp2f(s[i + 1] - m_run);
+      psum += p0 + p1;
+      pk[i / 2] = pack_bf16(p0, p1);
+    }
+    l_run += psum;
+#pragma unroll
+    for (int c = 0; c < kTcKeys / 8; ++c)
+      *reinterpret_cast<uint4*>(smem_raw + SM::P_OFF + (static_cast<size_t>(c) * kTcRows + row) * 16) =
+          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+    if (__any_sync(0xffffffffu, resc)) {   // tcgen05.ld / st are warp-collective
+      const float f = resc ? alpha : 1.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float o[32];
+        tc_ld32(tO + lrow + c0, o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= f;
+        tc_st32(tO + lrow + c0, o);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    fence_proxy_async_smem();   // P (generic-proxy stores) is read by the tensor cores
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kTcKeys / 16; ++kk)
+        tc_mma(tO, tc_desc(sbase + static_cast<uint32_t>(SM::P_OFF) + kk * 2 * kRowCells, kRowCells, 128),
+               tc_desc(vt + kk * 256, 128, kKeyCells), kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+      tc_commit(bar);
+    }
+    ok = mbar_wait(bar, phase);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+  }
+
+  if (failed) {
+    if (tid == 0) set_error(p.err, DEVERR_TIMEOUT);
+    cp_async_wait<0>();
+  } else if (ntiles > 0) {
+    // epilogue: O row / l, bf16, to the output; the row's log-normaliser.
+    // Every thread takes part in the (warp-collective) TMEM loads; rows past
+    // the prompt store nothing.
+    const int g = row % G;
+    const size_t rowi = (static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (vrow ? qpos : 0);
+    __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out) + rowi * DH;
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < DH; c0 += 32) {
+      float o[32];
+      tc_ld32(tO + lrow + c0, o);
+      if (vrow) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(og + c0 + 8 * c) =
+              make_uint4(pack_bf16(o[8 * c] * inv, o[8 * c + 1] * inv), pack_bf16(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
+                         pack_bf16(o[8 * c + 4] * inv, o[8 * c + 5] * inv), pack_bf16(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+      }
+    }
+    if (vrow && p.lse != nullptr) p.lse[rowi] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTcCols) : "memory");
+  }
+}
+
+template <int DH>
+int launch_attn_tc(const PaArgs& pa, int units, int n, cudaStream_t st) {
+  const size_t smem = TcSmem<DH>::bytes(pa.cand_cap);
+  if (cudaFuncSetAttribute(sparse_attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return -1;
+  dim3 grid((n + pa.qt - 1) / pa.qt, units);
+  sparse_attn_tc_kernel<DH><<<grid, kTcThreads, smem, st>>>(pa);
+  return 0;
+}
+
 template <int DH>
 int launch_attn_f32(const PaArgs& pa, int units, int n, cudaStream_t st) {
   const size_t smem = PaSmem<DH>::bytes(pa.cand_cap);
@@ -847,11 +1197,12 @@ int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPla
   pa.qt = p.qt;
   pa.cand_cap = p.cand_cap;
   pa.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.d));
+  pa.err = a.err;
   int r;
   if (dtype == 0)
     r = (a.d == 128) ? launch_attn_f32<128>(pa, a.units, p.n, st) : launch_attn_f32<64>(pa, a.units, p.n, st);
   else
-    r = (a.d == 128) ? launch_attn_bf16<128>(pa, a.units, p.n, st) : launch_attn_bf16<64>(pa, a.units, p.n, st);
+    r = (a.d == 128) ? launch_attn_tc<128>(pa, a.units, p.n, st) : launch_attn_tc<64>(pa, a.units, p.n, st);
   if (r != 0) return r;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
