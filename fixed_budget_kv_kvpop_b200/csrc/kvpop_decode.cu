@@ -213,49 +213,77 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
     if (!from_input && pos[rslot] != b) set_error(a.err, DEVERR_STATE_MISMATCH);
     if (sb != sb) set_error(a.err, DEVERR_NAN_SCORE);
   }
-  if (ntk < K) {
-    r.tgt = base + ntk;     // fill-up: next free long-range slot, nobody leaves
-    r.evict = -1;
-  } else if (K == 0) {
-    r.evict = r.bslot;
-  } else {
-    // block argmin of the long-range keys (keys are unique: positions are)
-    uint64_t best = ~0ull;
-    int mslot = -1;
-    for (int i0 = 0; i0 < K; i0 += 32 * kB) {
-      float sc[kB];
-      int32_t ps[kB];
-#pragma unroll
-      for (int t = 0; t < kB; ++t) {
-        const int i = i0 + lane + 32 * t;
-        if (i < K) { sc[t] = score[base + i]; ps[t] = pos[base + i]; }
-      }
-#pragma unroll
-      for (int t = 0; t < kB; ++t) {
-        const int i = i0 + lane + 32 * t;
-        if (i < K) {
-          const int sl = base + i;
-          const uint64_t key = (pending != nullptr && sl == pending->tgt) ? rank_key(pending->sb, pending->bpos)
-                                                                          : rank_key(sc[t], ps[t]);
-          if (key < best) { best = key; mslot = sl; }
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const uint64_t ok = __shfl_xor_sync(0xffffffffu, best, o);
-      const int os = __shfl_xor_sync(0xffffffffu, mslot, o);
-      if (ok < best) { best = ok; mslot = os; }
-    }
-    if (rank_key(sb, b) > best) {
-      r.tgt = mslot;
-      r.evict = mslot;
-    } else {
-      r.evict = r.bslot;
-    }
-  }
+  longrange_decide(a, u, ntk, pending, sb, b, r);
   return r;
 }
+
+#ifdef KVPOP_DECIDE_EARLY_ARRIVE
+// The decode kernel's deciders take the next step's decision in two halves,
+// so that a unit's merge (which commits this step's row moves) need not wait
+// for the next decision's scorer and argmin.  decide_load reads what the
+// commit can overwrite -- the next boundary token's row, or its caller score
+// -- into registers; decide_finish scores it and runs the argmin, whose only
+// slot the commit changes (the pending target) counts with the pending key.
+template <int DH>
+struct DecideInput {
+  double x[2 * DH / 32];   // this lane's scorer inputs
+  float sext;              // caller score
+  int b;                   // boundary token position, -1: none
+};
+
+template <typename T, int DH>
+__device__ __noinline__ void decide_load(const LayerArgs& a, int u, int N, const T* kn, const T* vn, float ext_new,
+                                         DecideInput<DH>& in) {
+  const int lane = threadIdx.x & 31;
+  const int S = a.S, W = a.W, D = a.D, NS = a.NS;
+  const int b = N - W - D;
+  in.b = -1;
+  in.sext = 0.f;
+  if (b < S) return;
+  in.b = b;
+  // before the pending commit: b is the token appended by that step (W = 1,
+  // D = 0), or still in its window slot (D <= 1), or in its staging slot
+  const bool from_input = (b == N - 1);
+  const int rslot = from_input ? -1 : (D <= 1 ? window_slot(b, S, W) : staging_slot(b, S, W, D));
+  const T* kv = reinterpret_cast<const T*>(a.kv + static_cast<size_t>(u) * NS * a.row_bytes);
+  const T* krow = from_input ? kn : kv + static_cast<size_t>(rslot) * (2 * DH);
+  const T* vrow = from_input ? vn : krow + DH;
+  if (a.flags & FLAG_EXTERNAL_SCORES)
+    in.sext = from_input ? ext_new : a.score[static_cast<size_t>(u) * NS + rslot];
+  else
+    load_scorer_input<T, 2 * DH>(krow, vrow, in.x);
+  if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0 && !from_input && a.pos[static_cast<size_t>(u) * NS + rslot] != b)
+    set_error(a.err, DEVERR_STATE_MISMATCH);
+}
+
+template <int DH>
+__device__ __noinline__ Decision decide_finish(const LayerArgs& a, int u, int N, int ntk, const Decision* pending,
+                                               const DecideInput<DH>& in) {
+  Decision r;
+  r.p = N; r.bpos = -1; r.bslot = -1; r.tgt = -1; r.evict = -1; r.sb = 0.f; r.pad[0] = r.pad[1] = 0;
+  if (in.b < 0) return r;
+  const int S = a.S, W = a.W, D = a.D;
+  const int b = in.b;
+  r.bpos = b;
+  r.bslot = (D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D);
+  float sb;
+  if (a.flags & FLAG_EXTERNAL_SCORES) {
+    sb = in.sext;
+  } else {
+    const int h = u % a.Hkv;
+    const float* w1 = head_w1(a, h);
+    if (a.hidden == 0) sb = linear_score_x<2 * DH>(in.x, w1, a.b2[h]);
+    else if (a.hidden == 32) sb = mlp_score_x<2 * DH, 32>(in.x, w1, head_b1(a, h), head_w2(a, h), a.b2[h]);
+    else if (a.hidden == 64) sb = mlp_score_x<2 * DH, 64>(in.x, w1, head_b1(a, h), head_w2(a, h), a.b2[h]);
+    else sb = mlp_score_x<2 * DH, 128>(in.x, w1, head_b1(a, h), head_w2(a, h), a.b2[h]);
+  }
+  sb = ranking_priority(a, u, N, sb);   // b becomes eligible at step b + W + D = N
+  r.sb = sb;
+  if ((a.flags & FLAG_DEBUG_CHECKS) && (threadIdx.x & 31) == 0 && sb != sb) set_error(a.err, DEVERR_NAN_SCORE);
+  longrange_decide(a, u, ntk, pending, sb, b, r);
+  return r;
+}
+#endif
 
 // Commit of the step appending token N for unit u (one warp): moves rows as
 // the decision says, writes the new token, updates the unit's counters.
@@ -686,12 +714,26 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     if (step) {
       const int dw = warp - NCW;
       for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
+#ifdef KVPOP_DECIDE_EARLY_ARRIVE
+        if (mode == MODE_STEP) {   // MODE_STEP_NODECIDE: the next step's kernel decides
+          const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
+          DecideInput<DH> din;
+          decide_load<T, DH>(a, u, N + 1, k_new + static_cast<size_t>(u) * DH, v_new + static_cast<size_t>(u) * DH,
+                             ext ? ext[u] : 0.f, din);
+          const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
+          if (prev == need_of(u) - 1) push_merge(u);
+          const Decision nx = decide_finish<DH>(a, u, N + 1, ntk_after, &cur, din);
+          if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+          continue;
+        }
+#else
         if (mode == MODE_STEP) {   // MODE_STEP_NODECIDE: the next step's kernel decides
           const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
           const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, &cur, k_new + static_cast<size_t>(u) * DH,
                                              v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f);
           if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
         }
+#endif
         const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
         if (prev == need_of(u) - 1) push_merge(u);
       }

@@ -272,9 +272,10 @@ __device__ __forceinline__ void set_error(int32_t* err, int32_t bits) {
 // warp reads the whole W1 row (coalesced: 4 cache lines per instruction), each
 // lane forms its X-term partial sum, and a butterfly reduction over 16 rows at
 // a time leaves lane l (< 16) with the pre-activation of row 16 * block + l.
-template <typename T, int D2, int HID>
-__device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, const float* w1, const float* b1,
-                                                const float* w2, float b2) {
+// Lane l of a warp loads inputs [l X, l X + X) of x = [k; v] (X = D2 / 32) as
+// fp64 (bf16 / fp32 inputs are exact in fp64).  krow, vrow 16-byte aligned.
+template <typename T, int D2>
+__device__ __forceinline__ void load_scorer_input(const T* krow, const T* vrow, double (&x)[D2 / 32]) {
   constexpr int X = D2 / 32;      // inputs per lane (4 or 8)
   constexpr int D = D2 / 2;
   const int lane = threadIdx.x & 31;
@@ -288,9 +289,24 @@ __device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, co
   } else {
     reinterpret_cast<uint2*>(xr)[0] = reinterpret_cast<const uint2*>(src)[0];
   }
-  double x[X];
 #pragma unroll
   for (int e = 0; e < X; ++e) x[e] = static_cast<double>(Elem<T>::to_f32(xr[e]));
+}
+
+// Scorer: s = w2 . relu(W1 x + b1) + b2 for x = [k; v] of one token (KVpop
+// page §E.1 headwise inputs, §E.2 stateless MLP scorer), computed by one warp
+// from the inputs load_scorer_input placed in its lanes.  Accumulated in fp64
+// and rounded once to fp32, the ranking precision (§F).  For each hidden row
+// the warp reads the whole W1 row (coalesced: 4 cache lines per instruction),
+// each lane forms its X-term partial sum, and a butterfly reduction over 16
+// rows at a time leaves lane l (< 16) with the pre-activation of row
+// 16 * block + l.
+template <int D2, int HID>
+__device__ __forceinline__ float mlp_score_x(const double (&x)[D2 / 32], const float* w1, const float* b1,
+                                             const float* w2, float b2) {
+  constexpr int X = D2 / 32;
+  const int lane = threadIdx.x & 31;
+  const int i0 = lane * X;
   double part = 0.0;
   for (int blk = 0; blk < HID; blk += 16) {
     // b1 and w2 of the row this lane finishes, issued with the block's W1 loads
@@ -333,36 +349,40 @@ __device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, co
   return static_cast<float>(part + static_cast<double>(b2));
 }
 
+template <typename T, int D2, int HID>
+__device__ __forceinline__ float mlp_score_rows(const T* krow, const T* vrow, const float* w1, const float* b1,
+                                                const float* w2, float b2) {
+  double x[D2 / 32];
+  load_scorer_input<T, D2>(krow, vrow, x);
+  return mlp_score_x<D2, HID>(x, w1, b1, w2, b2);
+}
+
 // Stateless headwise linear scorer s = w . [k; v] + b (page §E.2), one warp:
 // lane l holds inputs [l * X, l * X + X) and the matching weights; fp64 dot
 // product, warp reduction, one rounding to fp32.
-template <typename T, int D2>
-__device__ __forceinline__ float linear_score_rows(const T* krow, const T* vrow, const float* w, float b) {
+template <int D2>
+__device__ __forceinline__ float linear_score_x(const double (&x)[D2 / 32], const float* w, float b) {
   constexpr int X = D2 / 32;
-  constexpr int D = D2 / 2;
-  const int lane = threadIdx.x & 31;
-  const int i0 = lane * X;
-  const T* src = (i0 < D) ? krow + i0 : vrow + (i0 - D);
-  constexpr int kBytes = X * static_cast<int>(sizeof(T));
-  alignas(16) T xr[X];
-  if constexpr (kBytes % 16 == 0) {
-#pragma unroll
-    for (int q = 0; q < kBytes / 16; ++q) reinterpret_cast<uint4*>(xr)[q] = reinterpret_cast<const uint4*>(src)[q];
-  } else {
-    reinterpret_cast<uint2*>(xr)[0] = reinterpret_cast<const uint2*>(src)[0];
-  }
+  const int i0 = (threadIdx.x & 31) * X;
   double acc = 0.0;
 #pragma unroll
   for (int q = 0; q < X / 4; ++q) {
     const float4 wv = __ldg(reinterpret_cast<const float4*>(w + i0) + q);
-    acc = fma(static_cast<double>(wv.x), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 0])), acc);
-    acc = fma(static_cast<double>(wv.y), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 1])), acc);
-    acc = fma(static_cast<double>(wv.z), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 2])), acc);
-    acc = fma(static_cast<double>(wv.w), static_cast<double>(Elem<T>::to_f32(xr[4 * q + 3])), acc);
+    acc = fma(static_cast<double>(wv.x), x[4 * q + 0], acc);
+    acc = fma(static_cast<double>(wv.y), x[4 * q + 1], acc);
+    acc = fma(static_cast<double>(wv.z), x[4 * q + 2], acc);
+    acc = fma(static_cast<double>(wv.w), x[4 * q + 3], acc);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return static_cast<float>(acc + static_cast<double>(b));
+}
+
+template <typename T, int D2>
+__device__ __forceinline__ float linear_score_rows(const T* krow, const T* vrow, const float* w, float b) {
+  double x[D2 / 32];
+  load_scorer_input<T, D2>(krow, vrow, x);
+  return linear_score_x<D2>(x, w, b);
 }
 
 // hidden in {32, 64, 128} (MLP) or 0 (linear: w1 is the weight row, b2 the
@@ -383,6 +403,66 @@ __device__ __noinline__ float mlp_score_warp(const T* krow, const T* vrow, int d
   if (hidden == 32) return mlp_score_rows<T, 128, 32>(krow, vrow, w1, b1, w2, b2);
   if (hidden == 64) return mlp_score_rows<T, 128, 64>(krow, vrow, w1, b1, w2, b2);
   return mlp_score_rows<T, 128, 128>(krow, vrow, w1, b1, w2, b2);
+}
+
+// Eviction decision against the long-range set, taken by one warp for the
+// boundary token b (ranking priority sb) of unit u; r.bslot is set.  While
+// fewer than K long-range slots are used (ntk < K), b takes the next free
+// one.  Otherwise the warp finds the minimum key (score, -position) of the
+// long-range slots and b replaces it only if its own key is strictly larger;
+// else b is dropped.  pending: the previous step's decision when it is not
+// yet committed (its target slot then counts with pending's key), or null.
+// Keys are unique (positions are), so the argmin is unique.
+__device__ __forceinline__ void longrange_decide(const LayerArgs& a, int u, int ntk, const Decision* pending,
+                                                 float sb, int b, Decision& r) {
+  const int lane = threadIdx.x & 31;
+  const int K = a.K;
+  const int base = topk_base(a.S, a.W, a.D);
+  const int32_t* pos = a.pos + static_cast<size_t>(u) * a.NS;
+  const float* score = a.score + static_cast<size_t>(u) * a.NS;
+  if (ntk < K) {
+    r.tgt = base + ntk;     // fill-up: next free long-range slot, nobody leaves
+    r.evict = -1;
+    return;
+  }
+  if (K == 0) {
+    r.evict = r.bslot;
+    return;
+  }
+  constexpr int kB = 16;   // long-range keys per lane per round trip
+  uint64_t best = ~0ull;
+  int mslot = -1;
+  for (int i0 = 0; i0 < K; i0 += 32 * kB) {
+    float sc[kB];
+    int32_t ps[kB];
+#pragma unroll
+    for (int t = 0; t < kB; ++t) {
+      const int i = i0 + lane + 32 * t;
+      if (i < K) { sc[t] = score[base + i]; ps[t] = pos[base + i]; }
+    }
+#pragma unroll
+    for (int t = 0; t < kB; ++t) {
+      const int i = i0 + lane + 32 * t;
+      if (i < K) {
+        const int sl = base + i;
+        const uint64_t key = (pending != nullptr && sl == pending->tgt) ? rank_key(pending->sb, pending->bpos)
+                                                                        : rank_key(sc[t], ps[t]);
+        if (key < best) { best = key; mslot = sl; }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t ok = __shfl_xor_sync(0xffffffffu, best, o);
+    const int os = __shfl_xor_sync(0xffffffffu, mslot, o);
+    if (ok < best) { best = ok; mslot = os; }
+  }
+  if (rank_key(sb, b) > best) {
+    r.tgt = mslot;
+    r.evict = mslot;
+  } else {
+    r.evict = r.bslot;
+  }
 }
 
 // Packed fp32 FMA (sm_100 FFMA2): d = a * b + c on both halves, round-to-nearest.

@@ -209,45 +209,16 @@ __device__ __forceinline__ const T* row_ptr(const LayerArgs& a, int u, int slot)
 }
 
 // Eviction decision of the step appending token N from the boundary token's
-// priority sb, over the long-range set as committed after step N - 1 (warp
-// argmin of the keys (score, -position); see the decode kernel's deciders).
+// priority sb, over the long-range set as committed after step N - 1.
 __device__ Decision decide_with_priority(const LayerArgs& a, int u, int N, int ntk, float sb) {
-  const int lane = threadIdx.x & 31;
-  const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
   Decision r;
   r.p = N; r.bpos = -1; r.bslot = -1; r.tgt = -1; r.evict = -1; r.sb = 0.f; r.pad[0] = r.pad[1] = 0;
-  const int b = N - W - D;
-  if (b < S) return r;
-  const int base = topk_base(S, W, D);
-  const int32_t* pos = a.pos + static_cast<size_t>(u) * NS;
-  const float* score = a.score + static_cast<size_t>(u) * NS;
+  const int b = N - a.W - a.D;
+  if (b < a.S) return r;
   r.bpos = b;
-  r.bslot = (D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D);
+  r.bslot = (a.D == 0) ? window_slot(b, a.S, a.W) : staging_slot(b, a.S, a.W, a.D);
   r.sb = sb;
-  if (ntk < K) {
-    r.tgt = base + ntk;
-  } else if (K == 0) {
-    r.evict = r.bslot;
-  } else {
-    uint64_t best = ~0ull;
-    int mslot = -1;
-    for (int i = lane; i < K; i += 32) {
-      const uint64_t key = rank_key(score[base + i], pos[base + i]);
-      if (key < best) { best = key; mslot = base + i; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const uint64_t ok = __shfl_xor_sync(kFull, best, o);
-      const int os = __shfl_xor_sync(kFull, mslot, o);
-      if (ok < best) { best = ok; mslot = os; }
-    }
-    if (rank_key(sb, b) > best) {
-      r.tgt = mslot;
-      r.evict = mslot;
-    } else {
-      r.evict = r.bslot;
-    }
-  }
+  longrange_decide(a, u, ntk, nullptr, sb, b, r);
   return r;
 }
 
