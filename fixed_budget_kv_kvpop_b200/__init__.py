@@ -49,7 +49,7 @@ EXPORTED_SYMBOLS = (
     "kvpop_get_layout", "kvpop_get_error", "kvpop_clear_error", "kvpop_debug_poison_error",
     "kvpop_destroy", "kvpop_status_string", "kvpop_decode_step_noalloc",
     "kvpop_prefill_attention_workspace_bytes", "kvpop_prefill_attention", "kvpop_prefill_with_attention",
-    "kvpop_debug_set_hook",
+    "kvpop_debug_set_hook", "kvpop_prefill_attention_from_cutoffs",
 )
 
 
@@ -115,6 +115,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvpop_prefill_attention": ([P, I32, P, P, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
         "kvpop_prefill_with_attention": ([P, I32, P, P, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
         "kvpop_debug_set_hook": ([P, I32], ctypes.c_int),
+        "kvpop_prefill_attention_from_cutoffs": ([P, I32, P, P, P, I32, P, P, P, SZ, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -322,6 +323,15 @@ class KVPopCache:
                                            _ptr(out), _ptr(lse), _ptr(workspace),
                                            int(workspace.numel() * workspace.element_size()) if workspace is not None
                                            else 0, _stream_ptr(stream)), "kvpop_prefill_attention")
+
+    def prefill_attention_from_cutoffs(self, layer: int, q, k, v, out, lse=None, workspace=None, stream=None):
+        """The attention stage alone, from the cutoffs a previous
+        prefill_attention call of the same prompt left in `workspace`."""
+        n = self._check_prompt(q, k, v, out, lse, workspace, None)
+        _check(self._lib.kvpop_prefill_attention_from_cutoffs(
+            self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n, _ptr(out), _ptr(lse), _ptr(workspace),
+            int(workspace.numel() * workspace.element_size()) if workspace is not None else 0, _stream_ptr(stream)),
+            "kvpop_prefill_attention_from_cutoffs")
 
     def prefill_with_attention(self, layer: int, q, k, v, out, lse=None, workspace=None, ext_scores=None,
                                stream=None):

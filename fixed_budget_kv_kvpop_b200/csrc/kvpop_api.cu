@@ -417,6 +417,27 @@ int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const
   return r == 0 ? KVPOP_OK : KVPOP_ERR_CUDA;
 }
 
+int kvpop_prefill_attention_from_cutoffs(kvpop_handle* h, int32_t layer, const void* q, const void* k, const void* v,
+                                         int32_t n_tokens, void* out, float* lse, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers || n_tokens < 0) return KVPOP_ERR_INVALID_ARG;
+  if (n_tokens > h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
+  if (n_tokens == 0) return KVPOP_OK;
+  if (!q || !k || !v || !out || !workspace) return KVPOP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return KVPOP_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return KVPOP_ERR_INVALID_ARG;
+  const LayerArgs a = layer_args(h, layer);
+  PrefillAttnPlan p;
+  if (plan_prefill_attention(a, h->cfg.dtype, n_tokens, &p) != 0 || a.units > 65535) return KVPOP_ERR_BAD_SHAPE;
+  if (workspace_bytes < p.total) return KVPOP_ERR_INVALID_ARG;
+  const int r = launch_prefill_attention(a, h->cfg.dtype, p, q, k, v, nullptr, out, lse,
+                                         static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream),
+                                         true);
+  if (r == -2) return KVPOP_ERR_BAD_SHAPE;
+  return r == 0 ? KVPOP_OK : KVPOP_ERR_CUDA;
+}
+
 int kvpop_prefill_with_attention(kvpop_handle* h, int32_t layer, const void* q, const void* k, const void* v,
                                  int32_t n_tokens, const float* ext_scores, void* out, float* lse, void* workspace,
                                  size_t workspace_bytes, void* stream) {

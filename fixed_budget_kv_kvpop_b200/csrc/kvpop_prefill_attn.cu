@@ -811,7 +811,7 @@ __global__ void __launch_bounds__(kTcThreads) sparse_attn_tc_kernel(PaArgs p) {
   constexpr uint32_t kIdescPV = tc_idesc(kTcRows, DH, 1);
   constexpr uint32_t kRowCells = kTcRows * 16;   // bytes of one chunk column of Q or P
   constexpr uint32_t kKeyCells = kTcKeys * 16;   // bytes of one chunk column of a K or V tile
-  extern __shared__ __align__(128) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   int* kpos = reinterpret_cast<int*>(smem_raw + SM::META_OFF);   // [2][kTcKeys]
   int* kcut = kpos + 2 * kTcKeys;                                  // [2][kTcKeys]
@@ -1045,6 +1045,348 @@ int launch_attn_tc(const PaArgs& pa, int units, int n, cudaStream_t st) {
   return 0;
 }
 
+
+// ---------------- bf16 attention on tcgen05, two row blocks per CTA ----------------
+// 256 query rows per CTA (two blocks of 128, one per group of four softmax
+// warps), warp-specialized and pipelined through mbarriers:
+//   producer warps 8-11 gather each tile's K and V rows (cp.async, kT2Stages
+//     stages) and publish them with the keys' positions and cutoffs;
+//   one thread of warp 12 issues the MMAs in the order S_0(t+1), O_0 += P_0 V(t),
+//     S_1(t+1), O_1 += P_1 V(t), so the tensor cores work on one block while
+//     the other block's softmax runs; each tile's K and V serve both blocks;
+//   softmax warps 0-3 (block 0) and 4-7 (block 1): thread = query row = TMEM
+//     lane; S double-buffered in TMEM, P single-buffered in shared memory.
+// TMEM: S[block][buf] at columns 32 * (2 block + buf), O[block] at 128 + block * DH.
+constexpr int kT2Rows = 256;
+constexpr int kT2Keys = 32;
+constexpr int kT2Stages = 3;
+constexpr int kT2Threads = 13 * 32;
+constexpr int kT2Prod = 8;          // first producer warp
+constexpr int kT2Mma = 12;          // MMA warp
+constexpr uint32_t kT2Cols = 512;
+
+template <int DH>
+struct T2Smem {
+  static constexpr int QCH = DH / 8;
+  static constexpr size_t QBLK = static_cast<size_t>(QCH) * 128 * 16;          // one block of Q rows
+  static constexpr size_t Q_OFF = 0;
+  static constexpr size_t KV_TILE = static_cast<size_t>(QCH) * kT2Keys * 16;
+  static constexpr size_t KV_OFF = Q_OFF + 2 * QBLK;                             // [stage][K, V]
+  static constexpr size_t PBLK = static_cast<size_t>(kT2Keys / 8) * 128 * 16;
+  static constexpr size_t P_OFF = KV_OFF + 2 * kT2Stages * KV_TILE;             // [block]
+  static constexpr size_t META_OFF = P_OFF + 2 * PBLK;                           // [stage]{pos[keys], cut[keys], full}
+  static constexpr int META_INTS = 2 * kT2Keys + 4;
+  static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * kT2Stages * META_INTS;
+  static constexpr int NBAR = 2 * kT2Stages + 12;
+  static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
+  static constexpr size_t WT_OFF = TADDR_OFF + 16;
+  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);
+  static_assert(BAR_OFF % 8 == 0 && KV_OFF % 16 == 0 && P_OFF % 16 == 0, "shared-memory alignment");
+  // at least 116 KB: one CTA per SM, which then holds all 512 TMEM columns
+  static size_t bytes(int cand_cap) {
+    const size_t bb = CAND_OFF + sizeof(int) * static_cast<size_t>(cand_cap);
+    return bb > 116 * 1024 ? bb : 116 * 1024;
+  }
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p) {
+  using SM = T2Smem<DH>;
+  constexpr int QCH = SM::QCH;
+  constexpr uint32_t kIdescS = tc_idesc(128, kT2Keys, 0);
+  constexpr uint32_t kIdescPV = tc_idesc(128, DH, 1);
+  constexpr uint32_t kRowCells = 128 * 16;
+  constexpr uint32_t kKeyCells = kT2Keys * 16;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  int* meta = reinterpret_cast<int*>(smem_raw + SM::META_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + SM::BAR_OFF);
+  uint64_t* kv_full = bars;                       // [stage], 128 producer arrivals
+  uint64_t* kv_free = bars + kT2Stages;           // [stage], MMA commit
+  uint64_t* s_full = bars + 2 * kT2Stages;        // [block][buf], MMA commit
+  uint64_t* s_free = s_full + 4;                  // [block][buf], 128 softmax arrivals
+  uint64_t* p_full = s_free + 4;                  // [block], 128 softmax arrivals
+  uint64_t* o_done = p_full + 2;                  // [block], MMA commit
+  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_raw + SM::TADDR_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SM::TADDR_OFF + 4);
+  int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
+  int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int u = blockIdx.y;
+  const int b = u / p.Hkv, hk = u % p.Hkv;
+  const int n = p.n, S = p.S, WD = p.W + p.D, G = p.G;
+  const int q0 = blockIdx.x * p.qt;
+  const int q1 = min(n, q0 + p.qt);
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
+  const __nv_bfloat16* kgp = static_cast<const __nv_bfloat16*>(p.k) + static_cast<size_t>(u) * n * DH;
+  const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
+  const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
+
+  if (warp == kT2Mma) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(taddr_s)), "r"(kT2Cols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kT2Stages; ++i) {
+      mbar_init(&kv_full[i], 128);
+      mbar_init(&kv_free[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  // query rows of both blocks (row = position offset * G + head), zero past the prompt
+  for (int c = tid; c < kT2Rows * QCH; c += kT2Threads) {
+    const int row = c / QCH, ch = c % QCH;
+    const int qpos = q0 + row / G, g = row % G;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (qpos < q1)
+      x = *reinterpret_cast<const uint4*>(qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos) * DH + ch * 8);
+    *reinterpret_cast<uint4*>(smem_raw + SM::Q_OFF + (row >> 7) * SM::QBLK +
+                              (static_cast<size_t>(ch) * 128 + (row & 127)) * 16) = x;
+  }
+  fence_proxy_async_smem();
+  const int count = gather_candidates<kT2Threads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *taddr_s;
+  const int ntiles = (count + kT2Keys - 1) / kT2Keys;
+
+  // bounded wait; on expiry every role stops at its next check
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    if (lane == 0) set_error(p.err, DEVERR_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+  };
+
+  if (warp >= kT2Prod && warp < kT2Mma) {
+    // ---------------- producers ----------------
+    const int ptid = tid - kT2Prod * 32;
+    const int m1 = q1 - 1 - WD;
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t % kT2Stages;
+      if (t >= kT2Stages && !wait(&kv_free[st], ((t / kT2Stages) - 1) & 1)) break;
+      const uint32_t kbase = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
+      const uint32_t vbase = kbase + static_cast<uint32_t>(SM::KV_TILE);
+      for (int i = ptid; i < kT2Keys * QCH; i += 128) {
+        const int key = i / QCH, ch = i % QCH;
+        const int idx = t * kT2Keys + key;
+        const int j = idx < count ? cand[idx] : -1;
+        const size_t off = j >= 0 ? static_cast<size_t>(j) * DH + ch * 8 : 0;
+        const uint32_t so = static_cast<uint32_t>((ch * kT2Keys + key) * 16);
+        cp_async16(kbase + so, kgp + off, j >= 0 ? 16 : 0);
+        cp_async16(vbase + so, vgp + off, j >= 0 ? 16 : 0);
+      }
+      cp_async_commit();
+      if (ptid < kT2Keys) {
+        int* m = meta + st * SM::META_INTS;
+        const int idx = t * kT2Keys + ptid;
+        const int j = idx < count ? cand[idx] : -1;
+        const int c = j >= 0 ? cu[j] : 0;
+        m[ptid] = j;
+        m[kT2Keys + ptid] = c;
+        const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
+        const unsigned bal = __ballot_sync(0xffffffffu, full);
+        if (lane == 0) m[2 * kT2Keys] = (bal == 0xffffffffu);
+      }
+      if (t >= 1) {   // tile t - 1 has landed: publish it
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&kv_full[(t - 1) % kT2Stages]);
+      }
+    }
+    cp_async_wait<0>();
+    if (ntiles >= 1 && !*abort_flag) {
+      fence_proxy_async_smem();
+      mbar_arrive(&kv_full[(ntiles - 1) % kT2Stages]);
+    }
+  } else if (warp == kT2Mma) {
+    // ---------------- MMA issue (one thread) ----------------
+    if (lane == 0 && ntiles > 0) {
+      auto issue_s = [&](int X, int t) -> bool {
+        const int buf = t & 1, st = t % kT2Stages;
+        if (t >= 2 && !wait(&s_free[2 * X + buf], ((t - 2) >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t qb = sbase + static_cast<uint32_t>(SM::Q_OFF + X * SM::QBLK);
+        const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
+        const uint32_t d = tmem + 32u * (2 * X + buf);
+#pragma unroll
+        for (int ks = 0; ks < DH / 16; ++ks)
+          tc_mma(d, tc_desc(qb + ks * 2 * kRowCells, kRowCells, 128), tc_desc(kb + ks * 2 * kKeyCells, kKeyCells, 128),
+                 kIdescS, ks > 0 ? 1u : 0u);
+        tc_commit(&s_full[2 * X + buf]);
+        return true;
+      };
+      auto issue_pv = [&](int X, int t) -> bool {
+        const int st = t % kT2Stages;
+        if (!wait(&p_full[X], t & 1)) return false;
+        tc_fence_after();
+        const uint32_t pb = sbase + static_cast<uint32_t>(SM::P_OFF + X * SM::PBLK);
+        const uint32_t vb = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st + 1) * SM::KV_TILE);
+        const uint32_t d = tmem + 128u + static_cast<uint32_t>(X * DH);
+#pragma unroll
+        for (int kk = 0; kk < kT2Keys / 16; ++kk)
+          tc_mma(d, tc_desc(pb + kk * 2 * kRowCells, kRowCells, 128), tc_desc(vb + kk * 256, 128, kKeyCells),
+                 kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&o_done[X]);
+        return true;
+      };
+      bool ok = wait(&kv_full[0], 0) && issue_s(0, 0) && issue_s(1, 0);
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const bool next = t + 1 < ntiles;
+        if (next) ok = wait(&kv_full[(t + 1) % kT2Stages], ((t + 1) / kT2Stages) & 1) && issue_s(0, t + 1);
+        ok = ok && issue_pv(0, t);
+        if (next) ok = ok && issue_s(1, t + 1);
+        ok = ok && issue_pv(1, t);
+        if (ok) tc_commit(&kv_free[t % kT2Stages]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax: block X, thread = row = TMEM lane ----------------
+    const int X = warp >> 2;
+    const int row = tid & 127;
+    const int grow = X * 128 + row;
+    const int qpos = q0 + grow / G;
+    const bool vrow = qpos < q1;
+    const int mrow = qpos - WD;
+    const uint32_t lrow = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tO = tmem + 128u + static_cast<uint32_t>(X * DH);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int t = 0; t < ntiles; ++t) {
+      const int buf = t & 1, st = t % kT2Stages;
+      bool got = wait(&kv_full[st], (t / kT2Stages) & 1);
+      got = got && wait(&s_full[2 * X + buf], (t >> 1) & 1);
+      if (!__all_sync(0xffffffffu, got)) {   // the TMEM loads below are warp-collective
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[32];
+      tc_ld32(tmem + 32u * (2 * X + buf) + lrow, sv);
+      tc_fence_before();
+      mbar_arrive(&s_free[2 * X + buf]);
+      const int* m = meta + st * SM::META_INTS;
+      float tmax = -INFINITY;
+      if (m[2 * kT2Keys]) {
+#pragma unroll
+        for (int i = 0; i < kT2Keys; ++i) {
+          sv[i] = vrow ? sv[i] * p.scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, sv[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kT2Keys; ++i) {
+          const int j = m[i];
+          const bool vis = j >= 0 && vrow && j <= qpos && (j < S || j > mrow || m[kT2Keys + i] > mrow);
+          sv[i] = vis ? sv[i] * p.scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, sv[i]);
+        }
+      }
+      float alpha = 1.f;
+      bool resc = false;
+      if (tmax > m_run + kTcLazy) {
+        resc = (m_run != -INFINITY);
+        alpha = resc ? exp2f(m_run - tmax) : 0.f;
+        l_run *= alpha;
+        m_run = tmax;
+      }
+      float psum = 0.f;
+      uint32_t pk[kT2Keys / 2];
+#pragma unroll
+      for (int i = 0; i < kT2Keys; i += 2) {
+        const float p0 = sv[i] == -INFINITY ? 0.f : exp2f(sv[i] - m_run);
+        const float p1 = sv[i + 1] == -INFINITY ? 0.f : exp2f(sv[i + 1] - m_run);
+        psum += p0 + p1;
+        pk[i / 2] = pack_bf16(p0, p1);
+      }
+      l_run += psum;
+      // P_X and O_X are free once the previous tile's P V has completed
+      const bool freed = t == 0 || wait(&o_done[X], (t - 1) & 1);
+      if (!__all_sync(0xffffffffu, freed)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, resc)) {
+        const float f = resc ? alpha : 1.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+          float o[32];
+          tc_ld32(tO + lrow + c0, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= f;
+          tc_st32(tO + lrow + c0, o);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      }
+      uint8_t* pb = smem_raw + SM::P_OFF + X * SM::PBLK;
+#pragma unroll
+      for (int c = 0; c < kT2Keys / 8; ++c)
+        *reinterpret_cast<uint4*>(pb + (static_cast<size_t>(c) * 128 + row) * 16) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[X]);
+    }
+    bool fin = ok && ntiles > 0;
+    if (fin) fin = wait(&o_done[X], (ntiles - 1) & 1);
+    if (__all_sync(0xffffffffu, fin)) {
+      tc_fence_after();
+      const int g = grow % G;
+      const size_t rowi = (static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (vrow ? qpos : 0);
+      __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out) + rowi * DH;
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float o[32];
+        tc_ld32(tO + lrow + c0, o);
+        if (vrow) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(og + c0 + 8 * c) =
+                make_uint4(pack_bf16(o[8 * c] * inv, o[8 * c + 1] * inv),
+                           pack_bf16(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
+                           pack_bf16(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
+                           pack_bf16(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+        }
+      }
+      if (vrow && p.lse != nullptr) p.lse[rowi] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kT2Mma) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kT2Cols) : "memory");
+  }
+}
+
+template <int DH>
+int launch_attn_tc2(const PaArgs& pa, int units, int n, cudaStream_t st) {
+  const size_t smem = T2Smem<DH>::bytes(pa.cand_cap);
+  if (smem > 227 * 1024) return -2;
+  if (cudaFuncSetAttribute(sparse_attn_tc2_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return -1;
+  dim3 grid((n + pa.qt - 1) / pa.qt, units);
+  sparse_attn_tc2_kernel<DH><<<grid, kT2Threads, smem, st>>>(pa);
+  return 0;
+}
+
 template <int DH>
 int launch_attn_f32(const PaArgs& pa, int units, int n, cudaStream_t st) {
   const size_t smem = PaSmem<DH>::bytes(pa.cand_cap);
@@ -1161,25 +1503,27 @@ int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan
 
 int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPlan& p, const void* q, const void* k,
                              const void* v, const float* ext, void* out, float* lse, uint8_t* workspace,
-                             cudaStream_t st) {
+                             cudaStream_t st, bool reuse_cutoffs) {
   if (p.n == 0) return 0;
   if (a.units > 65535) return -2;
   int32_t* cut = reinterpret_cast<int32_t*>(workspace + p.cut_off);
   float* scores = reinterpret_cast<float*>(workspace + p.score_off);
   uint64_t* keys = reinterpret_cast<uint64_t*>(workspace + p.keys_off);
   uint32_t* bits = reinterpret_cast<uint32_t*>(workspace + p.bits_off);
-  if (p.ne > 0) {
+  if (!reuse_cutoffs && p.ne > 0) {
     const int r = launch_prompt_scores(a, dtype, k, v, p.n, ext, scores, p.ne, st);
     if (r != 0) return r;
   }
-  const size_t cut_smem = (p.keys_global ? 0 : static_cast<size_t>(p.npow) * 8) +
-                          (p.bits_global ? 0 : static_cast<size_t>(p.words) * 4);
-  if (cudaFuncSetAttribute(cutoff_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kPaSmemSortKeys * 8 + kPaSmemBitmapWords * 4) != cudaSuccess)
-    return -1;
-  cutoff_kernel<<<a.units, kCutThreads, cut_smem, st>>>(scores, max(p.ne, 1), cut, p.n, p.ne, p.npow, p.words, a.S,
-                                                        a.K, keys, bits, p.keys_global ? 1 : 0,
-                                                        p.bits_global ? 1 : 0, a.err);
+  if (!reuse_cutoffs) {
+    const size_t cut_smem = (p.keys_global ? 0 : static_cast<size_t>(p.npow) * 8) +
+                            (p.bits_global ? 0 : static_cast<size_t>(p.words) * 4);
+    if (cudaFuncSetAttribute(cutoff_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPaSmemSortKeys * 8 + kPaSmemBitmapWords * 4) != cudaSuccess)
+      return -1;
+    cutoff_kernel<<<a.units, kCutThreads, cut_smem, st>>>(scores, max(p.ne, 1), cut, p.n, p.ne, p.npow, p.words,
+                                                          a.S, a.K, keys, bits, p.keys_global ? 1 : 0,
+                                                          p.bits_global ? 1 : 0, a.err);
+  }
   PaArgs pa;
   pa.q = q;
   pa.k = k;

@@ -39,11 +39,13 @@ struct PrefillAttnPlan {
 // Plans the workspace and launch shapes; returns 0 or -2 (shape not supported).
 int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan* p);
 
-// Cutoffs then attention, on `st`.  cut, scores, keys and bits point into the
-// caller's workspace at the plan's offsets.  Returns 0, -1 (CUDA) or -2.
+// Prompt scores, cutoffs, then attention, on `st` (reuse_cutoffs: the
+// attention alone, from the cutoffs already in the workspace).  cut, scores,
+// keys and bits point into the caller's workspace at the plan's offsets.
+// Returns 0, -1 (CUDA) or -2.
 int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPlan& p, const void* q, const void* k,
                              const void* v, const float* ext, void* out, float* lse, uint8_t* workspace,
-                             cudaStream_t st);
+                             cudaStream_t st, bool reuse_cutoffs = false);
 
 // Whole-prompt cache build from the cutoffs of a launch_prefill_attention on
 // the same workspace (the layer must be empty): the tokens kept to the end

@@ -310,6 +310,19 @@ int kvpop_prefill_attention(kvpop_handle* h, int32_t layer, const void* q, const
                             int32_t n_tokens, const float* ext_scores, void* out, float* lse, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* The attention stage of kvpop_prefill_attention alone, from the running
+ * cutoffs that a previous kvpop_prefill_attention call of the same prompt
+ * (same layer's scorer, same k, v and n_tokens) left in `workspace`: the
+ * prompt is not scored again and the cutoffs are not recomputed (page §C.2:
+ * the cutoffs are computed once and the mask is evaluated from them on the
+ * fly).  For a caller that runs several query sets over one prompt's mask.
+ * The result equals that call's bit for bit when q, k and v are the same.
+ * Arguments, layouts and errors as kvpop_prefill_attention (no ext_scores);
+ * the workspace contents are the caller's responsibility. */
+int kvpop_prefill_attention_from_cutoffs(kvpop_handle* h, int32_t layer, const void* q, const void* k, const void* v,
+                                         int32_t n_tokens, void* out, float* lse, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
 /* kvpop_prefill and kvpop_prefill_attention in one call, for a whole prompt
  * on an empty layer: the prompt is scored once, its attention outputs (and
  * log-normalisers, if lse is not NULL) are computed under the running top-k

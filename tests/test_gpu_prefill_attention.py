@@ -171,6 +171,30 @@ def test_mask_edge_cases(S, W, D, K, n):
         np.testing.assert_allclose(r.out.double().cpu().numpy(), ref.numpy(), rtol=0, atol=gh.BF16_ATOL)
 
 
+def test_attention_from_cutoffs_equals_the_full_call():
+    """kvpop_prefill_attention_from_cutoffs (the attention stage alone, from
+    the cutoffs a first call left in the workspace) returns the full call's
+    outputs and normalisers bit for bit, and another query set over the same
+    mask matches the oracle."""
+    _need_gpu()
+    w = _case("bf16", 128, 8, 2, S=4, W=16, D=0, K=40, hidden=64)
+    r = run_prefill_attention(w, 300)
+    ws = torch.empty(r.cache.prefill_attention_workspace_bytes(300), dtype=torch.uint8, device="cuda")
+    out_full = torch.empty_like(r.q)
+    lse_full = torch.empty_like(r.lse)
+    r.cache.prefill_attention(0, r.q, r.k, r.v, out_full, lse_full, ws)
+    out2 = torch.full_like(r.q, float("nan"))
+    lse2 = torch.full_like(r.lse, float("nan"))
+    r.cache.prefill_attention_from_cutoffs(0, r.q, r.k, r.v, out2, lse2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_full, out2) and torch.equal(lse_full, lse2)
+    q2 = wl.prompt_queries(w, 0, 300, master=5).cuda()
+    r.cache.prefill_attention_from_cutoffs(0, q2, r.k, r.v, out2, lse2, ws)
+    torch.cuda.synchronize()
+    r.q, r.out, r.lse = q2, out2, lse2
+    check_all_rows(r)
+
+
 def test_repeat_call_is_deterministic_and_leaves_cache_alone():
     """Two calls give identical bits; the cache's position counter is untouched."""
     _need_gpu()
