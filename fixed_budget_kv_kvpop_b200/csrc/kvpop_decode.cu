@@ -217,7 +217,6 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
   return r;
 }
 
-#ifdef KVPOP_DECIDE_EARLY_ARRIVE
 // The decode kernel's deciders take the next step's decision in two halves,
 // so that a unit's merge (which commits this step's row moves) need not wait
 // for the next decision's scorer and argmin.  decide_load reads what the
@@ -283,7 +282,6 @@ __device__ __noinline__ Decision decide_finish(const LayerArgs& a, int u, int N,
   longrange_decide(a, u, ntk, pending, sb, b, r);
   return r;
 }
-#endif
 
 // Commit of the step appending token N for unit u (one warp): moves rows as
 // the decision says, writes the new token, updates the unit's counters.
@@ -699,8 +697,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     __syncwarp();
     if (lane == 0) {
       __threadfence();
+#ifdef KVPOP_CTA_FINISH
+      // count the CTA's warps in shared memory; its last warp reports the CTA
+      if (atomicAdd(&mq[kMergeCap + 3], 1) != NCW + NDW - 1) return;
+      __threadfence();
+      const int prev = atomicAdd(&a.layer->ticket, 1);
+      if (prev == static_cast<int>(gridDim.x) - 1) {
+#else
       const int prev = atomicAdd(&a.layer->ticket, 1);
       if (prev == static_cast<int>(gridDim.x) * (NCW + NDW) - 1) {
+#endif
         a.layer->n_seen = N + 1;
         a.layer->n_topk = ntk_after;
         a.layer->ticket = 0;
@@ -714,7 +720,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     if (step) {
       const int dw = warp - NCW;
       for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
-#ifdef KVPOP_DECIDE_EARLY_ARRIVE
         if (mode == MODE_STEP) {   // MODE_STEP_NODECIDE: the next step's kernel decides
           const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
           DecideInput<DH> din;
@@ -726,14 +731,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
           if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
           continue;
         }
-#else
-        if (mode == MODE_STEP) {   // MODE_STEP_NODECIDE: the next step's kernel decides
-          const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
-          const Decision nx = decide_warp<T>(a, u, N + 1, ntk_after, &cur, k_new + static_cast<size_t>(u) * DH,
-                                             v_new + static_cast<size_t>(u) * DH, ext ? ext[u] : 0.f);
-          if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
-        }
-#endif
         const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
         if (prev == need_of(u) - 1) push_merge(u);
       }

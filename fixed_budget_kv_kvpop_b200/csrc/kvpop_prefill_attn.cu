@@ -1479,7 +1479,7 @@ int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan
   P.ne = max(0, n - a.W - a.D - a.S);
   P.npow = next_pow2(max(P.ne, 1));
   P.words = max(1, (P.ne + 31) / 32);
-  P.qt = (dtype == 0 ? kPaRows : kPaMmaRows) / a.G;
+  P.qt = (dtype == 0 ? kPaRows : kT2Rows) / a.G;
   const int64_t cc = static_cast<int64_t>(a.S) + a.K + P.qt + a.W + a.D;
   if (cc > (1 << 14)) return -2;   // the candidate list lives in shared memory
   P.cand_cap = static_cast<int>(cc);
@@ -1546,7 +1546,7 @@ int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPla
   if (dtype == 0)
     r = (a.d == 128) ? launch_attn_f32<128>(pa, a.units, p.n, st) : launch_attn_f32<64>(pa, a.units, p.n, st);
   else
-    r = (a.d == 128) ? launch_attn_tc<128>(pa, a.units, p.n, st) : launch_attn_tc<64>(pa, a.units, p.n, st);
+    r = (a.d == 128) ? launch_attn_tc2<128>(pa, a.units, p.n, st) : launch_attn_tc2<64>(pa, a.units, p.n, st);
   if (r != 0) return r;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

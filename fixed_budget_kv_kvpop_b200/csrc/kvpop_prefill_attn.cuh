@@ -30,7 +30,7 @@ struct PrefillAttnPlan {
   int ne;           // tokens that become eligible in the prompt: max(0, n - W - D - S)
   int npow;         // sort length: next power of two >= max(ne, 1)
   int words;        // bitmap words: (ne + 31) / 32, at least 1
-  int qt;           // query positions per attention CTA: kPaRows / G (fp32) or kPaMmaRows / G (bf16)
+  int qt;           // query positions per attention CTA: 64 / G (fp32) or 256 / G (bf16)
   int cand_cap;     // candidate keys of one CTA at most: S + K + qt + W + D
   size_t cut_off, score_off, keys_off, bits_off, total;   // workspace layout (bytes)
   bool keys_global, bits_global;

@@ -302,7 +302,7 @@ int kvpop_decode_attend(kvpop_handle* h, int32_t layer, const void* q, void* out
  * Errors: KVPOP_ERR_INVALID_ARG (null or misaligned pointer, workspace too
  * small, bad layer), KVPOP_ERR_BAD_SHAPE (G not dividing 64, head_dim other
  * than 64/128, S + K + W + D + P above 16384 where P = 64/G for fp32 and
- * 128/G for bf16, more than 65535 units),
+ * 256/G for bf16, more than 65535 units, the mLSTM scorer),
  * KVPOP_ERR_CONTEXT_OVERFLOW (n_tokens > max_context); nothing is enqueued
  * then.  n_tokens = 0 is a no-op. */
 int kvpop_prefill_attention_workspace_bytes(const kvpop_handle* h, int32_t n_tokens, size_t* bytes);
