@@ -20,9 +20,9 @@
 // lane j ends with row j.  Weights are fp32 and inputs bf16 or fp32, both
 // exact in fp64.
 //
-// Decode: mlstm_step_kernel runs before each decode kernel of a layer.  It
-// folds the step's token into the state and takes that step's eviction
-// decision (the boundary token's score depends on the token that arrives in
+// Decode: mlstm_step_kernel (one CTA of four warps per unit) runs before each
+// decode kernel of a layer.  It folds the step's token into the state and
+// takes that step's eviction decision (the boundary token's score depends on the token that arrives in
 // the same step, so the decision cannot be taken one step ahead as the
 // stateless scorers' is).  Prefill: mlstm_prefill_kernel walks a chunk's
 // tokens in order and scores each token as it becomes eligible.
@@ -174,14 +174,13 @@ __device__ __forceinline__ void state_update(const double (&x)[X], const float* 
   s.m = m_new;
 }
 
-// Delayed readout of a token with inputs x from the state: the fp32 score.
-template <int X, int DV>
-__device__ __forceinline__ float state_score(const double (&x)[X], const float* __restrict__ hw, int p, int dv,
-                                             const LaneState<DV>& s) {
+// Delayed readout from the state of a token with read features r (feature f
+// in lane f): h = C^T r / max(|n . r|, e^-m), score = w_o . SiLU(h) + b_o,
+// rounded once to fp32 (tail: w_o, b_i, b_f, b_o of the head).
+template <int DV>
+__device__ __forceinline__ float state_readout(double r, const float* __restrict__ tail, int dv,
+                                               const LaneState<DV>& s) {
   const int lane = threadIdx.x & 31;
-  const int R = 2 * p + dv + 2;
-  const float* tail = hw + static_cast<size_t>(R) * (32 * X);
-  const double r = hedgehog_lane(project_rows<X>(x, hw, 0, p), p);
   // numerators (C^T r)_j: reduce-scatter over the feature lanes, lane j keeps j
   double v[32];
 #pragma unroll
@@ -203,61 +202,134 @@ __device__ __forceinline__ float state_score(const double (&x)[X], const float* 
   return static_cast<float>(warp_sum(t) + static_cast<double>(__ldg(tail + dv + 2)));
 }
 
+// Delayed readout of a token with inputs x from the state: the fp32 score.
+template <int X, int DV>
+__device__ __forceinline__ float state_score(const double (&x)[X], const float* __restrict__ hw, int p, int dv,
+                                             const LaneState<DV>& s) {
+  const float* tail = hw + static_cast<size_t>(2 * p + dv + 2) * (32 * X);
+  return state_readout<DV>(hedgehog_lane(project_rows<X>(x, hw, 0, p), p), tail, dv, s);
+}
+
+// Folds a token into the state from its projections: its Hedgehog features
+// (feature f in lane f), its value vector val[0, dv) and its gate
+// pre-activations gi, gf (biases included).  The same arithmetic as
+// state_update.
+template <int DV>
+__device__ __forceinline__ void state_fold(double phi, const double* val, double gi, double gf, int dv,
+                                           LaneState<DV>& s) {
+  const double lf = log_sigmoid(gf);
+  const double m_new = fmax(lf + s.m, gi);
+  const double ip = exp(gi - m_new);
+  const double fp = exp(lf + s.m - m_new);
+#pragma unroll
+  for (int j = 0; j < DV; ++j)
+    if (j < dv) s.c[j] = fp * s.c[j] + ip * (val[j] * phi);
+  s.n = fp * s.n + ip * phi;
+  s.m = m_new;
+}
+
 template <typename T>
 __device__ __forceinline__ const T* row_ptr(const LayerArgs& a, int u, int slot) {
   return reinterpret_cast<const T*>(a.kv + (static_cast<size_t>(u) * a.NS + slot) * a.row_bytes);
 }
 
-// Eviction decision of the step appending token N from the boundary token's
-// priority sb, over the long-range set as committed after step N - 1.
-__device__ Decision decide_with_priority(const LayerArgs& a, int u, int N, int ntk, float sb) {
-  Decision r;
-  r.p = N; r.bpos = -1; r.bslot = -1; r.tgt = -1; r.evict = -1; r.sb = 0.f; r.pad[0] = r.pad[1] = 0;
-  const int b = N - a.W - a.D;
-  if (b < a.S) return r;
-  r.bpos = b;
-  r.bslot = (a.D == 0) ? window_slot(b, a.S, a.W) : staging_slot(b, a.S, a.W, a.D);
-  r.sb = sb;
-  longrange_decide(a, u, ntk, nullptr, sb, b, r);
-  return r;
-}
-
+// One CTA of four warps per unit.  Warps 0-2 project the step's token (write
+// features, value, gates), warp 3 the boundary token's read features, all four
+// look for the long-range minimum; then warp 0 folds the token into the
+// state, reads the boundary token out and takes the step's decision.
 template <typename T, int X, int DV>
-__global__ void __launch_bounds__(32 * kMlstmWarps) mlstm_step_kernel(const LayerArgs a, const T* __restrict__ k_new,
-                                                                       const T* __restrict__ v_new) {
+__global__ void __launch_bounds__(128) mlstm_step_kernel(const LayerArgs a, const T* __restrict__ k_new,
+                                                         const T* __restrict__ v_new) {
   // Everything below reads the previous kernels' cache and counters.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int lane = threadIdx.x & 31;
-  const int u = blockIdx.x * kMlstmWarps + (threadIdx.x >> 5);
-  if (u >= a.units) return;
+  __shared__ double s_phi[32], s_val[32], s_r[32], s_g[2];
+  __shared__ unsigned long long s_best[4];
+  __shared__ int s_slot[4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x;
   const int N = a.layer->n_seen;
   const int ntk = a.layer->n_topk;
   if (N >= a.max_context) return;   // the decode kernel that follows reports the overflow
+  const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
   const int h = u % a.Hkv;
   const int p = a.mp, dv = a.mdv;
   const float* hw = a.mw + static_cast<size_t>(h) * mlstm_head_floats(p, dv, a.d);
-  double* st = a.mstate + static_cast<size_t>(u) * mlstm_state_doubles(p, dv);
-  LaneState<DV> s;
-  state_load<DV>(st, p, dv, s);
-  double x[X];
-  load_x<T, X>(k_new + static_cast<size_t>(u) * a.d, v_new + static_cast<size_t>(u) * a.d, x);
-  state_update<X, DV>(x, hw, p, dv, s);
-  state_store<DV>(st, p, dv, s);
-  const int b = N - a.W - a.D;
-  float sb = 0.f;
-  if (b >= a.S) {
-    const int bslot = (a.D == 0) ? window_slot(b, a.S, a.W) : staging_slot(b, a.S, a.W, a.D);
+  const float* tail = hw + static_cast<size_t>(2 * p + dv + 2) * (32 * X);
+  const int b = N - W - D;
+  const bool has_b = b >= S;
+  const int bslot = has_b ? ((D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D)) : -1;
+  const int base = topk_base(S, W, D);
+  const bool scan = has_b && ntk >= K && K > 0;
+  if (warp < 3) {
+    double x[X];
+    load_x<T, X>(k_new + static_cast<size_t>(u) * a.d, v_new + static_cast<size_t>(u) * a.d, x);
+    if (warp == 0) {
+      s_phi[lane] = hedgehog_lane(project_rows<X>(x, hw, p, p), p);
+    } else if (warp == 1) {
+      s_val[lane] = project_rows<X>(x, hw, 2 * p, dv);
+    } else {
+      const double g = project_rows<X>(x, hw, 2 * p + dv, 2);
+      if (lane < 2) s_g[lane] = g + static_cast<double>(__ldg(tail + dv + lane));
+    }
+  } else if (has_b) {
     const T* row = row_ptr<T>(a, u, bslot);
     double xb[X];
     load_x<T, X>(row, row + a.d, xb);
-    sb = ranking_priority(a, u, N, state_score<X, DV>(xb, hw, p, dv, s));
-    if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0) {
-      if (a.pos[static_cast<size_t>(u) * a.NS + bslot] != b) set_error(a.err, DEVERR_STATE_MISMATCH);
-      if (sb != sb) set_error(a.err, DEVERR_NAN_SCORE);
-    }
+    s_r[lane] = hedgehog_lane(project_rows<X>(xb, hw, 0, p), p);
+    if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0 && a.pos[static_cast<size_t>(u) * NS + bslot] != b)
+      set_error(a.err, DEVERR_STATE_MISMATCH);
   }
-  const Decision r = decide_with_priority(a, u, N, ntk, sb);
+  if (scan) {   // minimum key (score, -position) of the long-range set as committed after step N - 1
+    const int32_t* pos = a.pos + static_cast<size_t>(u) * NS + base;
+    const float* score = a.score + static_cast<size_t>(u) * NS + base;
+    uint64_t best = ~0ull;
+    int mslot = -1;
+    for (int i = threadIdx.x; i < K; i += 128) {
+      const uint64_t key = rank_key(score[i], pos[i]);
+      if (key < best) { best = key; mslot = base + i; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t ok = __shfl_xor_sync(kFull, best, o);
+      const int os = __shfl_xor_sync(kFull, mslot, o);
+      if (ok < best) { best = ok; mslot = os; }
+    }
+    if (lane == 0) { s_best[warp] = best; s_slot[warp] = mslot; }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  double* st = a.mstate + static_cast<size_t>(u) * mlstm_state_doubles(p, dv);
+  LaneState<DV> s;
+  state_load<DV>(st, p, dv, s);
+  state_fold<DV>(s_phi[lane], s_val, s_g[0], s_g[1], dv, s);
+  state_store<DV>(st, p, dv, s);
+  Decision r;
+  r.p = N; r.bpos = -1; r.bslot = -1; r.tgt = -1; r.evict = -1; r.sb = 0.f; r.pad[0] = r.pad[1] = 0;
+  if (has_b) {
+    const float sb = ranking_priority(a, u, N, state_readout<DV>(s_r[lane], tail, dv, s));
+    r.bpos = b;
+    r.bslot = bslot;
+    r.sb = sb;
+    if (ntk < K) {
+      r.tgt = base + ntk;   // fill-up: next free long-range slot, nobody leaves
+    } else if (K == 0) {
+      r.evict = bslot;
+    } else {
+      uint64_t best = s_best[0];
+      int mslot = s_slot[0];
+#pragma unroll
+      for (int w = 1; w < 4; ++w)
+        if (s_best[w] < best) { best = s_best[w]; mslot = s_slot[w]; }
+      if (rank_key(sb, b) > best) {
+        r.tgt = mslot;
+        r.evict = mslot;
+      } else {
+        r.evict = bslot;
+      }
+    }
+    if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0 && sb != sb) set_error(a.err, DEVERR_NAN_SCORE);
+  }
   if (lane == 0) a.dec[static_cast<size_t>(N & 1) * a.units + u] = r;
 }
 
@@ -314,8 +386,8 @@ __global__ void __launch_bounds__(32 * kMlstmWarps) mlstm_prefill_kernel(const L
 template <typename T, int X, int DV>
 int launch_step_t(const LayerArgs& a, const void* k_new, const void* v_new, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((a.units + kMlstmWarps - 1) / kMlstmWarps));
-  cfg.blockDim = dim3(32 * kMlstmWarps);
+  cfg.gridDim = dim3(static_cast<unsigned>(a.units));
+  cfg.blockDim = dim3(128);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
