@@ -1055,11 +1055,15 @@ int launch_attn_tc(const PaArgs& pa, int units, int n, cudaStream_t st) {
 //     S_1(t+1), O_1 += P_1 V(t), so the tensor cores work on one block while
 //     the other block's softmax runs; each tile's K and V serve both blocks;
 //   softmax warps 0-3 (block 0) and 4-7 (block 1): thread = query row = TMEM
-//     lane; S double-buffered in TMEM, P single-buffered in shared memory.
+//     lane; S double-buffered in TMEM, P double-buffered in shared memory, so
+//     a block's softmax of tile t + 1 need not wait for its P V of tile t
+//     (only a rescale of O, or reusing a P buffer, waits for an earlier P V).
 // TMEM: S[block][buf] at columns 32 * (2 block + buf), O[block] at 128 + block * DH.
+// Every mbarrier that a role may wait on twice in a row without an
+// intervening handoff is per buffer, so parity waits never alias.
 constexpr int kT2Rows = 256;
 constexpr int kT2Keys = 32;
-constexpr int kT2Stages = 3;
+constexpr int kT2Stages = 4;
 constexpr int kT2Threads = 13 * 32;
 constexpr int kT2Prod = 8;          // first producer warp
 constexpr int kT2Mma = 12;          // MMA warp
@@ -1073,11 +1077,11 @@ struct T2Smem {
   static constexpr size_t KV_TILE = static_cast<size_t>(QCH) * kT2Keys * 16;
   static constexpr size_t KV_OFF = Q_OFF + 2 * QBLK;                             // [stage][K, V]
   static constexpr size_t PBLK = static_cast<size_t>(kT2Keys / 8) * 128 * 16;
-  static constexpr size_t P_OFF = KV_OFF + 2 * kT2Stages * KV_TILE;             // [block]
-  static constexpr size_t META_OFF = P_OFF + 2 * PBLK;                           // [stage]{pos[keys], cut[keys], full}
+  static constexpr size_t P_OFF = KV_OFF + 2 * kT2Stages * KV_TILE;             // [block][buf]
+  static constexpr size_t META_OFF = P_OFF + 4 * PBLK;                           // [stage]{pos[keys], cut[keys], full}
   static constexpr int META_INTS = 2 * kT2Keys + 4;
   static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * kT2Stages * META_INTS;
-  static constexpr int NBAR = 2 * kT2Stages + 12;
+  static constexpr int NBAR = 2 * kT2Stages + 16;
   static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
   static constexpr size_t WT_OFF = TADDR_OFF + 16;
   static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);
@@ -1105,8 +1109,8 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
   uint64_t* kv_free = bars + kT2Stages;           // [stage], MMA commit
   uint64_t* s_full = bars + 2 * kT2Stages;        // [block][buf], MMA commit
   uint64_t* s_free = s_full + 4;                  // [block][buf], 128 softmax arrivals
-  uint64_t* p_full = s_free + 4;                  // [block], 128 softmax arrivals
-  uint64_t* o_done = p_full + 2;                  // [block], MMA commit
+  uint64_t* p_full = s_free + 4;                  // [block][buf], 128 softmax arrivals
+  uint64_t* o_done = p_full + 4;                  // [block][buf], MMA commit (P V of that buffer)
   uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_raw + SM::TADDR_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SM::TADDR_OFF + 4);
   int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
@@ -1136,8 +1140,6 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(&p_full[i], 128);
       mbar_init(&o_done[i], 1);
     }
@@ -1201,16 +1203,16 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         const unsigned bal = __ballot_sync(0xffffffffu, full);
         if (lane == 0) m[2 * kT2Keys] = (bal == 0xffffffffu);
       }
-      if (t >= 1) {   // tile t - 1 has landed: publish it
-        cp_async_wait<1>();
+      if (t >= kT2Stages - 1) {   // tile t - (stages - 1) has landed: publish it
+        cp_async_wait<kT2Stages - 1>();
         fence_proxy_async_smem();
-        mbar_arrive(&kv_full[(t - 1) % kT2Stages]);
+        mbar_arrive(&kv_full[(t - (kT2Stages - 1)) % kT2Stages]);
       }
     }
     cp_async_wait<0>();
-    if (ntiles >= 1 && !*abort_flag) {
+    if (!*abort_flag) {
       fence_proxy_async_smem();
-      mbar_arrive(&kv_full[(ntiles - 1) % kT2Stages]);
+      for (int t = max(0, ntiles - (kT2Stages - 1)); t < ntiles; ++t) mbar_arrive(&kv_full[t % kT2Stages]);
     }
   } else if (warp == kT2Mma) {
     // ---------------- MMA issue (one thread) ----------------
@@ -1230,17 +1232,17 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         return true;
       };
       auto issue_pv = [&](int X, int t) -> bool {
-        const int st = t % kT2Stages;
-        if (!wait(&p_full[X], t & 1)) return false;
+        const int st = t % kT2Stages, buf = t & 1;
+        if (!wait(&p_full[2 * X + buf], (t >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t pb = sbase + static_cast<uint32_t>(SM::P_OFF + X * SM::PBLK);
+        const uint32_t pb = sbase + static_cast<uint32_t>(SM::P_OFF + (2 * X + buf) * SM::PBLK);
         const uint32_t vb = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st + 1) * SM::KV_TILE);
         const uint32_t d = tmem + 128u + static_cast<uint32_t>(X * DH);
 #pragma unroll
         for (int kk = 0; kk < kT2Keys / 16; ++kk)
           tc_mma(d, tc_desc(pb + kk * 2 * kRowCells, kRowCells, 128), tc_desc(vb + kk * 256, 128, kKeyCells),
                  kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&o_done[X]);
+        tc_commit(&o_done[2 * X + buf]);
         return true;
       };
       bool ok = wait(&kv_full[0], 0) && issue_s(0, 0) && issue_s(1, 0);
@@ -1314,14 +1316,18 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         pk[i / 2] = pack_bf16(p0, p1);
       }
       l_run += psum;
-      // P_X and O_X are free once the previous tile's P V has completed
-      const bool freed = t == 0 || wait(&o_done[X], (t - 1) & 1);
+      // A rescale of O waits for every P V issued so far (the one of tile t - 1);
+      // reusing P buffer t & 1 waits for the P V of tile t - 2.
+      const bool any_resc = __any_sync(0xffffffffu, resc);
+      bool freed = true;
+      if (any_resc && t >= 1) freed = wait(&o_done[2 * X + ((t - 1) & 1)], ((t - 1) >> 1) & 1);
+      else if (t >= 2) freed = wait(&o_done[2 * X + (t & 1)], ((t - 2) >> 1) & 1);
       if (!__all_sync(0xffffffffu, freed)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (__any_sync(0xffffffffu, resc)) {
+      if (any_resc) {
         const float f = resc ? alpha : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < DH; c0 += 32) {
@@ -1333,17 +1339,17 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
-      uint8_t* pb = smem_raw + SM::P_OFF + X * SM::PBLK;
+      uint8_t* pb = smem_raw + SM::P_OFF + (2 * X + (t & 1)) * SM::PBLK;
 #pragma unroll
       for (int c = 0; c < kT2Keys / 8; ++c)
         *reinterpret_cast<uint4*>(pb + (static_cast<size_t>(c) * 128 + row) * 16) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[X]);
+      mbar_arrive(&p_full[2 * X + (t & 1)]);
     }
     bool fin = ok && ntiles > 0;
-    if (fin) fin = wait(&o_done[X], (ntiles - 1) & 1);
+    if (fin) fin = wait(&o_done[2 * X + ((ntiles - 1) & 1)], ((ntiles - 1) >> 1) & 1);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const int g = grow % G;
