@@ -111,11 +111,6 @@ struct kvpop_handle {
   std::vector<char> decoding;
   std::vector<CUtensorMap> maps;  // per layer: TMA view of the cache rows
   int test_hook = 0;              // failure injection (KVPOP_TEST_HOOKS builds only)
-  // Layer of the last enqueued call that wrote a layer's cache or counters
-  // (-1: none since creation, which synchronises).  A decode kernel whose
-  // layer differs may start loading cache rows before it waits for the
-  // kernel ahead of it in the stream (LayerArgs::early).
-  int last_write_layer = -1;
 };
 
 namespace {
@@ -271,13 +266,11 @@ int kvpop_prefill(kvpop_handle* h, int32_t layer, const void* k, const void* v, 
   if (launch_decide(a, h->cfg.dtype, n1, c1, static_cast<cudaStream_t>(stream)) != 0) return KVPOP_ERR_CUDA;
   h->n_seen[layer] = n1;
   h->n_topk[layer] = c1;
-  h->last_write_layer = layer;
   return KVPOP_OK;
 }
 
 namespace {
 void advance_mirror(kvpop_handle* h, int layer) {
-  h->last_write_layer = layer;
   const int S = h->cfg.sinks, W = h->cfg.window, D = h->cfg.delay;
   const int p = h->n_seen[layer];
   if (p - W - D >= S && h->n_topk[layer] < h->cfg.topk) h->n_topk[layer] += 1;
@@ -308,8 +301,7 @@ int kvpop_decode_attend(kvpop_handle* h, int32_t layer, const void* q, void* out
   if (!q || !out) return KVPOP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out)) return KVPOP_ERR_INVALID_ARG;
   if (h->n_seen[layer] == 0) return KVPOP_ERR_ORDER;
-  LayerArgs a = layer_args(h, layer);
-  a.early = h->last_write_layer != layer ? 1 : 0;
+  const LayerArgs a = layer_args(h, layer);
   const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, decode_scratch(h), MODE_ATTEND, q, nullptr, nullptr,
                               nullptr, out, h->num_sms, static_cast<cudaStream_t>(stream));
   if (r == -2) return KVPOP_ERR_BAD_SHAPE;
@@ -324,8 +316,7 @@ int kvpop_decode_step(kvpop_handle* h, int32_t layer, const void* q, const void*
   const bool ext = (h->cfg.flags & KVPOP_FLAG_EXTERNAL_SCORES) != 0;
   if (ext && !ext_score) return KVPOP_ERR_INVALID_ARG;
   if (h->n_seen[layer] >= h->cfg.max_context) return KVPOP_ERR_CONTEXT_OVERFLOW;
-  LayerArgs a = layer_args(h, layer);
-  a.early = h->last_write_layer != layer ? 1 : 0;
+  const LayerArgs a = layer_args(h, layer);
   if (a.mlstm && launch_mlstm_step(a, h->cfg.dtype, k_new, v_new, static_cast<cudaStream_t>(stream)) != 0)
     return KVPOP_ERR_CUDA;
   const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, decode_scratch(h), a.mlstm ? MODE_STEP_NODECIDE : MODE_STEP,
@@ -476,7 +467,6 @@ int kvpop_prefill_with_attention(kvpop_handle* h, int32_t layer, const void* q, 
   if (launch_decide(a, h->cfg.dtype, n_tokens, c1, st) != 0) return KVPOP_ERR_CUDA;
   h->n_seen[layer] = n_tokens;
   h->n_topk[layer] = c1;
-  h->last_write_layer = layer;
   return KVPOP_OK;
 }
 
@@ -581,8 +571,7 @@ extern "C" int kvpop_decode_step_noalloc(kvpop_handle* h, int32_t layer, const v
   // the tickets count arrivals from zero; a call that gave up on a wait can
   // leave them non-zero, and another handle may have used more units
   if (cudaMemsetAsync(sc.ticket, 0, ticket_bytes, st) != cudaSuccess) return KVPOP_ERR_CUDA;
-  LayerArgs a = layer_args(h, layer);
-  a.early = h->last_write_layer != layer ? 1 : 0;
+  const LayerArgs a = layer_args(h, layer);
   if (a.mlstm && launch_mlstm_step(a, h->cfg.dtype, k_new, v_new, st) != 0) return KVPOP_ERR_CUDA;
   const int r = launch_decode(h->maps[layer], a, h->cfg.dtype, sc, a.mlstm ? MODE_STEP_NODECIDE : MODE_STEP, q, k_new,
                               v_new, ext ? ext_score : nullptr, out, h->num_sms, st);

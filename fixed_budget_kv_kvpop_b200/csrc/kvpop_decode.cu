@@ -517,8 +517,7 @@ __device__ __forceinline__ void l2_warmup(const LayerArgs& a, bool step, int war
     if (gw >= nw) return;
     const int64_t lo = seg_lo(gw, total, nw);
     const int64_t cnt = seg_lo(gw + 1, total, nw) - lo;
-    const int first = (a.early && step) ? KVPOP_NSTG : 0;   // those stages are loaded before the wait
-    for (int i = first; i < first + kPrefetchTiles && i < cnt; ++i) {
+    for (int i = 0; i < kPrefetchTiles && i < cnt; ++i) {
       const int64_t t = lo + i;
       const int64_t u = t / tpu;
       const int jt = static_cast<int>(t - u * tpu);
@@ -580,39 +579,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   // prologue as SMs free up, and wait here until the previous one has
   // completed and its writes are visible (everything below reads its results).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // When the previous kernel in the stream did not write this layer (a.early),
-  // the layer's counters and cache rows are final already: consumer warps
-  // start loading their first NSTG tiles before waiting for that kernel.
-  const bool early = step && a.early && (smem_u32(smem) & 1023u) == 0u;
-  int Ne = 0, ntke = 0, pre_issued = 0;
-  if (early) {
-    __syncthreads();   // mbarrier initialisation visible to the TMA
-    Ne = ld_relaxed(&a.layer->n_seen);
-    ntke = ld_relaxed(&a.layer->n_topk);
-    if (warp < NCW && Ne >= 1 && Ne < a.max_context && ntke >= 0 && ntke <= a.K) {
-      const int tpu_e = (a.S + a.W + a.D + ntke + TS - 1) / TS;
-      const int64_t total_e = static_cast<int64_t>(a.units) * tpu_e;
-      const int64_t nw_e = decode_active_warps(total_e, tpu_e, static_cast<int64_t>(gridDim.x) * NCW);
-      const int64_t gw_e = static_cast<int64_t>(blockIdx.x) * NCW + warp;
-      if (gw_e < nw_e) {
-        const int64_t lo_e = seg_lo(gw_e, total_e, nw_e);
-        const int64_t cnt_e = seg_lo(gw_e + 1, total_e, nw_e) - lo_e;
-        pre_issued = static_cast<int>(cnt_e < NSTG ? cnt_e : NSTG);
-        uint8_t* ring_e = smem + SM::RINGS + warp * NSTG * GE::STAGE;
-        uint64_t* fb_e = full_bar + warp * NSTG;
-        for (int i = 0; i < pre_issued; ++i) {
-          const int64_t t = lo_e + i;
-          const int64_t u = t / tpu_e;
-          const int jt = static_cast<int>(t - u * tpu_e);
-          if (lane == 0) mbar_arrive_expect_tx(&fb_e[i], GE::STAGE);
-          __syncwarp();
-          if (lane < GE::NBLK)
-            tma_load_2d(ring_e + i * GE::STAGE + lane * GE::BOX, &tmap, lane * GE::BOXELEMS,
-                        static_cast<int>(u * a.NS + jt * TS), &fb_e[i]);
-        }
-      }
-    }
-  }
   l2_warmup<NCW>(a, step, warp, lane);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
@@ -621,11 +587,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     return;
   }
 
-  const int N = early ? Ne : a.layer->n_seen;      // the cache holds tokens 0..N-1
-  const int ntk = early ? ntke : a.layer->n_topk;
-  if (early && (a.flags & FLAG_DEBUG_CHECKS) && threadIdx.x == 0 &&
-      (a.layer->n_seen != Ne || a.layer->n_topk != ntke))
-    set_error(a.err, DEVERR_STATE_MISMATCH);
+  const int N = a.layer->n_seen;      // the cache holds tokens 0..N-1
+  const int ntk = a.layer->n_topk;
   const int S = a.S, W = a.W, D = a.D, K = a.K;
   if (step && N >= a.max_context) {
     if (threadIdx.x == 0) set_error(a.err, DEVERR_CONTEXT_OVERFLOW);
@@ -956,14 +919,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   issue_q(cu, 0);
   {
     const int npre = cnt < NSTG ? cnt : NSTG;
-    if (pre_issued == npre) {   // loaded before the wait: advance the issue cursor only
-      for (int i = 0; i < npre; ++i) {
-        if (++ij == tpu) { ij = 0; ++iu; }
-        if (++istage == NSTG) istage = 0;
-      }
-    } else {
-      for (int i = 0; i < npre; ++i) issue_next();
-    }
+    for (int i = 0; i < npre; ++i) issue_next();
   }
   int cstage = 0;
   uint32_t cphase = 0;

@@ -94,9 +94,6 @@ struct LayerArgs {
   const float* mw;      // this layer's weights [Hkv][mlstm_head_floats(p, dv, d)]
   double* mstate;       // this layer's states [units][mlstm_state_doubles(p, dv)]
   int test_hook;        // failure injection, honoured only by builds with KVPOP_TEST_HOOKS
-  int early;            // 1: the kernel just before this one in the stream did not write this layer's
-                        // cache or counters, so a decode kernel may start loading cache rows before
-                        // it waits for that kernel (programmatic dependent launch)
 };
 
 // test_hook values (KVPOP_TEST_HOOKS builds): consumer warp 0 of CTA 0 does

@@ -1061,9 +1061,17 @@ int launch_attn_tc(const PaArgs& pa, int units, int n, cudaStream_t st) {
 // TMEM: S[block][buf] at columns 32 * (2 block + buf), O[block] at 128 + block * DH.
 // Every mbarrier that a role may wait on twice in a row without an
 // intervening handoff is per buffer, so parity waits never alias.
+// 2^x with the hardware's approximate base-2 exponential (ftz; 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 constexpr int kT2Rows = 256;
 constexpr int kT2Keys = 32;
 constexpr int kT2Stages = 4;
+constexpr int kT2Lag = kT2Stages - 2;   // tiles a producer keeps in flight beyond the one it publishes
 constexpr int kT2Threads = 13 * 32;
 constexpr int kT2Prod = 8;          // first producer warp
 constexpr int kT2Mma = 12;          // MMA warp
@@ -1203,16 +1211,21 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         const unsigned bal = __ballot_sync(0xffffffffu, full);
         if (lane == 0) m[2 * kT2Keys] = (bal == 0xffffffffu);
       }
-      if (t >= kT2Stages - 1) {   // tile t - (stages - 1) has landed: publish it
-        cp_async_wait<kT2Stages - 1>();
+      // Publish tile t - kT2Lag once it has landed.  The lag is at most
+      // stages - 2: the MMA thread needs tile t + 1 (for S(t + 1)) before it
+      // issues P V(t), whose completion frees the stage that tile t + stages
+      // reuses, so tile t + 1 must be published before the producer waits for
+      // that stage.
+      if (t >= kT2Lag) {
+        cp_async_wait<kT2Lag>();
         fence_proxy_async_smem();
-        mbar_arrive(&kv_full[(t - (kT2Stages - 1)) % kT2Stages]);
+        mbar_arrive(&kv_full[(t - kT2Lag) % kT2Stages]);
       }
     }
     cp_async_wait<0>();
     if (!*abort_flag) {
       fence_proxy_async_smem();
-      for (int t = max(0, ntiles - (kT2Stages - 1)); t < ntiles; ++t) mbar_arrive(&kv_full[t % kT2Stages]);
+      for (int t = max(0, ntiles - kT2Lag); t < ntiles; ++t) mbar_arrive(&kv_full[t % kT2Stages]);
     }
   } else if (warp == kT2Mma) {
     // ---------------- MMA issue (one thread) ----------------
@@ -1281,12 +1294,14 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
       tc_ld32(tmem + 32u * (2 * X + buf) + lrow, sv);
       tc_fence_before();
       mbar_arrive(&s_free[2 * X + buf]);
+      // mask on the raw logits; the tile max commutes with the positive scale,
+      // so each weight is one FMA and one ex2: p = 2^(s * scale - m)
       const int* m = meta + st * SM::META_INTS;
       float tmax = -INFINITY;
       if (m[2 * kT2Keys]) {
 #pragma unroll
         for (int i = 0; i < kT2Keys; ++i) {
-          sv[i] = vrow ? sv[i] * p.scale_log2 : -INFINITY;
+          if (!vrow) sv[i] = -INFINITY;
           tmax = fmaxf(tmax, sv[i]);
         }
       } else {
@@ -1294,24 +1309,26 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         for (int i = 0; i < kT2Keys; ++i) {
           const int j = m[i];
           const bool vis = j >= 0 && vrow && j <= qpos && (j < S || j > mrow || m[kT2Keys + i] > mrow);
-          sv[i] = vis ? sv[i] * p.scale_log2 : -INFINITY;
+          sv[i] = vis ? sv[i] : -INFINITY;
           tmax = fmaxf(tmax, sv[i]);
         }
       }
+      const float tm = tmax * p.scale_log2;
       float alpha = 1.f;
       bool resc = false;
-      if (tmax > m_run + kTcLazy) {
+      if (tm > m_run + kTcLazy) {
         resc = (m_run != -INFINITY);
-        alpha = resc ? exp2f(m_run - tmax) : 0.f;
+        alpha = resc ? ex2_approx(m_run - tm) : 0.f;
         l_run *= alpha;
-        m_run = tmax;
+        m_run = tm;
       }
+      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;   // masked logits give 2^-inf = 0
       float psum = 0.f;
       uint32_t pk[kT2Keys / 2];
 #pragma unroll
       for (int i = 0; i < kT2Keys; i += 2) {
-        const float p0 = sv[i] == -INFINITY ? 0.f : exp2f(sv[i] - m_run);
-        const float p1 = sv[i + 1] == -INFINITY ? 0.f : exp2f(sv[i + 1] - m_run);
+        const float p0 = ex2_approx(fmaf(sv[i], p.scale_log2, nm));
+        const float p1 = ex2_approx(fmaf(sv[i + 1], p.scale_log2, nm));
         psum += p0 + p1;
         pk[i / 2] = pack_bf16(p0, p1);
       }
