@@ -53,21 +53,19 @@ constexpr float kLazy = 8.0f;                        // lazy rescale threshold (
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Launch shape of the decode kernel: consumer warps per CTA, shared-memory
-// stages per consumer warp, decider warps per CTA, tiles per consumer warp
-// prefetched into L2 before the wait for the previous kernel.
-#ifndef KVPOP_NCW
-#define KVPOP_NCW 10
-#endif
-#ifndef KVPOP_NSTG
-#define KVPOP_NSTG 2
-#endif
-#ifndef KVPOP_NDW
-#define KVPOP_NDW 2
-#endif
-#ifndef KVPOP_PFT
-#define KVPOP_PFT 2
-#endif
-constexpr int NDW = KVPOP_NDW;
+// stages per consumer warp, decider warps per CTA.  bf16 consumers run both
+// contractions on the tensor cores and need few warps to keep HBM busy;
+// keeping fewer tiles in flight also keeps the memory latency that the
+// deciders' dependent loads and the merges see short.  fp32 consumers (FMA
+// pipes) are issue-bound and take more warps.
+template <typename T, int G>
+struct LaunchShape {
+  static constexpr int NCW = sizeof(T) == 2 ? 6 : (G > 4 ? 8 : 10);
+  static constexpr int NSTG = 2;
+  static constexpr int NDW = sizeof(T) == 2 ? 4 : 2;
+};
+// Tiles per consumer warp prefetched into L2 before the wait for the previous kernel.
+constexpr int kPrefetchTiles = 2;
 
 // A tile is TS rows [k | v]; it lands in shared memory as NBLK boxes of
 // TS rows x 128 bytes (box b holds bytes [128 b, 128 b + 128) of every row),
@@ -499,9 +497,8 @@ __device__ __noinline__ void merge_unit(const LayerArgs& a, const DecodeScratch&
 // its array.  Consumer warps: the first kPrefetchTiles tiles of their range.
 // Decider warps: the long-range keys and candidate boundary rows of their
 // units, and (one CTA per KV head) that head's scorer weights.
-template <int NCW>
+template <int NCW, int NDW>
 __device__ __forceinline__ void l2_warmup(const LayerArgs& a, bool step, int warp, int lane) {
-  constexpr int kPrefetchTiles = KVPOP_PFT;
   if (lane != 0) return;
   const int N = ld_relaxed(&a.layer->n_seen);
   const int ntk = ld_relaxed(&a.layer->n_topk);
@@ -553,7 +550,7 @@ __device__ __forceinline__ void l2_warmup(const LayerArgs& a, bool step, int war
   }
 }
 
-template <typename T, int DH, int G, int NCW, int NSTG>
+template <typename T, int DH, int G, int NCW, int NSTG, int NDW>
 __global__ void __launch_bounds__((NCW + NDW) * 32, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ LayerArgs a,
               const __grid_constant__ DecodeScratch sc, const int mode, const T* __restrict__ q,
@@ -579,7 +576,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
   // prologue as SMs free up, and wait here until the previous one has
   // completed and its writes are visible (everything below reads its results).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  l2_warmup<NCW>(a, step, warp, lane);
+  l2_warmup<NCW, NDW>(a, step, warp, lane);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
   if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled boxes need 1024-byte alignment
@@ -613,21 +610,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     if (lane == 0) sc.ticket[unit] = 0;
   };
   // Queue a unit whose contributors have all arrived, for this CTA's merge
-  // helpers.  The queue is a ring of kMergeCap entries (0 = empty, else unit + 1);
-  // when it is full the pusher waits for the helpers (bounded).  If that wait
-  // gives up, the entry is not written (its ring slot still holds a unit not
-  // yet merged): the error word reports the timeout and the step's outputs
-  // are undefined, but no other unit's merge is lost.
+  // helpers: a ring of kMergeCap entries (0 = empty, else unit + 1) followed
+  // by its tail counter.  The pusher claims a slot, then fills its entry once
+  // the helper that took the previous value there has emptied it (bounded
+  // wait); helpers take entries by exchange with 0, so every value is taken
+  // once.  If the wait gives up, the unit is dropped: the error word reports
+  // the timeout and the step's outputs are undefined.
   auto push_merge = [&](int64_t unit) {
     if (lane == 0) {
       const int slot = atomicAdd(&mq[kMergeCap], 1);
       const uint64_t t0 = global_ns();
-      bool full = false;
-      while (slot - atomicAdd(&mq[kMergeCap + 1], 0) >= kMergeCap) {
-        if (global_ns() - t0 > kMergeWaitLimitNs) { set_error(a.err, DEVERR_TIMEOUT); full = true; break; }
-        __nanosleep(128);
+      while (atomicCAS(&mq[slot % kMergeCap], 0, static_cast<int>(unit) + 1) != 0) {
+        if (global_ns() - t0 > kMergeWaitLimitNs) { set_error(a.err, DEVERR_TIMEOUT); break; }
+        __nanosleep(64);
       }
-      if (!full) atomicExch(&mq[slot % kMergeCap], static_cast<int>(unit) + 1);
     }
     __syncwarp();
   };
@@ -658,6 +654,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
             got = v > 0 ? v - 1 : -3;
           }
         } else if (atomicAdd(&mq[kMergeCap + 2], 0) == NCW) {
+          __threadfence_block();
           if (head >= atomicAdd(&mq[kMergeCap], 0)) got = -2;
         }
       }
@@ -697,16 +694,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     __syncwarp();
     if (lane == 0) {
       __threadfence();
-#ifdef KVPOP_CTA_FINISH
-      // count the CTA's warps in shared memory; its last warp reports the CTA
-      if (atomicAdd(&mq[kMergeCap + 3], 1) != NCW + NDW - 1) return;
-      __threadfence();
-      const int prev = atomicAdd(&a.layer->ticket, 1);
-      if (prev == static_cast<int>(gridDim.x) - 1) {
-#else
       const int prev = atomicAdd(&a.layer->ticket, 1);
       if (prev == static_cast<int>(gridDim.x) * (NCW + NDW) - 1) {
-#endif
         a.layer->n_seen = N + 1;
         a.layer->n_topk = ntk_after;
         a.layer->ticket = 0;
@@ -787,125 +776,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     if (++ij == tpu) { ij = 0; ++iu; }
     if (++istage == NSTG) istage = 0;
   };
-
-  const int j = lane & 15;        // QK: slot of the tile
-  const int h = lane >> 4;        // QK: half of the dims
-  const int gq = lane / GE::LPS;  // PV: slot group
-  const int c = lane % GE::LPS;   // PV: chunk of the value row
-
-  float2 acc[G][GE::EPC / 2];
-  float m[G], lp[G];
-  int evict = -1;
-  int cur = -1;
-  int pend_unit = -1, pend_prev = 0;   // last finished segment, its ticket result
-  int qbuf = 0;
-  uint32_t qphase = 0;   // bit b = parity of raw buffer b's next completion
-
-  // Start a unit segment: q into the fp32 layout, reset the softmax state,
-  // fold the new token in if this warp holds the unit's first tile, and
-  // prefetch the next unit's q.
-  auto start_unit = [&](int unit, bool first_tile) {
-    if (!mbar_wait(&qb[qbuf], (qphase >> qbuf) & 1u)) {
-      if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
-    }
-    qphase ^= 1u << qbuf;
-    const uint8_t* raw = qraw + qbuf * SM::QRB;
-    __syncwarp();
-    float* qf = reinterpret_cast<float*>(qsm);
-    const T* qr = reinterpret_cast<const T*>(raw);
-    for (int idx = lane; idx < G * DH; idx += 32) {
-      const int g = idx / DH, dim = idx % DH;
-      const int ch = dim / GE::EPC, e = dim % GE::EPC;
-      const int hh = ch / GE::CH, cc = ch % GE::CH;
-      qf[hh * ((GE::QHALF + 16) / 4) + (cc * G + g) * GE::EPC + e] = Elem<T>::to_f32(qr[idx]) * qscale;
-    }
-    evict = step ? reinterpret_cast<const Decision*>(raw + G * DH * GE::ESZ + 2 * DH * GE::ESZ)->evict : -1;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      m[g] = kNegInf;
-      lp[g] = 0.f;
-#pragma unroll
-      for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = make_float2(0.f, 0.f);
-    }
-    if (step && first_tile) {
-      // the appended token: score q . k_new and take it as the first slot
-      constexpr int DPL = DH / 32;
-      const T* kn = reinterpret_cast<const T*>(raw + G * DH * GE::ESZ);
-      const T* vn = kn + DH;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float part = 0.f;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e)
-          part = fmaf(Elem<T>::to_f32(qr[g * DH + lane * DPL + e]), Elem<T>::to_f32(kn[lane * DPL + e]), part);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        m[g] = part * qscale;   // p = exp2(s - m) = 1
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) lp[g] = 1.f;
-      }
-      if (gq == 0) {
-        const uint4 vr = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vn) + c * 16);
-        float2 v2[GE::EPC / 2];
-        if constexpr (sizeof(T) == 2) {
-          v2[0] = bf2_to_f2(vr.x); v2[1] = bf2_to_f2(vr.y); v2[2] = bf2_to_f2(vr.z); v2[3] = bf2_to_f2(vr.w);
-        } else {
-          v2[0] = make_float2(__uint_as_float(vr.x), __uint_as_float(vr.y));
-          v2[1] = make_float2(__uint_as_float(vr.z), __uint_as_float(vr.w));
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = v2[e];
-      }
-    }
-    __syncwarp();
-    if (unit < last_unit) issue_q(unit + 1, qbuf ^ 1);
-    qbuf ^= 1;
-  };
-
-  auto finalize = [&](int unit) {
-    float l[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float v = lp[g];
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      l[g] = v;
-    }
-#pragma unroll
-    for (int o = GE::LPS; o < 32; o <<= 1)
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < GE::EPC / 2; ++e) {
-          acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, o);
-          acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, o);
-        }
-    const int64_t first = warp_of_tile(static_cast<int64_t>(unit) * tpu, total, nw);
-    const int seg = static_cast<int>(gw - first);
-    if (seg >= kMaxSeg) {  // cannot happen: decode_active_warps bounds the segments
-      if (lane == 0) set_error(a.err, DEVERR_BAD_INDEX);
-      return;
-    }
-    float* pa = sc.part_acc + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * DH);
-    float* pmv = sc.part_ml + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * 2);
-    if (lane < GE::LPS) {
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < GE::EPC / 2; ++e)
-          *reinterpret_cast<float2*>(pa + g * DH + c * GE::EPC + 2 * e) = acc[g][e];
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) { pmv[2 * g] = m[g]; pmv[2 * g + 1] = l[g]; }
-    }
-    pend_unit = unit;
-    pend_prev = arrive(unit);   // checked later, so the atomic's round trip overlaps streaming
-  };
+  // last finished segment and its ticket result, checked one segment later
+  int pend_unit = -1, pend_prev = 0;
   auto check_pending = [&]() {
     if (pend_unit < 0) return;
     const int prev = __shfl_sync(0xffffffffu, pend_prev, 0);
@@ -913,183 +785,536 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
     pend_unit = -1;
   };
 
-  // consume cursor
-  int cu = static_cast<int>(lo / tpu), cj = static_cast<int>(lo - static_cast<int64_t>(cu) * tpu);
-  // first unit's q before the tile burst (it would queue behind it otherwise)
-  issue_q(cu, 0);
-  {
-    const int npre = cnt < NSTG ? cnt : NSTG;
-    for (int i = 0; i < npre; ++i) issue_next();
-  }
-  int cstage = 0;
-  uint32_t cphase = 0;
-  bool failed = false;
-  int failed_at = -1;
-  for (int i = 0; i < cnt; ++i) {
-    const int s0 = cj * TS;
-    const int nsl = min(TS, vg.nse - s0);
-    if (cu != cur) {
-      if (cur >= 0) {
-        check_pending();
-        finalize(cur);
-      }
-      cur = cu;
-      start_unit(cu, cj == 0);
-    }
-    if (!mbar_wait(&fb[cstage], cphase)) {
-      if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
-      failed = true;
-      failed_at = i;
-      break;
-    }
-    const uint8_t* tile = ring + cstage * GE::STAGE;
+  if constexpr (sizeof(T) == 2) {
+    // ---- bf16: both contractions of a tile on the tensor cores ----
+    // mma.sync m16n8k16, fp32 accumulate.  S = Q K^T with the G query heads
+    // as the M rows (rows G..15 zero) and the tile's 16 slots as two n-blocks;
+    // O^T = V^T P^T with the head dims as M (DH / 16 blocks) and the heads as
+    // N, so the S fragment of a tile, rounded to bf16, is the B fragment of
+    // its P V as it stands.  Lane (gid, tig) = (lane / 4, lane % 4) keeps the
+    // softmax state of head gid over slots 2 tig, 2 tig + 1, 8 + 2 tig,
+    // 9 + 2 tig, and O^T of heads 2 tig, 2 tig + 1 at dims 16 mb + gid and
+    // 16 mb + gid + 8.  K and V fragments come from the swizzled tile by
+    // ldmatrix (row addresses of 8 consecutive slots hit 8 distinct bank
+    // groups).  Per tile and warp: 2 DH / 16 ldmatrix, 3 DH / 16 MMAs.
+    constexpr int KS = DH / 16;
+    const int gid = lane >> 2, tig = lane & 3;
+    const bool hreal = gid < G;
+    const int lslot = 8 * (lane >> 4) + (lane & 7);   // ldmatrix row: matrix lane / 8, row lane % 8
+    const int lhalf = (lane >> 3) & 1;                // second 8-element half of the 16
+    uint32_t qa[KS][2];
+    float o[KS][4];
+    float m_run = kNegInf, l_run = 0.f;
+    int evict = -1;
+    int cur = -1;
+    int qbuf = 0;
+    uint32_t qphase = 0;   // bit b = parity of raw buffer b's next completion
 
-    // ---- QK: lane (j, h) = slot j, dims of half h, all G heads ----
-    float s[G];
-    {
-      float2 sa[G][2];
+    // Start a unit segment: q into A fragments, reset the softmax state, fold
+    // the new token in if this warp holds the unit's first tile, and prefetch
+    // the next unit's q.
+    auto start_unit = [&](int unit, bool first_tile) {
+      if (!mbar_wait(&qb[qbuf], (qphase >> qbuf) & 1u)) {
+        if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+      }
+      qphase ^= 1u << qbuf;
+      const uint8_t* raw = qraw + qbuf * SM::QRB;
+      __syncwarp();
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(raw);   // q as bf16 pairs, [G][DH / 2]
 #pragma unroll
-      for (int g = 0; g < G; ++g) { sa[g][0] = make_float2(0.f, 0.f); sa[g][1] = make_float2(0.f, 0.f); }
-      const float* qh = reinterpret_cast<const float*>(qsm + h * (GE::QHALF + 16));
+      for (int ks = 0; ks < KS; ++ks) {
+        qa[ks][0] = hreal ? qw[(gid * DH + ks * 16 + 2 * tig) >> 1] : 0u;
+        qa[ks][1] = hreal ? qw[(gid * DH + ks * 16 + 8 + 2 * tig) >> 1] : 0u;
+      }
+      evict = step ? reinterpret_cast<const Decision*>(raw + G * DH * GE::ESZ + 2 * DH * GE::ESZ)->evict : -1;
+      m_run = kNegInf;
+      l_run = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < GE::CH; ++cc) {
-        const uint4 kr = *reinterpret_cast<const uint4*>(tile + GE::off(j, h * GE::CH + cc));
-        float2 k2[GE::EPC / 2];
-        if constexpr (sizeof(T) == 2) {
-          k2[0] = bf2_to_f2(kr.x); k2[1] = bf2_to_f2(kr.y); k2[2] = bf2_to_f2(kr.z); k2[3] = bf2_to_f2(kr.w);
-        } else {
-          k2[0] = make_float2(__uint_as_float(kr.x), __uint_as_float(kr.y));
-          k2[1] = make_float2(__uint_as_float(kr.z), __uint_as_float(kr.w));
-        }
+      for (int mb = 0; mb < KS; ++mb)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) o[mb][r] = 0.f;
+      if (step && first_tile) {
+        // the appended token: score q . k_new and take it as the first slot
+        constexpr int DPL = DH / 32;
+        const T* qr = reinterpret_cast<const T*>(raw);
+        const T* kn = qr + G * DH;
+        const T* vn = kn + DH;
+        float mnew = kNegInf;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float4* qp = reinterpret_cast<const float4*>(qh + (cc * G + g) * GE::EPC);
+          float part = 0.f;
 #pragma unroll
-          for (int e4 = 0; e4 < GE::EPC / 4; ++e4) {
-            const float4 qv = qp[e4];
-            sa[g][e4 & 1] = ffma2(make_float2(qv.x, qv.y), k2[2 * e4], sa[g][e4 & 1]);
-            sa[g][e4 & 1] = ffma2(make_float2(qv.z, qv.w), k2[2 * e4 + 1], sa[g][e4 & 1]);
-          }
+          for (int e = 0; e < DPL; ++e)
+            part = fmaf(Elem<T>::to_f32(qr[g * DH + lane * DPL + e]), Elem<T>::to_f32(kn[lane * DPL + e]), part);
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
+          if (g == gid) mnew = part * qscale;   // p = exp2(s - m) = 1
+        }
+        m_run = mnew;
+        l_run = (hreal && tig == 0) ? 1.f : 0.f;
+#pragma unroll
+        for (int mb = 0; mb < KS; ++mb) {
+          const float v0 = Elem<T>::to_f32(vn[16 * mb + gid]);
+          const float v1 = Elem<T>::to_f32(vn[16 * mb + gid + 8]);
+          o[mb][0] = v0; o[mb][1] = v0; o[mb][2] = v1; o[mb][3] = v1;
         }
       }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float v = (sa[g][0].x + sa[g][0].y) + (sa[g][1].x + sa[g][1].y);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        s[g] = v;
-      }
-    }
-    // Slot validity: a tile of occupied slots without the evicted one (the
-    // common case) needs no per-slot test.
-    bool valid = true;
-    uint32_t vmask = 0xffffu;
-    if (!(vg.full && s0 + TS <= vg.nse && (evict < s0 || evict >= s0 + TS))) {
-      const int slot = s0 + j;
-      valid = (j < nsl) && (slot != evict) && vg.slot_ok(slot);
-      vmask = __ballot_sync(0xffffffffu, valid) & 0xffffu;
-    }
-    // ---- online softmax (exp2 domain, lazy rescale) ----
-    float sv[G];
-    bool in_range = true;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      sv[g] = valid ? s[g] : kNegInf;
-      in_range = in_range && (sv[g] <= m[g] + kLazy);
-    }
-    // The running max moves only when a tile exceeds it by 2^kLazy; one vote
-    // tells whether any score of the tile does, else no tile max is needed.
-    if (!__all_sync(0xffffffffu, in_range)) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float mt = sv[g];
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-        if (mt > m[g] + kLazy) {   // warp-uniform
-          const float alpha = (m[g] == kNegInf) ? 0.f : fast_exp2(m[g] - mt);
-          m[g] = mt;
-          lp[g] *= alpha;
-#pragma unroll
-          for (int e = 0; e < GE::EPC / 2; ++e) {
-            acc[g][e].x *= alpha;
-            acc[g][e].y *= alpha;
-          }
-        }
-      }
-    }
-    float p[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      p[g] = valid ? fast_exp2(sv[g] - m[g]) : 0.f;
-      lp[g] += p[g];
-    }
-    if (h == 0) {
-      float* pd = reinterpret_cast<float*>(psm + j * GE::PSLOT + (j / GE::SPG) * 16);
-#pragma unroll
-      for (int g = 0; g < G; g += 2) {
-        if (g + 1 < G)
-          *reinterpret_cast<float4*>(pd + 2 * g) = make_float4(p[g], p[g], p[g + 1], p[g + 1]);
-        else
-          *reinterpret_cast<float2*>(pd + 2 * g) = make_float2(p[g], p[g]);
-      }
-    }
-    __syncwarp();
-    // ---- PV: lane (gq, c) = slots of group gq, value chunk c ----
-    auto pv_slot = [&](int j2) {
-      const float* pp = reinterpret_cast<const float*>(psm + j2 * GE::PSLOT + (j2 / GE::SPG) * 16);
-      float2 pr[G];
-#pragma unroll
-      for (int g = 0; g < G; g += 2) {
-        if (g + 1 < G) {
-          const float4 t4 = *reinterpret_cast<const float4*>(pp + 2 * g);
-          pr[g] = make_float2(t4.x, t4.y);
-          pr[g + 1] = make_float2(t4.z, t4.w);
-        } else {
-          pr[g] = *reinterpret_cast<const float2*>(pp + 2 * g);
-        }
-      }
-      const uint4 vr = *reinterpret_cast<const uint4*>(tile + GE::off(j2, GE::NCHK + c));
-      float2 v2[GE::EPC / 2];
-      if constexpr (sizeof(T) == 2) {
-        v2[0] = bf2_to_f2(vr.x); v2[1] = bf2_to_f2(vr.y); v2[2] = bf2_to_f2(vr.z); v2[3] = bf2_to_f2(vr.w);
-      } else {
-        v2[0] = make_float2(__uint_as_float(vr.x), __uint_as_float(vr.y));
-        v2[1] = make_float2(__uint_as_float(vr.z), __uint_as_float(vr.w));
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = ffma2(pr[g], v2[e], acc[g][e]);
+      __syncwarp();
+      if (unit < last_unit) issue_q(unit + 1, qbuf ^ 1);
+      qbuf ^= 1;
     };
-    if (vmask == 0xffffu) {
-#pragma unroll
-      for (int jj = 0; jj < GE::SPG; ++jj) pv_slot(gq * GE::SPG + jj);
-    } else {
-#pragma unroll
-      for (int jj = 0; jj < GE::SPG; ++jj) {
-        const int j2 = gq * GE::SPG + jj;
-        if ((vmask >> j2) & 1u) pv_slot(j2);
+
+    auto finalize = [&](int unit) {
+      float l = l_run;
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const int64_t first = warp_of_tile(static_cast<int64_t>(unit) * tpu, total, nw);
+      const int seg = static_cast<int>(gw - first);
+      if (seg >= kMaxSeg) {  // cannot happen: the split bounds the segments per unit
+        if (lane == 0) set_error(a.err, DEVERR_BAD_INDEX);
+        return;
       }
+      float* pa = sc.part_acc + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * DH);
+      float* pmv = sc.part_ml + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * 2);
+#pragma unroll
+      for (int mb = 0; mb < KS; ++mb)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int hh = 2 * tig + (r & 1);
+          if (hh < G) pa[hh * DH + 16 * mb + gid + 8 * (r >> 1)] = o[mb][r];
+        }
+      if (tig == 0 && hreal) {
+        pmv[2 * gid] = m_run;
+        pmv[2 * gid + 1] = l;
+      }
+      pend_unit = unit;
+      pend_prev = arrive(unit);   // checked later, so the atomic's round trip overlaps streaming
+    };
+
+    // consume cursor
+    int cu = static_cast<int>(lo / tpu), cj = static_cast<int>(lo - static_cast<int64_t>(cu) * tpu);
+    // first unit's q before the tile burst (it would queue behind it otherwise)
+    issue_q(cu, 0);
+    {
+      const int npre = cnt < NSTG ? cnt : NSTG;
+      for (int i = 0; i < npre; ++i) issue_next();
     }
-    __syncwarp();
-    if (i + NSTG < cnt) {
-      fence_proxy_async_smem();
-      issue_next();
+    int cstage = 0;
+    uint32_t cphase = 0;
+    bool failed = false;
+    int failed_at = -1;
+    for (int i = 0; i < cnt; ++i) {
+      const int s0 = cj * TS;
+      if (cu != cur) {
+        if (cur >= 0) {
+          check_pending();
+          finalize(cur);
+        }
+        cur = cu;
+        start_unit(cu, cj == 0);
+      }
+      if (!mbar_wait(&fb[cstage], cphase)) {
+        if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+        failed = true;
+        failed_at = i;
+        break;
+      }
+      uint8_t* tile = ring + cstage * GE::STAGE;
+      const uint32_t tb = smem_u32(tile);
+
+      // ---- S = Q K^T ----
+      float sacc[2][4];
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sacc[nb][r] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t kb[4];
+        ldsm_x4(tb + GE::off(lslot, 2 * ks + lhalf), kb);
+        const uint32_t qf[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+        mma_bf16_16816(sacc[0], qf, kb[0], kb[1]);
+        mma_bf16_16816(sacc[1], qf, kb[2], kb[3]);
+      }
+      float sv[4] = {sacc[0][0], sacc[0][1], sacc[1][0], sacc[1][1]};
+
+      // Slot validity: a tile of occupied slots without the evicted one (the
+      // common case) needs no per-slot test.  Rows of slots that hold no
+      // token may hold anything: their V rows are zeroed so that a weight of
+      // 0 cannot meet a non-finite value in the P V product (K rows need
+      // nothing: their scores are replaced).
+      if (!(vg.full && s0 + TS <= vg.nse && (evict < s0 || evict >= s0 + TS))) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int slot = s0 + 8 * (r >> 1) + 2 * tig + (r & 1);
+          if (slot == evict || !vg.slot_ok(slot)) sv[r] = kNegInf;
+        }
+        const int zslot = s0 + (lane & 15);
+        if (!vg.slot_ok(zslot)) {
+#pragma unroll
+          for (int cc = 0; cc < GE::NCHK / 2; ++cc)
+            *reinterpret_cast<uint4*>(tile + GE::off(lane & 15, GE::NCHK + (lane >> 4) * (GE::NCHK / 2) + cc)) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+      }
+      if (!hreal) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sv[r] = kNegInf;
+      }
+      // ---- online softmax of head gid (exp2 domain, lazy rescale) ----
+      float tmax = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+      const float tm = tmax * qscale;
+      if (__any_sync(0xffffffffu, tm > m_run + kLazy)) {
+        float alpha = 1.f;
+        if (tm > m_run + kLazy) {
+          alpha = (m_run == kNegInf) ? 0.f : fast_exp2(m_run - tm);
+          m_run = tm;
+          l_run *= alpha;
+        }
+        // this lane's O^T columns are heads 2 tig and 2 tig + 1 (quads 2 tig, 2 tig + 1)
+        const float aa = __shfl_sync(0xffffffffu, alpha, 8 * tig);
+        const float ab = __shfl_sync(0xffffffffu, alpha, 8 * tig + 4);
+#pragma unroll
+        for (int mb = 0; mb < KS; ++mb) {
+          o[mb][0] *= aa; o[mb][1] *= ab; o[mb][2] *= aa; o[mb][3] *= ab;
+        }
+      }
+      const float nm = (m_run == kNegInf) ? 0.f : -m_run;   // masked scores give 2^-inf = 0
+      float pw[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) pw[r] = fast_exp2(fmaf(sv[r], qscale, nm));
+      l_run += (pw[0] + pw[1]) + (pw[2] + pw[3]);
+      const uint32_t pb0 = pack_bf16(pw[0], pw[1]);   // P^T rows (slots) 2 tig, 2 tig + 1 of column (head) gid
+      const uint32_t pb1 = pack_bf16(pw[2], pw[3]);   // slots 8 + 2 tig, 9 + 2 tig
+
+      // ---- O^T += V^T P^T ----
+#pragma unroll
+      for (int mb = 0; mb < KS; ++mb) {
+        uint32_t va[4];
+        ldsm_x4_t(tb + GE::off(lslot, GE::NCHK + 2 * mb + lhalf), va);
+        mma_bf16_16816(o[mb], va, pb0, pb1);
+      }
+      __syncwarp();
+      if (i + NSTG < cnt) {
+        fence_proxy_async_smem();
+        issue_next();
+      }
+      if (++cj == tpu) { cj = 0; ++cu; }
+      if (++cstage == NSTG) { cstage = 0; cphase ^= 1u; }
     }
-    if (++cj == tpu) { cj = 0; ++cu; }
-    if (++cstage == NSTG) { cstage = 0; cphase ^= 1u; }
-  }
-  if (failed) {
-    // let this warp's copies still in flight land (bounded) before it exits
-    int st2 = cstage;
-    uint32_t ph2 = cphase;
-    for (int k2 = failed_at + 1; k2 < cnt && k2 < failed_at + NSTG; ++k2) {
-      if (++st2 == NSTG) { st2 = 0; ph2 ^= 1u; }
-      mbar_wait(&fb[st2], ph2);
+    if (failed) {
+      // let this warp's copies still in flight land (bounded) before it exits
+      int st2 = cstage;
+      uint32_t ph2 = cphase;
+      for (int k2 = failed_at + 1; k2 < cnt && k2 < failed_at + NSTG; ++k2) {
+        if (++st2 == NSTG) { st2 = 0; ph2 ^= 1u; }
+        mbar_wait(&fb[st2], ph2);
+      }
+    } else if (cur >= 0) {
+      check_pending();
+      finalize(cur);
+      check_pending();
     }
-  } else if (cur >= 0) {
-    check_pending();
-    finalize(cur);
-    check_pending();
+  } else {
+    const int j = lane & 15;        // QK: slot of the tile
+    const int h = lane >> 4;        // QK: half of the dims
+    const int gq = lane / GE::LPS;  // PV: slot group
+    const int c = lane % GE::LPS;   // PV: chunk of the value row
+
+    float2 acc[G][GE::EPC / 2];
+    float m[G], lp[G];
+    int evict = -1;
+    int cur = -1;
+    int qbuf = 0;
+    uint32_t qphase = 0;   // bit b = parity of raw buffer b's next completion
+
+    // Start a unit segment: q into the fp32 layout, reset the softmax state,
+    // fold the new token in if this warp holds the unit's first tile, and
+    // prefetch the next unit's q.
+    auto start_unit = [&](int unit, bool first_tile) {
+      if (!mbar_wait(&qb[qbuf], (qphase >> qbuf) & 1u)) {
+        if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+      }
+      qphase ^= 1u << qbuf;
+      const uint8_t* raw = qraw + qbuf * SM::QRB;
+      __syncwarp();
+      float* qf = reinterpret_cast<float*>(qsm);
+      const T* qr = reinterpret_cast<const T*>(raw);
+      for (int idx = lane; idx < G * DH; idx += 32) {
+        const int g = idx / DH, dim = idx % DH;
+        const int ch = dim / GE::EPC, e = dim % GE::EPC;
+        const int hh = ch / GE::CH, cc = ch % GE::CH;
+        qf[hh * ((GE::QHALF + 16) / 4) + (cc * G + g) * GE::EPC + e] = Elem<T>::to_f32(qr[idx]) * qscale;
+      }
+      evict = step ? reinterpret_cast<const Decision*>(raw + G * DH * GE::ESZ + 2 * DH * GE::ESZ)->evict : -1;
+  #pragma unroll
+      for (int g = 0; g < G; ++g) {
+        m[g] = kNegInf;
+        lp[g] = 0.f;
+  #pragma unroll
+        for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = make_float2(0.f, 0.f);
+      }
+      if (step && first_tile) {
+        // the appended token: score q . k_new and take it as the first slot
+        constexpr int DPL = DH / 32;
+        const T* kn = reinterpret_cast<const T*>(raw + G * DH * GE::ESZ);
+        const T* vn = kn + DH;
+  #pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float part = 0.f;
+  #pragma unroll
+          for (int e = 0; e < DPL; ++e)
+            part = fmaf(Elem<T>::to_f32(qr[g * DH + lane * DPL + e]), Elem<T>::to_f32(kn[lane * DPL + e]), part);
+  #pragma unroll
+          for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+          m[g] = part * qscale;   // p = exp2(s - m) = 1
+        }
+        if (lane == 0) {
+  #pragma unroll
+          for (int g = 0; g < G; ++g) lp[g] = 1.f;
+        }
+        if (gq == 0) {
+          const uint4 vr = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vn) + c * 16);
+          float2 v2[GE::EPC / 2];
+          if constexpr (sizeof(T) == 2) {
+            v2[0] = bf2_to_f2(vr.x); v2[1] = bf2_to_f2(vr.y); v2[2] = bf2_to_f2(vr.z); v2[3] = bf2_to_f2(vr.w);
+          } else {
+            v2[0] = make_float2(__uint_as_float(vr.x), __uint_as_float(vr.y));
+            v2[1] = make_float2(__uint_as_float(vr.z), __uint_as_float(vr.w));
+          }
+  #pragma unroll
+          for (int g = 0; g < G; ++g)
+  #pragma unroll
+            for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = v2[e];
+        }
+      }
+      __syncwarp();
+      if (unit < last_unit) issue_q(unit + 1, qbuf ^ 1);
+      qbuf ^= 1;
+    };
+
+    auto finalize = [&](int unit) {
+      float l[G];
+  #pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float v = lp[g];
+  #pragma unroll
+        for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        l[g] = v;
+      }
+  #pragma unroll
+      for (int o = GE::LPS; o < 32; o <<= 1)
+  #pragma unroll
+        for (int g = 0; g < G; ++g)
+  #pragma unroll
+          for (int e = 0; e < GE::EPC / 2; ++e) {
+            acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, o);
+            acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, o);
+          }
+      const int64_t first = warp_of_tile(static_cast<int64_t>(unit) * tpu, total, nw);
+      const int seg = static_cast<int>(gw - first);
+      if (seg >= kMaxSeg) {  // cannot happen: the split bounds the segments per unit
+        if (lane == 0) set_error(a.err, DEVERR_BAD_INDEX);
+        return;
+      }
+      float* pa = sc.part_acc + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * DH);
+      float* pmv = sc.part_ml + (static_cast<int64_t>(unit) * kMaxSeg + seg) * (G * 2);
+      if (lane < GE::LPS) {
+  #pragma unroll
+        for (int g = 0; g < G; ++g)
+  #pragma unroll
+          for (int e = 0; e < GE::EPC / 2; ++e)
+            *reinterpret_cast<float2*>(pa + g * DH + c * GE::EPC + 2 * e) = acc[g][e];
+      }
+      if (lane == 0) {
+  #pragma unroll
+        for (int g = 0; g < G; ++g) { pmv[2 * g] = m[g]; pmv[2 * g + 1] = l[g]; }
+      }
+      pend_unit = unit;
+      pend_prev = arrive(unit);   // checked later, so the atomic's round trip overlaps streaming
+    };
+
+    // consume cursor
+    int cu = static_cast<int>(lo / tpu), cj = static_cast<int>(lo - static_cast<int64_t>(cu) * tpu);
+    // first unit's q before the tile burst (it would queue behind it otherwise)
+    issue_q(cu, 0);
+    {
+      const int npre = cnt < NSTG ? cnt : NSTG;
+      for (int i = 0; i < npre; ++i) issue_next();
+    }
+    int cstage = 0;
+    uint32_t cphase = 0;
+    bool failed = false;
+    int failed_at = -1;
+    for (int i = 0; i < cnt; ++i) {
+      const int s0 = cj * TS;
+      const int nsl = min(TS, vg.nse - s0);
+      if (cu != cur) {
+        if (cur >= 0) {
+          check_pending();
+          finalize(cur);
+        }
+        cur = cu;
+        start_unit(cu, cj == 0);
+      }
+      if (!mbar_wait(&fb[cstage], cphase)) {
+        if (lane == 0) set_error(a.err, DEVERR_TIMEOUT);
+        failed = true;
+        failed_at = i;
+        break;
+      }
+      const uint8_t* tile = ring + cstage * GE::STAGE;
+
+      // ---- QK: lane (j, h) = slot j, dims of half h, all G heads ----
+      float s[G];
+      {
+        float2 sa[G][2];
+  #pragma unroll
+        for (int g = 0; g < G; ++g) { sa[g][0] = make_float2(0.f, 0.f); sa[g][1] = make_float2(0.f, 0.f); }
+        const float* qh = reinterpret_cast<const float*>(qsm + h * (GE::QHALF + 16));
+  #pragma unroll
+        for (int cc = 0; cc < GE::CH; ++cc) {
+          const uint4 kr = *reinterpret_cast<const uint4*>(tile + GE::off(j, h * GE::CH + cc));
+          float2 k2[GE::EPC / 2];
+          if constexpr (sizeof(T) == 2) {
+            k2[0] = bf2_to_f2(kr.x); k2[1] = bf2_to_f2(kr.y); k2[2] = bf2_to_f2(kr.z); k2[3] = bf2_to_f2(kr.w);
+          } else {
+            k2[0] = make_float2(__uint_as_float(kr.x), __uint_as_float(kr.y));
+            k2[1] = make_float2(__uint_as_float(kr.z), __uint_as_float(kr.w));
+          }
+  #pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float4* qp = reinterpret_cast<const float4*>(qh + (cc * G + g) * GE::EPC);
+  #pragma unroll
+            for (int e4 = 0; e4 < GE::EPC / 4; ++e4) {
+              const float4 qv = qp[e4];
+              sa[g][e4 & 1] = ffma2(make_float2(qv.x, qv.y), k2[2 * e4], sa[g][e4 & 1]);
+              sa[g][e4 & 1] = ffma2(make_float2(qv.z, qv.w), k2[2 * e4 + 1], sa[g][e4 & 1]);
+            }
+          }
+        }
+  #pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float v = (sa[g][0].x + sa[g][0].y) + (sa[g][1].x + sa[g][1].y);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          s[g] = v;
+        }
+      }
+      // Slot validity: a tile of occupied slots without the evicted one (the
+      // common case) needs no per-slot test.
+      bool valid = true;
+      uint32_t vmask = 0xffffu;
+      if (!(vg.full && s0 + TS <= vg.nse && (evict < s0 || evict >= s0 + TS))) {
+        const int slot = s0 + j;
+        valid = (j < nsl) && (slot != evict) && vg.slot_ok(slot);
+        vmask = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+      }
+      // ---- online softmax (exp2 domain, lazy rescale) ----
+      float sv[G];
+      bool in_range = true;
+  #pragma unroll
+      for (int g = 0; g < G; ++g) {
+        sv[g] = valid ? s[g] : kNegInf;
+        in_range = in_range && (sv[g] <= m[g] + kLazy);
+      }
+      // The running max moves only when a tile exceeds it by 2^kLazy; one vote
+      // tells whether any score of the tile does, else no tile max is needed.
+      if (!__all_sync(0xffffffffu, in_range)) {
+  #pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float mt = sv[g];
+  #pragma unroll
+          for (int o = 1; o < 16; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+          if (mt > m[g] + kLazy) {   // warp-uniform
+            const float alpha = (m[g] == kNegInf) ? 0.f : fast_exp2(m[g] - mt);
+            m[g] = mt;
+            lp[g] *= alpha;
+  #pragma unroll
+            for (int e = 0; e < GE::EPC / 2; ++e) {
+              acc[g][e].x *= alpha;
+              acc[g][e].y *= alpha;
+            }
+          }
+        }
+      }
+      float p[G];
+  #pragma unroll
+      for (int g = 0; g < G; ++g) {
+        p[g] = valid ? fast_exp2(sv[g] - m[g]) : 0.f;
+        lp[g] += p[g];
+      }
+      if (h == 0) {
+        float* pd = reinterpret_cast<float*>(psm + j * GE::PSLOT + (j / GE::SPG) * 16);
+  #pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          if (g + 1 < G)
+            *reinterpret_cast<float4*>(pd + 2 * g) = make_float4(p[g], p[g], p[g + 1], p[g + 1]);
+          else
+            *reinterpret_cast<float2*>(pd + 2 * g) = make_float2(p[g], p[g]);
+        }
+      }
+      __syncwarp();
+      // ---- PV: lane (gq, c) = slots of group gq, value chunk c ----
+      auto pv_slot = [&](int j2) {
+        const float* pp = reinterpret_cast<const float*>(psm + j2 * GE::PSLOT + (j2 / GE::SPG) * 16);
+        float2 pr[G];
+  #pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          if (g + 1 < G) {
+            const float4 t4 = *reinterpret_cast<const float4*>(pp + 2 * g);
+            pr[g] = make_float2(t4.x, t4.y);
+            pr[g + 1] = make_float2(t4.z, t4.w);
+          } else {
+            pr[g] = *reinterpret_cast<const float2*>(pp + 2 * g);
+          }
+        }
+        const uint4 vr = *reinterpret_cast<const uint4*>(tile + GE::off(j2, GE::NCHK + c));
+        float2 v2[GE::EPC / 2];
+        if constexpr (sizeof(T) == 2) {
+          v2[0] = bf2_to_f2(vr.x); v2[1] = bf2_to_f2(vr.y); v2[2] = bf2_to_f2(vr.z); v2[3] = bf2_to_f2(vr.w);
+        } else {
+          v2[0] = make_float2(__uint_as_float(vr.x), __uint_as_float(vr.y));
+          v2[1] = make_float2(__uint_as_float(vr.z), __uint_as_float(vr.w));
+        }
+  #pragma unroll
+        for (int g = 0; g < G; ++g)
+  #pragma unroll
+          for (int e = 0; e < GE::EPC / 2; ++e) acc[g][e] = ffma2(pr[g], v2[e], acc[g][e]);
+      };
+      if (vmask == 0xffffu) {
+  #pragma unroll
+        for (int jj = 0; jj < GE::SPG; ++jj) pv_slot(gq * GE::SPG + jj);
+      } else {
+  #pragma unroll
+        for (int jj = 0; jj < GE::SPG; ++jj) {
+          const int j2 = gq * GE::SPG + jj;
+          if ((vmask >> j2) & 1u) pv_slot(j2);
+        }
+      }
+      __syncwarp();
+      if (i + NSTG < cnt) {
+        fence_proxy_async_smem();
+        issue_next();
+      }
+      if (++cj == tpu) { cj = 0; ++cu; }
+      if (++cstage == NSTG) { cstage = 0; cphase ^= 1u; }
+    }
+    if (failed) {
+      // let this warp's copies still in flight land (bounded) before it exits
+      int st2 = cstage;
+      uint32_t ph2 = cphase;
+      for (int k2 = failed_at + 1; k2 < cnt && k2 < failed_at + NSTG; ++k2) {
+        if (++st2 == NSTG) { st2 = 0; ph2 ^= 1u; }
+        mbar_wait(&fb[st2], ph2);
+      }
+    } else if (cur >= 0) {
+      check_pending();
+      finalize(cur);
+      check_pending();
+    }
   }
   consumer_done();
   help();
@@ -1155,9 +1380,10 @@ __global__ void __launch_bounds__(128) decide_kernel(const LayerArgs a, int N, i
   }
 }
 
-template <typename T, int DH, int G, int NCW, int NSTG>
+template <typename T, int DH, int G>
 int launch_t(const CUtensorMap& tmap, const LayerArgs& a, const DecodeScratch& sc, int mode, const void* q,
              const void* kn, const void* vn, const float* ext, void* out, int num_sms, cudaStream_t st) {
+  constexpr int NCW = LaunchShape<T, G>::NCW, NSTG = LaunchShape<T, G>::NSTG, NDW = LaunchShape<T, G>::NDW;
   using SM = Smem<T, DH, G, NCW, NSTG>;
   // The shared-memory attribute belongs to the current device: set it once per
   // device (devices beyond the table get it on every call).
@@ -1166,7 +1392,7 @@ int launch_t(const CUtensorMap& tmap, const LayerArgs& a, const DecodeScratch& s
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
   if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_kernel<T, DH, G, NCW, NSTG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(decode_kernel<T, DH, G, NCW, NSTG, NDW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SM::TOTAL) != cudaSuccess)
       return -1;
     if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
@@ -1186,7 +1412,7 @@ int launch_t(const CUtensorMap& tmap, const LayerArgs& a, const DecodeScratch& s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<T, DH, G, NCW, NSTG>, tmap, a, sc, mode,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<T, DH, G, NCW, NSTG, NDW>, tmap, a, sc, mode,
                                            static_cast<const T*>(q), static_cast<const T*>(kn),
                                            static_cast<const T*>(vn), ext, static_cast<T*>(out));
   return e == cudaSuccess ? 0 : -1;
@@ -1229,8 +1455,7 @@ int launch_decode(const CUtensorMap& tmap, const LayerArgs& a, int dtype, const 
                   cudaStream_t st) {
 #define KVPOP_DISPATCH(TT, DD, GG) \
   if (a.d == DD && a.G == GG)      \
-    return launch_t<TT, DD, GG, (GG > 4 ? 8 : KVPOP_NCW), (GG > 4 ? 2 : KVPOP_NSTG)>(tmap, a, sc, mode, q, k_new,  \
-                                                                             v_new, ext_score, out, num_sms, st);
+    return launch_t<TT, DD, GG>(tmap, a, sc, mode, q, k_new, v_new, ext_score, out, num_sms, st);
   if (dtype == 1) {
     KVPOP_DISPATCH(__nv_bfloat16, 128, 4)
     KVPOP_DISPATCH(__nv_bfloat16, 128, 2)

@@ -153,13 +153,18 @@ template <> struct PaIo<float> {
 // Every key a query of the tile may attend to is among them.  Block-wide
 // (all NT threads); returns the count (at most cap).  Each thread scans 8
 // consecutive positions per round (8 cutoff loads in flight), and one block
-// scan per NT * 8 positions places the kept ones.
+// scan per NT * 8 positions places the kept ones.  With cand_cut, each
+// candidate's cutoff is stored beside it (0 for the sinks, which need none).
 template <int NT>
-__device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1, int cap) {
+__device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1, int cap,
+                                 int* cand_cut = nullptr) {
   constexpr int R = 8;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ns = min(S, q1);
-  for (int i = tid; i < ns; i += NT) cand[i] = i;
+  for (int i = tid; i < ns; i += NT) {
+    cand[i] = i;
+    if (cand_cut != nullptr) cand_cut[i] = 0;
+  }
   int count = ns;
   for (int base = S; base <= m0; base += NT * R) {
     const int j0 = base + tid * R;
@@ -189,7 +194,10 @@ __device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S,
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       if ((mine >> r) & 1u) {
-        if (off < cap) cand[off] = j0 + r;
+        if (off < cap) {
+          cand[off] = j0 + r;
+          if (cand_cut != nullptr) cand_cut[off] = c[r];
+        }
         ++off;
       }
     }
@@ -199,7 +207,10 @@ __device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S,
   const int r0 = max(S, m0 + 1);
   const int nr = max(0, q1 - r0);
   for (int i = tid; i < nr; i += NT)
-    if (count + i < cap) cand[count + i] = r0 + i;
+    if (count + i < cap) {
+      cand[count + i] = r0 + i;
+      if (cand_cut != nullptr) cand_cut[count + i] = cu[r0 + i];
+    }
   count += nr;
   __syncthreads();
   return min(count, cap);   // count <= cap always: S + K + qt + W + D bounds it
@@ -436,30 +447,12 @@ struct MmaSmem {
   static size_t bytes(int cand_cap) { return CAND_OFF + sizeof(int) * static_cast<size_t>(cand_cap); }
 };
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-               "{%8, %9}, {%0, %1, %2, %3};"
-               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
 
 template <int DH>
 __global__ void __launch_bounds__(kMmaThreads, 2) sparse_attn_mma_kernel(PaArgs p) {
@@ -1070,7 +1063,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 constexpr int kT2Rows = 256;
 constexpr int kT2Keys = 32;
-constexpr int kT2Stages = 4;
+constexpr int kT2Stages = 5;
 constexpr int kT2Lag = kT2Stages - 2;   // tiles a producer keeps in flight beyond the one it publishes
 constexpr int kT2Threads = 13 * 32;
 constexpr int kT2Prod = 8;          // first producer warp
@@ -1092,11 +1085,11 @@ struct T2Smem {
   static constexpr int NBAR = 2 * kT2Stages + 16;
   static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
   static constexpr size_t WT_OFF = TADDR_OFF + 16;
-  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);
+  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);     // [cand_cap] positions, then [cand_cap] cutoffs
   static_assert(BAR_OFF % 8 == 0 && KV_OFF % 16 == 0 && P_OFF % 16 == 0, "shared-memory alignment");
   // at least 116 KB: one CTA per SM, which then holds all 512 TMEM columns
   static size_t bytes(int cand_cap) {
-    const size_t bb = CAND_OFF + sizeof(int) * static_cast<size_t>(cand_cap);
+    const size_t bb = CAND_OFF + 2 * sizeof(int) * static_cast<size_t>(cand_cap);
     return bb > 116 * 1024 ? bb : 116 * 1024;
   }
 };
@@ -1123,6 +1116,7 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SM::TADDR_OFF + 4);
   int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
   int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
+  int* cand_cut = cand + p.cand_cap;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int u = blockIdx.y;
@@ -1134,6 +1128,19 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
   const __nv_bfloat16* kgp = static_cast<const __nv_bfloat16*>(p.k) + static_cast<size_t>(u) * n * DH;
   const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
   const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
+
+  // query rows of both blocks (row = position offset * G + head) by cp.async,
+  // zero past the prompt; they land while the candidates are gathered
+  for (int c = tid; c < kT2Rows * QCH; c += kT2Threads) {
+    const int row = c / QCH, ch = c % QCH;
+    const int qpos = q0 + row / G, g = row % G;
+    const bool in = qpos < q1;
+    const __nv_bfloat16* src = qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (in ? qpos : 0)) * DH + ch * 8;
+    cp_async16(sbase + static_cast<uint32_t>(SM::Q_OFF + (row >> 7) * SM::QBLK +
+                                             (static_cast<size_t>(ch) * 128 + (row & 127)) * 16),
+               src, in ? 16 : 0);
+  }
+  cp_async_commit();
 
   if (warp == kT2Mma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -1154,18 +1161,9 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
     *abort_flag = 0;
     mbar_fence_init();
   }
-  // query rows of both blocks (row = position offset * G + head), zero past the prompt
-  for (int c = tid; c < kT2Rows * QCH; c += kT2Threads) {
-    const int row = c / QCH, ch = c % QCH;
-    const int qpos = q0 + row / G, g = row % G;
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (qpos < q1)
-      x = *reinterpret_cast<const uint4*>(qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos) * DH + ch * 8);
-    *reinterpret_cast<uint4*>(smem_raw + SM::Q_OFF + (row >> 7) * SM::QBLK +
-                              (static_cast<size_t>(ch) * 128 + (row & 127)) * 16) = x;
-  }
+  const int count = gather_candidates<kT2Threads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap, cand_cut);
+  cp_async_wait<0>();
   fence_proxy_async_smem();
-  const int count = gather_candidates<kT2Threads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1204,7 +1202,7 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         int* m = meta + st * SM::META_INTS;
         const int idx = t * kT2Keys + ptid;
         const int j = idx < count ? cand[idx] : -1;
-        const int c = j >= 0 ? cu[j] : 0;
+        const int c = j >= 0 ? cand_cut[idx] : 0;
         m[ptid] = j;
         m[kT2Keys + ptid] = c;
         const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
