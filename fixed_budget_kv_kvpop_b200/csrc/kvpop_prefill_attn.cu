@@ -1079,8 +1079,8 @@ struct T2Smem {
   static constexpr size_t KV_OFF = Q_OFF + 2 * QBLK;                             // [stage][K, V]
   static constexpr size_t PBLK = static_cast<size_t>(kT2Keys / 8) * 128 * 16;
   static constexpr size_t P_OFF = KV_OFF + 2 * kT2Stages * KV_TILE;             // [block][buf]
-  static constexpr size_t META_OFF = P_OFF + 4 * PBLK;                           // [stage]{pos[keys], cut[keys], full}
-  static constexpr int META_INTS = 2 * kT2Keys + 4;
+  static constexpr size_t META_OFF = P_OFF + 4 * PBLK;                           // [stage][query position] key masks
+  static constexpr int META_INTS = kT2Rows;                                      // positions per CTA: 256 / G at most
   static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * kT2Stages * META_INTS;
   static constexpr int NBAR = 2 * kT2Stages + 16;
   static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
@@ -1182,7 +1182,6 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
   if (warp >= kT2Prod && warp < kT2Mma) {
     // ---------------- producers ----------------
     const int ptid = tid - kT2Prod * 32;
-    const int m1 = q1 - 1 - WD;
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % kT2Stages;
       if (t >= kT2Stages && !wait(&kv_free[st], ((t / kT2Stages) - 1) & 1)) break;
@@ -1198,16 +1197,21 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         cp_async16(vbase + so, vgp + off, j >= 0 ? 16 : 0);
       }
       cp_async_commit();
-      if (ptid < kT2Keys) {
-        int* m = meta + st * SM::META_INTS;
-        const int idx = t * kT2Keys + ptid;
+      {
+        // The tile's mask (§C.1) as one 32-bit word per query position of the
+        // CTA (bit i = key i visible): lane i of each producer warp holds key
+        // i, and one ballot per position collects the bits.  Key j (cutoff
+        // c) is visible at position q iff j <= q and (j is a sink or
+        // q - W - D < max(j, c)).
+        uint32_t* rm = reinterpret_cast<uint32_t*>(meta + st * SM::META_INTS);
+        const int idx = t * kT2Keys + lane;
         const int j = idx < count ? cand[idx] : -1;
-        const int c = j >= 0 ? cand_cut[idx] : 0;
-        m[ptid] = j;
-        m[kT2Keys + ptid] = c;
-        const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
-        const unsigned bal = __ballot_sync(0xffffffffu, full);
-        if (lane == 0) m[2 * kT2Keys] = (bal == 0xffffffffu);
+        const int mx = j >= 0 ? max(j, cand_cut[idx]) : 0;
+        for (int r = warp - kT2Prod; r < p.qt; r += kT2Mma - kT2Prod) {
+          const int qp = q0 + r;
+          const uint32_t bm = __ballot_sync(0xffffffffu, j >= 0 && j <= qp && (j < S || qp - WD < mx));
+          if (lane == 0) rm[r] = bm;
+        }
       }
       // Publish tile t - kT2Lag once it has landed.  The lag is at most
       // stages - 2: the MMA thread needs tile t + 1 (for S(t + 1)) before it
@@ -1272,9 +1276,9 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
     const int X = warp >> 2;
     const int row = tid & 127;
     const int grow = X * 128 + row;
-    const int qpos = q0 + grow / G;
+    const int posoff = grow / G;
+    const int qpos = q0 + posoff;
     const bool vrow = qpos < q1;
-    const int mrow = qpos - WD;
     const uint32_t lrow = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + 128u + static_cast<uint32_t>(X * DH);
     float m_run = -INFINITY, l_run = 0.f;
@@ -1294,20 +1298,15 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
       mbar_arrive(&s_free[2 * X + buf]);
       // mask on the raw logits; the tile max commutes with the positive scale,
       // so each weight is one FMA and one ex2: p = 2^(s * scale - m)
-      const int* m = meta + st * SM::META_INTS;
+      const uint32_t vm = vrow ? reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS)[posoff] : 0u;
       float tmax = -INFINITY;
-      if (m[2 * kT2Keys]) {
+      if (__all_sync(0xffffffffu, vm == 0xffffffffu)) {
 #pragma unroll
-        for (int i = 0; i < kT2Keys; ++i) {
-          if (!vrow) sv[i] = -INFINITY;
-          tmax = fmaxf(tmax, sv[i]);
-        }
+        for (int i = 0; i < kT2Keys; ++i) tmax = fmaxf(tmax, sv[i]);
       } else {
 #pragma unroll
         for (int i = 0; i < kT2Keys; ++i) {
-          const int j = m[i];
-          const bool vis = j >= 0 && vrow && j <= qpos && (j < S || j > mrow || m[kT2Keys + i] > mrow);
-          sv[i] = vis ? sv[i] : -INFINITY;
+          sv[i] = ((vm >> i) & 1u) ? sv[i] : -INFINITY;
           tmax = fmaxf(tmax, sv[i]);
         }
       }
