@@ -1420,18 +1420,26 @@ int launch_t(const CUtensorMap& tmap, const LayerArgs& a, const DecodeScratch& s
 
 }  // namespace
 
-int make_decode_tensor_map(CUtensorMap* map, void* layer_kv, int dtype, int d, int64_t rows, int row_bytes) {
-  // The driver entry point is fetched through the runtime, so the library
-  // needs no link-time dependency on libcuda.
+namespace {
+// The driver's tensor-map encoder, fetched through the runtime so that the
+// library needs no link-time dependency on libcuda; null if unavailable.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (encode == nullptr) {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult qres;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
         qres != cudaDriverEntryPointSuccess || fn == nullptr)
-      return -1;
+      return nullptr;
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
+  return encode;
+}
+}  // namespace
+
+int make_decode_tensor_map(CUtensorMap* map, void* layer_kv, int dtype, int d, int64_t rows, int row_bytes) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return -1;
   const int esz = dtype == 0 ? 4 : 2;
   const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(2 * d), static_cast<cuuint64_t>(rows)};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(row_bytes)};

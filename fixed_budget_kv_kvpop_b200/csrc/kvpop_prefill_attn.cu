@@ -1042,16 +1042,27 @@ int launch_attn_tc(const PaArgs& pa, int units, int n, cudaStream_t st) {
 // ---------------- bf16 attention on tcgen05, two row blocks per CTA ----------------
 // 256 query rows per CTA (two blocks of 128, one per group of four softmax
 // warps), warp-specialized and pipelined through mbarriers:
-//   producer warps 8-11 gather each tile's K and V rows (cp.async, kT2Stages
-//     stages) and publish them with the keys' positions and cutoffs;
-//   one thread of warp 12 issues the MMAs in the order S_0(t+1), O_0 += P_0 V(t),
-//     S_1(t+1), O_1 += P_1 V(t), so the tensor cores work on one block while
-//     the other block's softmax runs; each tile's K and V serve both blocks;
+//   copy warps 8-11 gather each tile's K and V rows by cp.async into the
+//     128-byte-swizzled operand layout (kT2Stages stages; each thread's
+//     copies arrive on the stage's mbarrier as they land, so nothing waits
+//     for its own copies); mask warps 12-13 build the tile's mask (one key
+//     bitmask per query position);
+//   one thread of warp 14 (block 0) and one of warp 15 (block 1) issue each
+//     block's MMAs in the order S(t+1), O += P V(t), so the tensor cores work
+//     on one block while the other block's softmax runs; each tile's K and V
+//     serve both blocks;
 //   softmax warps 0-3 (block 0) and 4-7 (block 1): thread = query row = TMEM
-//     lane; S double-buffered in TMEM, P double-buffered in shared memory, so
-//     a block's softmax of tile t + 1 need not wait for its P V of tile t
-//     (only a rescale of O, or reusing a P buffer, waits for an earlier P V).
-// TMEM: S[block][buf] at columns 32 * (2 block + buf), O[block] at 128 + block * DH.
+//     lane.
+// Q and P are the A operands and live in TMEM (rows = lanes, bf16 pairs per
+// 32-bit column), so the MMAs read only K and V from shared memory: with
+// 32-key tiles, re-reading a 128-row Q block from shared memory for every
+// tile would cost 4x the K bytes.  S is single-buffered per block (the
+// softmax reads it into registers and frees it at once); P is
+// double-buffered, so a block's softmax of tile t + 1 need not wait for its
+// P V of tile t (only a rescale of O, or reusing a P buffer, waits for an
+// earlier P V).
+// TMEM columns: O[block] at block * DH, Q[block] at 2 DH + block * DH / 2,
+// S[block] at 3 DH + 32 block, P[block][buf] at 3 DH + 64 + 16 (2 block + buf).
 // Every mbarrier that a role may wait on twice in a row without an
 // intervening handoff is per buffer, so parity waits never alias.
 // 2^x with the hardware's approximate base-2 exponential (ftz; 2^-inf = +0).
@@ -1060,33 +1071,67 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Shared-memory matrix descriptor, 128-byte swizzle (atoms of 8 rows x 128
+// bytes, 1024-byte aligned; start, leading and stride byte offsets in 16-byte
+// units; descriptor version 1, layout type 2).  K-major: stride offset =
+// 8-row group stride, leading offset unused (1), and the start moves by 32
+// bytes per 16 elements of K inside the atom.  MN-major: leading offset =
+// stride between 64-element groups of MN, stride offset = 8-row group stride
+// along K.
+__device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return tc_desc(saddr, lbo, sbo) | (2ull << 61);
+}
+// D (+)= A B with A in TMEM (row m = lane m, K pairs of bf16 per 32-bit
+// column) and B in shared memory (descriptor).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+      :: "r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tc_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};"
+      :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+         "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
 
 constexpr int kT2Rows = 256;
+// Lazy rescale threshold (log2 units): the running max of a row moves only
+// when a tile's max exceeds it by 2^20.  A rescale of O waits for the P V in
+// flight, so it must be rare; weights then stay below 2^20, far inside the
+// range of the fp32 accumulators (and of bf16 P, whose precision is
+// relative).
+constexpr float kT2Lazy = 20.0f;
 constexpr int kT2Keys = 32;
-constexpr int kT2Stages = 5;
-constexpr int kT2Lag = kT2Stages - 2;   // tiles a producer keeps in flight beyond the one it publishes
-constexpr int kT2Threads = 13 * 32;
-constexpr int kT2Prod = 8;          // first producer warp
-constexpr int kT2Mma = 12;          // MMA warp
+constexpr int kT2Stages = 10;
+constexpr int kT2Threads = 16 * 32;
+constexpr int kT2Prod = 8;          // first of the 4 copy warps
+constexpr int kT2Mask = 12;         // first of the 2 mask warps
+constexpr int kT2Mma = 14;          // MMA warps: one per row block
 constexpr uint32_t kT2Cols = 512;
 
+// A stage holds the tile's K then V, each as DH / 64 groups of 64 columns
+// (128 bytes per key row), each group 4 swizzle atoms of 8 keys x 128 bytes.
 template <int DH>
 struct T2Smem {
-  static constexpr int QCH = DH / 8;
-  static constexpr size_t QBLK = static_cast<size_t>(QCH) * 128 * 16;          // one block of Q rows
-  static constexpr size_t Q_OFF = 0;
-  static constexpr size_t KV_TILE = static_cast<size_t>(QCH) * kT2Keys * 16;
-  static constexpr size_t KV_OFF = Q_OFF + 2 * QBLK;                             // [stage][K, V]
-  static constexpr size_t PBLK = static_cast<size_t>(kT2Keys / 8) * 128 * 16;
-  static constexpr size_t P_OFF = KV_OFF + 2 * kT2Stages * KV_TILE;             // [block][buf]
-  static constexpr size_t META_OFF = P_OFF + 4 * PBLK;                           // [stage][query position] key masks
-  static constexpr int META_INTS = kT2Rows;                                      // positions per CTA: 256 / G at most
+  static constexpr int NGRP = DH / 64;                                           // 64-column groups per row
+  static constexpr size_t GRP = static_cast<size_t>(kT2Keys) * 128;              // one group of one tile: 4 KB
+  static constexpr size_t KV_TILE = NGRP * GRP;
+  static constexpr size_t STAGE = 2 * KV_TILE;
+  static constexpr size_t KV_OFF = 0;                                            // [stage][K, V]
+  static constexpr size_t META_OFF = KV_OFF + kT2Stages * STAGE;                // [stage][query position] key masks
+  static constexpr int META_INTS = kT2Rows + 4;                                  // 256 / G positions at most, then the full-tile flag
   static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * kT2Stages * META_INTS;
-  static constexpr int NBAR = 2 * kT2Stages + 16;
+  static constexpr int NBAR = 3 * kT2Stages + 13;
   static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
   static constexpr size_t WT_OFF = TADDR_OFF + 16;
   static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);     // [cand_cap] positions, then [cand_cap] cutoffs
-  static_assert(BAR_OFF % 8 == 0 && KV_OFF % 16 == 0 && P_OFF % 16 == 0, "shared-memory alignment");
+  static_assert(BAR_OFF % 8 == 0 && STAGE % 1024 == 0 && META_OFF % 16 == 0, "shared-memory alignment");
   // at least 116 KB: one CTA per SM, which then holds all 512 TMEM columns
   static size_t bytes(int cand_cap) {
     const size_t bb = CAND_OFF + 2 * sizeof(int) * static_cast<size_t>(cand_cap);
@@ -1095,23 +1140,27 @@ struct T2Smem {
 };
 
 template <int DH>
-__global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p) {
+__global__ void __launch_bounds__(kT2Threads, 1)
+sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   using SM = T2Smem<DH>;
-  constexpr int QCH = SM::QCH;
   constexpr uint32_t kIdescS = tc_idesc(128, kT2Keys, 0);
   constexpr uint32_t kIdescPV = tc_idesc(128, DH, 1);
-  constexpr uint32_t kRowCells = 128 * 16;
-  constexpr uint32_t kKeyCells = kT2Keys * 16;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
+  if ((sbase & 1023u) != 0u) {   // the swizzle atoms need 1024-byte alignment
+    if (threadIdx.x == 0) set_error(p.err, DEVERR_BAD_INDEX);
+    return;
+  }
   int* meta = reinterpret_cast<int*>(smem_raw + SM::META_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + SM::BAR_OFF);
-  uint64_t* kv_full = bars;                       // [stage], 128 producer arrivals
-  uint64_t* kv_free = bars + kT2Stages;           // [stage], MMA commit
-  uint64_t* s_full = bars + 2 * kT2Stages;        // [block][buf], MMA commit
-  uint64_t* s_free = s_full + 4;                  // [block][buf], 128 softmax arrivals
-  uint64_t* p_full = s_free + 4;                  // [block][buf], 128 softmax arrivals
+  uint64_t* kv_full = bars;                       // [stage], 128 producer arrivals as their copies land
+  uint64_t* kv_free = bars + kT2Stages;           // [stage], one MMA commit per row block
+  uint64_t* meta_full = bars + 2 * kT2Stages;     // [stage], the 4 producer warps (mask written)
+  uint64_t* s_full = bars + 3 * kT2Stages;        // [block], MMA commit
+  uint64_t* s_free = s_full + 2;                  // [block], 128 softmax arrivals
+  uint64_t* p_full = s_free + 2;                  // [block][buf], 128 softmax arrivals
   uint64_t* o_done = p_full + 4;                  // [block][buf], MMA commit (P V of that buffer)
+  uint64_t* q_full = o_done + 4;                  // 256 softmax arrivals: both Q blocks in TMEM
   uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_raw + SM::TADDR_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SM::TADDR_OFF + 4);
   int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
@@ -1129,18 +1178,21 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
   const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
   const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
 
-  // query rows of both blocks (row = position offset * G + head) by cp.async,
-  // zero past the prompt; they land while the candidates are gathered
-  for (int c = tid; c < kT2Rows * QCH; c += kT2Threads) {
-    const int row = c / QCH, ch = c % QCH;
-    const int qpos = q0 + row / G, g = row % G;
-    const bool in = qpos < q1;
-    const __nv_bfloat16* src = qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (in ? qpos : 0)) * DH + ch * 8;
-    cp_async16(sbase + static_cast<uint32_t>(SM::Q_OFF + (row >> 7) * SM::QBLK +
-                                             (static_cast<size_t>(ch) * 128 + (row & 127)) * 16),
-               src, in ? 16 : 0);
+  // softmax threads: their query row (row = position offset * G + head) into
+  // registers, zero past the prompt; the loads land while the candidates are
+  // gathered, and go to TMEM once its address is known
+  uint32_t qrow[DH / 2];
+  if (tid < kT2Rows) {
+    const int qp = q0 + tid / G, g = tid % G;
+    const bool in = qp < q1;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (in ? qp : 0)) * DH);
+#pragma unroll
+    for (int c = 0; c < DH / 8; ++c) {
+      const uint4 x = in ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      qrow[4 * c] = x.x; qrow[4 * c + 1] = x.y; qrow[4 * c + 2] = x.z; qrow[4 * c + 3] = x.w;
+    }
   }
-  cp_async_commit();
 
   if (warp == kT2Mma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -1150,25 +1202,41 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
   if (tid == 0) {
     for (int i = 0; i < kT2Stages; ++i) {
       mbar_init(&kv_full[i], 128);
-      mbar_init(&kv_free[i], 1);
+      mbar_init(&kv_free[i], 2);
+      mbar_init(&meta_full[i], kT2Mma - kT2Mask);
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&p_full[i], 128);
       mbar_init(&o_done[i], 1);
     }
+    mbar_init(q_full, kT2Rows);
     *abort_flag = 0;
     mbar_fence_init();
   }
   const int count = gather_candidates<kT2Threads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap, cand_cut);
-  cp_async_wait<0>();
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *taddr_s;
   const int ntiles = (count + kT2Keys - 1) / kT2Keys;
+  constexpr uint32_t kColQ = 2 * DH, kColS = 3 * DH, kColP = 3 * DH + 64;   // TMEM column bases (O at 0)
+  if (tid < kT2Rows) {
+    const uint32_t lq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kColQ + (tid >> 7) * (DH / 2);
+#pragma unroll
+    for (int c0 = 0; c0 < DH / 2; c0 += 16) {
+      uint32_t v16[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v16[i] = qrow[c0 + i];
+      tc_st16u(lq + c0, v16);
+    }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    tc_fence_before();
+    mbar_arrive(q_full);
+  }
 
   // bounded wait; on expiry every role stops at its next check
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -1179,94 +1247,116 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
     return false;
   };
 
-  if (warp >= kT2Prod && warp < kT2Mma) {
-    // ---------------- producers ----------------
-    const int ptid = tid - kT2Prod * 32;
+  if (warp >= kT2Prod && warp < kT2Mask) {
+    // ---------------- copy warps ----------------
+    // Their loop is bound by the load/store unit's rate for cp.async; the
+    // masks are built by other warps, so no shared-memory access of theirs
+    // queues behind these copies.
+    const int ptid = (warp - kT2Prod) * 32 + lane;
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % kT2Stages;
       if (t >= kT2Stages && !wait(&kv_free[st], ((t / kT2Stages) - 1) & 1)) break;
-      const uint32_t kbase = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
-      const uint32_t vbase = kbase + static_cast<uint32_t>(SM::KV_TILE);
-      for (int i = ptid; i < kT2Keys * QCH; i += 128) {
-        const int key = i / QCH, ch = i % QCH;
-        const int idx = t * kT2Keys + key;
-        const int j = idx < count ? cand[idx] : -1;
-        const size_t off = j >= 0 ? static_cast<size_t>(j) * DH + ch * 8 : 0;
-        const uint32_t so = static_cast<uint32_t>((ch * kT2Keys + key) * 16);
-        cp_async16(kbase + so, kgp + off, j >= 0 ? 16 : 0);
-        cp_async16(vbase + so, vgp + off, j >= 0 ? 16 : 0);
+      {
+        // The tile's K and V rows by cp.async into the swizzled layout: lane
+        // = 16-byte chunk of a 256-byte row (two rows per warp instruction),
+        // chunk c of key r at group c / 8, atom r / 8, row r % 8, position
+        // (c % 8) ^ (r % 8).  Past the candidates: zero-filled.  Each thread
+        // then arrives on kv_full[stage] when its copies have landed.
+        constexpr int CPR = DH / 8;                       // 16-byte chunks per row
+        const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE);
+#pragma unroll
+        for (int i = ptid; i < kT2Keys * CPR; i += 128) {
+          const int key = i / CPR, c = i % CPR;
+          const int kidx = t * kT2Keys + key;
+          const int jj = kidx < count ? cand[kidx] : -1;
+          const size_t off = jj >= 0 ? static_cast<size_t>(jj) * DH + c * 8 : 0;
+          const uint32_t so = static_cast<uint32_t>((c >> 3) * SM::GRP + (key >> 3) * 1024 + (key & 7) * 128 +
+                                                    (((c & 7) ^ (key & 7)) << 4));
+          cp_async16(kb + so, kgp + off, jj >= 0 ? 16 : 0);
+          cp_async16(kb + static_cast<uint32_t>(SM::KV_TILE) + so, vgp + off, jj >= 0 ? 16 : 0);
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(&kv_full[st])) : "memory");
       }
-      cp_async_commit();
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");   // nothing lands after the CTA's last barrier
+  } else if (warp >= kT2Mask && warp < kT2Mma) {
+    // ---------------- mask warps ----------------
+    const int mw = warp - kT2Mask;
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t % kT2Stages;
+      if (t >= kT2Stages && !wait(&kv_free[st], ((t / kT2Stages) - 1) & 1)) break;
+      const int idx = t * kT2Keys + lane;
+      const int j = idx < count ? cand[idx] : -1;
       {
         // The tile's mask (§C.1) as one 32-bit word per query position of the
-        // CTA (bit i = key i visible): lane i of each producer warp holds key
-        // i, and one ballot per position collects the bits.  Key j (cutoff
+        // CTA (bit i = key i visible): lane i of each mask warp holds key i,
+        // and one ballot per position collects the bits.  Key j (cutoff
         // c) is visible at position q iff j <= q and (j is a sink or
         // q - W - D < max(j, c)).
+        // A tile whose keys are all visible to every position of the CTA (the
+        // common case: long-range keys kept past the CTA's last position) is
+        // only flagged.
         uint32_t* rm = reinterpret_cast<uint32_t*>(meta + st * SM::META_INTS);
-        const int idx = t * kT2Keys + lane;
-        const int j = idx < count ? cand[idx] : -1;
         const int mx = j >= 0 ? max(j, cand_cut[idx]) : 0;
-        for (int r = warp - kT2Prod; r < p.qt; r += kT2Mma - kT2Prod) {
-          const int qp = q0 + r;
-          const uint32_t bm = __ballot_sync(0xffffffffu, j >= 0 && j <= qp && (j < S || qp - WD < mx));
-          if (lane == 0) rm[r] = bm;
+        const bool always = j >= 0 && j <= q0 && (j < S || q1 - 1 - WD < mx);
+        const bool full_tile = __ballot_sync(0xffffffffu, always) == 0xffffffffu;
+        if (mw == 0 && lane == 0) rm[kT2Rows] = full_tile ? 1u : 0u;
+        if (!full_tile) {
+          for (int r = mw; r < p.qt; r += kT2Mma - kT2Mask) {
+            const int qp = q0 + r;
+            const uint32_t bm = __ballot_sync(0xffffffffu, j >= 0 && j <= qp && (j < S || qp - WD < mx));
+            if (lane == 0) rm[r] = bm;
+          }
         }
-      }
-      // Publish tile t - kT2Lag once it has landed.  The lag is at most
-      // stages - 2: the MMA thread needs tile t + 1 (for S(t + 1)) before it
-      // issues P V(t), whose completion frees the stage that tile t + stages
-      // reuses, so tile t + 1 must be published before the producer waits for
-      // that stage.
-      if (t >= kT2Lag) {
-        cp_async_wait<kT2Lag>();
-        fence_proxy_async_smem();
-        mbar_arrive(&kv_full[(t - kT2Lag) % kT2Stages]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&meta_full[st]);
       }
     }
-    cp_async_wait<0>();
-    if (!*abort_flag) {
-      fence_proxy_async_smem();
-      for (int t = max(0, ntiles - kT2Lag); t < ntiles; ++t) mbar_arrive(&kv_full[t % kT2Stages]);
-    }
-  } else if (warp == kT2Mma) {
-    // ---------------- MMA issue (one thread) ----------------
+  } else if (warp >= kT2Mma) {
+    // ---------------- MMA issue: one thread per row block ----------------
+    // Each block's S(t + 1) is issued as soon as its softmax has read S(t),
+    // and its P V(t) as soon as P(t) is in TMEM, without waiting for the
+    // other block; a stage is free once both blocks' P V of it completed.
+    const int XB = warp - kT2Mma;
     if (lane == 0 && ntiles > 0) {
+      // S_X(t) = Q_X K(t)^T: A = Q_X in TMEM (8 columns per 16 dims), B = the K tile
       auto issue_s = [&](int X, int t) -> bool {
-        const int buf = t & 1, st = t % kT2Stages;
-        if (t >= 2 && !wait(&s_free[2 * X + buf], ((t - 2) >> 1) & 1)) return false;
+        const int st = t % kT2Stages;
+        if (t >= 1 && !wait(&s_free[X], (t - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t qb = sbase + static_cast<uint32_t>(SM::Q_OFF + X * SM::QBLK);
-        const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
-        const uint32_t d = tmem + 32u * (2 * X + buf);
+        const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE);
+        const uint32_t d = tmem + kColS + 32u * X;
+        const uint32_t aq = tmem + kColQ + static_cast<uint32_t>(X * (DH / 2));
+        // K-major B: 16 dims = 32 bytes of a 128-byte swizzled row; 8-key groups 1024 bytes apart
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks)
-          tc_mma(d, tc_desc(qb + ks * 2 * kRowCells, kRowCells, 128), tc_desc(kb + ks * 2 * kKeyCells, kKeyCells, 128),
-                 kIdescS, ks > 0 ? 1u : 0u);
-        tc_commit(&s_full[2 * X + buf]);
+          tc_mma_ts(d, aq + 8u * ks,
+                    tc_desc_sw128(kb + static_cast<uint32_t>((ks >> 2) * SM::GRP + (ks & 3) * 32), 16, 1024), kIdescS,
+                    ks > 0 ? 1u : 0u);
+        tc_commit(&s_full[X]);
         return true;
       };
+      // O_X += P_X(t) V(t): A = P_X(t) in TMEM (8 columns per 16 keys), B = the V tile
       auto issue_pv = [&](int X, int t) -> bool {
         const int st = t % kT2Stages, buf = t & 1;
         if (!wait(&p_full[2 * X + buf], (t >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t pb = sbase + static_cast<uint32_t>(SM::P_OFF + (2 * X + buf) * SM::PBLK);
-        const uint32_t vb = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st + 1) * SM::KV_TILE);
-        const uint32_t d = tmem + 128u + static_cast<uint32_t>(X * DH);
+        const uint32_t vb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE + SM::KV_TILE);
+        const uint32_t d = tmem + static_cast<uint32_t>(X * DH);
+        const uint32_t ap = tmem + kColP + 16u * (2 * X + buf);
+        // MN-major B: 64-dim groups GRP bytes apart (leading), 8-key groups 1024 bytes apart (stride);
+        // 16 keys per instruction = two 8-key groups
 #pragma unroll
         for (int kk = 0; kk < kT2Keys / 16; ++kk)
-          tc_mma(d, tc_desc(pb + kk * 2 * kRowCells, kRowCells, 128), tc_desc(vb + kk * 256, 128, kKeyCells),
-                 kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(d, ap + 8u * kk, tc_desc_sw128(vb + static_cast<uint32_t>(kk * 2048), SM::GRP, 1024), kIdescPV,
+                    (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&o_done[2 * X + buf]);
         return true;
       };
-      bool ok = wait(&kv_full[0], 0) && issue_s(0, 0) && issue_s(1, 0);
+      bool ok = wait(q_full, 0) && wait(&kv_full[0], 0) && issue_s(XB, 0);
       for (int t = 0; ok && t < ntiles; ++t) {
-        const bool next = t + 1 < ntiles;
-        if (next) ok = wait(&kv_full[(t + 1) % kT2Stages], ((t + 1) / kT2Stages) & 1) && issue_s(0, t + 1);
-        ok = ok && issue_pv(0, t);
-        if (next) ok = ok && issue_s(1, t + 1);
-        ok = ok && issue_pv(1, t);
+        if (t + 1 < ntiles) ok = wait(&kv_full[(t + 1) % kT2Stages], ((t + 1) / kT2Stages) & 1) && issue_s(XB, t + 1);
+        ok = ok && issue_pv(XB, t);
         if (ok) tc_commit(&kv_free[t % kT2Stages]);
       }
     }
@@ -1280,25 +1370,26 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
     const int qpos = q0 + posoff;
     const bool vrow = qpos < q1;
     const uint32_t lrow = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tO = tmem + 128u + static_cast<uint32_t>(X * DH);
+    const uint32_t tO = tmem + static_cast<uint32_t>(X * DH);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int t = 0; t < ntiles; ++t) {
-      const int buf = t & 1, st = t % kT2Stages;
-      bool got = wait(&kv_full[st], (t / kT2Stages) & 1);
-      got = got && wait(&s_full[2 * X + buf], (t >> 1) & 1);
+      const int st = t % kT2Stages;
+      bool got = wait(&meta_full[st], (t / kT2Stages) & 1);
+      got = got && wait(&s_full[X], t & 1);
       if (!__all_sync(0xffffffffu, got)) {   // the TMEM loads below are warp-collective
         ok = false;
         break;
       }
       tc_fence_after();
       float sv[32];
-      tc_ld32(tmem + 32u * (2 * X + buf) + lrow, sv);
+      tc_ld32(tmem + kColS + 32u * X + lrow, sv);
       tc_fence_before();
-      mbar_arrive(&s_free[2 * X + buf]);
+      mbar_arrive(&s_free[X]);
       // mask on the raw logits; the tile max commutes with the positive scale,
       // so each weight is one FMA and one ex2: p = 2^(s * scale - m)
-      const uint32_t vm = vrow ? reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS)[posoff] : 0u;
+      const uint32_t* rmk = reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS);
+      const uint32_t vm = !vrow ? 0u : (rmk[kT2Rows] ? 0xffffffffu : rmk[posoff]);
       float tmax = -INFINITY;
       if (__all_sync(0xffffffffu, vm == 0xffffffffu)) {
 #pragma unroll
@@ -1313,7 +1404,7 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
       const float tm = tmax * p.scale_log2;
       float alpha = 1.f;
       bool resc = false;
-      if (tm > m_run + kTcLazy) {
+      if (tm > m_run + kT2Lazy) {
         resc = (m_run != -INFINITY);
         alpha = resc ? ex2_approx(m_run - tm) : 0.f;
         l_run *= alpha;
@@ -1353,12 +1444,8 @@ __global__ void __launch_bounds__(kT2Threads, 1) sparse_attn_tc2_kernel(PaArgs p
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
-      uint8_t* pb = smem_raw + SM::P_OFF + (2 * X + (t & 1)) * SM::PBLK;
-#pragma unroll
-      for (int c = 0; c < kT2Keys / 8; ++c)
-        *reinterpret_cast<uint4*>(pb + (static_cast<size_t>(c) * 128 + row) * 16) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
+      tc_st16u(tmem + kColP + 16u * (2 * X + (t & 1)) + lrow, pk);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       mbar_arrive(&p_full[2 * X + (t & 1)]);
     }
@@ -1399,6 +1486,7 @@ template <int DH>
 int launch_attn_tc2(const PaArgs& pa, int units, int n, cudaStream_t st) {
   const size_t smem = T2Smem<DH>::bytes(pa.cand_cap);
   if (smem > 227 * 1024) return -2;
+  if (units == 0 || n == 0) return 0;
   if (cudaFuncSetAttribute(sparse_attn_tc2_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return -1;
