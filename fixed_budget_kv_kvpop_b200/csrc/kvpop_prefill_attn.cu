@@ -1391,15 +1391,16 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
       const uint32_t* rmk = reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS);
       const uint32_t vm = !vrow ? 0u : (rmk[kT2Rows] ? 0xffffffffu : rmk[posoff]);
       float tmax = -INFINITY;
-      if (__all_sync(0xffffffffu, vm == 0xffffffffu)) {
+      if (!__all_sync(0xffffffffu, vm == 0xffffffffu)) {
 #pragma unroll
-        for (int i = 0; i < kT2Keys; ++i) tmax = fmaxf(tmax, sv[i]);
-      } else {
+        for (int i = 0; i < kT2Keys; ++i) sv[i] = ((vm >> i) & 1u) ? sv[i] : -INFINITY;
+      }
+      {
+        // four independent max chains, then their max
+        float m4[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-        for (int i = 0; i < kT2Keys; ++i) {
-          sv[i] = ((vm >> i) & 1u) ? sv[i] : -INFINITY;
-          tmax = fmaxf(tmax, sv[i]);
-        }
+        for (int i = 4; i < kT2Keys; ++i) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
+        tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
       const float tm = tmax * p.scale_log2;
       float alpha = 1.f;
@@ -1411,16 +1412,17 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         m_run = tm;
       }
       const float nm = (m_run == -INFINITY) ? 0.f : -m_run;   // masked logits give 2^-inf = 0
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
       uint32_t pk[kT2Keys / 2];
 #pragma unroll
       for (int i = 0; i < kT2Keys; i += 2) {
-        const float p0 = ex2_approx(fmaf(sv[i], p.scale_log2, nm));
-        const float p1 = ex2_approx(fmaf(sv[i + 1], p.scale_log2, nm));
-        psum += p0 + p1;
+        const float x0 = fmaf(sv[i], p.scale_log2, nm), x1 = fmaf(sv[i + 1], p.scale_log2, nm);
+        const float p0 = ex2_approx(x0);
+        const float p1 = ex2_approx(x1);
+        ps[(i >> 1) & 3] += p0 + p1;
         pk[i / 2] = pack_bf16(p0, p1);
       }
-      l_run += psum;
+      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       // A rescale of O waits for every P V issued so far (the one of tile t - 1);
       // reusing P buffer t & 1 waits for the P V of tile t - 2.
       const bool any_resc = __any_sync(0xffffffffu, resc);
