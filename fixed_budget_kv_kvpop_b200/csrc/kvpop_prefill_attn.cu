@@ -1107,8 +1107,8 @@ constexpr int kT2Rows = 256;
 // range of the fp32 accumulators (and of bf16 P, whose precision is
 // relative).
 constexpr float kT2Lazy = 20.0f;
-constexpr int kT2Keys = 32;
-constexpr int kT2Stages = 10;
+constexpr int kT2Keys = 64;
+constexpr int kT2Stages = 5;
 constexpr int kT2Threads = 16 * 32;
 constexpr int kT2Prod = 8;          // first of the 4 copy warps
 constexpr int kT2Mask = 12;         // first of the 2 mask warps
@@ -1120,14 +1120,14 @@ constexpr uint32_t kT2Cols = 512;
 template <int DH>
 struct T2Smem {
   static constexpr int NGRP = DH / 64;                                           // 64-column groups per row
-  static constexpr size_t GRP = static_cast<size_t>(kT2Keys) * 128;              // one group of one tile: 4 KB
+  static constexpr size_t GRP = static_cast<size_t>(kT2Keys) * 128;              // one group of one tile: 8 KB
   static constexpr size_t KV_TILE = NGRP * GRP;
   static constexpr size_t STAGE = 2 * KV_TILE;
   static constexpr size_t KV_OFF = 0;                                            // [stage][K, V]
   static constexpr size_t META_OFF = KV_OFF + kT2Stages * STAGE;                // [stage][query position] key masks
-  static constexpr int META_INTS = kT2Rows + 4;                                  // 256 / G positions at most, then the full-tile flag
+  static constexpr int META_INTS = 2 * kT2Rows + 4;                              // 2 words per position (256 / G at most), then the full-tile flag
   static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * kT2Stages * META_INTS;
-  static constexpr int NBAR = 3 * kT2Stages + 13;
+  static constexpr int NBAR = 3 * kT2Stages + 7;
   static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
   static constexpr size_t WT_OFF = TADDR_OFF + 16;
   static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);     // [cand_cap] positions, then [cand_cap] cutoffs
@@ -1156,11 +1156,10 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   uint64_t* kv_full = bars;                       // [stage], 128 producer arrivals as their copies land
   uint64_t* kv_free = bars + kT2Stages;           // [stage], one MMA commit per row block
   uint64_t* meta_full = bars + 2 * kT2Stages;     // [stage], the 4 producer warps (mask written)
-  uint64_t* s_full = bars + 3 * kT2Stages;        // [block], MMA commit
-  uint64_t* s_free = s_full + 2;                  // [block], 128 softmax arrivals
-  uint64_t* p_full = s_free + 2;                  // [block][buf], 128 softmax arrivals
-  uint64_t* o_done = p_full + 4;                  // [block][buf], MMA commit (P V of that buffer)
-  uint64_t* q_full = o_done + 4;                  // 256 softmax arrivals: both Q blocks in TMEM
+  uint64_t* s_full = bars + 3 * kT2Stages;        // [block], MMA commit of S(t) (and of every P V before it)
+  uint64_t* p_full = s_full + 2;                  // [block], 128 softmax arrivals: P(t) in TMEM, S(t) read
+  uint64_t* o_done = p_full + 2;                  // [block], MMA commit after the block's last P V
+  uint64_t* q_full = o_done + 2;                  // 256 softmax arrivals: both Q blocks in TMEM
   uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_raw + SM::TADDR_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SM::TADDR_OFF + 4);
   int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
@@ -1207,9 +1206,6 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-    }
-    for (int i = 0; i < 4; ++i) {
       mbar_init(&p_full[i], 128);
       mbar_init(&o_done[i], 1);
     }
@@ -1223,7 +1219,7 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   tc_fence_after();
   const uint32_t tmem = *taddr_s;
   const int ntiles = (count + kT2Keys - 1) / kT2Keys;
-  constexpr uint32_t kColQ = 2 * DH, kColS = 3 * DH, kColP = 3 * DH + 64;   // TMEM column bases (O at 0)
+  constexpr uint32_t kColQ = 2 * DH, kColS = 3 * DH;   // TMEM column bases (O at 0; P(t) overwrites S(t))
   if (tid < kT2Rows) {
     const uint32_t lq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kColQ + (tid >> 7) * (DH / 2);
 #pragma unroll
@@ -1285,27 +1281,35 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % kT2Stages;
       if (t >= kT2Stages && !wait(&kv_free[st], ((t / kT2Stages) - 1) & 1)) break;
-      const int idx = t * kT2Keys + lane;
-      const int j = idx < count ? cand[idx] : -1;
       {
-        // The tile's mask (§C.1) as one 32-bit word per query position of the
-        // CTA (bit i = key i visible): lane i of each mask warp holds key i,
-        // and one ballot per position collects the bits.  Key j (cutoff
-        // c) is visible at position q iff j <= q and (j is a sink or
-        // q - W - D < max(j, c)).
-        // A tile whose keys are all visible to every position of the CTA (the
-        // common case: long-range keys kept past the CTA's last position) is
-        // only flagged.
+        // The tile's mask (§C.1) as two 32-bit words per query position of
+        // the CTA (bit i of word h = key 32 h + i visible): lane i of each
+        // mask warp holds keys i and 32 + i, and one ballot per word collects
+        // the bits.  Key j (cutoff c) is visible at position q iff j <= q and
+        // (j is a sink or q - W - D < max(j, c)).  A tile whose keys are all
+        // visible to every position of the CTA (the common case: long-range
+        // keys kept past the CTA's last position) is only flagged.
         uint32_t* rm = reinterpret_cast<uint32_t*>(meta + st * SM::META_INTS);
-        const int mx = j >= 0 ? max(j, cand_cut[idx]) : 0;
-        const bool always = j >= 0 && j <= q0 && (j < S || q1 - 1 - WD < mx);
-        const bool full_tile = __ballot_sync(0xffffffffu, always) == 0xffffffffu;
-        if (mw == 0 && lane == 0) rm[kT2Rows] = full_tile ? 1u : 0u;
+        int jh[2], mh[2];
+        bool always = true;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int idx = t * kT2Keys + 32 * h + lane;
+          jh[h] = idx < count ? cand[idx] : -1;
+          mh[h] = jh[h] >= 0 ? max(jh[h], cand_cut[idx]) : 0;
+          always = always && jh[h] >= 0 && jh[h] <= q0 && (jh[h] < S || q1 - 1 - WD < mh[h]);
+        }
+        const bool full_tile = __all_sync(0xffffffffu, always);
+        if (mw == 0 && lane == 0) rm[2 * kT2Rows] = full_tile ? 1u : 0u;
         if (!full_tile) {
           for (int r = mw; r < p.qt; r += kT2Mma - kT2Mask) {
             const int qp = q0 + r;
-            const uint32_t bm = __ballot_sync(0xffffffffu, j >= 0 && j <= qp && (j < S || qp - WD < mx));
-            if (lane == 0) rm[r] = bm;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t bm =
+                  __ballot_sync(0xffffffffu, jh[h] >= 0 && jh[h] <= qp && (jh[h] < S || qp - WD < mh[h]));
+              if (lane == 0) rm[2 * r + h] = bm;
+            }
           }
         }
         __syncwarp();
@@ -1314,18 +1318,19 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     }
   } else if (warp >= kT2Mma) {
     // ---------------- MMA issue: one thread per row block ----------------
-    // Each block's S(t + 1) is issued as soon as its softmax has read S(t),
-    // and its P V(t) as soon as P(t) is in TMEM, without waiting for the
-    // other block; a stage is free once both blocks' P V of it completed.
+    // Per block: S(0); then for each tile, once the softmax has read S(t) and
+    // written P(t) over it, O += P V(t) and S(t + 1).  The tensor cores run
+    // one thread's MMAs in issue order, so S(t + 1) overwrites those columns
+    // only after P V(t) has read them, and the commit after S(t + 1) also
+    // covers P V(t) (the softmax may then rescale O).  The blocks do not wait
+    // for each other; a stage is free once both blocks' P V of it completed.
     const int XB = warp - kT2Mma;
     if (lane == 0 && ntiles > 0) {
       // S_X(t) = Q_X K(t)^T: A = Q_X in TMEM (8 columns per 16 dims), B = the K tile
-      auto issue_s = [&](int X, int t) -> bool {
+      auto issue_s = [&](int X, int t) {
         const int st = t % kT2Stages;
-        if (t >= 1 && !wait(&s_free[X], (t - 1) & 1)) return false;
-        tc_fence_after();
         const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE);
-        const uint32_t d = tmem + kColS + 32u * X;
+        const uint32_t d = tmem + kColS + static_cast<uint32_t>(X * kT2Keys);
         const uint32_t aq = tmem + kColQ + static_cast<uint32_t>(X * (DH / 2));
         // K-major B: 16 dims = 32 bytes of a 128-byte swizzled row; 8-key groups 1024 bytes apart
 #pragma unroll
@@ -1334,30 +1339,37 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
                     tc_desc_sw128(kb + static_cast<uint32_t>((ks >> 2) * SM::GRP + (ks & 3) * 32), 16, 1024), kIdescS,
                     ks > 0 ? 1u : 0u);
         tc_commit(&s_full[X]);
-        return true;
       };
-      // O_X += P_X(t) V(t): A = P_X(t) in TMEM (8 columns per 16 keys), B = the V tile
-      auto issue_pv = [&](int X, int t) -> bool {
-        const int st = t % kT2Stages, buf = t & 1;
-        if (!wait(&p_full[2 * X + buf], (t >> 1) & 1)) return false;
-        tc_fence_after();
+      // O_X += P_X(t) V(t): A = P_X(t) in TMEM over S_X(t) (8 columns per 16 keys), B = the V tile
+      auto issue_pv = [&](int X, int t) {
+        const int st = t % kT2Stages;
         const uint32_t vb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE + SM::KV_TILE);
         const uint32_t d = tmem + static_cast<uint32_t>(X * DH);
-        const uint32_t ap = tmem + kColP + 16u * (2 * X + buf);
+        const uint32_t ap = tmem + kColS + static_cast<uint32_t>(X * kT2Keys);
         // MN-major B: 64-dim groups GRP bytes apart (leading), 8-key groups 1024 bytes apart (stride);
         // 16 keys per instruction = two 8-key groups
 #pragma unroll
         for (int kk = 0; kk < kT2Keys / 16; ++kk)
           tc_mma_ts(d, ap + 8u * kk, tc_desc_sw128(vb + static_cast<uint32_t>(kk * 2048), SM::GRP, 1024), kIdescPV,
                     (t > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&o_done[2 * X + buf]);
-        return true;
       };
-      bool ok = wait(q_full, 0) && wait(&kv_full[0], 0) && issue_s(XB, 0);
+      bool ok = wait(q_full, 0) && wait(&kv_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(XB, 0);
+      }
       for (int t = 0; ok && t < ntiles; ++t) {
-        if (t + 1 < ntiles) ok = wait(&kv_full[(t + 1) % kT2Stages], ((t + 1) / kT2Stages) & 1) && issue_s(XB, t + 1);
-        ok = ok && issue_pv(XB, t);
-        if (ok) tc_commit(&kv_free[t % kT2Stages]);
+        ok = wait(&p_full[XB], t & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(XB, t);
+        tc_commit(&kv_free[t % kT2Stages]);
+        if (t + 1 < ntiles) {
+          ok = wait(&kv_full[(t + 1) % kT2Stages], ((t + 1) / kT2Stages) & 1);
+          if (ok) issue_s(XB, t + 1);
+        } else {
+          tc_commit(&o_done[XB]);
+        }
       }
     }
     __syncwarp();
@@ -1382,18 +1394,32 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         break;
       }
       tc_fence_after();
-      float sv[32];
-      tc_ld32(tmem + kColS + 32u * X + lrow, sv);
-      tc_fence_before();
-      mbar_arrive(&s_free[X]);
+      // S(t) row: 64 fp32 columns (the commit after S(t) also covers every P V
+      // before it, so O may be rescaled below without another wait)
+      float sv[kT2Keys];
+      {
+        float lo[32], hi[32];
+        tc_ld32(tmem + kColS + static_cast<uint32_t>(X * kT2Keys) + lrow, lo);
+        tc_ld32(tmem + kColS + static_cast<uint32_t>(X * kT2Keys) + 32u + lrow, hi);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) { sv[i] = lo[i]; sv[32 + i] = hi[i]; }
+      }
       // mask on the raw logits; the tile max commutes with the positive scale,
       // so each weight is one FMA and one ex2: p = 2^(s * scale - m)
       const uint32_t* rmk = reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS);
-      const uint32_t vm = !vrow ? 0u : (rmk[kT2Rows] ? 0xffffffffu : rmk[posoff]);
+      uint32_t vm0 = 0u, vm1 = 0u;
+      if (vrow) {
+        const bool full = rmk[2 * kT2Rows] != 0u;
+        vm0 = full ? 0xffffffffu : rmk[2 * posoff];
+        vm1 = full ? 0xffffffffu : rmk[2 * posoff + 1];
+      }
       float tmax = -INFINITY;
-      if (!__all_sync(0xffffffffu, vm == 0xffffffffu)) {
+      if (!__all_sync(0xffffffffu, (vm0 & vm1) == 0xffffffffu)) {
 #pragma unroll
-        for (int i = 0; i < kT2Keys; ++i) sv[i] = ((vm >> i) & 1u) ? sv[i] : -INFINITY;
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = ((vm0 >> i) & 1u) ? sv[i] : -INFINITY;
+          sv[32 + i] = ((vm1 >> i) & 1u) ? sv[32 + i] : -INFINITY;
+        }
       }
       {
         // four independent max chains, then their max
@@ -1412,29 +1438,24 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         m_run = tm;
       }
       const float nm = (m_run == -INFINITY) ? 0.f : -m_run;   // masked logits give 2^-inf = 0
+      // P(t) in bf16 over the first 32 columns of S(t), 16 columns at a time
       float ps[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
-      uint32_t pk[kT2Keys / 2];
 #pragma unroll
-      for (int i = 0; i < kT2Keys; i += 2) {
-        const float x0 = fmaf(sv[i], p.scale_log2, nm), x1 = fmaf(sv[i + 1], p.scale_log2, nm);
-        const float p0 = ex2_approx(x0);
-        const float p1 = ex2_approx(x1);
-        ps[(i >> 1) & 3] += p0 + p1;
-        pk[i / 2] = pack_bf16(p0, p1);
+      for (int h = 0; h < kT2Keys / 32; ++h) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float x0 = fmaf(sv[32 * h + i], p.scale_log2, nm), x1 = fmaf(sv[32 * h + i + 1], p.scale_log2, nm);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          ps[(i >> 1) & 3] += p0 + p1;
+          pk[i / 2] = pack_bf16(p0, p1);
+        }
+        tc_st16u(tmem + kColS + static_cast<uint32_t>(X * kT2Keys + 16 * h) + lrow, pk);
       }
       l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      // A rescale of O waits for every P V issued so far (the one of tile t - 1);
-      // reusing P buffer t & 1 waits for the P V of tile t - 2.
-      const bool any_resc = __any_sync(0xffffffffu, resc);
-      bool freed = true;
-      if (any_resc && t >= 1) freed = wait(&o_done[2 * X + ((t - 1) & 1)], ((t - 1) >> 1) & 1);
-      else if (t >= 2) freed = wait(&o_done[2 * X + (t & 1)], ((t - 2) >> 1) & 1);
-      if (!__all_sync(0xffffffffu, freed)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (any_resc) {
+      if (__any_sync(0xffffffffu, resc)) {
+        // every P V before S(t) has completed (see above): rescale this row of O
         const float f = resc ? alpha : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < DH; c0 += 32) {
@@ -1444,15 +1465,13 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
           for (int i = 0; i < 32; ++i) o[i] *= f;
           tc_st32(tO + lrow + c0, o);
         }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
-      tc_st16u(tmem + kColP + 16u * (2 * X + (t & 1)) + lrow, pk);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(&p_full[2 * X + (t & 1)]);
+      mbar_arrive(&p_full[X]);
     }
     bool fin = ok && ntiles > 0;
-    if (fin) fin = wait(&o_done[2 * X + ((ntiles - 1) & 1)], ((ntiles - 1) >> 1) & 1);
+    if (fin) fin = wait(&o_done[X], 0);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const int g = grow % G;
