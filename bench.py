@@ -111,8 +111,8 @@ def step_bytes(w: wl.Workload) -> int:
 # of `bench.py --layers 2 --steps 2 --warmup 1` (the cr88 shape, 2 layers),
 # valid only for the kernel sources whose hash is recorded with it.
 TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024",
-                   "sources_sha256": "85a54fb15d497557650e5e985170016fa1eabd1f08cea0b8e3115cc976a3580b",
-                   "dram_bytes": 279_369_472 + 5_617_920, "algorithmic_bytes": 274_452_512}
+                   "sources_sha256": "e719b014f3cd4bd4534c1ceaa37d42b7bac5b13d3fdd0d4a3394611a2766e72f",
+                   "dram_bytes": 280_009_984 + 7_026_944, "algorithmic_bytes": 274_452_512}
 
 
 # ncu capture of the prefill attention's tensor-core kernel (the small case of
@@ -134,11 +134,11 @@ def _strip_code(src: str) -> str:
 
 def mma_kernel_sha256() -> str:
     """sha256 of the prefill attention's tensor-core kernel (its section of
-    kvpop_prefill_attn.cu, comments and blank lines removed)."""
+    kvpop_prefill_attn.cu with its launcher, comments and blank lines removed)."""
     import hashlib
     with open(os.path.join(ROOT, "fixed_budget_kv_kvpop_b200", "csrc", "kvpop_prefill_attn.cu")) as fh:
         src = fh.read()
-    a = src.index("bf16 attention on the tensor cores")
+    a = src.index("bf16 attention on tcgen05, two row blocks per CTA")
     b = src.index("int launch_attn_f32(")
     return hashlib.sha256(_strip_code(src[a:b]).encode()).hexdigest()
 

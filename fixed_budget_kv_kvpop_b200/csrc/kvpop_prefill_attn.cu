@@ -420,323 +420,10 @@ __global__ void __launch_bounds__(kPaThreads) sparse_attn_kernel(PaArgs p) {
   }
 }
 
-// ---------------- bf16 attention on the tensor cores (mma.sync) ----------------
-// One CTA of 8 warps per (unit, 128 / G query positions): each warp owns 16
-// query rows, the CTA streams its candidate keys in tiles of 32 through a
-// two-stage cp.async ring, S = Q K^T and O += P V run as m16n8k16 bf16 MMAs
-// with fp32 accumulators, and the mask and online softmax run on the S
-// fragments in registers.  Q fragments are re-read from shared memory for
-// every k-step and the key tile is 32 wide so that a thread needs at most 128
-// registers: two CTAs (16 warps) per SM hide each other's barrier and
-// latency stalls (measured 1.36x faster than 64-key tiles with Q held in
-// registers at one CTA per SM).
-constexpr int kMmaThreads = 256;
-constexpr int kMmaKeys = 32;
-constexpr int kMmaMetaWarps = kMmaKeys / 32;   // warps that publish a tile's key metadata
-
-template <int DH>
-struct MmaSmem {
-  static constexpr int RS = DH + 8;   // bf16 row stride: 16-byte pad keeps ldmatrix rows on distinct banks
-  static constexpr size_t Q_OFF = 0;
-  static constexpr size_t KV_OFF = Q_OFF + 2ull * kPaMmaRows * RS;
-  static constexpr size_t TILE = 2ull * kMmaKeys * RS;       // one K or V tile
-  static constexpr size_t POS_OFF = KV_OFF + 4 * TILE;       // stages x {K, V}
-  static constexpr size_t CUT_OFF = POS_OFF + sizeof(int) * 2 * kMmaKeys;
-  static constexpr size_t WT_OFF = CUT_OFF + sizeof(int) * 2 * kMmaKeys;
-  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);
-  static size_t bytes(int cand_cap) { return CAND_OFF + sizeof(int) * static_cast<size_t>(cand_cap); }
-};
-
+// ---------------- tcgen05 and copy helpers ----------------
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
-
-template <int DH>
-__global__ void __launch_bounds__(kMmaThreads, 2) sparse_attn_mma_kernel(PaArgs p) {
-  using SM = MmaSmem<DH>;
-  constexpr int KS = DH / 16;      // k-steps of Q K^T
-  constexpr int NT = kMmaKeys / 8; // key n-tiles of S
-  constexpr int DT = DH / 8;       // d n-tiles of O
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smem_raw + SM::Q_OFF);
-  int* kpos = reinterpret_cast<int*>(smem_raw + SM::POS_OFF);
-  int* kcut = reinterpret_cast<int*>(smem_raw + SM::CUT_OFF);
-  int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
-  int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g8 = lane >> 2, tig = lane & 3;
-  const int u = blockIdx.y;
-  const int b = u / p.Hkv, hk = u % p.Hkv;
-  const int n = p.n, S = p.S, WD = p.W + p.D, G = p.G;
-  const int q0 = blockIdx.x * p.qt;
-  const int q1 = min(n, q0 + p.qt);
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* kgp = static_cast<const __nv_bfloat16*>(p.k) + static_cast<size_t>(u) * n * DH;
-  const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
-  const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
-
-  // query rows (row = position offset * G + head), zero beyond the prompt
-  for (int c = tid; c < kPaMmaRows * (DH / 8); c += kMmaThreads) {
-    const int row = c / (DH / 8), ch = c % (DH / 8);
-    const int qpos = q0 + row / G, g = row % G;
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (qpos < q1) x = *reinterpret_cast<const uint4*>(qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos) * DH + ch * 8);
-    *reinterpret_cast<uint4*>(Qs + row * SM::RS + ch * 8) = x;
-  }
-  const int count = gather_candidates<kMmaThreads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
-  const int ntiles = (count + kMmaKeys - 1) / kMmaKeys;
-  const int m1 = q1 - 1 - WD;   // newest eligible position of the tile's last query
-  int* tile_full = wtot + 8;      // [stage][kMmaMetaWarps]: every key visible to every query of the tile
-
-  // Key metadata of tile t: the first kMmaKeys threads load (position,
-  // cutoff) early and publish them to shared memory after the current tile's
-  // math, so the cutoff loads' latency hides behind the MMAs.
-  auto load_meta = [&](int t, int& j, int& c) {
-    if (tid < kMmaKeys) {
-      const int idx = t * kMmaKeys + tid;
-      j = idx < count ? cand[idx] : -1;
-      c = j >= 0 ? cu[j] : 0;
-    }
-  };
-  auto store_meta = [&](int t, int j, int c) {
-    if (tid < kMmaKeys) {
-      const int st = t & 1;
-      kpos[st * kMmaKeys + tid] = j;
-      kcut[st * kMmaKeys + tid] = c;
-      const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
-      const unsigned bal = __ballot_sync(0xffffffffu, full);
-      if (lane == 0) tile_full[st * 2 + warp] = (bal == 0xffffffffu);
-    }
-  };
-  auto issue = [&](int t) {
-    const int st = t & 1;
-    const int t0 = t * kMmaKeys;
-    const uint32_t kbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st) * SM::TILE);
-    const uint32_t vbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st + 1) * SM::TILE);
-    for (int c = tid; c < kMmaKeys * (DH / 8); c += kMmaThreads) {
-      const int key = c / (DH / 8), ch = c % (DH / 8);
-      const int idx = t0 + key;
-      const int j = idx < count ? cand[idx] : -1;
-      const size_t off = j >= 0 ? static_cast<size_t>(j) * DH + ch * 8 : 0;
-      const uint32_t so = static_cast<uint32_t>((key * SM::RS + ch * 8) * 2);
-      cp_async16(kbase + so, kgp + off, j >= 0 ? 16 : 0);
-      cp_async16(vbase + so, vgp + off, j >= 0 ? 16 : 0);
-    }
-    cp_async_commit();
-  };
-  if (ntiles > 0) {
-    int j0 = -1, c0 = 0;
-    load_meta(0, j0, c0);
-    store_meta(0, j0, c0);
-    issue(0);
-  }
-
-  const int row_lo = warp * 16 + g8;
-  const int qlo = q0 + row_lo / G, qhi = q0 + (row_lo + 8) / G;
-  const int mlo = qlo - WD, mhi = qhi - WD;
-  const bool vlo = qlo < q1, vhi = qhi < q1;
-
-  float o[DT][4];
-#pragma unroll
-  for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-
-  for (int t = 0; t < ntiles; ++t) {
-    int jn = -1, cn = 0;
-    if (t + 1 < ntiles) {
-      load_meta(t + 1, jn, cn);
-      issue(t + 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int st = t & 1;
-    const uint32_t kbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st) * SM::TILE);
-    const uint32_t vbase = smem_u32(smem_raw + SM::KV_OFF + (2 * st + 1) * SM::TILE);
-
-    float sc[NT][4];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
-    {
-      const int mi = lane >> 3, ri = lane & 7;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        uint32_t qa[4];   // the warp's 16 query rows, k-step ks
-        {
-          const int row = warp * 16 + (mi & 1) * 8 + ri, col = ks * 16 + (mi >> 1) * 8;
-          ldsm_x4(smem_u32(Qs + row * SM::RS + col), qa);
-        }
-#pragma unroll
-        for (int jp = 0; jp < NT / 2; ++jp) {
-          uint32_t r[4];
-          const int key = jp * 16 + (mi >> 1) * 8 + ri, col = ks * 16 + (mi & 1) * 8;
-          ldsm_x4(kbase + static_cast<uint32_t>((key * SM::RS + col) * 2), r);
-          mma_bf16_16816(sc[2 * jp], qa, r[0], r[1]);
-          mma_bf16_16816(sc[2 * jp + 1], qa, r[2], r[3]);
-        }
-      }
-    }
-
-    // mask by the running top-k rule, base-2 logits, online softmax.  Most
-    // tiles hold only keys that every query of the CTA attends to.
-    float tmax_lo = -INFINITY, tmax_hi = -INFINITY;
-    bool all_full = true;
-#pragma unroll
-    for (int w = 0; w < kMmaMetaWarps; ++w) all_full = all_full && tile_full[st * 2 + w] != 0;
-    if (all_full) {
-#pragma unroll
-      for (int jn = 0; jn < NT; ++jn) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          sc[jn][e] = vlo ? sc[jn][e] * p.scale_log2 : -INFINITY;
-          sc[jn][2 + e] = vhi ? sc[jn][2 + e] * p.scale_log2 : -INFINITY;
-          tmax_lo = fmaxf(tmax_lo, sc[jn][e]);
-          tmax_hi = fmaxf(tmax_hi, sc[jn][2 + e]);
-        }
-      }
-    } else {
-      const int* kp = kpos + st * kMmaKeys;
-      const int* kc = kcut + st * kMmaKeys;
-#pragma unroll
-      for (int jn = 0; jn < NT; ++jn) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int key = jn * 8 + tig * 2 + e;
-          const int j = kp[key], c = kc[key];
-          const bool ok_lo = j >= 0 && vlo && j <= qlo && (j < S || j > mlo || c > mlo);
-          const bool ok_hi = j >= 0 && vhi && j <= qhi && (j < S || j > mhi || c > mhi);
-          sc[jn][e] = ok_lo ? sc[jn][e] * p.scale_log2 : -INFINITY;
-          sc[jn][2 + e] = ok_hi ? sc[jn][2 + e] * p.scale_log2 : -INFINITY;
-          tmax_lo = fmaxf(tmax_lo, sc[jn][e]);
-          tmax_hi = fmaxf(tmax_hi, sc[jn][2 + e]);
-        }
-      }
-    }
-    tmax_lo = fmaxf(tmax_lo, __shfl_xor_sync(0xffffffffu, tmax_lo, 1));
-    tmax_lo = fmaxf(tmax_lo, __shfl_xor_sync(0xffffffffu, tmax_lo, 2));
-    tmax_hi = fmaxf(tmax_hi, __shfl_xor_sync(0xffffffffu, tmax_hi, 1));
-    tmax_hi = fmaxf(tmax_hi, __shfl_xor_sync(0xffffffffu, tmax_hi, 2));
-    const float nm_lo = fmaxf(m_lo, tmax_lo), nm_hi = fmaxf(m_hi, tmax_hi);
-    const float a_lo = (nm_lo == -INFINITY) ? 1.f : exp2f(m_lo - nm_lo);
-    const float a_hi = (nm_hi == -INFINITY) ? 1.f : exp2f(m_hi - nm_hi);
-    float ps_lo = 0.f, ps_hi = 0.f;
-    uint32_t pa[NT / 2][4];
-#pragma unroll
-    for (int jn = 0; jn < NT; ++jn) {
-      const float p0 = sc[jn][0] == -INFINITY ? 0.f : exp2f(sc[jn][0] - nm_lo);
-      const float p1 = sc[jn][1] == -INFINITY ? 0.f : exp2f(sc[jn][1] - nm_lo);
-      const float p2 = sc[jn][2] == -INFINITY ? 0.f : exp2f(sc[jn][2] - nm_hi);
-      const float p3 = sc[jn][3] == -INFINITY ? 0.f : exp2f(sc[jn][3] - nm_hi);
-      ps_lo += p0 + p1;
-      ps_hi += p2 + p3;
-      pa[jn >> 1][(jn & 1) * 2 + 0] = pack_bf16(p0, p1);
-      pa[jn >> 1][(jn & 1) * 2 + 1] = pack_bf16(p2, p3);
-    }
-    ps_lo += __shfl_xor_sync(0xffffffffu, ps_lo, 1);
-    ps_lo += __shfl_xor_sync(0xffffffffu, ps_lo, 2);
-    ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 1);
-    ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 2);
-    l_lo = l_lo * a_lo + ps_lo;
-    l_hi = l_hi * a_hi + ps_hi;
-    m_lo = nm_lo;
-    m_hi = nm_hi;
-#pragma unroll
-    for (int i = 0; i < DT; ++i) {
-      o[i][0] *= a_lo;
-      o[i][1] *= a_lo;
-      o[i][2] *= a_hi;
-      o[i][3] *= a_hi;
-    }
-
-    // O += P V
-    {
-      const int mi = lane >> 3, ri = lane & 7;
-#pragma unroll
-      for (int kk = 0; kk < kMmaKeys / 16; ++kk) {
-#pragma unroll
-        for (int dp = 0; dp < DT / 2; ++dp) {
-          uint32_t r[4];
-          const int key = kk * 16 + (mi & 1) * 8 + ri, col = dp * 16 + (mi >> 1) * 8;
-          ldsm_x4_t(vbase + static_cast<uint32_t>((key * SM::RS + col) * 2), r);
-          mma_bf16_16816(o[2 * dp], pa[kk], r[0], r[1]);
-          mma_bf16_16816(o[2 * dp + 1], pa[kk], r[2], r[3]);
-        }
-      }
-    }
-    if (t + 1 < ntiles) store_meta(t + 1, jn, cn);   // stage (t+1)&1 was last read in tile t-1
-    __syncthreads();
-  }
-
-  __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out);
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int row = row_lo + 8 * h;
-    const int qpos = h ? qhi : qlo;
-    if (qpos >= q1) continue;
-    const int g = row % G;
-    const size_t rowi = (static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos;
-    const float inv = 1.f / (h ? l_hi : l_lo);
-#pragma unroll
-    for (int i = 0; i < DT; ++i)
-      *reinterpret_cast<uint32_t*>(og + rowi * DH + i * 8 + tig * 2) = pack_bf16(o[i][2 * h] * inv, o[i][2 * h + 1] * inv);
-    if (p.lse != nullptr && tig == 0)
-      p.lse[rowi] = ((h ? m_hi : m_lo) + log2f(h ? l_hi : l_lo)) * 0.69314718055994531f;
-  }
-}
-
-
-// ---------------- bf16 attention on the 5th-generation tensor cores ----------------
-// One CTA of 4 warps per (unit, 128 / G query positions): thread t owns query
-// row t, which is also TMEM lane t.  Per tile of kTcKeys candidate keys:
-//   1. all threads gather the tile's K and V rows with cp.async into shared
-//      memory (one tile ahead, two stages);
-//   2. one thread issues S = Q K^T as tcgen05.mma (bf16 operands from shared
-//      memory, fp32 accumulator in TMEM, M = 128, N = kTcKeys, K = 16 per
-//      instruction) and commits it to an mbarrier;
-//   3. every thread loads its row of S from TMEM (tcgen05.ld), applies the
-//      running top-k mask and an exp2-domain online softmax (the running max
-//      moves only when a tile exceeds it by 2^8; the O row in TMEM is then
-//      rescaled by tcgen05.ld / st), and writes its row of P (bf16) to shared
-//      memory;
-//   4. one thread issues O += P V (M = 128, N = d, K = 16 per instruction)
-//      into the TMEM accumulator.
-// Operands use the canonical no-swizzle layout: 16-byte cells stored
-// chunk-major ([16-byte chunk][row]), so every 8 x 16-byte core matrix is
-// 128 contiguous bytes.  K-major (Q, K, P): leading offset = the chunk stride,
-// stride offset = 128 bytes (8 rows).  V is the MN-major B operand of P V:
-// stride offset = the chunk stride (8 more dims), leading offset = 128 bytes
-// (8 more keys).  Two CTAs share an SM (shared memory and 2 x 256 TMEM
-// columns), so one CTA's softmax overlaps the other's MMAs.
-constexpr int kTcThreads = 128;
-constexpr int kTcKeys = 32;
-constexpr int kTcRows = 128;
-constexpr uint32_t kTcCols = 256;          // TMEM columns per CTA: S at 0, O at 128
-constexpr size_t kTcMinSmem = 80 * 1024;   // keeps at most two CTAs (2 x 256 TMEM columns) per SM
-constexpr float kTcLazy = 8.0f;            // lazy rescale threshold (log2 units)
-
-template <int DH>
-struct TcSmem {
-  static constexpr int QCH = DH / 8;                                   // 16-byte chunks per row
-  static constexpr size_t Q_OFF = 0;                                   // [QCH][kTcRows] cells
-  static constexpr size_t KV_TILE = static_cast<size_t>(QCH) * kTcKeys * 16;   // [QCH][kTcKeys] cells
-  static constexpr size_t KV_OFF = Q_OFF + static_cast<size_t>(QCH) * kTcRows * 16;   // [stage][K, V]
-  static constexpr size_t P_OFF = KV_OFF + 4 * KV_TILE;                // [kTcKeys / 8][kTcRows] cells
-  static constexpr size_t META_OFF = P_OFF + static_cast<size_t>(kTcKeys / 8) * kTcRows * 16;
-  static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * (4 * kTcKeys + 4);
-  static constexpr size_t TADDR_OFF = BAR_OFF + 16;
-  static constexpr size_t WT_OFF = TADDR_OFF + 16;
-  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);
-  static_assert(BAR_OFF % 8 == 0 && KV_OFF % 16 == 0 && P_OFF % 16 == 0, "shared-memory alignment");
-  static size_t bytes(int cand_cap) {
-    const size_t b = CAND_OFF + sizeof(int) * static_cast<size_t>(cand_cap);
-    return b > kTcMinSmem ? b : kTcMinSmem;
-  }
-};
 
 // Shared-memory matrix descriptor, no swizzle (start, leading and stride
 // byte offsets in 16-byte units; descriptor version 1).
@@ -749,13 +436,6 @@ __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t lbo, uint32
 __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -795,249 +475,6 @@ __device__ __forceinline__ void tc_st32(uint32_t taddr, const float (&v)[32]) {
          "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
-
-template <int DH>
-__global__ void __launch_bounds__(kTcThreads) sparse_attn_tc_kernel(PaArgs p) {
-  using SM = TcSmem<DH>;
-  constexpr int QCH = SM::QCH;
-  constexpr uint32_t kIdescS = tc_idesc(kTcRows, kTcKeys, 0);
-  constexpr uint32_t kIdescPV = tc_idesc(kTcRows, DH, 1);
-  constexpr uint32_t kRowCells = kTcRows * 16;   // bytes of one chunk column of Q or P
-  constexpr uint32_t kKeyCells = kTcKeys * 16;   // bytes of one chunk column of a K or V tile
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  const uint32_t sbase = smem_u32(smem_raw);
-  int* kpos = reinterpret_cast<int*>(smem_raw + SM::META_OFF);   // [2][kTcKeys]
-  int* kcut = kpos + 2 * kTcKeys;                                  // [2][kTcKeys]
-  int* tfull = kcut + 2 * kTcKeys;                                 // [2]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + SM::BAR_OFF);
-  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_raw + SM::TADDR_OFF);
-  int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
-  int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int u = blockIdx.y;
-  const int b = u / p.Hkv, hk = u % p.Hkv;
-  const int n = p.n, S = p.S, WD = p.W + p.D, G = p.G;
-  const int q0 = blockIdx.x * p.qt;
-  const int q1 = min(n, q0 + p.qt);
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* kgp = static_cast<const __nv_bfloat16*>(p.k) + static_cast<size_t>(u) * n * DH;
-  const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
-  const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
-
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 :: "r"(smem_u32(taddr_s)), "r"(kTcCols) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    mbar_fence_init();
-  }
-  // query rows (row = position offset * G + head), zero beyond the prompt
-  for (int c = tid; c < kTcRows * QCH; c += kTcThreads) {
-    const int row = c / QCH, ch = c % QCH;
-    const int qpos = q0 + row / G, g = row % G;
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (qpos < q1)
-      x = *reinterpret_cast<const uint4*>(qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + qpos) * DH + ch * 8);
-    *reinterpret_cast<uint4*>(smem_raw + SM::Q_OFF + (static_cast<size_t>(ch) * kTcRows + row) * 16) = x;
-  }
-  fence_proxy_async_smem();   // Q (generic-proxy stores) is read by the tensor cores
-  const int count = gather_candidates<kTcThreads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *taddr_s;
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lrow = static_cast<uint32_t>(warp * 32) << 16;   // this warp's TMEM lanes
-  const int ntiles = (count + kTcKeys - 1) / kTcKeys;
-  const int m1 = q1 - 1 - WD;
-
-  // gather tile t into stage t & 1: K and V rows (16-byte cells, zero past the
-  // candidates) and the keys' positions and cutoffs
-  auto issue = [&](int t) {
-    const int st = t & 1;
-    const uint32_t kbase = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
-    const uint32_t vbase = kbase + static_cast<uint32_t>(SM::KV_TILE);
-    for (int i = tid; i < kTcKeys * QCH; i += kTcThreads) {
-      const int key = i / QCH, ch = i % QCH;
-      const int idx = t * kTcKeys + key;
-      const int j = idx < count ? cand[idx] : -1;
-      const size_t off = j >= 0 ? static_cast<size_t>(j) * DH + ch * 8 : 0;
-      const uint32_t so = static_cast<uint32_t>((ch * kTcKeys + key) * 16);
-      cp_async16(kbase + so, kgp + off, j >= 0 ? 16 : 0);
-      cp_async16(vbase + so, vgp + off, j >= 0 ? 16 : 0);
-    }
-    cp_async_commit();
-    if (tid < kTcKeys) {
-      const int idx = t * kTcKeys + tid;
-      const int j = idx < count ? cand[idx] : -1;
-      const int c = j >= 0 ? cu[j] : 0;
-      kpos[st * kTcKeys + tid] = j;
-      kcut[st * kTcKeys + tid] = c;
-      const bool full = j >= 0 && j <= q0 && (j < S || j > m1 || c > m1);
-      const unsigned bal = __ballot_sync(0xffffffffu, full);
-      if (lane == 0) tfull[st] = (bal == 0xffffffffu);
-    }
-  };
-
-  const int row = tid;
-  const int qpos = q0 + row / G;
-  const bool vrow = qpos < q1;
-  const int mrow = qpos - WD;
-  float m_run = -INFINITY, l_run = 0.f;
-  uint32_t phase = 0;
-  bool failed = false;
-
-  if (ntiles > 0) issue(0);
-  for (int t = 0; t < ntiles; ++t) {
-    const int st = t & 1;
-    if (t + 1 < ntiles) {
-      issue(t + 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    fence_proxy_async_smem();   // this thread's cp.async rows -> the tensor cores' view
-    __syncthreads();
-    const uint32_t kt = sbase + static_cast<uint32_t>(SM::KV_OFF + (2 * st) * SM::KV_TILE);
-    const uint32_t vt = kt + static_cast<uint32_t>(SM::KV_TILE);
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < DH / 16; ++ks)
-        tc_mma(tS, tc_desc(sbase + static_cast<uint32_t>(SM::Q_OFF) + ks * 2 * kRowCells, kRowCells, 128),
-               tc_desc(kt + ks * 2 * kKeyCells, kKeyCells, 128), kIdescS, ks > 0 ? 1u : 0u);
-      tc_commit(bar);
-    }
-    bool ok = mbar_wait(bar, phase);
-    phase ^= 1u;
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
-    tc_fence_after();
-    float s[32];
-    tc_ld32(tS + lrow, s);
-
-    // running top-k mask, base-2 logits, online softmax with lazy rescaling
-    float tmax = -INFINITY;
-    if (tfull[st]) {
-#pragma unroll
-      for (int i = 0; i < kTcKeys; ++i) {
-        s[i] = vrow ? s[i] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, s[i]);
-      }
-    } else {
-      const int* kp = kpos + st * kTcKeys;
-      const int* kc = kcut + st * kTcKeys;
-#pragma unroll
-      for (int i = 0; i < kTcKeys; ++i) {
-        const int j = kp[i];
-        const bool vis = j >= 0 && vrow && j <= qpos && (j < S || j > mrow || kc[i] > mrow);
-        s[i] = vis ? s[i] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, s[i]);
-      }
-    }
-    float alpha = 1.f;
-    bool resc = false;
-    if (tmax > m_run + kTcLazy) {
-      resc = (m_run != -INFINITY);   // an O row that has seen no key is still zero
-      alpha = resc ? exp2f(m_run - tmax) : 0.f;
-      l_run *= alpha;
-      m_run = tmax;
-    }
-    float psum = 0.f;
-    uint32_t pk[kTcKeys / 2];
-#pragma unroll
-    for (int i = 0; i < kTcKeys; i += 2) {
-      const float p0 = s[i] == -INFINITY ? 0.f : exp2f(s[i] - m_run);
-      const float p1 = s[i + 1] == -INFINITY ? 0.f : exp2f(s[i + 1] - m_run);
-      psum += p0 + p1;
-      pk[i / 2] = pack_bf16(p0, p1);
-    }
-    l_run += psum;
-#pragma unroll
-    for (int c = 0; c < kTcKeys / 8; ++c)
-      *reinterpret_cast<uint4*>(smem_raw + SM::P_OFF + (static_cast<size_t>(c) * kTcRows + row) * 16) =
-          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-    if (__any_sync(0xffffffffu, resc)) {   // tcgen05.ld / st are warp-collective
-      const float f = resc ? alpha : 1.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float o[32];
-        tc_ld32(tO + lrow + c0, o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] *= f;
-        tc_st32(tO + lrow + c0, o);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    }
-    fence_proxy_async_smem();   // P (generic-proxy stores) is read by the tensor cores
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTcKeys / 16; ++kk)
-        tc_mma(tO, tc_desc(sbase + static_cast<uint32_t>(SM::P_OFF) + kk * 2 * kRowCells, kRowCells, 128),
-               tc_desc(vt + kk * 256, 128, kKeyCells), kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(bar);
-    }
-    ok = mbar_wait(bar, phase);
-    phase ^= 1u;
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
-    tc_fence_after();
-  }
-
-  if (failed) {
-    if (tid == 0) set_error(p.err, DEVERR_TIMEOUT);
-    cp_async_wait<0>();
-  } else if (ntiles > 0) {
-    // epilogue: O row / l, bf16, to the output; the row's log-normaliser.
-    // Every thread takes part in the (warp-collective) TMEM loads; rows past
-    // the prompt store nothing.
-    const int g = row % G;
-    const size_t rowi = (static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (vrow ? qpos : 0);
-    __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out) + rowi * DH;
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll 1
-    for (int c0 = 0; c0 < DH; c0 += 32) {
-      float o[32];
-      tc_ld32(tO + lrow + c0, o);
-      if (vrow) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(og + c0 + 8 * c) =
-              make_uint4(pack_bf16(o[8 * c] * inv, o[8 * c + 1] * inv), pack_bf16(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
-                         pack_bf16(o[8 * c + 4] * inv, o[8 * c + 5] * inv), pack_bf16(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
-      }
-    }
-    if (vrow && p.lse != nullptr) p.lse[rowi] = (m_run + log2f(l_run)) * 0.69314718055994531f;
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTcCols) : "memory");
-  }
-}
-
-template <int DH>
-int launch_attn_tc(const PaArgs& pa, int units, int n, cudaStream_t st) {
-  const size_t smem = TcSmem<DH>::bytes(pa.cand_cap);
-  if (cudaFuncSetAttribute(sparse_attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return -1;
-  dim3 grid((n + pa.qt - 1) / pa.qt, units);
-  sparse_attn_tc_kernel<DH><<<grid, kTcThreads, smem, st>>>(pa);
-  return 0;
-}
-
 
 // ---------------- bf16 attention on tcgen05, two row blocks per CTA ----------------
 // 256 query rows per CTA (two blocks of 128, one per group of four softmax
@@ -1145,14 +582,14 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   using SM = T2Smem<DH>;
   constexpr uint32_t kIdescS = tc_idesc(128, kT2Keys, 0);
   constexpr uint32_t kIdescPV = tc_idesc(128, DH, 1);
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const uint32_t sbase = smem_u32(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_t2[];
+  const uint32_t sbase = smem_u32(smem_t2);
   if ((sbase & 1023u) != 0u) {   // the swizzle atoms need 1024-byte alignment
     if (threadIdx.x == 0) set_error(p.err, DEVERR_BAD_INDEX);
     return;
   }
-  int* meta = reinterpret_cast<int*>(smem_raw + SM::META_OFF);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + SM::BAR_OFF);
+  int* meta = reinterpret_cast<int*>(smem_t2 + SM::META_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_t2 + SM::BAR_OFF);
   uint64_t* kv_full = bars;                       // [stage], 128 producer arrivals as their copies land
   uint64_t* kv_free = bars + kT2Stages;           // [stage], one MMA commit per row block
   uint64_t* meta_full = bars + 2 * kT2Stages;     // [stage], the 4 producer warps (mask written)
@@ -1160,10 +597,10 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   uint64_t* p_full = s_full + 2;                  // [block], 128 softmax arrivals: P(t) in TMEM, S(t) read
   uint64_t* o_done = p_full + 2;                  // [block], MMA commit after the block's last P V
   uint64_t* q_full = o_done + 2;                  // 256 softmax arrivals: both Q blocks in TMEM
-  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_raw + SM::TADDR_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + SM::TADDR_OFF + 4);
-  int* wtot = reinterpret_cast<int*>(smem_raw + SM::WT_OFF);
-  int* cand = reinterpret_cast<int*>(smem_raw + SM::CAND_OFF);
+  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_t2 + SM::TADDR_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_t2 + SM::TADDR_OFF + 4);
+  int* wtot = reinterpret_cast<int*>(smem_t2 + SM::WT_OFF);
+  int* cand = reinterpret_cast<int*>(smem_t2 + SM::CAND_OFF);
   int* cand_cut = cand + p.cand_cap;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1526,18 +963,6 @@ int launch_attn_f32(const PaArgs& pa, int units, int n, cudaStream_t st) {
     return -1;
   dim3 grid((n + pa.qt - 1) / pa.qt, units);
   sparse_attn_kernel<float, DH><<<grid, kPaThreads, smem, st>>>(pa);
-  return 0;
-}
-
-template <int DH>
-int launch_attn_bf16(const PaArgs& pa, int units, int n, cudaStream_t st) {
-  const size_t smem = MmaSmem<DH>::bytes(pa.cand_cap);
-  if (smem > 48 * 1024 && cudaFuncSetAttribute(sparse_attn_mma_kernel<DH>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem)) != cudaSuccess)
-    return -1;
-  dim3 grid((n + pa.qt - 1) / pa.qt, units);
-  sparse_attn_mma_kernel<DH><<<grid, kMmaThreads, smem, st>>>(pa);
   return 0;
 }
 

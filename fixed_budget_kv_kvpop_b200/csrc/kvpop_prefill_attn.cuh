@@ -14,10 +14,9 @@ namespace kvpop {
 int launch_prompt_scores(const LayerArgs& a, int dtype, const void* k, const void* v, int n, const float* ext,
                          float* out, int cap, cudaStream_t st);
 
-// Rows of query heads one attention CTA computes (query positions x G):
-// fp32 kernel (FMA pipes) and bf16 kernel (tensor cores).
+// Rows of query heads one fp32 attention CTA computes (query positions x G;
+// the bf16 tensor-core kernel takes 256 rows).
 constexpr int kPaRows = 64;
-constexpr int kPaMmaRows = 128;
 // Candidate keys staged per tile.
 constexpr int kPaKeys = 32;
 // Largest sort handled in shared memory (keys); larger sorts run in the workspace.
