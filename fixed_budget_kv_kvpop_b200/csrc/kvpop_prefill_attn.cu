@@ -479,27 +479,22 @@ __device__ __forceinline__ void tc_st32(uint32_t taddr, const float (&v)[32]) {
 // ---------------- bf16 attention on tcgen05, two row blocks per CTA ----------------
 // 256 query rows per CTA (two blocks of 128, one per group of four softmax
 // warps), warp-specialized and pipelined through mbarriers:
-//   copy warps 8-11 gather each tile's K and V rows by cp.async into the
-//     128-byte-swizzled operand layout (kT2Stages stages; each thread's
-//     copies arrive on the stage's mbarrier as they land, so nothing waits
-//     for its own copies); mask warps 12-13 build the tile's mask (one key
-//     bitmask per query position);
+//   copy warps 8-11 gather each 64-key tile's K and V rows by cp.async into
+//     the 128-byte-swizzled operand layout (NST stages; each thread's copies
+//     arrive on the stage's mbarrier as they land, so nothing waits for its
+//     own copies); mask warps 12-13 build the tile's mask (64 key bits per
+//     query position);
 //   one thread of warp 14 (block 0) and one of warp 15 (block 1) issue each
-//     block's MMAs in the order S(t+1), O += P V(t), so the tensor cores work
-//     on one block while the other block's softmax runs; each tile's K and V
-//     serve both blocks;
+//     block's MMAs: S(0), S(1), then per tile O += P V(t) and S(t + 2); each
+//     tile's K and V serve both blocks;
 //   softmax warps 0-3 (block 0) and 4-7 (block 1): thread = query row = TMEM
 //     lane.
-// Q and P are the A operands and live in TMEM (rows = lanes, bf16 pairs per
-// 32-bit column), so the MMAs read only K and V from shared memory: with
-// 32-key tiles, re-reading a 128-row Q block from shared memory for every
-// tile would cost 4x the K bytes.  S is single-buffered per block (the
-// softmax reads it into registers and frees it at once); P is
-// double-buffered, so a block's softmax of tile t + 1 need not wait for its
-// P V of tile t (only a rescale of O, or reusing a P buffer, waits for an
-// earlier P V).
-// TMEM columns: O[block] at block * DH, Q[block] at 2 DH + block * DH / 2,
-// S[block] at 3 DH + 32 block, P[block][buf] at 3 DH + 64 + 16 (2 block + buf).
+// Q (A of S = Q K^T) sits in shared memory; S is double-buffered in TMEM per
+// block, so S(t + 1) is computed while the softmax works on S(t); the softmax
+// writes P(t) in bf16 over S(t) (A of P V from TMEM).  One thread's MMAs run
+// in issue order, so S(t + 2) overwrites that buffer only after P V(t) has
+// read it.  An O rescale (rare: lazy threshold) waits for the P V before.
+// TMEM columns: O[block] at block * DH, S[block][buf] at 2 DH + 64 (2 block + buf).
 // Every mbarrier that a role may wait on twice in a row without an
 // intervening handoff is per buffer, so parity waits never alias.
 // 2^x with the hardware's approximate base-2 exponential (ftz; 2^-inf = +0).
@@ -517,6 +512,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // along K.
 __device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return tc_desc(saddr, lbo, sbo) | (2ull << 61);
+}
+// D (+)= A B with A and B in shared memory (descriptors).
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
 // D (+)= A B with A in TMEM (row m = lane m, K pairs of bf16 per 32-bit
 // column) and B in shared memory (descriptor).
@@ -545,30 +548,36 @@ constexpr int kT2Rows = 256;
 // relative).
 constexpr float kT2Lazy = 20.0f;
 constexpr int kT2Keys = 64;
-constexpr int kT2Stages = 5;
 constexpr int kT2Threads = 16 * 32;
 constexpr int kT2Prod = 8;          // first of the 4 copy warps
 constexpr int kT2Mask = 12;         // first of the 2 mask warps
 constexpr int kT2Mma = 14;          // MMA warps: one per row block
 constexpr uint32_t kT2Cols = 512;
 
-// A stage holds the tile's K then V, each as DH / 64 groups of 64 columns
-// (128 bytes per key row), each group 4 swizzle atoms of 8 keys x 128 bytes.
-template <int DH>
+// Shared memory: Q of both blocks, then NST stages each holding the tile's K
+// then V, all in the K-major / MN-major 128-byte-swizzled layout: rows of 64
+// columns (128 bytes) in swizzle atoms of 8 rows x 128 bytes.  Q: per block
+// DH / 64 groups of 16 atoms (128 rows); K and V: DH / 64 groups of 8 atoms
+// (64 keys).
+template <int DH, int NST>
 struct T2Smem {
   static constexpr int NGRP = DH / 64;                                           // 64-column groups per row
+  static constexpr size_t QGRP = 128 * 128;                                      // one group of one Q block: 16 KB
+  static constexpr size_t QBLK = NGRP * QGRP;
+  static constexpr size_t Q_OFF = 0;
   static constexpr size_t GRP = static_cast<size_t>(kT2Keys) * 128;              // one group of one tile: 8 KB
   static constexpr size_t KV_TILE = NGRP * GRP;
   static constexpr size_t STAGE = 2 * KV_TILE;
-  static constexpr size_t KV_OFF = 0;                                            // [stage][K, V]
-  static constexpr size_t META_OFF = KV_OFF + kT2Stages * STAGE;                // [stage][query position] key masks
+  static constexpr size_t KV_OFF = Q_OFF + 2 * QBLK;                            // [stage][K, V]
+  static constexpr size_t META_OFF = KV_OFF + NST * STAGE;                      // [stage][query position] key masks
   static constexpr int META_INTS = 2 * kT2Rows + 4;                              // 2 words per position (256 / G at most), then the full-tile flag
-  static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * kT2Stages * META_INTS;
-  static constexpr int NBAR = 3 * kT2Stages + 7;
+  static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * NST * META_INTS;
+  static constexpr int NBAR = 3 * NST + 13;
   static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
   static constexpr size_t WT_OFF = TADDR_OFF + 16;
   static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);     // [cand_cap] positions, then [cand_cap] cutoffs
-  static_assert(BAR_OFF % 8 == 0 && STAGE % 1024 == 0 && META_OFF % 16 == 0, "shared-memory alignment");
+  static_assert(BAR_OFF % 8 == 0 && STAGE % 1024 == 0 && KV_OFF % 1024 == 0 && META_OFF % 16 == 0,
+                "shared-memory alignment");
   // at least 116 KB: one CTA per SM, which then holds all 512 TMEM columns
   static size_t bytes(int cand_cap) {
     const size_t bb = CAND_OFF + 2 * sizeof(int) * static_cast<size_t>(cand_cap);
@@ -576,10 +585,10 @@ struct T2Smem {
   }
 };
 
-template <int DH>
+template <int DH, int NST>
 __global__ void __launch_bounds__(kT2Threads, 1)
 sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
-  using SM = T2Smem<DH>;
+  using SM = T2Smem<DH, NST>;
   constexpr uint32_t kIdescS = tc_idesc(128, kT2Keys, 0);
   constexpr uint32_t kIdescPV = tc_idesc(128, DH, 1);
   extern __shared__ __align__(1024) uint8_t smem_t2[];
@@ -590,13 +599,13 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   }
   int* meta = reinterpret_cast<int*>(smem_t2 + SM::META_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_t2 + SM::BAR_OFF);
-  uint64_t* kv_full = bars;                       // [stage], 128 producer arrivals as their copies land
-  uint64_t* kv_free = bars + kT2Stages;           // [stage], one MMA commit per row block
-  uint64_t* meta_full = bars + 2 * kT2Stages;     // [stage], the 4 producer warps (mask written)
-  uint64_t* s_full = bars + 3 * kT2Stages;        // [block], MMA commit of S(t) (and of every P V before it)
-  uint64_t* p_full = s_full + 2;                  // [block], 128 softmax arrivals: P(t) in TMEM, S(t) read
-  uint64_t* o_done = p_full + 2;                  // [block], MMA commit after the block's last P V
-  uint64_t* q_full = o_done + 2;                  // 256 softmax arrivals: both Q blocks in TMEM
+  uint64_t* kv_full = bars;                       // [stage], 128 copy-thread arrivals as their copies land
+  uint64_t* kv_free = bars + NST;                 // [stage], one MMA commit per row block
+  uint64_t* meta_full = bars + 2 * NST;           // [stage], the 2 mask warps
+  uint64_t* s_full = bars + 3 * NST;              // [block][buf], MMA commit of S(t)
+  uint64_t* p_full = s_full + 4;                  // [block][buf], 128 softmax arrivals: P(t) over S(t)
+  uint64_t* o_done = p_full + 4;                  // [block], MMA commit after each P V
+  uint64_t* q_full = o_done + 2;                  // 256 softmax arrivals: both Q blocks in shared memory
   uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_t2 + SM::TADDR_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_t2 + SM::TADDR_OFF + 4);
   int* wtot = reinterpret_cast<int*>(smem_t2 + SM::WT_OFF);
@@ -636,16 +645,16 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    for (int i = 0; i < kT2Stages; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&kv_full[i], 128);
       mbar_init(&kv_free[i], 2);
       mbar_init(&meta_full[i], kT2Mma - kT2Mask);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
-      mbar_init(&o_done[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
     mbar_init(q_full, kT2Rows);
     *abort_flag = 0;
     mbar_fence_init();
@@ -656,18 +665,17 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   tc_fence_after();
   const uint32_t tmem = *taddr_s;
   const int ntiles = (count + kT2Keys - 1) / kT2Keys;
-  constexpr uint32_t kColQ = 2 * DH, kColS = 3 * DH;   // TMEM column bases (O at 0; P(t) overwrites S(t))
+  constexpr uint32_t kColS = 2 * DH;   // TMEM: O[block] at block * DH, S[block][buf] at kColS + 64 (2 block + buf)
   if (tid < kT2Rows) {
-    const uint32_t lq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kColQ + (tid >> 7) * (DH / 2);
+    // this thread's query row into the swizzled Q block: 16-byte chunk c of
+    // row r at group c / 8, atom r / 8, row r % 8, position (c % 8) ^ (r % 8)
+    const int r = tid & 127;
+    uint8_t* qb = smem_t2 + SM::Q_OFF + (tid >> 7) * SM::QBLK + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-    for (int c0 = 0; c0 < DH / 2; c0 += 16) {
-      uint32_t v16[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v16[i] = qrow[c0 + i];
-      tc_st16u(lq + c0, v16);
-    }
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    tc_fence_before();
+    for (int c = 0; c < DH / 8; ++c)
+      *reinterpret_cast<uint4*>(qb + (c >> 3) * SM::QGRP + (((c & 7) ^ (r & 7)) << 4)) =
+          make_uint4(qrow[4 * c], qrow[4 * c + 1], qrow[4 * c + 2], qrow[4 * c + 3]);
+    fence_proxy_async_smem();   // generic stores, read by the tensor cores (async proxy)
     mbar_arrive(q_full);
   }
 
@@ -687,8 +695,8 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     // queues behind these copies.
     const int ptid = (warp - kT2Prod) * 32 + lane;
     for (int t = 0; t < ntiles; ++t) {
-      const int st = t % kT2Stages;
-      if (t >= kT2Stages && !wait(&kv_free[st], ((t / kT2Stages) - 1) & 1)) break;
+      const int st = t % NST;
+      if (t >= NST && !wait(&kv_free[st], ((t / NST) - 1) & 1)) break;
       {
         // The tile's K and V rows by cp.async into the swizzled layout: lane
         // = 16-byte chunk of a 256-byte row (two rows per warp instruction),
@@ -716,8 +724,8 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     // ---------------- mask warps ----------------
     const int mw = warp - kT2Mask;
     for (int t = 0; t < ntiles; ++t) {
-      const int st = t % kT2Stages;
-      if (t >= kT2Stages && !wait(&kv_free[st], ((t / kT2Stages) - 1) & 1)) break;
+      const int st = t % NST;
+      if (t >= NST && !wait(&kv_free[st], ((t / NST) - 1) & 1)) break;
       {
         // The tile's mask (§C.1) as two 32-bit words per query position of
         // the CTA (bit i of word h = key 32 h + i visible): lane i of each
@@ -739,14 +747,20 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         const bool full_tile = __all_sync(0xffffffffu, always);
         if (mw == 0 && lane == 0) rm[2 * kT2Rows] = full_tile ? 1u : 0u;
         if (!full_tile) {
-          for (int r = mw; r < p.qt; r += kT2Mma - kT2Mask) {
-            const int qp = q0 + r;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t bm =
-                  __ballot_sync(0xffffffffu, jh[h] >= 0 && jh[h] <= qp && (jh[h] < S || qp - WD < mh[h]));
-              if (lane == 0) rm[2 * r + h] = bm;
+          // positions in groups of 32, alternating between the two mask warps;
+          // lane i keeps position 32 g + i's two words and stores them once
+          // (one shared-memory store per lane and group, so little queues
+          // behind the copy warps' traffic)
+          for (int r0 = 32 * mw; r0 < p.qt; r0 += 32 * (kT2Mma - kT2Mask)) {
+            uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i) {
+              const int qp = q0 + r0 + i;
+              const uint32_t b0 = __ballot_sync(0xffffffffu, jh[0] >= 0 && jh[0] <= qp && (jh[0] < S || qp - WD < mh[0]));
+              const uint32_t b1 = __ballot_sync(0xffffffffu, jh[1] >= 0 && jh[1] <= qp && (jh[1] < S || qp - WD < mh[1]));
+              if (lane == i) { w0 = b0; w1 = b1; }
             }
+            if (r0 + lane < p.qt) *reinterpret_cast<uint2*>(rm + 2 * (r0 + lane)) = make_uint2(w0, w1);
           }
         }
         __syncwarp();
@@ -755,57 +769,57 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     }
   } else if (warp >= kT2Mma) {
     // ---------------- MMA issue: one thread per row block ----------------
-    // Per block: S(0); then for each tile, once the softmax has read S(t) and
-    // written P(t) over it, O += P V(t) and S(t + 1).  The tensor cores run
-    // one thread's MMAs in issue order, so S(t + 1) overwrites those columns
-    // only after P V(t) has read them, and the commit after S(t + 1) also
-    // covers P V(t) (the softmax may then rescale O).  The blocks do not wait
-    // for each other; a stage is free once both blocks' P V of it completed.
+    // Per block: S(0), S(1); then per tile, once the softmax has written
+    // P(t) over S(t): O += P V(t), and S(t + 2) into the same buffer (after
+    // P V(t) in issue order).  The blocks do not wait for each other; a stage
+    // is free once both blocks' P V of it completed.
     const int XB = warp - kT2Mma;
     if (lane == 0 && ntiles > 0) {
-      // S_X(t) = Q_X K(t)^T: A = Q_X in TMEM (8 columns per 16 dims), B = the K tile
+      // S_X(t) = Q_X K(t)^T: A = Q_X and B = the K tile, both K-major swizzled in shared memory
       auto issue_s = [&](int X, int t) {
-        const int st = t % kT2Stages;
+        const int st = t % NST;
         const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE);
-        const uint32_t d = tmem + kColS + static_cast<uint32_t>(X * kT2Keys);
-        const uint32_t aq = tmem + kColQ + static_cast<uint32_t>(X * (DH / 2));
-        // K-major B: 16 dims = 32 bytes of a 128-byte swizzled row; 8-key groups 1024 bytes apart
+        const uint32_t qb = sbase + static_cast<uint32_t>(SM::Q_OFF + X * SM::QBLK);
+        const uint32_t d = tmem + kColS + static_cast<uint32_t>((2 * X + (t & 1)) * kT2Keys);
+        // 16 dims = 32 bytes of a 128-byte swizzled row; 8-row groups 1024 bytes apart
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks)
-          tc_mma_ts(d, aq + 8u * ks,
-                    tc_desc_sw128(kb + static_cast<uint32_t>((ks >> 2) * SM::GRP + (ks & 3) * 32), 16, 1024), kIdescS,
-                    ks > 0 ? 1u : 0u);
-        tc_commit(&s_full[X]);
+          tc_mma(d, tc_desc_sw128(qb + static_cast<uint32_t>((ks >> 2) * SM::QGRP + (ks & 3) * 32), 16, 1024),
+                 tc_desc_sw128(kb + static_cast<uint32_t>((ks >> 2) * SM::GRP + (ks & 3) * 32), 16, 1024), kIdescS,
+                 ks > 0 ? 1u : 0u);
+        tc_commit(&s_full[2 * X + (t & 1)]);
       };
       // O_X += P_X(t) V(t): A = P_X(t) in TMEM over S_X(t) (8 columns per 16 keys), B = the V tile
       auto issue_pv = [&](int X, int t) {
-        const int st = t % kT2Stages;
+        const int st = t % NST;
         const uint32_t vb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE + SM::KV_TILE);
         const uint32_t d = tmem + static_cast<uint32_t>(X * DH);
-        const uint32_t ap = tmem + kColS + static_cast<uint32_t>(X * kT2Keys);
+        const uint32_t ap = tmem + kColS + static_cast<uint32_t>((2 * X + (t & 1)) * kT2Keys);
         // MN-major B: 64-dim groups GRP bytes apart (leading), 8-key groups 1024 bytes apart (stride);
         // 16 keys per instruction = two 8-key groups
 #pragma unroll
         for (int kk = 0; kk < kT2Keys / 16; ++kk)
           tc_mma_ts(d, ap + 8u * kk, tc_desc_sw128(vb + static_cast<uint32_t>(kk * 2048), SM::GRP, 1024), kIdescPV,
                     (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&o_done[X]);
       };
-      bool ok = wait(q_full, 0) && wait(&kv_full[0], 0);
-      if (ok) {
-        tc_fence_after();
-        issue_s(XB, 0);
+      bool ok = wait(q_full, 0);
+      for (int t = 0; ok && t < 2 && t < ntiles; ++t) {
+        ok = wait(&kv_full[t % NST], (t / NST) & 1);
+        if (ok) {
+          tc_fence_after();
+          issue_s(XB, t);
+        }
       }
       for (int t = 0; ok && t < ntiles; ++t) {
-        ok = wait(&p_full[XB], t & 1);
+        ok = wait(&p_full[2 * XB + (t & 1)], (t >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
         issue_pv(XB, t);
-        tc_commit(&kv_free[t % kT2Stages]);
-        if (t + 1 < ntiles) {
-          ok = wait(&kv_full[(t + 1) % kT2Stages], ((t + 1) / kT2Stages) & 1);
-          if (ok) issue_s(XB, t + 1);
-        } else {
-          tc_commit(&o_done[XB]);
+        tc_commit(&kv_free[t % NST]);
+        if (t + 2 < ntiles) {
+          ok = wait(&kv_full[(t + 2) % NST], ((t + 2) / NST) & 1);
+          if (ok) issue_s(XB, t + 2);
         }
       }
     }
@@ -823,21 +837,21 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int t = 0; t < ntiles; ++t) {
-      const int st = t % kT2Stages;
-      bool got = wait(&meta_full[st], (t / kT2Stages) & 1);
-      got = got && wait(&s_full[X], t & 1);
+      const int st = t % NST;
+      bool got = wait(&meta_full[st], (t / NST) & 1);
+      got = got && wait(&s_full[2 * X + (t & 1)], (t >> 1) & 1);
       if (!__all_sync(0xffffffffu, got)) {   // the TMEM loads below are warp-collective
         ok = false;
         break;
       }
       tc_fence_after();
-      // S(t) row: 64 fp32 columns (the commit after S(t) also covers every P V
-      // before it, so O may be rescaled below without another wait)
+      // S(t) row: 64 fp32 columns of buffer t & 1
+      const uint32_t tS = tmem + kColS + static_cast<uint32_t>((2 * X + (t & 1)) * kT2Keys);
       float sv[kT2Keys];
       {
         float lo[32], hi[32];
-        tc_ld32(tmem + kColS + static_cast<uint32_t>(X * kT2Keys) + lrow, lo);
-        tc_ld32(tmem + kColS + static_cast<uint32_t>(X * kT2Keys) + 32u + lrow, hi);
+        tc_ld32(tS + lrow, lo);
+        tc_ld32(tS + 32u + lrow, hi);
 #pragma unroll
         for (int i = 0; i < 32; ++i) { sv[i] = lo[i]; sv[32 + i] = hi[i]; }
       }
@@ -888,11 +902,17 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
           ps[(i >> 1) & 3] += p0 + p1;
           pk[i / 2] = pack_bf16(p0, p1);
         }
-        tc_st16u(tmem + kColS + static_cast<uint32_t>(X * kT2Keys + 16 * h) + lrow, pk);
+        tc_st16u(tS + static_cast<uint32_t>(16 * h) + lrow, pk);
       }
       l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       if (__any_sync(0xffffffffu, resc)) {
-        // every P V before S(t) has completed (see above): rescale this row of O
+        // rescale this row of O once the P V before (of tile t - 1) has completed
+        const bool done = t == 0 || wait(&o_done[X], (t - 1) & 1);
+        if (!__all_sync(0xffffffffu, done)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const float f = resc ? alpha : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < DH; c0 += 32) {
@@ -905,10 +925,10 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(&p_full[X]);
+      mbar_arrive(&p_full[2 * X + (t & 1)]);
     }
     bool fin = ok && ntiles > 0;
-    if (fin) fin = wait(&o_done[X], 0);
+    if (fin) fin = wait(&o_done[X], (ntiles - 1) & 1);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const int g = grow % G;
@@ -940,17 +960,26 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   }
 }
 
-template <int DH>
-int launch_attn_tc2(const PaArgs& pa, int units, int n, cudaStream_t st) {
-  const size_t smem = T2Smem<DH>::bytes(pa.cand_cap);
-  if (smem > 227 * 1024) return -2;
-  if (units == 0 || n == 0) return 0;
-  if (cudaFuncSetAttribute(sparse_attn_tc2_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int DH, int NST>
+int launch_attn_tc2_stages(const PaArgs& pa, int units, int n, size_t smem, cudaStream_t st) {
+  if (cudaFuncSetAttribute(sparse_attn_tc2_kernel<DH, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return -1;
   dim3 grid((n + pa.qt - 1) / pa.qt, units);
-  sparse_attn_tc2_kernel<DH><<<grid, kT2Threads, smem, st>>>(pa);
+  sparse_attn_tc2_kernel<DH, NST><<<grid, kT2Threads, smem, st>>>(pa);
   return 0;
+}
+
+// Four stages when they fit in shared memory beside the candidate lists, else three.
+template <int DH>
+int launch_attn_tc2(const PaArgs& pa, int units, int n, cudaStream_t st) {
+  constexpr size_t kMax = 227 * 1024;
+  if (units == 0 || n == 0) return 0;
+  const size_t smem4 = T2Smem<DH, 4>::bytes(pa.cand_cap);
+  if (smem4 <= kMax) return launch_attn_tc2_stages<DH, 4>(pa, units, n, smem4, st);
+  const size_t smem3 = T2Smem<DH, 3>::bytes(pa.cand_cap);
+  if (smem3 <= kMax) return launch_attn_tc2_stages<DH, 3>(pa, units, n, smem3, st);
+  return -2;
 }
 
 template <int DH>
