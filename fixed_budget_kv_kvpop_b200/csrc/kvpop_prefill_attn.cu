@@ -25,9 +25,9 @@
 // the recent positions of its queries.  It then streams them in tiles of
 // kPaKeys through shared memory with an online softmax in fp32 (FMA pipes),
 // masking each (query, key) pair by the rule above.  bf16 inputs take the
-// tensor-core kernel instead (sparse_attn_mma_kernel: 128 rows per CTA,
-// m16n8k16 bf16 MMAs with fp32 accumulation, keys gathered by cp.async);
-// fp32 inputs keep the FMA kernel so that they are never rounded to a
+// tcgen05 kernel instead (sparse_attn_tc2_kernel: 256 rows per CTA, S and O
+// accumulated in TMEM, keys gathered by cp.async into swizzled operand
+// tiles); fp32 inputs keep the FMA kernel so that they are never rounded to a
 // tensor-core input type.
 //
 // Cache build.  The tokens whose cutoff is "never" are the running top-k at
