@@ -138,7 +138,7 @@ def mma_kernel_sha256() -> str:
     import hashlib
     with open(os.path.join(ROOT, "fixed_budget_kv_kvpop_b200", "csrc", "kvpop_prefill_attn.cu")) as fh:
         src = fh.read()
-    a = src.index("bf16 attention on tcgen05, two row blocks per CTA")
+    a = src.index("bf16 attention on tcgen05: persistent, two row blocks per work item")
     b = src.index("int launch_attn_f32(")
     return hashlib.sha256(_strip_code(src[a:b]).encode()).hexdigest()
 

@@ -25,10 +25,10 @@
 // the recent positions of its queries.  It then streams them in tiles of
 // kPaKeys through shared memory with an online softmax in fp32 (FMA pipes),
 // masking each (query, key) pair by the rule above.  bf16 inputs take the
-// tcgen05 kernel instead (sparse_attn_tc2_kernel: 256 rows per CTA, S and O
-// accumulated in TMEM, keys gathered by cp.async into swizzled operand
-// tiles); fp32 inputs keep the FMA kernel so that they are never rounded to a
-// tensor-core input type.
+// tcgen05 kernel instead (sparse_attn_tcp_kernel: persistent, one CTA per SM
+// walking work items of 256 query rows, S and O accumulated in TMEM, keys
+// gathered by cp.async into swizzled operand tiles); fp32 inputs keep the FMA
+// kernel so that they are never rounded to a tensor-core input type.
 //
 // Cache build.  The tokens whose cutoff is "never" are the running top-k at
 // the last prompt position; place_kept_kernel writes them to the long-range
@@ -153,18 +153,13 @@ template <> struct PaIo<float> {
 // Every key a query of the tile may attend to is among them.  Block-wide
 // (all NT threads); returns the count (at most cap).  Each thread scans 8
 // consecutive positions per round (8 cutoff loads in flight), and one block
-// scan per NT * 8 positions places the kept ones.  With cand_cut, each
-// candidate's cutoff is stored beside it (0 for the sinks, which need none).
+// scan per NT * 8 positions places the kept ones.
 template <int NT>
-__device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1, int cap,
-                                 int* cand_cut = nullptr) {
+__device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1, int cap) {
   constexpr int R = 8;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ns = min(S, q1);
-  for (int i = tid; i < ns; i += NT) {
-    cand[i] = i;
-    if (cand_cut != nullptr) cand_cut[i] = 0;
-  }
+  for (int i = tid; i < ns; i += NT) cand[i] = i;
   int count = ns;
   for (int base = S; base <= m0; base += NT * R) {
     const int j0 = base + tid * R;
@@ -194,10 +189,7 @@ __device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S,
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       if ((mine >> r) & 1u) {
-        if (off < cap) {
-          cand[off] = j0 + r;
-          if (cand_cut != nullptr) cand_cut[off] = c[r];
-        }
+        if (off < cap) cand[off] = j0 + r;
         ++off;
       }
     }
@@ -207,10 +199,7 @@ __device__ int gather_candidates(int* cand, int* wtot, const int32_t* cu, int S,
   const int r0 = max(S, m0 + 1);
   const int nr = max(0, q1 - r0);
   for (int i = tid; i < nr; i += NT)
-    if (count + i < cap) {
-      cand[count + i] = r0 + i;
-      if (cand_cut != nullptr) cand_cut[count + i] = cu[r0 + i];
-    }
+    if (count + i < cap) cand[count + i] = r0 + i;
   count += nr;
   __syncthreads();
   return min(count, cap);   // count <= cap always: S + K + qt + W + D bounds it
@@ -476,27 +465,6 @@ __device__ __forceinline__ void tc_st32(uint32_t taddr, const float (&v)[32]) {
       : "memory");
 }
 
-// ---------------- bf16 attention on tcgen05, two row blocks per CTA ----------------
-// 256 query rows per CTA (two blocks of 128, one per group of four softmax
-// warps), warp-specialized and pipelined through mbarriers:
-//   copy warps 8-11 gather each 64-key tile's K and V rows by cp.async into
-//     the 128-byte-swizzled operand layout (NST stages; each thread's copies
-//     arrive on the stage's mbarrier as they land, so nothing waits for its
-//     own copies); mask warps 12-13 build the tile's mask (64 key bits per
-//     query position);
-//   one thread of warp 14 (block 0) and one of warp 15 (block 1) issue each
-//     block's MMAs: S(0), S(1), then per tile O += P V(t) and S(t + 2); each
-//     tile's K and V serve both blocks;
-//   softmax warps 0-3 (block 0) and 4-7 (block 1): thread = query row = TMEM
-//     lane.
-// Q (A of S = Q K^T) sits in shared memory; S is double-buffered in TMEM per
-// block, so S(t + 1) is computed while the softmax works on S(t); the softmax
-// writes P(t) in bf16 over S(t) (A of P V from TMEM).  One thread's MMAs run
-// in issue order, so S(t + 2) overwrites that buffer only after P V(t) has
-// read it.  An O rescale (rare: lazy threshold) waits for the P V before.
-// TMEM columns: O[block] at block * DH, S[block][buf] at 2 DH + 64 (2 block + buf).
-// Every mbarrier that a role may wait on twice in a row without an
-// intervening handoff is per buffer, so parity waits never alias.
 // 2^x with the hardware's approximate base-2 exponential (ftz; 2^-inf = +0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -540,6 +508,37 @@ __device__ __forceinline__ void tc_st16u(uint32_t taddr, const uint32_t (&v)[16]
       : "memory");
 }
 
+// ---------------- bf16 attention on tcgen05: persistent, two row blocks per work item ----------------
+// One CTA per SM walks its share of the work items (unit, 256 query rows =
+// 256 / G positions x G heads), items blockIdx.x, blockIdx.x + gridDim.x, ...
+// in order.  Warp-specialized and pipelined through mbarriers, with the
+// pipeline running on across item boundaries (a global tile counter T picks
+// every stage, buffer and parity):
+//   copy warps 8-11 gather the next item's candidate keys while the current
+//     item's last tiles are still being computed, then each 64-key tile's K
+//     and V rows by cp.async into the 128-byte-swizzled operand layout (NST
+//     stages; each thread's copies arrive on the stage's mbarrier as they
+//     land); mask warps 12-13 build each tile's mask (64 key bits per query
+//     position);
+//   one thread of warp 14 (block 0) and one of warp 15 (block 1) issue each
+//     block's MMAs: S(T), S(T + 1), then per tile O += P V(T) and S(T + 2);
+//     each tile's K and V serve both blocks.  The same thread loads its
+//     block's Q rows of the next item by TMA as soon as the current item's
+//     last S has read them;
+//   softmax warps 0-3 (block 0) and 4-7 (block 1): thread = query row = TMEM
+//     lane; each item ends with its rows' epilogue, while the next item's
+//     first S tiles are already computed.
+// Q (A of S = Q K^T) sits in shared memory; S is double-buffered in TMEM per
+// block; the softmax writes P(T) in bf16 over S(T) (A of P V from TMEM).  One
+// thread's MMAs run in issue order, so S(T + 2) overwrites that buffer only
+// after P V(T) has read it.  An O rescale (rare: lazy threshold) waits for
+// the P V before.  TMEM columns: O[block] at block * DH, S[block][buf] at
+// 2 DH + 64 (2 block + buf).  Block X holds query positions X * 128 / G ..
+// (X + 1) * 128 / G - 1 of the item; its row r is head r / (128 / G) at
+// position r % (128 / G), so each head's rows are one TMA box of Q.  Every
+// mbarrier that a role may wait on twice in a row without an intervening
+// handoff is per buffer, so parity waits never alias.
+
 constexpr int kT2Rows = 256;
 // Lazy rescale threshold (log2 units): the running max of a row moves only
 // when a tile's max exceeds it by 2^20.  A rescale of O waits for the P V in
@@ -553,12 +552,15 @@ constexpr int kT2Prod = 8;          // first of the 4 copy warps
 constexpr int kT2Mask = 12;         // first of the 2 mask warps
 constexpr int kT2Mma = 14;          // MMA warps: one per row block
 constexpr uint32_t kT2Cols = 512;
+constexpr int kT2Ring = 8;          // tile counts of items in flight (more than NST + 1 items)
+constexpr int kT2CopyBar = 1;       // named barrier of the 128 copy threads
 
 // Shared memory: Q of both blocks, then NST stages each holding the tile's K
 // then V, all in the K-major / MN-major 128-byte-swizzled layout: rows of 64
 // columns (128 bytes) in swizzle atoms of 8 rows x 128 bytes.  Q: per block
 // DH / 64 groups of 16 atoms (128 rows); K and V: DH / 64 groups of 8 atoms
-// (64 keys).
+// (64 keys).  Then the masks, the barriers, a few words, and the candidate
+// positions of two items (the current one and the next, gathered ahead).
 template <int DH, int NST>
 struct T2Smem {
   static constexpr int NGRP = DH / 64;                                           // 64-column groups per row
@@ -572,12 +574,12 @@ struct T2Smem {
   static constexpr size_t META_OFF = KV_OFF + NST * STAGE;                      // [stage][query position] key masks
   static constexpr int META_INTS = 2 * kT2Rows + 4;                              // 2 words per position (256 / G at most), then the full-tile flag
   static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * NST * META_INTS;
-  static constexpr int NBAR = 3 * NST + 13;
-  static constexpr size_t TADDR_OFF = BAR_OFF + 8 * NBAR;
-  static constexpr size_t WT_OFF = TADDR_OFF + 16;
-  static constexpr size_t CAND_OFF = WT_OFF + 16 * sizeof(int);     // [cand_cap] positions, then [cand_cap] cutoffs
-  static_assert(BAR_OFF % 8 == 0 && STAGE % 1024 == 0 && KV_OFF % 1024 == 0 && META_OFF % 16 == 0,
-                "shared-memory alignment");
+  static constexpr int NBAR = 3 * NST + 4 + 4 + 2 + 2 + 2 + kT2Ring + 2;
+  static constexpr size_t MISC_OFF = BAR_OFF + 8 * NBAR;                        // TMEM address, abort flag, tile-count ring, warp totals
+  static constexpr size_t CAND_OFF = MISC_OFF + 64;                             // [item % 2][cand_cap] positions
+  static_assert(BAR_OFF % 8 == 0 && STAGE % 1024 == 0 && KV_OFF % 1024 == 0 && META_OFF % 16 == 0 &&
+                    2 + kT2Ring + 4 <= 16,
+                "shared-memory layout");
   // at least 116 KB: one CTA per SM, which then holds all 512 TMEM columns
   static size_t bytes(int cand_cap) {
     const size_t bb = CAND_OFF + 2 * sizeof(int) * static_cast<size_t>(cand_cap);
@@ -585,9 +587,133 @@ struct T2Smem {
   }
 };
 
+// Named barrier over `nthreads` threads (whole warps); the second form
+// returns whether any participating thread passed true.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r) : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads) : "memory");
+  return r != 0;
+}
+// 32 bytes to global memory in one store (the address 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               :: "l"(ptr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+// Non-blocking test of an mbarrier phase (acquire on success).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Test of an mbarrier phase that may suspend the thread (no issue slots) for
+// up to about `ns` nanoseconds while the phase is incomplete.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(ns) : "memory");
+  return ok != 0;
+}
+// One box of a 3-D tensor map into shared memory (no multicast), completion
+// counted in bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// The candidates of one work item (the keys gather_candidates lists, in the
+// same ascending order), computed by the 128 copy
+// threads (ptid 0..127) alone, synchronised by named barrier kT2CopyBar.
+// Each warp scans 32 x R consecutive cutoffs per round with coalesced loads
+// (lane i reads position base + 32 r + i), ballots the kept ones and places
+// them after the earlier warps' (one scan over the four warp totals per
+// round of 128 x R positions).  Returns the count (at most cap).
+__device__ __forceinline__ int gather_candidates_copy(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1,
+                                                      int cap, int ptid) {
+  constexpr int NT = 128, R = 16;
+  const int lane = ptid & 31, w = ptid >> 5;
+  const int ns = min(S, q1);
+  for (int i = ptid; i < ns; i += NT) cand[i] = i;
+  int count = ns;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = S; base <= m0; base += NT * R) {
+    const int wb = base + w * 32 * R;
+    int c[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int j = wb + 32 * r + lane;
+      c[r] = j <= m0 ? cu[j] : 0;
+    }
+    uint32_t bal[R];
+    int tot = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int j = wb + 32 * r + lane;
+      bal[r] = __ballot_sync(0xffffffffu, j <= m0 && c[r] > m0);
+      tot += __popc(bal[r]);
+    }
+    if (lane == 0) wtot[w] = tot;
+    named_bar_sync(kT2CopyBar, NT);
+    int off = count, total = 0;
+#pragma unroll
+    for (int x = 0; x < NT / 32; ++x) {
+      const int t = wtot[x];
+      off += (x < w) ? t : 0;
+      total += t;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if ((bal[r] >> lane) & 1u) {
+        const int o = off + __popc(bal[r] & lt);
+        if (o < cap) cand[o] = wb + 32 * r + lane;
+      }
+      off += __popc(bal[r]);
+    }
+    count += total;
+    named_bar_sync(kT2CopyBar, NT);   // wtot is rewritten next round
+  }
+  const int r0 = max(S, m0 + 1);
+  const int nr = max(0, q1 - r0);
+  for (int i = ptid; i < nr; i += NT)
+    if (count + i < cap) cand[count + i] = r0 + i;
+  count += nr;
+  named_bar_sync(kT2CopyBar, NT);
+  return min(count, cap);   // count <= cap always: S + K + qt + W + D bounds it
+}
+
+// A work item: 256 / G query positions [q0, q1) of unit u (batch row b, KV head hk).
+struct T2Item {
+  int u, b, hk, q0, q1;
+};
+__device__ __forceinline__ T2Item t2_item(const PaArgs& p, int ntq, int it) {
+  T2Item w;
+  w.u = it / ntq;
+  w.b = w.u / p.Hkv;
+  w.hk = w.u % p.Hkv;
+  w.q0 = (it % ntq) * p.qt;
+  w.q1 = min(p.n, w.q0 + p.qt);
+  return w;
+}
+
 template <int DH, int NST>
 __global__ void __launch_bounds__(kT2Threads, 1)
-sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
+sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ PaArgs p, int nitems) {
   using SM = T2Smem<DH, NST>;
   constexpr uint32_t kIdescS = tc_idesc(128, kT2Keys, 0);
   constexpr uint32_t kIdescPV = tc_idesc(128, DH, 1);
@@ -602,42 +728,26 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   uint64_t* kv_full = bars;                       // [stage], 128 copy-thread arrivals as their copies land
   uint64_t* kv_free = bars + NST;                 // [stage], one MMA commit per row block
   uint64_t* meta_full = bars + 2 * NST;           // [stage], the 2 mask warps
-  uint64_t* s_full = bars + 3 * NST;              // [block][buf], MMA commit of S(t)
-  uint64_t* p_full = s_full + 4;                  // [block][buf], 128 softmax arrivals: P(t) over S(t)
+  uint64_t* s_full = bars + 3 * NST;              // [block][buf], MMA commit of S(T)
+  uint64_t* p_full = s_full + 4;                  // [block][buf], 128 softmax arrivals: P(T) over S(T)
   uint64_t* o_done = p_full + 4;                  // [block], MMA commit after each P V
-  uint64_t* q_full = o_done + 2;                  // 256 softmax arrivals: both Q blocks in shared memory
-  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(smem_t2 + SM::TADDR_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_t2 + SM::TADDR_OFF + 4);
-  int* wtot = reinterpret_cast<int*>(smem_t2 + SM::WT_OFF);
-  int* cand = reinterpret_cast<int*>(smem_t2 + SM::CAND_OFF);
-  int* cand_cut = cand + p.cand_cap;
+  uint64_t* q_full = o_done + 2;                  // [block], the block's Q rows of an item landed (TMA bytes)
+  uint64_t* q_free = q_full + 2;                  // [block], MMA commit after an item's last S
+  uint64_t* item_full = q_free + 2;               // [item % ring], the item's candidates and tile count are ready
+  uint64_t* cand_free = item_full + kT2Ring;      // [item % 2], the mask warps are done with the item's candidates
+  int* misc = reinterpret_cast<int*>(smem_t2 + SM::MISC_OFF);
+  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(misc);
+  volatile int* abort_flag = misc + 1;
+  int* count_ring = misc + 2;                     // [item % ring] candidate count of the item
+  int* wtot = misc + 2 + kT2Ring;                 // copy warps' totals (gather scan)
+  int* cand2 = reinterpret_cast<int*>(smem_t2 + SM::CAND_OFF);   // item i's candidates at cand2 + (i & 1) * cand_cap
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int u = blockIdx.y;
-  const int b = u / p.Hkv, hk = u % p.Hkv;
   const int n = p.n, S = p.S, WD = p.W + p.D, G = p.G;
-  const int q0 = blockIdx.x * p.qt;
-  const int q1 = min(n, q0 + p.qt);
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* kgp = static_cast<const __nv_bfloat16*>(p.k) + static_cast<size_t>(u) * n * DH;
-  const __nv_bfloat16* vgp = static_cast<const __nv_bfloat16*>(p.v) + static_cast<size_t>(u) * n * DH;
-  const int32_t* cu = p.cut + static_cast<size_t>(u) * n;
-
-  // softmax threads: their query row (row = position offset * G + head) into
-  // registers, zero past the prompt; the loads land while the candidates are
-  // gathered, and go to TMEM once its address is known
-  uint32_t qrow[DH / 2];
-  if (tid < kT2Rows) {
-    const int qp = q0 + tid / G, g = tid % G;
-    const bool in = qp < q1;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        qg + ((static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (in ? qp : 0)) * DH);
-#pragma unroll
-    for (int c = 0; c < DH / 8; ++c) {
-      const uint4 x = in ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-      qrow[4 * c] = x.x; qrow[4 * c + 1] = x.y; qrow[4 * c + 2] = x.z; qrow[4 * c + 3] = x.w;
-    }
-  }
+  const int ntq = (n + p.qt - 1) / p.qt;
+  const int PB = 128 / G;                          // query positions per row block
+  const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k);
+  const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(p.v);
 
   if (warp == kT2Mma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -654,30 +764,21 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
-    mbar_init(q_full, kT2Rows);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&o_done[i], 1);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_free[i], 1);
+    }
+    for (int i = 0; i < kT2Ring; ++i) mbar_init(&item_full[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&cand_free[i], kT2Mma - kT2Mask);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  const int count = gather_candidates<kT2Threads>(cand, wtot, cu, S, q0 - WD, q1, p.cand_cap, cand_cut);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *taddr_s;
-  const int ntiles = (count + kT2Keys - 1) / kT2Keys;
   constexpr uint32_t kColS = 2 * DH;   // TMEM: O[block] at block * DH, S[block][buf] at kColS + 64 (2 block + buf)
-  if (tid < kT2Rows) {
-    // this thread's query row into the swizzled Q block: 16-byte chunk c of
-    // row r at group c / 8, atom r / 8, row r % 8, position (c % 8) ^ (r % 8)
-    const int r = tid & 127;
-    uint8_t* qb = smem_t2 + SM::Q_OFF + (tid >> 7) * SM::QBLK + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-    for (int c = 0; c < DH / 8; ++c)
-      *reinterpret_cast<uint4*>(qb + (c >> 3) * SM::QGRP + (((c & 7) ^ (r & 7)) << 4)) =
-          make_uint4(qrow[4 * c], qrow[4 * c + 1], qrow[4 * c + 2], qrow[4 * c + 3]);
-    fence_proxy_async_smem();   // generic stores, read by the tensor cores (async proxy)
-    mbar_arrive(q_full);
-  }
 
   // bounded wait; on expiry every role stops at its next check
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -687,17 +788,58 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     *abort_flag = 1;
     return false;
   };
+  auto ntiles_of = [](int count) { return (count + kT2Keys - 1) / kT2Keys; };
 
   if (warp >= kT2Prod && warp < kT2Mask) {
-    // ---------------- copy warps ----------------
+    // ---------------- copy warps: candidates, then K and V tiles ----------------
     // Their loop is bound by the load/store unit's rate for cp.async; the
     // masks are built by other warps, so no shared-memory access of theirs
-    // queues behind these copies.
+    // queues behind these copies.  The candidates of item i + 1 are gathered
+    // once item i's first NST tiles are issued (or after all of them, if it
+    // has fewer), into the buffer of item i - 1 (released by the mask
+    // warps); the softmax and MMA roles only need the count, kept in a ring.
+    // Every named barrier and every exit is taken by all 128 threads alike: a
+    // thread whose wait failed skips its work but keeps the same path.
     const int ptid = (warp - kT2Prod) * 32 + lane;
-    for (int t = 0; t < ntiles; ++t) {
-      const int st = t % NST;
-      if (t >= NST && !wait(&kv_free[st], ((t / NST) - 1) & 1)) break;
-      {
+    bool failed = false;
+    auto gather = [&](int i) {   // item i's candidates into its buffer; count to the ring
+      const T2Item w = t2_item(p, ntq, blockIdx.x + i * gridDim.x);
+      const int count = gather_candidates_copy(cand2 + (i & 1) * p.cand_cap, wtot, p.cut + static_cast<size_t>(w.u) * n,
+                                               S, w.q0 - WD, w.q1, p.cand_cap, ptid);
+      if (ptid == 0) {
+        count_ring[i % kT2Ring] = count;
+        mbar_arrive(&item_full[i % kT2Ring]);
+      }
+      return count;
+    };
+    int next_count = gather(0);
+    int T = 0;
+    for (int i = 0;; ++i) {
+      const int it = blockIdx.x + i * gridDim.x;
+      if (it >= nitems) break;
+      const T2Item w = t2_item(p, ntq, it);
+      const bool has_next = it + static_cast<int>(gridDim.x) < nitems;
+      const int* cand = cand2 + (i & 1) * p.cand_cap;
+      const int count = next_count;
+      const int nt = ntiles_of(count);
+      const int gat = min(NST, nt);
+      const __nv_bfloat16* kgp = kbase + static_cast<size_t>(w.u) * n * DH;
+      const __nv_bfloat16* vgp = vbase + static_cast<size_t>(w.u) * n * DH;
+      for (int t = 0; t <= nt; ++t) {
+        if (t == gat && has_next) {
+          const bool good = failed || i == 0 || wait(&cand_free[(i - 1) & 1], ((i - 1) >> 1) & 1);
+          if (named_bar_or(kT2CopyBar, 128, failed || !good || *abort_flag != 0))
+            failed = true;
+          else
+            next_count = gather(i + 1);
+        }
+        if (t == nt) break;
+        const int st = T % NST;
+        ++T;
+        if (failed || (T > NST && !wait(&kv_free[st], (((T - 1) / NST) - 1) & 1))) {
+          failed = true;
+          continue;
+        }
         // The tile's K and V rows by cp.async into the swizzled layout: lane
         // = 16-byte chunk of a 256-byte row (two rows per warp instruction),
         // chunk c of key r at group c / 8, atom r / 8, row r % 8, position
@@ -706,8 +848,8 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         constexpr int CPR = DH / 8;                       // 16-byte chunks per row
         const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE);
 #pragma unroll
-        for (int i = ptid; i < kT2Keys * CPR; i += 128) {
-          const int key = i / CPR, c = i % CPR;
+        for (int x = ptid; x < kT2Keys * CPR; x += 128) {
+          const int key = x / CPR, c = x % CPR;
           const int kidx = t * kT2Keys + key;
           const int jj = kidx < count ? cand[kidx] : -1;
           const size_t off = jj >= 0 ? static_cast<size_t>(jj) * DH + c * 8 : 0;
@@ -718,22 +860,37 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         }
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(&kv_full[st])) : "memory");
       }
+      if (named_bar_or(kT2CopyBar, 128, failed || *abort_flag != 0)) break;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");   // nothing lands after the CTA's last barrier
   } else if (warp >= kT2Mask && warp < kT2Mma) {
     // ---------------- mask warps ----------------
     const int mw = warp - kT2Mask;
-    for (int t = 0; t < ntiles; ++t) {
-      const int st = t % NST;
-      if (t >= NST && !wait(&kv_free[st], ((t / NST) - 1) & 1)) break;
-      {
+    int T = 0;
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int it = blockIdx.x + i * gridDim.x;
+      if (it >= nitems) break;
+      if (!__all_sync(0xffffffffu, wait(&item_full[i % kT2Ring], (i / kT2Ring) & 1))) break;
+      const T2Item w = t2_item(p, ntq, it);
+      const int q0 = w.q0, q1 = w.q1;
+      const int count = count_ring[i % kT2Ring];
+      const int nt = ntiles_of(count);
+      const int* cand = cand2 + (i & 1) * p.cand_cap;
+      const int32_t* cu = p.cut + static_cast<size_t>(w.u) * n;
+      for (int t = 0; t < nt; ++t, ++T) {
+        const int st = T % NST;
+        if (!__all_sync(0xffffffffu, T < NST || wait(&kv_free[st], ((T / NST) - 1) & 1))) {
+          ok = false;
+          break;
+        }
         // The tile's mask (§C.1) as two 32-bit words per query position of
-        // the CTA (bit i of word h = key 32 h + i visible): lane i of each
+        // the item (bit i of word h = key 32 h + i visible): lane i of each
         // mask warp holds keys i and 32 + i, and one ballot per word collects
         // the bits.  Key j (cutoff c) is visible at position q iff j <= q and
         // (j is a sink or q - W - D < max(j, c)).  A tile whose keys are all
-        // visible to every position of the CTA (the common case: long-range
-        // keys kept past the CTA's last position) is only flagged.
+        // visible to every position of the item (the common case: long-range
+        // keys kept past the item's last position) is only flagged.
         uint32_t* rm = reinterpret_cast<uint32_t*>(meta + st * SM::META_INTS);
         int jh[2], mh[2];
         bool always = true;
@@ -741,7 +898,7 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         for (int h = 0; h < 2; ++h) {
           const int idx = t * kT2Keys + 32 * h + lane;
           jh[h] = idx < count ? cand[idx] : -1;
-          mh[h] = jh[h] >= 0 ? max(jh[h], cand_cut[idx]) : 0;
+          mh[h] = jh[h] >= 0 ? max(jh[h], cu[jh[h]]) : 0;
           always = always && jh[h] >= 0 && jh[h] <= q0 && (jh[h] < S || q1 - 1 - WD < mh[h]);
         }
         const bool full_tile = __all_sync(0xffffffffu, always);
@@ -749,16 +906,14 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         if (!full_tile) {
           // positions in groups of 32, alternating between the two mask warps;
           // lane i keeps position 32 g + i's two words and stores them once
-          // (one shared-memory store per lane and group, so little queues
-          // behind the copy warps' traffic)
           for (int r0 = 32 * mw; r0 < p.qt; r0 += 32 * (kT2Mma - kT2Mask)) {
             uint32_t w0 = 0u, w1 = 0u;
 #pragma unroll 4
-            for (int i = 0; i < 32; ++i) {
-              const int qp = q0 + r0 + i;
+            for (int x = 0; x < 32; ++x) {
+              const int qp = q0 + r0 + x;
               const uint32_t b0 = __ballot_sync(0xffffffffu, jh[0] >= 0 && jh[0] <= qp && (jh[0] < S || qp - WD < mh[0]));
               const uint32_t b1 = __ballot_sync(0xffffffffu, jh[1] >= 0 && jh[1] <= qp && (jh[1] < S || qp - WD < mh[1]));
-              if (lane == i) { w0 = b0; w1 = b1; }
+              if (lane == x) { w0 = b0; w1 = b1; }
             }
             if (r0 + lane < p.qt) *reinterpret_cast<uint2*>(rm + 2 * (r0 + lane)) = make_uint2(w0, w1);
           }
@@ -766,60 +921,122 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&meta_full[st]);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cand_free[i & 1]);
     }
   } else if (warp >= kT2Mma) {
     // ---------------- MMA issue: one thread per row block ----------------
-    // Per block: S(0), S(1); then per tile, once the softmax has written
-    // P(t) over S(t): O += P V(t), and S(t + 2) into the same buffer (after
-    // P V(t) in issue order).  The blocks do not wait for each other; a stage
-    // is free once both blocks' P V of it completed.
+    // Per block, over the CTA's tiles T of all its items: O += P V(T) once
+    // the softmax has written P(T) over S(T) (accumulating unless T is its
+    // item's first), and S(T) = Q K(T)^T once its K tile, its item's tile
+    // count and Q rows are in and P V(T - 2) has been issued (S(T) reuses
+    // that buffer; one thread's MMAs run in issue order).  The thread polls
+    // all three conditions, so a P V never waits behind the next item's
+    // first S; and it loads the next item's Q rows by TMA as soon as the
+    // current item's last S has completed.  The blocks do not wait for each
+    // other; a stage is free once both blocks' P V of it completed.
     const int XB = warp - kT2Mma;
-    if (lane == 0 && ntiles > 0) {
-      // S_X(t) = Q_X K(t)^T: A = Q_X and B = the K tile, both K-major swizzled in shared memory
-      auto issue_s = [&](int X, int t) {
-        const int st = t % NST;
+    if (lane == 0) {
+      const uint32_t qb = sbase + static_cast<uint32_t>(SM::Q_OFF + XB * SM::QBLK);
+      // Q rows of block XB of item i: per head one box of PB positions x 64 dims per 64-dim group
+      auto load_q = [&](int i) {
+        const T2Item w = t2_item(p, ntq, blockIdx.x + i * gridDim.x);
+        mbar_arrive_expect_tx(&q_full[XB], static_cast<uint32_t>(SM::QBLK));
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int c = 0; c < SM::NGRP; ++c)
+            tma_load_3d(qb + static_cast<uint32_t>(c * SM::QGRP + g * PB * 128), &qmap, 64 * c, w.q0 + XB * PB,
+                        w.b * p.Hq + w.hk * G + g, &q_full[XB]);
+      };
+      // S_X(T) = Q_X K(T)^T: A = Q_X and B = the K tile, both K-major swizzled in shared memory
+      auto issue_s = [&](int T) {
+        const int st = T % NST;
         const uint32_t kb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE);
-        const uint32_t qb = sbase + static_cast<uint32_t>(SM::Q_OFF + X * SM::QBLK);
-        const uint32_t d = tmem + kColS + static_cast<uint32_t>((2 * X + (t & 1)) * kT2Keys);
+        const uint32_t d = tmem + kColS + static_cast<uint32_t>((2 * XB + (T & 1)) * kT2Keys);
         // 16 dims = 32 bytes of a 128-byte swizzled row; 8-row groups 1024 bytes apart
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks)
           tc_mma(d, tc_desc_sw128(qb + static_cast<uint32_t>((ks >> 2) * SM::QGRP + (ks & 3) * 32), 16, 1024),
                  tc_desc_sw128(kb + static_cast<uint32_t>((ks >> 2) * SM::GRP + (ks & 3) * 32), 16, 1024), kIdescS,
                  ks > 0 ? 1u : 0u);
-        tc_commit(&s_full[2 * X + (t & 1)]);
+        tc_commit(&s_full[2 * XB + (T & 1)]);
       };
-      // O_X += P_X(t) V(t): A = P_X(t) in TMEM over S_X(t) (8 columns per 16 keys), B = the V tile
-      auto issue_pv = [&](int X, int t) {
-        const int st = t % NST;
+      // O_X (+)= P_X(T) V(T): A = P_X(T) in TMEM over S_X(T) (8 columns per 16 keys), B = the V tile
+      auto issue_pv = [&](int T, bool first) {
+        const int st = T % NST;
         const uint32_t vb = sbase + static_cast<uint32_t>(SM::KV_OFF + st * SM::STAGE + SM::KV_TILE);
-        const uint32_t d = tmem + static_cast<uint32_t>(X * DH);
-        const uint32_t ap = tmem + kColS + static_cast<uint32_t>((2 * X + (t & 1)) * kT2Keys);
+        const uint32_t d = tmem + static_cast<uint32_t>(XB * DH);
+        const uint32_t ap = tmem + kColS + static_cast<uint32_t>((2 * XB + (T & 1)) * kT2Keys);
         // MN-major B: 64-dim groups GRP bytes apart (leading), 8-key groups 1024 bytes apart (stride);
         // 16 keys per instruction = two 8-key groups
 #pragma unroll
         for (int kk = 0; kk < kT2Keys / 16; ++kk)
           tc_mma_ts(d, ap + 8u * kk, tc_desc_sw128(vb + static_cast<uint32_t>(kk * 2048), SM::GRP, 1024), kIdescPV,
-                    (t > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&o_done[X]);
+                    (!first || kk > 0) ? 1u : 0u);
+        tc_commit(&o_done[XB]);
       };
-      bool ok = wait(q_full, 0);
-      for (int t = 0; ok && t < 2 && t < ntiles; ++t) {
-        ok = wait(&kv_full[t % NST], (t / NST) & 1);
-        if (ok) {
-          tc_fence_after();
-          issue_s(XB, t);
+      // S cursor: item si (tile count snt once known, -1 before), its tile st_; Ts = next S, Tp = next P V
+      int si = 0, st_ = 0, snt = -1, Ts = 0, Tp = 0, q_loaded = 0;
+      uint32_t first_bits = 0u;   // bit T % 4: tile T is its item's first
+      bool more = true;
+      load_q(0);
+      uint64_t idle_since = 0;
+      while (more || Tp < Ts) {
+        bool prog = false;
+        // the next item's Q, once the item before's last S has read Q
+        if (more && q_loaded < si && mbar_test(&q_free[XB], (si - 1) & 1)) {
+          load_q(si);
+          q_loaded = si;
+          prog = true;
         }
-      }
-      for (int t = 0; ok && t < ntiles; ++t) {
-        ok = wait(&p_full[2 * XB + (t & 1)], (t >> 1) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(XB, t);
-        tc_commit(&kv_free[t % NST]);
-        if (t + 2 < ntiles) {
-          ok = wait(&kv_full[(t + 2) % NST], ((t + 2) / NST) & 1);
-          if (ok) issue_s(XB, t + 2);
+        // with no S waiting for its inputs, the thread suspends on the next P
+        // (up to ~200 ns a time) instead of spinning on the softmax warps' issue slots
+        const bool s_waits = more && Ts < Tp + 2;
+        if (Tp < Ts && (s_waits ? mbar_test(&p_full[2 * XB + (Tp & 1)], (Tp >> 1) & 1)
+                                : mbar_try_wait_ns(&p_full[2 * XB + (Tp & 1)], (Tp >> 1) & 1, 200u))) {
+          tc_fence_after();
+          issue_pv(Tp, ((first_bits >> (Tp & 3)) & 1u) != 0u);
+          tc_commit(&kv_free[Tp % NST]);
+          ++Tp;
+          prog = true;
+        }
+        if (more && Ts < Tp + 2) {
+          bool ready = true;
+          if (snt < 0) {
+            ready = mbar_test(&item_full[si % kT2Ring], (si / kT2Ring) & 1);
+            if (ready) {
+              snt = ntiles_of(count_ring[si % kT2Ring]);
+              st_ = 0;
+            }
+          }
+          if (ready && st_ == 0) ready = q_loaded == si && mbar_test(&q_full[XB], si & 1);
+          if (ready && mbar_test(&kv_full[Ts % NST], (Ts / NST) & 1)) {
+            tc_fence_after();
+            issue_s(Ts);
+            first_bits = (first_bits & ~(1u << (Ts & 3))) | ((st_ == 0 ? 1u : 0u) << (Ts & 3));
+            ++Ts;
+            if (++st_ == snt) {
+              tc_commit(&q_free[XB]);   // completes once this item's S MMAs have read Q
+              ++si;
+              snt = -1;
+              more = static_cast<int>(blockIdx.x) + si * static_cast<int>(gridDim.x) < nitems;
+            }
+            prog = true;
+          }
+        }
+        if (prog) {
+          idle_since = 0;
+        } else {
+          if (*abort_flag) break;
+          const uint64_t now = global_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs) {
+            set_error(p.err, DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+          if (s_waits || Tp == Ts) __nanosleep(32);   // otherwise the P wait above suspended
         }
       }
     }
@@ -828,111 +1045,128 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
     // ---------------- softmax: block X, thread = row = TMEM lane ----------------
     const int X = warp >> 2;
     const int row = tid & 127;
-    const int grow = X * 128 + row;
-    const int posoff = grow / G;
-    const int qpos = q0 + posoff;
-    const bool vrow = qpos < q1;
+    const int g = row / PB;
+    const int posoff = X * PB + row % PB;
     const uint32_t lrow = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + static_cast<uint32_t>(X * DH);
-    float m_run = -INFINITY, l_run = 0.f;
+    const bool out32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0u;   // output rows 32-byte aligned
+    int T = 0;
     bool ok = true;
-    for (int t = 0; t < ntiles; ++t) {
-      const int st = t % NST;
-      bool got = wait(&meta_full[st], (t / NST) & 1);
-      got = got && wait(&s_full[2 * X + (t & 1)], (t >> 1) & 1);
-      if (!__all_sync(0xffffffffu, got)) {   // the TMEM loads below are warp-collective
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // S(t) row: 64 fp32 columns of buffer t & 1
-      const uint32_t tS = tmem + kColS + static_cast<uint32_t>((2 * X + (t & 1)) * kT2Keys);
-      float sv[kT2Keys];
-      {
-        float lo[32], hi[32];
-        tc_ld32(tS + lrow, lo);
-        tc_ld32(tS + 32u + lrow, hi);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { sv[i] = lo[i]; sv[32 + i] = hi[i]; }
-      }
-      // mask on the raw logits; the tile max commutes with the positive scale,
-      // so each weight is one FMA and one ex2: p = 2^(s * scale - m)
-      const uint32_t* rmk = reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS);
-      uint32_t vm0 = 0u, vm1 = 0u;
-      if (vrow) {
-        const bool full = rmk[2 * kT2Rows] != 0u;
-        vm0 = full ? 0xffffffffu : rmk[2 * posoff];
-        vm1 = full ? 0xffffffffu : rmk[2 * posoff + 1];
-      }
-      float tmax = -INFINITY;
-      if (!__all_sync(0xffffffffu, (vm0 & vm1) == 0xffffffffu)) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = ((vm0 >> i) & 1u) ? sv[i] : -INFINITY;
-          sv[32 + i] = ((vm1 >> i) & 1u) ? sv[32 + i] : -INFINITY;
-        }
-      }
-      {
-        // four independent max chains, then their max
-        float m4[4] = {sv[0], sv[1], sv[2], sv[3]};
-#pragma unroll
-        for (int i = 4; i < kT2Keys; ++i) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
-        tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      }
-      const float tm = tmax * p.scale_log2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (tm > m_run + kT2Lazy) {
-        resc = (m_run != -INFINITY);
-        alpha = resc ? ex2_approx(m_run - tm) : 0.f;
-        l_run *= alpha;
-        m_run = tm;
-      }
-      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;   // masked logits give 2^-inf = 0
-      // P(t) in bf16 over the first 32 columns of S(t), 16 columns at a time
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
-#pragma unroll
-      for (int h = 0; h < kT2Keys / 32; ++h) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float x0 = fmaf(sv[32 * h + i], p.scale_log2, nm), x1 = fmaf(sv[32 * h + i + 1], p.scale_log2, nm);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          ps[(i >> 1) & 3] += p0 + p1;
-          pk[i / 2] = pack_bf16(p0, p1);
-        }
-        tc_st16u(tS + static_cast<uint32_t>(16 * h) + lrow, pk);
-      }
-      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      if (__any_sync(0xffffffffu, resc)) {
-        // rescale this row of O once the P V before (of tile t - 1) has completed
-        const bool done = t == 0 || wait(&o_done[X], (t - 1) & 1);
-        if (!__all_sync(0xffffffffu, done)) {
+    for (int i = 0; ok; ++i) {
+      const int it = blockIdx.x + i * gridDim.x;
+      if (it >= nitems) break;
+      if (!__all_sync(0xffffffffu, wait(&item_full[i % kT2Ring], (i / kT2Ring) & 1))) break;
+      const T2Item w = t2_item(p, ntq, it);
+      const int nt = ntiles_of(count_ring[i % kT2Ring]);
+      const int qpos = w.q0 + posoff;
+      const bool vrow = qpos < w.q1;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int t = 0; t < nt; ++t, ++T) {
+        const int st = T % NST;
+        bool got = wait(&meta_full[st], (T / NST) & 1);
+        got = got && wait(&s_full[2 * X + (T & 1)], (T >> 1) & 1);
+        if (!__all_sync(0xffffffffu, got)) {   // the TMEM loads below are warp-collective
           ok = false;
           break;
         }
         tc_fence_after();
-        const float f = resc ? alpha : 1.f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < DH; c0 += 32) {
-          float o[32];
-          tc_ld32(tO + lrow + c0, o);
+        // S(T) row: 64 fp32 columns of buffer T & 1
+        const uint32_t tS = tmem + kColS + static_cast<uint32_t>((2 * X + (T & 1)) * kT2Keys);
+        float sv[kT2Keys];
+        {
+          float lo[32], hi[32];
+          tc_ld32(tS + lrow, lo);
+          tc_ld32(tS + 32u + lrow, hi);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= f;
-          tc_st32(tO + lrow + c0, o);
+          for (int x = 0; x < 32; ++x) { sv[x] = lo[x]; sv[32 + x] = hi[x]; }
         }
+        // mask on the raw logits; the tile max commutes with the positive scale,
+        // so each weight is one FMA and one ex2: p = 2^(s * scale - m)
+        const uint32_t* rmk = reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS);
+        uint32_t vm0 = 0u, vm1 = 0u;
+        if (vrow) {
+          const bool full = rmk[2 * kT2Rows] != 0u;
+          vm0 = full ? 0xffffffffu : rmk[2 * posoff];
+          vm1 = full ? 0xffffffffu : rmk[2 * posoff + 1];
+        }
+        float tmax = -INFINITY;
+        if (!__all_sync(0xffffffffu, (vm0 & vm1) == 0xffffffffu)) {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            sv[x] = ((vm0 >> x) & 1u) ? sv[x] : -INFINITY;
+            sv[32 + x] = ((vm1 >> x) & 1u) ? sv[32 + x] : -INFINITY;
+          }
+        }
+        {
+          // four independent max chains, then their max
+          float m4[4] = {sv[0], sv[1], sv[2], sv[3]};
+#pragma unroll
+          for (int x = 4; x < kT2Keys; ++x) m4[x & 3] = fmaxf(m4[x & 3], sv[x]);
+          tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        }
+        const float tm = tmax * p.scale_log2;
+        float alpha = 1.f;
+        bool resc = false;
+        if (tm > m_run + kT2Lazy) {
+          resc = (m_run != -INFINITY);
+          alpha = resc ? ex2_approx(m_run - tm) : 0.f;
+          l_run *= alpha;
+          m_run = tm;
+        }
+        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;   // masked logits give 2^-inf = 0
+        // P(T) in bf16 over the first 32 columns of S(T), 16 columns at a time
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
+#pragma unroll
+        for (int h = 0; h < kT2Keys / 32; ++h) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            const float x0 = fmaf(sv[32 * h + x], p.scale_log2, nm), x1 = fmaf(sv[32 * h + x + 1], p.scale_log2, nm);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            ps[(x >> 1) & 3] += p0 + p1;
+            pk[x / 2] = pack_bf16(p0, p1);
+          }
+          tc_st16u(tS + static_cast<uint32_t>(16 * h) + lrow, pk);
+        }
+        l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        if (__any_sync(0xffffffffu, resc)) {
+          // rescale this row of O once the P V before (of tile T - 1, same item: t > 0) has completed
+          const bool done = wait(&o_done[X], (T - 1) & 1);
+          if (!__all_sync(0xffffffffu, done)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = resc ? alpha : 1.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < DH; c0 += 32) {
+            float o[32];
+            tc_ld32(tO + lrow + c0, o);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] *= f;
+            tc_st32(tO + lrow + c0, o);
+          }
+        }
+        // A parity wait on o_done (one phase per P V) is exact only while at
+        // most one phase separates it from the barrier's: here P V(T - 2) has
+        // completed (S(T) was issued after it) and P V(T) waits for this
+        // arrival.  So the item's last tile waits here for P V(T - 1), and the
+        // epilogue then waits for P V(T) alone.
+        if (t == nt - 1 && t > 0 && !__all_sync(0xffffffffu, wait(&o_done[X], (T - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(&p_full[2 * X + (T & 1)]);
       }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(&p_full[2 * X + (t & 1)]);
-    }
-    bool fin = ok && ntiles > 0;
-    if (fin) fin = wait(&o_done[X], (ntiles - 1) & 1);
-    if (__all_sync(0xffffffffu, fin)) {
+      if (!ok) break;
+      // epilogue: O of this row once the item's last P V (tile T - 1) has completed; the
+      // next item's first P V overwrites O only after this thread's next p_full arrival
+      if (!__all_sync(0xffffffffu, wait(&o_done[X], (T - 1) & 1))) break;
       tc_fence_after();
-      const int g = grow % G;
-      const size_t rowi = (static_cast<size_t>(b) * p.Hq + hk * G + g) * n + (vrow ? qpos : 0);
+      const size_t rowi = (static_cast<size_t>(w.b) * p.Hq + w.hk * G + g) * n + (vrow ? qpos : 0);
       __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out) + rowi * DH;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
@@ -940,16 +1174,21 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
         float o[32];
         tc_ld32(tO + lrow + c0, o);
         if (vrow) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(og + c0 + 8 * c) =
-                make_uint4(pack_bf16(o[8 * c] * inv, o[8 * c + 1] * inv),
-                           pack_bf16(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
-                           pack_bf16(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
-                           pack_bf16(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(o[2 * c] * inv, o[2 * c + 1] * inv);
+          if (out32) {   // one full 32-byte sector per store
+#pragma unroll
+            for (int c = 0; c < 2; ++c) st_global_v8(og + c0 + 16 * c, pk + 8 * c);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(og + c0 + 8 * c) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
         }
       }
       if (vrow && p.lse != nullptr) p.lse[rowi] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      tc_fence_before();
     }
   }
   tc_fence_before();
@@ -960,25 +1199,48 @@ sparse_attn_tc2_kernel(const __grid_constant__ PaArgs p) {
   }
 }
 
+// One CTA per SM (at most one per work item); Q through a 3-D tensor map
+// (head dim, position, batch row x query head) with one box per head and
+// 64-dim group.
 template <int DH, int NST>
-int launch_attn_tc2_stages(const PaArgs& pa, int units, int n, size_t smem, cudaStream_t st) {
-  if (cudaFuncSetAttribute(sparse_attn_tc2_kernel<DH, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+int launch_attn_tcp_stages(const PaArgs& pa, int units, int n, size_t smem, cudaStream_t st) {
+  if (cudaFuncSetAttribute(sparse_attn_tcp_kernel<DH, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return -1;
-  dim3 grid((n + pa.qt - 1) / pa.qt, units);
-  sparse_attn_tc2_kernel<DH, NST><<<grid, kT2Threads, smem, st>>>(pa);
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return -1;
+  const int B = units / pa.Hkv;
+  CUtensorMap qmap;
+  const cuuint64_t gdim[3] = {static_cast<cuuint64_t>(DH), static_cast<cuuint64_t>(n),
+                              static_cast<cuuint64_t>(B) * pa.Hq};
+  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(DH) * 2, static_cast<cuuint64_t>(n) * DH * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(128 / pa.G), 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  if (encode(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pa.q), gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return -1;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+    return -1;
+  const int64_t nitems = static_cast<int64_t>(units) * ((n + pa.qt - 1) / pa.qt);
+  if (nitems > (1ll << 30)) return -2;
+  const int grid = static_cast<int>(nitems < nsm ? nitems : nsm);
+  sparse_attn_tcp_kernel<DH, NST><<<grid, kT2Threads, smem, st>>>(qmap, pa, static_cast<int>(nitems));
   return 0;
 }
 
 // Four stages when they fit in shared memory beside the candidate lists, else three.
 template <int DH>
-int launch_attn_tc2(const PaArgs& pa, int units, int n, cudaStream_t st) {
+int launch_attn_tcp(const PaArgs& pa, int units, int n, cudaStream_t st) {
   constexpr size_t kMax = 227 * 1024;
   if (units == 0 || n == 0) return 0;
+  if (pa.G > 16 || 128 % pa.G != 0) return -2;   // one TMA box of at least 8 rows per head
   const size_t smem4 = T2Smem<DH, 4>::bytes(pa.cand_cap);
-  if (smem4 <= kMax) return launch_attn_tc2_stages<DH, 4>(pa, units, n, smem4, st);
+  if (smem4 <= kMax) return launch_attn_tcp_stages<DH, 4>(pa, units, n, smem4, st);
   const size_t smem3 = T2Smem<DH, 3>::bytes(pa.cand_cap);
-  if (smem3 <= kMax) return launch_attn_tc2_stages<DH, 3>(pa, units, n, smem3, st);
+  if (smem3 <= kMax) return launch_attn_tcp_stages<DH, 3>(pa, units, n, smem3, st);
   return -2;
 }
 
@@ -1055,6 +1317,7 @@ int launch_place_kept(const LayerArgs& a, int dtype, const PrefillAttnPlan& p, c
 
 int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan* p) {
   if (n < 0 || kPaRows % a.G != 0) return -2;
+  if (dtype != 0 && a.G > 16) return -2;   // bf16: each head's rows of a row block are one TMA box of >= 8 rows (a cache has G <= 8)
   if (a.mlstm) return -2;   // the prompt scores come from the stateless scorers or the caller
   if (a.d != 64 && a.d != 128) return -2;
   PrefillAttnPlan P{};
@@ -1129,7 +1392,7 @@ int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPla
   if (dtype == 0)
     r = (a.d == 128) ? launch_attn_f32<128>(pa, a.units, p.n, st) : launch_attn_f32<64>(pa, a.units, p.n, st);
   else
-    r = (a.d == 128) ? launch_attn_tc2<128>(pa, a.units, p.n, st) : launch_attn_tc2<64>(pa, a.units, p.n, st);
+    r = (a.d == 128) ? launch_attn_tcp<128>(pa, a.units, p.n, st) : launch_attn_tcp<64>(pa, a.units, p.n, st);
   if (r != 0) return r;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -29,8 +29,9 @@ class PaRun:
 
 
 def run_prefill_attention(w, n, *, external=False, tie_levels=0, log_decay=None, layer=0, master=0,
-                          gen_device="cpu", with_lse=True):
-    """One prefill-attention call for `layer` of a one-layer-per-call cache."""
+                          gen_device="cpu", with_lse=True, out_offset=0):
+    """One prefill-attention call for `layer` of a one-layer-per-call cache
+    (out_offset: the output starts that many elements into its allocation)."""
     import fixed_budget_kv_kvpop_b200 as kp
     n_layers = layer + 1
     weights = None
@@ -45,7 +46,7 @@ def run_prefill_attention(w, n, *, external=False, tie_levels=0, log_decay=None,
     ext = None
     if external:
         ext = wl.external_scores(w, layer, n, master=master, device=gen_device, tie_levels=tie_levels).cuda()
-    out = torch.full_like(q, float("nan"))
+    out = torch.full((q.numel() + out_offset,), float("nan"), dtype=q.dtype, device="cuda")[out_offset:].view(q.shape)
     lse = torch.full((w.batch, w.n_q_heads, n), float("nan"), device="cuda") if with_lse else None
     ws = torch.empty(cache.prefill_attention_workspace_bytes(n), dtype=torch.uint8, device="cuda")
     cache.prefill_attention(layer, q, k, v, out, lse, ws, ext)
@@ -138,6 +139,16 @@ def test_gpu_scorer(dtype, d, hq, hkv, S, W, D, K, hidden, n):
     _need_gpu()
     w = _case(dtype, d, hq, hkv, S=S, W=W, D=D, K=K, hidden=hidden, batch=2)
     r = run_prefill_attention(w, n)
+    check_all_rows(r)
+
+
+def test_output_rows_16_byte_aligned():
+    """An output buffer that is 16- but not 32-byte aligned (the tensor-core
+    kernel then writes 16 bytes per store instead of 32): same parity."""
+    _need_gpu()
+    w = _case("bf16", 128, 8, 2, S=4, W=16, D=0, K=40, hidden=64, batch=2)
+    r = run_prefill_attention(w, 333, out_offset=8)
+    assert r.out.data_ptr() % 32 == 16
     check_all_rows(r)
 
 
