@@ -539,6 +539,32 @@ __device__ __forceinline__ void tc_st16u(uint32_t taddr, const uint32_t (&v)[16]
 // mbarrier that a role may wait on twice in a row without an intervening
 // handoff is per buffer, so parity waits never alias.
 
+// 64 consecutive fp32 columns of this thread's TMEM lane in one load, waited
+// for inside the same statement (warp-collective).
+__device__ __forceinline__ void tc_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+      "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, "
+      "%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, "
+      "%34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, "
+      "%50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63"
+      "}, [%64];\n"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 constexpr int kT2Rows = 256;
 // Lazy rescale threshold (log2 units): the running max of a row moves only
 // when a tile's max exceeds it by 2^20.  A rescale of O waits for the P V in
@@ -638,18 +664,26 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 
 // The candidates of one work item (the keys gather_candidates lists, in the
-// same ascending order), computed by the 128 copy
-// threads (ptid 0..127) alone, synchronised by named barrier kT2CopyBar.
-// Each warp scans 32 x R consecutive cutoffs per round with coalesced loads
-// (lane i reads position base + 32 r + i), ballots the kept ones and places
-// them after the earlier warps' (one scan over the four warp totals per
-// round of 128 x R positions).  Returns the count (at most cap).
-__device__ __forceinline__ int gather_candidates_copy(int* cand, int* wtot, const int32_t* cu, int S, int m0, int q1,
-                                                      int cap, int ptid) {
+// same ascending order), computed by the 128 copy threads (ptid 0..127)
+// alone, synchronised by named barrier kT2CopyBar.  Each warp scans 32 x R
+// consecutive cutoffs per round with coalesced loads (lane i reads position
+// base + 32 r + i), ballots the kept ones and places them after the earlier
+// warps' (one scan over the four warp totals per round of 128 x R
+// positions).  Entry: the position j, or, with `packed` (prompts of at most
+// 65,535 tokens), j | min(max(j, c_j), 65535) << 16, so that the mask needs
+// no cutoff load (positions and query indices stay below 65,535, so the
+// clamp never changes q - W - D < max(j, c_j)).  Returns the count (at most
+// cap).
+__device__ __forceinline__ uint32_t cand_entry(int j, int c, bool packed) {
+  return packed ? static_cast<uint32_t>(j) | (static_cast<uint32_t>(min(max(j, c), 65535)) << 16)
+                : static_cast<uint32_t>(j);
+}
+__device__ __forceinline__ int gather_candidates_copy(uint32_t* cand, int* wtot, const int32_t* cu, int S, int m0,
+                                                      int q1, int cap, int ptid, bool packed) {
   constexpr int NT = 128, R = 16;
   const int lane = ptid & 31, w = ptid >> 5;
   const int ns = min(S, q1);
-  for (int i = ptid; i < ns; i += NT) cand[i] = i;
+  for (int i = ptid; i < ns; i += NT) cand[i] = cand_entry(i, 0, packed);
   int count = ns;
   const uint32_t lt = (1u << lane) - 1u;
   for (int base = S; base <= m0; base += NT * R) {
@@ -681,7 +715,7 @@ __device__ __forceinline__ int gather_candidates_copy(int* cand, int* wtot, cons
     for (int r = 0; r < R; ++r) {
       if ((bal[r] >> lane) & 1u) {
         const int o = off + __popc(bal[r] & lt);
-        if (o < cap) cand[o] = wb + 32 * r + lane;
+        if (o < cap) cand[o] = cand_entry(wb + 32 * r + lane, c[r], packed);
       }
       off += __popc(bal[r]);
     }
@@ -691,7 +725,7 @@ __device__ __forceinline__ int gather_candidates_copy(int* cand, int* wtot, cons
   const int r0 = max(S, m0 + 1);
   const int nr = max(0, q1 - r0);
   for (int i = ptid; i < nr; i += NT)
-    if (count + i < cap) cand[count + i] = r0 + i;
+    if (count + i < cap) cand[count + i] = cand_entry(r0 + i, packed ? cu[r0 + i] : 0, packed);
   count += nr;
   named_bar_sync(kT2CopyBar, NT);
   return min(count, cap);   // count <= cap always: S + K + qt + W + D bounds it
@@ -740,12 +774,13 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
   volatile int* abort_flag = misc + 1;
   int* count_ring = misc + 2;                     // [item % ring] candidate count of the item
   int* wtot = misc + 2 + kT2Ring;                 // copy warps' totals (gather scan)
-  int* cand2 = reinterpret_cast<int*>(smem_t2 + SM::CAND_OFF);   // item i's candidates at cand2 + (i & 1) * cand_cap
+  uint32_t* cand2 = reinterpret_cast<uint32_t*>(smem_t2 + SM::CAND_OFF);   // item i's candidates at cand2 + (i & 1) * cand_cap
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = p.n, S = p.S, WD = p.W + p.D, G = p.G;
   const int ntq = (n + p.qt - 1) / p.qt;
   const int PB = 128 / G;                          // query positions per row block
+  const bool packed = n <= 65535;                  // candidate entries carry max(j, c_j) (cand_entry)
   const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k);
   const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(p.v);
 
@@ -805,7 +840,7 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
     auto gather = [&](int i) {   // item i's candidates into its buffer; count to the ring
       const T2Item w = t2_item(p, ntq, blockIdx.x + i * gridDim.x);
       const int count = gather_candidates_copy(cand2 + (i & 1) * p.cand_cap, wtot, p.cut + static_cast<size_t>(w.u) * n,
-                                               S, w.q0 - WD, w.q1, p.cand_cap, ptid);
+                                               S, w.q0 - WD, w.q1, p.cand_cap, ptid, packed);
       if (ptid == 0) {
         count_ring[i % kT2Ring] = count;
         mbar_arrive(&item_full[i % kT2Ring]);
@@ -819,7 +854,7 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
       if (it >= nitems) break;
       const T2Item w = t2_item(p, ntq, it);
       const bool has_next = it + static_cast<int>(gridDim.x) < nitems;
-      const int* cand = cand2 + (i & 1) * p.cand_cap;
+      const uint32_t* cand = cand2 + (i & 1) * p.cand_cap;
       const int count = next_count;
       const int nt = ntiles_of(count);
       const int gat = min(NST, nt);
@@ -851,7 +886,7 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
         for (int x = ptid; x < kT2Keys * CPR; x += 128) {
           const int key = x / CPR, c = x % CPR;
           const int kidx = t * kT2Keys + key;
-          const int jj = kidx < count ? cand[kidx] : -1;
+          const int jj = kidx < count ? static_cast<int>(packed ? cand[kidx] & 0xffffu : cand[kidx]) : -1;
           const size_t off = jj >= 0 ? static_cast<size_t>(jj) * DH + c * 8 : 0;
           const uint32_t so = static_cast<uint32_t>((c >> 3) * SM::GRP + (key >> 3) * 1024 + (key & 7) * 128 +
                                                     (((c & 7) ^ (key & 7)) << 4));
@@ -876,46 +911,65 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
       const int q0 = w.q0, q1 = w.q1;
       const int count = count_ring[i % kT2Ring];
       const int nt = ntiles_of(count);
-      const int* cand = cand2 + (i & 1) * p.cand_cap;
+      const uint32_t* cand = cand2 + (i & 1) * p.cand_cap;
       const int32_t* cu = p.cut + static_cast<size_t>(w.u) * n;
+      // lane's keys 32 h + lane of tile t: position (-1 past the candidates) and max(position, cutoff)
+      auto load_keys = [&](int t, int (&jj)[2], int (&mm)[2]) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int idx = t * kT2Keys + 32 * h + lane;
+          const uint32_t e = idx < count ? cand[idx] : 0xffffffffu;
+          jj[h] = idx < count ? static_cast<int>(packed ? e & 0xffffu : e) : -1;
+          mm[h] = jj[h] < 0 ? 0 : packed ? static_cast<int>(e >> 16) : max(jj[h], cu[jj[h]]);
+        }
+      };
+      int jn[2], mn[2];   // the next tile's keys, loaded one tile ahead (long prompts read the cutoffs from global memory)
+      load_keys(0, jn, mn);
       for (int t = 0; t < nt; ++t, ++T) {
         const int st = T % NST;
         if (!__all_sync(0xffffffffu, T < NST || wait(&kv_free[st], ((T / NST) - 1) & 1))) {
           ok = false;
           break;
         }
+        const int jh[2] = {jn[0], jn[1]}, mh[2] = {mn[0], mn[1]};
+        if (t + 1 < nt) load_keys(t + 1, jn, mn);
         // The tile's mask (§C.1) as two 32-bit words per query position of
-        // the item (bit i of word h = key 32 h + i visible): lane i of each
-        // mask warp holds keys i and 32 + i, and one ballot per word collects
-        // the bits.  Key j (cutoff c) is visible at position q iff j <= q and
-        // (j is a sink or q - W - D < max(j, c)).  A tile whose keys are all
-        // visible to every position of the item (the common case: long-range
-        // keys kept past the item's last position) is only flagged.
+        // the item (bit i of word h = key 32 h + i visible).  Key j (cutoff c)
+        // is visible at position q iff j <= q and (j is a sink or
+        // q - W - D < max(j, c)): an interval of positions starting at j.
+        // Lane i holds keys i and 32 + i; one ballot per word finds the keys
+        // visible to every position of the item (the base words) and one the
+        // others (exceptions: keys evicted or admitted inside the item's
+        // range).  A tile without exceptions is only flagged; otherwise lane i
+        // builds the words of position 32 g + i from the base words and a
+        // test of each exception key's interval (broadcast by shuffles).
         uint32_t* rm = reinterpret_cast<uint32_t*>(meta + st * SM::META_INTS);
-        int jh[2], mh[2];
-        bool always = true;
+        int lo[2], lim[2];
+        uint32_t base[2], exc[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int idx = t * kT2Keys + 32 * h + lane;
-          jh[h] = idx < count ? cand[idx] : -1;
-          mh[h] = jh[h] >= 0 ? max(jh[h], cu[jh[h]]) : 0;
-          always = always && jh[h] >= 0 && jh[h] <= q0 && (jh[h] < S || q1 - 1 - WD < mh[h]);
+          lo[h] = jh[h] >= 0 ? jh[h] : INT_MAX;              // past the candidates: never visible
+          lim[h] = jh[h] < S ? INT_MAX : mh[h];              // visible while q - W - D < lim
+          const bool always = lo[h] <= q0 && q1 - 1 - WD < lim[h];
+          base[h] = __ballot_sync(0xffffffffu, always);
+          exc[h] = __ballot_sync(0xffffffffu, jh[h] >= 0 && !always);
         }
-        const bool full_tile = __all_sync(0xffffffffu, always);
+        const bool full_tile = (base[0] & base[1]) == 0xffffffffu;
         if (mw == 0 && lane == 0) rm[2 * kT2Rows] = full_tile ? 1u : 0u;
         if (!full_tile) {
-          // positions in groups of 32, alternating between the two mask warps;
-          // lane i keeps position 32 g + i's two words and stores them once
+          // positions in groups of 32, alternating between the two mask warps
           for (int r0 = 32 * mw; r0 < p.qt; r0 += 32 * (kT2Mma - kT2Mask)) {
-            uint32_t w0 = 0u, w1 = 0u;
-#pragma unroll 4
-            for (int x = 0; x < 32; ++x) {
-              const int qp = q0 + r0 + x;
-              const uint32_t b0 = __ballot_sync(0xffffffffu, jh[0] >= 0 && jh[0] <= qp && (jh[0] < S || qp - WD < mh[0]));
-              const uint32_t b1 = __ballot_sync(0xffffffffu, jh[1] >= 0 && jh[1] <= qp && (jh[1] < S || qp - WD < mh[1]));
-              if (lane == x) { w0 = b0; w1 = b1; }
-            }
-            if (r0 + lane < p.qt) *reinterpret_cast<uint2*>(rm + 2 * (r0 + lane)) = make_uint2(w0, w1);
+            const int qp = q0 + r0 + lane;
+            uint32_t wd[2] = {base[0], base[1]};
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              for (uint32_t m = exc[h]; m != 0u; m &= m - 1u) {
+                const int e = __ffs(m) - 1;
+                const int l = __shfl_sync(0xffffffffu, lo[h], e);
+                const int L = __shfl_sync(0xffffffffu, lim[h], e);
+                if (l <= qp && qp - WD < L) wd[h] |= 1u << e;
+              }
+            if (r0 + lane < p.qt) *reinterpret_cast<uint2*>(rm + 2 * (r0 + lane)) = make_uint2(wd[0], wd[1]);
           }
         }
         __syncwarp();
@@ -1072,14 +1126,9 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
         tc_fence_after();
         // S(T) row: 64 fp32 columns of buffer T & 1
         const uint32_t tS = tmem + kColS + static_cast<uint32_t>((2 * X + (T & 1)) * kT2Keys);
+        static_assert(kT2Keys == 64, "one 64-column TMEM load per tile");
         float sv[kT2Keys];
-        {
-          float lo[32], hi[32];
-          tc_ld32(tS + lrow, lo);
-          tc_ld32(tS + 32u + lrow, hi);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) { sv[x] = lo[x]; sv[32 + x] = hi[x]; }
-        }
+        tc_ld64(tS + lrow, sv);
         // mask on the raw logits; the tile max commutes with the positive scale,
         // so each weight is one FMA and one ex2: p = 2^(s * scale - m)
         const uint32_t* rmk = reinterpret_cast<const uint32_t*>(meta + st * SM::META_INTS);

@@ -314,6 +314,24 @@ def test_cutoffs_with_the_bitmap_in_the_workspace():
     assert torch.isfinite(r.out).all()
 
 
+def test_bf16_prompt_above_65535_tokens():
+    """A bf16 prompt of 66,236 tokens (one unit, G 4, d 128, S 4 + W 16 + D 2 +
+    K 300): past 65,535 positions the tensor-core kernel keeps plain positions
+    in its candidate lists and reads the cutoffs for the mask from global
+    memory.  Cutoffs against the Fenwick tree and the running top-k at sampled
+    positions, and sampled output rows."""
+    _need_gpu()
+    w = _case("bf16", 128, 4, 1, S=4, W=16, D=2, K=300, hidden=64)
+    n = 65536 + 700
+    r = run_prefill_attention(w, n, gen_device="cuda")
+    rng = np.random.default_rng(5)
+    m_last = n - 1 - w.window - w.delay
+    ms = sorted(set([w.sinks, w.sinks + w.topk, 65600, m_last] + list(rng.integers(w.sinks, m_last + 1, 3))))
+    rows = sorted(set([0, 65534, 65535, 65536, n - 1] + list(rng.integers(0, n, 5))))
+    _check_large_unit(r, 0, ms, rows, gh.BF16_ATOL)
+    assert torch.isfinite(r.out).all()
+
+
 def test_full_size_8b_delayed_shape_sampled_rows():
     """The Qwen3-8B delayed-scoring shape at full size (32 rows x 8 KV heads,
     prompt 32768, S 4 + W 256 + D 32 + K 3836, G 4, bf16, MLP scorer): 32,476
