@@ -471,6 +471,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 // Shared-memory matrix descriptor, 128-byte swizzle (atoms of 8 rows x 128
 // bytes, 1024-byte aligned; start, leading and stride byte offsets in 16-byte
 // units; descriptor version 1, layout type 2).  K-major: stride offset =
@@ -602,9 +608,10 @@ struct T2Smem {
   static constexpr size_t BAR_OFF = META_OFF + sizeof(int) * NST * META_INTS;
   static constexpr int NBAR = 3 * NST + 4 + 4 + 2 + 2 + 2 + kT2Ring + 2;
   static constexpr size_t MISC_OFF = BAR_OFF + 8 * NBAR;                        // TMEM address, abort flag, tile-count ring, warp totals
-  static constexpr size_t CAND_OFF = MISC_OFF + 64;                             // [item % 2][cand_cap] positions
+  static constexpr size_t EXC_OFF = MISC_OFF + 128;                             // gather scratch: the item's evicted long-range keys
+  static constexpr size_t CAND_OFF = EXC_OFF + sizeof(int) * kT2Rows;           // [item % 2][cand_cap] positions
   static_assert(BAR_OFF % 8 == 0 && STAGE % 1024 == 0 && KV_OFF % 1024 == 0 && META_OFF % 16 == 0 &&
-                    2 + kT2Ring + 4 <= 16,
+                    2 + kT2Ring + 8 <= 32,
                 "shared-memory layout");
   // at least 116 KB: one CTA per SM, which then holds all 512 TMEM columns
   static size_t bytes(int cand_cap) {
@@ -613,6 +620,25 @@ struct T2Smem {
   }
 };
 
+// 32 x 32 bit-matrix transpose across a warp: lane i holds row i (bit j =
+// column j) on entry and column i (bit j = row j) on return.  Five rounds
+// swap off-diagonal blocks of 16, 8, 4, 2 and 1 between lanes i and i ^ k.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+  constexpr uint32_t kMask[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    const int k = 16 >> s;
+    const uint32_t m = kMask[s];
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, k);
+    x = (lane & k) ? ((x & ~m) | ((y >> k) & m)) : ((x & m) | ((y << k) & ~m));
+  }
+  return x;
+}
+// Bits a..b (inclusive) of a 32-bit word, clipped to 0..31; 0 when empty.
+__device__ __forceinline__ uint32_t bit_range32(int a, int b) {
+  if (a > b || a > 31 || b < 0) return 0u;
+  return (0xffffffffu >> (31 - min(b, 31))) & (0xffffffffu << max(a, 0));
+}
 // Named barrier over `nthreads` threads (whole warps); the second form
 // returns whether any participating thread passed true.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -663,28 +689,31 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// The candidates of one work item (the keys gather_candidates lists, in the
-// same ascending order), computed by the 128 copy threads (ptid 0..127)
-// alone, synchronised by named barrier kT2CopyBar.  Each warp scans 32 x R
-// consecutive cutoffs per round with coalesced loads (lane i reads position
-// base + 32 r + i), ballots the kept ones and places them after the earlier
-// warps' (one scan over the four warp totals per round of 128 x R
-// positions).  Entry: the position j, or, with `packed` (prompts of at most
-// 65,535 tokens), j | min(max(j, c_j), 65535) << 16, so that the mask needs
-// no cutoff load (positions and query indices stay below 65,535, so the
-// clamp never changes q - W - D < max(j, c_j)).  Returns the count (at most
-// cap).
+// The candidates of one work item (the keys gather_candidates lists),
+// computed by the 128 copy threads (ptid 0..127) alone, synchronised by
+// named barrier kT2CopyBar, in the order: sinks, the long-range keys still
+// kept at the item's last query (visible to all its positions), the ones
+// evicted inside the item's range (at most one per position, kept in `exc`
+// until the scan ends), then the recent block; so that only the last few
+// tiles of an item need a mask.  Each warp scans 32 x R consecutive cutoffs
+// per round with coalesced loads (lane i reads position base + 32 r + i),
+// ballots the kept ones and places them after the earlier warps' (one scan
+// over the four warps' two totals per round of 128 x R positions).  Entry:
+// the position j, or, with `packed` (prompts of at most 65,535 tokens),
+// j | min(max(j, c_j), 65535) << 16, so that the mask needs no cutoff load
+// (positions and query indices stay below 65,535, so the clamp never changes
+// q - W - D < max(j, c_j)).  Returns the count (at most cap).
 __device__ __forceinline__ uint32_t cand_entry(int j, int c, bool packed) {
   return packed ? static_cast<uint32_t>(j) | (static_cast<uint32_t>(min(max(j, c), 65535)) << 16)
                 : static_cast<uint32_t>(j);
 }
-__device__ __forceinline__ int gather_candidates_copy(uint32_t* cand, int* wtot, const int32_t* cu, int S, int m0,
-                                                      int q1, int cap, int ptid, bool packed) {
-  constexpr int NT = 128, R = 16;
+__device__ __forceinline__ int gather_candidates_copy(uint32_t* cand, uint32_t* exc, int* wtot, const int32_t* cu,
+                                                      int S, int m0, int m1, int q1, int cap, int ptid, bool packed) {
+  constexpr int NT = 128, R = 8;
   const int lane = ptid & 31, w = ptid >> 5;
   const int ns = min(S, q1);
   for (int i = ptid; i < ns; i += NT) cand[i] = cand_entry(i, 0, packed);
-  int count = ns;
+  int na = ns, ne = 0;   // entries placed: sinks and kept keys / evicted keys
   const uint32_t lt = (1u << lane) - 1u;
   for (int base = S; base <= m0; base += NT * R) {
     const int wb = base + w * 32 * R;
@@ -694,34 +723,52 @@ __device__ __forceinline__ int gather_candidates_copy(uint32_t* cand, int* wtot,
       const int j = wb + 32 * r + lane;
       c[r] = j <= m0 ? cu[j] : 0;
     }
-    uint32_t bal[R];
-    int tot = 0;
+    uint32_t ba[R], be[R];
+    int ta = 0, te = 0;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int j = wb + 32 * r + lane;
-      bal[r] = __ballot_sync(0xffffffffu, j <= m0 && c[r] > m0);
-      tot += __popc(bal[r]);
+      ba[r] = __ballot_sync(0xffffffffu, j <= m0 && c[r] > m1);
+      be[r] = __ballot_sync(0xffffffffu, j <= m0 && c[r] > m0 && c[r] <= m1);
+      ta += __popc(ba[r]);
+      te += __popc(be[r]);
     }
-    if (lane == 0) wtot[w] = tot;
+    if (lane == 0) {
+      wtot[w] = ta;
+      wtot[4 + w] = te;
+    }
     named_bar_sync(kT2CopyBar, NT);
-    int off = count, total = 0;
+    int oa = na, oe = ne, sa = 0, se = 0;
 #pragma unroll
     for (int x = 0; x < NT / 32; ++x) {
-      const int t = wtot[x];
-      off += (x < w) ? t : 0;
-      total += t;
+      const int xa = wtot[x], xe = wtot[4 + x];
+      oa += (x < w) ? xa : 0;
+      oe += (x < w) ? xe : 0;
+      sa += xa;
+      se += xe;
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      if ((bal[r] >> lane) & 1u) {
-        const int o = off + __popc(bal[r] & lt);
-        if (o < cap) cand[o] = cand_entry(wb + 32 * r + lane, c[r], packed);
+      const int j = wb + 32 * r + lane;
+      if ((ba[r] >> lane) & 1u) {
+        const int o = oa + __popc(ba[r] & lt);
+        if (o < cap) cand[o] = cand_entry(j, c[r], packed);
       }
-      off += __popc(bal[r]);
+      if ((be[r] >> lane) & 1u) {
+        const int o = oe + __popc(be[r] & lt);
+        if (o < kT2Rows) exc[o] = cand_entry(j, c[r], packed);
+      }
+      oa += __popc(ba[r]);
+      oe += __popc(be[r]);
     }
-    count += total;
-    named_bar_sync(kT2CopyBar, NT);   // wtot is rewritten next round
+    na += sa;
+    ne += se;
+    named_bar_sync(kT2CopyBar, NT);   // wtot is rewritten next round; exc complete
   }
+  ne = min(ne, kT2Rows);   // at most m1 - m0 < qt <= kT2Rows evictions
+  for (int i = ptid; i < ne; i += NT)
+    if (na + i < cap) cand[na + i] = exc[i];
+  int count = na + ne;
   const int r0 = max(S, m0 + 1);
   const int nr = max(0, q1 - r0);
   for (int i = ptid; i < nr; i += NT)
@@ -773,7 +820,9 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
   uint32_t* taddr_s = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = misc + 1;
   int* count_ring = misc + 2;                     // [item % ring] candidate count of the item
-  int* wtot = misc + 2 + kT2Ring;                 // copy warps' totals (gather scan)
+  int* wtot = misc + 2 + kT2Ring;                 // copy warps' two totals each (gather scan)
+  uint32_t* exc = reinterpret_cast<uint32_t*>(smem_t2 + SM::EXC_OFF);
+
   uint32_t* cand2 = reinterpret_cast<uint32_t*>(smem_t2 + SM::CAND_OFF);   // item i's candidates at cand2 + (i & 1) * cand_cap
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -839,8 +888,9 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
     bool failed = false;
     auto gather = [&](int i) {   // item i's candidates into its buffer; count to the ring
       const T2Item w = t2_item(p, ntq, blockIdx.x + i * gridDim.x);
-      const int count = gather_candidates_copy(cand2 + (i & 1) * p.cand_cap, wtot, p.cut + static_cast<size_t>(w.u) * n,
-                                               S, w.q0 - WD, w.q1, p.cand_cap, ptid, packed);
+      const int count = gather_candidates_copy(cand2 + (i & 1) * p.cand_cap, exc, wtot,
+                                               p.cut + static_cast<size_t>(w.u) * n, S, w.q0 - WD, w.q1 - 1 - WD,
+                                               w.q1, p.cand_cap, ptid, packed);
       if (ptid == 0) {
         count_ring[i % kT2Ring] = count;
         mbar_arrive(&item_full[i % kT2Ring]);
@@ -936,39 +986,34 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
         // The tile's mask (§C.1) as two 32-bit words per query position of
         // the item (bit i of word h = key 32 h + i visible).  Key j (cutoff c)
         // is visible at position q iff j <= q and (j is a sink or
-        // q - W - D < max(j, c)): an interval of positions starting at j.
-        // Lane i holds keys i and 32 + i; one ballot per word finds the keys
-        // visible to every position of the item (the base words) and one the
-        // others (exceptions: keys evicted or admitted inside the item's
-        // range).  A tile without exceptions is only flagged; otherwise lane i
-        // builds the words of position 32 g + i from the base words and a
-        // test of each exception key's interval (broadcast by shuffles).
+        // q - W - D < max(j, c)): positions lo = j .. hi = max(j, c) + W + D - 1
+        // (no end for a sink).  Lane i holds keys i and 32 + i.  A tile whose
+        // keys all see every position of the item is only flagged; otherwise,
+        // per 32 positions, lane i forms the row of key 32 h + i (bit x =
+        // position x of the group visible) and a bit transpose across the
+        // warp turns the 32 rows into the 32 positions' words.
         uint32_t* rm = reinterpret_cast<uint32_t*>(meta + st * SM::META_INTS);
-        int lo[2], lim[2];
-        uint32_t base[2], exc[2];
+        int lo[2], hi[2];
+        uint32_t always_b[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           lo[h] = jh[h] >= 0 ? jh[h] : INT_MAX;              // past the candidates: never visible
-          lim[h] = jh[h] < S ? INT_MAX : mh[h];              // visible while q - W - D < lim
-          const bool always = lo[h] <= q0 && q1 - 1 - WD < lim[h];
-          base[h] = __ballot_sync(0xffffffffu, always);
-          exc[h] = __ballot_sync(0xffffffffu, jh[h] >= 0 && !always);
+          hi[h] = (jh[h] < S || mh[h] > INT_MAX - WD) ? INT_MAX : mh[h] + WD - 1;
+          always_b[h] = __ballot_sync(0xffffffffu, lo[h] <= q0 && hi[h] >= q1 - 1);
         }
-        const bool full_tile = (base[0] & base[1]) == 0xffffffffu;
+        const bool full_tile = (always_b[0] & always_b[1]) == 0xffffffffu;
         if (mw == 0 && lane == 0) rm[2 * kT2Rows] = full_tile ? 1u : 0u;
         if (!full_tile) {
           // positions in groups of 32, alternating between the two mask warps
           for (int r0 = 32 * mw; r0 < p.qt; r0 += 32 * (kT2Mma - kT2Mask)) {
-            const int qp = q0 + r0 + lane;
-            uint32_t wd[2] = {base[0], base[1]};
+            const int g0 = q0 + r0;
+            uint32_t wd[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-              for (uint32_t m = exc[h]; m != 0u; m &= m - 1u) {
-                const int e = __ffs(m) - 1;
-                const int l = __shfl_sync(0xffffffffu, lo[h], e);
-                const int L = __shfl_sync(0xffffffffu, lim[h], e);
-                if (l <= qp && qp - WD < L) wd[h] |= 1u << e;
-              }
+            for (int h = 0; h < 2; ++h) {
+              const int a = lo[h] == INT_MAX ? 32 : max(lo[h] - g0, -1);
+              const int b = hi[h] == INT_MAX ? 31 : min(hi[h] - g0, 32);
+              wd[h] = warp_transpose32(bit_range32(a, b), lane);
+            }
             if (r0 + lane < p.qt) *reinterpret_cast<uint2*>(rm + 2 * (r0 + lane)) = make_uint2(wd[0], wd[1]);
           }
         }
@@ -1063,7 +1108,9 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
               st_ = 0;
             }
           }
-          if (ready && st_ == 0) ready = q_loaded == si && mbar_test(&q_full[XB], si & 1);
+          // an item's first S waits for its Q rows, and for the item before's
+          // last P V to be issued, which the epilogue of that item waits for
+          if (ready && st_ == 0) ready = q_loaded == si && (si == 0 || Tp == Ts) && mbar_test(&q_full[XB], si & 1);
           if (ready && mbar_test(&kv_full[Ts % NST], (Ts / NST) & 1)) {
             tc_fence_after();
             issue_s(Ts);
@@ -1099,7 +1146,6 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
     // ---------------- softmax: block X, thread = row = TMEM lane ----------------
     const int X = warp >> 2;
     const int row = tid & 127;
-    const int g = row / PB;
     const int posoff = X * PB + row % PB;
     const uint32_t lrow = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + static_cast<uint32_t>(X * DH);
@@ -1147,11 +1193,16 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
           }
         }
         {
-          // four independent max chains, then their max
-          float m4[4] = {sv[0], sv[1], sv[2], sv[3]};
+          // four independent chains of three-input maxima (chain c: columns c, c + 4, ...), then their max
+          float m4[4];
 #pragma unroll
-          for (int x = 4; x < kT2Keys; ++x) m4[x & 3] = fmaxf(m4[x & 3], sv[x]);
-          tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          for (int c = 0; c < 4; ++c) {
+            m4[c] = fmax3(sv[c], sv[c + 4], sv[c + 8]);
+#pragma unroll
+            for (int x = c + 12; x < kT2Keys - 4; x += 8) m4[c] = fmax3(m4[c], sv[x], sv[x + 4]);
+            m4[c] = fmaxf(m4[c], sv[kT2Keys - 4 + c]);
+          }
+          tmax = fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], m4[3]);
         }
         const float tm = tmax * p.scale_log2;
         float alpha = 1.f;
@@ -1163,22 +1214,23 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
           m_run = tm;
         }
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;   // masked logits give 2^-inf = 0
-        // P(T) in bf16 over the first 32 columns of S(T), 16 columns at a time
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
+        // P(T) in bf16 over the first 32 columns of S(T), 16 columns at a time;
+        // the exponent arguments and the row sum on pairs (fp32x2 FMA and add)
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nm, nm);
+        float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};   // two independent partial sums of pairs
 #pragma unroll
         for (int h = 0; h < kT2Keys / 32; ++h) {
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            const float x0 = fmaf(sv[32 * h + x], p.scale_log2, nm), x1 = fmaf(sv[32 * h + x + 1], p.scale_log2, nm);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
-            ps[(x >> 1) & 3] += p0 + p1;
-            pk[x / 2] = pack_bf16(p0, p1);
+            const float2 xx = __ffma2_rn(make_float2(sv[32 * h + x], sv[32 * h + x + 1]), sc2, nm2);
+            const float2 pp = make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
+            ps2[(x >> 1) & 1] = __fadd2_rn(ps2[(x >> 1) & 1], pp);
+            pk[x / 2] = pack_bf16(pp.x, pp.y);
           }
           tc_st16u(tS + static_cast<uint32_t>(16 * h) + lrow, pk);
         }
-        l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        l_run += (ps2[0].x + ps2[1].x) + (ps2[0].y + ps2[1].y);
         if (__any_sync(0xffffffffu, resc)) {
           // rescale this row of O once the P V before (of tile T - 1, same item: t > 0) has completed
           const bool done = wait(&o_done[X], (T - 1) & 1);
@@ -1215,7 +1267,7 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
       // next item's first P V overwrites O only after this thread's next p_full arrival
       if (!__all_sync(0xffffffffu, wait(&o_done[X], (T - 1) & 1))) break;
       tc_fence_after();
-      const size_t rowi = (static_cast<size_t>(w.b) * p.Hq + w.hk * G + g) * n + (vrow ? qpos : 0);
+      const size_t rowi = (static_cast<size_t>(w.b) * p.Hq + w.hk * G + row / PB) * n + (vrow ? qpos : 0);
       __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out) + rowi * DH;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
