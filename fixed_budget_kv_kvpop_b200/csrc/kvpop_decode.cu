@@ -1420,6 +1420,9 @@ int launch_t(const CUtensorMap& tmap, const LayerArgs& a, const DecodeScratch& s
 
 }  // namespace
 
+namespace {
+// The driver's tensor-map encoder, fetched through the runtime so that the
+// library needs no link-time dependency on libcuda; null if unavailable.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (encode == nullptr) {
@@ -1432,6 +1435,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   }
   return encode;
 }
+}  // namespace
 
 int make_decode_tensor_map(CUtensorMap* map, void* layer_kv, int dtype, int d, int64_t rows, int row_bytes) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();

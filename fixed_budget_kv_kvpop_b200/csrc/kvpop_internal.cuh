@@ -27,7 +27,6 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -517,9 +516,6 @@ enum DecodeMode : int { MODE_STEP = 0, MODE_ATTEND = 1, MODE_STEP_NODECIDE = 2 }
 int launch_decode(const CUtensorMap& tmap, const LayerArgs& a, int dtype, const DecodeScratch& sc, int mode,
                   const void* q, const void* k_new, const void* v_new, const float* ext_score, void* out, int num_sms,
                   cudaStream_t st);
-// The driver's tensor-map encoder, fetched through the runtime so that the
-// library needs no link-time dependency on libcuda; null if unavailable.
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // Tensor map over one layer's cache rows for the decode kernel's TMA loads.
 int make_decode_tensor_map(CUtensorMap* map, void* layer_kv, int dtype, int d, int64_t rows, int row_bytes);
 // The cache update of a decode step without attention.

@@ -34,6 +34,8 @@
 // the last prompt position; place_kept_kernel writes them to the long-range
 // slots in ascending position order (what a one-chunk prefill places), so a
 // whole-prompt prefill and its attention outputs share one scoring pass.
+#include <cudaTypedefs.h>
+
 #include "kvpop_prefill_attn.cuh"
 
 namespace kvpop {
@@ -1271,19 +1273,19 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
       __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.out) + rowi * DH;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float o[32];
-        tc_ld32(tO + lrow + c0, o);
+      for (int c0 = 0; c0 < DH; c0 += 64) {
+        float o[64];
+        tc_ld64(tO + lrow + c0, o);
         if (vrow) {
-          uint32_t pk[16];
+          uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(o[2 * c] * inv, o[2 * c + 1] * inv);
+          for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(o[2 * c] * inv, o[2 * c + 1] * inv);
           if (out32) {   // one full 32-byte sector per store
 #pragma unroll
-            for (int c = 0; c < 2; ++c) st_global_v8(og + c0 + 16 * c, pk + 8 * c);
+            for (int c = 0; c < 4; ++c) st_global_v8(og + c0 + 16 * c, pk + 8 * c);
           } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 8; ++c)
               *reinterpret_cast<uint4*>(og + c0 + 8 * c) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
           }
         }
@@ -1300,6 +1302,21 @@ sparse_attn_tcp_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_co
   }
 }
 
+// The driver's tensor-map encoder, fetched through the runtime (no link-time
+// dependency on libcuda); null if unavailable.
+PFN_cuTensorMapEncodeTiled_v12000 attn_tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess || fn == nullptr)
+      return nullptr;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return encode;
+}
+
 // One CTA per SM (at most one per work item); Q through a 3-D tensor map
 // (head dim, position, batch row x query head) with one box per head and
 // 64-dim group.
@@ -1308,7 +1325,7 @@ int launch_attn_tcp_stages(const PaArgs& pa, int units, int n, size_t smem, cuda
   if (cudaFuncSetAttribute(sparse_attn_tcp_kernel<DH, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return -1;
-  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  PFN_cuTensorMapEncodeTiled_v12000 encode = attn_tensor_map_encoder();
   if (encode == nullptr) return -1;
   const int B = units / pa.Hkv;
   CUtensorMap qmap;
