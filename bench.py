@@ -116,13 +116,13 @@ TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024",
 
 
 # ncu capture of the prefill attention's tensor-core kernel (the small case of
-# profiles/sparse_attn_tc2_kernel_cr88_b4_full.md: 4 rows x 8 KV heads =
+# profiles/sparse_attn_tcp_kernel_cr88_b4_full.md: 4 rows x 8 KV heads =
 # 32 units, prompt 8192): DRAM read + write of one launch.  Traffic grows with
 # the units a launch covers (every unit reads its own q, k, v and writes its
 # own output), so a launch of U units moves dram_bytes * U / 32.
 PA_TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024", "units": 32,
-                      "kernel_sha256": "7385e8788803a77d0a9c3116f389047326352182b5eb6f59b175ac56cfcf8365",
-                      "dram_bytes": 403_767_040 + 235_346_176}
+                      "kernel_sha256": "beca722c9380e6e50b89152aefac4c8391a573c3bc8487aa3d4ab72b68a25f90",
+                      "dram_bytes": 403_797_248 + 239_627_520}
 
 
 def _strip_code(src: str) -> str:
