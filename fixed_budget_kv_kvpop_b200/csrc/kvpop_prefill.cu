@@ -149,139 +149,129 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, Chunk
 }
 
 // P1 for the common shapes (2d in {128, 256}, hidden in {32, 64}): the same
-// scores as score_kernel, with W1 (transposed) and the token tile held in
-// shared memory as fp64, so the inner loop is 4 shared loads of 2 doubles per
-// 16 fp64 FMAs and nothing is converted there.  Thread (tq, hq) computes the
-// pre-activations of tokens 4tq..4tq+3 x hidden 4hq..4hq+3; the 16 threads of
-// a token quad then finish w2 . relu(. + b1) by shuffles.  Each block keeps
-// W1 resident and walks kTilesPerBlock token tiles of its unit.
+// scores as score_kernel, with the pre-activations W1 x on the fp64 tensor
+// cores (mma.sync m8n8k4 f64: fp64 products and sums, as score_kernel's fp64
+// FMAs).  Shared memory holds W1 transposed and a tile of TT tokens' inputs
+// [k; v], both in fp32 (exact for fp32 weights and bf16/fp32 inputs; each
+// operand fragment is widened to fp64 as it is loaded), with row pitches
+// that make every fragment load conflict-free.  Warp w owns tokens 32 w ..
+// 32 w + 31 of the tile (4 row tiles of 8) x all hidden units (HID / 8
+// column tiles): per 4 inputs it loads 4 + HID / 8 fragments and issues
+// 4 HID / 8 MMAs.  The epilogue finishes w2 . relu(. + b1) per token from
+// the accumulators and sums the 4 lanes of each row by shuffles.  Each block
+// keeps W1 resident and walks kTilesPerBlock token tiles of its unit.
 constexpr int kScore64Threads = 128;
 constexpr int kTilesPerBlock = 8;
 
 template <int D2, int HID>
 struct Score64Geom {
-  static constexpr int TT = 4 * (kScore64Threads / (HID / 4));   // tokens per tile: 32 (HID 64) or 64 (HID 32)
-  static constexpr int WP = HID + 2;                             // padded row of the transposed W1 (doubles)
-  static constexpr int XP = TT + 2;                              // padded row of the transposed tile (doubles)
-  static constexpr int SMEM = (D2 * WP + D2 * XP) * 8;
+  static constexpr int TT = (kScore64Threads / 32) * 32;      // tokens per tile: 32 per warp
+  static constexpr int XP = D2 + 4;                            // floats per token row (pitch = 4 mod 32)
+  static constexpr int WP = HID + 8;                           // floats per input row of W1^T (pitch = 8 mod 32)
+  static constexpr int SMEM = (D2 * WP + TT * XP) * 4;
 };
 
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d[0]), "+d"(d[1]) : "d"(a), "d"(b));
+}
+
 template <typename T, int D2, int HID>
-__global__ void __launch_bounds__(kScore64Threads) score64_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k,
-                                                                  const T* __restrict__ v, int n,
-                                                                  float* __restrict__ out, int cap) {
+__global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a, ChunkGeom cg,
+                                                                     const T* __restrict__ k,
+                                                                     const T* __restrict__ v, int n,
+                                                                     float* __restrict__ out, int cap) {
   using SG = Score64Geom<D2, HID>;
-  constexpr int TT = SG::TT, WP = SG::WP, XP = SG::XP;
-  constexpr int HQN = HID / 4;   // threads per token quad
-  extern __shared__ __align__(16) double sm64[];
-  double* Wd = sm64;             // [D2][WP]: Wd[i][j] = W1[j][i]
-  double* Xd = sm64 + D2 * WP;   // [D2][XP]: Xd[i][t] = x_t[i]
+  constexpr int TT = SG::TT, XP = SG::XP, WP = SG::WP;
+  constexpr int NT = HID / 8;                                   // column tiles (hidden)
+  constexpr int EPU = 16 / static_cast<int>(sizeof(T));        // inputs per 16-byte load
+  constexpr int UPT = D2 / EPU;                                 // 16-byte loads per token row
+  extern __shared__ __align__(16) float smf[];
+  float* Wt = smf;                                              // [D2][WP]: Wt[i][j] = W1[j][i]
+  float* Xs = smf + D2 * WP;                                    // [TT][XP]: Xs[t][i] = x_t[i]
   const int u = blockIdx.y;
   const int h = u % a.Hkv;
   const int n_new = cg.e1 - cg.e0;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile0 = blockIdx.x * kTilesPerBlock;
   if (tile0 * TT >= n_new) return;
 
-  const float* w1 = a.w1 + static_cast<size_t>(h) * HID * D2;
   {
-    // thread -> a contiguous stretch of one W1 row; 8 float4 loads in flight
-    constexpr int FPT = HID * D2 / kScore64Threads;   // floats per thread (a divisor of D2)
-    const int j = (tid * FPT) / D2, i0 = (tid * FPT) % D2;
-    const float4* src = reinterpret_cast<const float4*>(w1 + static_cast<size_t>(j) * D2 + i0);
-#pragma unroll
-    for (int q0 = 0; q0 < FPT / 4; q0 += 8) {
-      float4 wv[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) wv[q] = __ldg(src + q0 + q);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int i = i0 + 4 * (q0 + q);
-        Wd[(i + 0) * WP + j] = static_cast<double>(wv[q].x);
-        Wd[(i + 1) * WP + j] = static_cast<double>(wv[q].y);
-        Wd[(i + 2) * WP + j] = static_cast<double>(wv[q].z);
-        Wd[(i + 3) * WP + j] = static_cast<double>(wv[q].w);
-      }
+    // W1 [HID][D2] -> Wt: thread -> hidden j = e % HID, inputs 4 q .. 4 q + 3
+    // (consecutive lanes write consecutive j of one input row)
+    const float* w1 = a.w1 + static_cast<size_t>(h) * HID * D2;
+    for (int e = tid; e < HID * D2 / 4; e += kScore64Threads) {
+      const int j = e % HID, q = e / HID;
+      const float4 wv = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(j) * D2) + q);
+      float* dst = Wt + (4 * q) * WP + j;
+      dst[0] = wv.x;
+      dst[WP] = wv.y;
+      dst[2 * WP] = wv.z;
+      dst[3 * WP] = wv.w;
     }
   }
-  const int tq = tid / HQN, hq = tid % HQN;
-  const float* b1 = a.b1 + static_cast<size_t>(h) * HID;
-  const float* w2 = a.w2 + static_cast<size_t>(h) * HID;
-  double b1v[4], w2v[4];
+  const int gr = lane >> 2, gc = lane & 3;                      // fragment row / column within a tile
+  // this lane's hidden units in the accumulators: 8 c + 2 gc + {0, 1}, c < NT
+  double b1v[NT][2], w2v[NT][2];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    b1v[c] = static_cast<double>(b1[4 * hq + c]);
-    w2v[c] = static_cast<double>(w2[4 * hq + c]);
-  }
+  for (int c = 0; c < NT; ++c)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      b1v[c][e] = static_cast<double>(a.b1[static_cast<size_t>(h) * HID + 8 * c + 2 * gc + e]);
+      w2v[c][e] = static_cast<double>(a.w2[static_cast<size_t>(h) * HID + 8 * c + 2 * gc + e]);
+    }
   const double b2 = static_cast<double>(a.b2[h]);
 
   for (int tile = tile0; tile < tile0 + kTilesPerBlock && tile * TT < n_new; ++tile) {
     const int tok0 = tile * TT;
-    const int ntok = min(TT, n_new - tok0);
     __syncthreads();   // W1 written (first tile) / previous tile's reads done
-    {
-      // thread -> (token tt, part p): a contiguous stretch of EPT inputs, all
-      // within k or within v; every 16-byte load is issued before any is used
-      constexpr int TPT = kScore64Threads / TT;   // threads per token (2 or 4)
-      constexpr int EPT = D2 / TPT;               // inputs per thread
-      constexpr int NV = EPT * static_cast<int>(sizeof(T)) / 16;
-      const int tt = tid / TPT, p = tid % TPT;
-      alignas(16) T xr[EPT];
-      if (tt < ntok) {
-        const int t = cg.e0 + tok0 + tt;
+    for (int e = tid; e < TT * UPT; e += kScore64Threads) {
+      const int tt = e / UPT, c = e % UPT;
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (tok0 + tt < n_new) {
         const uint8_t* vs;
-        const uint8_t* ks = token_row<T>(a, cg, u, t, k, v, n, vs);
-        const int i0 = p * EPT;
-        const uint4* src = reinterpret_cast<const uint4*>(
-            (i0 < D2 / 2) ? ks + i0 * sizeof(T) : vs + (i0 - D2 / 2) * sizeof(T));
-#pragma unroll
-        for (int q = 0; q < NV; ++q) reinterpret_cast<uint4*>(xr)[q] = src[q];
-      } else {
-#pragma unroll
-        for (int q = 0; q < NV; ++q) reinterpret_cast<uint4*>(xr)[q] = make_uint4(0u, 0u, 0u, 0u);
+        const uint8_t* ks = token_row<T>(a, cg, u, cg.e0 + tok0 + tt, k, v, n, vs);
+        const int i0 = c * EPU;
+        raw = *reinterpret_cast<const uint4*>((i0 < D2 / 2) ? ks + i0 * sizeof(T) : vs + (i0 - D2 / 2) * sizeof(T));
       }
+      const T* xe = reinterpret_cast<const T*>(&raw);
 #pragma unroll
-      for (int e = 0; e < EPT; ++e) Xd[(p * EPT + e) * XP + tt] = static_cast<double>(Elem<T>::to_f32(xr[e]));
+      for (int q = 0; q < EPU; ++q) Xs[tt * XP + c * EPU + q] = Elem<T>::to_f32(xe[q]);
     }
     __syncthreads();
-    double acc[4][4];
+    double acc[4][NT][2];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
-#pragma unroll 4
-    for (int i = 0; i < D2; ++i) {
-      const double2 x01 = *reinterpret_cast<const double2*>(Xd + i * XP + 4 * tq);
-      const double2 x23 = *reinterpret_cast<const double2*>(Xd + i * XP + 4 * tq + 2);
-      const double2 w01 = *reinterpret_cast<const double2*>(Wd + i * WP + 4 * hq);
-      const double2 w23 = *reinterpret_cast<const double2*>(Wd + i * WP + 4 * hq + 2);
-      const double xr[4] = {x01.x, x01.y, x23.x, x23.y};
-      const double wc[4] = {w01.x, w01.y, w23.x, w23.y};
+      for (int c = 0; c < NT; ++c) acc[m][c][0] = acc[m][c][1] = 0.0;
+    const float* xa = Xs + (32 * warp + gr) * XP + gc;            // A: row gr of tile m at + 8 m XP, inputs i0 + gc
+    const float* wb = Wt + gc * WP + gr;                          // B: input i0 + gc, hidden 8 c + gr
+#pragma unroll 2
+    for (int i0 = 0; i0 < D2; i0 += 4) {
+      double af[4], bf[NT];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int m = 0; m < 4; ++m) af[m] = static_cast<double>(xa[8 * m * XP + i0]);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fma(xr[r], wc[c], acc[r][c]);
+      for (int c = 0; c < NT; ++c) bf[c] = static_cast<double>(wb[i0 * WP + 8 * c]);
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int c = 0; c < NT; ++c) dmma_8x8x4(acc[m][c], af[m], bf[c]);
     }
-    double part[4];
+    // w2 . relu(W1 x + b1) + b2: this lane holds tokens 32 warp + 8 m + gr, 2 NT hidden units each
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      part[r] = 0.0;
+    for (int m = 0; m < 4; ++m) {
+      double part = 0.0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) part[r] = fma(w2v[c], fmax(acc[r][c] + b1v[c], 0.0), part[r]);
-    }
-    // reduce over the HQN threads of a token quad (consecutive lanes, HQN | 32)
+      for (int c = 0; c < NT; ++c)
 #pragma unroll
-    for (int off = 1; off < HQN; off <<= 1)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], off);
-    if (hq == 0) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int tt = 4 * tq + r;
-        if (tt < ntok)
-          out[static_cast<size_t>(u) * cap + tok0 + tt] =
-              ranking_priority(a, u, cg.e0 + tok0 + tt + a.W + a.D, static_cast<float>(part[r] + b2));
-      }
+        for (int e = 0; e < 2; ++e) part = fma(w2v[c][e], fmax(acc[m][c][e] + b1v[c][e], 0.0), part);
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      const int tt = 32 * warp + 8 * m + gr;
+      if (gc == 0 && tok0 + tt < n_new)
+        out[static_cast<size_t>(u) * cap + tok0 + tt] =
+            ranking_priority(a, u, cg.e0 + tok0 + tt + a.W + a.D, static_cast<float>(part + b2));
     }
   }
 }
