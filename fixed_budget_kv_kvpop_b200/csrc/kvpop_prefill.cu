@@ -154,21 +154,23 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, Chunk
 // FMAs).  Shared memory holds W1 transposed and a tile of TT tokens' inputs
 // [k; v], both in fp32 (exact for fp32 weights and bf16/fp32 inputs; each
 // operand fragment is widened to fp64 as it is loaded), with row pitches
-// that make every fragment load conflict-free.  Warp w owns tokens 32 w ..
-// 32 w + 31 of the tile (4 row tiles of 8) x all hidden units (HID / 8
-// column tiles): per 4 inputs it loads 4 + HID / 8 fragments and issues
-// 4 HID / 8 MMAs.  The epilogue finishes w2 . relu(. + b1) per token from
-// the accumulators and sums the 4 lanes of each row by shuffles.  Each block
-// keeps W1 resident and walks kTilesPerBlock token tiles of its unit.
-constexpr int kScore64Threads = 128;
+// that make every fragment load conflict-free.  Warp w owns tokens 32 (w % 4)
+// .. + 31 of the tile (4 row tiles of 8) x half w / 4 of the hidden units
+// (HID / 16 column tiles of 8): per 4 inputs it loads 4 + HID / 16 fragments
+// and issues HID / 4 MMAs; two warps per scheduler hide each other's MMA
+// latency.  The epilogue forms w2 . relu(. + b1) over the warp's hidden half
+// per token, sums the 4 lanes of each row by shuffles and the two halves in
+// a fixed order through shared memory.  Each block keeps W1 resident and
+// walks kTilesPerBlock token tiles of its unit.
+constexpr int kScore64Threads = 256;
 constexpr int kTilesPerBlock = 8;
 
 template <int D2, int HID>
 struct Score64Geom {
-  static constexpr int TT = (kScore64Threads / 32) * 32;      // tokens per tile: 32 per warp
+  static constexpr int TT = 128;                               // tokens per tile: 32 per warp pair
   static constexpr int XP = D2 + 4;                            // floats per token row (pitch = 4 mod 32)
   static constexpr int WP = HID + 8;                           // floats per input row of W1^T (pitch = 8 mod 32)
-  static constexpr int SMEM = (D2 * WP + TT * XP) * 4;
+  static constexpr int SMEM = (D2 * WP + TT * XP) * 4 + 2 * TT * 8;   // + the halves' partial sums
 };
 
 __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
@@ -183,12 +185,13 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
                                                                      float* __restrict__ out, int cap) {
   using SG = Score64Geom<D2, HID>;
   constexpr int TT = SG::TT, XP = SG::XP, WP = SG::WP;
-  constexpr int NT = HID / 8;                                   // column tiles (hidden)
+  constexpr int NT = HID / 16;                                  // column tiles of this warp's hidden half
   constexpr int EPU = 16 / static_cast<int>(sizeof(T));        // inputs per 16-byte load
   constexpr int UPT = D2 / EPU;                                 // 16-byte loads per token row
   extern __shared__ __align__(16) float smf[];
   float* Wt = smf;                                              // [D2][WP]: Wt[i][j] = W1[j][i]
   float* Xs = smf + D2 * WP;                                    // [TT][XP]: Xs[t][i] = x_t[i]
+  double* pp = reinterpret_cast<double*>(Xs + TT * XP);         // [half][TT] partial sums
   const int u = blockIdx.y;
   const int h = u % a.Hkv;
   const int n_new = cg.e1 - cg.e0;
@@ -198,45 +201,71 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
 
   {
     // W1 [HID][D2] -> Wt: thread -> hidden j = e % HID, inputs 4 q .. 4 q + 3
-    // (consecutive lanes write consecutive j of one input row)
+    // with q = e / HID (consecutive lanes write consecutive j of one input
+    // row), 4 loads in flight per thread before any is stored
     const float* w1 = a.w1 + static_cast<size_t>(h) * HID * D2;
-    for (int e = tid; e < HID * D2 / 4; e += kScore64Threads) {
-      const int j = e % HID, q = e / HID;
-      const float4 wv = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(j) * D2) + q);
-      float* dst = Wt + (4 * q) * WP + j;
-      dst[0] = wv.x;
-      dst[WP] = wv.y;
-      dst[2 * WP] = wv.z;
-      dst[3 * WP] = wv.w;
+    static_assert((HID * D2 / 4) % (4 * kScore64Threads) == 0, "whole batches of loads");
+#pragma unroll 1
+    for (int e0 = 0; e0 < HID * D2 / 4; e0 += 4 * kScore64Threads) {
+      float4 wv[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int e = e0 + tid + x * kScore64Threads;
+        wv[x] = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(e % HID) * D2) + e / HID);
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int e = e0 + tid + x * kScore64Threads;
+        float* dst = Wt + (4 * (e / HID)) * WP + e % HID;
+        dst[0] = wv[x].x;
+        dst[WP] = wv[x].y;
+        dst[2 * WP] = wv[x].z;
+        dst[3 * WP] = wv[x].w;
+      }
     }
   }
   const int gr = lane >> 2, gc = lane & 3;                      // fragment row / column within a tile
-  // this lane's hidden units in the accumulators: 8 c + 2 gc + {0, 1}, c < NT
+  const int tg = warp & 3, hh = warp >> 2;                      // token group, hidden half
+  const int j0 = hh * (HID / 2);
+  // this lane's hidden units in the accumulators: j0 + 8 c + 2 gc + {0, 1}, c < NT
   double b1v[NT][2], w2v[NT][2];
 #pragma unroll
   for (int c = 0; c < NT; ++c)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      b1v[c][e] = static_cast<double>(a.b1[static_cast<size_t>(h) * HID + 8 * c + 2 * gc + e]);
-      w2v[c][e] = static_cast<double>(a.w2[static_cast<size_t>(h) * HID + 8 * c + 2 * gc + e]);
+      b1v[c][e] = static_cast<double>(a.b1[static_cast<size_t>(h) * HID + j0 + 8 * c + 2 * gc + e]);
+      w2v[c][e] = static_cast<double>(a.w2[static_cast<size_t>(h) * HID + j0 + 8 * c + 2 * gc + e]);
     }
   const double b2 = static_cast<double>(a.b2[h]);
 
   for (int tile = tile0; tile < tile0 + kTilesPerBlock && tile * TT < n_new; ++tile) {
     const int tok0 = tile * TT;
     __syncthreads();   // W1 written (first tile) / previous tile's reads done
-    for (int e = tid; e < TT * UPT; e += kScore64Threads) {
-      const int tt = e / UPT, c = e % UPT;
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (tok0 + tt < n_new) {
-        const uint8_t* vs;
-        const uint8_t* ks = token_row<T>(a, cg, u, cg.e0 + tok0 + tt, k, v, n, vs);
-        const int i0 = c * EPU;
-        raw = *reinterpret_cast<const uint4*>((i0 < D2 / 2) ? ks + i0 * sizeof(T) : vs + (i0 - D2 / 2) * sizeof(T));
-      }
-      const T* xe = reinterpret_cast<const T*>(&raw);
+    // the tile's rows, 8 16-byte loads in flight per thread before any is stored
+    static_assert((TT * UPT) % (8 * kScore64Threads) == 0, "whole batches of loads");
+#pragma unroll 1
+    for (int e0 = 0; e0 < TT * UPT; e0 += 8 * kScore64Threads) {
+      uint4 raw[8];
 #pragma unroll
-      for (int q = 0; q < EPU; ++q) Xs[tt * XP + c * EPU + q] = Elem<T>::to_f32(xe[q]);
+      for (int x = 0; x < 8; ++x) {
+        const int e = e0 + tid + x * kScore64Threads;
+        const int tt = e / UPT, c = e % UPT;
+        raw[x] = make_uint4(0u, 0u, 0u, 0u);
+        if (tok0 + tt < n_new) {
+          const uint8_t* vs;
+          const uint8_t* ks = token_row<T>(a, cg, u, cg.e0 + tok0 + tt, k, v, n, vs);
+          const int i0 = c * EPU;
+          raw[x] = *reinterpret_cast<const uint4*>((i0 < D2 / 2) ? ks + i0 * sizeof(T) : vs + (i0 - D2 / 2) * sizeof(T));
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int e = e0 + tid + x * kScore64Threads;
+        const int tt = e / UPT, c = e % UPT;
+        const T* xe = reinterpret_cast<const T*>(&raw[x]);
+#pragma unroll
+        for (int q = 0; q < EPU; ++q) Xs[tt * XP + c * EPU + q] = Elem<T>::to_f32(xe[q]);
+      }
     }
     __syncthreads();
     double acc[4][NT][2];
@@ -244,8 +273,8 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
     for (int m = 0; m < 4; ++m)
 #pragma unroll
       for (int c = 0; c < NT; ++c) acc[m][c][0] = acc[m][c][1] = 0.0;
-    const float* xa = Xs + (32 * warp + gr) * XP + gc;            // A: row gr of tile m at + 8 m XP, inputs i0 + gc
-    const float* wb = Wt + gc * WP + gr;                          // B: input i0 + gc, hidden 8 c + gr
+    const float* xa = Xs + (32 * tg + gr) * XP + gc;              // A: row gr of tile m at + 8 m XP, inputs i0 + gc
+    const float* wb = Wt + gc * WP + j0 + gr;                     // B: input i0 + gc, hidden j0 + 8 c + gr
 #pragma unroll 2
     for (int i0 = 0; i0 < D2; i0 += 4) {
       double af[4], bf[NT];
@@ -258,7 +287,8 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
 #pragma unroll
         for (int c = 0; c < NT; ++c) dmma_8x8x4(acc[m][c], af[m], bf[c]);
     }
-    // w2 . relu(W1 x + b1) + b2: this lane holds tokens 32 warp + 8 m + gr, 2 NT hidden units each
+    // w2 . relu(W1 x + b1) over this warp's hidden half: this lane holds
+    // tokens 32 tg + 8 m + gr, 2 NT hidden units each
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       double part = 0.0;
@@ -268,11 +298,13 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
         for (int e = 0; e < 2; ++e) part = fma(w2v[c][e], fmax(acc[m][c][e] + b1v[c][e], 0.0), part);
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
-      const int tt = 32 * warp + 8 * m + gr;
-      if (gc == 0 && tok0 + tt < n_new)
-        out[static_cast<size_t>(u) * cap + tok0 + tt] =
-            ranking_priority(a, u, cg.e0 + tok0 + tt + a.W + a.D, static_cast<float>(part + b2));
+      if (gc == 0) pp[hh * TT + 32 * tg + 8 * m + gr] = part;
     }
+    __syncthreads();
+    // the two halves in a fixed order, + b2, one token per thread
+    if (tid < TT && tok0 + tid < n_new)
+      out[static_cast<size_t>(u) * cap + tok0 + tid] =
+          ranking_priority(a, u, cg.e0 + tok0 + tid + a.W + a.D, static_cast<float>(pp[tid] + pp[TT + tid] + b2));
   }
 }
 
