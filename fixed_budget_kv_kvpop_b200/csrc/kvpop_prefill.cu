@@ -155,14 +155,15 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, Chunk
 // [k; v], both in fp32 (exact for fp32 weights and bf16/fp32 inputs; each
 // operand fragment is widened to fp64 as it is loaded), with row pitches
 // that make every fragment load conflict-free.  Warp w owns tokens 32 (w % 4)
-// .. + 31 of the tile (4 row tiles of 8) x half w / 4 of the hidden units
-// (HID / 16 column tiles of 8): per 4 inputs it loads 4 + HID / 16 fragments
-// and issues HID / 4 MMAs; two warps per scheduler hide each other's MMA
-// latency.  The epilogue forms w2 . relu(. + b1) over the warp's hidden half
-// per token, sums the 4 lanes of each row by shuffles and the two halves in
-// a fixed order through shared memory.  Each block keeps W1 resident and
-// walks kTilesPerBlock token tiles of its unit.
-constexpr int kScore64Threads = 256;
+// .. + 31 of the tile (4 row tiles of 8) x part w / 4 of HS equal parts of
+// the hidden units: per 4 inputs it loads 4 + HID / (8 HS) fragments and
+// issues 4 HID / (8 HS) MMAs; HS warps per scheduler hide each other's MMA
+// latency.  The epilogue forms w2 . relu(. + b1) over the warp's part per
+// token, sums the 4 lanes of each row by shuffles and the HS parts in a
+// fixed order through shared memory.  Each block keeps W1 resident and walks
+// kTilesPerBlock token tiles of its unit.
+constexpr int kScore64Threads = 512;
+constexpr int kScore64Parts = kScore64Threads / 128;   // HS: hidden parts, one warp each per token group
 constexpr int kTilesPerBlock = 8;
 
 template <int D2, int HID>
@@ -170,7 +171,7 @@ struct Score64Geom {
   static constexpr int TT = 128;                               // tokens per tile: 32 per warp pair
   static constexpr int XP = D2 + 4;                            // floats per token row (pitch = 4 mod 32)
   static constexpr int WP = HID + 8;                           // floats per input row of W1^T (pitch = 8 mod 32)
-  static constexpr int SMEM = (D2 * WP + TT * XP) * 4 + 2 * TT * 8;   // + the halves' partial sums
+  static constexpr int SMEM = (D2 * WP + TT * XP) * 4 + kScore64Parts * TT * 8;   // + the parts' partial sums
 };
 
 __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
@@ -185,13 +186,15 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
                                                                      float* __restrict__ out, int cap) {
   using SG = Score64Geom<D2, HID>;
   constexpr int TT = SG::TT, XP = SG::XP, WP = SG::WP;
-  constexpr int NT = HID / 16;                                  // column tiles of this warp's hidden half
+  constexpr int HS = kScore64Parts;
+  constexpr int NT = HID / (8 * HS);                            // column tiles of this warp's hidden part
+  static_assert(NT >= 1 && HID % (8 * HS) == 0, "whole column tiles per part");
   constexpr int EPU = 16 / static_cast<int>(sizeof(T));        // inputs per 16-byte load
   constexpr int UPT = D2 / EPU;                                 // 16-byte loads per token row
   extern __shared__ __align__(16) float smf[];
   float* Wt = smf;                                              // [D2][WP]: Wt[i][j] = W1[j][i]
   float* Xs = smf + D2 * WP;                                    // [TT][XP]: Xs[t][i] = x_t[i]
-  double* pp = reinterpret_cast<double*>(Xs + TT * XP);         // [half][TT] partial sums
+  double* pp = reinterpret_cast<double*>(Xs + TT * XP);         // [part][TT] partial sums
   const int u = blockIdx.y;
   const int h = u % a.Hkv;
   const int n_new = cg.e1 - cg.e0;
@@ -202,31 +205,29 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
   {
     // W1 [HID][D2] -> Wt: thread -> hidden j = e % HID, inputs 4 q .. 4 q + 3
     // with q = e / HID (consecutive lanes write consecutive j of one input
-    // row), 4 loads in flight per thread before any is stored
+    // row), all of a thread's loads in flight before any is stored
     const float* w1 = a.w1 + static_cast<size_t>(h) * HID * D2;
-    static_assert((HID * D2 / 4) % (4 * kScore64Threads) == 0, "whole batches of loads");
-#pragma unroll 1
-    for (int e0 = 0; e0 < HID * D2 / 4; e0 += 4 * kScore64Threads) {
-      float4 wv[4];
+    constexpr int WL = HID * D2 / 4 / kScore64Threads;          // float4 loads per thread
+    static_assert(WL >= 1 && WL * kScore64Threads == HID * D2 / 4, "whole loads per thread");
+    float4 wv[WL];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int e = e0 + tid + x * kScore64Threads;
-        wv[x] = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(e % HID) * D2) + e / HID);
-      }
+    for (int x = 0; x < WL; ++x) {
+      const int e = tid + x * kScore64Threads;
+      wv[x] = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(e % HID) * D2) + e / HID);
+    }
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int e = e0 + tid + x * kScore64Threads;
-        float* dst = Wt + (4 * (e / HID)) * WP + e % HID;
-        dst[0] = wv[x].x;
-        dst[WP] = wv[x].y;
-        dst[2 * WP] = wv[x].z;
-        dst[3 * WP] = wv[x].w;
-      }
+    for (int x = 0; x < WL; ++x) {
+      const int e = tid + x * kScore64Threads;
+      float* dst = Wt + (4 * (e / HID)) * WP + e % HID;
+      dst[0] = wv[x].x;
+      dst[WP] = wv[x].y;
+      dst[2 * WP] = wv[x].z;
+      dst[3 * WP] = wv[x].w;
     }
   }
   const int gr = lane >> 2, gc = lane & 3;                      // fragment row / column within a tile
-  const int tg = warp & 3, hh = warp >> 2;                      // token group, hidden half
-  const int j0 = hh * (HID / 2);
+  const int tg = warp & 3, hh = warp >> 2;                      // token group, hidden part
+  const int j0 = hh * (HID / HS);
   // this lane's hidden units in the accumulators: j0 + 8 c + 2 gc + {0, 1}, c < NT
   double b1v[NT][2], w2v[NT][2];
 #pragma unroll
@@ -241,13 +242,14 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
   for (int tile = tile0; tile < tile0 + kTilesPerBlock && tile * TT < n_new; ++tile) {
     const int tok0 = tile * TT;
     __syncthreads();   // W1 written (first tile) / previous tile's reads done
-    // the tile's rows, 8 16-byte loads in flight per thread before any is stored
-    static_assert((TT * UPT) % (8 * kScore64Threads) == 0, "whole batches of loads");
+    // the tile's rows, up to 8 16-byte loads in flight per thread before any is stored
+    constexpr int XL = TT * UPT / kScore64Threads < 8 ? TT * UPT / kScore64Threads : 8;   // loads per batch
+    static_assert(XL >= 1 && (TT * UPT) % (XL * kScore64Threads) == 0, "whole batches of loads");
 #pragma unroll 1
-    for (int e0 = 0; e0 < TT * UPT; e0 += 8 * kScore64Threads) {
-      uint4 raw[8];
+    for (int e0 = 0; e0 < TT * UPT; e0 += XL * kScore64Threads) {
+      uint4 raw[XL];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) {
+      for (int x = 0; x < XL; ++x) {
         const int e = e0 + tid + x * kScore64Threads;
         const int tt = e / UPT, c = e % UPT;
         raw[x] = make_uint4(0u, 0u, 0u, 0u);
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
         }
       }
 #pragma unroll
-      for (int x = 0; x < 8; ++x) {
+      for (int x = 0; x < XL; ++x) {
         const int e = e0 + tid + x * kScore64Threads;
         const int tt = e / UPT, c = e % UPT;
         const T* xe = reinterpret_cast<const T*>(&raw[x]);
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
 #pragma unroll
         for (int c = 0; c < NT; ++c) dmma_8x8x4(acc[m][c], af[m], bf[c]);
     }
-    // w2 . relu(W1 x + b1) over this warp's hidden half: this lane holds
+    // w2 . relu(W1 x + b1) over this warp's hidden part: this lane holds
     // tokens 32 tg + 8 m + gr, 2 NT hidden units each
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -301,10 +303,14 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
       if (gc == 0) pp[hh * TT + 32 * tg + 8 * m + gr] = part;
     }
     __syncthreads();
-    // the two halves in a fixed order, + b2, one token per thread
-    if (tid < TT && tok0 + tid < n_new)
+    // the parts in a fixed order, + b2, one token per thread
+    if (tid < TT && tok0 + tid < n_new) {
+      double sum = pp[tid];
+#pragma unroll
+      for (int q = 1; q < HS; ++q) sum += pp[q * TT + tid];
       out[static_cast<size_t>(u) * cap + tok0 + tid] =
-          ranking_priority(a, u, cg.e0 + tok0 + tid + a.W + a.D, static_cast<float>(pp[tid] + pp[TT + tid] + b2));
+          ranking_priority(a, u, cg.e0 + tok0 + tid + a.W + a.D, static_cast<float>(sum + b2));
+    }
   }
 }
 
