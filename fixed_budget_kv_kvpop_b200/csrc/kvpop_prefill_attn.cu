@@ -52,26 +52,22 @@ __host__ __device__ inline int next_pow2(int x) {
   return p;
 }
 
-// ---------------- cutoffs: one CTA per unit ----------------
+// ---------------- cutoffs: sort (one CTA per unit), then walk (one warp per unit) ----------------
 __global__ void __launch_bounds__(kCutThreads) cutoff_kernel(const float* __restrict__ scores, int score_cap,
-                                                             int32_t* __restrict__ cut, int n, int ne, int npow,
-                                                             int words, int S, int K, uint64_t* keys_g,
-                                                             uint32_t* bits_g, int keys_global, int bits_global,
-                                                             int32_t* err) {
+                                                             int32_t* __restrict__ cut, int32_t* __restrict__ order,
+                                                             int n, int ne, int npow, int S, uint64_t* keys_g,
+                                                             int keys_global) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   int32_t* cu = cut + static_cast<size_t>(u) * n;
   uint64_t* keys = keys_global ? keys_g + static_cast<size_t>(u) * npow : reinterpret_cast<uint64_t*>(smem_raw);
-  uint32_t* bits = bits_global ? bits_g + static_cast<size_t>(u) * words
-                               : reinterpret_cast<uint32_t*>(smem_raw + (keys_global ? 0 : static_cast<size_t>(npow) * 8));
   // tokens that never become eligible in the prompt
   for (int t = tid; t < n; t += blockDim.x)
     if (t < S || t >= S + ne) cu[t] = -1;
   if (ne == 0) return;
   const float* su = scores + static_cast<size_t>(u) * score_cap;
   for (int i = tid; i < npow; i += blockDim.x) keys[i] = (i < ne) ? rank_key(su[i], S + i) : 0ull;
-  for (int i = tid; i < words; i += blockDim.x) bits[i] = 0u;
   __syncthreads();
   // bitonic sort, descending (best first); padding keys (0) sink to the end
   for (int kk = 2; kk <= npow; kk <<= 1) {
@@ -90,39 +86,100 @@ __global__ void __launch_bounds__(kCutThreads) cutoff_kernel(const float* __rest
       __syncthreads();
     }
   }
-  if (tid != 0) return;
-  // best-first walk; T = K-th smallest position among the tokens seen so far
+  // the positions in best-first order, for the walk
+  int32_t* ou = order + static_cast<size_t>(u) * ne;
+  for (int r = tid; r < ne; r += blockDim.x) ou[r] = static_cast<int>(0xffffffffu - static_cast<uint32_t>(keys[r]));
+}
+
+// Best-first walk of one unit per warp: T = the K-th smallest position
+// among the tokens seen so far; c_j = "never" for the first K, else
+// max(j, T) before j is inserted (j below T moves T to its predecessor in a
+// bitmap of inserted positions).  The warp takes 32 tokens at a time (lane i
+// = the i-th best of the batch; the next batch's positions load meanwhile):
+// the first K set their bits and raise T together; after them the tokens at
+// or above T change nothing, so one ballot finds the next one below T, the
+// tokens before it take c = their own position, and only that one is
+// inserted (a predecessor not in T's word is found 32 words at a time by
+// ballot).  The batch's cutoffs are stored at once.
+constexpr int kWalkWarps = 4;
+__global__ void __launch_bounds__(32 * kWalkWarps) walk_kernel(const int32_t* __restrict__ order,
+                                                               int32_t* __restrict__ cut, int n, int ne, int words,
+                                                               int S, int K, int units, uint32_t* bits_g,
+                                                               int bits_global, int32_t* err) {
+  extern __shared__ __align__(16) uint32_t bsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * kWalkWarps + warp;
+  if (u >= units || ne == 0) return;
+  uint32_t* bits = bits_global ? bits_g + static_cast<size_t>(u) * words : bsm + static_cast<size_t>(warp) * words;
+  for (int i = lane; i < words; i += 32) bits[i] = 0u;
+  __syncwarp();
+  const int32_t* ord = order + static_cast<size_t>(u) * ne;
+  int32_t* cu = cut + static_cast<size_t>(u) * n;
   int T = -1;
   bool bad = false;
-  for (int r = 0; r < ne; ++r) {
-    const int pos = static_cast<int>(0xffffffffu - static_cast<uint32_t>(keys[r]));
-    int c;
-    if (K == 0) {
-      c = pos;
-    } else if (r < K) {
-      c = kNever;
-      T = max(T, pos);
-      const int idx = pos - S;
-      bits[idx >> 5] |= 1u << (idx & 31);
-    } else {
-      c = max(pos, T);
-      if (pos < T) {
-        const int idx = pos - S;
-        bits[idx >> 5] |= 1u << (idx & 31);
-        const int ti = T - S;
-        int w = ti >> 5;
-        uint32_t m = bits[w] & ((1u << (ti & 31)) - 1u);
-        while (m == 0u && w > 0) m = bits[--w];
-        if (m == 0u) {  // cannot happen: pos < T was just inserted
-          bad = true;
-          break;
+  int cur = lane < ne ? ord[lane] : 0;
+  for (int r0 = 0; r0 < ne && !bad; r0 += 32) {
+    const int nxt = r0 + 32 + lane < ne ? ord[r0 + 32 + lane] : 0;   // the next batch, in flight meanwhile
+    const int lim = min(32, ne - r0);
+    const bool valid = lane < lim;
+    int myc = cur;   // K = 0: c = j
+    if (K > 0) {
+      // the batch's tokens among the first K: "never", their bits set, T = max
+      const bool first_k = valid && r0 + lane < K;
+      if (__any_sync(0xffffffffu, first_k)) {
+        if (first_k) {
+          const int idx = cur - S;
+          atomicOr(&bits[idx >> 5], 1u << (idx & 31));
+          myc = kNever;
         }
-        T = S + (w << 5) + 31 - __clz(m);
+        int tm = first_k ? cur : -1;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tm = max(tm, __shfl_xor_sync(0xffffffffu, tm, o));
+        T = max(T, tm);
+        __syncwarp();
+      }
+      // the rest in best-first order: up to the next token below T, c = max(j, T) = j
+      int x = r0 >= K ? 0 : K - r0;
+      while (x < lim) {
+        const uint32_t below = __ballot_sync(0xffffffffu, valid && lane >= x && cur < T);
+        const int xi = below != 0u ? __ffs(below) - 1 : lim;
+        if (lane >= x && lane < xi) myc = max(cur, T);
+        if (xi == lim) break;
+        // token xi is below T: c = T, insert it, T moves to its predecessor
+        const int pos = __shfl_sync(0xffffffffu, cur, xi);
+        if (lane == xi) myc = T;
+        const int idx = pos - S;
+        if (lane == 0) bits[idx >> 5] |= 1u << (idx & 31);
+        __syncwarp();
+        const int ti = T - S;
+        const int w = ti >> 5;
+        const uint32_t m = bits[w] & ((1u << (ti & 31)) - 1u);
+        if (m != 0u) {
+          T = S + (w << 5) + 31 - __clz(m);
+        } else {
+          bool found = false;
+          for (int base = w - 1; base >= 0 && !found; base -= 32) {
+            const int wi = base - lane;
+            const uint32_t bv = wi >= 0 ? bits[wi] : 0u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, bv != 0u);
+            if (bal != 0u) {
+              const int l = __ffs(bal) - 1;   // the lowest lane holds the highest word
+              T = S + ((base - l) << 5) + 31 - __clz(__shfl_sync(0xffffffffu, bv, l));
+              found = true;
+            }
+          }
+          if (!found) {   // cannot happen: pos < T was just inserted
+            bad = true;
+            break;
+          }
+        }
+        x = xi + 1;
       }
     }
-    cu[pos] = c;
+    if (!bad && valid) cu[cur] = myc;
+    cur = nxt;
   }
-  if (bad) set_error(err, DEVERR_STATE_MISMATCH);
+  if (bad && lane == 0) set_error(err, DEVERR_STATE_MISMATCH);
 }
 
 // ---------------- attention: one CTA per (query tile, unit) ----------------
@@ -1456,6 +1513,8 @@ int plan_prefill_attention(const LayerArgs& a, int dtype, int n, PrefillAttnPlan
   off += al(units * max(n, 1) * sizeof(int32_t));
   P.score_off = off;
   off += al(units * max(P.ne, 1) * sizeof(float));
+  P.order_off = off;
+  off += al(units * max(P.ne, 1) * sizeof(int32_t));
   P.keys_off = off;
   if (P.keys_global) off += al(units * P.npow * sizeof(uint64_t));
   P.bits_off = off;
@@ -1474,19 +1533,24 @@ int launch_prefill_attention(const LayerArgs& a, int dtype, const PrefillAttnPla
   float* scores = reinterpret_cast<float*>(workspace + p.score_off);
   uint64_t* keys = reinterpret_cast<uint64_t*>(workspace + p.keys_off);
   uint32_t* bits = reinterpret_cast<uint32_t*>(workspace + p.bits_off);
+  int32_t* order = reinterpret_cast<int32_t*>(workspace + p.order_off);
   if (!reuse_cutoffs && p.ne > 0) {
     const int r = launch_prompt_scores(a, dtype, k, v, p.n, ext, scores, p.ne, st);
     if (r != 0) return r;
   }
   if (!reuse_cutoffs) {
-    const size_t cut_smem = (p.keys_global ? 0 : static_cast<size_t>(p.npow) * 8) +
-                            (p.bits_global ? 0 : static_cast<size_t>(p.words) * 4);
-    if (cudaFuncSetAttribute(cutoff_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kPaSmemSortKeys * 8 + kPaSmemBitmapWords * 4) != cudaSuccess)
+    const size_t cut_smem = p.keys_global ? 0 : static_cast<size_t>(p.npow) * 8;
+    if (cudaFuncSetAttribute(cutoff_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPaSmemSortKeys * 8) !=
+        cudaSuccess)
       return -1;
-    cutoff_kernel<<<a.units, kCutThreads, cut_smem, st>>>(scores, max(p.ne, 1), cut, p.n, p.ne, p.npow, p.words,
-                                                          a.S, a.K, keys, bits, p.keys_global ? 1 : 0,
-                                                          p.bits_global ? 1 : 0, a.err);
+    cutoff_kernel<<<a.units, kCutThreads, cut_smem, st>>>(scores, max(p.ne, 1), cut, order, p.n, p.ne, p.npow, a.S,
+                                                          keys, p.keys_global ? 1 : 0);
+    const size_t walk_smem = p.bits_global ? 0 : static_cast<size_t>(kWalkWarps) * p.words * 4;
+    if (cudaFuncSetAttribute(walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kWalkWarps * kPaSmemBitmapWords * 4) != cudaSuccess)
+      return -1;
+    walk_kernel<<<(a.units + kWalkWarps - 1) / kWalkWarps, 32 * kWalkWarps, walk_smem, st>>>(
+        order, cut, p.n, p.ne, p.words, a.S, a.K, a.units, bits, p.bits_global ? 1 : 0, a.err);
   }
   PaArgs pa;
   pa.q = q;

@@ -31,7 +31,7 @@ struct PrefillAttnPlan {
   int words;        // bitmap words: (ne + 31) / 32, at least 1
   int qt;           // query positions per attention CTA: 64 / G (fp32) or 256 / G (bf16)
   int cand_cap;     // candidate keys of one CTA at most: S + K + qt + W + D
-  size_t cut_off, score_off, keys_off, bits_off, total;   // workspace layout (bytes)
+  size_t cut_off, score_off, order_off, keys_off, bits_off, total;   // workspace layout (bytes)
   bool keys_global, bits_global;
 };
 
