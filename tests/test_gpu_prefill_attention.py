@@ -298,8 +298,8 @@ def test_cutoffs_sorted_in_the_workspace():
 
 
 def test_cutoffs_with_the_bitmap_in_the_workspace():
-    """More than 131,072 eligible tokens in a unit: cutoff_kernel keeps both
-    the sort keys and the position bitmap in the workspace.  One unit of
+    """More than 131,072 eligible tokens in a unit: the sort keys (cutoff_kernel)
+    and the walk's position bitmap (walk_kernel) both live in the workspace.  One unit of
     131,594 prompt tokens (131,572 eligible), fp32 d 64 G 2, S 4 + W 16 +
     D 2 + K 300, the library's MLP scorer."""
     _need_gpu()
