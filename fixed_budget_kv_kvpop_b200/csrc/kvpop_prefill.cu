@@ -21,6 +21,8 @@
 //              assignment by block prefix sums and row copies.
 //   P3 move:   window tokens that enter the staging ring move there.
 //   P4 write:  chunk tokens go to their sink / window / staging slots.
+#include <type_traits>
+
 #include "kvpop_internal.cuh"
 #include "kvpop_prefill_attn.cuh"
 
@@ -314,6 +316,179 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
   }
 }
 
+// score64_kernel for bf16 inputs, with each tile's rows copied while the
+// tile before is computed.  The rows land by cp.async as they are (bf16
+// pairs in 32-bit words, two buffers of TT rows) and are widened to fp64 as
+// the fragments are loaded, so no thread waits for a tile's loads or
+// converts it in shared memory.  W1 is kept transposed with the two inputs
+// of each pair side by side (one 8-byte load per fragment serves two MMAs);
+// in pass p0 lane (gr, gc) holds inputs 2 (p0 + gc) and 2 (p0 + gc) + 1 of
+// its A row and B column, and the two MMAs of the pass take the first and
+// the second of them: the same products, summed over the same inputs, as
+// score64_kernel.  Row pitches: XW = 4 (mod 32) words and WP2 = 4 (mod 16)
+// pairs keep every fragment load conflict-free.
+template <int D2, int HID>
+struct Score64BGeom {
+  static constexpr int TT = 128;
+  static constexpr int XW = D2 / 2 + 4;                       // 32-bit words per token row (16-byte multiple)
+  static constexpr int WP2 = HID + 4;                         // float pairs per pair row of W1^T
+  static constexpr size_t XBUF = static_cast<size_t>(TT) * XW * 4;
+  static constexpr size_t W_OFF = 2 * XBUF;
+  static constexpr size_t PP_OFF = W_OFF + static_cast<size_t>(D2 / 2) * WP2 * 8;
+  static constexpr size_t SMEM = PP_OFF + static_cast<size_t>(kScore64Parts) * TT * 8;
+  static_assert((XW * 4) % 16 == 0 && XW % 32 == 4 && WP2 % 16 == 4, "row pitches");
+};
+
+__device__ __forceinline__ void score_cp16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+template <int D2, int HID>
+__global__ void __launch_bounds__(kScore64Threads, 1) score64_bf16_kernel(LayerArgs a, ChunkGeom cg,
+                                                                          const __nv_bfloat16* __restrict__ k,
+                                                                          const __nv_bfloat16* __restrict__ v,
+                                                                          int n, float* __restrict__ out, int cap) {
+  using SG = Score64BGeom<D2, HID>;
+  using T = __nv_bfloat16;
+  constexpr int TT = SG::TT, XW = SG::XW, WP2 = SG::WP2;
+  constexpr int HS = kScore64Parts;
+  constexpr int NT = HID / (8 * HS);                            // column tiles of this warp's hidden part
+  static_assert(NT >= 1 && HID % (8 * HS) == 0, "whole column tiles per part");
+  constexpr int UPT = D2 / 8;                                   // 16-byte chunks per token row
+  constexpr int CPT = TT * UPT / kScore64Threads;               // chunks per thread per tile
+  static_assert(CPT >= 1 && CPT * kScore64Threads == TT * UPT, "whole chunks per thread");
+  extern __shared__ __align__(16) uint8_t smb[];
+  const uint32_t* Xw = reinterpret_cast<const uint32_t*>(smb);  // [buf][TT][XW]: bf16 pairs of x_t
+  float2* Wt2 = reinterpret_cast<float2*>(smb + SG::W_OFF);     // [D2 / 2][WP2]: (W1[j][2p], W1[j][2p + 1])
+  double* pp = reinterpret_cast<double*>(smb + SG::PP_OFF);     // [part][TT] partial sums
+  const int u = blockIdx.y;
+  const int h = u % a.Hkv;
+  const int n_new = cg.e1 - cg.e0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile0 = blockIdx.x * kTilesPerBlock;
+  const int ntile = min(kTilesPerBlock, (n_new + TT - 1) / TT - tile0);
+  if (ntile <= 0) return;
+  const uint32_t xs0 = smem_u32(smb);
+
+  // a tile's rows into buffer b: thread -> chunks tid + x * threads (chunk c
+  // of token tt = inputs 8 c .. 8 c + 7, from k for the first half of the
+  // row, v for the second); tokens past the chunk's end are zero-filled
+  auto issue = [&](int tile, int b) {
+    const int tok0 = tile * TT;
+#pragma unroll
+    for (int x = 0; x < CPT; ++x) {
+      const int e = tid + x * kScore64Threads;
+      const int tt = e / UPT, c = e % UPT;
+      const void* src = k;
+      int bytes = 0;
+      if (tok0 + tt < n_new) {
+        const uint8_t* vs;
+        const uint8_t* ks = token_row<T>(a, cg, u, cg.e0 + tok0 + tt, k, v, n, vs);
+        const int i0 = c * 8;
+        src = (i0 < D2 / 2) ? ks + i0 * sizeof(T) : vs + (i0 - D2 / 2) * sizeof(T);
+        bytes = 16;
+      }
+      score_cp16(xs0 + static_cast<uint32_t>(b * SG::XBUF + (static_cast<size_t>(tt) * XW + c * 4) * 4), src, bytes);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  issue(tile0, 0);
+
+  {
+    // W1 [HID][D2] -> Wt2 while the first tile is in flight: thread -> hidden
+    // j = e % HID, inputs 4 q .. 4 q + 3 with q = e / HID (pairs 2 q, 2 q + 1)
+    const float* w1 = a.w1 + static_cast<size_t>(h) * HID * D2;
+    constexpr int WL = HID * D2 / 4 / kScore64Threads;          // float4 loads per thread
+    static_assert(WL >= 1 && WL * kScore64Threads == HID * D2 / 4, "whole loads per thread");
+    float4 wv[WL];
+#pragma unroll
+    for (int x = 0; x < WL; ++x) {
+      const int e = tid + x * kScore64Threads;
+      wv[x] = __ldg(reinterpret_cast<const float4*>(w1 + static_cast<size_t>(e % HID) * D2) + e / HID);
+    }
+#pragma unroll
+    for (int x = 0; x < WL; ++x) {
+      const int e = tid + x * kScore64Threads;
+      float2* dst = Wt2 + (2 * (e / HID)) * WP2 + e % HID;
+      dst[0] = make_float2(wv[x].x, wv[x].y);
+      dst[WP2] = make_float2(wv[x].z, wv[x].w);
+    }
+  }
+  const int gr = lane >> 2, gc = lane & 3;                      // fragment row / column within a tile
+  const int tg = warp & 3, hh = warp >> 2;                      // token group, hidden part
+  const int j0 = hh * (HID / HS);
+  // this lane's hidden units in the accumulators: j0 + 8 c + 2 gc + {0, 1}, c < NT
+  double b1v[NT][2], w2v[NT][2];
+#pragma unroll
+  for (int c = 0; c < NT; ++c)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      b1v[c][e] = static_cast<double>(a.b1[static_cast<size_t>(h) * HID + j0 + 8 * c + 2 * gc + e]);
+      w2v[c][e] = static_cast<double>(a.w2[static_cast<size_t>(h) * HID + j0 + 8 * c + 2 * gc + e]);
+    }
+  const double b2 = static_cast<double>(a.b2[h]);
+
+  for (int i = 0; i < ntile; ++i) {
+    const int tok0 = (tile0 + i) * TT;
+    if (i + 1 < ntile) issue(tile0 + i + 1, (i + 1) & 1);      // its buffer was last read before the barrier below
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");       // this tile's rows (and only the next tile's in flight)
+    __syncthreads();                                            // every thread's rows (and W1) visible
+    double acc[4][NT][2];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int c = 0; c < NT; ++c) acc[m][c][0] = acc[m][c][1] = 0.0;
+    const uint32_t* xa = Xw + (i & 1) * TT * XW + (32 * tg + gr) * XW + gc;   // A: row gr of tile m at + 8 m XW
+    const float2* wb = Wt2 + gc * WP2 + j0 + gr;                // B: pair row p0 + gc, hidden j0 + 8 c + gr
+#pragma unroll 2
+    for (int p0 = 0; p0 < D2 / 2; p0 += 4) {
+      uint32_t aw[4];
+      float2 bw[NT];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) aw[m] = xa[8 * m * XW + p0];
+#pragma unroll
+      for (int c = 0; c < NT; ++c) bw[c] = wb[p0 * WP2 + 8 * c];
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        double af[4], bf[NT];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          af[m] = static_cast<double>(__uint_as_float(s == 0 ? aw[m] << 16 : aw[m] & 0xffff0000u));
+#pragma unroll
+        for (int c = 0; c < NT; ++c) bf[c] = static_cast<double>(s == 0 ? bw[c].x : bw[c].y);
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+          for (int c = 0; c < NT; ++c) dmma_8x8x4(acc[m][c], af[m], bf[c]);
+      }
+    }
+    // w2 . relu(W1 x + b1) over this warp's hidden part: this lane holds
+    // tokens 32 tg + 8 m + gr, 2 NT hidden units each
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      double part = 0.0;
+#pragma unroll
+      for (int c = 0; c < NT; ++c)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) part = fma(w2v[c][e], fmax(acc[m][c][e] + b1v[c][e], 0.0), part);
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      if (gc == 0) pp[hh * TT + 32 * tg + 8 * m + gr] = part;
+    }
+    __syncthreads();   // pp complete; every read of this tile's buffer done
+    // the parts in a fixed order, + b2, one token per thread
+    if (tid < TT && tok0 + tid < n_new) {
+      double sum = pp[tid];
+#pragma unroll
+      for (int q = 1; q < HS; ++q) sum += pp[q * TT + tid];
+      out[static_cast<size_t>(u) * cap + tok0 + tid] =
+          ranking_priority(a, u, cg.e0 + tok0 + tid + a.W + a.D, static_cast<float>(sum + b2));
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // P1 with the stateless headwise linear scorer (page §E.2), s = w . [k; v] + b:
 // one warp per token, the weight row in registers, fp64 dot product.
 constexpr int kLinearThreads = 256;
@@ -539,14 +714,24 @@ __global__ void write_kernel(LayerArgs a, ChunkGeom cg, const T* __restrict__ k,
 template <typename T, int D2, int HID>
 int launch_score64(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T* v, int n, float* out, int cap,
                    int n_new, cudaStream_t st) {
-  using SG = Score64Geom<D2, HID>;
-  // set on every call: the attribute belongs to the current device
-  if (cudaFuncSetAttribute(score64_kernel<T, D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM) !=
-      cudaSuccess)
-    return -1;
-  const int tiles = (n_new + SG::TT - 1) / SG::TT;
-  dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
-  score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap);
+  // the shared-memory attribute is set on every call: it belongs to the current device
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    using SG = Score64BGeom<D2, HID>;
+    if (cudaFuncSetAttribute(score64_bf16_kernel<D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(SG::SMEM)) != cudaSuccess)
+      return -1;
+    const int tiles = (n_new + SG::TT - 1) / SG::TT;
+    dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
+    score64_bf16_kernel<D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap);
+  } else {
+    using SG = Score64Geom<D2, HID>;
+    if (cudaFuncSetAttribute(score64_kernel<T, D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM) !=
+        cudaSuccess)
+      return -1;
+    const int tiles = (n_new + SG::TT - 1) / SG::TT;
+    dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
+    score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap);
+  }
   return 0;
 }
 
