@@ -64,6 +64,7 @@ struct LaunchShape {
   static constexpr int NSTG = 2;
   static constexpr int NDW = sizeof(T) == 2 ? 4 : 2;
 };
+constexpr int kMaxDeciders = 8;   // decider warps per CTA at most (team slots in shared memory)
 // Tiles per consumer warp prefetched into L2 before the wait for the previous kernel.
 constexpr int kPrefetchTiles = 2;
 
@@ -109,7 +110,8 @@ struct Smem {
   static constexpr int QRAW = P + NCW * GE::PBYTES;
   static constexpr int MQ = QRAW + NCW * 2 * QRB;
   static constexpr int BAR = MQ + (kMergeCap + 4) * 4;
-  static constexpr int TOTAL = BAR + NCW * (NSTG + 2) * 8;
+  static constexpr int TEAM = BAR + NCW * (NSTG + 2) * 8;             // the deciders' parts (decide_finish in teams)
+  static constexpr int TOTAL = TEAM + kMaxDeciders * 24;
   static_assert(GE::STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(Q % 16 == 0 && P % 16 == 0 && QRAW % 16 == 0 && QRB % 16 == 0 && MQ % 16 == 0 &&
                     BAR % 8 == 0,
@@ -173,18 +175,16 @@ template <typename T>
 __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, int ntk, const Decision* pending,
                                 const T* kn, const T* vn, float ext_new) {
   const int lane = threadIdx.x & 31;
-  const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
+  const int S = a.S, W = a.W, D = a.D, NS = a.NS;
   Decision r;
   r.p = N; r.bpos = -1; r.bslot = -1; r.tgt = -1; r.evict = -1; r.sb = 0.f; r.pad[0] = r.pad[1] = 0;
   const int b = N - W - D;
   if (b < S) return r;
-  const int base = topk_base(S, W, D);
   const T* kv = reinterpret_cast<const T*>(a.kv + static_cast<size_t>(u) * NS * a.row_bytes);
   const int32_t* pos = a.pos + static_cast<size_t>(u) * NS;
   const float* score = a.score + static_cast<size_t>(u) * NS;
   r.bpos = b;
   r.bslot = (D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D);
-  constexpr int kB = 16;   // long-range keys per lane per round trip
   // where b's row is now
   const T* krow;
   bool from_input = false;
@@ -253,13 +253,37 @@ __device__ __noinline__ void decide_load(const LayerArgs& a, int u, int N, const
     set_error(a.err, DEVERR_STATE_MISMATCH);
 }
 
+// decide_finish: the decision from what decide_load read, taken by one warp
+// (nteam = 1) or by the nteam decider warps of a CTA together (team index
+// dw), in launches where each CTA decides one unit at most.  Warp dw forms
+// the MLP terms of the hidden blocks [dw nb / nteam, (dw + 1) nb / nteam)
+// (nb = hidden / 16) and scans the dw-th of nteam equal parts of the
+// long-range keys, so a team pays one round trip of loads for each of the
+// two steps instead of several.  The parts meet in shared memory (named
+// barrier kDecideBar over the team): the MLP parts are summed in team order
+// and the partial minima compared (keys are unique), and every warp returns
+// the same decision.  A team sums the score's fp64 terms in another order
+// than one warp does; both round once to fp32.
+constexpr int kDecideBar = 1;
+struct DecideTeam {
+  double part;
+  unsigned long long best;
+  int slot, pad;
+};
+static_assert(sizeof(DecideTeam) == 24, "team slot size");
+
+__device__ __forceinline__ void team_bar_sync(int nthreads) {
+  asm volatile("bar.sync %0, %1;" :: "r"(kDecideBar), "r"(nthreads) : "memory");
+}
+
 template <int DH>
 __device__ __noinline__ Decision decide_finish(const LayerArgs& a, int u, int N, int ntk, const Decision* pending,
-                                               const DecideInput<DH>& in) {
+                                               const DecideInput<DH>& in, int dw, int nteam, DecideTeam* team) {
   Decision r;
   r.p = N; r.bpos = -1; r.bslot = -1; r.tgt = -1; r.evict = -1; r.sb = 0.f; r.pad[0] = r.pad[1] = 0;
-  if (in.b < 0) return r;
-  const int S = a.S, W = a.W, D = a.D;
+  if (in.b < 0) return r;   // the same in every warp of a team
+  const int lane = threadIdx.x & 31;
+  const int S = a.S, W = a.W, D = a.D, K = a.K;
   const int b = in.b;
   r.bpos = b;
   r.bslot = (D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D);
@@ -269,15 +293,57 @@ __device__ __noinline__ Decision decide_finish(const LayerArgs& a, int u, int N,
   } else {
     const int h = u % a.Hkv;
     const float* w1 = head_w1(a, h);
-    if (a.hidden == 0) sb = linear_score_x<2 * DH>(in.x, w1, a.b2[h]);
-    else if (a.hidden == 32) sb = mlp_score_x<2 * DH, 32>(in.x, w1, head_b1(a, h), head_w2(a, h), a.b2[h]);
-    else if (a.hidden == 64) sb = mlp_score_x<2 * DH, 64>(in.x, w1, head_b1(a, h), head_w2(a, h), a.b2[h]);
-    else sb = mlp_score_x<2 * DH, 128>(in.x, w1, head_b1(a, h), head_w2(a, h), a.b2[h]);
+    if (a.hidden == 0) {
+      sb = linear_score_x<2 * DH>(in.x, w1, a.b2[h]);
+    } else {
+      const int nb = a.hidden / 16;
+      const int j0 = 16 * (dw * nb / nteam), j1 = 16 * ((dw + 1) * nb / nteam);
+      double part;
+      if (a.hidden == 32) part = mlp_part_x<2 * DH, 32>(in.x, w1, head_b1(a, h), head_w2(a, h), j0, j1);
+      else if (a.hidden == 64) part = mlp_part_x<2 * DH, 64>(in.x, w1, head_b1(a, h), head_w2(a, h), j0, j1);
+      else part = mlp_part_x<2 * DH, 128>(in.x, w1, head_b1(a, h), head_w2(a, h), j0, j1);
+      if (nteam > 1) {
+        if (lane == 0) team[dw].part = part;
+        team_bar_sync(nteam * 32);
+        part = 0.0;
+        for (int t = 0; t < nteam; ++t) part += team[t].part;
+      }
+      sb = static_cast<float>(part + static_cast<double>(a.b2[h]));
+    }
   }
   sb = ranking_priority(a, u, N, sb);   // b becomes eligible at step b + W + D = N
   r.sb = sb;
-  if ((a.flags & FLAG_DEBUG_CHECKS) && (threadIdx.x & 31) == 0 && sb != sb) set_error(a.err, DEVERR_NAN_SCORE);
-  longrange_decide(a, u, ntk, pending, sb, b, r);
+  if ((a.flags & FLAG_DEBUG_CHECKS) && dw == 0 && lane == 0 && sb != sb) set_error(a.err, DEVERR_NAN_SCORE);
+  const int base = topk_base(S, W, D);
+  if (ntk < K) {
+    r.tgt = base + ntk;     // fill-up: next free long-range slot, nobody leaves
+    r.evict = -1;
+  } else if (K == 0) {
+    r.evict = r.bslot;
+  } else {
+    const int q = (K + nteam - 1) / nteam;
+    int mslot;
+    uint64_t best = longrange_min(a, u, pending, min(K, dw * q), min(K, (dw + 1) * q), mslot);
+    if (nteam > 1) {
+      if (lane == 0) {
+        team[dw].best = best;
+        team[dw].slot = mslot;
+      }
+      team_bar_sync(nteam * 32);
+      best = ~0ull;
+      for (int t = 0; t < nteam; ++t) {
+        const uint64_t k = team[t].best;
+        if (k < best) { best = k; mslot = team[t].slot; }
+      }
+    }
+    if (rank_key(sb, b) > best) {
+      r.tgt = mslot;
+      r.evict = mslot;
+    } else {
+      r.evict = r.bslot;
+    }
+  }
+  if (nteam > 1) team_bar_sync(nteam * 32);   // every warp has read the slots: free for the next unit
   return r;
 }
 
@@ -527,7 +593,9 @@ __device__ __forceinline__ void l2_warmup(const LayerArgs& a, bool step, int war
   const int dw = warp - NCW;
   const int base = topk_base(S, W, D);
   const int b = N + 1 - W - D;   // boundary token of the decision taken in this launch
-  for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
+  const bool team = a.units <= static_cast<int>(gridDim.x);   // as the deciders split their units
+  if (team && dw != 0) return;
+  for (int u = team ? blockIdx.x : blockIdx.x * NDW + dw; u < a.units; u += team ? gridDim.x : gridDim.x * NDW) {
     if (K > 0) {
       // [lo, hi) byte range of the unit's long-range scores / positions, in 16-byte units
       const int64_t lo = (static_cast<int64_t>(u) * NS + base) * 4 / 16 * 16;
@@ -706,22 +774,34 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
 
   if (warp >= NCW) {
     // ---------------- deciders, then merge helpers ----------------
+    static_assert(NDW <= kMaxDeciders, "team slots");
     if (step) {
       const int dw = warp - NCW;
-      for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
+      // with at most one unit per CTA, the CTA's decider warps take it together
+      const bool team = a.units <= static_cast<int>(gridDim.x);
+      const bool lead = !team || dw == 0;   // the warp that arrives and stores the decision
+      DecideTeam* team_sm = reinterpret_cast<DecideTeam*>(smem + SM::TEAM);
+      for (int u = team ? blockIdx.x : blockIdx.x * NDW + dw; u < a.units;
+           u += team ? gridDim.x : gridDim.x * NDW) {
         if (mode == MODE_STEP) {   // MODE_STEP_NODECIDE: the next step's kernel decides
           const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
           DecideInput<DH> din;
           decide_load<T, DH>(a, u, N + 1, k_new + static_cast<size_t>(u) * DH, v_new + static_cast<size_t>(u) * DH,
                              ext ? ext[u] : 0.f, din);
-          const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
-          if (prev == need_of(u) - 1) push_merge(u);
-          const Decision nx = decide_finish<DH>(a, u, N + 1, ntk_after, &cur, din);
-          if (lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
+          if (team) team_bar_sync(NDW * 32);   // every warp holds the row before the merge may overwrite it
+          if (lead) {
+            const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
+            if (prev == need_of(u) - 1) push_merge(u);
+          }
+          const Decision nx = decide_finish<DH>(a, u, N + 1, ntk_after, &cur, din, team ? dw : 0, team ? NDW : 1,
+                                                team_sm);
+          if (lead && lane == 0) a.dec[static_cast<size_t>((N + 1) & 1) * a.units + u] = nx;
           continue;
         }
-        const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
-        if (prev == need_of(u) - 1) push_merge(u);
+        if (lead) {
+          const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
+          if (prev == need_of(u) - 1) push_merge(u);
+        }
       }
     }
     help();

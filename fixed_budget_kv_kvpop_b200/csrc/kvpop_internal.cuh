@@ -301,15 +301,16 @@ __device__ __forceinline__ void load_scorer_input(const T* krow, const T* vrow, 
 // the warp reads the whole W1 row (coalesced: 4 cache lines per instruction),
 // each lane forms its X-term partial sum, and a butterfly reduction over 16
 // rows at a time leaves lane l (< 16) with the pre-activation of row
-// 16 * block + l.
+// 16 * block + l.  mlp_part_x sums w2_j relu(.) over the hidden rows
+// [j0, j1) (whole blocks of 16) and returns it in every lane, without b2.
 template <int D2, int HID>
-__device__ __forceinline__ float mlp_score_x(const double (&x)[D2 / 32], const float* w1, const float* b1,
-                                             const float* w2, float b2) {
+__device__ __forceinline__ double mlp_part_x(const double (&x)[D2 / 32], const float* w1, const float* b1,
+                                             const float* w2, int j0, int j1) {
   constexpr int X = D2 / 32;
   const int lane = threadIdx.x & 31;
   const int i0 = lane * X;
   double part = 0.0;
-  for (int blk = 0; blk < HID; blk += 16) {
+  for (int blk = j0; blk < j1; blk += 16) {
     // b1 and w2 of the row this lane finishes, issued with the block's W1 loads
     const float b1j = (lane < 16) ? __ldg(b1 + blk + lane) : 0.f;
     const float w2j = (lane < 16) ? __ldg(w2 + blk + lane) : 0.f;
@@ -347,7 +348,13 @@ __device__ __forceinline__ float mlp_score_x(const double (&x)[D2 / 32], const f
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  return static_cast<float>(part + static_cast<double>(b2));
+  return part;
+}
+
+template <int D2, int HID>
+__device__ __forceinline__ float mlp_score_x(const double (&x)[D2 / 32], const float* w1, const float* b1,
+                                             const float* w2, float b2) {
+  return static_cast<float>(mlp_part_x<D2, HID>(x, w1, b1, w2, 0, HID) + static_cast<double>(b2));
 }
 
 template <typename T, int D2, int HID>
@@ -406,45 +413,30 @@ __device__ __noinline__ float mlp_score_warp(const T* krow, const T* vrow, int d
   return mlp_score_rows<T, 128, 128>(krow, vrow, w1, b1, w2, b2);
 }
 
-// Eviction decision against the long-range set, taken by one warp for the
-// boundary token b (ranking priority sb) of unit u; r.bslot is set.  While
-// fewer than K long-range slots are used (ntk < K), b takes the next free
-// one.  Otherwise the warp finds the minimum key (score, -position) of the
-// long-range slots and b replaces it only if its own key is strictly larger;
-// else b is dropped.  pending: the previous step's decision when it is not
-// yet committed (its target slot then counts with pending's key), or null.
-// Keys are unique (positions are), so the argmin is unique.
-__device__ __forceinline__ void longrange_decide(const LayerArgs& a, int u, int ntk, const Decision* pending,
-                                                 float sb, int b, Decision& r) {
+// Minimum key (score, -position) of the long-range slots base + [i_lo, i_hi)
+// (pending's target counting with pending's key), in every lane of the warp;
+// ~0 and slot -1 for an empty range.
+__device__ __forceinline__ uint64_t longrange_min(const LayerArgs& a, int u, const Decision* pending, int i_lo,
+                                                  int i_hi, int& mslot) {
   const int lane = threadIdx.x & 31;
-  const int K = a.K;
   const int base = topk_base(a.S, a.W, a.D);
   const int32_t* pos = a.pos + static_cast<size_t>(u) * a.NS;
   const float* score = a.score + static_cast<size_t>(u) * a.NS;
-  if (ntk < K) {
-    r.tgt = base + ntk;     // fill-up: next free long-range slot, nobody leaves
-    r.evict = -1;
-    return;
-  }
-  if (K == 0) {
-    r.evict = r.bslot;
-    return;
-  }
   constexpr int kB = 16;   // long-range keys per lane per round trip
   uint64_t best = ~0ull;
-  int mslot = -1;
-  for (int i0 = 0; i0 < K; i0 += 32 * kB) {
+  mslot = -1;
+  for (int i0 = i_lo; i0 < i_hi; i0 += 32 * kB) {
     float sc[kB];
     int32_t ps[kB];
 #pragma unroll
     for (int t = 0; t < kB; ++t) {
       const int i = i0 + lane + 32 * t;
-      if (i < K) { sc[t] = score[base + i]; ps[t] = pos[base + i]; }
+      if (i < i_hi) { sc[t] = score[base + i]; ps[t] = pos[base + i]; }
     }
 #pragma unroll
     for (int t = 0; t < kB; ++t) {
       const int i = i0 + lane + 32 * t;
-      if (i < K) {
+      if (i < i_hi) {
         const int sl = base + i;
         const uint64_t key = (pending != nullptr && sl == pending->tgt) ? rank_key(pending->sb, pending->bpos)
                                                                         : rank_key(sc[t], ps[t]);
@@ -458,6 +450,32 @@ __device__ __forceinline__ void longrange_decide(const LayerArgs& a, int u, int 
     const int os = __shfl_xor_sync(0xffffffffu, mslot, o);
     if (ok < best) { best = ok; mslot = os; }
   }
+  return best;
+}
+
+// Eviction decision against the long-range set, taken by one warp for the
+// boundary token b (ranking priority sb) of unit u; r.bslot is set.  While
+// fewer than K long-range slots are used (ntk < K), b takes the next free
+// one.  Otherwise the warp finds the minimum key (score, -position) of the
+// long-range slots and b replaces it only if its own key is strictly larger;
+// else b is dropped.  pending: the previous step's decision when it is not
+// yet committed (its target slot then counts with pending's key), or null.
+// Keys are unique (positions are), so the argmin is unique.
+__device__ __forceinline__ void longrange_decide(const LayerArgs& a, int u, int ntk, const Decision* pending,
+                                                 float sb, int b, Decision& r) {
+  const int K = a.K;
+  const int base = topk_base(a.S, a.W, a.D);
+  if (ntk < K) {
+    r.tgt = base + ntk;     // fill-up: next free long-range slot, nobody leaves
+    r.evict = -1;
+    return;
+  }
+  if (K == 0) {
+    r.evict = r.bslot;
+    return;
+  }
+  int mslot;
+  const uint64_t best = longrange_min(a, u, pending, 0, K, mslot);
   if (rank_key(sb, b) > best) {
     r.tgt = mslot;
     r.evict = mslot;

@@ -163,10 +163,26 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(LayerArgs a, Chunk
 // latency.  The epilogue forms w2 . relu(. + b1) over the warp's part per
 // token, sums the 4 lanes of each row by shuffles and the HS parts in a
 // fixed order through shared memory.  Each block keeps W1 resident and walks
-// kTilesPerBlock token tiles of its unit.
+// tpb consecutive token tiles of its unit (score64_tiles_per_block).
 constexpr int kScore64Threads = 512;
 constexpr int kScore64Parts = kScore64Threads / 128;   // HS: hidden parts, one warp each per token group
-constexpr int kTilesPerBlock = 8;
+
+// Tiles per block: the split of each unit's tiles into blocks that
+// minimises (waves of one-block-per-SM) x (tiles per block + the cost of a
+// block's start, about 0.15 of a tile: W1 and the first tile's rows).
+inline int score64_tiles_per_block(int tiles, int units, int nsm) {
+  if (tiles <= 0) return 1;
+  int best = tiles;
+  double best_cost = 1e300;
+  for (int c = 1; c <= tiles; ++c) {
+    const int tpb = (tiles + c - 1) / c;
+    if (c > 1 && tpb == (tiles + c - 2) / (c - 1)) continue;   // same split as c - 1
+    const long long blocks = static_cast<long long>(units) * ((tiles + tpb - 1) / tpb);
+    const double cost = static_cast<double>((blocks + nsm - 1) / nsm) * (tpb + 0.15);
+    if (cost < best_cost) { best_cost = cost; best = tpb; }
+  }
+  return best;
+}
 
 template <int D2, int HID>
 struct Score64Geom {
@@ -185,7 +201,7 @@ template <typename T, int D2, int HID>
 __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a, ChunkGeom cg,
                                                                      const T* __restrict__ k,
                                                                      const T* __restrict__ v, int n,
-                                                                     float* __restrict__ out, int cap) {
+                                                                     float* __restrict__ out, int cap, int tpb) {
   using SG = Score64Geom<D2, HID>;
   constexpr int TT = SG::TT, XP = SG::XP, WP = SG::WP;
   constexpr int HS = kScore64Parts;
@@ -201,7 +217,7 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
   const int h = u % a.Hkv;
   const int n_new = cg.e1 - cg.e0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile0 = blockIdx.x * kTilesPerBlock;
+  const int tile0 = blockIdx.x * tpb;
   if (tile0 * TT >= n_new) return;
 
   {
@@ -241,7 +257,7 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_kernel(LayerArgs a
     }
   const double b2 = static_cast<double>(a.b2[h]);
 
-  for (int tile = tile0; tile < tile0 + kTilesPerBlock && tile * TT < n_new; ++tile) {
+  for (int tile = tile0; tile < tile0 + tpb && tile * TT < n_new; ++tile) {
     const int tok0 = tile * TT;
     __syncthreads();   // W1 written (first tile) / previous tile's reads done
     // the tile's rows, up to 8 16-byte loads in flight per thread before any is stored
@@ -335,7 +351,7 @@ struct Score64BGeom {
   static constexpr size_t XBUF = static_cast<size_t>(TT) * XW * 4;
   static constexpr size_t W_OFF = 2 * XBUF;
   static constexpr size_t PP_OFF = W_OFF + static_cast<size_t>(D2 / 2) * WP2 * 8;
-  static constexpr size_t SMEM = PP_OFF + static_cast<size_t>(kScore64Parts) * TT * 8;
+  static constexpr size_t SMEM = PP_OFF + 2 * static_cast<size_t>(kScore64Parts) * TT * 8;
   static_assert((XW * 4) % 16 == 0 && XW % 32 == 4 && WP2 % 16 == 4, "row pitches");
 };
 
@@ -347,7 +363,8 @@ template <int D2, int HID>
 __global__ void __launch_bounds__(kScore64Threads, 1) score64_bf16_kernel(LayerArgs a, ChunkGeom cg,
                                                                           const __nv_bfloat16* __restrict__ k,
                                                                           const __nv_bfloat16* __restrict__ v,
-                                                                          int n, float* __restrict__ out, int cap) {
+                                                                          int n, float* __restrict__ out, int cap,
+                                                                          int tpb) {
   using SG = Score64BGeom<D2, HID>;
   using T = __nv_bfloat16;
   constexpr int TT = SG::TT, XW = SG::XW, WP2 = SG::WP2;
@@ -360,13 +377,13 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_bf16_kernel(LayerA
   extern __shared__ __align__(16) uint8_t smb[];
   const uint32_t* Xw = reinterpret_cast<const uint32_t*>(smb);  // [buf][TT][XW]: bf16 pairs of x_t
   float2* Wt2 = reinterpret_cast<float2*>(smb + SG::W_OFF);     // [D2 / 2][WP2]: (W1[j][2p], W1[j][2p + 1])
-  double* pp = reinterpret_cast<double*>(smb + SG::PP_OFF);     // [part][TT] partial sums
+  double* pp = reinterpret_cast<double*>(smb + SG::PP_OFF);     // [tile % 2][part][TT] partial sums
   const int u = blockIdx.y;
   const int h = u % a.Hkv;
   const int n_new = cg.e1 - cg.e0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile0 = blockIdx.x * kTilesPerBlock;
-  const int ntile = min(kTilesPerBlock, (n_new + TT - 1) / TT - tile0);
+  const int tile0 = blockIdx.x * tpb;
+  const int ntile = min(tpb, (n_new + TT - 1) / TT - tile0);
   if (ntile <= 0) return;
   const uint32_t xs0 = smem_u32(smb);
 
@@ -428,12 +445,26 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_bf16_kernel(LayerA
     }
   const double b2 = static_cast<double>(a.b2[h]);
 
-  for (int i = 0; i < ntile; ++i) {
+  // tile i's scores: the parts in a fixed order, + b2, one token per thread
+  auto finish = [&](int i) {
     const int tok0 = (tile0 + i) * TT;
-    if (i + 1 < ntile) issue(tile0 + i + 1, (i + 1) & 1);      // its buffer was last read before the barrier below
-    else asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 1;" ::: "memory");       // this tile's rows (and only the next tile's in flight)
-    __syncthreads();                                            // every thread's rows (and W1) visible
+    const double* q = pp + (i & 1) * HS * TT;
+    if (tid < TT && tok0 + tid < n_new) {
+      double sum = q[tid];
+#pragma unroll
+      for (int x = 1; x < HS; ++x) sum += q[x * TT + tid];
+      out[static_cast<size_t>(u) * cap + tok0 + tid] =
+          ranking_priority(a, u, cg.e0 + tok0 + tid + a.W + a.D, static_cast<float>(sum + b2));
+    }
+  };
+  for (int i = 0; i < ntile; ++i) {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");       // this tile's rows
+    // one barrier per tile: the rows (and W1) are visible, every thread is
+    // done reading the other buffer (tile i - 1) and has written its parts
+    // of tile i - 1, which are summed while tile i + 1's rows are copied
+    __syncthreads();
+    if (i > 0) finish(i - 1);
+    if (i + 1 < ntile) issue(tile0 + i + 1, (i + 1) & 1);
     double acc[4][NT][2];
 #pragma unroll
     for (int m = 0; m < 4; ++m)
@@ -474,18 +505,11 @@ __global__ void __launch_bounds__(kScore64Threads, 1) score64_bf16_kernel(LayerA
         for (int e = 0; e < 2; ++e) part = fma(w2v[c][e], fmax(acc[m][c][e] + b1v[c][e], 0.0), part);
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
-      if (gc == 0) pp[hh * TT + 32 * tg + 8 * m + gr] = part;
-    }
-    __syncthreads();   // pp complete; every read of this tile's buffer done
-    // the parts in a fixed order, + b2, one token per thread
-    if (tid < TT && tok0 + tid < n_new) {
-      double sum = pp[tid];
-#pragma unroll
-      for (int q = 1; q < HS; ++q) sum += pp[q * TT + tid];
-      out[static_cast<size_t>(u) * cap + tok0 + tid] =
-          ranking_priority(a, u, cg.e0 + tok0 + tid + a.W + a.D, static_cast<float>(sum + b2));
+      if (gc == 0) pp[(i & 1) * HS * TT + hh * TT + 32 * tg + 8 * m + gr] = part;
     }
   }
+  __syncthreads();
+  finish(ntile - 1);
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
@@ -715,22 +739,28 @@ template <typename T, int D2, int HID>
 int launch_score64(const LayerArgs& a, const ChunkGeom& cg, const T* k, const T* v, int n, float* out, int cap,
                    int n_new, cudaStream_t st) {
   // the shared-memory attribute is set on every call: it belongs to the current device
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+    return -1;
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
     using SG = Score64BGeom<D2, HID>;
     if (cudaFuncSetAttribute(score64_bf16_kernel<D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(SG::SMEM)) != cudaSuccess)
       return -1;
     const int tiles = (n_new + SG::TT - 1) / SG::TT;
-    dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
-    score64_bf16_kernel<D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap);
+    const int tpb = score64_tiles_per_block(tiles, a.units, nsm);
+    dim3 grid((tiles + tpb - 1) / tpb, a.units);
+    score64_bf16_kernel<D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap, tpb);
   } else {
     using SG = Score64Geom<D2, HID>;
     if (cudaFuncSetAttribute(score64_kernel<T, D2, HID>, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM) !=
         cudaSuccess)
       return -1;
     const int tiles = (n_new + SG::TT - 1) / SG::TT;
-    dim3 grid((tiles + kTilesPerBlock - 1) / kTilesPerBlock, a.units);
-    score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap);
+    const int tpb = score64_tiles_per_block(tiles, a.units, nsm);
+    dim3 grid((tiles + tpb - 1) / tpb, a.units);
+    score64_kernel<T, D2, HID><<<grid, kScore64Threads, SG::SMEM, st>>>(a, cg, k, v, n, out, cap, tpb);
   }
   return 0;
 }
