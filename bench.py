@@ -111,8 +111,8 @@ def step_bytes(w: wl.Workload) -> int:
 # of `bench.py --layers 2 --steps 2 --warmup 1` (the cr88 shape, 2 layers),
 # valid only for the kernel sources whose hash is recorded with it.
 TRAFFIC_CAPTURE = {"workload": "qwen3_4b_cr88_b64_B1024",
-                   "sources_sha256": "e719b014f3cd4bd4534c1ceaa37d42b7bac5b13d3fdd0d4a3394611a2766e72f",
-                   "dram_bytes": 280_009_984 + 7_026_944, "algorithmic_bytes": 274_452_512}
+                   "sources_sha256": "9b3c42ad75e0dfdd3a80099795cac9f95def999cb44b67e34a6f3c33d411fb84",
+                   "dram_bytes": 280_001_792 + 6_511_872, "algorithmic_bytes": 274_452_512}
 
 
 # ncu capture of the prefill attention's tensor-core kernel (the small case of

@@ -221,6 +221,14 @@ __device__ __noinline__ Decision decide_warp(const LayerArgs& a, int u, int N, i
 // commit can overwrite -- the next boundary token's row, or its caller score
 // -- into registers; decide_finish scores it and runs the argmin, whose only
 // slot the commit changes (the pending target) counts with the pending key.
+// With team_threads > 0 the warps of a deciding team meet at kDecideBar once
+// each holds what it read, before their lead lets the merge commit.
+// Named barrier of a CTA's decider warps when they decide one unit together.
+constexpr int kDecideBar = 1;
+__device__ __forceinline__ void team_bar_sync(int nthreads) {
+  asm volatile("bar.sync %0, %1;" :: "r"(kDecideBar), "r"(nthreads) : "memory");
+}
+
 template <int DH>
 struct DecideInput {
   double x[2 * DH / 32];   // this lane's scorer inputs
@@ -230,13 +238,16 @@ struct DecideInput {
 
 template <typename T, int DH>
 __device__ __noinline__ void decide_load(const LayerArgs& a, int u, int N, const T* kn, const T* vn, float ext_new,
-                                         DecideInput<DH>& in) {
+                                         DecideInput<DH>& in, int team_threads) {
   const int lane = threadIdx.x & 31;
   const int S = a.S, W = a.W, D = a.D, NS = a.NS;
   const int b = N - W - D;
   in.b = -1;
   in.sext = 0.f;
-  if (b < S) return;
+  if (b < S) {
+    if (team_threads > 0) team_bar_sync(team_threads);
+    return;
+  }
   in.b = b;
   // before the pending commit: b is the token appended by that step (W = 1,
   // D = 0), or still in its window slot (D <= 1), or in its staging slot
@@ -251,6 +262,7 @@ __device__ __noinline__ void decide_load(const LayerArgs& a, int u, int N, const
     load_scorer_input<T, 2 * DH>(krow, vrow, in.x);
   if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0 && !from_input && a.pos[static_cast<size_t>(u) * NS + rslot] != b)
     set_error(a.err, DEVERR_STATE_MISMATCH);
+  if (team_threads > 0) team_bar_sync(team_threads);
 }
 
 // decide_finish: the decision from what decide_load read, taken by one warp
@@ -264,7 +276,6 @@ __device__ __noinline__ void decide_load(const LayerArgs& a, int u, int N, const
 // and the partial minima compared (keys are unique), and every warp returns
 // the same decision.  A team sums the score's fp64 terms in another order
 // than one warp does; both round once to fp32.
-constexpr int kDecideBar = 1;
 struct DecideTeam {
   double part;
   unsigned long long best;
@@ -272,9 +283,6 @@ struct DecideTeam {
 };
 static_assert(sizeof(DecideTeam) == 24, "team slot size");
 
-__device__ __forceinline__ void team_bar_sync(int nthreads) {
-  asm volatile("bar.sync %0, %1;" :: "r"(kDecideBar), "r"(nthreads) : "memory");
-}
 
 template <int DH>
 __device__ __noinline__ Decision decide_finish(const LayerArgs& a, int u, int N, int ntk, const Decision* pending,
@@ -593,9 +601,7 @@ __device__ __forceinline__ void l2_warmup(const LayerArgs& a, bool step, int war
   const int dw = warp - NCW;
   const int base = topk_base(S, W, D);
   const int b = N + 1 - W - D;   // boundary token of the decision taken in this launch
-  const bool team = a.units <= static_cast<int>(gridDim.x);   // as the deciders split their units
-  if (team && dw != 0) return;
-  for (int u = team ? blockIdx.x : blockIdx.x * NDW + dw; u < a.units; u += team ? gridDim.x : gridDim.x * NDW) {
+  for (int u = blockIdx.x * NDW + dw; u < a.units; u += gridDim.x * NDW) {
     if (K > 0) {
       // [lo, hi) byte range of the unit's long-range scores / positions, in 16-byte units
       const int64_t lo = (static_cast<int64_t>(u) * NS + base) * 4 / 16 * 16;
@@ -787,8 +793,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ 
           const Decision cur = a.dec[static_cast<size_t>(N & 1) * a.units + u];
           DecideInput<DH> din;
           decide_load<T, DH>(a, u, N + 1, k_new + static_cast<size_t>(u) * DH, v_new + static_cast<size_t>(u) * DH,
-                             ext ? ext[u] : 0.f, din);
-          if (team) team_bar_sync(NDW * 32);   // every warp holds the row before the merge may overwrite it
+                             ext ? ext[u] : 0.f, din, team ? NDW * 32 : 0);
           if (lead) {
             const int prev = __shfl_sync(0xffffffffu, arrive(u), 0);
             if (prev == need_of(u) - 1) push_merge(u);
