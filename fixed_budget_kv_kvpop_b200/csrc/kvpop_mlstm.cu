@@ -16,12 +16,14 @@
 //
 // One warp per (batch row, KV head) unit.  Lane l holds inputs
 // [l X, l X + X) of x (X = 2d / 32) in fp64; a projection onto up to 32 rows
-// is a per-lane partial dot product per row followed by a reduce-scatter, so
-// lane j ends with row j.  Weights are fp32 and inputs bf16 or fp32, both
+// is a per-lane partial dot product per row followed by a warp sum that lane
+// j keeps for row j (a rolled loop: the step kernel runs from a cold
+// instruction cache after every decode kernel, so its code is kept short).  Weights are fp32 and inputs bf16 or fp32, both
 // exact in fp64.
 //
-// Decode: mlstm_step_kernel (one CTA of four warps per unit) runs before each
-// decode kernel of a layer.  It folds the step's token into the state and
+// Decode: mlstm_step_kernel (one CTA of four warps per unit, the head's
+// projection weights staged in shared memory) runs before each decode
+// kernel of a layer.  It folds the step's token into the state and
 // takes that step's eviction decision (the boundary token's score depends on the token that arrives in
 // the same step, so the decision cannot be taken one step ahead as the
 // stateless scorers' is).  Prefill: mlstm_prefill_kernel walks a chunk's
@@ -66,39 +68,29 @@ __device__ __forceinline__ void load_x(const T* krow, const T* vrow, double (&x)
 
 // Dot products of x with rows [r0, r0 + nr) (nr <= 32) of a row-major fp32
 // matrix with 32 X columns; row r0 + j ends in lane j (0 in lanes >= nr).
-template <int X>
+// kShared: w is in shared memory (plain loads), else global (read-only loads).
+template <int X, bool kShared = false>
 __device__ __forceinline__ double project_rows(const double (&x)[X], const float* __restrict__ w, int r0, int nr) {
   const int lane = threadIdx.x & 31;
-  double v[32];
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
+  double out = 0.0;
+#pragma unroll 1
+  for (int r = 0; r < nr; ++r) {
+    const float4* wr = reinterpret_cast<const float4*>(w + static_cast<size_t>(r0 + r) * (32 * X) + lane * X);
     double acc = 0.0;
-    if (r < nr) {
-      const float4* wr = reinterpret_cast<const float4*>(w + static_cast<size_t>(r0 + r) * (32 * X) + lane * X);
 #pragma unroll
-      for (int q = 0; q < X / 4; ++q) {
-        const float4 c = __ldg(wr + q);
-        acc = fma(static_cast<double>(c.x), x[4 * q + 0], acc);
-        acc = fma(static_cast<double>(c.y), x[4 * q + 1], acc);
-        acc = fma(static_cast<double>(c.z), x[4 * q + 2], acc);
-        acc = fma(static_cast<double>(c.w), x[4 * q + 3], acc);
-      }
+    for (int q = 0; q < X / 4; ++q) {
+      float4 c;
+      if constexpr (kShared) c = wr[q];
+      else c = __ldg(wr + q);
+      acc = fma(static_cast<double>(c.x), x[4 * q + 0], acc);
+      acc = fma(static_cast<double>(c.y), x[4 * q + 1], acc);
+      acc = fma(static_cast<double>(c.z), x[4 * q + 2], acc);
+      acc = fma(static_cast<double>(c.w), x[4 * q + 3], acc);
     }
-    v[r] = acc;
+    acc = warp_sum(acc);
+    if (lane == r) out = acc;
   }
-  // reduce-scatter: after the step with offset o, lane l keeps the half of
-  // its partial sums whose row index has bit o equal to l's; lane l ends with row l
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const double keep = up ? v[i + o] : v[i];
-      const double send = up ? v[i] : v[i + o];
-      v[i] = keep + __shfl_xor_sync(kFull, send, o);
-    }
-  }
-  return lane < nr ? v[0] : 0.0;
+  return out;
 }
 
 // Hedgehog features of z (z_j in lane j < p): [softmax(z); softmax(-z)],
@@ -233,29 +225,65 @@ __device__ __forceinline__ const T* row_ptr(const LayerArgs& a, int u, int slot)
   return reinterpret_cast<const T*>(a.kv + (static_cast<size_t>(u) * a.NS + slot) * a.row_bytes);
 }
 
-// One CTA of four warps per unit.  Warps 0-2 project the step's token (write
-// features, value, gates), warp 3 the boundary token's read features, all four
-// look for the long-range minimum; then warp 0 folds the token into the
-// state, reads the boundary token out and takes the step's decision.
+__device__ __forceinline__ void ml_cp16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Dynamic shared memory of mlstm_step_kernel: the head's W_q, W_k, W_v rows
+// (fp32), then the unit's state.
+__host__ __device__ __forceinline__ int mlstm_step_smem(int p, int dv, int d) {
+  return (2 * p + dv) * 2 * d * 4 + mlstm_state_doubles(p, dv) * 8;
+}
+
+// One CTA of four warps per unit.  The head's W_q, W_k, W_v rows (the
+// caller's constants) are copied into shared memory before the wait for the
+// previous kernel; after it, warp 2 copies the unit's state while the
+// projections run.  Warps 0-2 project the step's token (write features,
+// value, gates), warp 3 the boundary token's read features, all four look
+// for the long-range minimum (each thread's keys loaded in one batch); then
+// warp 0 folds the token into the state, reads the boundary token out and
+// takes the step's decision.  The copies put every chain of dependent loads
+// at one round trip.
 template <typename T, int X, int DV>
 __global__ void __launch_bounds__(128) mlstm_step_kernel(const LayerArgs a, const T* __restrict__ k_new,
                                                          const T* __restrict__ v_new) {
-  // Everything below reads the previous kernels' cache and counters.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  extern __shared__ __align__(16) uint8_t ml_sm[];
   __shared__ double s_phi[32], s_val[32], s_r[32], s_g[2];
   __shared__ unsigned long long s_best[4];
   __shared__ int s_slot[4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x;
-  const int N = a.layer->n_seen;
-  const int ntk = a.layer->n_topk;
-  if (N >= a.max_context) return;   // the decode kernel that follows reports the overflow
-  const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
   const int h = u % a.Hkv;
   const int p = a.mp, dv = a.mdv;
   const float* hw = a.mw + static_cast<size_t>(h) * mlstm_head_floats(p, dv, a.d);
   const float* tail = hw + static_cast<size_t>(2 * p + dv + 2) * (32 * X);
+  float* w_sm = reinterpret_cast<float*>(ml_sm);                                                  // [2p + dv][32 X]
+  double* st_sm = reinterpret_cast<double*>(ml_sm + static_cast<size_t>(2 * p + dv) * 32 * X * 4);
+  {
+    const int nch = (2 * p + dv) * 32 * X / 4;   // 16-byte chunks
+    for (int c = threadIdx.x; c < nch; c += 128) ml_cp16(w_sm + 4 * c, hw + 4 * c);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  // Everything below reads the previous kernels' cache, states and counters.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int N = a.layer->n_seen;
+  const int ntk = a.layer->n_topk;
+  if (N >= a.max_context) {   // the decode kernel that follows reports the overflow
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    return;
+  }
+  const int S = a.S, W = a.W, D = a.D, K = a.K, NS = a.NS;
+  double* st = a.mstate + static_cast<size_t>(u) * mlstm_state_doubles(p, dv);
+  if (warp == 2) {   // the state (16-byte multiple per unit) behind the weights
+    const int nch = mlstm_state_doubles(p, dv) / 2;
+    for (int c = lane; c < nch; c += 32) ml_cp16(st_sm + 2 * c, st + 2 * c);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+  } else {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  }
+  __syncthreads();   // the weights in shared memory
   const int b = N - W - D;
   const bool has_b = b >= S;
   const int bslot = has_b ? ((D == 0) ? window_slot(b, S, W) : staging_slot(b, S, W, D)) : -1;
@@ -265,9 +293,9 @@ __global__ void __launch_bounds__(128) mlstm_step_kernel(const LayerArgs a, cons
     double x[X];
     load_x<T, X>(k_new + static_cast<size_t>(u) * a.d, v_new + static_cast<size_t>(u) * a.d, x);
     if (warp == 0) {
-      s_phi[lane] = hedgehog_lane(project_rows<X>(x, hw, p, p), p);
+      s_phi[lane] = hedgehog_lane(project_rows<X, true>(x, w_sm, p, p), p);
     } else if (warp == 1) {
-      s_val[lane] = project_rows<X>(x, hw, 2 * p, dv);
+      s_val[lane] = project_rows<X, true>(x, w_sm, 2 * p, dv);
     } else {
       const double g = project_rows<X>(x, hw, 2 * p + dv, 2);
       if (lane < 2) s_g[lane] = g + static_cast<double>(__ldg(tail + dv + lane));
@@ -276,18 +304,32 @@ __global__ void __launch_bounds__(128) mlstm_step_kernel(const LayerArgs a, cons
     const T* row = row_ptr<T>(a, u, bslot);
     double xb[X];
     load_x<T, X>(row, row + a.d, xb);
-    s_r[lane] = hedgehog_lane(project_rows<X>(xb, hw, 0, p), p);
+    s_r[lane] = hedgehog_lane(project_rows<X, true>(xb, w_sm, 0, p), p);
     if ((a.flags & FLAG_DEBUG_CHECKS) && lane == 0 && a.pos[static_cast<size_t>(u) * NS + bslot] != b)
       set_error(a.err, DEVERR_STATE_MISMATCH);
   }
   if (scan) {   // minimum key (score, -position) of the long-range set as committed after step N - 1
     const int32_t* pos = a.pos + static_cast<size_t>(u) * NS + base;
     const float* score = a.score + static_cast<size_t>(u) * NS + base;
+    constexpr int kB = 8;   // keys per thread per round trip
     uint64_t best = ~0ull;
     int mslot = -1;
-    for (int i = threadIdx.x; i < K; i += 128) {
-      const uint64_t key = rank_key(score[i], pos[i]);
-      if (key < best) { best = key; mslot = base + i; }
+    for (int i0 = 0; i0 < K; i0 += 128 * kB) {
+      float sc[kB];
+      int32_t ps[kB];
+#pragma unroll
+      for (int t = 0; t < kB; ++t) {
+        const int i = i0 + threadIdx.x + 128 * t;
+        if (i < K) { sc[t] = score[i]; ps[t] = pos[i]; }
+      }
+#pragma unroll
+      for (int t = 0; t < kB; ++t) {
+        const int i = i0 + threadIdx.x + 128 * t;
+        if (i < K) {
+          const uint64_t key = rank_key(sc[t], ps[t]);
+          if (key < best) { best = key; mslot = base + i; }
+        }
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -297,11 +339,11 @@ __global__ void __launch_bounds__(128) mlstm_step_kernel(const LayerArgs a, cons
     }
     if (lane == 0) { s_best[warp] = best; s_slot[warp] = mslot; }
   }
-  __syncthreads();
+  if (warp == 2) asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();   // projections, minima and the state in shared memory
   if (warp != 0) return;
-  double* st = a.mstate + static_cast<size_t>(u) * mlstm_state_doubles(p, dv);
   LaneState<DV> s;
-  state_load<DV>(st, p, dv, s);
+  state_load<DV>(st_sm, p, dv, s);
   state_fold<DV>(s_phi[lane], s_val, s_g[0], s_g[1], dv, s);
   state_store<DV>(st, p, dv, s);
   Decision r;
@@ -386,8 +428,23 @@ __global__ void __launch_bounds__(32 * kMlstmWarps) mlstm_prefill_kernel(const L
 template <typename T, int X, int DV>
 int launch_step_t(const LayerArgs& a, const void* k_new, const void* v_new, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
+  const int smem = mlstm_step_smem(a.mp, a.mdv, a.d);
+  // The shared-memory attribute (the most any p <= 16, dv <= DV needs)
+  // belongs to the current device: set once per device (devices beyond the
+  // table get it on every call).
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
+    if (cudaFuncSetAttribute(mlstm_step_kernel<T, X, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mlstm_step_smem(16, DV, 16 * X)) != cudaSuccess)
+      return -1;
+    if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
+  }
   cfg.gridDim = dim3(static_cast<unsigned>(a.units));
   cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
