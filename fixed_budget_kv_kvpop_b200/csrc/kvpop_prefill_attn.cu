@@ -53,6 +53,72 @@ __host__ __device__ inline int next_pow2(int x) {
 }
 
 // ---------------- cutoffs: sort (one CTA per unit), then walk (one warp per unit) ----------------
+// The bitonic network (descending) over npow = E * kCutThreads keys in
+// shared memory, with thread t holding keys t E .. t E + E - 1 in registers:
+// strides below E compare within a thread, strides E .. 16 E between the
+// lanes of a warp (shuffles), and only larger strides go through shared
+// memory.  The same compare-exchanges as the all-shared-memory network, so
+// the same order.
+template <int E>
+__device__ __forceinline__ void bitonic_sort_regs(uint64_t* keys, int npow) {
+  const int t = threadIdx.x;
+  uint64_t e[E];
+#pragma unroll
+  for (int k = 0; k < E; ++k) e[k] = keys[t * E + k];
+  for (int kk = 2; kk <= npow; kk <<= 1) {
+    int j = kk >> 1;
+    if (j >= 32 * E) {   // strides across warps
+#pragma unroll
+      for (int k = 0; k < E; ++k) keys[t * E + k] = e[k];
+      __syncthreads();
+      for (; j >= 32 * E; j >>= 1) {
+        for (int i = t; i < npow; i += blockDim.x) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const uint64_t x = keys[i], y = keys[ixj];
+            const bool desc = (i & kk) == 0;
+            if (desc ? (x < y) : (x > y)) {
+              keys[i] = y;
+              keys[ixj] = x;
+            }
+          }
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int k = 0; k < E; ++k) e[k] = keys[t * E + k];
+    }
+    for (; j >= E; j >>= 1) {   // strides across the lanes of a warp: element k of thread t ^ (j / E)
+      const int lm = j / E;
+      const bool lower = (t & lm) == 0;
+#pragma unroll
+      for (int k = 0; k < E; ++k) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, e[k], lm);
+        const bool desc = ((t * E + k) & kk) == 0;
+        e[k] = (desc == lower) ? (e[k] > y ? e[k] : y) : (e[k] < y ? e[k] : y);
+      }
+    }
+#pragma unroll
+    for (int jj = E / 2; jj >= 1; jj >>= 1) {   // strides within the thread
+      if (jj > j) continue;
+#pragma unroll
+      for (int k = 0; k < E; ++k) {
+        if ((k & jj) != 0) continue;
+        const uint64_t x = e[k], y = e[k | jj];
+        const bool desc = ((t * E + k) & kk) == 0;
+        if (desc ? (x < y) : (x > y)) {
+          e[k] = y;
+          e[k | jj] = x;
+        }
+      }
+    }
+  }
+  __syncthreads();   // every thread's last shared-memory reads are done
+#pragma unroll
+  for (int k = 0; k < E; ++k) keys[t * E + k] = e[k];
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kCutThreads) cutoff_kernel(const float* __restrict__ scores, int score_cap,
                                                              int32_t* __restrict__ cut, int32_t* __restrict__ order,
                                                              int n, int ne, int npow, int S, uint64_t* keys_g,
@@ -70,20 +136,24 @@ __global__ void __launch_bounds__(kCutThreads) cutoff_kernel(const float* __rest
   for (int i = tid; i < npow; i += blockDim.x) keys[i] = (i < ne) ? rank_key(su[i], S + i) : 0ull;
   __syncthreads();
   // bitonic sort, descending (best first); padding keys (0) sink to the end
-  for (int kk = 2; kk <= npow; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < npow; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint64_t x = keys[i], y = keys[ixj];
-          const bool desc = (i & kk) == 0;
-          if (desc ? (x < y) : (x > y)) {
-            keys[i] = y;
-            keys[ixj] = x;
+  if (!keys_global && npow == 16 * kCutThreads) {   // 4097 .. 8192 eligible tokens
+    bitonic_sort_regs<16>(keys, npow);
+  } else {
+    for (int kk = 2; kk <= npow; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < npow; i += blockDim.x) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const uint64_t x = keys[i], y = keys[ixj];
+            const bool desc = (i & kk) == 0;
+            if (desc ? (x < y) : (x > y)) {
+              keys[i] = y;
+              keys[ixj] = x;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
   // the positions in best-first order, for the walk

@@ -279,6 +279,26 @@ def _check_large_unit(r, unit, m_samples, rows, atol):
             np.testing.assert_allclose(lse[qp], orc.attention_lse(q[qp], k[A]), rtol=0, atol=LSE_ATOL[w.dtype])
 
 
+def test_cutoffs_from_the_register_sort():
+    """4097 .. 8192 eligible tokens per unit: cutoff_kernel sorts the 8192
+    rank keys with 16 per thread in registers (shuffles between lanes,
+    shared memory only for strides of 512 and more).  Two units, 6,000 and
+    8,324 prompt tokens (5,868 and 8,192 eligible), bf16 d 128 G 4, the 87.5%
+    budget, caller scores with ties: every cutoff equal to the Fenwick tree,
+    the running top-k at sampled positions, sampled rows."""
+    _need_gpu()
+    w = _case("bf16", 128, 8, 2, S=4, W=128, D=0, K=892, hidden=64)
+    for n in (6000, 8324):
+        r = run_prefill_attention(w, n, external=True, tie_levels=3, gen_device="cuda")
+        rng = np.random.default_rng(n)
+        m_last = n - 1 - w.window - w.delay
+        ms = sorted(set([w.sinks, w.sinks + w.topk - 1, w.sinks + w.topk, m_last] +
+                        list(rng.integers(w.sinks, m_last + 1, 4))))
+        rows = sorted(set([0, n - 1] + list(rng.integers(0, n, 4))))
+        for unit in range(2):
+            _check_large_unit(r, unit, ms, rows, gh.BF16_ATOL)
+
+
 def test_cutoffs_sorted_in_the_workspace():
     """More than 16,384 eligible tokens in a unit: cutoff_kernel sorts the
     rank keys in the caller's workspace instead of shared memory (bitmap
