@@ -129,6 +129,31 @@ def test_split_append_attend_matches_fused_step(S, W, D, K):
         gh.check_unit(b, 0, unit, exact_slots=False, atol=gh.BF16_ATOL)
 
 
+@pytest.mark.parametrize("external", [True, False])
+def test_team_decision_with_several_key_batches(external):
+    """Two units (fewer than CTAs): a CTA's four decider warps share each
+    decision, and with K = 2100 each warp scans 525 long-range keys in two
+    batches of loads.  Prompt 2400 (the long-range set full), 6 decode
+    steps; slot maps bit-exact against the slot simulator with tie-heavy
+    caller scores, exact fp32 scores with the MLP."""
+    _need_gpu()
+    w = wl.Workload("team_case", batch=1, n_layers=1, n_q_heads=8, n_kv_heads=2, head_dim=128, dtype="bf16",
+                    sinks=4, window=16, topk=2100, delay=0, prefill=2400, decode=6, scorer_hidden=64,
+                    heavy_hitter_frac=0.02)
+    run = gh.run_gpu(w, n_layers=1, n_steps=w.decode, external=external, tie_levels=3 if external else 0)
+    for unit in range(2):
+        gh.check_unit(run, 0, unit, exact_slots=external, atol=gh.BF16_ATOL)
+    if not external:
+        pos, score, _ = run.cache.inspect(0)
+        base = w.sinks + w.window + w.delay
+        for unit in range(2):
+            k_all, v_all, _ = gh.unit_inputs(run, 0, unit)
+            ref = gh.unit_scores(run, 0, unit, k_all, v_all)
+            got = [(int(pos[unit, sl]), float(score[unit, sl])) for sl in range(base, pos.shape[1]) if pos[unit, sl] >= 0]
+            assert len(got) == w.topk
+            assert all(np.float32(ref[p_]) == s_ for p_, s_ in got), f"unit {unit}: scores differ"
+
+
 def test_mlp_scores_match_oracle_exactly_in_fp32():
     """The scorer accumulates in fp64 and rounds once, so the long-range slots'
     fp32 scores equal the oracle's float64-then-float32 scores."""
